@@ -1,0 +1,220 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant online KV-cache vector quantization and
+ * decode attention over the packed cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "TurboQuant-MLX: quantizzare pesi e KV cache per LLM
+ * open-weight su Mac", section "Il metodo TurboQuant, in breve"): each head
+ * vector x is rotated by a seeded random orthogonal matrix Pi, every rotated
+ * coordinate is quantized on its own to the nearest Lloyd-Max centroid of the
+ * known post-rotation coordinate density, and the b-bit codes are packed next
+ * to the vector's norm.  The inner-product ("prod") variant spends one of the
+ * b bits per channel on a 1-bit QJL sketch sign(S r) of the residual r so that
+ * <q, x> is estimated without bias.  No calibration: everything depends only
+ * on (d, b, seed).
+ *
+ * Conventions for every call below
+ *  - Memory: the caller owns all memory.  Device pointers are plain CUDA
+ *    device addresses (for example from torch tensors); host pointers are
+ *    plain host arrays.  No call on the data path allocates; tq_params_create
+ *    allocates the parameter tables once and tq_params_destroy frees them.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream).  Device calls only enqueue work and never synchronize.
+ *  - Errors: every call returns a tq_status; TQ_OK is 0.  On failure nothing
+ *    is enqueued and tq_last_error() returns a message for the calling host
+ *    thread.  Inputs must be finite: NaN or Inf inputs give unspecified codes
+ *    but never an out-of-bounds access.
+ *  - Sizes: d = 128 and m = 128 in this version (TQ_ERR_UNSUPPORTED
+ *    otherwise); bits in 1..4 (MSE) or 1..4 total (prod, 1 = QJL only).
+ *
+ * Packed row format (both sides of the library agree on it; the pages only
+ * say that codes live at "unconventional bit widths", NVIDIA forum post "Why
+ * TurboQuant saves DGX twice"):
+ *  - codes: code j of rotated coordinate j sits at bit offset sum_{i<j} w_i of
+ *    the row, least-significant bit first inside little-endian bytes.  w_j is
+ *    the MSE bit width (bits for MSE, bits-1 for prod); a mixed row uses
+ *    bits+1 for j < d/2.  Row bytes: 16*w (uniform) or 8*(2w+1) (mixed).
+ *  - code value = number of Lloyd-Max decision bounds strictly below the
+ *    rotated unit-vector coordinate (ties go to the lower centroid).
+ *  - norms: fp32 ||x||.  qjl (prod): m/8 bytes per row, bit i = 1 iff
+ *    (S r)_i >= 0.  res_norms (prod): fp32 ||r||.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_ARG = 1,          /* NULL pointer, negative size, bad enum */
+  TQ_ERR_UNSUPPORTED = 2,  /* a size or format this build does not handle */
+  TQ_ERR_ALIGN = 3,        /* a device plane not 16-byte aligned */
+  TQ_ERR_CAPACITY = 4,     /* workspace or cache too small */
+  TQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (message says which) */
+  TQ_ERR_NOMEM = 6         /* tq_params_create could not allocate */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+typedef enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1 } tq_mode;
+typedef enum { TQ_K = 0, TQ_V = 1 } tq_which;
+
+/* Parameters of one quantizer pair (keys and values may differ: the
+ * asymmetric K/V setting of "Greetings from TurboQuant-MLX" (turboquant_plus
+ * issue 59) and of the TurboQuant-MLX article, section "Cosa aggiunge").
+ * bits_*: total bits per channel.  mixed_*: 1 puts the first d/2 rotated
+ * channels at bits+1 ("3.5 bits per channel" with bits = 3, article section
+ * "Il metodo TurboQuant, in breve"); MSE mode only.  seed drives Pi and S. */
+typedef struct {
+  int d;
+  int bits_k, bits_v;
+  int mode_k, mode_v;    /* tq_mode */
+  int mixed_k, mixed_v;  /* 0 or 1 */
+  int m;                 /* QJL sketch size */
+  uint64_t seed;
+} tq_config;
+
+typedef struct tq_params tq_params;
+
+/* One packed plane set (device pointers).  codes: [n][code_bytes];
+ * norms: [n] fp32; qjl: [n][m/8] (prod only, else NULL); res_norms: [n] fp32
+ * (prod only, else NULL).  Planes must be 16-byte aligned (TQ_ERR_ALIGN). */
+typedef struct {
+  uint8_t* codes;
+  float* norms;
+  uint8_t* qjl;
+  float* res_norms;
+} tq_packed;
+
+/* ---- host tables ------------------------------------------------------ */
+
+/* Lloyd-Max codebook of one coordinate of a uniform point on S^{d-1}
+ * (density proportional to (1-x^2)^((d-3)/2)), article section "Il metodo
+ * TurboQuant, in breve" (optimal scalar quantizer for the known distribution)
+ * and section "Cosa aggiunge turboquant-mlx" (Lloyd-Max).  Writes 2^bits
+ * ascending centroids and the 2^bits - 1 midpoints between them (host
+ * arrays, caller-owned).  Any d >= 3 and bits in 1..8.  Pure host function. */
+tq_status tq_codebook(int d, int bits, double* centroids, double* bounds);
+
+/* Seeded random rotation Pi (d x d row-major, y = Pi u): Haar orthogonal,
+ * the QR factor of a Gaussian matrix with diag(R) made positive.  Gaussians
+ * from SplitMix64 (stream seed ^ (0 << 32)) and Box-Muller, filled row-major.
+ * Host array of d*d doubles, caller-owned.  Pure host function. */
+tq_status tq_rotation(uint64_t seed, int d, double* pi);
+
+/* QJL matrix S (m x d row-major, i.i.d. N(0,1)) from the stream
+ * seed ^ (1 << 32).  Host array of m*d doubles.  Pure host function. */
+tq_status tq_qjl_matrix(uint64_t seed, int m, int d, double* s);
+
+/* ---- parameters ------------------------------------------------------- */
+
+/* Build the tables for cfg on the current CUDA device (allocates device
+ * memory once, copies with the legacy stream and synchronizes; not for the
+ * data path).  *out is owned by the caller and freed by tq_params_destroy. */
+tq_status tq_params_create(const tq_config* cfg, tq_params** out);
+void tq_params_destroy(tq_params* p);
+
+/* Bytes per packed row for K (which = TQ_K) or V: code bytes and QJL bytes
+ * (0 in MSE mode). */
+tq_status tq_row_bytes(const tq_params* p, int which, int* code_bytes, int* qjl_bytes);
+
+/* ---- quantize / dequantize ------------------------------------------- */
+
+/* Rotate, quantize and pack n vectors x ([n][d], fp32 or bf16, device) with
+ * the K or V format of p into `out` (device planes sized for n rows).
+ * Article section "Il metodo TurboQuant, in breve".  n = 0 is a no-op. */
+tq_status tq_quantize(const tq_params* p, const void* x, int x_dtype, int64_t n, int which,
+                      const tq_packed* out, void* stream);
+
+/* x_hat = ||x|| (Pi^T c[idx] + sqrt(pi/2)/m * ||r|| * S^T z) for n packed rows
+ * (device) into out ([n][d] fp32, device); accumulates in fp64.  A boundary
+ * and test call: decode attention never materializes x_hat. */
+tq_status tq_dequantize(const tq_params* p, const tq_packed* in, int64_t n, int which,
+                        float* out, void* stream);
+
+/* ---- packed KV cache ---------------------------------------------------- */
+
+/* A cache for n_seq sequences x n_kv_heads heads.  Token t of a sequence is
+ * kept unquantized in bf16 if t < n_sink (attention sink, "Greetings from
+ * TurboQuant-MLX", item 1) and is quantized row t - n_sink otherwise.
+ * Every plane is laid out [n_seq][n_kv_heads][capacity][row] (sink planes
+ * [n_seq][n_kv_heads][n_sink][d]); capacity is a multiple of 64 and counts
+ * quantized rows.  lens: device int32 [n_seq], tokens held per sequence
+ * (sink included); the caller zeroes it for an empty cache.  status: device
+ * int32 word; kernels OR error bits into it (1 = append past capacity,
+ * 2 = a length above the bound given to tq_decode_attn). */
+typedef struct {
+  int n_seq, n_kv_heads, capacity, n_sink;
+  uint8_t* k_codes; float* k_norms; uint8_t* k_qjl; float* k_res_norms;
+  uint8_t* v_codes; float* v_norms; uint8_t* v_qjl; float* v_res_norms;
+  uint16_t* k_sink; uint16_t* v_sink;
+  int32_t* lens;
+  int32_t* status;
+} tq_cache;
+
+/* Bytes of one contiguous buffer holding every plane of such a cache (each
+ * plane 256-byte aligned); 0 on bad arguments. */
+size_t tq_cache_bytes(const tq_params* p, int n_seq, int n_kv_heads, int capacity, int n_sink);
+
+/* Fill *out with plane pointers carved from `base` (device, >= tq_cache_bytes
+ * bytes, 256-byte aligned).  lens and status are separate caller buffers. */
+tq_status tq_cache_bind(const tq_params* p, void* base, size_t bytes, int n_seq, int n_kv_heads,
+                        int capacity, int n_sink, int32_t* lens, int32_t* status, tq_cache* out);
+
+/* Append n_tok new tokens to each of n_seq sequences (streaming append,
+ * "Greetings from TurboQuant-MLX", item 2: 64-token chunks; the method is
+ * online, article section "Il metodo TurboQuant, in breve").  seq_ids:
+ * device int32 [n_seq], distinct cache sequence indices.  k, v: device
+ * [n_seq][n_tok][n_kv_heads][d] in dtype.  Tokens land at positions
+ * lens[s] .. lens[s] + n_tok - 1 (sink or quantized row), then lens[s] grows
+ * by n_tok, all in stream order.  A sequence that would pass
+ * n_sink + capacity is left unchanged and bit 1 is set in cache->status. */
+tq_status tq_append(const tq_params* p, const tq_cache* cache, const int32_t* seq_ids,
+                    const void* k, const void* v, int dtype, int n_tok, int n_seq, void* stream);
+
+/* ---- decode attention --------------------------------------------------- */
+
+/* sparse_v_threshold: V of a quantized token is left out when an upper bound
+ * on its softmax weight is below this value (0 = off); the softmax
+ * denominator keeps every token ("Greetings from TurboQuant-MLX", item 3:
+ * 1e-6).  The bound used is exp(s - m)/l over the tokens seen so far, which
+ * is never below the final weight, so no token the exact rule keeps is
+ * skipped. */
+typedef struct {
+  float sparse_v_threshold;
+  int reserved;
+} tq_attn_flags;
+
+/* Workspace bytes for tq_decode_attn on B sequences with n_kv_heads heads,
+ * Hq query heads and lengths up to max_len. */
+size_t tq_decode_workspace_bytes(const tq_params* p, int B, int hq, int n_kv_heads, int max_len);
+
+/* Zero the bookkeeping part of a fresh workspace (once per workspace; the
+ * decode kernel leaves it zeroed after each call). */
+tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* One decode step for sequences b = 0..B-1 of the cache: q [B][hq][d]
+ * (q_dtype), out [B][hq][d] (out_dtype), GQA: query head h reads kv-head
+ * h / (hq / n_kv_heads), hq / n_kv_heads <= 8.  Score <q, k>/sqrt(d) with the
+ * key read through its codes: s = ||k|| (<Pi q, c[idx]> + sqrt(pi/2)/m ||r||
+ * <S q, z>) / sqrt(d); softmax over all held tokens; V accumulated in the
+ * rotated domain and Pi^T (and S^T) applied once per output.  Sink tokens use
+ * their bf16 keys and values directly.  A sequence with no tokens gives a
+ * zero output.  max_len: host bound on lens (longer sequences are cut to it
+ * and bit 2 is set in cache->status). */
+tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
+                         int B, int hq, int max_len, void* out, int out_dtype,
+                         void* workspace, size_t ws_bytes, const tq_attn_flags* flags,
+                         void* stream);
+
+/* Message for the last failed call on this host thread ("" if none). */
+const char* tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */
