@@ -1,0 +1,80 @@
+// Internal declarations shared by the host code and the CUDA kernels of libtq.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kDim = 128;       // head dimension handled by the kernels
+constexpr int kSketch = 128;    // QJL sketch size m
+constexpr int kMaxBits = 4;     // largest MSE code width used by the kernels
+constexpr int kBookSlots = 16;  // centroid slots per width in device tables
+
+// One quantizer format (keys or values).
+//   mse_bits: width of the uniform MSE part (bits, or bits-1 in prod mode);
+//   mixed:    the first d/2 rotated coordinates use mse_bits+1;
+//   prod:     a QJL sign row (m/8 bytes) and a residual norm follow.
+// id packs the three into one small integer used to pick kernel variants.
+struct FormatSpec {
+  int total_bits = 0;
+  int mse_bits = 0;
+  int mixed = 0;
+  int prod = 0;
+  int code_bytes = 0;
+  int qjl_bytes = 0;
+  int id() const { return mse_bits | (mixed << 3) | (prod << 4); }
+  int width(int j) const { return (mixed && j < kDim / 2) ? mse_bits + 1 : mse_bits; }
+};
+
+}  // namespace tq
+
+struct tq_params {
+  tq_config cfg;
+  tq::FormatSpec fk, fv;
+  int device = 0;
+  // host copies (fp64)
+  std::vector<double> pi, s;
+  // device tables, carved from one allocation
+  void* block = nullptr;
+  float* pi32 = nullptr;   // Pi   [d][d] row-major (y = Pi u)
+  float* pit32 = nullptr;  // Pi^T [d][d]
+  float* s32 = nullptr;    // S    [m][d]
+  float* st32 = nullptr;   // S^T  [d][m]
+  float* mt32 = nullptr;   // (S Pi^T)^T [d][m]: sketch of a rotated-domain residual
+  double* pi64 = nullptr;  // Pi [d][d] fp64 (dequantize)
+  double* s64 = nullptr;   // S  [m][d] fp64 (dequantize)
+  float* cb32 = nullptr;   // centroids [kMaxBits+1][16] (row b = width b)
+  float* bd32 = nullptr;   // decision bounds [kMaxBits+1][16]
+  double* cb64 = nullptr;  // centroids fp64 [kMaxBits+1][16]
+};
+
+namespace tq {
+
+tq_status fail(tq_status st, const std::string& msg);
+tq_status cuda_fail(cudaError_t e, const char* what);
+
+// Kernel launchers (defined in the .cu files).
+tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x, int x_bf16,
+                          int64_t n, const tq_packed* out, cudaStream_t st);
+tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* seq_ids,
+                        const void* k, const void* v, int x_bf16, int n_tok, int n_seq,
+                        cudaStream_t st);
+tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_packed* in,
+                            int64_t n, float* out, cudaStream_t st);
+
+struct DecodePlan {
+  int B, hq, hkv, group, max_len, n_splits, split_tokens, part_floats;
+  size_t ws_partials_bytes, ws_total_bytes;
+};
+DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len);
+tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c,
+                        const DecodePlan& plan, void* out, int out_bf16, void* ws,
+                        float sparse_thr, cudaStream_t st);
+
+}  // namespace tq

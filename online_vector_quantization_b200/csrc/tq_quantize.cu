@@ -1,0 +1,472 @@
+// Rotate + quantize + pack kernels (plain rows and streaming cache append) and
+// the fp64 dequantizer.
+//
+// Method: page "TurboQuant-MLX: quantizzare pesi e KV cache per LLM
+// open-weight su Mac", section "Il metodo TurboQuant, in breve" -- rotate by
+// Pi, quantize each rotated coordinate of the unit vector to its Lloyd-Max
+// centroid, keep the norm; the prod variant adds sign(S r) of the residual.
+// Streaming append in 64-token chunks: "Greetings from TurboQuant-MLX"
+// (turboquant_plus issue 59), item 2.
+//
+// Kernel shape: persistent CTAs of 256 threads; Pi^T (and the residual sketch
+// matrix (S Pi^T)^T in prod mode) stay in shared memory for the CTA's life;
+// each 64-vector tile is staged transposed in shared memory and multiplied
+// with 4x8 register blocking in fp32 (the decision needs fp32-level rotation
+// accuracy: a coordinate within ~1e-6 of a bound is the only place the code
+// may differ from an fp64 reference).
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int kTile = 64;       // vectors per tile
+constexpr int kThreads = 256;
+
+struct QuantArgs {
+  const void* x;
+  int x_bf16;
+  int64_t n;
+  int mse_bits, mixed, prod, code_bytes;
+  const float* pit;  // Pi^T [d][d]
+  const float* mt;   // (S Pi^T)^T [d][m]
+  const float* cb;   // [5][16]
+  const float* bd;   // [5][16]
+  // plain destination (row = vector index)
+  uint8_t* codes;
+  float* norms;
+  uint8_t* qjl;
+  float* res;
+  // append destination
+  int append;
+  const int32_t* seq_ids;
+  const int32_t* lens;
+  int n_tok, hkv, capacity, n_sink, cache_seqs;
+  uint16_t* sink;  // bf16 [n_seq][hkv][n_sink][d]
+};
+
+struct SmemQuant {
+  float pit[kDim][kDim];     // pit[k][j] = Pi[j][k]
+  float xs[kDim][kTile];     // x transposed: xs[k][v]
+  float nu[kTile];
+  float inv_nu[kTile];
+  uint8_t codes[kTile][kDim];
+  int64_t row[kTile];        // destination row, -1 = none (tail or sink token)
+};
+
+struct SmemProd {
+  float mt[kDim][kSketch];   // mt[j][i] = M[i][j], M = S Pi^T
+  float rs[kDim][kTile];     // rotated-domain residual, transposed
+};
+
+// Destination row of vector v for an append: (seq, head, pos - n_sink);
+// also copies sink tokens.  Returns -1 when there is nothing to quantize.
+__device__ int64_t append_row(const QuantArgs& a, int64_t v, int* seq_out, int* head_out, int* pos_out) {
+  const int head = static_cast<int>(v % a.hkv);
+  const int64_t st = v / a.hkv;
+  const int tok = static_cast<int>(st % a.n_tok);
+  const int s_local = static_cast<int>(st / a.n_tok);
+  const int seq = a.seq_ids[s_local];
+  *seq_out = seq;
+  *head_out = head;
+  *pos_out = 0;
+  if (seq < 0 || seq >= a.cache_seqs) return -1;          // rejected by the length update
+  const int len = a.lens[seq];
+  *pos_out = len + tok;
+  if (len < 0 || len + a.n_tok > a.n_sink + a.capacity) return -1;
+  const int pos = len + tok;
+  if (pos < a.n_sink) return -2;                           // sink token
+  return (static_cast<int64_t>(seq) * a.hkv + head) * a.capacity + (pos - a.n_sink);
+}
+
+template <int BF16>
+__device__ void load_tile(const QuantArgs& a, SmemQuant& s, int64_t v0) {
+  // 16-byte chunks; lanes walk vectors so the transposed shared stores of a
+  // warp hit 32 consecutive banks.
+  constexpr int kElems = BF16 ? 8 : 4;
+  constexpr int kChunks = kDim / kElems;
+  const int tid = threadIdx.x;
+  for (int it = tid; it < kTile * kChunks; it += kThreads) {
+    const int v = (it & 31) + 32 * ((it >> 5) & 1);
+    const int chunk = it >> 6;
+    const int64_t gv = v0 + v;
+    float vals[kElems];
+    if (gv < a.n) {
+      const char* src = static_cast<const char*>(a.x) + (gv * kDim + chunk * kElems) * (BF16 ? 2 : 4);
+      uint4 raw = *reinterpret_cast<const uint4*>(src);
+      if (BF16) {
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int e = 0; e < kElems; ++e) vals[e] = __bfloat162float(h[e]);
+      } else {
+        const float* f = reinterpret_cast<const float*>(&raw);
+#pragma unroll
+        for (int e = 0; e < kElems; ++e) vals[e] = f[e];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kElems; ++e) vals[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < kElems; ++e) s.xs[chunk * kElems + e][v] = vals[e];
+  }
+}
+
+__device__ __forceinline__ int quantize_coord(float u, const float* bd, int bits) {
+  // number of bounds strictly below u (bounds ascending, unused slots +inf)
+  int idx = 0;
+  for (int step = (1 << bits) >> 1; step > 0; step >>= 1)
+    if (bd[idx + step - 1] < u) idx += step;
+  return idx;
+}
+
+// Bits [32w, 32w+32) of a packed row whose codes sit in smem (one byte each).
+__device__ __forceinline__ uint32_t pack_word(const uint8_t* codes, int w, int mse_bits, int mixed) {
+  uint32_t out = 0;
+  const int lo = 32 * w, hi = lo + 32;
+  // segment 0: coordinates [0, n0) at width b0 from bit 0; segment 1 after it
+  const int b0 = mixed ? mse_bits + 1 : mse_bits;
+  const int n0 = mixed ? kDim / 2 : kDim;
+  const int seg1_bit = n0 * b0;
+  for (int seg = 0; seg < (mixed ? 2 : 1); ++seg) {
+    const int b = seg ? mse_bits : b0;
+    const int base_bit = seg ? seg1_bit : 0;
+    const int j0 = seg ? n0 : 0, j1 = seg ? kDim : n0;
+    int first = j0 + max(0, (lo - base_bit) / b - 1);
+    for (int j = first; j < j1; ++j) {
+      const int bit = base_bit + (j - j0) * b;
+      if (bit >= hi) break;
+      if (bit + b <= lo) continue;
+      const uint32_t c = codes[j];
+      const int sh = bit - lo;
+      out |= sh >= 0 ? (c << sh) : (c >> (-sh));
+    }
+  }
+  return out;
+}
+
+template <int BF16>
+__global__ void __launch_bounds__(kThreads, 1) quantize_kernel(QuantArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SmemQuant& s = *reinterpret_cast<SmemQuant*>(smem_raw);
+  SmemProd* sp = a.prod ? reinterpret_cast<SmemProd*>(smem_raw + sizeof(SmemQuant)) : nullptr;
+  __shared__ float cb_s[kMaxBits + 1][kBookSlots];
+  __shared__ float bd_s[kMaxBits + 1][kBookSlots];
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < kDim * kDim / 4; i += kThreads)
+    reinterpret_cast<float4*>(&s.pit[0][0])[i] = reinterpret_cast<const float4*>(a.pit)[i];
+  if (a.prod)
+    for (int i = tid; i < kDim * kSketch / 4; i += kThreads)
+      reinterpret_cast<float4*>(&sp->mt[0][0])[i] = reinterpret_cast<const float4*>(a.mt)[i];
+  for (int i = tid; i < (kMaxBits + 1) * kBookSlots; i += kThreads) {
+    cb_s[i / kBookSlots][i % kBookSlots] = a.cb[i];
+    bd_s[i / kBookSlots][i % kBookSlots] = a.bd[i];
+  }
+
+  const int tv = tid >> 4;  // vectors 4tv .. 4tv+3
+  const int tj = tid & 15;  // dims 8tj .. 8tj+7
+  const int64_t n_tiles = (a.n + kTile - 1) / kTile;
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int64_t v0 = tile * kTile;
+    __syncthreads();  // previous tile fully consumed
+    load_tile<BF16>(a, s, v0);
+    if (tid < kTile) {
+      const int64_t gv = v0 + tid;
+      int64_t row = -1;
+      if (gv < a.n) {
+        if (a.append) {
+          int seq, head, pos;
+          row = append_row(a, gv, &seq, &head, &pos);
+          if (row == -2) {
+            // sink token: keep the bf16 value (input converted) and skip
+            uint16_t* dst = a.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
+            const char* src = static_cast<const char*>(a.x) + gv * kDim * (BF16 ? 2 : 4);
+            for (int k = 0; k < kDim; ++k) {
+              float f = BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[k])
+                             : reinterpret_cast<const float*>(src)[k];
+              __nv_bfloat16 h = __float2bfloat16_rn(f);
+              dst[k] = *reinterpret_cast<uint16_t*>(&h);
+            }
+            row = -1;
+          }
+        } else {
+          row = gv;
+        }
+      }
+      s.row[tid] = row;
+    }
+    __syncthreads();
+    if (tid < kTile) {
+      float ss = 0.f;
+      for (int k = 0; k < kDim; ++k) ss = fmaf(s.xs[k][tid], s.xs[k][tid], ss);
+      const float nu = sqrtf(ss);
+      s.nu[tid] = nu;
+      s.inv_nu[tid] = nu > 0.f ? 1.f / nu : 0.f;
+    }
+
+    // y = Pi x for 4 vectors x 8 dims per thread
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < kDim; ++k) {
+      const float4 xv = *reinterpret_cast<const float4*>(&s.xs[k][4 * tv]);
+      const float4 p0 = *reinterpret_cast<const float4*>(&s.pit[k][8 * tj]);
+      const float4 p1 = *reinterpret_cast<const float4*>(&s.pit[k][8 * tj + 4]);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float pa[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xa[i], pa[j], acc[i][j]);
+    }
+    __syncthreads();  // nu ready; xs no longer needed
+
+    float g2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int v = 4 * tv + i;
+      const float inv = s.inv_nu[v];
+      const bool zero = !(s.nu[v] > 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int dim = 8 * tj + j;
+        const int b = (a.mixed && dim < kDim / 2) ? a.mse_bits + 1 : a.mse_bits;
+        const float u = acc[i][j] * inv;
+        int idx = 0;
+        float c = 0.f;
+        if (b > 0 && !zero) {
+          idx = quantize_coord(u, bd_s[b], b);
+          c = cb_s[b][idx];
+        }
+        s.codes[v][dim] = static_cast<uint8_t>(idx);
+        if (a.prod) {
+          const float r = zero ? 0.f : u - c;
+          sp->rs[dim][v] = r;
+          g2[i] = fmaf(r, r, g2[i]);
+        }
+      }
+    }
+    __syncthreads();
+
+    // pack codes and write norms
+    const int words = a.code_bytes / 4;
+    for (int it = tid; it < kTile * words; it += kThreads) {
+      const int v = it / words, w = it % words;
+      const int64_t row = s.row[v];
+      if (row < 0) continue;
+      reinterpret_cast<uint32_t*>(a.codes + row * a.code_bytes)[w] =
+          pack_word(s.codes[v], w, a.mse_bits, a.mixed);
+    }
+    if (tid < kTile && s.row[tid] >= 0) a.norms[s.row[tid]] = s.nu[tid];
+
+    if (a.prod) {
+      // gamma = ||r||: reduce over the 16 threads sharing tv (lanes of one half-warp)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) g2[i] += __shfl_xor_sync(0xffffffffu, g2[i], off);
+      // sketch t = M r for 4 vectors x 8 sketch rows
+      float t[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[i][j] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < kDim; ++k) {
+        const float4 rv = *reinterpret_cast<const float4*>(&sp->rs[k][4 * tv]);
+        const float4 m0 = *reinterpret_cast<const float4*>(&sp->mt[k][8 * tj]);
+        const float4 m1 = *reinterpret_cast<const float4*>(&sp->mt[k][8 * tj + 4]);
+        const float ra[4] = {rv.x, rv.y, rv.z, rv.w};
+        const float ma[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) t[i][j] = fmaf(ra[i], ma[j], t[i][j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int v = 4 * tv + i;
+        const int64_t row = s.row[v];
+        if (row < 0) continue;
+        const bool zero = !(s.nu[v] > 0.f);
+        uint32_t byte = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) byte |= (t[i][j] >= 0.f ? 1u : 0u) << j;
+        a.qjl[row * (kSketch / 8) + tj] = zero ? 0 : static_cast<uint8_t>(byte);
+        if (tj == 0) a.res[row] = zero ? 0.f : sqrtf(g2[i]);
+      }
+    }
+  }
+}
+
+// Status bit 1: the append of a sequence was refused (capacity exceeded, or a
+// sequence index / stored length out of range); its length is unchanged.
+__global__ void bump_lens_kernel(const int32_t* seq_ids, int32_t* lens, int32_t* status, int n_seq,
+                                 int n_tok, int limit, int cache_seqs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_seq) return;
+  const int seq = seq_ids[i];
+  if (seq < 0 || seq >= cache_seqs || lens[seq] < 0 || lens[seq] + n_tok > limit)
+    atomicOr(status, 1);
+  else
+    lens[seq] += n_tok;
+}
+
+// x_hat = nu (Pi^T c + sqrt(pi/2)/m gamma S^T z), fp64 accumulation.
+constexpr int kDeqVecs = 8;
+__global__ void __launch_bounds__(kDim) dequantize_kernel(
+    const uint8_t* codes, const float* norms, const uint8_t* qjl, const float* res, int64_t n,
+    int mse_bits, int mixed, int prod, int code_bytes, const double* pi64, const double* s64,
+    const double* cb64, float* out) {
+  __shared__ double chat[kDeqVecs][kDim];
+  __shared__ double zs[kDeqVecs][kSketch];
+  const int i = threadIdx.x;
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kDeqVecs;
+  for (int v = 0; v < kDeqVecs; ++v) {
+    const int64_t gv = v0 + v;
+    double c = 0.0, z = 0.0;
+    if (gv < n) {
+      const int b = (mixed && i < kDim / 2) ? mse_bits + 1 : mse_bits;
+      if (b > 0) {
+        const int bit = (mixed && i >= kDim / 2) ? (kDim / 2) * (mse_bits + 1) + (i - kDim / 2) * b : i * b;
+        const uint8_t* row = codes + gv * code_bytes;
+        uint32_t w = row[bit >> 3];
+        if ((bit & 7) + b > 8) w |= static_cast<uint32_t>(row[(bit >> 3) + 1]) << 8;
+        const int idx = (w >> (bit & 7)) & ((1u << b) - 1);
+        c = cb64[b * kBookSlots + idx];
+      }
+      if (prod) z = ((qjl[gv * (kSketch / 8) + (i >> 3)] >> (i & 7)) & 1) ? 1.0 : -1.0;
+    }
+    chat[v][i] = c;
+    zs[v][i] = z;
+  }
+  __syncthreads();
+  double acc[kDeqVecs], accz[kDeqVecs];
+  for (int v = 0; v < kDeqVecs; ++v) acc[v] = accz[v] = 0.0;
+  for (int j = 0; j < kDim; ++j) {
+    const double pji = pi64[j * kDim + i];
+    for (int v = 0; v < kDeqVecs; ++v) acc[v] = fma(pji, chat[v][j], acc[v]);
+  }
+  if (prod)
+    for (int l = 0; l < kSketch; ++l) {
+      const double sli = s64[l * kDim + i];
+      for (int v = 0; v < kDeqVecs; ++v) accz[v] = fma(sli, zs[v][l], accz[v]);
+    }
+  const double kappa = 1.2533141373155002512078826424055 / kSketch;  // sqrt(pi/2)/m
+  for (int v = 0; v < kDeqVecs; ++v) {
+    const int64_t gv = v0 + v;
+    if (gv >= n) break;
+    double xh = acc[v];
+    if (prod) xh += kappa * static_cast<double>(res[gv]) * accz[v];
+    out[gv * kDim + i] = static_cast<float>(static_cast<double>(norms[gv]) * xh);
+  }
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+size_t quant_smem(int prod) { return sizeof(SmemQuant) + (prod ? sizeof(SmemProd) : 0); }
+
+tq_status run_quantize(QuantArgs& a, cudaStream_t st) {
+  const size_t smem = quant_smem(a.prod);
+  const int64_t tiles = (a.n + kTile - 1) / kTile;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  cudaError_t e;
+  if (a.x_bf16) {
+    e = cudaFuncSetAttribute(quantize_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) quantize_kernel<1><<<grid, kThreads, smem, st>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(quantize_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) quantize_kernel<0><<<grid, kThreads, smem, st>>>(a);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "quantize kernel launch");
+}
+
+void fill_format(QuantArgs& a, const tq_params* p, const FormatSpec& f) {
+  a.mse_bits = f.mse_bits;
+  a.mixed = f.mixed;
+  a.prod = f.prod;
+  a.code_bytes = f.code_bytes;
+  a.pit = p->pit32;
+  a.mt = p->mt32;
+  a.cb = p->cb32;
+  a.bd = p->bd32;
+}
+
+}  // namespace
+
+tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x, int x_bf16, int64_t n,
+                          const tq_packed* out, cudaStream_t st) {
+  QuantArgs a{};
+  fill_format(a, p, f);
+  a.x = x;
+  a.x_bf16 = x_bf16;
+  a.n = n;
+  a.codes = out->codes;
+  a.norms = out->norms;
+  a.qjl = out->qjl;
+  a.res = out->res_norms;
+  return run_quantize(a, st);
+}
+
+tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* seq_ids, const void* k,
+                        const void* v, int x_bf16, int n_tok, int n_seq, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(n_seq) * n_tok * c->n_kv_heads;
+  for (int which = 0; which < 2; ++which) {
+    const FormatSpec& f = which ? p->fv : p->fk;
+    QuantArgs a{};
+    fill_format(a, p, f);
+    a.x = which ? v : k;
+    a.x_bf16 = x_bf16;
+    a.n = n;
+    a.codes = which ? c->v_codes : c->k_codes;
+    a.norms = which ? c->v_norms : c->k_norms;
+    a.qjl = which ? c->v_qjl : c->k_qjl;
+    a.res = which ? c->v_res_norms : c->k_res_norms;
+    a.append = 1;
+    a.seq_ids = seq_ids;
+    a.lens = c->lens;
+    a.n_tok = n_tok;
+    a.hkv = c->n_kv_heads;
+    a.capacity = c->capacity;
+    a.n_sink = c->n_sink;
+    a.cache_seqs = c->n_seq;
+    a.sink = which ? c->v_sink : c->k_sink;
+    tq_status s = run_quantize(a, st);
+    if (s != TQ_OK) return s;
+  }
+  bump_lens_kernel<<<(n_seq + 127) / 128, 128, 0, st>>>(seq_ids, c->lens, c->status, n_seq, n_tok,
+                                                        c->n_sink + c->capacity, c->n_seq);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "append length update");
+}
+
+tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_packed* in, int64_t n,
+                            float* out, cudaStream_t st) {
+  const int64_t blocks = (n + kDeqVecs - 1) / kDeqVecs;
+  if (blocks > 0x7fffffff) return fail(TQ_ERR_UNSUPPORTED, "tq_dequantize: n too large");
+  dequantize_kernel<<<static_cast<unsigned>(blocks), kDim, 0, st>>>(
+      in->codes, in->norms, in->qjl, in->res_norms, n, f.mse_bits, f.mixed, f.prod, f.code_bytes, p->pi64,
+      p->s64, p->cb64, out);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "dequantize kernel launch");
+}
+
+}  // namespace tq

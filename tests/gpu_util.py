@@ -1,0 +1,126 @@
+"""Helpers shared by the GPU parity tests: build matching GPU / oracle
+parameter sets, move packed rows between the two, and compare results with
+the tolerances of the parity contract."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import online_vector_quantization_b200 as tq
+from oracle import tq_oracle as o
+
+# Tolerances (the parity contract).
+BOUNDARY_EPS = 1e-5        # codes may differ only within this distance of a bound
+MISMATCH_FRACTION = 1e-4   # ... and on fewer than this fraction of coordinates
+DEQUANT_ATOL = 1e-5        # fp32 dequantization on identical packed input
+ATTN_REL_L2 = 2e-3         # decode attention, bf16 queries and outputs
+
+
+def fmt(bits, prod=False, mixed=False):
+    return o.Format(bits, prod=prod, mixed=mixed)
+
+
+def make_params(fk: o.Format, fv: o.Format, seed: int = 0):
+    gp = tq.Params(fk.bits, fv.bits, tq.TQ_MODE_PROD if fk.prod else tq.TQ_MODE_MSE,
+                   tq.TQ_MODE_PROD if fv.prod else tq.TQ_MODE_MSE, int(fk.mixed), int(fv.mixed), seed=seed)
+    op = o.Params(128, fk, fv, seed=seed)
+    return gp, op
+
+
+def widths(f: o.Format):
+    return [f.mse_bits(j, 128) for j in range(128)]
+
+
+def gpu_packed_to_numpy(pk: tq.Packed) -> o.Packed:
+    n = pk.norms.shape[0]
+    codes = pk.codes.cpu().numpy() if pk.codes is not None else np.zeros((n, 0), np.uint8)
+    qjl = pk.qjl.cpu().numpy() if pk.qjl is not None else np.zeros((n, 0), np.uint8)
+    res = pk.res_norms.cpu().numpy() if pk.res_norms is not None else np.zeros(n, np.float32)
+    return o.Packed(codes, pk.norms.cpu().numpy(), qjl, res)
+
+
+def numpy_packed_to_gpu(pk: o.Packed) -> tq.Packed:
+    def t(a, dtype):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dtype=dtype, device="cuda")
+    n = pk.norms.shape[0]
+    return tq.Packed(t(pk.codes, torch.uint8) if pk.codes.shape[1] else None,
+                     t(pk.norms, torch.float32),
+                     t(pk.qjl, torch.uint8) if pk.qjl.shape[1] else None,
+                     t(pk.res_norms, torch.float32) if pk.qjl.shape[1] else None)
+
+
+def rotated_unit(op: o.Params, x: np.ndarray) -> np.ndarray:
+    nu = np.linalg.norm(x, axis=1, keepdims=True)
+    return (x / np.where(nu == 0, 1, nu)) @ op.pi.T
+
+
+def compare_codes(op: o.Params, f: o.Format, x: np.ndarray, got: o.Packed, want: o.Packed):
+    """Codes bit-exact except coordinates within BOUNDARY_EPS of a bound, and
+    those fewer than MISMATCH_FRACTION of all.  Returns the set of vectors
+    whose codes differ (their QJL sketch legitimately differs too)."""
+    w = widths(f)
+    gi = o.unpack_codes(got.codes, w)
+    wi = o.unpack_codes(want.codes, w)
+    bad = np.argwhere(gi != wi)
+    y = rotated_unit(op, x)
+    for v, j in bad:
+        b = op.books[w[j]].bounds
+        assert np.min(np.abs(y[v, j] - b)) < BOUNDARY_EPS, (v, j, y[v, j], gi[v, j], wi[v, j])
+    total = gi.size
+    assert len(bad) <= max(1, MISMATCH_FRACTION * total), (len(bad), total)
+    return set(int(v) for v in bad[:, 0])
+
+
+def compare_qjl(op: o.Params, f: o.Format, x: np.ndarray, got: o.Packed, want: o.Packed, skip: set):
+    if not f.prod:
+        return
+    gb = o.unpack_codes(got.qjl, [1] * 128)
+    wb = o.unpack_codes(want.qjl, [1] * 128)
+    # S r in fp64 from the oracle's own codes
+    chat = np.zeros((x.shape[0], 128))
+    wi = o.unpack_codes(want.codes, widths(f)) if want.codes.shape[1] else None
+    for j, wj in enumerate(widths(f)):
+        if wj:
+            chat[:, j] = op.books[wj].centroids[wi[:, j]]
+    nu = np.linalg.norm(x, axis=1, keepdims=True)
+    u = x / np.where(nu == 0, 1, nu)
+    proj = (u - chat @ op.pi) @ op.s.T
+    for v, i in np.argwhere(gb != wb):
+        if int(v) in skip:
+            continue
+        assert abs(proj[v, i]) < BOUNDARY_EPS, (v, i, proj[v, i])
+    keep = np.array([v not in skip for v in range(x.shape[0])])
+    assert np.allclose(got.res_norms[keep], want.res_norms[keep], rtol=1e-5, atol=1e-6)
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def fill_cache_from_oracle(cache: tq.Cache, op: o.Params, ocache: o.Cache, lens, B, hkv):
+    """Write oracle-packed rows and bf16 sink rows into a GPU cache."""
+    gp_planes = {}
+    for name, dtype, elems in (("k_codes", torch.uint8, op.fmt_k.code_bytes(128)),
+                               ("v_codes", torch.uint8, op.fmt_v.code_bytes(128)),
+                               ("k_norms", torch.float32, 1), ("v_norms", torch.float32, 1),
+                               ("k_qjl", torch.uint8, 16), ("v_qjl", torch.uint8, 16),
+                               ("k_res_norms", torch.float32, 1), ("v_res_norms", torch.float32, 1),
+                               ("k_sink", torch.bfloat16, 128), ("v_sink", torch.bfloat16, 128)):
+        gp_planes[name] = cache.plane(name, dtype, elems)
+    for b in range(B):
+        for h in range(hkv):
+            ns = min(cache.n_sink, lens[b])
+            nq = lens[b] - ns
+            for side, rows, sink in (("k", ocache.k_rows[b, h], ocache.k_sink[b, h]),
+                                     ("v", ocache.v_rows[b, h], ocache.v_sink[b, h])):
+                if gp_planes[side + "_codes"] is not None and rows.codes.shape[1]:
+                    gp_planes[side + "_codes"][b, h, :nq] = torch.from_numpy(rows.codes[:nq]).cuda()
+                gp_planes[side + "_norms"][b, h, :nq, 0] = torch.from_numpy(rows.norms[:nq]).cuda()
+                if gp_planes[side + "_qjl"] is not None:
+                    gp_planes[side + "_qjl"][b, h, :nq] = torch.from_numpy(rows.qjl[:nq]).cuda()
+                    gp_planes[side + "_res_norms"][b, h, :nq, 0] = torch.from_numpy(rows.res_norms[:nq]).cuda()
+                if ns:
+                    gp_planes[side + "_sink"][b, h, :ns] = torch.from_numpy(sink[:ns]).to(torch.bfloat16).cuda()
+    cache.lens.copy_(torch.tensor(lens, dtype=torch.int32))

@@ -1,0 +1,61 @@
+"""Host-side checks of libtq (no GPU needed): the library loads, exports every
+entry point include/tq.h declares, rejects bad arguments, and its host tables
+(an independent second implementation) agree with the oracle."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import online_vector_quantization_b200 as tq
+from oracle import tq_oracle as o
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "tq.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(tq._lib, n), n
+        assert n in tq.EXPORTED, n
+
+
+@pytest.mark.parametrize("d,b", [(128, 1), (128, 2), (128, 3), (128, 4), (64, 3), (256, 2)])
+def test_codebook_matches_oracle(d, b):
+    c, t = tq.tq_codebook(d, b)
+    ref = o.lloyd_max(d, b)
+    assert np.max(np.abs(c - ref.centroids)) < 1e-12
+    assert np.max(np.abs(t - ref.bounds)) < 1e-12
+
+
+@pytest.mark.parametrize("seed,d", [(0, 128), (12345, 128), (7, 16)])
+def test_rotation_matches_oracle(seed, d):
+    assert np.max(np.abs(tq.tq_rotation(seed, d) - o.rotation(seed, d))) < 1e-12
+
+
+def test_qjl_matrix_matches_oracle():
+    assert np.max(np.abs(tq.tq_qjl_matrix(3, 128, 128) - o.qjl_matrix(3, 128, 128))) < 1e-14
+
+
+def test_host_argument_errors():
+    with pytest.raises(tq.TqError) as e:
+        tq.tq_codebook(2, 3)
+    assert e.value.status == 1
+    with pytest.raises(tq.TqError) as e:
+        tq.Params(3, 3, d=64)
+    assert e.value.status == 2
+    with pytest.raises(tq.TqError) as e:
+        tq.Params(5, 3)
+    assert e.value.status == 2
+    with pytest.raises(tq.TqError) as e:
+        tq.Params(3, 3, mixed_k=1, mode_k=tq.TQ_MODE_PROD)
+    assert e.value.status == 2
+    assert tq._lib.tq_cache_bytes(None, 1, 1, 64, 0) == 0
+    assert tq._lib.tq_decode_workspace_bytes(None, 1, 8, 8, 128) == 0
