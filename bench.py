@@ -1,0 +1,489 @@
+"""Benchmark of the TurboQuant KV-cache path on B200.
+
+One step = one pass of the hot path over one batch: a 64-token bf16 chunk is
+appended to every sequence (fused rotate / quantize / pack / append) and one
+decode-attention step runs over the packed cache.  Workload (streaming append
++ decode): 16 sequences, contexts uniform in [8192, 65536], 8 kv-heads and 32
+query heads of d = 128, mixed 3.5-bit keys and values (64 rotated channels at
+4 bits, 64 at 3 bits).  The cache read per step (~570 MB) is larger than L2.
+
+`value` is the packed-KV throughput of the whole step in GB/s: algorithmic
+bytes (chunk read + packed rows written + packed cache, queries and outputs
+read/written by the decode) over the step time.  Auxiliary measurements of
+the other workloads (quantize sweep, prod-mode GQA decode, long-context
+asymmetric decode with sink and sparse V, tiny fp32 case) ride along.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 launch with torch.distributed.run: every rank runs its own copy of
+the workload (independent sequences, no data exchange: weak scaling); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_SEQ, HKV, HQ, D, CHUNK = 16, 8, 32, 128, 64
+LEN_LO, LEN_HI = 8192, 65536
+ROW_BYTES = 56 + 4  # mixed 3.5-bit code row + fp32 norm, per K or V
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device):
+    """Config: streaming append + decode.  Returns the state the step uses."""
+    lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", rank))
+    params = tq.Params(3, 3, mixed_k=1, mixed_v=1, seed=0)
+    cap = ((max(lens) + (n_steps + 1) * CHUNK + 63) // 64) * 64
+    cache = tq.Cache(params, N_SEQ, HKV, cap, 0, device=device)
+    # prefill (untimed): the prefix of each sequence through tq_append
+    for s, n in enumerate(lens):
+        ids = torch.tensor([s], dtype=torch.int32, device=device)
+        done = 0
+        while done < n:
+            m = min(16384, n - done)
+            k = kv_inputs.kv_vectors(m * HKV, D, key=("stream-k", rank, s, done), device=device,
+                                     dtype=torch.bfloat16).view(1, m, HKV, D)
+            v = kv_inputs.kv_vectors(m * HKV, D, key=("stream-v", rank, s, done), device=device,
+                                     dtype=torch.bfloat16).view(1, m, HKV, D)
+            tq.tq_append(params, cache, ids, k, v)
+            done += m
+    torch.cuda.synchronize()
+    assert cache.lens.cpu().tolist() == lens
+    chunks_k = [kv_inputs.kv_vectors(N_SEQ * CHUNK * HKV, D, key=("chunk-k", rank, i), device=device,
+                                     dtype=torch.bfloat16).view(N_SEQ, CHUNK, HKV, D) for i in range(n_steps)]
+    chunks_v = [kv_inputs.kv_vectors(N_SEQ * CHUNK * HKV, D, key=("chunk-v", rank, i), device=device,
+                                     dtype=torch.bfloat16).view(N_SEQ, CHUNK, HKV, D) for i in range(n_steps)]
+    qs = [kv_inputs.queries((N_SEQ, HQ, D), key=("stream-q", rank, i), device=device) for i in range(n_steps)]
+    ids = torch.arange(N_SEQ, dtype=torch.int32, device=device)
+    ws = tq.decode_workspace(params, N_SEQ, HQ, HKV, cap, device=device)
+    out = torch.empty(N_SEQ, HQ, D, dtype=torch.bfloat16, device=device)
+    return dict(params=params, cache=cache, lens=lens, cap=cap, ck=chunks_k, cv=chunks_v, qs=qs, ids=ids, ws=ws,
+                out=out)
+
+
+def step_bytes(lens_now):
+    append = 2 * N_SEQ * CHUNK * HKV * D * 2 + 2 * N_SEQ * CHUNK * HKV * ROW_BYTES
+    decode = sum(HKV * (n + CHUNK) * 2 * ROW_BYTES for n in lens_now) + 2 * N_SEQ * HQ * D * 2
+    return append, decode
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import kv_inputs
+    import online_vector_quantization_b200 as tq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device, timeout=__import__("datetime").timedelta(seconds=300))
+    n_steps = args.warmup + args.steps
+    st = build_stream_workload(tq, torch, kv_inputs, rank, n_steps, device)
+    params, cache = st["params"], st["cache"]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        tq.tq_append(params, cache, st["ids"], st["ck"][i], st["cv"][i])
+        ev_d0.record(stream)
+        tq.tq_decode_attn(params, st["qs"][i], cache, st["cap"], st["out"], st["ws"])
+        ev_d1.record(stream)
+
+    ev_d0, ev_d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    lens_at_timing = [n + args.warmup * CHUNK for n in st["lens"]]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    d_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for j in range(args.steps):
+        ev_d0, ev_d1 = d_events[j]
+        step(args.warmup + j)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    decode_ms = [a.elapsed_time(b) for a, b in d_events]
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    append_b, decode_b = 0, 0
+    for j in range(args.steps):
+        a, d = step_bytes([n + j * CHUNK for n in lens_at_timing])
+        append_b += a
+        decode_b += d
+    ms_per_step = total_ms / args.steps
+    value = (append_b + decode_b) * world / (total_ms * 1e-3) / 1e9
+    assert int(cache.status.item()) == 0
+
+    # e2e: same step through the public API from pinned host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        e2e = run_e2e(tq, torch, kv_inputs, args, st, rank, device, world)
+
+    peak, peak_kind = peaks()
+    avg_decode_s = sum(decode_ms) / len(decode_ms) * 1e-3
+    decode_bytes_per_launch = decode_b / args.steps
+    achieved = decode_bytes_per_launch / avg_decode_s / 1e9
+    aux = {} if args.no_aux or rank != 0 else run_aux(tq, torch, kv_inputs, device, args)
+    cpu = None if (rank != 0 or world > 1 or args.no_cpu) else cpu_baseline_stream(args)
+    if rank == 0:
+        line = {
+            "metric": "decode-attn packed-KV GB/s (streaming append + decode step)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc", "data": "synthetic",
+            "config": {"workload": "streaming append + decode: 16 seqs, ctx U[8192,65536], 64-token bf16 chunk "
+                                   "appended (fused rotate/quantize/pack), 1 decode step, mixed 3.5-bit K/V, "
+                                   "32 q / 8 kv heads, d=128",
+                       "seq_lens": st["lens"], "l2": "inputs larger than L2 (cache read ~570 MB per step)",
+                       "tokens_per_s_per_seq": round(1000.0 / ms_per_step, 2),
+                       "decode_ms": round(avg_decode_s * 1e3, 4),
+                       "append_plus_decode_bytes_per_step": (append_b + decode_b) // args.steps,
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"kernel": "decode_kernel<mixed3.5,mixed3.5> (+qrot)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "bytes_per_launch": int(decode_bytes_per_launch), "traffic": args.traffic},
+            "clocks": clocks,
+            "gpu_launches": args.steps * 5,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "aux": aux,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
+    import torch.distributed as dist
+    params, cache = st["params"], st["cache"]
+    stream = torch.cuda.current_stream()
+    hk = [t.cpu().pin_memory() for t in st["ck"][:args.steps]]
+    hv = [t.cpu().pin_memory() for t in st["cv"][:args.steps]]
+    hq = [t.cpu().pin_memory() for t in st["qs"][:args.steps]]
+    hout = torch.empty(N_SEQ, HQ, D, dtype=torch.bfloat16).pin_memory()
+    dk = torch.empty_like(st["ck"][0])
+    dv = torch.empty_like(st["cv"][0])
+    dq = torch.empty_like(st["qs"][0])
+    # rewind the lengths so the e2e steps see the same contexts as the timed ones
+    lens0 = torch.tensor([n + args.warmup * CHUNK for n in st["lens"]], dtype=torch.int32, device=device)
+    cache.lens.copy_(lens0)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for j in range(args.steps):
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dq.copy_(hq[j], non_blocking=True)
+        tq.tq_append(params, cache, st["ids"], dk, dv)
+        tq.tq_decode_attn(params, dq, cache, st["cap"], st["out"], st["ws"])
+        hout.copy_(st["out"], non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    total = 0
+    for j in range(args.steps):
+        a, d = step_bytes([n + (args.warmup + j) * CHUNK for n in st["lens"]])
+        total += a + d
+    h2d = 2 * N_SEQ * CHUNK * HKV * D * 2 + N_SEQ * HQ * D * 2
+    return {"value": round(total * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms / args.steps, 4),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": N_SEQ * HQ * D * 2}
+
+
+def _flush_l2(torch, buf):
+    buf.add_(1)
+
+
+def _time_call(torch, fn, iters, flush=None):
+    """Median device time (ms) of fn over iters calls, L2 flushed between calls."""
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(iters):
+        if flush is not None:
+            _flush_l2(torch, flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def run_aux(tq, torch, kv_inputs, device, args):
+    """The other workloads, measured on the same GPU in the same run."""
+    out = {}
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MB > L2
+    iters = 10
+    # quantize sweep: 32 kv-heads x 32768 tokens, bf16 with 4 outlier channels
+    n = 32 * 32768
+    x = kv_inputs.kv_vectors(n, D, key="sweep", device=device, dtype=torch.bfloat16, outliers=True)
+    sweep = {}
+    for mode, name in ((tq.TQ_MODE_MSE, "mse"), (tq.TQ_MODE_PROD, "prod")):
+        for b in (1, 2, 3, 4):
+            p = tq.Params(b, b, mode, mode)
+            pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
+            ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
+            cb, qb = p.row_bytes(tq.TQ_K)
+            by = n * (D * 2 + cb + 4 + (qb + 4 if qb else 0))
+            sweep[f"{name}{b}"] = {"mvec_per_s": round(n / (ms * 1e-3) / 1e6, 1), "ms": round(ms, 4),
+                                   "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1)}
+    out["quantize_sweep_1M_bf16"] = sweep
+    del x
+    # GQA decode, prod mode: B=1, 32 q / 8 kv heads, T=32768, K/V 3-bit (2-bit MSE + QJL)
+    T = 32768
+    p = tq.Params(3, 3, tq.TQ_MODE_PROD, tq.TQ_MODE_PROD)
+    cache = tq.Cache(p, 1, 8, T, 0, device=device)
+    k = kv_inputs.kv_vectors(T * 8, D, key="c3k", device=device).view(1, T, 8, D)
+    v = kv_inputs.kv_vectors(T * 8, D, key="c3v", device=device).view(1, T, 8, D)
+    tq.tq_append(p, cache, torch.zeros(1, dtype=torch.int32, device=device), k, v)
+    q = kv_inputs.queries((1, 32, D), key="c3q", device=device)
+    ws = tq.decode_workspace(p, 1, 32, 8, T, device=device)
+    o = torch.empty(1, 32, D, dtype=torch.bfloat16, device=device)
+    ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, T, o, ws), iters, flush)
+    by = 8 * T * 2 * (32 + 16 + 8)
+    out["decode_prod3_gqa_T32k"] = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1),
+                                    "bytes": by, "l2": "flushed between calls"}
+    del cache, k, v
+    # long-context asymmetric: B=4, 64 q / 8 kv, T=131072, sink 128 bf16, K4/V3, sparse V 1e-6
+    T = 131072
+    p = tq.Params(4, 3)
+    cache = tq.Cache(p, 4, 8, T - 128, 128, device=device)
+    q = kv_inputs.queries((4, 64, D), key="c4q", device=device)
+    for s in range(4):
+        ids = torch.tensor([s], dtype=torch.int32, device=device)
+        ks, vs = [], []
+        for h in range(8):
+            kk = kv_inputs.kv_vectors(T, D, key=("c4k", s, h), device=device, dtype=torch.bfloat16)
+            kk = kv_inputs.planted_keys(kk, q[s, 8 * h:8 * h + 8], 8, 128, key=("c4p", s, h))
+            ks.append(kk)
+            vs.append(kv_inputs.kv_vectors(T, D, key=("c4v", s, h), device=device, dtype=torch.bfloat16))
+        kt = torch.stack(ks, 1).view(1, T, 8, D)
+        vt = torch.stack(vs, 1).view(1, T, 8, D)
+        del ks, vs
+        for c0 in range(0, T, 32768):
+            tq.tq_append(p, cache, ids, kt[:, c0:c0 + 32768].contiguous(), vt[:, c0:c0 + 32768].contiguous())
+        del kt, vt
+    ws = tq.decode_workspace(p, 4, 64, 8, T, device=device)
+    o = torch.empty(4, 64, D, dtype=torch.bfloat16, device=device)
+    for thr, name in ((1e-6, "sparse_v"), (0.0, "dense")):
+        ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, T, o, ws, thr), iters, flush)
+        by = 4 * 8 * ((T - 128) * (68 + 52) + 128 * 512)
+        out[f"decode_k4v3_sink_T128k_{name}"] = {"ms": round(ms, 4), "gb_per_s_dense_equiv": round(by / (ms * 1e-3) / 1e9, 1),
+                                                 "dense_bytes": by}
+    assert int(cache.status.item()) == 0
+    del cache
+    # tiny fp32 case: 4096 vectors, b=3, 1 head
+    p = tq.Params(3, 3)
+    x = kv_inputs.kv_vectors(4096, D, key="c1", device=device)
+    cache = tq.Cache(p, 1, 1, 4096, 0, device=device)
+    tq.tq_append(p, cache, torch.zeros(1, dtype=torch.int32, device=device), x.view(1, 4096, 1, D), x.view(1, 4096, 1, D))
+    q = kv_inputs.queries((1, 1, D), key="c1q", device=device, dtype=torch.float32)
+    ws = tq.decode_workspace(p, 1, 1, 1, 4096, device=device)
+    o = torch.empty(1, 1, D, dtype=torch.float32, device=device)
+    ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, 4096, o, ws), iters)
+    out["decode_tiny_fp32_T4096"] = {"ms": round(ms, 4)}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Oracle timing (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_unit_sample(n_units: int):
+    """Build oracle state for n_units (sequence, kv-head) units of the
+    streaming workload (untimed) and return a function doing one step on them:
+    quantize a 64-token chunk of K and V and decode the unit's 4 query heads."""
+    import numpy as np
+    import torch
+
+    import kv_inputs
+    from oracle import tq_oracle as o
+
+    lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", 0))
+    f = o.Format(3, mixed=True)
+    op = o.Params(128, f, f)
+    units = []
+    for u in range(n_units):
+        s = u % N_SEQ
+        n = lens[s]
+        k = kv_inputs.kv_vectors(n, D, key=("oracle-k", s, u), dtype=torch.bfloat16).double().numpy()
+        v = kv_inputs.kv_vectors(n, D, key=("oracle-v", s, u), dtype=torch.bfloat16).double().numpy()
+        ck = kv_inputs.kv_vectors(CHUNK, D, key=("oracle-ck", s, u), dtype=torch.bfloat16).double().numpy()
+        cv = kv_inputs.kv_vectors(CHUNK, D, key=("oracle-cv", s, u), dtype=torch.bfloat16).double().numpy()
+        q = kv_inputs.queries((1, HQ // HKV, D), key=("oracle-q", s, u)).double().numpy()
+        cache = o.cache_from_vectors(op, k[None, None], v[None, None], 0)
+        units.append((n, ck, cv, q, cache))
+
+    def one_step():
+        nbytes = 0
+        for n, ck, cv, q, cache in units:
+            kr, vr = o.quantize(op, ck, "k"), o.quantize(op, cv, "v")
+            c = o.Cache(0)
+            c.k_sink[0, 0] = c.v_sink[0, 0] = np.zeros((0, D))
+            c.k_rows[0, 0] = o.Packed(np.concatenate([cache.k_rows[0, 0].codes, kr.codes]),
+                                      np.concatenate([cache.k_rows[0, 0].norms, kr.norms]), np.zeros((n + CHUNK, 0), np.uint8),
+                                      np.zeros(n + CHUNK, np.float32))
+            c.v_rows[0, 0] = o.Packed(np.concatenate([cache.v_rows[0, 0].codes, vr.codes]),
+                                      np.concatenate([cache.v_rows[0, 0].norms, vr.norms]), np.zeros((n + CHUNK, 0), np.uint8),
+                                      np.zeros(n + CHUNK, np.float32))
+            o.decode_attention(op, q, c, [n + CHUNK], 1)
+            nbytes += 2 * CHUNK * D * 2 + 2 * CHUNK * ROW_BYTES + (n + CHUNK) * 2 * ROW_BYTES + 2 * (HQ // HKV) * D * 2
+        return nbytes
+
+    return one_step
+
+
+def _threads():
+    try:
+        import numpy  # noqa: F401
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_stream(args):
+    step = _oracle_unit_sample(args.cpu_units)
+    t = time.perf_counter()
+    nbytes = step()
+    dt = time.perf_counter() - t
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{args.cpu_units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step "
+                      f"(64-token append + 4-head decode each), fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    step = _oracle_unit_sample(args.cpu_units)
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += step()
+    dt = time.perf_counter() - t
+    value = nbytes / dt / 1e9
+    sample = (f"{args.cpu_units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step per step "
+              "(64-token append + 4-head decode each), fp64 numpy oracle on host cores")
+    line = {"impl": "reference", "metric": "decode-attn packed-KV GB/s (streaming append + decode step)",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "streaming append + decode: 16 seqs, ctx U[8192,65536], 64-token bf16 chunk, "
+                                   "mixed 3.5-bit K/V, 32 q / 8 kv heads, d=128 (bounded sample)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--no-aux", action="store_true", help="skip the auxiliary workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--cpu-units", type=int, default=2)
+    ap.add_argument("--traffic", type=float, default=None, help=argparse.SUPPRESS)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

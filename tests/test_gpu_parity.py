@@ -76,6 +76,9 @@ def _decode_case(fk, fv, B, hq, hkv, T, lens, n_sink, thr, q_dtype=torch.bfloat1
     torch.cuda.synchronize()
     got = out.float().cpu().numpy()
     assert int(cache.status.item()) == 0
+    if out_dtype == torch.bfloat16:
+        floor = gu.rel_l2(torch.from_numpy(want).to(torch.bfloat16).double().numpy(), want)
+        print(f"decode rel L2 {gu.rel_l2(got, want):.3e} (bf16 rounding of the exact output alone: {floor:.3e})")
     return got, want, (gp, op, cache, ws, q, out, max_len)
 
 
