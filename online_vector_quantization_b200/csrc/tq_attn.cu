@@ -41,7 +41,11 @@ constexpr int kTok = 16;       // tokens per warp tile
 constexpr int kMaxG = 8;       // query heads per kv-head (MMA N = 8)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kQjlScale = 1.2533141373155003f / kSketch;  // sqrt(pi/2)/m
-constexpr int kQfragWords = 2 * 16 * 32;                    // [kstep 16][b0,b1][lane 32]
+// Query fragments per (sequence, kv-head): [kstep 16][b0,b1][hi,lo][lane 32].
+// The rotated query is split as hi = fp16(x), lo = fp16(x - hi), and both
+// halves are multiplied with the same code fragment, so the query enters the
+// scores with fp32-level accuracy.
+constexpr int kQfragWords = 16 * 2 * 2 * 32;
 
 // ---------------------------------------------------------------------------
 // Formats (id = mse_bits | mixed << 3 | prod << 4).  Segments of the MSE row:
@@ -60,6 +64,7 @@ struct Fmt {
   static constexpr int b1 = mse;
   static constexpr int byte1 = mixed ? 8 * (mse + 1) : 0;
   static constexpr bool uses(int b) { return (nseg > 0 && b0 == b) || (nseg > 1 && b1 == b); }
+  __host__ __device__ static constexpr int width(int j) { return (mixed && j < 64) ? mse + 1 : mse; }
 };
 
 // Shared-memory lookup tables.  Region A (row stride 256 B): bytes [0,128) of
@@ -318,7 +323,8 @@ struct DecodeArgs {
   const float* st;   // S^T
   const float* pi;   // Pi
   const float* s;    // S
-  const float* cb;   // centroids [5][16]
+  const float* cbs;  // sigma-scaled centroids [5][16] (the values the MMAs see)
+  const float* sig;  // sigma per width [5]
   float sparse_thr;
 };
 
@@ -351,14 +357,15 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
       acc = fmaf(a.pit[k * kDim + j], qs[h][k], acc);
       if (FK::prod) acs = fmaf(a.st[k * kSketch + j], qs[h][k], acs);
     }
-    qt[h][j] = acc * scale;
+    const int wj = FK::width(j);
+    qt[h][j] = wj > 0 ? acc * scale / a.sig[wj] : 0.f;
     qsk[h][j] = acs * scale;
   }
   __syncthreads();
   // B fragments: lane (g, t) supplies head g; k-steps 0..7 from the MSE
   // segments, 8..15 from the QJL segment.
   uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  for (int i = tid; i < kQfragWords / 2; i += kThreads) {
+  for (int i = tid; i < 16 * 32; i += kThreads) {
     const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
     int dims[4] = {0, 0, 0, 0};
     const float* src = qt[g];
@@ -376,13 +383,20 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
       for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
       src = qsk[g];
     }
-    uint32_t b0 = 0, b1 = 0;
+    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
     if (valid) {
-      b0 = h2bits(src[dims[0]], src[dims[1]]);
-      b1 = h2bits(src[dims[2]], src[dims[3]]);
+      for (int r = 0; r < 2; ++r) {
+        const float x0 = src[dims[2 * r]], x1 = src[dims[2 * r + 1]];
+        const __half2 h = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(h);
+        hi[r] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[r] = h2bits(x0 - hf.x, x1 - hf.y);
+      }
     }
-    dst[(ks * 2 + 0) * 32 + lane] = b0;
-    dst[(ks * 2 + 1) * 32 + lane] = b1;
+    for (int r = 0; r < 2; ++r) {
+      dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
+      dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
+    }
   }
 }
 
@@ -390,8 +404,9 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
 // Split merge (last CTA of a (sequence, kv-head)): combine the partials and
 // apply Pi^T (and S^T) once per output.
 // ---------------------------------------------------------------------------
-template <bool VPROD>
+template <int VF>
 __device__ void merge_unit(const DecodeArgs& a, int b, int kvh, int n_real, bool has_sink, float* sm) {
+  constexpr bool VPROD = Fmt<VF>::prod;
   const int tid = threadIdx.x, G = a.group;
   const int PF = a.part_floats;
   const float* base = a.parts + (static_cast<int64_t>(b) * a.hkv + kvh) * (a.n_splits + 1) * kMaxG * PF;
@@ -424,6 +439,7 @@ __device__ void merge_unit(const DecodeArgs& a, int b, int kvh, int n_real, bool
       const float* pp = base + (sp * kMaxG + h) * PF;
       s += __ldcg(pp + 2 + j) * exp2f(__ldcg(pp) - mm[h]);
     }
+    if (j < kDim) s = Fmt<VF>::width(j) > 0 ? s / a.sig[Fmt<VF>::width(j)] : 0.f;
     acc[h * 2 * kDim + j] = s;
   }
   for (int i = tid; i < G * kDim; i += kThreads) {
@@ -457,7 +473,7 @@ __device__ void merge_unit(const DecodeArgs& a, int b, int kvh, int n_real, bool
 }
 
 // Publish this CTA's partial; the CTA that completes the set merges.
-template <bool VPROD>
+template <int VF>
 __device__ void finish_cta(const DecodeArgs& a, int b, int kvh, int expected, int n_real, bool has_sink,
                            float* sm) {
   __shared__ int s_last;
@@ -471,7 +487,7 @@ __device__ void finish_cta(const DecodeArgs& a, int b, int kvh, int expected, in
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  merge_unit<VPROD>(a, b, kvh, n_real, has_sink, sm);
+  merge_unit<VF>(a, b, kvh, n_real, has_sink, sm);
   if (threadIdx.x == 0) *ticket = 0;  // leave the workspace ready for the next call
 }
 
@@ -479,7 +495,7 @@ __device__ void finish_cta(const DecodeArgs& a, int b, int kvh, int expected, in
 // 2. decode kernel
 // ---------------------------------------------------------------------------
 template <int KF, int VF>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1 : 2) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
   using KR = KRow<KF>;
@@ -568,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       part_base[(a.n_splits * kMaxG + tid) * PF + 1] = red[2 * tid + 1];
     }
     __syncthreads();
-    finish_cta<FV::prod>(a, b, kvh, expected, n_real, has_sink, sm);
+    finish_cta<VF>(a, b, kvh, expected, n_real, has_sink, sm);
     return;
   }
 
@@ -577,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   // ---- quantized split ----------------------------------------------------
   // lookup tables
   {
-    const float* cb = a.cb;
+    const float* cb = a.cbs;
     if constexpr (L::t4) {
       for (int i = tid; i < 256 * 32; i += kThreads) {
         const int r = i >> 5, ln = i & 31;
@@ -603,22 +619,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   const unsigned char* lut_a = smem;
   const unsigned char* lut_b = smem + L::region_b_off;
   const uint32_t lane4 = lane * 4, lane8 = lane * 8;
-  const uint32_t c1k = FK::mse == 1 ? h2bits(a.cb[1 * kBookSlots + 1], a.cb[1 * kBookSlots + 1]) : 0u;
-  const uint32_t c1v = FV::mse == 1 ? h2bits(a.cb[1 * kBookSlots + 1], a.cb[1 * kBookSlots + 1]) : 0u;
+  const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
+  const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
 
   // query B-fragments
   const uint32_t* qf = a.qfrag + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  uint32_t bq[8][2], bqs[8][2];
+  uint32_t bq[8][2][2], bqs[8][2][2];  // [kstep][b0,b1][hi,lo]
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    bq[s][0] = qf[(s * 2 + 0) * 32 + lane];
-    bq[s][1] = qf[(s * 2 + 1) * 32 + lane];
-    if constexpr (FK::prod) {
-      bqs[s][0] = qf[((8 + s) * 2 + 0) * 32 + lane];
-      bqs[s][1] = qf[((8 + s) * 2 + 1) * 32 + lane];
-    }
-  }
+  for (int s = 0; s < 8; ++s)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        bq[s][r][x] = qf[((s * 2 + r) * 2 + x) * 32 + lane];
+        if constexpr (FK::prod) bqs[s][r][x] = qf[(((8 + s) * 2 + r) * 2 + x) * 32 + lane];
+      }
   __syncthreads();
 
   constexpr int VMT = 8 + (FV::prod ? 8 : 0);  // m-tiles of the V accumulator
@@ -699,7 +715,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         uint32_t la, ha, lb, hb;
         k0A.decode(s, lk, lane4, lane8, c1k, la, ha);
         k0B.decode(s, lk, lane4, lane8, c1k, lb, hb);
-        mma16816(sc, la, lb, ha, hb, bq[s][0], bq[s][1]);
+        mma16816(sc, la, lb, ha, hb, bq[s][0][0], bq[s][1][0]);
+        mma16816(sc, la, lb, ha, hb, bq[s][0][1], bq[s][1][1]);
       }
     }
     if constexpr (FK::nseg > 1) {
@@ -708,7 +725,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         uint32_t la, ha, lb, hb;
         k1A.decode(s, lut_a, lane4, lane8, c1k, la, ha);
         k1B.decode(s, lut_a, lane4, lane8, c1k, lb, hb);
-        mma16816(sc, la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0], bq[KR::S0::KSTEPS + s][1]);
+        mma16816(sc, la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][0], bq[KR::S0::KSTEPS + s][1][0]);
+        mma16816(sc, la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][1], bq[KR::S0::KSTEPS + s][1][1]);
       }
     }
     if constexpr (FK::prod) {
@@ -717,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         uint32_t la, ha, lb, hb;
         kqA.decode(s, lut_a, lane4, lane8, one2, la, ha);
         kqB.decode(s, lut_a, lane4, lane8, one2, lb, hb);
-        mma16816(sq, la, lb, ha, hb, bqs[s][0], bqs[s][1]);
+        mma16816(sq, la, lb, ha, hb, bqs[s][0][0], bqs[s][1][0]);
+        mma16816(sq, la, lb, ha, hb, bqs[s][0][1], bqs[s][1][1]);
       }
     }
     // s (base 2): c0,c1 = token g, heads 2t, 2t+1; c2,c3 = token g+8
@@ -865,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
-  finish_cta<FV::prod>(a, b, kvh, expected, n_real, has_sink, sm);
+  finish_cta<VF>(a, b, kvh, expected, n_real, has_sink, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -967,7 +986,8 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.st = p->st32;
   a.pi = p->pi32;
   a.s = p->s32;
-  a.cb = p->cb32;
+  a.cbs = p->cbs32;
+  a.sig = p->sig32;
   a.sparse_thr = sparse_thr;
   const int sink_floats = kMaxG * kDim + kMaxG * c->n_sink + 2 * kMaxG + 64;
 

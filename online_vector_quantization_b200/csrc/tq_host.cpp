@@ -198,6 +198,38 @@ static tq_status lloyd_max(int d, int bits, double* centroids, double* bounds) {
   return TQ_OK;
 }
 
+// Round a positive double to the nearest fp16 value (normal range).
+static double round_to_f16(double v) {
+  int e = 0;
+  std::frexp(v, &e);                       // v = m 2^e, m in [0.5, 1)
+  const double ulp = std::ldexp(1.0, e - 11);  // 11 significant bits
+  return std::nearbyint(v / ulp) * ulp;
+}
+
+// Scale sigma for one codebook: the MMAs see sigma * c_k in fp16 and the
+// result is divided by sigma in fp32, so pick sigma (a power of two times a
+// factor in [1, 2), searched on a grid) that makes every centroid nearly
+// exact in fp16.  One-bit codebooks get sigma = 1/c_1 (values exactly +-1).
+static double codebook_sigma(const double* c, int levels) {
+  double cmax = 0.0;
+  for (int k = 0; k < levels; ++k) cmax = std::max(cmax, std::fabs(c[k]));
+  if (levels == 2) return 1.0 / cmax;
+  int e = 0;
+  std::frexp(cmax, &e);
+  const double base = std::ldexp(1.0, 1 - e);  // cmax * base in [1, 2)
+  double best_err = 1e300, best = base;
+  for (int i = 0; i < (1 << 16); ++i) {
+    const double sg = base * (1.0 + i / 65536.0);
+    double err = 0.0;
+    for (int k = 0; k < levels; ++k) {
+      const double v = std::fabs(c[k]) * sg;
+      err = std::max(err, std::fabs(round_to_f16(v) - v) / v);
+    }
+    if (err < best_err) { best_err = err; best = sg; }
+  }
+  return best;
+}
+
 static bool make_format(int bits, int mode, int mixed, FormatSpec* f, std::string* why) {
   if (mode != TQ_MODE_MSE && mode != TQ_MODE_PROD) { *why = "mode must be MSE or PROD"; return false; }
   if (bits < 1 || bits > 4) { *why = "bits must be in 1..4"; return false; }
@@ -266,6 +298,7 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   // host staging of every device table
   std::vector<float> pi32(d * d), pit32(d * d), s32(m * d), st32(d * m), mt32(d * m);
   std::vector<float> cb32((kMaxBits + 1) * kBookSlots, 0.f), bd32((kMaxBits + 1) * kBookSlots, 0.f);
+  std::vector<float> cbs32((kMaxBits + 1) * kBookSlots, 0.f), sig32(kMaxBits + 1, 1.f);
   std::vector<double> cb64((kMaxBits + 1) * kBookSlots, 0.0);
   for (int r = 0; r < d; ++r)
     for (int c = 0; c < d; ++c) {
@@ -290,8 +323,11 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
     if (!used) continue;
     double c[16], t[15];
     lloyd_max(d, b, c, t);
+    const double sg = codebook_sigma(c, 1 << b);
+    sig32[b] = static_cast<float>(sg);
     for (int k = 0; k < (1 << b); ++k) {
       cb32[b * kBookSlots + k] = static_cast<float>(c[k]);
+      cbs32[b * kBookSlots + k] = static_cast<float>(c[k] * static_cast<double>(sig32[b]));
       cb64[b * kBookSlots + k] = c[k];
     }
     for (int k = 0; k + 1 < (1 << b); ++k) bd32[b * kBookSlots + k] = static_cast<float>(t[k]);
@@ -304,7 +340,7 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   size_t o_pi = take(pi32.size() * 4), o_pit = take(pit32.size() * 4), o_s = take(s32.size() * 4),
          o_st = take(st32.size() * 4), o_mt = take(mt32.size() * 4), o_pi64 = take(p->pi.size() * 8),
          o_s64 = take(p->s.size() * 8), o_cb = take(cb32.size() * 4), o_bd = take(bd32.size() * 4),
-         o_cb64 = take(cb64.size() * 8);
+         o_cb64 = take(cb64.size() * 8), o_cbs = take(cbs32.size() * 4), o_sig = take(sig32.size() * 4);
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->block, off);
   if (e != cudaSuccess) {
@@ -323,12 +359,15 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   p->cb32 = reinterpret_cast<float*>(base + o_cb);
   p->bd32 = reinterpret_cast<float*>(base + o_bd);
   p->cb64 = reinterpret_cast<double*>(base + o_cb64);
+  p->cbs32 = reinterpret_cast<float*>(base + o_cbs);
+  p->sig32 = reinterpret_cast<float*>(base + o_sig);
   struct { void* dst; const void* src; size_t n; } copies[] = {
       {p->pi32, pi32.data(), pi32.size() * 4},   {p->pit32, pit32.data(), pit32.size() * 4},
       {p->s32, s32.data(), s32.size() * 4},      {p->st32, st32.data(), st32.size() * 4},
       {p->mt32, mt32.data(), mt32.size() * 4},   {p->pi64, p->pi.data(), p->pi.size() * 8},
       {p->s64, p->s.data(), p->s.size() * 8},    {p->cb32, cb32.data(), cb32.size() * 4},
-      {p->bd32, bd32.data(), bd32.size() * 4},   {p->cb64, cb64.data(), cb64.size() * 8}};
+      {p->bd32, bd32.data(), bd32.size() * 4},   {p->cb64, cb64.data(), cb64.size() * 8},
+      {p->cbs32, cbs32.data(), cbs32.size() * 4}, {p->sig32, sig32.data(), sig32.size() * 4}};
   for (auto& c : copies) {
     e = cudaMemcpy(c.dst, c.src, c.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {

@@ -50,6 +50,8 @@ struct tq_params {
   double* pi64 = nullptr;  // Pi [d][d] fp64 (dequantize)
   double* s64 = nullptr;   // S  [m][d] fp64 (dequantize)
   float* cb32 = nullptr;   // centroids [kMaxBits+1][16] (row b = width b)
+  float* cbs32 = nullptr;  // centroids times sigma_b, the values fed to fp16 MMAs
+  float* sig32 = nullptr;  // sigma_b [kMaxBits+1]: scale making sigma_b*c near-exact in fp16
   float* bd32 = nullptr;   // decision bounds [kMaxBits+1][16]
   double* cb64 = nullptr;  // centroids fp64 [kMaxBits+1][16]
 };
