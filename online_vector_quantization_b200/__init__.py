@@ -152,9 +152,9 @@ class Params:
         return cb.value, qb.value
 
     def close(self):
-        if getattr(self, "handle", None):
+        if getattr(self, "handle", None) and _lib is not None:
             _lib.tq_params_destroy(self.handle)
-            self.handle = None
+        self.handle = None
 
     def __del__(self):
         self.close()

@@ -87,6 +87,18 @@ __device__ __forceinline__ uint32_t h2bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+template <int N>
+struct IntC {
+  static constexpr int value = N;
+};
+template <int N, int I = 0, typename Fn>
+__device__ __forceinline__ void static_for(Fn&& fn) {
+  if constexpr (I < N) {
+    fn(IntC<I>{});
+    static_for<N, I + 1>(fn);
+  }
+}
+
 __device__ __forceinline__ uint32_t lds32(const unsigned char* smem, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(smem + off);
 }
@@ -115,10 +127,66 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// ---- TMA bulk copies and mbarriers (PTX) ----------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
+// addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for a phase with a time limit (~0.5 s of SM clocks); false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > (1ll << 30)) return false;
+  return true;
+}
+
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
   return d;
+}
+
+// LUT address of the 6-bit field at bit `off` of x: (field << 8) | lb, in a
+// shift and one logic op.
+template <int OFF>
+__device__ __forceinline__ uint32_t addr6(uint64_t x, uint32_t lb) {
+  uint32_t v;
+  if constexpr (OFF >= 8)
+    v = static_cast<uint32_t>(x >> (OFF - 8));
+  else
+    v = static_cast<uint32_t>(x) << (8 - OFF);
+  return (v & 0x3F00u) | lb;
 }
 
 template <int N>
@@ -165,22 +233,30 @@ struct KChunk {
     }
   }
 
-  __device__ __forceinline__ uint32_t field6(int p) const {
-    const int bit = 6 * p, i = bit >> 5, sh = bit & 31;
-    if (sh + 6 <= 32 || i + 1 >= WORDS) return (w[i] >> sh) & 63u;
-    return __funnelshift_r(w[i], w[i + 1], sh) & 63u;
+  // 64-bit window holding the 6-bit field p (3-bit chunks)
+  template <int P>
+  __device__ __forceinline__ uint32_t pair3(uint32_t lb) const {
+    if constexpr (6 * P + 6 <= 64) {
+      const uint64_t x = static_cast<uint64_t>(w[0]) | (static_cast<uint64_t>(w[WORDS > 1 ? 1 : 0]) << 32);
+      return addr6<6 * P>(x, lb);
+    } else {
+      const uint64_t x = static_cast<uint64_t>(w[1]) | (static_cast<uint64_t>(w[WORDS > 2 ? 2 : 1]) << 32);
+      return addr6<6 * P - 32>(x, lb);
+    }
   }
 
-  // k-step s: (lo, hi) = A-fragment registers for k = 2t..2t+1 and 2t+8..2t+9
-  __device__ __forceinline__ void decode(int s, const unsigned char* smem, uint32_t lane4, uint32_t lane8,
+  // k-step S: (lo, hi) = A-fragment registers for k = 2t..2t+1 and 2t+8..2t+9
+  template <int S>
+  __device__ __forceinline__ void decode(const unsigned char* smem, uint32_t lane4, uint32_t lane8,
                                          uint32_t c_bits, uint32_t& lo, uint32_t& hi) const {
+    constexpr int s = S;
     if constexpr (B == 4) {
       const uint32_t ww = w[s >> 1];
       lo = lds32(smem, byte_addr(ww, lane4, 2 * (s & 1)));
       hi = lds32(smem, byte_addr(ww, lane4, 2 * (s & 1) + 1));
     } else if constexpr (B == 3) {
-      lo = lds32(smem, (field6(2 * s) << 8) | (lane4 + 128));
-      hi = lds32(smem, (field6(2 * s + 1) << 8) | (lane4 + 128));
+      lo = lds32(smem, pair3<2 * S>(lane4 + 128));
+      hi = lds32(smem, pair3<2 * S + 1>(lane4 + 128));
     } else if constexpr (B == 2) {
       const uint2 v = lds64(smem, byte_addr(w[s >> 2], lane8, s & 3));
       lo = v.x;
@@ -252,11 +328,12 @@ struct VChunk {
       const uint64_t m = field_mask3<MT>();
       const uint64_t ev = (a.x & m) | ((b.x & m) << 3);
       const uint64_t od = ((a.x >> 3) & m) | (b.x & (m << 3));
-#pragma unroll
-      for (int k = 0; k < MT; ++k) {
-        rg[k] = lds32(smem, ((static_cast<uint32_t>(ev >> (6 * k)) & 63u) << 8) | (lane4 + 128));
-        rg8[k] = lds32(smem, ((static_cast<uint32_t>(od >> (6 * k)) & 63u) << 8) | (lane4 + 128));
-      }
+      const uint32_t lb = lane4 + 128;
+      static_for<MT>([&](auto kk) {
+        constexpr int k = decltype(kk)::value;
+        rg[k] = lds32(smem, addr6<6 * k>(ev, lb));
+        rg8[k] = lds32(smem, addr6<6 * k>(od, lb));
+      });
     } else if constexpr (B == 2) {
       const uint32_t xa = static_cast<uint32_t>(a.x), xb = static_cast<uint32_t>(b.x);
       const uint32_t ev = (xa & 0x33333333u) | ((xb & 0x33333333u) << 2);
@@ -326,6 +403,7 @@ struct DecodeArgs {
   const float* cbs;  // sigma-scaled centroids [5][16] (the values the MMAs see)
   const float* sig;  // sigma per width [5]
   float sparse_thr;
+  int pack;          // 1: group <= 4, query hi/lo halves share one MMA (columns g and g+4)
 };
 
 __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
@@ -333,7 +411,9 @@ __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
 }
 
 // ---------------------------------------------------------------------------
-// 1. query rotation: one CTA per (sequence, kv-head)
+// 1. query rotation: one CTA per (sequence, kv-head).  Threads 0..127 form
+//    Pi q for all heads (one output coordinate each), threads 128..255 form
+//    S q (prod keys); then the fp16 B-fragments are written.
 // ---------------------------------------------------------------------------
 template <int KF>
 __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
@@ -350,27 +430,43 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
   }
   __syncthreads();
   const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
-  for (int i = tid; i < kMaxG * kDim; i += kThreads) {
-    const int h = i / kDim, j = i % kDim;
-    float acc = 0.f, acs = 0.f;
-    for (int k = 0; k < kDim; ++k) {
-      acc = fmaf(a.pit[k * kDim + j], qs[h][k], acc);
-      if (FK::prod) acs = fmaf(a.st[k * kSketch + j], qs[h][k], acs);
+  {
+    const int j = tid & (kDim - 1);
+    const bool sketch = tid >= kDim;
+    if (!sketch || FK::prod) {
+      const float* mat = sketch ? a.st : a.pit;  // [k][j] layouts, coalesced over j
+      float acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < kDim; ++k) {
+        const float m = __ldg(mat + k * kDim + j);
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) acc[h] = fmaf(m, qs[h][k], acc[h]);
+      }
+      if (sketch) {
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) qsk[h][j] = acc[h] * scale;
+      } else {
+        const int wj = FK::width(j);
+        const float f = wj > 0 ? scale / a.sig[wj] : 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) qt[h][j] = acc[h] * f;
+      }
     }
-    const int wj = FK::width(j);
-    qt[h][j] = wj > 0 ? acc * scale / a.sig[wj] : 0.f;
-    qsk[h][j] = acs * scale;
   }
   __syncthreads();
-  // B fragments: lane (g, t) supplies head g; k-steps 0..7 from the MSE
-  // segments, 8..15 from the QJL segment.
+  // B fragments: lane (g, t) supplies column g; k-steps 0..7 from the MSE
+  // segments, 8..15 from the QJL segment.  Unpacked: column g = head g, halves
+  // hi (x = 0) and lo (x = 1).  Packed (group <= 4): column g < 4 = hi of head
+  // g, column g >= 4 = lo of head g - 4, in x = 0.
   uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
   for (int i = tid; i < 16 * 32; i += kThreads) {
     const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
     int dims[4] = {0, 0, 0, 0};
-    const float* src = qt[g];
     bool valid = true;
-    if (ks < 8) {
+    const bool qjl = ks >= 8;
+    if (!qjl) {
       if (FK::nseg == 0) {
         valid = false;
       } else if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
@@ -381,8 +477,9 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
     } else {
       if (!FK::prod) valid = false;
       for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
-      src = qsk[g];
     }
+    const int head = a.pack ? (g & 3) : g;
+    const float* src = qjl ? qsk[head] : qt[head];
     uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
     if (valid) {
       for (int r = 0; r < 2; ++r) {
@@ -394,8 +491,13 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
       }
     }
     for (int r = 0; r < 2; ++r) {
-      dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
-      dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
+      if (a.pack) {
+        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = g < 4 ? hi[r] : lo[r];
+        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = 0;
+      } else {
+        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
+        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
+      }
     }
   }
 }
@@ -492,9 +594,261 @@ __device__ void finish_cta(const DecodeArgs& a, int b, int kvh, int expected, in
 }
 
 // ---------------------------------------------------------------------------
-// 2. decode kernel
+// One warp tile: 16 tokens, the registers a lane needs from them.
 // ---------------------------------------------------------------------------
 template <int KF, int VF>
+struct Tile {
+  typename KRow<KF>::S0 k0A, k0B;
+  typename KRow<KF>::S1 k1A, k1B;
+  typename KRow<KF>::Q kqA, kqB;
+  typename VRow<VF>::S0 v0[4];
+  typename VRow<VF>::S1 v1[4];
+  typename VRow<VF>::Q vq[4];
+  float nkA, nkB, nvA, nvB, gkA, gkB, gvA, gvB;
+};
+
+struct UnitPlanes {
+  const uint8_t* kcodes;
+  const uint8_t* vcodes;
+  const float* knorm;
+  const float* vnorm;
+  const uint8_t* kq;
+  const uint8_t* vq;
+  const float* kres;
+  const float* vres;
+};
+
+// One pipeline stage in shared memory: the planes of kChunk consecutive
+// tokens, each copied by one bulk copy.
+constexpr int kChunk = kTok * kWarps;  // 128 tokens: one tile per warp
+template <int KF, int VF>
+struct StageLayout {
+  static constexpr int kc = 0;
+  static constexpr int vc = kc + kChunk * Fmt<KF>::code_bytes;
+  static constexpr int kn = vc + kChunk * Fmt<VF>::code_bytes;
+  static constexpr int vn = kn + kChunk * 4;
+  static constexpr int kq = vn + kChunk * 4;
+  static constexpr int kr = kq + (Fmt<KF>::prod ? kChunk * (kSketch / 8) : 0);
+  static constexpr int vq = kr + (Fmt<KF>::prod ? kChunk * 4 : 0);
+  static constexpr int vr = vq + (Fmt<VF>::prod ? kChunk * (kSketch / 8) : 0);
+  static constexpr int bytes = vr + (Fmt<VF>::prod ? kChunk * 4 : 0);
+  // bytes of a stage holding `rows` tokens (rows a multiple of 16)
+  __host__ __device__ static constexpr uint32_t tx_bytes(int rows) {
+    return static_cast<uint32_t>(rows) * (bytes / kChunk);
+  }
+};
+
+// Pipeline depth: three stages when two CTAs (LUT + stages each, plus the
+// 1 KB the driver reserves per CTA) still fit in the SM's 228 KB, else two.
+template <int KF, int VF>
+__host__ __device__ constexpr int decode_stages() {
+  return 2 * (Lut<KF, VF>::bytes + 3 * StageLayout<KF, VF>::bytes + 2048) <= 228 * 1024 ? 3 : 2;
+}
+
+// Lane loads of one tile from a staged chunk (or any planes with the same row
+// layout); rows row0 .. row0+15 exist in every plane, rows at or past the
+// sequence length hold stale data and are masked when used.
+template <int KF, int VF>
+__device__ __forceinline__ void load_tile(Tile<KF, VF>& T, const UnitPlanes& u, int row0, int g, int t) {
+  using FK = Fmt<KF>;
+  using FV = Fmt<VF>;
+  const int rA = row0 + g, rB = row0 + g + 8;
+  const uint8_t* ka = u.kcodes + static_cast<int64_t>(rA) * FK::code_bytes;
+  const uint8_t* kb = u.kcodes + static_cast<int64_t>(rB) * FK::code_bytes;
+  if constexpr (FK::nseg > 0) { T.k0A.load(ka, t); T.k0B.load(kb, t); }
+  if constexpr (FK::nseg > 1) { T.k1A.load(ka, t); T.k1B.load(kb, t); }
+  if constexpr (FK::prod) {
+    T.kqA.load(u.kq + rA * (kSketch / 8), t);
+    T.kqB.load(u.kq + rB * (kSketch / 8), t);
+    T.gkA = u.kres[rA];
+    T.gkB = u.kres[rB];
+  }
+  T.nkA = u.knorm[rA];
+  T.nkB = u.knorm[rB];
+  T.nvA = u.vnorm[rA];
+  T.nvB = u.vnorm[rB];
+  if constexpr (FV::prod) {
+    T.gvA = u.vres[rA];
+    T.gvB = u.vres[rB];
+  }
+  const int v0 = row0 + 2 * t;  // tokens v0, v0+1, v0+8, v0+9
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = v0 + (i & 1) + 8 * (i >> 1);
+    const uint8_t* vr = u.vcodes + static_cast<int64_t>(r) * FV::code_bytes;
+    if constexpr (FV::nseg > 0) T.v0[i].load(vr, g);
+    if constexpr (FV::nseg > 1) T.v1[i].load(vr, g);
+    if constexpr (FV::prod) T.vq[i].load(u.vq + r * (kSketch / 8), g);
+  }
+}
+
+template <int KF, int VF, bool PACK>
+struct WarpState {
+  static constexpr int VMT = 8 + (Fmt<VF>::prod ? 8 : 0);  // m-tiles of the V accumulator
+  float oacc[VMT][4];
+  float m0, m1, l0, l1;
+};
+
+template <int KF, int VF, bool PACK>
+__device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF, VF, PACK>& W,
+                                             const uint32_t (&bq)[8][2][PACK ? 1 : 2],
+                                             const uint32_t (&bqs)[8][2][PACK ? 1 : 2], int row0, int t_end,
+                                             int g, const unsigned char* lut_a, const unsigned char* lut_b,
+                                             uint32_t lane4, uint32_t lane8, uint32_t c1k, uint32_t c1v,
+                                             float thr) {
+  using FK = Fmt<KF>;
+  using FV = Fmt<VF>;
+  using KR = KRow<KF>;
+  using VR = VRow<VF>;
+  constexpr int NX = PACK ? 1 : 2;
+  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
+  const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
+  const bool okA = row0 + g < t_end, okB = row0 + g + 8 < t_end;
+
+  // ---- scores S^T (tokens x columns), four independent MMA accumulator chains
+  float ca[4][4], cq[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ca[i][j] = cq[i][j] = 0.f;
+  if constexpr (FK::nseg > 0) {
+    const unsigned char* lk = FK::b0 == 2 ? lut_b : lut_a;
+    static_for<KR::S0::KSTEPS>([&](auto ss) {
+      constexpr int s = decltype(ss)::value;
+      uint32_t la, ha, lb, hb;
+      T.k0A.template decode<s>(lk, lane4, lane8, c1k, la, ha);
+      T.k0B.template decode<s>(lk, lane4, lane8, c1k, lb, hb);
+#pragma unroll
+      for (int x = 0; x < NX; ++x) mma16816(ca[(NX * s + x) & 3], la, lb, ha, hb, bq[s][0][x], bq[s][1][x]);
+    });
+  }
+  if constexpr (FK::nseg > 1) {
+    static_for<KR::S1::KSTEPS>([&](auto ss) {
+      constexpr int s = decltype(ss)::value;
+      uint32_t la, ha, lb, hb;
+      T.k1A.template decode<s>(lut_a, lane4, lane8, c1k, la, ha);
+      T.k1B.template decode<s>(lut_a, lane4, lane8, c1k, lb, hb);
+#pragma unroll
+      for (int x = 0; x < NX; ++x)
+        mma16816(ca[(NX * s + x + 2) & 3], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
+    });
+  }
+  if constexpr (FK::prod) {
+    static_for<8>([&](auto ss) {
+      constexpr int s = decltype(ss)::value;
+      uint32_t la, ha, lb, hb;
+      T.kqA.template decode<s>(lut_a, lane4, lane8, one2, la, ha);
+      T.kqB.template decode<s>(lut_a, lane4, lane8, one2, lb, hb);
+#pragma unroll
+      for (int x = 0; x < NX; ++x) mma16816(cq[(NX * s + x) & 3], la, lb, ha, hb, bqs[s][0][x], bqs[s][1][x]);
+    });
+  }
+  float sc[4], sq[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    sc[j] = (ca[0][j] + ca[1][j]) + (ca[2][j] + ca[3][j]);
+    sq[j] = (cq[0][j] + cq[1][j]) + (cq[2][j] + cq[3][j]);
+  }
+  if constexpr (PACK) {
+    // columns c and c+4 hold the hi and lo halves of one head: add them
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sc[i] += __shfl_xor_sync(0xffffffffu, sc[i], 2);
+      if constexpr (FK::prod) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], 2);
+    }
+  }
+  // s (base 2): c0,c1 = token g, columns 2t, 2t+1; c2,c3 = token g+8
+  const float gkA = FK::prod ? T.gkA : 0.f, gkB = FK::prod ? T.gkB : 0.f;
+  float s2[4];
+  s2[0] = okA ? T.nkA * (sc[0] + kQjlScale * gkA * sq[0]) : -INFINITY;
+  s2[1] = okA ? T.nkA * (sc[1] + kQjlScale * gkA * sq[1]) : -INFINITY;
+  s2[2] = okB ? T.nkB * (sc[2] + kQjlScale * gkB * sq[2]) : -INFINITY;
+  s2[3] = okB ? T.nkB * (sc[3] + kQjlScale * gkB * sq[3]) : -INFINITY;
+  float mx0 = fmaxf(s2[0], s2[2]), mx1 = fmaxf(s2[1], s2[3]);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
+  const float al0 = exp2f(W.m0 - mn0), al1 = exp2f(W.m1 - mn1);
+  float p[4];
+  p[0] = exp2f(s2[0] - mn0);
+  p[1] = exp2f(s2[1] - mn1);
+  p[2] = exp2f(s2[2] - mn0);
+  p[3] = exp2f(s2[3] - mn1);
+  float rs0 = p[0] + p[2], rs1 = p[1] + p[3];
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
+    rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
+  }
+  W.l0 = W.l0 * al0 + rs0;
+  W.l1 = W.l1 * al1 + rs1;
+  W.m0 = mn0;
+  W.m1 = mn1;
+  if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
+#pragma unroll
+    for (int i = 0; i < VMT; ++i) {
+      W.oacc[i][0] *= al0;
+      W.oacc[i][1] *= al1;
+      W.oacc[i][2] *= al0;
+      W.oacc[i][3] *= al1;
+    }
+  }
+  // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
+  if (thr > 0.f) {
+    const float c0 = thr * W.l0, c1 = thr * W.l1;
+    p[0] = p[0] >= c0 ? p[0] : 0.f;
+    p[1] = p[1] >= c1 ? p[1] : 0.f;
+    p[2] = p[2] >= c0 ? p[2] : 0.f;
+    p[3] = p[3] >= c1 ? p[3] : 0.f;
+    const bool any = (p[0] + p[1] + p[2] + p[3]) > 0.f;
+    if (!__any_sync(0xffffffffu, any)) return;
+  }
+
+  // ---- P'^T fragments: P' = p * ||v|| (and * ||r_v|| for the sketch part)
+  const float wA = okA ? T.nvA : 0.f, wB = okB ? T.nvB : 0.f;
+  const uint32_t pb0 = movmatrix_t(h2bits(p[0] * wA, p[1] * wA));
+  const uint32_t pb1 = movmatrix_t(h2bits(p[2] * wB, p[3] * wB));
+  uint32_t qb0 = 0, qb1 = 0;
+  if constexpr (FV::prod) {
+    const float uA = okA ? wA * T.gvA : 0.f, uB = okB ? wB * T.gvB : 0.f;
+    qb0 = movmatrix_t(h2bits(p[0] * uA, p[1] * uA));
+    qb1 = movmatrix_t(h2bits(p[2] * uB, p[3] * uB));
+  }
+  // ---- O^T += C_v^T P'^T
+  if constexpr (FV::nseg > 0) {
+    constexpr int MT = VR::S0::MT;
+    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
+    const unsigned char* lut = FV::b0 == 2 ? lut_b : lut_a;
+    VR::S0::decode(T.v0[0], T.v0[1], lut, lane4, lane8, c1v, r0, r08);
+    VR::S0::decode(T.v0[2], T.v0[3], lut, lane4, lane8, c1v, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mma16816(W.oacc[mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
+  }
+  if constexpr (FV::nseg > 1) {
+    constexpr int MT = VR::S1::MT;
+    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
+    VR::S1::decode(T.v1[0], T.v1[1], lut_a, lane4, lane8, c1v, r0, r08);
+    VR::S1::decode(T.v1[2], T.v1[3], lut_a, lane4, lane8, c1v, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+      mma16816(W.oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
+  }
+  if constexpr (FV::prod) {
+    uint32_t r0[8], r08[8], r1[8], r18[8];
+    VR::Q::decode(T.vq[0], T.vq[1], lut_a, lane4, lane8, one2, r0, r08);
+    VR::Q::decode(T.vq[2], T.vq[3], lut_a, lane4, lane8, one2, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) mma16816(W.oacc[8 + mt], r0[mt], r08[mt], r1[mt], r18[mt], qb0, qb1);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. decode kernel
+// ---------------------------------------------------------------------------
+template <int KF, int VF, bool PACK>
 __global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1 : 2) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
@@ -621,208 +975,123 @@ __global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1
   const uint32_t lane4 = lane * 4, lane8 = lane * 8;
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
-  const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
 
   // query B-fragments
+  constexpr int NX = PACK ? 1 : 2;
   const uint32_t* qf = a.qfrag + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  uint32_t bq[8][2][2], bqs[8][2][2];  // [kstep][b0,b1][hi,lo]
+  uint32_t bq[8][2][NX], bqs[8][2][NX];  // [kstep][b0,b1][hi,lo]
 #pragma unroll
   for (int s = 0; s < 8; ++s)
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
+      for (int x = 0; x < NX; ++x) {
         bq[s][r][x] = qf[((s * 2 + r) * 2 + x) * 32 + lane];
         if constexpr (FK::prod) bqs[s][r][x] = qf[(((8 + s) * 2 + r) * 2 + x) * 32 + lane];
       }
   __syncthreads();
 
-  constexpr int VMT = 8 + (FV::prod ? 8 : 0);  // m-tiles of the V accumulator
-  float oacc[VMT][4];
+  WarpState<KF, VF, PACK> wst;
+  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
 #pragma unroll
-  for (int i = 0; i < VMT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  for (int i = 0; i < VMT; ++i) wst.oacc[i][0] = wst.oacc[i][1] = wst.oacc[i][2] = wst.oacc[i][3] = 0.f;
+  wst.m0 = wst.m1 = -INFINITY;
+  wst.l0 = wst.l1 = 0.f;
 
   const int t_begin = split * a.split_tokens;
   const int t_end = min(nq, t_begin + a.split_tokens);
-  const int n_tiles = (t_end - t_begin + kTok - 1) / kTok;
   const int64_t ubase = (static_cast<int64_t>(b) * a.hkv + kvh) * a.capacity;
-  const uint8_t* kcodes = a.k_codes + ubase * FK::code_bytes;
-  const uint8_t* vcodes = a.v_codes + ubase * FV::code_bytes;
-  const float* knorm = a.k_norms + ubase;
-  const float* vnorm = a.v_norms + ubase;
-  const uint8_t* kq = FK::prod ? a.k_qjl + ubase * (kSketch / 8) : nullptr;
-  const uint8_t* vq = FV::prod ? a.v_qjl + ubase * (kSketch / 8) : nullptr;
-  const float* kres = FK::prod ? a.k_res + ubase : nullptr;
-  const float* vres = FV::prod ? a.v_res + ubase : nullptr;
+  UnitPlanes u;
+  u.kcodes = a.k_codes + ubase * FK::code_bytes;
+  u.vcodes = a.v_codes + ubase * FV::code_bytes;
+  u.knorm = a.k_norms + ubase;
+  u.vnorm = a.v_norms + ubase;
+  u.kq = FK::prod ? a.k_qjl + ubase * (kSketch / 8) : nullptr;
+  u.vq = FV::prod ? a.v_qjl + ubase * (kSketch / 8) : nullptr;
+  u.kres = FK::prod ? a.k_res + ubase : nullptr;
+  u.vres = FV::prod ? a.v_res + ubase : nullptr;
   const float thr = a.sparse_thr;
 
-  for (int it = warp; it < n_tiles; it += kWarps) {
-    const int row0 = t_begin + it * kTok;
-    const int rA = row0 + g, rB = row0 + g + 8;
-    const bool okA = rA < t_end, okB = rB < t_end;
-
-    // ---- loads
-    typename KR::S0 k0A, k0B;
-    typename KR::S1 k1A, k1B;
-    typename KR::Q kqA, kqB;
-    if constexpr (FK::nseg > 0) {
-      k0A.load(kcodes + static_cast<int64_t>(rA) * FK::code_bytes, t);
-      k0B.load(kcodes + static_cast<int64_t>(rB) * FK::code_bytes, t);
-    }
-    if constexpr (FK::nseg > 1) {
-      k1A.load(kcodes + static_cast<int64_t>(rA) * FK::code_bytes, t);
-      k1B.load(kcodes + static_cast<int64_t>(rB) * FK::code_bytes, t);
-    }
+  // software pipeline: the loads of the warp's next tile are in flight while
+  // the current one is decoded (two register buffers, no copies)
+  // TMA pipeline: thread 0 streams kChunk-token chunks of the split into a
+  // ring of shared-memory stages (one bulk copy per plane); warp w decodes
+  // tile w of each chunk.
+  using SL = StageLayout<KF, VF>;
+  constexpr int kStages = decode_stages<KF, VF>();
+  unsigned char* stages = smem + L::bytes;
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ int s_abort;
+  const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
+  const int t_end16 = (t_end + kTok - 1) / kTok * kTok;  // <= capacity (a multiple of 64)
+  auto issue = [&](int c) {
+    unsigned char* st = stages + (c % kStages) * SL::bytes;
+    const int r0 = t_begin + c * kChunk;
+    const int rows = min(kChunk, t_end16 - r0);
+    uint64_t* bar = &full_bar[c % kStages];
+    mbar_expect_tx(bar, SL::tx_bytes(rows));
+    if constexpr (FK::code_bytes > 0)
+      bulk_g2s(st + SL::kc, u.kcodes + static_cast<int64_t>(r0) * FK::code_bytes, rows * FK::code_bytes, bar);
+    if constexpr (FV::code_bytes > 0)
+      bulk_g2s(st + SL::vc, u.vcodes + static_cast<int64_t>(r0) * FV::code_bytes, rows * FV::code_bytes, bar);
+    bulk_g2s(st + SL::kn, u.knorm + r0, rows * 4, bar);
+    bulk_g2s(st + SL::vn, u.vnorm + r0, rows * 4, bar);
     if constexpr (FK::prod) {
-      kqA.load(kq + rA * (kSketch / 8), t);
-      kqB.load(kq + rB * (kSketch / 8), t);
-    }
-    const float nkA = knorm[rA], nkB = knorm[rB];
-    const float nvA = vnorm[rA], nvB = vnorm[rB];
-    float gkA = 0.f, gkB = 0.f, gvA = 0.f, gvB = 0.f;
-    if constexpr (FK::prod) { gkA = kres[rA]; gkB = kres[rB]; }
-    if constexpr (FV::prod) { gvA = okA ? vres[rA] : 0.f; gvB = okB ? vres[rB] : 0.f; }
-    const int v0 = row0 + 2 * t;  // tokens v0, v0+1, v0+8, v0+9
-    typename VR::S0 v0a, v0b, v0c, v0d;
-    typename VR::S1 v1a, v1b, v1c, v1d;
-    typename VR::Q vqa, vqb, vqc, vqd;
-    if constexpr (FV::nseg > 0) {
-      v0a.load(vcodes + static_cast<int64_t>(v0) * FV::code_bytes, g);
-      v0b.load(vcodes + static_cast<int64_t>(v0 + 1) * FV::code_bytes, g);
-      v0c.load(vcodes + static_cast<int64_t>(v0 + 8) * FV::code_bytes, g);
-      v0d.load(vcodes + static_cast<int64_t>(v0 + 9) * FV::code_bytes, g);
-    }
-    if constexpr (FV::nseg > 1) {
-      v1a.load(vcodes + static_cast<int64_t>(v0) * FV::code_bytes, g);
-      v1b.load(vcodes + static_cast<int64_t>(v0 + 1) * FV::code_bytes, g);
-      v1c.load(vcodes + static_cast<int64_t>(v0 + 8) * FV::code_bytes, g);
-      v1d.load(vcodes + static_cast<int64_t>(v0 + 9) * FV::code_bytes, g);
+      bulk_g2s(st + SL::kq, u.kq + r0 * (kSketch / 8), rows * (kSketch / 8), bar);
+      bulk_g2s(st + SL::kr, u.kres + r0, rows * 4, bar);
     }
     if constexpr (FV::prod) {
-      vqa.load(vq + v0 * (kSketch / 8), g);
-      vqb.load(vq + (v0 + 1) * (kSketch / 8), g);
-      vqc.load(vq + (v0 + 8) * (kSketch / 8), g);
-      vqd.load(vq + (v0 + 9) * (kSketch / 8), g);
+      bulk_g2s(st + SL::vq, u.vq + r0 * (kSketch / 8), rows * (kSketch / 8), bar);
+      bulk_g2s(st + SL::vr, u.vres + r0, rows * 4, bar);
     }
-
-    // ---- scores S^T (tokens x heads)
-    float sc[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (FK::nseg > 0) {
-      const unsigned char* lk = FK::b0 == 2 ? lut_b : lut_a;
+  };
+  if (tid == 0) {
+    s_abort = 0;
 #pragma unroll
-      for (int s = 0; s < KR::S0::KSTEPS; ++s) {
-        uint32_t la, ha, lb, hb;
-        k0A.decode(s, lk, lane4, lane8, c1k, la, ha);
-        k0B.decode(s, lk, lane4, lane8, c1k, lb, hb);
-        mma16816(sc, la, lb, ha, hb, bq[s][0][0], bq[s][1][0]);
-        mma16816(sc, la, lb, ha, hb, bq[s][0][1], bq[s][1][1]);
-      }
+    for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int c = 0; c < min(kStages, n_chunks); ++c) issue(c);
+  int issued = min(kStages, n_chunks);
+  for (int c = 0; c < n_chunks; ++c) {
+    if (!mbar_wait(&full_bar[c % kStages], (c / kStages) & 1)) s_abort = 1;
+    const int row0 = t_begin + c * kChunk + warp * kTok;
+    if (row0 < t_end && !s_abort) {
+      const unsigned char* st = stages + (c % kStages) * SL::bytes;
+      UnitPlanes sp;
+      sp.kcodes = st + SL::kc;
+      sp.vcodes = st + SL::vc;
+      sp.knorm = reinterpret_cast<const float*>(st + SL::kn);
+      sp.vnorm = reinterpret_cast<const float*>(st + SL::vn);
+      sp.kq = st + SL::kq;
+      sp.kres = reinterpret_cast<const float*>(st + SL::kr);
+      sp.vq = st + SL::vq;
+      sp.vres = reinterpret_cast<const float*>(st + SL::vr);
+      Tile<KF, VF> tl;
+      load_tile(tl, sp, warp * kTok, g, t);
+      compute_tile<KF, VF, PACK>(tl, wst, bq, bqs, row0, t_end, g, lut_a, lut_b, lane4, lane8, c1k, c1v, thr);
     }
-    if constexpr (FK::nseg > 1) {
-#pragma unroll
-      for (int s = 0; s < KR::S1::KSTEPS; ++s) {
-        uint32_t la, ha, lb, hb;
-        k1A.decode(s, lut_a, lane4, lane8, c1k, la, ha);
-        k1B.decode(s, lut_a, lane4, lane8, c1k, lb, hb);
-        mma16816(sc, la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][0], bq[KR::S0::KSTEPS + s][1][0]);
-        mma16816(sc, la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][1], bq[KR::S0::KSTEPS + s][1][1]);
-      }
-    }
-    if constexpr (FK::prod) {
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        uint32_t la, ha, lb, hb;
-        kqA.decode(s, lut_a, lane4, lane8, one2, la, ha);
-        kqB.decode(s, lut_a, lane4, lane8, one2, lb, hb);
-        mma16816(sq, la, lb, ha, hb, bqs[s][0][0], bqs[s][1][0]);
-        mma16816(sq, la, lb, ha, hb, bqs[s][0][1], bqs[s][1][1]);
-      }
-    }
-    // s (base 2): c0,c1 = token g, heads 2t, 2t+1; c2,c3 = token g+8
-    float s2[4];
-    s2[0] = okA ? nkA * (sc[0] + kQjlScale * gkA * sq[0]) : -INFINITY;
-    s2[1] = okA ? nkA * (sc[1] + kQjlScale * gkA * sq[1]) : -INFINITY;
-    s2[2] = okB ? nkB * (sc[2] + kQjlScale * gkB * sq[2]) : -INFINITY;
-    s2[3] = okB ? nkB * (sc[3] + kQjlScale * gkB * sq[3]) : -INFINITY;
-    float mx0 = fmaxf(s2[0], s2[2]), mx1 = fmaxf(s2[1], s2[3]);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-    float p[4];
-    p[0] = exp2f(s2[0] - mn0);
-    p[1] = exp2f(s2[1] - mn1);
-    p[2] = exp2f(s2[2] - mn0);
-    p[3] = exp2f(s2[3] - mn1);
-    float rs0 = p[0] + p[2], rs1 = p[1] + p[3];
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
-      rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
-    }
-    l0 = l0 * al0 + rs0;
-    l1 = l1 * al1 + rs1;
-    m0 = mn0;
-    m1 = mn1;
-#pragma unroll
-    for (int i = 0; i < VMT; ++i) {
-      oacc[i][0] *= al0;
-      oacc[i][1] *= al1;
-      oacc[i][2] *= al0;
-      oacc[i][3] *= al1;
-    }
-    // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
-    if (thr > 0.f) {
-      const float c0 = thr * l0, c1 = thr * l1;
-      p[0] = p[0] >= c0 ? p[0] : 0.f;
-      p[1] = p[1] >= c1 ? p[1] : 0.f;
-      p[2] = p[2] >= c0 ? p[2] : 0.f;
-      p[3] = p[3] >= c1 ? p[3] : 0.f;
-    }
-    const bool any = (p[0] + p[1] + p[2] + p[3]) > 0.f;
-    if (!__any_sync(0xffffffffu, any)) continue;
-
-    // ---- P'^T fragments: P' = p * ||v|| (and * ||r_v|| for the sketch part)
-    const float wA = okA ? nvA : 0.f, wB = okB ? nvB : 0.f;
-    const uint32_t x0 = h2bits(p[0] * wA, p[1] * wA), x1 = h2bits(p[2] * wB, p[3] * wB);
-    const uint32_t pb0 = movmatrix_t(x0), pb1 = movmatrix_t(x1);
-    uint32_t qb0 = 0, qb1 = 0;
-    if constexpr (FV::prod) {
-      const uint32_t y0 = h2bits(p[0] * wA * gvA, p[1] * wA * gvA), y1 = h2bits(p[2] * wB * gvB, p[3] * wB * gvB);
-      qb0 = movmatrix_t(y0);
-      qb1 = movmatrix_t(y1);
-    }
-    // ---- O^T += C_v^T P'^T
-    if constexpr (FV::nseg > 0) {
-      constexpr int MT = VR::S0::MT;
-      uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
-      const unsigned char* lut = Fmt<VF>::b0 == 2 ? lut_b : lut_a;
-      VR::S0::decode(v0a, v0b, lut, lane4, lane8, c1v, r0, r08);
-      VR::S0::decode(v0c, v0d, lut, lane4, lane8, c1v, r1, r18);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) mma16816(oacc[mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
-    }
-    if constexpr (FV::nseg > 1) {
-      constexpr int MT = VR::S1::MT;
-      uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
-      VR::S1::decode(v1a, v1b, lut_a, lane4, lane8, c1v, r0, r08);
-      VR::S1::decode(v1c, v1d, lut_a, lane4, lane8, c1v, r1, r18);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-        mma16816(oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
-    }
-    if constexpr (FV::prod) {
-      uint32_t r0[8], r08[8], r1[8], r18[8];
-      VR::Q::decode(vqa, vqb, lut_a, lane4, lane8, one2, r0, r08);
-      VR::Q::decode(vqc, vqd, lut_a, lane4, lane8, one2, r1, r18);
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) mma16816(oacc[8 + mt], r0[mt], r08[mt], r1[mt], r18[mt], qb0, qb1);
+    __syncthreads();  // stage c % kStages is free again
+    if (s_abort) break;
+    if (tid == 0 && issued < n_chunks) {
+      fence_proxy_async();
+      issue(issued);
+      ++issued;
     }
   }
+  if (s_abort) {
+    // a copy never completed: flag it, drain what was issued (bounded) and
+    // leave without publishing a partial
+    if (tid == 0) {
+      atomicOr(a.status, 4);
+      for (int c = 0; c < issued; ++c) mbar_wait(&full_bar[c % kStages], (c / kStages) & 1);
+    }
+    return;
+  }
+  float (&oacc)[VMT][4] = wst.oacc;
+  const float m0 = wst.m0, m1 = wst.m1, l0 = wst.l0, l1 = wst.l1;
 
   // ---- merge the warps of this CTA (shared memory reused after the loop)
   __syncthreads();
@@ -893,25 +1162,32 @@ __global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1
 template <int KF, int VF>
 size_t decode_smem_bytes() {
   using L = Lut<KF, VF>;
+  const size_t pipeline = static_cast<size_t>(L::bytes) + decode_stages<KF, VF>() * StageLayout<KF, VF>::bytes;
   const size_t W = Fmt<VF>::prod ? 2 * kDim : kDim;
   const size_t combine = (2 * kWarps * kMaxG + kWarps * kMaxG * W) * sizeof(float);
   const size_t merge = (kMaxG * 2 * kDim + kMaxG * kDim + 2 * kMaxG) * sizeof(float);
-  return std::max<size_t>({static_cast<size_t>(L::bytes), combine, merge, 24 * 1024});
+  return std::max<size_t>({pipeline, combine, merge, 24 * 1024});
+}
+
+template <int KF, int VF, bool PACK>
+tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF, PACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
+  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, 0, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
+  decode_kernel<KF, VF, PACK><<<dim3(plan.n_splits + 1, plan.hkv, plan.B), kThreads, smem, st>>>(a);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "decode kernel launch");
 }
 
 template <int KF, int VF>
 tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, int sink_smem_floats, cudaStream_t st) {
   size_t smem = decode_smem_bytes<KF, VF>();
   smem = std::max<size_t>(smem, static_cast<size_t>(sink_smem_floats) * sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
-  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, 0, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
-  decode_kernel<KF, VF><<<dim3(plan.n_splits + 1, plan.hkv, plan.B), kThreads, smem, st>>>(a);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "decode kernel launch");
+  a.pack = plan.group <= 4;
+  return a.pack ? run_decode_v<KF, VF, true>(a, plan, smem, st) : run_decode_v<KF, VF, false>(a, plan, smem, st);
 }
 
 constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 3) | (prod << 4); }
