@@ -87,6 +87,13 @@ __device__ __forceinline__ uint32_t h2bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int N>
 struct IntC {
   static constexpr int value = N;
@@ -120,7 +127,7 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t c_bits
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -136,9 +143,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -173,7 +177,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
   uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
   return d;
 }
 
@@ -390,7 +394,7 @@ struct DecodeArgs {
   const uint16_t* v_sink;
   const int32_t* lens;
   int32_t* status;
-  int hkv, group, hq, capacity, n_sink, max_len, n_splits, split_tokens, part_floats;
+  int B, hkv, group, hq, capacity, n_sink, max_len, part_floats;
   float* parts;
   int32_t* tickets;
   const uint32_t* qfrag;
@@ -503,97 +507,6 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Split merge (last CTA of a (sequence, kv-head)): combine the partials and
-// apply Pi^T (and S^T) once per output.
-// ---------------------------------------------------------------------------
-template <int VF>
-__device__ void merge_unit(const DecodeArgs& a, int b, int kvh, int n_real, bool has_sink, float* sm) {
-  constexpr bool VPROD = Fmt<VF>::prod;
-  const int tid = threadIdx.x, G = a.group;
-  const int PF = a.part_floats;
-  const float* base = a.parts + (static_cast<int64_t>(b) * a.hkv + kvh) * (a.n_splits + 1) * kMaxG * PF;
-  float* acc = sm;                         // [kMaxG][2*kDim] rotated | sketch
-  float* osk = sm + kMaxG * 2 * kDim;      // [kMaxG][kDim] sink, original domain
-  float* mm = osk + kMaxG * kDim;          // [kMaxG]: M
-  float* ll = mm + kMaxG;                  // [kMaxG]: L
-  if (tid < kMaxG) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < n_real; ++sp) M = fmaxf(M, __ldcg(base + (sp * kMaxG + tid) * PF));
-    if (has_sink) M = fmaxf(M, __ldcg(base + (a.n_splits * kMaxG + tid) * PF));
-    float L = 0.f;
-    for (int sp = 0; sp < n_real; ++sp) {
-      const float* pp = base + (sp * kMaxG + tid) * PF;
-      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - M);
-    }
-    if (has_sink) {
-      const float* pp = base + (a.n_splits * kMaxG + tid) * PF;
-      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - M);
-    }
-    mm[tid] = M;
-    ll[tid] = L;
-  }
-  __syncthreads();
-  const int width = VPROD ? 2 * kDim : kDim;
-  for (int i = tid; i < G * width; i += kThreads) {
-    const int h = i / width, j = i % width;
-    float s = 0.f;
-    for (int sp = 0; sp < n_real; ++sp) {
-      const float* pp = base + (sp * kMaxG + h) * PF;
-      s += __ldcg(pp + 2 + j) * exp2f(__ldcg(pp) - mm[h]);
-    }
-    if (j < kDim) s = Fmt<VF>::width(j) > 0 ? s / a.sig[Fmt<VF>::width(j)] : 0.f;
-    acc[h * 2 * kDim + j] = s;
-  }
-  for (int i = tid; i < G * kDim; i += kThreads) {
-    const int h = i / kDim, j = i % kDim;
-    float s = 0.f;
-    if (has_sink) {
-      const float* pp = base + (a.n_splits * kMaxG + h) * PF;
-      s = __ldcg(pp + 2 + j) * exp2f(__ldcg(pp) - mm[h]);
-    }
-    osk[h * kDim + j] = s;
-  }
-  __syncthreads();
-  for (int i = tid; i < G * kDim; i += kThreads) {
-    const int h = i / kDim, o = i % kDim;
-    float r = 0.f;
-    const float* ah = acc + h * 2 * kDim;
-    for (int j = 0; j < kDim; ++j) r = fmaf(a.pi[j * kDim + o], ah[j], r);
-    if (VPROD) {
-      float z = 0.f;
-      for (int l = 0; l < kSketch; ++l) z = fmaf(a.s[l * kDim + o], ah[kDim + l], z);
-      r = fmaf(kQjlScale, z, r);
-    }
-    const float L = ll[h];
-    const float val = L > 0.f ? (r + osk[h * kDim + o]) / L : 0.f;
-    const int64_t oi = (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + o;
-    if (a.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(val);
-    else
-      reinterpret_cast<float*>(a.out)[oi] = val;
-  }
-}
-
-// Publish this CTA's partial; the CTA that completes the set merges.
-template <int VF>
-__device__ void finish_cta(const DecodeArgs& a, int b, int kvh, int expected, int n_real, bool has_sink,
-                           float* sm) {
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  int32_t* ticket = a.tickets + static_cast<int64_t>(b) * a.hkv + kvh;
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(ticket, 1);
-    s_last = prev == expected - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  merge_unit<VF>(a, b, kvh, n_real, has_sink, sm);
-  if (threadIdx.x == 0) *ticket = 0;  // leave the workspace ready for the next call
-}
-
-// ---------------------------------------------------------------------------
 // One warp tile: 16 tokens, the registers a lane needs from them.
 // ---------------------------------------------------------------------------
 template <int KF, int VF>
@@ -620,7 +533,9 @@ struct UnitPlanes {
 
 // One pipeline stage in shared memory: the planes of kChunk consecutive
 // tokens, each copied by one bulk copy.
-constexpr int kChunk = kTok * kWarps;  // 128 tokens: one tile per warp
+constexpr int kConsumers = 15;                // consumer warps of the persistent kernel
+constexpr int kThreadsP = (kConsumers + 1) * 32;  // + one producer warp
+constexpr int kChunk = kTok * kConsumers;       // 240 tokens: one tile per consumer warp
 template <int KF, int VF>
 struct StageLayout {
   static constexpr int kc = 0;
@@ -638,11 +553,21 @@ struct StageLayout {
   }
 };
 
-// Pipeline depth: three stages when two CTAs (LUT + stages each, plus the
-// 1 KB the driver reserves per CTA) still fit in the SM's 228 KB, else two.
+// Shared memory of the persistent kernel: LUT | pipeline stages | scratch
+// (warp combine in 64-coordinate slices, split merge, sink scores).
+constexpr int kSliceDims = 64;
+__host__ __device__ constexpr int scratch_bytes(int n_sink) {
+  const int combine = (kConsumers * kMaxG * kSliceDims + 2 * kConsumers * kMaxG) * 4;
+  const int merge = (kMaxG * 3 * kDim + 2 * kMaxG) * 4;
+  const int sink = (kMaxG * kDim + kMaxG * n_sink + 2 * kMaxG) * 4;
+  return combine > merge ? (combine > sink ? combine : sink) : (merge > sink ? merge : sink);
+}
+constexpr int kSmemBudget = 227 * 1024 - 1024;  // per block, minus static shared memory
 template <int KF, int VF>
 __host__ __device__ constexpr int decode_stages() {
-  return 2 * (Lut<KF, VF>::bytes + 3 * StageLayout<KF, VF>::bytes + 2048) <= 228 * 1024 ? 3 : 2;
+  return Lut<KF, VF>::bytes + 4 * StageLayout<KF, VF>::bytes + scratch_bytes(128) <= kSmemBudget   ? 4
+         : Lut<KF, VF>::bytes + 3 * StageLayout<KF, VF>::bytes + scratch_bytes(128) <= kSmemBudget ? 3
+                                                                                                  : 2;
 }
 
 // Lane loads of one tile from a staged chunk (or any planes with the same row
@@ -771,12 +696,12 @@ __device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
   }
   const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
-  const float al0 = exp2f(W.m0 - mn0), al1 = exp2f(W.m1 - mn1);
+  const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
   float p[4];
-  p[0] = exp2f(s2[0] - mn0);
-  p[1] = exp2f(s2[1] - mn1);
-  p[2] = exp2f(s2[2] - mn0);
-  p[3] = exp2f(s2[3] - mn1);
+  p[0] = fast_exp2(s2[0] - mn0);
+  p[1] = fast_exp2(s2[1] - mn1);
+  p[2] = fast_exp2(s2[2] - mn0);
+  p[3] = fast_exp2(s2[3] - mn1);
   float rs0 = p[0] + p[2], rs1 = p[1] + p[3];
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
@@ -845,123 +770,320 @@ __device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF
   }
 }
 
+
 // ---------------------------------------------------------------------------
-// 2. decode kernel
+// 2. persistent decode kernel
+//
+// One CTA per SM: consumer warps 0..14 decode, warp 15 streams the packed
+// cache with bulk copies (full / empty mbarriers, bounded waits).
+//
+// Schedule.  Unit u = b * hkv + h (sequence b, kv-head h).  Its quantized
+// tokens form ceil(nq / kChunk) chunks; the chunks of all units, in unit
+// order, make one list of C chunks cut into gridDim.x equal contiguous ranges,
+// one per CTA, so every CTA streams the same number of bytes.  A unit may span
+// several CTAs (its pieces).  Piece (u, cta) publishes partial slot u + cta:
+// both indices only grow along the list, so slots are distinct and there are
+// at most U + P - 1 of them.  The bf16 sink of unit u is one more piece
+// (slot U + P + u), done by CTA u mod P.  The CTA that completes a unit's set
+// of pieces (atomic ticket, no spin-wait) merges them and applies Pi^T / S^T.
 // ---------------------------------------------------------------------------
+struct UnitInfo {
+  int len, ns, nq, chunks;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u) {
+  const int b = u / a.hkv;
+  const int len = min(max(a.lens[b], 0), a.max_len);
+  UnitInfo r;
+  r.len = len;
+  r.ns = min(a.n_sink, len);
+  r.nq = len - r.ns;
+  r.chunks = (r.nq + kChunk - 1) / kChunk;
+  return r;
+}
+
+__device__ __forceinline__ int64_t range_start(int i, int64_t C, int P) { return static_cast<int64_t>(i) * C / P; }
+
+// CTA whose range holds chunk c: the largest i with i*C/P <= c.
+__device__ __forceinline__ int cta_of_chunk(int64_t c, int64_t C, int P) {
+  return static_cast<int>(((c + 1) * P - 1) / C);
+}
+
+// Ranges are empty when C < P; such CTAs hold no piece of any unit.
+__device__ __forceinline__ bool cta_has_chunks(int i, int64_t C, int P) {
+  return range_start(i + 1, C, P) > range_start(i, C, P);
+}
+
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers * 32) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ float* part_slot(const DecodeArgs& a, int64_t slot) {
+  return a.parts + slot * kMaxG * a.part_floats;
+}
+
+__device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t i, float v) {
+  if (a.out_bf16)
+    reinterpret_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(a.out)[i] = v;
+}
+
+// Merge the pieces of unit u (consumer threads): main slots u + i for
+// i in [first, last] (none when first > last) and the sink slot.
+template <int VF>
+__device__ void merge_unit(const DecodeArgs& a, int u, int first, int last, bool has_sink, float* sm, int64_t C) {
+  constexpr bool VPROD = Fmt<VF>::prod;
+  constexpr int NT = kConsumers * 32;
+  const int tid = threadIdx.x, G = a.group;
+  const int PF = a.part_floats;
+  const int U = a.B * a.hkv, P = gridDim.x;
+  const float* sink = part_slot(a, U + P + u);
+  float* acc = sm;                     // [kMaxG][2*kDim] rotated | sketch
+  float* osk = sm + kMaxG * 2 * kDim;  // [kMaxG][kDim] sink, original domain
+  float* mm = osk + kMaxG * kDim;      // [kMaxG]: M
+  float* ll = mm + kMaxG;              // [kMaxG]: L
+  if (tid < kMaxG) {
+    float M = -INFINITY;
+    for (int i = first; i <= last; ++i)
+      if (cta_has_chunks(i, C, P)) M = fmaxf(M, __ldcg(part_slot(a, u + i) + tid * PF));
+    if (has_sink) M = fmaxf(M, __ldcg(sink + tid * PF));
+    float L = 0.f;
+    for (int i = first; i <= last; ++i) {
+      if (!cta_has_chunks(i, C, P)) continue;
+      const float* pp = part_slot(a, u + i) + tid * PF;
+      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - M);
+    }
+    if (has_sink) L += __ldcg(sink + tid * PF + 1) * exp2f(__ldcg(sink + tid * PF) - M);
+    mm[tid] = M;
+    ll[tid] = L;
+  }
+  consumers_sync();
+  const int width = VPROD ? 2 * kDim : kDim;
+  for (int i = tid; i < G * width; i += NT) {
+    const int h = i / width, j = i % width;
+    float s = 0.f;
+    for (int k = first; k <= last; ++k) {
+      if (!cta_has_chunks(k, C, P)) continue;
+      const float* pp = part_slot(a, u + k) + h * PF;
+      s += __ldcg(pp + 2 + j) * exp2f(__ldcg(pp) - mm[h]);
+    }
+    if (j < kDim) s = Fmt<VF>::width(j) > 0 ? s / a.sig[Fmt<VF>::width(j)] : 0.f;
+    acc[h * 2 * kDim + j] = s;
+  }
+  for (int i = tid; i < G * kDim; i += NT) {
+    const int h = i / kDim, j = i % kDim;
+    osk[h * kDim + j] = has_sink ? __ldcg(sink + h * PF + 2 + j) * exp2f(__ldcg(sink + h * PF) - mm[h]) : 0.f;
+  }
+  consumers_sync();
+  const int b = u / a.hkv, kvh = u % a.hkv;
+  for (int i = tid; i < G * kDim; i += NT) {
+    const int h = i / kDim, o = i % kDim;
+    float r = 0.f;
+    const float* ah = acc + h * 2 * kDim;
+    for (int j = 0; j < kDim; ++j) r = fmaf(a.pi[j * kDim + o], ah[j], r);
+    if (VPROD) {
+      float z = 0.f;
+      for (int l = 0; l < kSketch; ++l) z = fmaf(a.s[l * kDim + o], ah[kDim + l], z);
+      r = fmaf(kQjlScale, z, r);
+    }
+    const float L = ll[h];
+    store_out(a, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + o, L > 0.f ? (r + osk[h * kDim + o]) / L : 0.f);
+  }
+}
+
+// Count this piece of unit u; the piece that completes the set merges.
+template <int VF>
+__device__ void publish_piece(const DecodeArgs& a, int u, int first, int last, bool has_sink, float* sm,
+                              volatile int* s_flag, volatile int* s_abort, int64_t C) {
+  __threadfence();
+  consumers_sync();
+  if (threadIdx.x == 0) {
+    int last_piece = 0;
+    if (!*s_abort) {
+      int expected = has_sink ? 1 : 0;
+      for (int i = first; i <= last; ++i) expected += cta_has_chunks(i, C, gridDim.x);
+      last_piece = atomicAdd(a.tickets + u, 1) == expected - 1;
+    }
+    *s_flag = last_piece;
+  }
+  consumers_sync();
+  if (*s_flag) {
+    __threadfence();
+    merge_unit<VF>(a, u, first, last, has_sink, sm, C);
+    if (threadIdx.x == 0) a.tickets[u] = 0;  // ready for the next call
+  }
+  consumers_sync();
+}
+
+// Cross-warp combine of one piece into partial slot `slot`, in 64-coordinate
+// slices of the accumulator (consumer threads).
 template <int KF, int VF, bool PACK>
-__global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1 : 2) decode_kernel(DecodeArgs a) {
+__device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& W, int64_t slot, float* sm,
+                            int warp, int g, int t) {
+  using FV = Fmt<VF>;
+  using VR = VRow<VF>;
+  constexpr int NT = kConsumers * 32;
+  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
+  constexpr int WD = FV::prod ? 2 * kDim : kDim;
+  const int tid = threadIdx.x;
+  float* wm = sm;                          // [warp][head]
+  float* wl = wm + kConsumers * kMaxG;     // [warp][head]
+  float* wacc = wl + kConsumers * kMaxG;   // [warp][head][kSliceDims]
+  float* dst = part_slot(a, slot);
+  const int PF = a.part_floats;
+  if (g == 0) {
+    wm[warp * kMaxG + 2 * t] = W.m0;
+    wm[warp * kMaxG + 2 * t + 1] = W.m1;
+    wl[warp * kMaxG + 2 * t] = W.l0;
+    wl[warp * kMaxG + 2 * t + 1] = W.l1;
+  }
+#pragma unroll 1
+  for (int pass = 0; pass < WD / kSliceDims; ++pass) {
+    const int lo = pass * kSliceDims;
+#pragma unroll
+    for (int mt = 0; mt < VMT; ++mt) {
+      int d0, d1;
+      if (mt < 8) {
+        if (FV::nseg > 1 && mt >= VR::S0::MT) {
+          d0 = VR::S1::dim(64, g, mt - VR::S0::MT, 0);
+          d1 = VR::S1::dim(64, g, mt - VR::S0::MT, 1);
+        } else {
+          d0 = VR::S0::dim(0, g, mt, 0);
+          d1 = VR::S0::dim(0, g, mt, 1);
+        }
+      } else {
+        d0 = kDim + VR::Q::dim(0, g, mt - 8, 0);
+        d1 = kDim + VR::Q::dim(0, g, mt - 8, 1);
+      }
+      float* w0 = wacc + (warp * kMaxG + 2 * t) * kSliceDims - lo;
+      float* w1 = wacc + (warp * kMaxG + 2 * t + 1) * kSliceDims - lo;
+      if (d0 >= lo && d0 < lo + kSliceDims) {
+        w0[d0] = W.oacc[mt][0];
+        w1[d0] = W.oacc[mt][1];
+      }
+      if (d1 >= lo && d1 < lo + kSliceDims) {
+        w0[d1] = W.oacc[mt][2];
+        w1[d1] = W.oacc[mt][3];
+      }
+    }
+    consumers_sync();
+    for (int i = tid; i < kMaxG * kSliceDims; i += NT) {
+      const int h = i / kSliceDims, j = i % kSliceDims;
+      float M = -INFINITY;
+      for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
+      float s = 0.f, l = 0.f;
+      for (int w = 0; w < kConsumers; ++w) {
+        const float mw = wm[w * kMaxG + h];
+        if (mw > -INFINITY) {
+          const float f = exp2f(mw - M);
+          s += wacc[(w * kMaxG + h) * kSliceDims + j] * f;
+          l += wl[w * kMaxG + h] * f;
+        }
+      }
+      dst[h * PF + 2 + lo + j] = s;
+      if (pass == 0 && j == 0) {
+        dst[h * PF + 0] = M;
+        dst[h * PF + 1] = l;
+      }
+    }
+    consumers_sync();
+  }
+}
+
+// Sink piece of unit u: bf16 keys/values of tokens [0, ns) in the original
+// domain (consumer threads), into slot U + P + u.
+__device__ void sink_piece(const DecodeArgs& a, int u, int ns, float* sm) {
+  constexpr int NT = kConsumers * 32;
+  const int tid = threadIdx.x, G = a.group;
+  const int b = u / a.hkv, kvh = u % a.hkv;
+  const int U = a.B * a.hkv, P = gridDim.x;
+  float* qs = sm;                      // [8][128]
+  float* sc = qs + kMaxG * kDim;       // [8][n_sink]
+  float* red = sc + kMaxG * a.n_sink;  // [8][2]
+  float* dst = part_slot(a, U + P + u);
+  const int PF = a.part_floats;
+  for (int i = tid; i < kMaxG * kDim; i += NT) {
+    const int h = i / kDim, d = i % kDim;
+    qs[i] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
+  }
+  consumers_sync();
+  const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
+  const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
+  const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
+  for (int i = tid; i < G * ns; i += NT) {
+    const int h = i / ns, tok = i % ns;
+    float acc = 0.f;
+    for (int d = 0; d < kDim; ++d) acc = fmaf(__bfloat162float(ks[tok * kDim + d]), qs[h * kDim + d], acc);
+    sc[h * a.n_sink + tok] = acc * scale;
+  }
+  consumers_sync();
+  if (tid < G) {
+    float m = -INFINITY;
+    for (int tok = 0; tok < ns; ++tok) m = fmaxf(m, sc[tid * a.n_sink + tok]);
+    float l = 0.f;
+    for (int tok = 0; tok < ns; ++tok) {
+      const float p = exp2f(sc[tid * a.n_sink + tok] - m);
+      sc[tid * a.n_sink + tok] = p;
+      l += p;
+    }
+    red[2 * tid] = m;
+    red[2 * tid + 1] = l;
+  }
+  consumers_sync();
+  for (int i = tid; i < G * kDim; i += NT) {
+    const int h = i / kDim, d = i % kDim;
+    float acc = 0.f;
+    for (int tok = 0; tok < ns; ++tok) acc = fmaf(sc[h * a.n_sink + tok], __bfloat162float(vs[tok * kDim + d]), acc);
+    dst[h * PF + 2 + d] = acc;
+  }
+  if (tid < G) {
+    dst[tid * PF + 0] = red[2 * tid];
+    dst[tid * PF + 1] = red[2 * tid + 1];
+  }
+}
+
+template <int KF, int VF, bool PACK>
+__global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
-  using KR = KRow<KF>;
-  using VR = VRow<VF>;
   using L = Lut<KF, VF>;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  using SL = StageLayout<KF, VF>;
+  constexpr int S = decode_stages<KF, VF>();
+  constexpr int NX = PACK ? 1 : 2;
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* stages = smem + L::bytes;
+  float* scratch = reinterpret_cast<float*>(smem + L::bytes + S * SL::bytes);
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ long long s_C, s_c0, s_c1;
+  __shared__ int s_u0, s_lc0;
+  __shared__ volatile int s_abort, s_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int G = a.group;
+  const int P = gridDim.x, cta = blockIdx.x;
+  const int U = a.B * a.hkv;
 
-  int len = a.lens[b];
-  if (len > a.max_len) {
-    if (split == 0 && kvh == 0 && tid == 0) atomicOr(a.status, 2);
-    len = a.max_len;
-  }
-  if (len < 0) len = 0;
-  const int ns = min(a.n_sink, len);
-  const int nq = len - ns;
-  const int n_real = (nq + a.split_tokens - 1) / a.split_tokens;
-  const bool has_sink = ns > 0;
-  const int expected = n_real + (has_sink ? 1 : 0);
-  const int PF = a.part_floats;
-  float* part_base = a.parts + (static_cast<int64_t>(b) * a.hkv + kvh) * (a.n_splits + 1) * kMaxG * PF;
-  float* sm = reinterpret_cast<float*>(smem);
-
-  if (expected == 0) {
-    if (split == 0)
-      for (int i = tid; i < G * kDim; i += kThreads) {
-        const int64_t oi = (static_cast<int64_t>(b) * a.hq + kvh * G) * kDim + i;
-        if (a.out_bf16)
-          reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(0.f);
-        else
-          reinterpret_cast<float*>(a.out)[oi] = 0.f;
-      }
-    return;
-  }
-
-  if (split == a.n_splits) {
-    // ---- sink CTA: bf16 keys/values of tokens [0, ns), original domain ----
-    if (!has_sink) return;
-    float* qs = sm;                        // [8][128]
-    float* sc = qs + kMaxG * kDim;         // [8][n_sink]
-    float* red = sc + kMaxG * a.n_sink;    // [8][2]
-    for (int i = tid; i < kMaxG * kDim; i += kThreads) {
-      const int h = i / kDim, d = i % kDim;
-      qs[i] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
-    }
-    __syncthreads();
-    const uint16_t* ks = a.k_sink + (static_cast<int64_t>(b) * a.hkv + kvh) * a.n_sink * kDim;
-    const uint16_t* vs = a.v_sink + (static_cast<int64_t>(b) * a.hkv + kvh) * a.n_sink * kDim;
-    const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
-    for (int i = tid; i < G * ns; i += kThreads) {
-      const int h = i / ns, tok = i % ns;
-      float acc = 0.f;
-      for (int d = 0; d < kDim; ++d) {
-        const uint16_t kb = ks[tok * kDim + d];
-        acc = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&kb)), qs[h * kDim + d], acc);
-      }
-      sc[h * a.n_sink + tok] = acc * scale;
-    }
-    __syncthreads();
-    if (tid < G) {
-      float m = -INFINITY;
-      for (int tok = 0; tok < ns; ++tok) m = fmaxf(m, sc[tid * a.n_sink + tok]);
-      float l = 0.f;
-      for (int tok = 0; tok < ns; ++tok) {
-        const float p = exp2f(sc[tid * a.n_sink + tok] - m);
-        sc[tid * a.n_sink + tok] = p;
-        l += p;
-      }
-      red[2 * tid] = m;
-      red[2 * tid + 1] = l;
-    }
-    __syncthreads();
-    for (int i = tid; i < G * kDim; i += kThreads) {
-      const int h = i / kDim, d = i % kDim;
-      float acc = 0.f;
-      for (int tok = 0; tok < ns; ++tok) {
-        const uint16_t vb = vs[tok * kDim + d];
-        acc = fmaf(sc[h * a.n_sink + tok], __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&vb)), acc);
-      }
-      part_base[(a.n_splits * kMaxG + h) * PF + 2 + d] = acc;
-    }
-    if (tid < G) {
-      part_base[(a.n_splits * kMaxG + tid) * PF + 0] = red[2 * tid];
-      part_base[(a.n_splits * kMaxG + tid) * PF + 1] = red[2 * tid + 1];
-    }
-    __syncthreads();
-    finish_cta<VF>(a, b, kvh, expected, n_real, has_sink, sm);
-    return;
-  }
-
-  if (split >= n_real) return;
-
-  // ---- quantized split ----------------------------------------------------
-  // lookup tables
+  // ---- lookup tables (all threads), schedule and barriers (thread 0)
   {
     const float* cb = a.cbs;
     if constexpr (L::t4) {
-      for (int i = tid; i < 256 * 32; i += kThreads) {
+      for (int i = tid; i < 256 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
         *reinterpret_cast<uint32_t*>(smem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
       }
     }
     if constexpr (L::t3) {
-      for (int i = tid; i < 64 * 32; i += kThreads) {
+      for (int i = tid; i < 64 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
         *reinterpret_cast<uint32_t*>(smem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (r & 7)], cb[3 * kBookSlots + (r >> 3)]);
       }
     }
     if constexpr (L::t2) {
-      for (int i = tid; i < 256 * 32; i += kThreads) {
+      for (int i = tid; i < 256 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
         uint2 v;
         v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
@@ -970,96 +1092,155 @@ __global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1
       }
     }
   }
+  if (tid == 0) {
+    long long C = 0;
+    for (int u = 0; u < U; ++u) C += unit_info(a, u).chunks;
+    const long long c0 = range_start(cta, C, P), c1 = range_start(cta + 1, C, P);
+    int u0 = U, lc0 = 0;
+    long long acc = 0;
+    for (int u = 0; u < U && c0 < c1; ++u) {
+      const int ch = unit_info(a, u).chunks;
+      if (c0 < acc + ch) {
+        u0 = u;
+        lc0 = static_cast<int>(c0 - acc);
+        break;
+      }
+      acc += ch;
+    }
+    s_C = C;
+    s_c0 = c0;
+    s_c1 = c1;
+    s_u0 = u0;
+    s_lc0 = lc0;
+    s_abort = 0;
+    s_flag = 0;
+    if (cta == 0)
+      for (int b = 0; b < a.B; ++b)
+        if (a.lens[b] > a.max_len) atomicOr(a.status, 2);
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kConsumers);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const long long C = s_C, c0 = s_c0, c1 = s_c1;
+
+  if (warp == kConsumers) {
+    // ---- producer: one lane streams the CTA's chunks through the stages
+    if (lane == 0 && c0 < c1) {
+      int u = s_u0, lc = s_lc0;
+      UnitInfo ui = unit_info(a, u);
+      long long k = 0;
+      for (long long c = c0; c < c1; ++c, ++k) {
+        while (lc >= ui.chunks) {
+          ++u;
+          lc = 0;
+          ui = unit_info(a, u);
+        }
+        const int s = static_cast<int>(k % S);
+        if (k >= S && !mbar_wait(&empty_bar[s], static_cast<uint32_t>((k / S - 1) & 1))) s_abort = 1;
+        if (s_abort) break;
+        const int64_t ubase = static_cast<int64_t>(u) * a.capacity;
+        const int r0 = lc * kChunk;
+        const int rows = min(kChunk, (ui.nq + kTok - 1) / kTok * kTok - r0);  // <= capacity - r0
+        unsigned char* st = stages + s * SL::bytes;
+        uint64_t* bar = &full_bar[s];
+        mbar_expect_tx(bar, SL::tx_bytes(rows));
+        const int64_t row = ubase + r0;
+        if constexpr (FK::code_bytes > 0) bulk_g2s(st + SL::kc, a.k_codes + row * FK::code_bytes, rows * FK::code_bytes, bar);
+        if constexpr (FV::code_bytes > 0) bulk_g2s(st + SL::vc, a.v_codes + row * FV::code_bytes, rows * FV::code_bytes, bar);
+        bulk_g2s(st + SL::kn, a.k_norms + row, rows * 4, bar);
+        bulk_g2s(st + SL::vn, a.v_norms + row, rows * 4, bar);
+        if constexpr (FK::prod) {
+          bulk_g2s(st + SL::kq, a.k_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
+          bulk_g2s(st + SL::kr, a.k_res + row, rows * 4, bar);
+        }
+        if constexpr (FV::prod) {
+          bulk_g2s(st + SL::vq, a.v_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
+          bulk_g2s(st + SL::vr, a.v_res + row, rows * 4, bar);
+        }
+        ++lc;
+      }
+    }
+    return;
+  }
+
+  // ---- consumers
   const unsigned char* lut_a = smem;
   const unsigned char* lut_b = smem + L::region_b_off;
   const uint32_t lane4 = lane * 4, lane8 = lane * 8;
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
-
-  // query B-fragments
-  constexpr int NX = PACK ? 1 : 2;
-  const uint32_t* qf = a.qfrag + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  uint32_t bq[8][2][NX], bqs[8][2][NX];  // [kstep][b0,b1][hi,lo]
-#pragma unroll
-  for (int s = 0; s < 8; ++s)
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int x = 0; x < NX; ++x) {
-        bq[s][r][x] = qf[((s * 2 + r) * 2 + x) * 32 + lane];
-        if constexpr (FK::prod) bqs[s][r][x] = qf[(((8 + s) * 2 + r) * 2 + x) * 32 + lane];
-      }
-  __syncthreads();
-
-  WarpState<KF, VF, PACK> wst;
-  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
-#pragma unroll
-  for (int i = 0; i < VMT; ++i) wst.oacc[i][0] = wst.oacc[i][1] = wst.oacc[i][2] = wst.oacc[i][3] = 0.f;
-  wst.m0 = wst.m1 = -INFINITY;
-  wst.l0 = wst.l1 = 0.f;
-
-  const int t_begin = split * a.split_tokens;
-  const int t_end = min(nq, t_begin + a.split_tokens);
-  const int64_t ubase = (static_cast<int64_t>(b) * a.hkv + kvh) * a.capacity;
-  UnitPlanes u;
-  u.kcodes = a.k_codes + ubase * FK::code_bytes;
-  u.vcodes = a.v_codes + ubase * FV::code_bytes;
-  u.knorm = a.k_norms + ubase;
-  u.vnorm = a.v_norms + ubase;
-  u.kq = FK::prod ? a.k_qjl + ubase * (kSketch / 8) : nullptr;
-  u.vq = FV::prod ? a.v_qjl + ubase * (kSketch / 8) : nullptr;
-  u.kres = FK::prod ? a.k_res + ubase : nullptr;
-  u.vres = FV::prod ? a.v_res + ubase : nullptr;
   const float thr = a.sparse_thr;
 
-  // software pipeline: the loads of the warp's next tile are in flight while
-  // the current one is decoded (two register buffers, no copies)
-  // TMA pipeline: thread 0 streams kChunk-token chunks of the split into a
-  // ring of shared-memory stages (one bulk copy per plane); warp w decodes
-  // tile w of each chunk.
-  using SL = StageLayout<KF, VF>;
-  constexpr int kStages = decode_stages<KF, VF>();
-  unsigned char* stages = smem + L::bytes;
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ int s_abort;
-  const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
-  const int t_end16 = (t_end + kTok - 1) / kTok * kTok;  // <= capacity (a multiple of 64)
-  auto issue = [&](int c) {
-    unsigned char* st = stages + (c % kStages) * SL::bytes;
-    const int r0 = t_begin + c * kChunk;
-    const int rows = min(kChunk, t_end16 - r0);
-    uint64_t* bar = &full_bar[c % kStages];
-    mbar_expect_tx(bar, SL::tx_bytes(rows));
-    if constexpr (FK::code_bytes > 0)
-      bulk_g2s(st + SL::kc, u.kcodes + static_cast<int64_t>(r0) * FK::code_bytes, rows * FK::code_bytes, bar);
-    if constexpr (FV::code_bytes > 0)
-      bulk_g2s(st + SL::vc, u.vcodes + static_cast<int64_t>(r0) * FV::code_bytes, rows * FV::code_bytes, bar);
-    bulk_g2s(st + SL::kn, u.knorm + r0, rows * 4, bar);
-    bulk_g2s(st + SL::vn, u.vnorm + r0, rows * 4, bar);
-    if constexpr (FK::prod) {
-      bulk_g2s(st + SL::kq, u.kq + r0 * (kSketch / 8), rows * (kSketch / 8), bar);
-      bulk_g2s(st + SL::kr, u.kres + r0, rows * 4, bar);
+  // sink pieces and empty sequences of the units u = cta (mod P)
+  for (int u = cta; u < U; u += P) {
+    const UnitInfo ui = unit_info(a, u);
+    if (ui.len == 0) {
+      const int b = u / a.hkv, kvh = u % a.hkv;
+      for (int i = tid; i < a.group * kDim; i += kConsumers * 32)
+        store_out(a, (static_cast<int64_t>(b) * a.hq + kvh * a.group) * kDim + i, 0.f);
+      continue;
     }
-    if constexpr (FV::prod) {
-      bulk_g2s(st + SL::vq, u.vq + r0 * (kSketch / 8), rows * (kSketch / 8), bar);
-      bulk_g2s(st + SL::vr, u.vres + r0, rows * 4, bar);
+    if (ui.ns == 0) continue;
+    sink_piece(a, u, ui.ns, scratch);
+    int first = 1, last = 0;
+    if (ui.chunks > 0) {
+      long long cu0 = 0;
+      for (int v = 0; v < u; ++v) cu0 += unit_info(a, v).chunks;
+      first = cta_of_chunk(cu0, C, P);
+      last = cta_of_chunk(cu0 + ui.chunks - 1, C, P);
     }
-  };
-  if (tid == 0) {
-    s_abort = 0;
-#pragma unroll
-    for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
-    mbar_fence_init();
+    publish_piece<VF>(a, u, first, last, true, scratch, &s_flag, &s_abort, C);
   }
-  __syncthreads();
-  if (tid == 0)
-    for (int c = 0; c < min(kStages, n_chunks); ++c) issue(c);
-  int issued = min(kStages, n_chunks);
-  for (int c = 0; c < n_chunks; ++c) {
-    if (!mbar_wait(&full_bar[c % kStages], (c / kStages) & 1)) s_abort = 1;
-    const int row0 = t_begin + c * kChunk + warp * kTok;
-    if (row0 < t_end && !s_abort) {
-      const unsigned char* st = stages + (c % kStages) * SL::bytes;
+
+  WarpState<KF, VF, PACK> wst;
+  uint32_t bq[8][2][NX], bqs[8][2][NX];
+  int u = -1;
+  UnitInfo ui{};
+  long long cu0 = 0;
+  int walk_u = s_u0, walk_lc = s_lc0;
+  UnitInfo wui = c0 < c1 ? unit_info(a, walk_u) : UnitInfo{};
+  long long walk_cu0 = c0 - s_lc0;
+  long long k = 0;
+  for (long long c = c0; c < c1; ++c, ++k) {
+    while (walk_lc >= wui.chunks) {
+      walk_cu0 += wui.chunks;
+      ++walk_u;
+      walk_lc = 0;
+      wui = unit_info(a, walk_u);
+    }
+    if (walk_u != u) {
+      if (u >= 0) {
+        write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
+        publish_piece<VF>(a, u, cta_of_chunk(cu0, C, P), cta_of_chunk(cu0 + ui.chunks - 1, C, P), ui.ns > 0,
+                          scratch, &s_flag, &s_abort, C);
+      }
+      u = walk_u;
+      ui = wui;
+      cu0 = walk_cu0;
+      const uint32_t* qf = a.qfrag + static_cast<int64_t>(u) * kQfragWords;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int x = 0; x < NX; ++x) {
+            bq[s][r][x] = qf[((s * 2 + r) * 2 + x) * 32 + lane];
+            if constexpr (FK::prod) bqs[s][r][x] = qf[(((8 + s) * 2 + r) * 2 + x) * 32 + lane];
+          }
+#pragma unroll
+      for (int i = 0; i < WarpState<KF, VF, PACK>::VMT; ++i) wst.oacc[i][0] = wst.oacc[i][1] = wst.oacc[i][2] = wst.oacc[i][3] = 0.f;
+      wst.m0 = wst.m1 = -INFINITY;
+      wst.l0 = wst.l1 = 0.f;
+    }
+    const int s = static_cast<int>(k % S);
+    if (!s_abort && !mbar_wait(&full_bar[s], static_cast<uint32_t>((k / S) & 1))) s_abort = 1;
+    const int row0 = walk_lc * kChunk + warp * kTok;
+    if (!s_abort && row0 < ui.nq) {
+      const unsigned char* st = stages + s * SL::bytes;
       UnitPlanes sp;
       sp.kcodes = st + SL::kc;
       sp.vcodes = st + SL::vc;
@@ -1071,102 +1252,37 @@ __global__ void __launch_bounds__(kThreads, (Fmt<KF>::prod || Fmt<VF>::prod) ? 1
       sp.vres = reinterpret_cast<const float*>(st + SL::vr);
       Tile<KF, VF> tl;
       load_tile(tl, sp, warp * kTok, g, t);
-      compute_tile<KF, VF, PACK>(tl, wst, bq, bqs, row0, t_end, g, lut_a, lut_b, lane4, lane8, c1k, c1v, thr);
+      compute_tile<KF, VF, PACK>(tl, wst, bq, bqs, row0, ui.nq, g, lut_a, lut_b, lane4, lane8, c1k, c1v, thr);
     }
-    __syncthreads();  // stage c % kStages is free again
-    if (s_abort) break;
-    if (tid == 0 && issued < n_chunks) {
-      fence_proxy_async();
-      issue(issued);
-      ++issued;
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    ++walk_lc;
   }
-  if (s_abort) {
-    // a copy never completed: flag it, drain what was issued (bounded) and
-    // leave without publishing a partial
-    if (tid == 0) {
-      atomicOr(a.status, 4);
-      for (int c = 0; c < issued; ++c) mbar_wait(&full_bar[c % kStages], (c / kStages) & 1);
-    }
-    return;
+  if (u >= 0) {
+    write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
+    publish_piece<VF>(a, u, cta_of_chunk(cu0, C, P), cta_of_chunk(cu0 + ui.chunks - 1, C, P), ui.ns > 0, scratch,
+                      &s_flag, &s_abort, C);
   }
-  float (&oacc)[VMT][4] = wst.oacc;
-  const float m0 = wst.m0, m1 = wst.m1, l0 = wst.l0, l1 = wst.l1;
-
-  // ---- merge the warps of this CTA (shared memory reused after the loop)
-  __syncthreads();
-  constexpr int W = FV::prod ? 2 * kDim : kDim;  // accumulator width per head
-  float* wm = sm;                                // [warp][head]
-  float* wl = wm + kWarps * kMaxG;
-  float* wacc = wl + kWarps * kMaxG;             // [warp][head][W]
-  if (g == 0) {
-    wm[warp * kMaxG + 2 * t] = m0;
-    wm[warp * kMaxG + 2 * t + 1] = m1;
-    wl[warp * kMaxG + 2 * t] = l0;
-    wl[warp * kMaxG + 2 * t + 1] = l1;
-  }
-#pragma unroll
-  for (int mt = 0; mt < VMT; ++mt) {
-    int d0, d1;
-    if (mt < 8) {
-      if (FV::nseg > 1 && mt >= VR::S0::MT) {
-        d0 = VR::S1::dim(64, g, mt - VR::S0::MT, 0);
-        d1 = VR::S1::dim(64, g, mt - VR::S0::MT, 1);
-      } else {
-        d0 = VR::S0::dim(0, g, mt, 0);
-        d1 = VR::S0::dim(0, g, mt, 1);
-      }
-    } else {
-      d0 = kDim + VR::Q::dim(0, g, mt - 8, 0);
-      d1 = kDim + VR::Q::dim(0, g, mt - 8, 1);
-    }
-    float* w0 = wacc + (warp * kMaxG + 2 * t) * W;
-    float* w1 = wacc + (warp * kMaxG + 2 * t + 1) * W;
-    w0[d0] = oacc[mt][0];
-    w1[d0] = oacc[mt][1];
-    w0[d1] = oacc[mt][2];
-    w1[d1] = oacc[mt][3];
-  }
-  __syncthreads();
-  float* mine = part_base + static_cast<int64_t>(split) * kMaxG * PF;
-  for (int i = tid; i < kMaxG * W; i += kThreads) {
-    const int h = i / W, j = i % W;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = wm[w * kMaxG + h];
-      if (mw > -INFINITY) s += wacc[(w * kMaxG + h) * W + j] * exp2f(mw - M);
-    }
-    mine[h * PF + 2 + j] = s;
-    if (j == 0) {
-      float l = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = wm[w * kMaxG + h];
-        if (mw > -INFINITY) l += wl[w * kMaxG + h] * exp2f(mw - M);
-      }
-      mine[h * PF + 0] = M;
-      mine[h * PF + 1] = l;
-    }
-  }
-  __syncthreads();
-  finish_cta<VF>(a, b, kvh, expected, n_real, has_sink, sm);
+  if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+int num_sms_cached() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
 template <int KF, int VF>
-size_t decode_smem_bytes() {
-  using L = Lut<KF, VF>;
-  const size_t pipeline = static_cast<size_t>(L::bytes) + decode_stages<KF, VF>() * StageLayout<KF, VF>::bytes;
-  const size_t W = Fmt<VF>::prod ? 2 * kDim : kDim;
-  const size_t combine = (2 * kWarps * kMaxG + kWarps * kMaxG * W) * sizeof(float);
-  const size_t merge = (kMaxG * 2 * kDim + kMaxG * kDim + 2 * kMaxG) * sizeof(float);
-  return std::max<size_t>({pipeline, combine, merge, 24 * 1024});
+size_t decode_smem_bytes(int n_sink) {
+  return static_cast<size_t>(Lut<KF, VF>::bytes) + decode_stages<KF, VF>() * StageLayout<KF, VF>::bytes +
+         scratch_bytes(n_sink);
 }
 
 template <int KF, int VF, bool PACK>
@@ -1177,15 +1293,16 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
-  decode_kernel<KF, VF, PACK><<<dim3(plan.n_splits + 1, plan.hkv, plan.B), kThreads, smem, st>>>(a);
+  decode_kernel<KF, VF, PACK><<<plan.ctas, kThreadsP, smem, st>>>(a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "decode kernel launch");
 }
 
 template <int KF, int VF>
-tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, int sink_smem_floats, cudaStream_t st) {
-  size_t smem = decode_smem_bytes<KF, VF>();
-  smem = std::max<size_t>(smem, static_cast<size_t>(sink_smem_floats) * sizeof(float));
+tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
+  const size_t smem = decode_smem_bytes<KF, VF>(a.n_sink);
+  if (smem > static_cast<size_t>(kSmemBudget))
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink too large for the shared-memory plan");
   a.pack = plan.group <= 4;
   return a.pack ? run_decode_v<KF, VF, true>(a, plan, smem, st) : run_decode_v<KF, VF, false>(a, plan, smem, st);
 }
@@ -1201,25 +1318,13 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) 
   pl.hkv = hkv;
   pl.group = hq / hkv;
   pl.max_len = max_len;
-  int sms = 148;
-  {
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  const int64_t units = static_cast<int64_t>(B) * hkv;
-  const int64_t target = static_cast<int64_t>(sms) * 2 * 8;  // about eight waves of resident CTAs
-  int64_t per = (static_cast<int64_t>(std::max(max_len, 1)) * units + target - 1) / target;
-  const int quantum = kTok * kWarps;  // 128 tokens: one tile per warp
-  per = std::max<int64_t>(per, 4 * quantum);
-  per = (per + quantum - 1) / quantum * quantum;
-  pl.split_tokens = static_cast<int>(per);
-  pl.n_splits = std::max(1, static_cast<int>((std::max(max_len, 1) + per - 1) / per));
+  pl.ctas = num_sms_cached();
   pl.part_floats = 2 + (p->fv.prod ? 2 * kDim : kDim);
-  const size_t tickets = (static_cast<size_t>(units) * sizeof(int32_t) + 255) & ~size_t(255);
-  const size_t qfrag = static_cast<size_t>(units) * kQfragWords * sizeof(uint32_t);
-  pl.ws_partials_bytes = static_cast<size_t>(units) * (pl.n_splits + 1) * kMaxG * pl.part_floats * sizeof(float);
-  pl.ws_total_bytes = tickets + ((qfrag + 255) & ~size_t(255)) + pl.ws_partials_bytes;
+  const size_t units = static_cast<size_t>(B) * hkv;
+  const size_t tickets = (units * sizeof(int32_t) + 255) & ~size_t(255);
+  const size_t qfrag = (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
+  const size_t slots = 2 * units + pl.ctas;
+  pl.ws_total_bytes = tickets + qfrag + slots * kMaxG * pl.part_floats * sizeof(float);
   return pl;
 }
 
@@ -1240,14 +1345,13 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.v_sink = c->v_sink;
   a.lens = c->lens;
   a.status = c->status;
+  a.B = plan.B;
   a.hkv = plan.hkv;
   a.group = plan.group;
   a.hq = plan.hq;
   a.capacity = c->capacity;
   a.n_sink = c->n_sink;
   a.max_len = plan.max_len;
-  a.n_splits = plan.n_splits;
-  a.split_tokens = plan.split_tokens;
   a.part_floats = plan.part_floats;
   const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
   char* w = static_cast<char*>(ws);
@@ -1265,11 +1369,10 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.cbs = p->cbs32;
   a.sig = p->sig32;
   a.sparse_thr = sparse_thr;
-  const int sink_floats = kMaxG * kDim + kMaxG * c->n_sink + 2 * kMaxG + 64;
 
   const int kf = p->fk.id(), vf = p->fv.id();
 #define TQ_CASE(K, V) \
-  if (kf == (K) && vf == (V)) return run_decode<(K), (V)>(a, plan, sink_floats, st);
+  if (kf == (K) && vf == (V)) return run_decode<(K), (V)>(a, plan, st);
   // symmetric formats
   TQ_CASE(fid(1, 0, 0), fid(1, 0, 0))
   TQ_CASE(fid(2, 0, 0), fid(2, 0, 0))

@@ -71,8 +71,8 @@ tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_pa
                             int64_t n, float* out, cudaStream_t st);
 
 struct DecodePlan {
-  int B, hq, hkv, group, max_len, n_splits, split_tokens, part_floats;
-  size_t ws_partials_bytes, ws_total_bytes;
+  int B, hq, hkv, group, max_len, ctas, part_floats;
+  size_t ws_total_bytes;
 };
 DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len);
 tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c,
