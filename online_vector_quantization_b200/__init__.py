@@ -30,7 +30,7 @@ class TqError(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libtq.so is not built ({LIB_PATH}); run python -m online_vector_quantization_b200.build")
+    raise ImportError(f"libtq.so is not built ({LIB_PATH}); run python online_vector_quantization_b200/build.py")
 _lib = ctypes.CDLL(LIB_PATH)
 
 c_int, c_void_p, c_size_t, c_float, c_uint64, c_int64 = (
@@ -265,3 +265,4 @@ def tq_decode_attn(params: Params, q, cache: Cache, max_len: int, out, workspace
                                max_len, _ptr(out), _dtype_code(out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), ctypes.byref(flags),
                                _stream(stream)))
+

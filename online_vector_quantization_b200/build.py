@@ -1,6 +1,7 @@
 """Build libtq.so in-tree with nvcc for sm_100a (B200).
 
-Run as ``python -m online_vector_quantization_b200.build`` or call build().
+Run as ``python online_vector_quantization_b200/build.py`` (not with -m: the
+package import loads the library this script builds) or call build().
 The shared library exports the C ABI declared in include/tq.h.
 """
 from __future__ import annotations
