@@ -210,6 +210,23 @@ tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const t
                          void* workspace, size_t ws_bytes, const tq_attn_flags* flags,
                          void* stream);
 
+/* The same decode step as tq_decode_attn for callers that cannot allocate
+ * device memory (for example an engine that reserves all device memory for its
+ * own pool and calls this library from plugin code without a handle on that
+ * pool, or a decode loop that cannot afford cudaMalloc's implicit device
+ * synchronization).  No counterpart in the method's pages: it only changes
+ * where the workspace lives.  The workspace is a fixed 8 MiB array in device
+ * memory defined by the library (every GPU that loads the library holds it
+ * until the process exits); a call that would need more returns
+ * TQ_ERR_CAPACITY.  No cudaMalloc, cudaFree or other allocation happens.  The
+ * first call on each device looks up the array's address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array and each one clears what must start at zero, so
+ * calls that overlap on the GPU (for example on two streams) race. */
+tq_status tq_decode_attn_noalloc(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
+                                 int B, int hq, int max_len, void* out, int out_dtype,
+                                 const tq_attn_flags* flags, void* stream);
+
 /* Message for the last failed call on this host thread ("" if none). */
 const char* tq_last_error(void);
 

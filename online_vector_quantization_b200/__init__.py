@@ -77,6 +77,8 @@ _SIGS = {
     "tq_decode_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
     "tq_decode_attn": (c_int, [c_void_p, c_void_p, c_int, ctypes.POINTER(TqCache), c_int, c_int, c_int, c_void_p,
                                c_int, c_void_p, c_size_t, ctypes.POINTER(TqAttnFlags), c_void_p]),
+    "tq_decode_attn_noalloc": (c_int, [c_void_p, c_void_p, c_int, ctypes.POINTER(TqCache), c_int, c_int, c_int,
+                                       c_void_p, c_int, ctypes.POINTER(TqAttnFlags), c_void_p]),
     "tq_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -266,3 +268,12 @@ def tq_decode_attn(params: Params, q, cache: Cache, max_len: int, out, workspace
                                workspace.numel() * workspace.element_size(), ctypes.byref(flags),
                                _stream(stream)))
 
+
+def tq_decode_attn_noalloc(params: Params, q, cache: Cache, max_len: int, out, sparse_v_threshold: float = 0.0,
+                           stream=None):
+    """tq_decode_attn with the library's fixed device scratch instead of a
+    caller workspace (see include/tq.h)."""
+    B, hq = q.shape[0], q.shape[1]
+    flags = TqAttnFlags(sparse_v_threshold, 0)
+    _check(_lib.tq_decode_attn_noalloc(params.handle, _ptr(q), _dtype_code(q), ctypes.byref(cache.struct), B, hq,
+                                       max_len, _ptr(out), _dtype_code(out), ctypes.byref(flags), _stream(stream)))
