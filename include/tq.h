@@ -145,7 +145,9 @@ tq_status tq_dequantize(const tq_params* p, const tq_packed* in, int64_t n, int 
  * quantized rows.  lens: device int32 [n_seq], tokens held per sequence
  * (sink included); the caller zeroes it for an empty cache.  status: device
  * int32 word; kernels OR error bits into it (1 = append past capacity,
- * 2 = a length above the bound given to tq_decode_attn). */
+ * 2 = a length above the bound given to tq_decode_attn, 4 = a decode wait on
+ * the copy pipeline gave up after its time limit, 8 = the decode kernel's
+ * shared-memory layout did not fit; after 4 or 8 the outputs are invalid). */
 typedef struct {
   int n_seq, n_kv_heads, capacity, n_sink;
   uint8_t* k_codes; float* k_norms; uint8_t* k_qjl; float* k_res_norms;

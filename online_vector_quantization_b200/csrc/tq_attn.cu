@@ -77,10 +77,15 @@ struct Lut {
   static constexpr bool t4 = Fmt<KF>::uses(4) || Fmt<VF>::uses(4);
   static constexpr bool t3 = Fmt<KF>::uses(3) || Fmt<VF>::uses(3);
   static constexpr bool t2 = Fmt<KF>::uses(2) || Fmt<VF>::uses(2);
-  static constexpr int region_a = t4 ? 65536 : (t3 ? 16384 : 0);
-  static constexpr int region_b_off = region_a;
+  static constexpr int region_a = (t4 || (t3 && t2)) ? 65536 : (t3 ? 16384 : 0);
+  static constexpr int region_b_off = region_a;  // 0 or 65536: a 64 KB boundary
   static constexpr int bytes = region_a + (t2 ? 65536 : 0);
 };
+
+// The tables live at shared-window address kLutAddr (64 KB aligned), so a
+// lookup address is (code byte << 8) | lane offset | table base, formed by a
+// single byte permute or logic op with the base folded into the lane offset.
+constexpr uint32_t kLutAddr = 0x10000;
 
 __device__ __forceinline__ uint32_t h2bits(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -106,17 +111,29 @@ __device__ __forceinline__ void static_for(Fn&& fn) {
   }
 }
 
-__device__ __forceinline__ uint32_t lds32(const unsigned char* smem, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(smem + off);
+// Shared-memory loads on 32-bit shared-window addresses (`base` is the
+// shared address of a table or stage, `off` a byte offset).
+__device__ __forceinline__ uint32_t lds32(uint32_t base, uint32_t off) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(base + off));
+  return v;
 }
-
-__device__ __forceinline__ uint2 lds64(const unsigned char* smem, uint32_t off) {
-  return *reinterpret_cast<const uint2*>(smem + off);
+__device__ __forceinline__ uint2 lds64(uint32_t base, uint32_t off) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(base + off));
+  return v;
 }
+__device__ __forceinline__ uint4 lds128(uint32_t base, uint32_t off) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(base + off));
+  return v;
+}
+__device__ __forceinline__ float ldsf(uint32_t base, uint32_t off) { return __uint_as_float(lds32(base, off)); }
 
-// byte k of w placed at bits 8..15, lane offset `lb` (< 256) at bits 0..7
+// byte k of w placed at bits 8..15; bits 0..7 and 16..31 from lb (the lane
+// offset and the table base; lb's bits 8..15 are zero)
 __device__ __forceinline__ uint32_t byte_addr(uint32_t w, uint32_t lb, int k) {
-  return __byte_perm(w, lb, 0x5504 | (k << 4));
+  return __byte_perm(w, lb, 0x7604 | (k << 4));
 }
 
 // half2 of +-c from bits p and p+16 of w (bit set -> +c); c_bits = half2(c, c)
@@ -148,12 +165,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
-// addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+// 1-D bulk copy global -> this CTA's shared memory at shared address `dst`
+// (no multicast); both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s_addr(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-          smem_u32(dst)),
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
@@ -213,27 +229,26 @@ struct KChunk {
   static constexpr int KSTEPS = ND / 16;
   uint32_t w[WORDS];
 
-  __device__ __forceinline__ void load(const uint8_t* row, int t) {
+  // row: shared address of the token's code row
+  __device__ __forceinline__ void load(uint32_t row, int t) {
     const int o = BYTE0 + t * BYTES;
     if constexpr (BYTES == 16) {
-      const uint4 v = *reinterpret_cast<const uint4*>(row + o);
+      const uint4 v = lds128(row, o);
       w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     } else if constexpr (BYTES == 12) {
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(row + o);
-      w[0] = p[0]; w[1] = p[1]; w[2] = p[2];
+      w[0] = lds32(row, o); w[1] = lds32(row, o + 4); w[2] = lds32(row, o + 8);
     } else if constexpr (BYTES == 8) {
-      const uint2 v = *reinterpret_cast<const uint2*>(row + o);
+      const uint2 v = lds64(row, o);
       w[0] = v.x; w[1] = v.y;
     } else if constexpr (BYTES == 6) {
       const int al = o & ~3;
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(row + al);
-      const uint32_t lo = p[0], hi = p[1];
+      const uint32_t lo = lds32(row, al), hi = lds32(row, al + 4);
       const int sh = (o & 3) * 8;
       w[0] = __funnelshift_r(lo, hi, sh);
       w[1] = hi >> sh;
     } else {
       static_assert(BYTES == 4, "unsupported K chunk");
-      w[0] = *reinterpret_cast<const uint32_t*>(row + o);
+      w[0] = lds32(row, o);
     }
   }
 
@@ -251,7 +266,7 @@ struct KChunk {
 
   // k-step S: (lo, hi) = A-fragment registers for k = 2t..2t+1 and 2t+8..2t+9
   template <int S>
-  __device__ __forceinline__ void decode(const unsigned char* smem, uint32_t lane4, uint32_t lane8,
+  __device__ __forceinline__ void decode(uint32_t smem, uint32_t lane4, uint32_t lane8,
                                          uint32_t c_bits, uint32_t& lo, uint32_t& hi) const {
     constexpr int s = S;
     if constexpr (B == 4) {
@@ -288,31 +303,31 @@ struct VChunk {
   static constexpr int MT = ND / 16;          // m-tiles of the segment
   uint64_t x;
 
-  __device__ __forceinline__ void load(const uint8_t* row, int g) {
+  __device__ __forceinline__ void load(uint32_t row, int g) {
     constexpr int bits = ND * B / 8;
     if constexpr (bits == 64) {
-      x = *reinterpret_cast<const uint64_t*>(row + BYTE0 + 8 * g);
+      const uint2 v = lds64(row, BYTE0 + 8 * g);
+      x = static_cast<uint64_t>(v.x) | (static_cast<uint64_t>(v.y) << 32);
     } else if constexpr (bits == 32) {
-      x = *reinterpret_cast<const uint32_t*>(row + BYTE0 + 4 * g);
+      x = lds32(row, BYTE0 + 4 * g);
     } else if constexpr (bits == 16) {
-      x = *reinterpret_cast<const uint16_t*>(row + BYTE0 + 2 * g);
+      const int o = BYTE0 + 2 * g;
+      x = (lds32(row, o & ~3) >> ((o & 2) * 8)) & 0xFFFFu;
     } else if constexpr (bits == 48) {
       const int o = BYTE0 + 6 * g, al = o & ~3;
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(row + al);
-      const uint64_t v = static_cast<uint64_t>(p[0]) | (static_cast<uint64_t>(p[1]) << 32);
+      const uint64_t v = static_cast<uint64_t>(lds32(row, al)) | (static_cast<uint64_t>(lds32(row, al + 4)) << 32);
       x = (v >> ((o & 3) * 8)) & 0xFFFFFFFFFFFFull;
     } else {
       static_assert(bits == 24, "unsupported V chunk");
       const int o = BYTE0 + 3 * g, al = o & ~3, sh = (o & 3) * 8;
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(row + al);
-      uint64_t v = p[0];
-      if (sh > 8) v |= static_cast<uint64_t>(p[1]) << 32;  // field crosses into the next word
+      uint64_t v = lds32(row, al);
+      if (sh > 8) v |= static_cast<uint64_t>(lds32(row, al + 4)) << 32;  // field crosses into the next word
       x = (v >> sh) & 0xFFFFFFull;
     }
   }
 
   // rows g (coordinate 2mt) and g+8 (2mt+1) for every m-tile, tokens (A, B)
-  __device__ __forceinline__ static void decode(const VChunk& a, const VChunk& b, const unsigned char* smem,
+  __device__ __forceinline__ static void decode(const VChunk& a, const VChunk& b, uint32_t smem,
                                                 uint32_t lane4, uint32_t lane8, uint32_t c_bits,
                                                 uint32_t (&rg)[MT], uint32_t (&rg8)[MT]) {
     if constexpr (B == 4) {
@@ -329,14 +344,20 @@ struct VChunk {
         }
       }
     } else if constexpr (B == 3) {
-      const uint64_t m = field_mask3<MT>();
-      const uint64_t ev = (a.x & m) | ((b.x & m) << 3);
-      const uint64_t od = ((a.x >> 3) & m) | (b.x & (m << 3));
+      // 24-bit halves of 8 codes: interleave the two tokens' 3-bit fields
+      // into 6-bit (A | B << 3) fields, evens and odds apart
+      constexpr uint32_t E = 0x1C71C7u;  // 3-bit fields at bits 0, 6, 12, 18
       const uint32_t lb = lane4 + 128;
-      static_for<MT>([&](auto kk) {
-        constexpr int k = decltype(kk)::value;
-        rg[k] = lds32(smem, addr6<6 * k>(ev, lb));
-        rg8[k] = lds32(smem, addr6<6 * k>(od, lb));
+      static_for<MT / 4>([&](auto hh) {
+        constexpr int h = decltype(hh)::value;
+        const uint32_t xa = static_cast<uint32_t>(a.x >> (24 * h)), xb = static_cast<uint32_t>(b.x >> (24 * h));
+        const uint32_t ev = (xa & E) | ((xb << 3) & ~E);
+        const uint32_t od = ((xa >> 3) & E) | (xb & ~E);
+        static_for<4>([&](auto kk) {
+          constexpr int k = decltype(kk)::value;
+          rg[4 * h + k] = lds32(smem, addr6<6 * k>(ev, lb));
+          rg8[4 * h + k] = lds32(smem, addr6<6 * k>(od, lb));
+        });
       });
     } else if constexpr (B == 2) {
       const uint32_t xa = static_cast<uint32_t>(a.x), xb = static_cast<uint32_t>(b.x);
@@ -408,6 +429,7 @@ struct DecodeArgs {
   const float* sig;  // sigma per width [5]
   float sparse_thr;
   int pack;          // 1: group <= 4, query hi/lo halves share one MMA (columns g and g+4)
+  uint32_t dyn_bytes;  // dynamic shared memory granted to the decode kernel
 };
 
 __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
@@ -506,37 +528,16 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// One warp tile: 16 tokens, the registers a lane needs from them.
-// ---------------------------------------------------------------------------
-template <int KF, int VF>
-struct Tile {
-  typename KRow<KF>::S0 k0A, k0B;
-  typename KRow<KF>::S1 k1A, k1B;
-  typename KRow<KF>::Q kqA, kqB;
-  typename VRow<VF>::S0 v0[4];
-  typename VRow<VF>::S1 v1[4];
-  typename VRow<VF>::Q vq[4];
-  float nkA, nkB, nvA, nvB, gkA, gkB, gvA, gvB;
-};
-
+// Shared addresses of the planes of one staged chunk.
 struct UnitPlanes {
-  const uint8_t* kcodes;
-  const uint8_t* vcodes;
-  const float* knorm;
-  const float* vnorm;
-  const uint8_t* kq;
-  const uint8_t* vq;
-  const float* kres;
-  const float* vres;
+  uint32_t kcodes, vcodes, knorm, vnorm, kq, vq, kres, vres;
 };
 
-// One pipeline stage in shared memory: the planes of kChunk consecutive
-// tokens, each copied by one bulk copy.
+// One pipeline stage in shared memory: the planes of CH consecutive tokens,
+// each copied by one bulk copy.
 constexpr int kConsumers = 15;                // consumer warps of the persistent kernel
 constexpr int kThreadsP = (kConsumers + 1) * 32;  // + one producer warp
-constexpr int kChunk = kTok * kConsumers;       // 240 tokens: one tile per consumer warp
-template <int KF, int VF>
+template <int KF, int VF, int kChunk>
 struct StageLayout {
   static constexpr int kc = 0;
   static constexpr int vc = kc + kChunk * Fmt<KF>::code_bytes;
@@ -553,59 +554,47 @@ struct StageLayout {
   }
 };
 
-// Shared memory of the persistent kernel: LUT | pipeline stages | scratch
-// (warp combine in 64-coordinate slices, split merge, sink scores).
+// Shared memory of the persistent kernel: pipeline stages, the lookup tables at
+// kLutAddr, and a scratch area (warp combine in 64-coordinate slices, split
+// merge, sink scores).  Stages go below kLutAddr while they fit, the rest
+// above the tables.
 constexpr int kSliceDims = 64;
 __host__ __device__ constexpr int scratch_bytes(int n_sink) {
   const int combine = (kConsumers * kMaxG * kSliceDims + 2 * kConsumers * kMaxG) * 4;
-  const int merge = (kMaxG * 3 * kDim + 2 * kMaxG) * 4;
+  const int merge = (kMaxG * 5 * kDim + 2 * kMaxG) * 4;
   const int sink = (kMaxG * kDim + kMaxG * n_sink + 2 * kMaxG) * 4;
   return combine > merge ? (combine > sink ? combine : sink) : (merge > sink ? merge : sink);
 }
-constexpr int kSmemBudget = 227 * 1024 - 1024;  // per block, minus static shared memory
-template <int KF, int VF>
-__host__ __device__ constexpr int decode_stages() {
-  return Lut<KF, VF>::bytes + 4 * StageLayout<KF, VF>::bytes + scratch_bytes(128) <= kSmemBudget   ? 4
-         : Lut<KF, VF>::bytes + 3 * StageLayout<KF, VF>::bytes + scratch_bytes(128) <= kSmemBudget ? 3
-                                                                                                  : 2;
+constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic bytes requested per block
+constexpr int kDynBaseMax = 4096;                // assumed upper bound of the dynamic base address
+constexpr int kSmemEnd = 227 * 1024;             // assumed end of the usable shared window
+
+__host__ __device__ constexpr int plan_end(int stage, int n_stages, int lut, int scratch) {
+  int cur = kDynBaseMax, in_gap = 0;
+  while (in_gap < n_stages && cur + stage <= static_cast<int>(kLutAddr)) {
+    cur += stage;
+    ++in_gap;
+  }
+  const bool scratch_low = cur + scratch <= static_cast<int>(kLutAddr);
+  return static_cast<int>(kLutAddr) + lut + (n_stages - in_gap) * stage + (scratch_low ? 0 : scratch);
 }
 
-// Lane loads of one tile from a staged chunk (or any planes with the same row
-// layout); rows row0 .. row0+15 exist in every plane, rows at or past the
-// sequence length hold stale data and are masked when used.
+// Chunk shape of a format pair: tokens per consumer warp (32 or 16) and the
+// number of stages, the deepest that fits.
 template <int KF, int VF>
-__device__ __forceinline__ void load_tile(Tile<KF, VF>& T, const UnitPlanes& u, int row0, int g, int t) {
-  using FK = Fmt<KF>;
-  using FV = Fmt<VF>;
-  const int rA = row0 + g, rB = row0 + g + 8;
-  const uint8_t* ka = u.kcodes + static_cast<int64_t>(rA) * FK::code_bytes;
-  const uint8_t* kb = u.kcodes + static_cast<int64_t>(rB) * FK::code_bytes;
-  if constexpr (FK::nseg > 0) { T.k0A.load(ka, t); T.k0B.load(kb, t); }
-  if constexpr (FK::nseg > 1) { T.k1A.load(ka, t); T.k1B.load(kb, t); }
-  if constexpr (FK::prod) {
-    T.kqA.load(u.kq + rA * (kSketch / 8), t);
-    T.kqB.load(u.kq + rB * (kSketch / 8), t);
-    T.gkA = u.kres[rA];
-    T.gkB = u.kres[rB];
-  }
-  T.nkA = u.knorm[rA];
-  T.nkB = u.knorm[rB];
-  T.nvA = u.vnorm[rA];
-  T.nvB = u.vnorm[rB];
-  if constexpr (FV::prod) {
-    T.gvA = u.vres[rA];
-    T.gvB = u.vres[rB];
-  }
-  const int v0 = row0 + 2 * t;  // tokens v0, v0+1, v0+8, v0+9
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = v0 + (i & 1) + 8 * (i >> 1);
-    const uint8_t* vr = u.vcodes + static_cast<int64_t>(r) * FV::code_bytes;
-    if constexpr (FV::nseg > 0) T.v0[i].load(vr, g);
-    if constexpr (FV::nseg > 1) T.v1[i].load(vr, g);
-    if constexpr (FV::prod) T.vq[i].load(u.vq + r * (kSketch / 8), g);
-  }
-}
+struct DecodeCfg {
+  static constexpr int lut = Lut<KF, VF>::bytes;
+  static constexpr int scr = scratch_bytes(128);
+  static constexpr int s32 = StageLayout<KF, VF, 32 * kConsumers>::bytes;
+  static constexpr int s16 = StageLayout<KF, VF, 16 * kConsumers>::bytes;
+  static constexpr bool fit32 = plan_end(s32, 2, lut, scr) <= kSmemEnd;
+  static constexpr int WT = fit32 ? 32 : 16;
+  static constexpr int CH = WT * kConsumers;
+  static constexpr int stage = fit32 ? s32 : s16;
+  static constexpr int S = plan_end(stage, 4, lut, scr) <= kSmemEnd   ? 4
+                           : plan_end(stage, 3, lut, scr) <= kSmemEnd ? 3
+                                                                       : 2;
+};
 
 template <int KF, int VF, bool PACK>
 struct WarpState {
@@ -614,65 +603,75 @@ struct WarpState {
   float m0, m1, l0, l1;
 };
 
-template <int KF, int VF, bool PACK>
-__device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF, VF, PACK>& W,
-                                             const uint32_t (&bq)[8][2][PACK ? 1 : 2],
-                                             const uint32_t (&bqs)[8][2][PACK ? 1 : 2], int row0, int t_end,
-                                             int g, const unsigned char* lut_a, const unsigned char* lut_b,
-                                             uint32_t lane4, uint32_t lane8, uint32_t c1k, uint32_t c1v,
-                                             float thr) {
-  using FK = Fmt<KF>;
-  using FV = Fmt<VF>;
-  using KR = KRow<KF>;
-  using VR = VRow<VF>;
-  constexpr int NX = PACK ? 1 : 2;
-  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
-  const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
-  const bool okA = row0 + g < t_end, okB = row0 + g + 8 < t_end;
+template <bool PACK>
+using QFrag = uint32_t[8][2][PACK ? 1 : 2];
 
-  // ---- scores S^T (tokens x columns), four independent MMA accumulator chains
-  float ca[4][4], cq[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) ca[i][j] = cq[i][j] = 0.f;
+// Scores of one 16-token subtile whose rows start at `srow` of the staged
+// planes: s2 (base 2) for tokens g (s2[0], s2[1]) and g+8 (s2[2], s2[3]),
+// columns 2t, 2t+1; masked tokens get -inf.  Two MMA accumulator chains.
+template <int KF, bool PACK>
+__device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, bool okA, bool okB, int g, int t,
+                                               const QFrag<PACK>& bq, const QFrag<PACK>& bqs,
+                                               uint32_t lut_a, uint32_t lut_b,
+                                               uint32_t lane4, uint32_t lane8, uint32_t c1k, float (&s2)[4]) {
+  using FK = Fmt<KF>;
+  using KR = KRow<KF>;
+  constexpr int NX = PACK ? 1 : 2;
+  const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
+  const int rA = srow + g, rB = srow + g + 8;
+  const uint32_t ka = u.kcodes + rA * FK::code_bytes;
+  const uint32_t kb = u.kcodes + rB * FK::code_bytes;
+  float ca[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float cq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   if constexpr (FK::nseg > 0) {
-    const unsigned char* lk = FK::b0 == 2 ? lut_b : lut_a;
+    typename KR::S0 xa, xb;
+    xa.load(ka, t);
+    xb.load(kb, t);
+    const uint32_t lk = FK::b0 == 2 ? lut_b : lut_a;
     static_for<KR::S0::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      T.k0A.template decode<s>(lk, lane4, lane8, c1k, la, ha);
-      T.k0B.template decode<s>(lk, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s>(lk, lane4, lane8, c1k, la, ha);
+      xb.template decode<s>(lk, lane4, lane8, c1k, lb, hb);
 #pragma unroll
-      for (int x = 0; x < NX; ++x) mma16816(ca[(NX * s + x) & 3], la, lb, ha, hb, bq[s][0][x], bq[s][1][x]);
+      for (int x = 0; x < NX; ++x) mma16816(ca[(NX * s + x) & 1], la, lb, ha, hb, bq[s][0][x], bq[s][1][x]);
     });
   }
   if constexpr (FK::nseg > 1) {
+    typename KR::S1 xa, xb;
+    xa.load(ka, t);
+    xb.load(kb, t);
     static_for<KR::S1::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      T.k1A.template decode<s>(lut_a, lane4, lane8, c1k, la, ha);
-      T.k1B.template decode<s>(lut_a, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s>(lut_a, lane4, lane8, c1k, la, ha);
+      xb.template decode<s>(lut_a, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x)
-        mma16816(ca[(NX * s + x + 2) & 3], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
+        mma16816(ca[(NX * s + x + 1) & 1], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
     });
   }
+  float gA = 0.f, gB = 0.f;
   if constexpr (FK::prod) {
+    typename KR::Q xa, xb;
+    xa.load(u.kq + rA * (kSketch / 8), t);
+    xb.load(u.kq + rB * (kSketch / 8), t);
     static_for<8>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      T.kqA.template decode<s>(lut_a, lane4, lane8, one2, la, ha);
-      T.kqB.template decode<s>(lut_a, lane4, lane8, one2, lb, hb);
+      xa.template decode<s>(lut_a, lane4, lane8, one2, la, ha);
+      xb.template decode<s>(lut_a, lane4, lane8, one2, lb, hb);
 #pragma unroll
-      for (int x = 0; x < NX; ++x) mma16816(cq[(NX * s + x) & 3], la, lb, ha, hb, bqs[s][0][x], bqs[s][1][x]);
+      for (int x = 0; x < NX; ++x) mma16816(cq[(NX * s + x) & 1], la, lb, ha, hb, bqs[s][0][x], bqs[s][1][x]);
     });
+    gA = kQjlScale * ldsf(u.kres, rA * 4);
+    gB = kQjlScale * ldsf(u.kres, rB * 4);
   }
   float sc[4], sq[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    sc[j] = (ca[0][j] + ca[1][j]) + (ca[2][j] + ca[3][j]);
-    sq[j] = (cq[0][j] + cq[1][j]) + (cq[2][j] + cq[3][j]);
+    sc[j] = ca[0][j] + ca[1][j];
+    sq[j] = cq[0][j] + cq[1][j];
   }
   if constexpr (PACK) {
     // columns c and c+4 hold the hi and lo halves of one head: add them
@@ -682,14 +681,105 @@ __device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF
       if constexpr (FK::prod) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], 2);
     }
   }
-  // s (base 2): c0,c1 = token g, columns 2t, 2t+1; c2,c3 = token g+8
-  const float gkA = FK::prod ? T.gkA : 0.f, gkB = FK::prod ? T.gkB : 0.f;
-  float s2[4];
-  s2[0] = okA ? T.nkA * (sc[0] + kQjlScale * gkA * sq[0]) : -INFINITY;
-  s2[1] = okA ? T.nkA * (sc[1] + kQjlScale * gkA * sq[1]) : -INFINITY;
-  s2[2] = okB ? T.nkB * (sc[2] + kQjlScale * gkB * sq[2]) : -INFINITY;
-  s2[3] = okB ? T.nkB * (sc[3] + kQjlScale * gkB * sq[3]) : -INFINITY;
-  float mx0 = fmaxf(s2[0], s2[2]), mx1 = fmaxf(s2[1], s2[3]);
+  const float nA = ldsf(u.knorm, rA * 4), nB = ldsf(u.knorm, rB * 4);
+  if constexpr (FK::prod) {
+    s2[0] = nA * fmaf(gA, sq[0], sc[0]);
+    s2[1] = nA * fmaf(gA, sq[1], sc[1]);
+    s2[2] = nB * fmaf(gB, sq[2], sc[2]);
+    s2[3] = nB * fmaf(gB, sq[3], sc[3]);
+  } else {
+    s2[0] = nA * sc[0];
+    s2[1] = nA * sc[1];
+    s2[2] = nB * sc[2];
+    s2[3] = nB * sc[3];
+  }
+  if (!okA) s2[0] = s2[1] = -INFINITY;
+  if (!okB) s2[2] = s2[3] = -INFINITY;
+}
+
+// O^T += C_v^T P'^T for one 16-token subtile (rows from `srow`); p holds the
+// softmax weights of tokens g (p[0], p[1]) and g+8 (p[2], p[3]).
+template <int VF, int VMT>
+__device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, bool okA, bool okB, int g, int t,
+                                           const float (&p)[4], uint32_t lut_a,
+                                           uint32_t lut_b, uint32_t lane4, uint32_t lane8, uint32_t c1v,
+                                           float (&oacc)[VMT][4]) {
+  using FV = Fmt<VF>;
+  using VR = VRow<VF>;
+  const uint32_t one2 = 0x3C003C00u;
+  const float wA = okA ? ldsf(u.vnorm, (srow + g) * 4) : 0.f, wB = okB ? ldsf(u.vnorm, (srow + g + 8) * 4) : 0.f;
+  const uint32_t pb0 = movmatrix_t(h2bits(p[0] * wA, p[1] * wA));
+  const uint32_t pb1 = movmatrix_t(h2bits(p[2] * wB, p[3] * wB));
+  const int v0 = srow + 2 * t;  // tokens v0, v0+1, v0+8, v0+9
+  const uint32_t r0p = u.vcodes + v0 * FV::code_bytes;
+  const uint32_t r1p = r0p + FV::code_bytes;
+  const uint32_t r8p = r0p + 8 * FV::code_bytes;
+  const uint32_t r9p = r0p + 9 * FV::code_bytes;
+  if constexpr (FV::nseg > 0) {
+    constexpr int MT = VR::S0::MT;
+    typename VR::S0 xa, xb, xc, xd;
+    xa.load(r0p, g);
+    xb.load(r1p, g);
+    xc.load(r8p, g);
+    xd.load(r9p, g);
+    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
+    const uint32_t lut = FV::b0 == 2 ? lut_b : lut_a;
+    VR::S0::decode(xa, xb, lut, lane4, lane8, c1v, r0, r08);
+    VR::S0::decode(xc, xd, lut, lane4, lane8, c1v, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mma16816(oacc[mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
+  }
+  if constexpr (FV::nseg > 1) {
+    constexpr int MT = VR::S1::MT;
+    typename VR::S1 xa, xb, xc, xd;
+    xa.load(r0p, g);
+    xb.load(r1p, g);
+    xc.load(r8p, g);
+    xd.load(r9p, g);
+    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
+    VR::S1::decode(xa, xb, lut_a, lane4, lane8, c1v, r0, r08);
+    VR::S1::decode(xc, xd, lut_a, lane4, lane8, c1v, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mma16816(oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
+  }
+  if constexpr (FV::prod) {
+    const float uA = okA ? wA * ldsf(u.vres, (srow + g) * 4) : 0.f, uB = okB ? wB * ldsf(u.vres, (srow + g + 8) * 4) : 0.f;
+    const uint32_t qb0 = movmatrix_t(h2bits(p[0] * uA, p[1] * uA));
+    const uint32_t qb1 = movmatrix_t(h2bits(p[2] * uB, p[3] * uB));
+    typename VR::Q xa, xb, xc, xd;
+    xa.load(u.vq + v0 * (kSketch / 8), g);
+    xb.load(u.vq + (v0 + 1) * (kSketch / 8), g);
+    xc.load(u.vq + (v0 + 8) * (kSketch / 8), g);
+    xd.load(u.vq + (v0 + 9) * (kSketch / 8), g);
+    uint32_t r0[8], r08[8], r1[8], r18[8];
+    VR::Q::decode(xa, xb, lut_a, lane4, lane8, one2, r0, r08);
+    VR::Q::decode(xc, xd, lut_a, lane4, lane8, one2, r1, r18);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) mma16816(oacc[8 + mt], r0[mt], r08[mt], r1[mt], r18[mt], qb0, qb1);
+  }
+}
+
+// One warp tile of 32 tokens (two 16-token subtiles) starting at stage row
+// `srow`, unit-relative row `row0`; tokens at or past `nq` are masked.
+template <int KF, int VF, bool PACK, int WT>
+__device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int row0, int nq,
+                                             WarpState<KF, VF, PACK>& W, const QFrag<PACK>& bq,
+                                             const QFrag<PACK>& bqs, int g, int t, uint32_t lut_a,
+                                             uint32_t lut_b, uint32_t lane4, uint32_t lane8,
+                                             uint32_t c1k, uint32_t c1v, float thr) {
+  constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
+  const bool second = WT == 2 * kTok && row0 + kTok < nq;  // warp-uniform: the second subtile holds tokens
+  const bool ok0A = row0 + g < nq, ok0B = row0 + g + 8 < nq;
+  const bool ok1A = row0 + kTok + g < nq, ok1B = row0 + kTok + g + 8 < nq;
+  float s0[4], s1[4];
+  subtile_scores<KF, PACK>(u, srow, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
+  if (second)
+    subtile_scores<KF, PACK>(u, srow + kTok, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
+  else
+    s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
+  // online softmax over the 32 tokens (base 2), columns 2t and 2t+1
+  float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
+  float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -697,19 +787,23 @@ __device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF
   }
   const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
   const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
-  float p[4];
-  p[0] = fast_exp2(s2[0] - mn0);
-  p[1] = fast_exp2(s2[1] - mn1);
-  p[2] = fast_exp2(s2[2] - mn0);
-  p[3] = fast_exp2(s2[3] - mn1);
-  float rs0 = p[0] + p[2], rs1 = p[1] + p[3];
+  float p0[4], p1[4];
+  p0[0] = fast_exp2(s0[0] - mn0);
+  p0[1] = fast_exp2(s0[1] - mn1);
+  p0[2] = fast_exp2(s0[2] - mn0);
+  p0[3] = fast_exp2(s0[3] - mn1);
+  p1[0] = fast_exp2(s1[0] - mn0);
+  p1[1] = fast_exp2(s1[1] - mn1);
+  p1[2] = fast_exp2(s1[2] - mn0);
+  p1[3] = fast_exp2(s1[3] - mn1);
+  float rs0 = (p0[0] + p0[2]) + (p1[0] + p1[2]), rs1 = (p0[1] + p0[3]) + (p1[1] + p1[3]);
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
     rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
   }
-  W.l0 = W.l0 * al0 + rs0;
-  W.l1 = W.l1 * al1 + rs1;
+  W.l0 = fmaf(W.l0, al0, rs0);
+  W.l1 = fmaf(W.l1, al1, rs1);
   W.m0 = mn0;
   W.m1 = mn1;
   if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
@@ -721,55 +815,23 @@ __device__ __forceinline__ void compute_tile(const Tile<KF, VF>& T, WarpState<KF
       W.oacc[i][3] *= al1;
     }
   }
-  // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
+  bool keep0 = true, keep1 = second;
   if (thr > 0.f) {
+    // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
     const float c0 = thr * W.l0, c1 = thr * W.l1;
-    p[0] = p[0] >= c0 ? p[0] : 0.f;
-    p[1] = p[1] >= c1 ? p[1] : 0.f;
-    p[2] = p[2] >= c0 ? p[2] : 0.f;
-    p[3] = p[3] >= c1 ? p[3] : 0.f;
-    const bool any = (p[0] + p[1] + p[2] + p[3]) > 0.f;
-    if (!__any_sync(0xffffffffu, any)) return;
-  }
-
-  // ---- P'^T fragments: P' = p * ||v|| (and * ||r_v|| for the sketch part)
-  const float wA = okA ? T.nvA : 0.f, wB = okB ? T.nvB : 0.f;
-  const uint32_t pb0 = movmatrix_t(h2bits(p[0] * wA, p[1] * wA));
-  const uint32_t pb1 = movmatrix_t(h2bits(p[2] * wB, p[3] * wB));
-  uint32_t qb0 = 0, qb1 = 0;
-  if constexpr (FV::prod) {
-    const float uA = okA ? wA * T.gvA : 0.f, uB = okB ? wB * T.gvB : 0.f;
-    qb0 = movmatrix_t(h2bits(p[0] * uA, p[1] * uA));
-    qb1 = movmatrix_t(h2bits(p[2] * uB, p[3] * uB));
-  }
-  // ---- O^T += C_v^T P'^T
-  if constexpr (FV::nseg > 0) {
-    constexpr int MT = VR::S0::MT;
-    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
-    const unsigned char* lut = FV::b0 == 2 ? lut_b : lut_a;
-    VR::S0::decode(T.v0[0], T.v0[1], lut, lane4, lane8, c1v, r0, r08);
-    VR::S0::decode(T.v0[2], T.v0[3], lut, lane4, lane8, c1v, r1, r18);
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) mma16816(W.oacc[mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
+    for (int i = 0; i < 4; i += 2) {
+      p0[i] = p0[i] >= c0 ? p0[i] : 0.f;
+      p0[i + 1] = p0[i + 1] >= c1 ? p0[i + 1] : 0.f;
+      p1[i] = p1[i] >= c0 ? p1[i] : 0.f;
+      p1[i + 1] = p1[i + 1] >= c1 ? p1[i + 1] : 0.f;
+    }
+    keep0 = __any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f);
+    keep1 = second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f);
   }
-  if constexpr (FV::nseg > 1) {
-    constexpr int MT = VR::S1::MT;
-    uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
-    VR::S1::decode(T.v1[0], T.v1[1], lut_a, lane4, lane8, c1v, r0, r08);
-    VR::S1::decode(T.v1[2], T.v1[3], lut_a, lane4, lane8, c1v, r1, r18);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-      mma16816(W.oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
-  }
-  if constexpr (FV::prod) {
-    uint32_t r0[8], r08[8], r1[8], r18[8];
-    VR::Q::decode(T.vq[0], T.vq[1], lut_a, lane4, lane8, one2, r0, r08);
-    VR::Q::decode(T.vq[2], T.vq[3], lut_a, lane4, lane8, one2, r1, r18);
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) mma16816(W.oacc[8 + mt], r0[mt], r08[mt], r1[mt], r18[mt], qb0, qb1);
-  }
+  if (keep0) subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+  if (keep1) subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
 }
-
 
 // ---------------------------------------------------------------------------
 // 2. persistent decode kernel
@@ -791,7 +853,7 @@ struct UnitInfo {
   int len, ns, nq, chunks;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u) {
+__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u, int kChunk) {
   const int b = u / a.hkv;
   const int len = min(max(a.lens[b], 0), a.max_len);
   UnitInfo r;
@@ -803,6 +865,20 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u) {
 }
 
 __device__ __forceinline__ int64_t range_start(int i, int64_t C, int P) { return static_cast<int64_t>(i) * C / P; }
+
+// Chunks of each kv-head unit of sequence b (all units of a sequence are alike).
+__device__ __forceinline__ int seq_chunks(const DecodeArgs& a, int b, int kChunk) {
+  const int len = min(max(a.lens[b], 0), a.max_len);
+  return (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
+}
+
+// First global chunk index of unit u.
+__device__ __forceinline__ int64_t unit_first_chunk(const DecodeArgs& a, int u, int kChunk) {
+  const int b = u / a.hkv, h = u % a.hkv;
+  int64_t before = 0;
+  for (int v = 0; v < b; ++v) before += seq_chunks(a, v, kChunk);
+  return before * a.hkv + static_cast<int64_t>(h) * seq_chunks(a, b, kChunk);
+}
 
 // CTA whose range holds chunk c: the largest i with i*C/P <= c.
 __device__ __forceinline__ int cta_of_chunk(int64_t c, int64_t C, int P) {
@@ -864,6 +940,7 @@ __device__ void merge_unit(const DecodeArgs& a, int u, int first, int last, bool
   }
   consumers_sync();
   const int width = VPROD ? 2 * kDim : kDim;
+  for (int i = tid + G * 2 * kDim; i < kMaxG * 2 * kDim; i += NT) acc[i] = 0.f;
   for (int i = tid; i < G * width; i += NT) {
     const int h = i / width, j = i % width;
     float s = 0.f;
@@ -880,17 +957,35 @@ __device__ void merge_unit(const DecodeArgs& a, int u, int first, int last, bool
     osk[h * kDim + j] = has_sink ? __ldcg(sink + h * PF + 2 + j) * exp2f(__ldcg(sink + h * PF) - mm[h]) : 0.f;
   }
   consumers_sync();
+  // un-rotate: thread o < 128 forms (Pi^T A_h)_o for every head, threads
+  // 128..255 form (S^T B_h)_o (prod values); Pi and S rows are read once,
+  // coalesced, eight in flight
+  float* outr = ll + kMaxG;            // [kMaxG][kDim]
+  float* outs = outr + kMaxG * kDim;   // [kMaxG][kDim]
+  if (tid < (VPROD ? 2 : 1) * kDim) {
+    const bool sk = tid >= kDim;
+    const int o = tid & (kDim - 1);
+    const float* mat = sk ? a.s : a.pi;
+    const float* src = acc + (sk ? kDim : 0);
+    float r[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) r[h] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < kDim; ++j) {
+      const float mj = __ldg(mat + j * kDim + o);
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) r[h] = fmaf(mj, src[h * 2 * kDim + j], r[h]);
+    }
+    float* dst = sk ? outs : outr;
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) dst[h * kDim + o] = r[h];
+  }
+  consumers_sync();
   const int b = u / a.hkv, kvh = u % a.hkv;
   for (int i = tid; i < G * kDim; i += NT) {
     const int h = i / kDim, o = i % kDim;
-    float r = 0.f;
-    const float* ah = acc + h * 2 * kDim;
-    for (int j = 0; j < kDim; ++j) r = fmaf(a.pi[j * kDim + o], ah[j], r);
-    if (VPROD) {
-      float z = 0.f;
-      for (int l = 0; l < kSketch; ++l) z = fmaf(a.s[l * kDim + o], ah[kDim + l], z);
-      r = fmaf(kQjlScale, z, r);
-    }
+    float r = outr[h * kDim + o];
+    if (VPROD) r = fmaf(kQjlScale, outs[h * kDim + o], r);
     const float L = ll[h];
     store_out(a, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + o, L > 0.f ? (r + osk[h * kDim + o]) / L : 0.f);
   }
@@ -1052,12 +1147,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
   using L = Lut<KF, VF>;
-  using SL = StageLayout<KF, VF>;
-  constexpr int S = decode_stages<KF, VF>();
+  using CF = DecodeCfg<KF, VF>;
+  constexpr int CH = CF::CH, WT = CF::WT, S = CF::S;
+  using SL = StageLayout<KF, VF, CH>;
   constexpr int NX = PACK ? 1 : 2;
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* stages = smem + L::bytes;
-  float* scratch = reinterpret_cast<float*>(smem + L::bytes + S * SL::bytes);
+  // Shared-memory layout (shared-window addresses): stages below kLutAddr
+  // while they fit, the tables at kLutAddr, then the other stages and the
+  // scratch area.  Checked against the allocation before anything runs.
+  const uint32_t dyn0 = smem_u32(smem);
+  uint32_t low0 = (dyn0 + 127u) & ~127u, n_low = 0;
+  while (n_low < S && low0 + (n_low + 1) * SL::bytes <= kLutAddr) ++n_low;
+  const uint32_t high0 = kLutAddr + L::bytes;
+  uint32_t end = high0 + (S - n_low) * SL::bytes, scratch_addr;
+  const uint32_t scr_bytes = scratch_bytes(a.n_sink);
+  if (low0 + n_low * SL::bytes + scr_bytes <= kLutAddr) {
+    scratch_addr = low0 + n_low * SL::bytes;
+  } else {
+    scratch_addr = end;
+    end += scr_bytes;
+  }
+  if (dyn0 > kLutAddr || end > dyn0 + a.dyn_bytes) {
+    if (threadIdx.x == 0) atomicOr(a.status, 8);
+    return;
+  }
+  auto stage_addr = [&](int s) -> uint32_t {
+    return s < static_cast<int>(n_low) ? low0 + s * SL::bytes : high0 + (s - n_low) * SL::bytes;
+  };
+  float* scratch = reinterpret_cast<float*>(smem + (scratch_addr - dyn0));
+  unsigned char* lut_mem = smem + (kLutAddr - dyn0);
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ long long s_C, s_c0, s_c1;
@@ -1073,13 +1191,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     if constexpr (L::t4) {
       for (int i = tid; i < 256 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(smem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
       }
     }
     if constexpr (L::t3) {
       for (int i = tid; i < 64 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(smem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (r & 7)], cb[3 * kBookSlots + (r >> 3)]);
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (r & 7)], cb[3 * kBookSlots + (r >> 3)]);
       }
     }
     if constexpr (L::t2) {
@@ -1088,35 +1206,63 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
         uint2 v;
         v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
         v.y = h2bits(cb[2 * kBookSlots + ((r >> 4) & 3)], cb[2 * kBookSlots + (r >> 6)]);
-        *reinterpret_cast<uint2*>(smem + L::region_b_off + r * 256 + ln * 8) = v;
+        *reinterpret_cast<uint2*>(lut_mem + L::region_b_off + r * 256 + ln * 8) = v;
       }
     }
   }
-  if (tid == 0) {
+  if (warp == 0) {
+    // schedule (one warp): total chunks C, this CTA's range [c0, c1) and the
+    // unit / local chunk where it starts
     long long C = 0;
-    for (int u = 0; u < U; ++u) C += unit_info(a, u).chunks;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      int ch = b0 + lane < a.B ? seq_chunks(a, b0 + lane, CH) : 0;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, off);
+      C += ch;
+    }
+    C *= a.hkv;
     const long long c0 = range_start(cta, C, P), c1 = range_start(cta + 1, C, P);
     int u0 = U, lc0 = 0;
-    long long acc = 0;
-    for (int u = 0; u < U && c0 < c1; ++u) {
-      const int ch = unit_info(a, u).chunks;
-      if (c0 < acc + ch) {
-        u0 = u;
-        lc0 = static_cast<int>(c0 - acc);
+    long long base = 0;
+    for (int b0 = 0; b0 < a.B && c0 < c1; b0 += 32) {
+      const int b = b0 + lane;
+      const long long ch = b < a.B ? seq_chunks(a, b, CH) : 0;
+      long long incl = ch;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const long long lo = base + (incl - ch) * a.hkv, hi = base + incl * a.hkv;
+      const unsigned hit = __ballot_sync(0xffffffffu, b < a.B && ch > 0 && c0 >= lo && c0 < hi);
+      if (hit) {
+        const int src = __ffs(hit) - 1;
+        if (lane == src) {
+          const long long off = c0 - lo;
+          const int h = static_cast<int>(off / ch);
+          u0 = b * a.hkv + h;
+          lc0 = static_cast<int>(off - h * ch);
+        }
+        u0 = __shfl_sync(0xffffffffu, u0, src);
+        lc0 = __shfl_sync(0xffffffffu, lc0, src);
         break;
       }
-      acc += ch;
+      base += __shfl_sync(0xffffffffu, incl, 31) * a.hkv;
     }
-    s_C = C;
-    s_c0 = c0;
-    s_c1 = c1;
-    s_u0 = u0;
-    s_lc0 = lc0;
-    s_abort = 0;
-    s_flag = 0;
     if (cta == 0)
-      for (int b = 0; b < a.B; ++b)
+      for (int b = lane; b < a.B; b += 32)
         if (a.lens[b] > a.max_len) atomicOr(a.status, 2);
+    if (lane == 0) {
+      s_C = C;
+      s_c0 = c0;
+      s_c1 = c1;
+      s_u0 = u0;
+      s_lc0 = lc0;
+      s_abort = 0;
+      s_flag = 0;
+    }
+  }
+  if (tid == 32) {
 #pragma unroll
     for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
@@ -1131,35 +1277,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     // ---- producer: one lane streams the CTA's chunks through the stages
     if (lane == 0 && c0 < c1) {
       int u = s_u0, lc = s_lc0;
-      UnitInfo ui = unit_info(a, u);
+      UnitInfo ui = unit_info(a, u, CH);
       long long k = 0;
       for (long long c = c0; c < c1; ++c, ++k) {
         while (lc >= ui.chunks) {
           ++u;
           lc = 0;
-          ui = unit_info(a, u);
+          ui = unit_info(a, u, CH);
         }
         const int s = static_cast<int>(k % S);
         if (k >= S && !mbar_wait(&empty_bar[s], static_cast<uint32_t>((k / S - 1) & 1))) s_abort = 1;
         if (s_abort) break;
         const int64_t ubase = static_cast<int64_t>(u) * a.capacity;
-        const int r0 = lc * kChunk;
-        const int rows = min(kChunk, (ui.nq + kTok - 1) / kTok * kTok - r0);  // <= capacity - r0
-        unsigned char* st = stages + s * SL::bytes;
+        const int r0 = lc * CH;
+        const int rows = min(CH, (ui.nq + kTok - 1) / kTok * kTok - r0);  // <= capacity - r0
+        const uint32_t st = stage_addr(s);
         uint64_t* bar = &full_bar[s];
         mbar_expect_tx(bar, SL::tx_bytes(rows));
         const int64_t row = ubase + r0;
-        if constexpr (FK::code_bytes > 0) bulk_g2s(st + SL::kc, a.k_codes + row * FK::code_bytes, rows * FK::code_bytes, bar);
-        if constexpr (FV::code_bytes > 0) bulk_g2s(st + SL::vc, a.v_codes + row * FV::code_bytes, rows * FV::code_bytes, bar);
-        bulk_g2s(st + SL::kn, a.k_norms + row, rows * 4, bar);
-        bulk_g2s(st + SL::vn, a.v_norms + row, rows * 4, bar);
+        if constexpr (FK::code_bytes > 0) bulk_g2s_addr(st + SL::kc, a.k_codes + row * FK::code_bytes, rows * FK::code_bytes, bar);
+        if constexpr (FV::code_bytes > 0) bulk_g2s_addr(st + SL::vc, a.v_codes + row * FV::code_bytes, rows * FV::code_bytes, bar);
+        bulk_g2s_addr(st + SL::kn, a.k_norms + row, rows * 4, bar);
+        bulk_g2s_addr(st + SL::vn, a.v_norms + row, rows * 4, bar);
         if constexpr (FK::prod) {
-          bulk_g2s(st + SL::kq, a.k_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
-          bulk_g2s(st + SL::kr, a.k_res + row, rows * 4, bar);
+          bulk_g2s_addr(st + SL::kq, a.k_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
+          bulk_g2s_addr(st + SL::kr, a.k_res + row, rows * 4, bar);
         }
         if constexpr (FV::prod) {
-          bulk_g2s(st + SL::vq, a.v_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
-          bulk_g2s(st + SL::vr, a.v_res + row, rows * 4, bar);
+          bulk_g2s_addr(st + SL::vq, a.v_qjl + row * (kSketch / 8), rows * (kSketch / 8), bar);
+          bulk_g2s_addr(st + SL::vr, a.v_res + row, rows * 4, bar);
         }
         ++lc;
       }
@@ -1168,16 +1314,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   }
 
   // ---- consumers
-  const unsigned char* lut_a = smem;
-  const unsigned char* lut_b = smem + L::region_b_off;
-  const uint32_t lane4 = lane * 4, lane8 = lane * 8;
+  // table bases are folded into the lane offsets (see kLutAddr)
+  const uint32_t lut_a = 0, lut_b = 0;
+  const uint32_t lane4 = kLutAddr | (lane * 4), lane8 = (kLutAddr + L::region_b_off) | (lane * 8);
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const float thr = a.sparse_thr;
 
   // sink pieces and empty sequences of the units u = cta (mod P)
   for (int u = cta; u < U; u += P) {
-    const UnitInfo ui = unit_info(a, u);
+    const UnitInfo ui = unit_info(a, u, CH);
     if (ui.len == 0) {
       const int b = u / a.hkv, kvh = u % a.hkv;
       for (int i = tid; i < a.group * kDim; i += kConsumers * 32)
@@ -1188,8 +1334,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     sink_piece(a, u, ui.ns, scratch);
     int first = 1, last = 0;
     if (ui.chunks > 0) {
-      long long cu0 = 0;
-      for (int v = 0; v < u; ++v) cu0 += unit_info(a, v).chunks;
+      const long long cu0 = unit_first_chunk(a, u, CH);
       first = cta_of_chunk(cu0, C, P);
       last = cta_of_chunk(cu0 + ui.chunks - 1, C, P);
     }
@@ -1197,12 +1342,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   }
 
   WarpState<KF, VF, PACK> wst;
-  uint32_t bq[8][2][NX], bqs[8][2][NX];
+  QFrag<PACK> bq, bqs;
+  constexpr int kMaxPending = 32;
+  __shared__ int s_pend[kMaxPending][4];
+  int n_pend = 0;  // same value in every consumer thread
   int u = -1;
   UnitInfo ui{};
   long long cu0 = 0;
   int walk_u = s_u0, walk_lc = s_lc0;
-  UnitInfo wui = c0 < c1 ? unit_info(a, walk_u) : UnitInfo{};
+  UnitInfo wui = c0 < c1 ? unit_info(a, walk_u, CH) : UnitInfo{};
   long long walk_cu0 = c0 - s_lc0;
   long long k = 0;
   for (long long c = c0; c < c1; ++c, ++k) {
@@ -1210,13 +1358,25 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       walk_cu0 += wui.chunks;
       ++walk_u;
       walk_lc = 0;
-      wui = unit_info(a, walk_u);
+      wui = unit_info(a, walk_u, CH);
     }
     if (walk_u != u) {
       if (u >= 0) {
+        // publish the partial now; count it (and merge, if it completes the
+        // unit) after the range, so no merge stalls the stream
         write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
-        publish_piece<VF>(a, u, cta_of_chunk(cu0, C, P), cta_of_chunk(cu0 + ui.chunks - 1, C, P), ui.ns > 0,
-                          scratch, &s_flag, &s_abort, C);
+        const int first = cta_of_chunk(cu0, C, P), last = cta_of_chunk(cu0 + ui.chunks - 1, C, P);
+        if (n_pend < kMaxPending) {
+          if (tid == 0) {
+            s_pend[n_pend][0] = u;
+            s_pend[n_pend][1] = first;
+            s_pend[n_pend][2] = last;
+            s_pend[n_pend][3] = ui.ns > 0;
+          }
+          ++n_pend;
+        } else {
+          publish_piece<VF>(a, u, first, last, ui.ns > 0, scratch, &s_flag, &s_abort, C);
+        }
       }
       u = walk_u;
       ui = wui;
@@ -1238,21 +1398,20 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     }
     const int s = static_cast<int>(k % S);
     if (!s_abort && !mbar_wait(&full_bar[s], static_cast<uint32_t>((k / S) & 1))) s_abort = 1;
-    const int row0 = walk_lc * kChunk + warp * kTok;
+    const int row0 = walk_lc * CH + warp * WT;
     if (!s_abort && row0 < ui.nq) {
-      const unsigned char* st = stages + s * SL::bytes;
+      const uint32_t st = stage_addr(s);
       UnitPlanes sp;
       sp.kcodes = st + SL::kc;
       sp.vcodes = st + SL::vc;
-      sp.knorm = reinterpret_cast<const float*>(st + SL::kn);
-      sp.vnorm = reinterpret_cast<const float*>(st + SL::vn);
+      sp.knorm = st + SL::kn;
+      sp.vnorm = st + SL::vn;
       sp.kq = st + SL::kq;
-      sp.kres = reinterpret_cast<const float*>(st + SL::kr);
+      sp.kres = st + SL::kr;
       sp.vq = st + SL::vq;
-      sp.vres = reinterpret_cast<const float*>(st + SL::vr);
-      Tile<KF, VF> tl;
-      load_tile(tl, sp, warp * kTok, g, t);
-      compute_tile<KF, VF, PACK>(tl, wst, bq, bqs, row0, ui.nq, g, lut_a, lut_b, lane4, lane8, c1k, c1v, thr);
+      sp.vres = st + SL::vr;
+      compute_tile<KF, VF, PACK, WT>(sp, warp * WT, row0, ui.nq, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
+                                 c1k, c1v, thr);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
@@ -1263,6 +1422,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     publish_piece<VF>(a, u, cta_of_chunk(cu0, C, P), cta_of_chunk(cu0 + ui.chunks - 1, C, P), ui.ns > 0, scratch,
                       &s_flag, &s_abort, C);
   }
+  consumers_sync();  // the pending list written by thread 0 is visible
+  for (int i = 0; i < n_pend; ++i)
+    publish_piece<VF>(a, s_pend[i][0], s_pend[i][1], s_pend[i][2], s_pend[i][3] != 0, scratch, &s_flag, &s_abort, C);
   if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
 
@@ -1281,8 +1443,8 @@ int num_sms_cached() {
 
 template <int KF, int VF>
 size_t decode_smem_bytes(int n_sink) {
-  return static_cast<size_t>(Lut<KF, VF>::bytes) + decode_stages<KF, VF>() * StageLayout<KF, VF>::bytes +
-         scratch_bytes(n_sink);
+  using CF = DecodeCfg<KF, VF>;
+  return static_cast<size_t>(plan_end(CF::stage, CF::S, CF::lut, scratch_bytes(n_sink)) - kDynBaseMax);
 }
 
 template <int KF, int VF, bool PACK>
@@ -1300,9 +1462,10 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
 
 template <int KF, int VF>
 tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
-  const size_t smem = decode_smem_bytes<KF, VF>(a.n_sink);
-  if (smem > static_cast<size_t>(kSmemBudget))
+  if (decode_smem_bytes<KF, VF>(a.n_sink) + kDynBaseMax > static_cast<size_t>(kSmemEnd))
     return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink too large for the shared-memory plan");
+  const size_t smem = kSmemBudget;  // the whole window: one CTA per SM
+  a.dyn_bytes = static_cast<uint32_t>(smem);
   a.pack = plan.group <= 4;
   return a.pack ? run_decode_v<KF, VF, true>(a, plan, smem, st) : run_decode_v<KF, VF, false>(a, plan, smem, st);
 }
