@@ -194,8 +194,9 @@ typedef struct {
  * Hq query heads and lengths up to max_len. */
 size_t tq_decode_workspace_bytes(const tq_params* p, int B, int hq, int n_kv_heads, int max_len);
 
-/* Zero the bookkeeping part of a fresh workspace (once per workspace; the
- * decode kernel leaves it zeroed after each call). */
+/* Zero-fill a workspace.  Optional: the decode kernels keep no state in the
+ * workspace between calls and read only what they wrote earlier in the same
+ * call. */
 tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* One decode step for sequences b = 0..B-1 of the cache: q [B][hq][d]
@@ -206,7 +207,11 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
  * rotated domain and Pi^T (and S^T) applied once per output.  Sink tokens use
  * their bf16 keys and values directly.  A sequence with no tokens gives a
  * zero output.  max_len: host bound on lens (longer sequences are cut to it
- * and bit 2 is set in cache->status). */
+ * and bit 2 is set in cache->status).  n_sink above 12288 gives
+ * TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the query rotation,
+ * the persistent decode kernel and the merge; the last two are launched with
+ * programmatic stream serialization and overlap their prologues with the
+ * previous kernel's tail. */
 tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
                          int B, int hq, int max_len, void* out, int out_dtype,
                          void* workspace, size_t ws_bytes, const tq_attn_flags* flags,

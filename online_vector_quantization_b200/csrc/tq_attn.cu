@@ -12,17 +12,19 @@
 // Kernels of one decode step
 //   1. qrot_kernel: q -> Pi q (and S q), scaled by log2(e)/sqrt(d), stored as
 //      fp16 MMA B-fragments in the workspace, once per (sequence, kv-head).
-//   2. decode_kernel: grid (split, kv-head, sequence) + one sink CTA per
-//      (sequence, kv-head).  Each warp walks 16-token tiles of its split:
+//   2. decode_kernel: persistent, one CTA per SM; a producer warp streams
+//      the packed cache into shared memory with bulk copies, fifteen consumer
+//      warps walk 16-token tiles of it:
 //        scores S^T[16 tok x 8 heads] = C_k[16 x 128] Q~^T  (mma.sync m16n8k16)
 //        online softmax (base 2), sparse-V mask, P' = p * ||v||
 //        O^T[128 x 8 heads] += C_v^T[128 x 16 tok] P'^T    (mma.sync m16n8k16)
 //      The dequantized codebook values for both MMAs come straight from
 //      per-lane-replicated shared-memory tables indexed by packed code bytes
 //      (two or four codes per lookup, no bank conflicts), so no fp16 tile is
-//      ever written back to memory.  Warps merge in shared memory, the CTA
-//      writes (m, l, acc) partials, and the last CTA of a (sequence, kv-head)
-//      (atomic ticket, no spin-waits) merges the splits and applies Pi^T/S^T.
+//      ever written back to memory.  Warps merge in shared memory and the CTA
+//      writes one (m, l, acc) partial per piece of a (sequence, kv-head).
+//   3. merge_kernel: one CTA per (sequence, query head) attends the bf16 sink,
+//      combines the pieces and applies Pi^T / S^T once.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -416,8 +418,9 @@ struct DecodeArgs {
   const int32_t* lens;
   int32_t* status;
   int B, hkv, group, hq, capacity, n_sink, max_len, part_floats;
+  int ctas;   // CTAs of the decode grid (pieces a unit can be cut into)
+  int chunk;  // quantized tokens per scheduled chunk
   float* parts;
-  int32_t* tickets;
   const uint32_t* qfrag;
   void* out;
   int out_bf16;
@@ -436,6 +439,15 @@ __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]) : reinterpret_cast<const float*>(q)[i];
 }
 
+// Programmatic dependent launch.  The three kernels of one decode call run
+// back to back on one stream; the second and third are launched with
+// programmatic stream serialization, so they may start while the previous one
+// still runs.  pdl_launch lets the next kernel be scheduled; pdl_wait blocks
+// the calling thread until the previous kernel has finished and its writes
+// are visible (a no-op in a kernel launched without the attribute).
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // 1. query rotation: one CTA per (sequence, kv-head).  Threads 0..127 form
 //    Pi q for all heads (one output coordinate each), threads 128..255 form
@@ -450,6 +462,7 @@ __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
   __shared__ float qsk[kMaxG][kSketch];
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = a.group;
+  pdl_launch();  // the decode kernel's prologue and cache stream may start
   for (int i = tid; i < kMaxG * kDim; i += kThreads) {
     const int h = i / kDim, d = i % kDim;
     qs[h][d] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
@@ -559,12 +572,9 @@ struct StageLayout {
 // merge, sink scores).  Stages go below kLutAddr while they fit, the rest
 // above the tables.
 constexpr int kSliceDims = 64;
-__host__ __device__ constexpr int scratch_bytes(int n_sink) {
-  const int combine = (kConsumers * kMaxG * kSliceDims + 2 * kConsumers * kMaxG) * 4;
-  const int merge = (kMaxG * 5 * kDim + 2 * kMaxG) * 4;
-  const int sink = (kMaxG * kDim + kMaxG * n_sink + 2 * kMaxG) * 4;
-  return combine > merge ? (combine > sink ? combine : sink) : (merge > sink ? merge : sink);
-}
+// Cross-warp combine area of write_piece: per warp and head the running max,
+// the sum and one slice of the accumulator.
+constexpr int kScratchBytes = (kConsumers * kMaxG * kSliceDims + 2 * kConsumers * kMaxG) * 4;
 constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic bytes requested per block
 constexpr int kDynBaseMax = 4096;                // assumed upper bound of the dynamic base address
 constexpr int kSmemEnd = 227 * 1024;             // assumed end of the usable shared window
@@ -584,7 +594,7 @@ __host__ __device__ constexpr int plan_end(int stage, int n_stages, int lut, int
 template <int KF, int VF>
 struct DecodeCfg {
   static constexpr int lut = Lut<KF, VF>::bytes;
-  static constexpr int scr = scratch_bytes(128);
+  static constexpr int scr = kScratchBytes;
   static constexpr int s32 = StageLayout<KF, VF, 32 * kConsumers>::bytes;
   static constexpr int s16 = StageLayout<KF, VF, 16 * kConsumers>::bytes;
   static constexpr bool fit32 = plan_end(s32, 2, lut, scr) <= kSmemEnd;
@@ -843,11 +853,10 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
 // tokens form ceil(nq / kChunk) chunks; the chunks of all units, in unit
 // order, make one list of C chunks cut into gridDim.x equal contiguous ranges,
 // one per CTA, so every CTA streams the same number of bytes.  A unit may span
-// several CTAs (its pieces).  Piece (u, cta) publishes partial slot u + cta:
+// several CTAs (its pieces).  Piece (u, cta) writes partial slot u + cta:
 // both indices only grow along the list, so slots are distinct and there are
-// at most U + P - 1 of them.  The bf16 sink of unit u is one more piece
-// (slot U + P + u), done by CTA u mod P.  The CTA that completes a unit's set
-// of pieces (atomic ticket, no spin-wait) merges them and applies Pi^T / S^T.
+// at most U + P - 1 of them.  The merge kernel finds a unit's pieces from the
+// same schedule.  No CTA waits for another.
 // ---------------------------------------------------------------------------
 struct UnitInfo {
   int len, ns, nq, chunks;
@@ -872,14 +881,6 @@ __device__ __forceinline__ int seq_chunks(const DecodeArgs& a, int b, int kChunk
   return (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
 }
 
-// First global chunk index of unit u.
-__device__ __forceinline__ int64_t unit_first_chunk(const DecodeArgs& a, int u, int kChunk) {
-  const int b = u / a.hkv, h = u % a.hkv;
-  int64_t before = 0;
-  for (int v = 0; v < b; ++v) before += seq_chunks(a, v, kChunk);
-  return before * a.hkv + static_cast<int64_t>(h) * seq_chunks(a, b, kChunk);
-}
-
 // CTA whose range holds chunk c: the largest i with i*C/P <= c.
 __device__ __forceinline__ int cta_of_chunk(int64_t c, int64_t C, int P) {
   return static_cast<int>(((c + 1) * P - 1) / C);
@@ -898,8 +899,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Partial slot: per head of the unit's group, [max, sum, accumulator].
 __device__ __forceinline__ float* part_slot(const DecodeArgs& a, int64_t slot) {
-  return a.parts + slot * kMaxG * a.part_floats;
+  return a.parts + slot * a.group * a.part_floats;
 }
 
 __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t i, float v) {
@@ -907,112 +909,6 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t i, float 
     reinterpret_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(v);
   else
     reinterpret_cast<float*>(a.out)[i] = v;
-}
-
-// Merge the pieces of unit u (consumer threads): main slots u + i for
-// i in [first, last] (none when first > last) and the sink slot.
-template <int VF>
-__device__ void merge_unit(const DecodeArgs& a, int u, int first, int last, bool has_sink, float* sm, int64_t C) {
-  constexpr bool VPROD = Fmt<VF>::prod;
-  constexpr int NT = kConsumers * 32;
-  const int tid = threadIdx.x, G = a.group;
-  const int PF = a.part_floats;
-  const int U = a.B * a.hkv, P = gridDim.x;
-  const float* sink = part_slot(a, U + P + u);
-  float* acc = sm;                     // [kMaxG][2*kDim] rotated | sketch
-  float* osk = sm + kMaxG * 2 * kDim;  // [kMaxG][kDim] sink, original domain
-  float* mm = osk + kMaxG * kDim;      // [kMaxG]: M
-  float* ll = mm + kMaxG;              // [kMaxG]: L
-  if (tid < kMaxG) {
-    float M = -INFINITY;
-    for (int i = first; i <= last; ++i)
-      if (cta_has_chunks(i, C, P)) M = fmaxf(M, __ldcg(part_slot(a, u + i) + tid * PF));
-    if (has_sink) M = fmaxf(M, __ldcg(sink + tid * PF));
-    float L = 0.f;
-    for (int i = first; i <= last; ++i) {
-      if (!cta_has_chunks(i, C, P)) continue;
-      const float* pp = part_slot(a, u + i) + tid * PF;
-      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - M);
-    }
-    if (has_sink) L += __ldcg(sink + tid * PF + 1) * exp2f(__ldcg(sink + tid * PF) - M);
-    mm[tid] = M;
-    ll[tid] = L;
-  }
-  consumers_sync();
-  const int width = VPROD ? 2 * kDim : kDim;
-  for (int i = tid + G * 2 * kDim; i < kMaxG * 2 * kDim; i += NT) acc[i] = 0.f;
-  for (int i = tid; i < G * width; i += NT) {
-    const int h = i / width, j = i % width;
-    float s = 0.f;
-    for (int k = first; k <= last; ++k) {
-      if (!cta_has_chunks(k, C, P)) continue;
-      const float* pp = part_slot(a, u + k) + h * PF;
-      s += __ldcg(pp + 2 + j) * exp2f(__ldcg(pp) - mm[h]);
-    }
-    if (j < kDim) s = Fmt<VF>::width(j) > 0 ? s / a.sig[Fmt<VF>::width(j)] : 0.f;
-    acc[h * 2 * kDim + j] = s;
-  }
-  for (int i = tid; i < G * kDim; i += NT) {
-    const int h = i / kDim, j = i % kDim;
-    osk[h * kDim + j] = has_sink ? __ldcg(sink + h * PF + 2 + j) * exp2f(__ldcg(sink + h * PF) - mm[h]) : 0.f;
-  }
-  consumers_sync();
-  // un-rotate: thread o < 128 forms (Pi^T A_h)_o for every head, threads
-  // 128..255 form (S^T B_h)_o (prod values); Pi and S rows are read once,
-  // coalesced, eight in flight
-  float* outr = ll + kMaxG;            // [kMaxG][kDim]
-  float* outs = outr + kMaxG * kDim;   // [kMaxG][kDim]
-  if (tid < (VPROD ? 2 : 1) * kDim) {
-    const bool sk = tid >= kDim;
-    const int o = tid & (kDim - 1);
-    const float* mat = sk ? a.s : a.pi;
-    const float* src = acc + (sk ? kDim : 0);
-    float r[kMaxG];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) r[h] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < kDim; ++j) {
-      const float mj = __ldg(mat + j * kDim + o);
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h) r[h] = fmaf(mj, src[h * 2 * kDim + j], r[h]);
-    }
-    float* dst = sk ? outs : outr;
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) dst[h * kDim + o] = r[h];
-  }
-  consumers_sync();
-  const int b = u / a.hkv, kvh = u % a.hkv;
-  for (int i = tid; i < G * kDim; i += NT) {
-    const int h = i / kDim, o = i % kDim;
-    float r = outr[h * kDim + o];
-    if (VPROD) r = fmaf(kQjlScale, outs[h * kDim + o], r);
-    const float L = ll[h];
-    store_out(a, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + o, L > 0.f ? (r + osk[h * kDim + o]) / L : 0.f);
-  }
-}
-
-// Count this piece of unit u; the piece that completes the set merges.
-template <int VF>
-__device__ void publish_piece(const DecodeArgs& a, int u, int first, int last, bool has_sink, float* sm,
-                              volatile int* s_flag, volatile int* s_abort, int64_t C) {
-  __threadfence();
-  consumers_sync();
-  if (threadIdx.x == 0) {
-    int last_piece = 0;
-    if (!*s_abort) {
-      int expected = has_sink ? 1 : 0;
-      for (int i = first; i <= last; ++i) expected += cta_has_chunks(i, C, gridDim.x);
-      last_piece = atomicAdd(a.tickets + u, 1) == expected - 1;
-    }
-    *s_flag = last_piece;
-  }
-  consumers_sync();
-  if (*s_flag) {
-    __threadfence();
-    merge_unit<VF>(a, u, first, last, has_sink, sm, C);
-    if (threadIdx.x == 0) a.tickets[u] = 0;  // ready for the next call
-  }
-  consumers_sync();
 }
 
 // Cross-warp combine of one piece into partial slot `slot`, in 64-coordinate
@@ -1067,7 +963,7 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
       }
     }
     consumers_sync();
-    for (int i = tid; i < kMaxG * kSliceDims; i += NT) {
+    for (int i = tid; i < a.group * kSliceDims; i += NT) {
       const int h = i / kSliceDims, j = i % kSliceDims;
       float M = -INFINITY;
       for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
@@ -1090,55 +986,188 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
   }
 }
 
-// Sink piece of unit u: bf16 keys/values of tokens [0, ns) in the original
-// domain (consumer threads), into slot U + P + u.
-__device__ void sink_piece(const DecodeArgs& a, int u, int ns, float* sm) {
-  constexpr int NT = kConsumers * 32;
-  const int tid = threadIdx.x, G = a.group;
+// ---------------------------------------------------------------------------
+// 3. merge: one CTA per (unit, query head).  The unit's quantized tokens were
+//    streamed as pieces by consecutive CTAs of the decode grid; its bf16 sink
+//    tokens are attended here.  Partial results are combined by their maxima
+//    (the usual online-softmax merge), Pi^T (and S^T for prod values) is
+//    applied once, and the result is divided by the softmax sum.  Everything
+//    that does not read the pieces runs before pdl_wait, overlapping the tail
+//    of the decode kernel.
+// ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 512;
+constexpr int kMaxPieces = 1024;  // bound on the decode grid size
+constexpr int kMaxSink = 12288;   // sink scores live in 48 KB of shared memory
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();  // red may still be read by an earlier reduction
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = red[0];
+  for (int w = 1; w < kMergeThreads / 32; ++w) v = is_max ? fmaxf(v, red[w]) : v + red[w];
+  return v;
+}
+
+template <int VF>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
+  using FV = Fmt<VF>;
+  constexpr int NT = kMergeThreads;
+  constexpr int WD = FV::prod ? 2 * kDim : kDim;  // accumulator: rotated | sketch
+  constexpr int NS = NT / WD;                     // piece slices of the accumulation
+  constexpr int RS = WD / 4;                      // matrix rows per un-rotation slice
+  extern __shared__ float s_sc[];                 // [n_sink] sink scores, then weights
+  __shared__ float s_f[kMaxPieces];               // per piece: max, then weight
+  __shared__ float s_red[NT];
+  __shared__ float s_acc[WD];
+  __shared__ float s_osk[kDim];
+  __shared__ float s_q[kDim];
+  __shared__ float s_w[NT / 32];
+  __shared__ long long s_C, s_cu0;
+  const int u = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = a.group, P = a.ctas, CH = a.chunk, PF = a.part_floats;
   const int b = u / a.hkv, kvh = u % a.hkv;
-  const int U = a.B * a.hkv, P = gridDim.x;
-  float* qs = sm;                      // [8][128]
-  float* sc = qs + kMaxG * kDim;       // [8][n_sink]
-  float* red = sc + kMaxG * a.n_sink;  // [8][2]
-  float* dst = part_slot(a, U + P + u);
-  const int PF = a.part_floats;
-  for (int i = tid; i < kMaxG * kDim; i += NT) {
-    const int h = i / kDim, d = i % kDim;
-    qs[i] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
+  const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim;
+  const UnitInfo ui = unit_info(a, u, CH);
+  if (ui.len == 0) {
+    if (tid < kDim) store_out(a, orow + tid, 0.f);
+    return;
   }
-  consumers_sync();
-  const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
-  const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
-  const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
-  for (int i = tid; i < G * ns; i += NT) {
-    const int h = i / ns, tok = i % ns;
-    float acc = 0.f;
-    for (int d = 0; d < kDim; ++d) acc = fmaf(__bfloat162float(ks[tok * kDim + d]), qs[h * kDim + d], acc);
-    sc[h * a.n_sink + tok] = acc * scale;
-  }
-  consumers_sync();
-  if (tid < G) {
-    float m = -INFINITY;
-    for (int tok = 0; tok < ns; ++tok) m = fmaxf(m, sc[tid * a.n_sink + tok]);
-    float l = 0.f;
-    for (int tok = 0; tok < ns; ++tok) {
-      const float p = exp2f(sc[tid * a.n_sink + tok] - m);
-      sc[tid * a.n_sink + tok] = p;
-      l += p;
+  // where the unit's chunks sit in the decode schedule (warp 0)
+  if (warp == 0 && ui.chunks > 0) {
+    long long tot = 0, before = 0;
+    for (int v = lane; v < a.B; v += 32) {
+      const int ch = seq_chunks(a, v, CH);
+      tot += ch;
+      if (v < b) before += ch;
     }
-    red[2 * tid] = m;
-    red[2 * tid + 1] = l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, off);
+      before += __shfl_xor_sync(0xffffffffu, before, off);
+    }
+    if (lane == 0) {
+      s_C = tot * a.hkv;
+      s_cu0 = before * a.hkv + static_cast<long long>(kvh) * ui.chunks;
+    }
   }
-  consumers_sync();
-  for (int i = tid; i < G * kDim; i += NT) {
-    const int h = i / kDim, d = i % kDim;
-    float acc = 0.f;
-    for (int tok = 0; tok < ns; ++tok) acc = fmaf(sc[h * a.n_sink + tok], __bfloat162float(vs[tok * kDim + d]), acc);
-    dst[h * PF + 2 + d] = acc;
+  // sink: scores with the original query, softmax weights, weighted values
+  float ms = -INFINITY, ls = 0.f;
+  if (ui.ns > 0) {
+    if (tid < kDim) s_q[tid] = load_q(a.q, a.q_bf16, orow + tid);
+    __syncthreads();
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
+    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
+    const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
+    for (int t = warp; t < ui.ns; t += NT / 32) {
+      const __nv_bfloat16* kr = ks + static_cast<int64_t>(t) * kDim + 4 * lane;
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d = fmaf(__bfloat162float(kr[e]), s_q[4 * lane + e], d);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if (lane == 0) s_sc[t] = d * scale;
+    }
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int t = tid; t < ui.ns; t += NT) mx = fmaxf(mx, s_sc[t]);
+    ms = block_reduce(mx, true, s_w);
+    float sum = 0.f;
+    for (int t = tid; t < ui.ns; t += NT) {
+      const float p = exp2f(s_sc[t] - ms);
+      s_sc[t] = p;
+      sum += p;
+    }
+    ls = block_reduce(sum, false, s_w);  // its barriers also publish s_sc
+    {
+      const int j = tid & (kDim - 1), sl = tid >> 7;
+      float acc = 0.f;
+      for (int t = sl; t < ui.ns; t += NT / kDim) acc = fmaf(s_sc[t], __bfloat162float(vs[static_cast<int64_t>(t) * kDim + j]), acc);
+      s_red[sl * kDim + j] = acc;
+    }
+    __syncthreads();
+    if (tid < kDim) {
+      float v = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < NT / kDim; ++sl) v += s_red[sl * kDim + tid];
+      s_osk[tid] = v;
+    }
   }
-  if (tid < G) {
-    dst[tid * PF + 0] = red[2 * tid];
-    dst[tid * PF + 1] = red[2 * tid + 1];
+  __syncthreads();
+  // the pieces: written by the decode kernel
+  pdl_wait();
+  float M = ms, L = 0.f;
+  const bool has_pieces = ui.chunks > 0;
+  int first = 0, n_p = 0;
+  if (has_pieces) {
+    const long long C = s_C, cu0 = s_cu0;
+    first = cta_of_chunk(cu0, C, P);
+    n_p = cta_of_chunk(cu0 + ui.chunks - 1, C, P) - first + 1;
+    float mx = -INFINITY;
+    for (int i = tid; i < n_p; i += NT) {
+      const float m = cta_has_chunks(first + i, C, P) ? __ldcg(part_slot(a, u + first + i) + h * PF) : -INFINITY;
+      s_f[i] = m;
+      mx = fmaxf(mx, m);
+    }
+    M = fmaxf(M, block_reduce(mx, true, s_w));
+    float lsum = 0.f;
+    for (int i = tid; i < n_p; i += NT) {
+      const float m = s_f[i];
+      const float f = m > -INFINITY ? exp2f(m - M) : 0.f;
+      if (f != 0.f) lsum = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 1), f, lsum);
+      s_f[i] = f;
+    }
+    L = block_reduce(lsum, false, s_w);  // its barriers also publish s_f
+    {
+      const int j = tid % WD, sl = tid / WD;
+      float acc = 0.f;
+      for (int i = sl; i < n_p; i += NS) {
+        const float f = s_f[i];
+        if (f != 0.f) acc = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 2 + j), f, acc);
+      }
+      s_red[sl * WD + j] = acc;
+    }
+    __syncthreads();
+    for (int j = tid; j < WD; j += NT) {
+      float v = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < NS; ++sl) v += s_red[sl * WD + j];
+      if (j < kDim) v = FV::width(j) > 0 ? v / a.sig[FV::width(j)] : 0.f;
+      s_acc[j] = v;
+    }
+    __syncthreads();
+  }
+  const float fs = ui.ns > 0 ? exp2f(ms - M) : 0.f;
+  L = fmaf(ls, fs, L);
+  // un-rotation: out_o = sum_j Pi[j][o] A_j + sqrt(pi/2)/m sum_j S[j][o] B_j;
+  // thread (o, slice) sums RS consecutive rows j, rows read coalesced over o
+  {
+    const int o = tid & (kDim - 1), sl = tid >> 7;
+    float r = 0.f;
+    if (has_pieces) {
+      const int j0 = sl * RS;
+      const bool sk = FV::prod && j0 >= kDim;
+      const float* mat = sk ? a.s + (j0 - kDim) * kDim : a.pi + j0 * kDim;
+      const float* src = s_acc + j0;
+#pragma unroll 8
+      for (int jj = 0; jj < RS; ++jj) r = fmaf(__ldg(mat + jj * kDim + o), src[jj], r);
+      if (sk) r *= kQjlScale;
+    }
+    s_red[sl * kDim + o] = r;
+  }
+  __syncthreads();
+  if (tid < kDim) {
+    float v = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) v += s_red[sl * kDim + tid];
+    if (ui.ns > 0) v = fmaf(fs, s_osk[tid], v);
+    store_out(a, orow + tid, L > 0.f ? v / L : 0.f);
   }
 }
 
@@ -1152,6 +1181,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using SL = StageLayout<KF, VF, CH>;
   constexpr int NX = PACK ? 1 : 2;
   extern __shared__ __align__(128) unsigned char smem[];
+  pdl_launch();  // the merge kernel may be scheduled as CTAs retire
   // Shared-memory layout (shared-window addresses): stages below kLutAddr
   // while they fit, the tables at kLutAddr, then the other stages and the
   // scratch area.  Checked against the allocation before anything runs.
@@ -1160,7 +1190,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   while (n_low < S && low0 + (n_low + 1) * SL::bytes <= kLutAddr) ++n_low;
   const uint32_t high0 = kLutAddr + L::bytes;
   uint32_t end = high0 + (S - n_low) * SL::bytes, scratch_addr;
-  const uint32_t scr_bytes = scratch_bytes(a.n_sink);
+  const uint32_t scr_bytes = kScratchBytes;
   if (low0 + n_low * SL::bytes + scr_bytes <= kLutAddr) {
     scratch_addr = low0 + n_low * SL::bytes;
   } else {
@@ -1178,9 +1208,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   unsigned char* lut_mem = smem + (kLutAddr - dyn0);
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
-  __shared__ long long s_C, s_c0, s_c1;
+  __shared__ long long s_c0, s_c1;
   __shared__ int s_u0, s_lc0;
-  __shared__ volatile int s_abort, s_flag;
+  __shared__ volatile int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int P = gridDim.x, cta = blockIdx.x;
   const int U = a.B * a.hkv;
@@ -1253,13 +1283,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       for (int b = lane; b < a.B; b += 32)
         if (a.lens[b] > a.max_len) atomicOr(a.status, 2);
     if (lane == 0) {
-      s_C = C;
       s_c0 = c0;
       s_c1 = c1;
       s_u0 = u0;
       s_lc0 = lc0;
       s_abort = 0;
-      s_flag = 0;
     }
   }
   if (tid == 32) {
@@ -1271,7 +1299,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     mbar_fence_init();
   }
   __syncthreads();
-  const long long C = s_C, c0 = s_c0, c1 = s_c1;
+  const long long c0 = s_c0, c1 = s_c1;
 
   if (warp == kConsumers) {
     // ---- producer: one lane streams the CTA's chunks through the stages
@@ -1321,66 +1349,25 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const float thr = a.sparse_thr;
 
-  // sink pieces and empty sequences of the units u = cta (mod P)
-  for (int u = cta; u < U; u += P) {
-    const UnitInfo ui = unit_info(a, u, CH);
-    if (ui.len == 0) {
-      const int b = u / a.hkv, kvh = u % a.hkv;
-      for (int i = tid; i < a.group * kDim; i += kConsumers * 32)
-        store_out(a, (static_cast<int64_t>(b) * a.hq + kvh * a.group) * kDim + i, 0.f);
-      continue;
-    }
-    if (ui.ns == 0) continue;
-    sink_piece(a, u, ui.ns, scratch);
-    int first = 1, last = 0;
-    if (ui.chunks > 0) {
-      const long long cu0 = unit_first_chunk(a, u, CH);
-      first = cta_of_chunk(cu0, C, P);
-      last = cta_of_chunk(cu0 + ui.chunks - 1, C, P);
-    }
-    publish_piece<VF>(a, u, first, last, true, scratch, &s_flag, &s_abort, C);
-  }
+  pdl_wait();  // the rotated query fragments
 
   WarpState<KF, VF, PACK> wst;
   QFrag<PACK> bq, bqs;
-  constexpr int kMaxPending = 32;
-  __shared__ int s_pend[kMaxPending][4];
-  int n_pend = 0;  // same value in every consumer thread
   int u = -1;
   UnitInfo ui{};
-  long long cu0 = 0;
   int walk_u = s_u0, walk_lc = s_lc0;
   UnitInfo wui = c0 < c1 ? unit_info(a, walk_u, CH) : UnitInfo{};
-  long long walk_cu0 = c0 - s_lc0;
   long long k = 0;
   for (long long c = c0; c < c1; ++c, ++k) {
     while (walk_lc >= wui.chunks) {
-      walk_cu0 += wui.chunks;
       ++walk_u;
       walk_lc = 0;
       wui = unit_info(a, walk_u, CH);
     }
     if (walk_u != u) {
-      if (u >= 0) {
-        // publish the partial now; count it (and merge, if it completes the
-        // unit) after the range, so no merge stalls the stream
-        write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
-        const int first = cta_of_chunk(cu0, C, P), last = cta_of_chunk(cu0 + ui.chunks - 1, C, P);
-        if (n_pend < kMaxPending) {
-          if (tid == 0) {
-            s_pend[n_pend][0] = u;
-            s_pend[n_pend][1] = first;
-            s_pend[n_pend][2] = last;
-            s_pend[n_pend][3] = ui.ns > 0;
-          }
-          ++n_pend;
-        } else {
-          publish_piece<VF>(a, u, first, last, ui.ns > 0, scratch, &s_flag, &s_abort, C);
-        }
-      }
+      if (u >= 0) write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
       u = walk_u;
       ui = wui;
-      cu0 = walk_cu0;
       const uint32_t* qf = a.qfrag + static_cast<int64_t>(u) * kQfragWords;
 #pragma unroll
       for (int s = 0; s < 8; ++s)
@@ -1417,14 +1404,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     if (lane == 0) mbar_arrive(&empty_bar[s]);
     ++walk_lc;
   }
-  if (u >= 0) {
-    write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
-    publish_piece<VF>(a, u, cta_of_chunk(cu0, C, P), cta_of_chunk(cu0 + ui.chunks - 1, C, P), ui.ns > 0, scratch,
-                      &s_flag, &s_abort, C);
-  }
-  consumers_sync();  // the pending list written by thread 0 is visible
-  for (int i = 0; i < n_pend; ++i)
-    publish_piece<VF>(a, s_pend[i][0], s_pend[i][1], s_pend[i][2], s_pend[i][3] != 0, scratch, &s_flag, &s_abort, C);
+  if (u >= 0) write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
   if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
 
@@ -1442,9 +1422,28 @@ int num_sms_cached() {
 }
 
 template <int KF, int VF>
-size_t decode_smem_bytes(int n_sink) {
+size_t decode_smem_bytes() {
   using CF = DecodeCfg<KF, VF>;
-  return static_cast<size_t>(plan_end(CF::stage, CF::S, CF::lut, scratch_bytes(n_sink)) - kDynBaseMax);
+  return static_cast<size_t>(plan_end(CF::stage, CF::S, CF::lut, kScratchBytes) - kDynBaseMax);
+}
+
+// Launch with programmatic stream serialization: the kernel may start before
+// the previous kernel on the stream has finished (it calls pdl_wait before
+// reading that kernel's output).
+template <typename Kernel>
+cudaError_t launch_overlapped(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t st,
+                              const DecodeArgs& a) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 template <int KF, int VF, bool PACK>
@@ -1452,21 +1451,27 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF, PACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
+  // the query rotation waits for all earlier work on the stream (the appends
+  // that filled the cache); the two kernels after it overlap their prologues
+  // with its tail
   qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
-  decode_kernel<KF, VF, PACK><<<plan.ctas, kThreadsP, smem, st>>>(a);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "decode kernel launch");
+  e = launch_overlapped(decode_kernel<KF, VF, PACK>, dim3(plan.ctas), kThreadsP, smem, st, a);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  const size_t merge_smem = static_cast<size_t>(a.n_sink) * sizeof(float);
+  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv, plan.group), kMergeThreads, merge_smem, st, a);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "merge kernel launch");
 }
 
 template <int KF, int VF>
 tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
-  if (decode_smem_bytes<KF, VF>(a.n_sink) + kDynBaseMax > static_cast<size_t>(kSmemEnd))
-    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink too large for the shared-memory plan");
+  if (decode_smem_bytes<KF, VF>() + kDynBaseMax > static_cast<size_t>(kSmemEnd))
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: no shared-memory plan for this format");
   const size_t smem = kSmemBudget;  // the whole window: one CTA per SM
   a.dyn_bytes = static_cast<uint32_t>(smem);
   a.pack = plan.group <= 4;
+  a.chunk = DecodeCfg<KF, VF>::CH;
   return a.pack ? run_decode_v<KF, VF, true>(a, plan, smem, st) : run_decode_v<KF, VF, false>(a, plan, smem, st);
 }
 
@@ -1481,13 +1486,13 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) 
   pl.hkv = hkv;
   pl.group = hq / hkv;
   pl.max_len = max_len;
-  pl.ctas = num_sms_cached();
+  pl.ctas = num_sms_cached() < kMaxPieces ? num_sms_cached() : kMaxPieces;
   pl.part_floats = 2 + (p->fv.prod ? 2 * kDim : kDim);
   const size_t units = static_cast<size_t>(B) * hkv;
-  const size_t tickets = (units * sizeof(int32_t) + 255) & ~size_t(255);
   const size_t qfrag = (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
-  const size_t slots = 2 * units + pl.ctas;
-  pl.ws_total_bytes = tickets + qfrag + slots * kMaxG * pl.part_floats * sizeof(float);
+  // piece (u, cta) uses slot u + cta: fewer than units + ctas slots
+  const size_t slots = units + pl.ctas;
+  pl.ws_total_bytes = qfrag + slots * pl.group * pl.part_floats * sizeof(float);
   return pl;
 }
 
@@ -1516,10 +1521,10 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.n_sink = c->n_sink;
   a.max_len = plan.max_len;
   a.part_floats = plan.part_floats;
+  a.ctas = plan.ctas;
+  if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 12288");
   const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
   char* w = static_cast<char*>(ws);
-  a.tickets = reinterpret_cast<int32_t*>(w);
-  w += (units * sizeof(int32_t) + 255) & ~size_t(255);
   a.qfrag = reinterpret_cast<uint32_t*>(w);
   w += (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
   a.parts = reinterpret_cast<float*>(w);

@@ -1,7 +1,7 @@
 // Decode attention for callers that cannot allocate device memory.
 //
-// tq_decode_attn needs a caller-provided workspace (per-call tickets, query
-// fragments and split partials).  Some callers cannot obtain one: an
+// tq_decode_attn needs a caller-provided workspace (query fragments and split
+// partials).  Some callers cannot obtain one: an
 // inference engine that reserves all device memory up front for its own pool
 // and runs our call from plugin code that has no handle on that pool, or a
 // latency-critical decode loop where cudaMalloc's implicit device
@@ -81,11 +81,8 @@ extern "C" tq_status tq_decode_attn_noalloc(const tq_params* p, const void* q, i
   void* scratch = nullptr;
   tq_status st = scratch_address(&scratch);
   if (st != TQ_OK) return st;
-  // The arrival tickets at the head of the scratch must start at zero; the
-  // rest is written before it is read.
-  const size_t tickets = (static_cast<size_t>(B) * hkv * sizeof(int32_t) + 255) & ~size_t(255);
-  cudaError_t e = cudaMemsetAsync(scratch, 0, tickets, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return tq::cuda_fail(e, "tq_decode_attn_noalloc: clearing the tickets");
+  // Nothing in the scratch needs to start at zero: every word a kernel reads
+  // was written earlier in the same call.
   return tq::launch_decode(p, q, q_dtype == TQ_BF16, cache, plan, out, out_dtype == TQ_BF16, scratch, thr,
                            static_cast<cudaStream_t>(stream));
 }
