@@ -217,12 +217,14 @@ def run_gpu(args):
                        "decode_ms": round(avg_decode_s * 1e3, 4),
                        "append_plus_decode_bytes_per_step": (append_b + decode_b) // args.steps,
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"kernel": "decode_kernel<mixed3.5,mixed3.5> (+qrot)", "bound": "hbm",
+            "roofline": {"kernel": "decode_kernel<mixed3.5,mixed3.5> (+qrot, merge)", "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                          "bytes_per_launch": int(decode_bytes_per_launch), "traffic": args.traffic},
             "clocks": clocks,
-            "gpu_launches": args.steps * 5,
+            # per step: append = quantize K, quantize V, length update;
+            # decode = query rotation, decode kernel, merge
+            "gpu_launches": args.steps * 6,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "aux": aux,

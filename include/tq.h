@@ -207,7 +207,7 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
  * rotated domain and Pi^T (and S^T) applied once per output.  Sink tokens use
  * their bf16 keys and values directly.  A sequence with no tokens gives a
  * zero output.  max_len: host bound on lens (longer sequences are cut to it
- * and bit 2 is set in cache->status).  n_sink above 12288 gives
+ * and bit 2 is set in cache->status).  n_sink above 4096 gives
  * TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the query rotation,
  * the persistent decode kernel and the merge; the last two are launched with
  * programmatic stream serialization and overlap their prologues with the

@@ -439,6 +439,11 @@ __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]) : reinterpret_cast<const float*>(q)[i];
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
 // Programmatic dependent launch.  The three kernels of one decode call run
 // back to back on one stream; the second and third are launched with
 // programmatic stream serialization, so they may start while the previous one
@@ -457,31 +462,54 @@ template <int KF>
 __global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
   using KR = KRow<KF>;
   using FK = Fmt<KF>;
-  __shared__ float qs[kMaxG][kDim];
+  extern __shared__ float4 s_mat4[];              // Pi^T [k][j], then S^T [k][j] (prod keys)
+  __shared__ __align__(16) float qsT[kDim][kMaxG];  // query, [k][head]
   __shared__ float qt[kMaxG][kDim];
   __shared__ float qsk[kMaxG][kSketch];
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = a.group;
   pdl_launch();  // the decode kernel's prologue and cache stream may start
-  for (int i = tid; i < kMaxG * kDim; i += kThreads) {
-    const int h = i / kDim, d = i % kDim;
-    qs[h][d] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
+  {
+    // stage the matrices with asynchronous 16-byte copies, all in flight
+    constexpr int N4 = kDim * kDim / 4 / kThreads;
+    const float4* pit4 = reinterpret_cast<const float4*>(a.pit);
+#pragma unroll
+    for (int i = 0; i < N4; ++i) cp_async16(smem_u32(s_mat4 + i * kThreads + tid), pit4 + i * kThreads + tid);
+    if constexpr (FK::prod) {
+      const float4* st4 = reinterpret_cast<const float4*>(a.st);
+#pragma unroll
+      for (int i = 0; i < N4; ++i)
+        cp_async16(smem_u32(s_mat4 + kDim * kDim / 4 + i * kThreads + tid), st4 + i * kThreads + tid);
+    }
   }
+  for (int i = tid; i < kMaxG * kDim; i += kThreads) {
+    const int h = i % kMaxG, d = i / kMaxG;
+    qsT[d][h] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
+  }
+  cp_async_wait_all();
   __syncthreads();
   const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
   {
     const int j = tid & (kDim - 1);
     const bool sketch = tid >= kDim;
     if (!sketch || FK::prod) {
-      const float* mat = sketch ? a.st : a.pit;  // [k][j] layouts, coalesced over j
+      const float* mat = reinterpret_cast<const float*>(s_mat4) + (sketch ? kDim * kDim : 0);
+      const float4* q4 = reinterpret_cast<const float4*>(&qsT[0][0]);
       float acc[kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
 #pragma unroll 8
       for (int k = 0; k < kDim; ++k) {
-        const float m = __ldg(mat + k * kDim + j);
-#pragma unroll
-        for (int h = 0; h < kMaxG; ++h) acc[h] = fmaf(m, qs[h][k], acc[h]);
+        const float m = mat[k * kDim + j];
+        const float4 x0 = q4[2 * k], x1 = q4[2 * k + 1];
+        acc[0] = fmaf(m, x0.x, acc[0]);
+        acc[1] = fmaf(m, x0.y, acc[1]);
+        acc[2] = fmaf(m, x0.z, acc[2]);
+        acc[3] = fmaf(m, x0.w, acc[3]);
+        acc[4] = fmaf(m, x1.x, acc[4]);
+        acc[5] = fmaf(m, x1.y, acc[5]);
+        acc[6] = fmaf(m, x1.z, acc[6]);
+        acc[7] = fmaf(m, x1.w, acc[7]);
       }
       if (sketch) {
 #pragma unroll
@@ -770,20 +798,24 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, bool o
 }
 
 // One warp tile of 32 tokens (two 16-token subtiles) starting at stage row
-// `srow`, unit-relative row `row0`; tokens at or past `nq` are masked.
-template <int KF, int VF, bool PACK, int WT>
+// `srow`, unit-relative row `row0`; tokens at or past `nq` are masked (their
+// scores are -inf and their value weights 0, so a subtile past the end adds
+// nothing; computing it anyway keeps the two subtiles free of branches, which
+// lets their lookup and MMA chains interleave).  SPARSE: skip the PV MMAs of
+// a subtile whose weights are all below the sparse-V threshold.
+template <int KF, int VF, bool PACK, int WT, bool SPARSE>
 __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int row0, int nq,
                                              WarpState<KF, VF, PACK>& W, const QFrag<PACK>& bq,
                                              const QFrag<PACK>& bqs, int g, int t, uint32_t lut_a,
                                              uint32_t lut_b, uint32_t lane4, uint32_t lane8,
                                              uint32_t c1k, uint32_t c1v, float thr) {
   constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
-  const bool second = WT == 2 * kTok && row0 + kTok < nq;  // warp-uniform: the second subtile holds tokens
+  constexpr bool second = WT == 2 * kTok;
   const bool ok0A = row0 + g < nq, ok0B = row0 + g + 8 < nq;
   const bool ok1A = row0 + kTok + g < nq, ok1B = row0 + kTok + g + 8 < nq;
   float s0[4], s1[4];
   subtile_scores<KF, PACK>(u, srow, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
-  if (second)
+  if constexpr (second)
     subtile_scores<KF, PACK>(u, srow + kTok, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
@@ -825,8 +857,11 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
       W.oacc[i][3] *= al1;
     }
   }
-  bool keep0 = true, keep1 = second;
-  if (thr > 0.f) {
+  if constexpr (!SPARSE) {
+    subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+    if constexpr (second)
+      subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+  } else {
     // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
     const float c0 = thr * W.l0, c1 = thr * W.l1;
 #pragma unroll
@@ -836,11 +871,11 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
       p1[i] = p1[i] >= c0 ? p1[i] : 0.f;
       p1[i + 1] = p1[i + 1] >= c1 ? p1[i + 1] : 0.f;
     }
-    keep0 = __any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f);
-    keep1 = second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f);
+    if (__any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f))
+      subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+    if (second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f))
+      subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   }
-  if (keep0) subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
-  if (keep1) subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
 }
 
 // ---------------------------------------------------------------------------
@@ -987,31 +1022,33 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
 }
 
 // ---------------------------------------------------------------------------
-// 3. merge: one CTA per (unit, query head).  The unit's quantized tokens were
-//    streamed as pieces by consecutive CTAs of the decode grid; its bf16 sink
-//    tokens are attended here.  Partial results are combined by their maxima
-//    (the usual online-softmax merge), Pi^T (and S^T for prod values) is
-//    applied once, and the result is divided by the softmax sum.  Everything
-//    that does not read the pieces runs before pdl_wait, overlapping the tail
-//    of the decode kernel.
+// 3. merge: one CTA per unit (sequence, kv-head), all heads of its group.
+//    The unit's quantized tokens were streamed as pieces by consecutive CTAs
+//    of the decode grid; its bf16 sink tokens are attended here.  Partial
+//    results are combined by their maxima (the usual online-softmax merge),
+//    Pi^T (and S^T for prod values) is applied once, and the result is
+//    divided by the softmax sum.  The matrix rows and the sink run before
+//    pdl_wait, overlapping the tail of the decode kernel.
 // ---------------------------------------------------------------------------
 constexpr int kMergeThreads = 512;
 constexpr int kMaxPieces = 1024;  // bound on the decode grid size
-constexpr int kMaxSink = 12288;   // sink scores live in 48 KB of shared memory
+constexpr int kMaxSink = 4096;    // sink weights live in shared memory
 
-__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = is_max ? fmaxf(v, o) : v + o;
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();  // red may still be read by an earlier reduction
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  v = red[0];
-  for (int w = 1; w < kMergeThreads / 32; ++w) v = is_max ? fmaxf(v, red[w]) : v + red[w];
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
   return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Merge shared memory beyond the static arrays: sink weights [n_sink][8] and
+// piece weights [ctas][8].
+inline size_t merge_dyn_bytes(int n_sink, int ctas) {
+  return (static_cast<size_t>(n_sink) + ctas) * kMaxG * sizeof(float);
 }
 
 template <int VF>
@@ -1021,23 +1058,35 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   constexpr int WD = FV::prod ? 2 * kDim : kDim;  // accumulator: rotated | sketch
   constexpr int NS = NT / WD;                     // piece slices of the accumulation
   constexpr int RS = WD / 4;                      // matrix rows per un-rotation slice
-  extern __shared__ float s_sc[];                 // [n_sink] sink scores, then weights
-  __shared__ float s_f[kMaxPieces];               // per piece: max, then weight
-  __shared__ float s_red[NT];
-  __shared__ float s_acc[WD];
-  __shared__ float s_osk[kDim];
-  __shared__ float s_q[kDim];
-  __shared__ float s_w[NT / 32];
+  extern __shared__ float4 s_dyn4[];
+  __shared__ float s_red[4 * kMaxG * kDim];       // slice partials
+  __shared__ __align__(16) float s_acc[WD][kMaxG];  // merged accumulator, [j][head]
+  __shared__ float s_osk[kMaxG][kDim];            // sink values, original domain
+  __shared__ float s_q[kMaxG][kDim];
+  __shared__ float s_ms[kMaxG], s_ls[kMaxG], s_M[kMaxG], s_L[kMaxG];
   __shared__ long long s_C, s_cu0;
-  const int u = blockIdx.x, h = blockIdx.y;
+  float* s_sc = reinterpret_cast<float*>(s_dyn4);  // [n_sink][8]
+  float* s_f = s_sc + a.n_sink * kMaxG;             // [pieces][8]
+  const int u = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.group, P = a.ctas, CH = a.chunk, PF = a.part_floats;
   const int b = u / a.hkv, kvh = u % a.hkv;
-  const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim;
+  const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * G) * kDim;  // head 0 of the group
   const UnitInfo ui = unit_info(a, u, CH);
   if (ui.len == 0) {
-    if (tid < kDim) store_out(a, orow + tid, 0.f);
+    for (int i = tid; i < G * kDim; i += NT) store_out(a, orow + i, 0.f);
     return;
+  }
+  // this thread's matrix rows for the un-rotation: column o, rows
+  // [sl*RS, (sl+1)*RS) of [Pi; sqrt(pi/2)/m S]
+  const int o = tid & (kDim - 1), sl4 = tid >> 7;
+  float pm[RS];
+  if (ui.chunks > 0) {
+    const int j0 = sl4 * RS;
+    const bool sk = FV::prod && j0 >= kDim;
+    const float* mat = sk ? a.s + (j0 - kDim) * kDim : a.pi + j0 * kDim;
+#pragma unroll
+    for (int jj = 0; jj < RS; ++jj) pm[jj] = __ldg(mat + jj * kDim + o) * (sk ? kQjlScale : 1.f);
   }
   // where the unit's chunks sit in the decode schedule (warp 0)
   if (warp == 0 && ui.chunks > 0) {
@@ -1058,120 +1107,173 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     }
   }
   // sink: scores with the original query, softmax weights, weighted values
-  float ms = -INFINITY, ls = 0.f;
   if (ui.ns > 0) {
-    if (tid < kDim) s_q[tid] = load_q(a.q, a.q_bf16, orow + tid);
+    for (int i = tid; i < kMaxG * kDim; i += NT) (&s_q[0][0])[i] = i < G * kDim ? load_q(a.q, a.q_bf16, orow + i) : 0.f;
     __syncthreads();
     const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
     const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
     const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
     for (int t = warp; t < ui.ns; t += NT / 32) {
       const __nv_bfloat16* kr = ks + static_cast<int64_t>(t) * kDim + 4 * lane;
-      float d = 0.f;
+      float k4[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) d = fmaf(__bfloat162float(kr[e]), s_q[4 * lane + e], d);
+      for (int e = 0; e < 4; ++e) k4[e] = __bfloat162float(kr[e]);
+      for (int h = 0; h < G; ++h) {
+        float d = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      if (lane == 0) s_sc[t] = d * scale;
+        for (int e = 0; e < 4; ++e) d = fmaf(k4[e], s_q[h][4 * lane + e], d);
+        d = warp_sum(d);
+        if (lane == 0) s_sc[t * kMaxG + h] = d * scale;
+      }
     }
     __syncthreads();
-    float mx = -INFINITY;
-    for (int t = tid; t < ui.ns; t += NT) mx = fmaxf(mx, s_sc[t]);
-    ms = block_reduce(mx, true, s_w);
-    float sum = 0.f;
-    for (int t = tid; t < ui.ns; t += NT) {
-      const float p = exp2f(s_sc[t] - ms);
-      s_sc[t] = p;
-      sum += p;
+    if (warp < G) {  // warp h: max, weights and sum of head h
+      const int h = warp;
+      float mx = -INFINITY;
+      for (int t = lane; t < ui.ns; t += 32) mx = fmaxf(mx, s_sc[t * kMaxG + h]);
+      mx = warp_max(mx);
+      float sum = 0.f;
+      for (int t = lane; t < ui.ns; t += 32) {
+        const float p = exp2f(s_sc[t * kMaxG + h] - mx);
+        s_sc[t * kMaxG + h] = p;
+        sum += p;
+      }
+      sum = warp_sum(sum);
+      if (lane == 0) {
+        s_ms[h] = mx;
+        s_ls[h] = sum;
+      }
     }
-    ls = block_reduce(sum, false, s_w);  // its barriers also publish s_sc
+    __syncthreads();
     {
-      const int j = tid & (kDim - 1), sl = tid >> 7;
-      float acc = 0.f;
-      for (int t = sl; t < ui.ns; t += NT / kDim) acc = fmaf(s_sc[t], __bfloat162float(vs[static_cast<int64_t>(t) * kDim + j]), acc);
-      s_red[sl * kDim + j] = acc;
+      float acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+      for (int t = sl4; t < ui.ns; t += 4) {
+        const float v = __bfloat162float(vs[static_cast<int64_t>(t) * kDim + o]);
+        const float4 p0 = s_dyn4[t * 2], p1 = s_dyn4[t * 2 + 1];
+        acc[0] = fmaf(p0.x, v, acc[0]);
+        acc[1] = fmaf(p0.y, v, acc[1]);
+        acc[2] = fmaf(p0.z, v, acc[2]);
+        acc[3] = fmaf(p0.w, v, acc[3]);
+        acc[4] = fmaf(p1.x, v, acc[4]);
+        acc[5] = fmaf(p1.y, v, acc[5]);
+        acc[6] = fmaf(p1.z, v, acc[6]);
+        acc[7] = fmaf(p1.w, v, acc[7]);
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) s_red[(sl4 * kMaxG + h) * kDim + o] = acc[h];
     }
     __syncthreads();
-    if (tid < kDim) {
-      float v = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < NT / kDim; ++sl) v += s_red[sl * kDim + tid];
-      s_osk[tid] = v;
+    for (int i = tid; i < G * kDim; i += NT) {
+      const int h = i / kDim, j = i % kDim;
+      s_osk[h][j] = s_red[(0 * kMaxG + h) * kDim + j] + s_red[(1 * kMaxG + h) * kDim + j] +
+                    s_red[(2 * kMaxG + h) * kDim + j] + s_red[(3 * kMaxG + h) * kDim + j];
     }
+  } else if (tid < kMaxG) {
+    s_ms[tid] = -INFINITY;
+    s_ls[tid] = 0.f;
   }
   __syncthreads();
   // the pieces: written by the decode kernel
   pdl_wait();
-  float M = ms, L = 0.f;
   const bool has_pieces = ui.chunks > 0;
   int first = 0, n_p = 0;
+  long long C = 0;
   if (has_pieces) {
-    const long long C = s_C, cu0 = s_cu0;
+    C = s_C;
+    const long long cu0 = s_cu0;
     first = cta_of_chunk(cu0, C, P);
     n_p = cta_of_chunk(cu0 + ui.chunks - 1, C, P) - first + 1;
-    float mx = -INFINITY;
-    for (int i = tid; i < n_p; i += NT) {
-      const float m = cta_has_chunks(first + i, C, P) ? __ldcg(part_slot(a, u + first + i) + h * PF) : -INFINITY;
-      s_f[i] = m;
-      mx = fmaxf(mx, m);
-    }
-    M = fmaxf(M, block_reduce(mx, true, s_w));
-    float lsum = 0.f;
-    for (int i = tid; i < n_p; i += NT) {
-      const float m = s_f[i];
-      const float f = m > -INFINITY ? exp2f(m - M) : 0.f;
-      if (f != 0.f) lsum = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 1), f, lsum);
-      s_f[i] = f;
-    }
-    L = block_reduce(lsum, false, s_w);  // its barriers also publish s_f
-    {
-      const int j = tid % WD, sl = tid / WD;
-      float acc = 0.f;
-      for (int i = sl; i < n_p; i += NS) {
-        const float f = s_f[i];
-        if (f != 0.f) acc = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 2 + j), f, acc);
-      }
-      s_red[sl * WD + j] = acc;
-    }
-    __syncthreads();
-    for (int j = tid; j < WD; j += NT) {
-      float v = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < NS; ++sl) v += s_red[sl * WD + j];
-      if (j < kDim) v = FV::width(j) > 0 ? v / a.sig[FV::width(j)] : 0.f;
-      s_acc[j] = v;
-    }
-    __syncthreads();
   }
-  const float fs = ui.ns > 0 ? exp2f(ms - M) : 0.f;
-  L = fmaf(ls, fs, L);
-  // un-rotation: out_o = sum_j Pi[j][o] A_j + sqrt(pi/2)/m sum_j S[j][o] B_j;
-  // thread (o, slice) sums RS consecutive rows j, rows read coalesced over o
-  {
-    const int o = tid & (kDim - 1), sl = tid >> 7;
-    float r = 0.f;
-    if (has_pieces) {
-      const int j0 = sl * RS;
-      const bool sk = FV::prod && j0 >= kDim;
-      const float* mat = sk ? a.s + (j0 - kDim) * kDim : a.pi + j0 * kDim;
-      const float* src = s_acc + j0;
-#pragma unroll 8
-      for (int jj = 0; jj < RS; ++jj) r = fmaf(__ldg(mat + jj * kDim + o), src[jj], r);
-      if (sk) r *= kQjlScale;
+  if (warp < G) {  // warp h: the pieces' maxima, weights and sums for head h
+    const int h = warp;
+    float M = s_ms[h];
+    for (int i = lane; i < n_p; i += 32) {
+      const float m = cta_has_chunks(first + i, C, P) ? __ldcg(part_slot(a, u + first + i) + h * PF) : -INFINITY;
+      s_f[i * kMaxG + h] = m;
+      M = fmaxf(M, m);
     }
-    s_red[sl * kDim + o] = r;
+    M = warp_max(M);
+    float L = 0.f;
+    for (int i = lane; i < n_p; i += 32) {
+      const float m = s_f[i * kMaxG + h];
+      const float f = m > -INFINITY ? exp2f(m - M) : 0.f;
+      if (f != 0.f) L = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 1), f, L);
+      s_f[i * kMaxG + h] = f;
+    }
+    L = warp_sum(L);
+    if (lane == 0) {
+      const float fs = s_ms[h] > -INFINITY ? exp2f(s_ms[h] - M) : 0.f;
+      s_M[h] = fs;  // sink weight relative to the merged maximum
+      s_L[h] = fmaf(s_ls[h], fs, L);
+    }
   }
   __syncthreads();
-  if (tid < kDim) {
-    float v = 0.f;
+  if (has_pieces) {
+    {
+      const int j = tid % WD, sl = tid / WD;
+      float acc[kMaxG];
 #pragma unroll
-    for (int sl = 0; sl < 4; ++sl) v += s_red[sl * kDim + tid];
-    if (ui.ns > 0) v = fmaf(fs, s_osk[tid], v);
-    store_out(a, orow + tid, L > 0.f ? v / L : 0.f);
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+      for (int i = sl; i < n_p; i += NS) {
+        const float* pp = part_slot(a, u + first + i) + 2 + j;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          if (h < G) {
+            const float f = s_f[i * kMaxG + h];
+            if (f != 0.f) acc[h] = fmaf(__ldcg(pp + h * PF), f, acc[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) s_red[(sl * kMaxG + h) * WD + j] = acc[h];
+    }
+    __syncthreads();
+    for (int i = tid; i < kMaxG * WD; i += NT) {
+      const int j = i / kMaxG, h = i % kMaxG;
+      float v = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < NS; ++sl) v += s_red[(sl * kMaxG + h) * WD + j];
+      if (j < kDim) v = FV::width(j) > 0 ? v / a.sig[FV::width(j)] : 0.f;
+      s_acc[j][h] = h < G ? v : 0.f;
+    }
+    __syncthreads();
+    // un-rotation: out_h[o] = sum_j Pi[j][o] A_h[j] + sqrt(pi/2)/m sum_j S[j][o] B_h[j]
+    float r[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) r[h] = 0.f;
+    const float4* acc4 = reinterpret_cast<const float4*>(&s_acc[sl4 * RS][0]);
+#pragma unroll
+    for (int jj = 0; jj < RS; ++jj) {
+      const float4 x0 = acc4[2 * jj], x1 = acc4[2 * jj + 1];
+      r[0] = fmaf(pm[jj], x0.x, r[0]);
+      r[1] = fmaf(pm[jj], x0.y, r[1]);
+      r[2] = fmaf(pm[jj], x0.z, r[2]);
+      r[3] = fmaf(pm[jj], x0.w, r[3]);
+      r[4] = fmaf(pm[jj], x1.x, r[4]);
+      r[5] = fmaf(pm[jj], x1.y, r[5]);
+      r[6] = fmaf(pm[jj], x1.z, r[6]);
+      r[7] = fmaf(pm[jj], x1.w, r[7]);
+    }
+    __syncthreads();  // s_red is reused
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) s_red[(sl4 * kMaxG + h) * kDim + o] = r[h];
+    __syncthreads();
+  }
+  for (int i = tid; i < G * kDim; i += NT) {
+    const int h = i / kDim, j = i % kDim;
+    float v = 0.f;
+    if (has_pieces)
+      v = s_red[(0 * kMaxG + h) * kDim + j] + s_red[(1 * kMaxG + h) * kDim + j] + s_red[(2 * kMaxG + h) * kDim + j] +
+          s_red[(3 * kMaxG + h) * kDim + j];
+    if (ui.ns > 0) v = fmaf(s_M[h], s_osk[h][j], v);
+    const float L = s_L[h];
+    store_out(a, orow + i, L > 0.f ? v / L : 0.f);
   }
 }
 
-template <int KF, int VF, bool PACK>
+template <int KF, int VF, bool PACK, bool SPARSE>
 __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
@@ -1217,7 +1319,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
 
   // ---- lookup tables (all threads), schedule and barriers (thread 0)
   {
-    const float* cb = a.cbs;
+    __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
+    if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
+    __syncthreads();
+    const float* cb = s_cb;
     if constexpr (L::t4) {
       for (int i = tid; i < 256 * 32; i += kThreadsP) {
         const int r = i >> 5, ln = i & 31;
@@ -1397,7 +1502,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       sp.kres = st + SL::kr;
       sp.vq = st + SL::vq;
       sp.vres = st + SL::vr;
-      compute_tile<KF, VF, PACK, WT>(sp, warp * WT, row0, ui.nq, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
+      compute_tile<KF, VF, PACK, WT, SPARSE>(sp, warp * WT, row0, ui.nq, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
                                  c1k, c1v, thr);
     }
     __syncwarp();
@@ -1446,21 +1551,28 @@ cudaError_t launch_overlapped(Kernel kernel, dim3 grid, int threads, size_t smem
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int KF, int VF, bool PACK>
+template <int KF, int VF, bool PACK, bool SPARSE>
 tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF, PACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF, PACK, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
   // the query rotation waits for all earlier work on the stream (the appends
   // that filled the cache); the two kernels after it overlap their prologues
   // with its tail
-  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, 0, st>>>(a);
+  const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
+  e = cudaFuncSetAttribute(qrot_kernel<KF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(qrot_smem));
+  if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
+  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, qrot_smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
-  e = launch_overlapped(decode_kernel<KF, VF, PACK>, dim3(plan.ctas), kThreadsP, smem, st, a);
+  e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-  const size_t merge_smem = static_cast<size_t>(a.n_sink) * sizeof(float);
-  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv, plan.group), kMergeThreads, merge_smem, st, a);
+  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas);
+  if (merge_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(merge_kernel<VF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(merge_smem));
+    if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
+  }
+  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv), kMergeThreads, merge_smem, st, a);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "merge kernel launch");
 }
 
@@ -1472,7 +1584,9 @@ tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
   a.dyn_bytes = static_cast<uint32_t>(smem);
   a.pack = plan.group <= 4;
   a.chunk = DecodeCfg<KF, VF>::CH;
-  return a.pack ? run_decode_v<KF, VF, true>(a, plan, smem, st) : run_decode_v<KF, VF, false>(a, plan, smem, st);
+  if (a.sparse_thr > 0.f)
+    return a.pack ? run_decode_v<KF, VF, true, true>(a, plan, smem, st) : run_decode_v<KF, VF, false, true>(a, plan, smem, st);
+  return a.pack ? run_decode_v<KF, VF, true, false>(a, plan, smem, st) : run_decode_v<KF, VF, false, false>(a, plan, smem, st);
 }
 
 constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 3) | (prod << 4); }
@@ -1522,7 +1636,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.max_len = plan.max_len;
   a.part_floats = plan.part_floats;
   a.ctas = plan.ctas;
-  if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 12288");
+  if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 4096");
   const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
   char* w = static_cast<char*>(ws);
   a.qfrag = reinterpret_cast<uint32_t*>(w);
