@@ -117,6 +117,13 @@ tq_status tq_qjl_matrix(uint64_t seed, int m, int d, double* s);
 tq_status tq_params_create(const tq_config* cfg, tq_params** out);
 void tq_params_destroy(tq_params* p);
 
+/* Error bits that tq_quantize kernels recorded on the device for p (appends
+ * record into their cache's status word instead): 4 = a wait in the copy /
+ * tensor-core pipeline gave up after its time limit (the outputs of that call
+ * are invalid).  Copies the word to *out (synchronizing the device); clear != 0
+ * then resets it.  Not for the data path. */
+tq_status tq_params_status(const tq_params* p, int32_t* out, int clear);
+
 /* Bytes per packed row for K (which = TQ_K) or V: code bytes and QJL bytes
  * (0 in MSE mode). */
 tq_status tq_row_bytes(const tq_params* p, int which, int* code_bytes, int* qjl_bytes);
@@ -125,7 +132,10 @@ tq_status tq_row_bytes(const tq_params* p, int which, int* code_bytes, int* qjl_
 
 /* Rotate, quantize and pack n vectors x ([n][d], fp32 or bf16, device) with
  * the K or V format of p into `out` (device planes sized for n rows).
- * Article section "Il metodo TurboQuant, in breve".  n = 0 is a no-op. */
+ * Article section "Il metodo TurboQuant, in breve".  n = 0 is a no-op.
+ * bf16 input in MSE or mixed formats (x 16-byte aligned) runs the rotation on
+ * the tensor cores (tcgen05, Pi split into two bf16 halves, fp32
+ * accumulation); fp32 input and prod formats use an fp32 SIMT kernel. */
 tq_status tq_quantize(const tq_params* p, const void* x, int x_dtype, int64_t n, int which,
                       const tq_packed* out, void* stream);
 

@@ -65,6 +65,7 @@ _SIGS = {
     "tq_qjl_matrix": (c_int, [c_uint64, c_int, c_int, _dp]),
     "tq_params_create": (c_int, [ctypes.POINTER(TqConfig), ctypes.POINTER(c_void_p)]),
     "tq_params_destroy": (None, [c_void_p]),
+    "tq_params_status": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_int32), c_int]),
     "tq_row_bytes": (c_int, [c_void_p, c_int, ctypes.POINTER(c_int), ctypes.POINTER(c_int)]),
     "tq_quantize": (c_int, [c_void_p, c_void_p, c_int, c_int64, c_int, ctypes.POINTER(TqPacked), c_void_p]),
     "tq_dequantize": (c_int, [c_void_p, ctypes.POINTER(TqPacked), c_int64, c_int, c_void_p, c_void_p]),
@@ -147,6 +148,12 @@ class Params:
         _check(_lib.tq_params_create(ctypes.byref(self.config), ctypes.byref(h)))
         self.handle = h.value
         self.d, self.m = d, m
+
+    def status(self, clear: bool = False) -> int:
+        """Error bits recorded by quantize kernels for these parameters (see tq.h)."""
+        out = ctypes.c_int32()
+        _check(_lib.tq_params_status(self.handle, ctypes.byref(out), int(clear)))
+        return out.value
 
     def row_bytes(self, which: int):
         cb, qb = c_int(), c_int()

@@ -340,7 +340,8 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   size_t o_pi = take(pi32.size() * 4), o_pit = take(pit32.size() * 4), o_s = take(s32.size() * 4),
          o_st = take(st32.size() * 4), o_mt = take(mt32.size() * 4), o_pi64 = take(p->pi.size() * 8),
          o_s64 = take(p->s.size() * 8), o_cb = take(cb32.size() * 4), o_bd = take(bd32.size() * 4),
-         o_cb64 = take(cb64.size() * 8), o_cbs = take(cbs32.size() * 4), o_sig = take(sig32.size() * 4);
+         o_cb64 = take(cb64.size() * 8), o_cbs = take(cbs32.size() * 4), o_sig = take(sig32.size() * 4),
+         o_status = take(sizeof(int32_t));
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->block, off);
   if (e != cudaSuccess) {
@@ -361,6 +362,13 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   p->cb64 = reinterpret_cast<double*>(base + o_cb64);
   p->cbs32 = reinterpret_cast<float*>(base + o_cbs);
   p->sig32 = reinterpret_cast<float*>(base + o_sig);
+  p->status32 = reinterpret_cast<int32_t*>(base + o_status);
+  e = cudaMemset(p->status32, 0, sizeof(int32_t));
+  if (e != cudaSuccess) {
+    cudaFree(p->block);
+    delete p;
+    return cuda_fail(e, "tq_params_create: status word");
+  }
   struct { void* dst; const void* src; size_t n; } copies[] = {
       {p->pi32, pi32.data(), pi32.size() * 4},   {p->pit32, pit32.data(), pit32.size() * 4},
       {p->s32, s32.data(), s32.size() * 4},      {p->st32, st32.data(), st32.size() * 4},
@@ -384,6 +392,13 @@ void tq_params_destroy(tq_params* p) {
   if (!p) return;
   if (p->block) cudaFree(p->block);
   delete p;
+}
+
+tq_status tq_params_status(const tq_params* p, int32_t* out, int clear) {
+  if (!p || !out) return fail(TQ_ERR_ARG, "tq_params_status: bad arguments");
+  cudaError_t e = cudaMemcpy(out, p->status32, sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && clear) e = cudaMemset(p->status32, 0, sizeof(int32_t));
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_params_status");
 }
 
 tq_status tq_row_bytes(const tq_params* p, int which, int* code_bytes, int* qjl_bytes) {

@@ -54,6 +54,7 @@ struct tq_params {
   float* sig32 = nullptr;  // sigma_b [kMaxBits+1]: scale making sigma_b*c near-exact in fp16
   float* bd32 = nullptr;   // decision bounds [kMaxBits+1][16]
   double* cb64 = nullptr;  // centroids fp64 [kMaxBits+1][16]
+  int32_t* status32 = nullptr;  // device word that plain quantize kernels OR error bits into
 };
 
 namespace tq {

@@ -15,10 +15,12 @@
 // accuracy: a coordinate within ~1e-6 of a bound is the only place the code
 // may differ from an fp64 reference).
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "tq_internal.h"
+#include "tq_sm100.cuh"
 
 namespace tq {
 namespace {
@@ -31,6 +33,7 @@ struct QuantArgs {
   int x_bf16;
   int64_t n;
   int mse_bits, mixed, prod, code_bytes;
+  const float* pi;   // Pi [d][d] (y = Pi u)
   const float* pit;  // Pi^T [d][d]
   const float* mt;   // (S Pi^T)^T [d][m]
   const float* cb;   // [5][16]
@@ -46,6 +49,7 @@ struct QuantArgs {
   const int32_t* lens;
   int n_tok, hkv, capacity, n_sink, cache_seqs;
   uint16_t* sink;  // bf16 [n_seq][hkv][n_sink][d]
+  int32_t* status;  // device word; bit 4 = a pipeline wait timed out
 };
 
 struct SmemQuant {
@@ -306,6 +310,280 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_kernel(QuantArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core rotate + quantize + pack (bf16 input, MSE and mixed formats).
+//
+// y = Pi x for a tile of 128 vectors is one 128 x 128 x 128 product on the
+// fifth-generation tensor cores: A = the bf16 tile (exact input), B = Pi split
+// as Pi_hi + Pi_lo in bf16 (16 mantissa bits together; the rounding error of
+// a rotated unit-vector coordinate stays near 1e-6, under the 1e-5 band in
+// which a code may legitimately differ), both products accumulated in fp32 in
+// tensor memory.  Warp roles in a persistent CTA (one per SM):
+//   warp 8      TMA producer: tiles of x, 128 rows x 256 B, into a 4-deep ring
+//               (two 64-column boxes, 128-byte swizzle);
+//   warp 9      allocates 256 TMEM columns and issues the MMAs (one thread);
+//   warps 0..7  two epilogue groups taking alternate tiles, each with its own
+//               128-column accumulator: thread = one vector (TMEM lane); norm
+//               from the staged bf16 row, 32-column TMEM loads, codes by a
+//               branch-free search over the symmetric decision bounds, packing
+//               in registers, 16- or 8-byte stores of the packed row.
+// ---------------------------------------------------------------------------
+constexpr int kTcRows = 128;                      // vectors per tile (MMA M)
+constexpr int kTcStages = 4;                      // x tiles in flight
+constexpr int kTcBox = kTcRows * 128;             // one 64-column box: 16 KB
+constexpr int kTcTile = 2 * kTcBox;               // one 128 x 128 bf16 tile: 32 KB
+constexpr int kTcThreads = 10 * 32;
+constexpr int kTcSmem = 2 * kTcTile + kTcStages * kTcTile + 1024;  // Pi hi/lo, x ring, alignment slack
+constexpr int kTcCols = 256;                      // TMEM columns: two 128-column accumulators
+
+// Code of u for a width-W codebook whose decision bounds are symmetric about
+// 0: pb[i] = the i-th positive bound (pb[0] = 0 is the middle one).  Equals the
+// count of bounds strictly below u except on exact ties with a bound.
+template <int W>
+__device__ __forceinline__ uint32_t sym_code(float u, const float (&pb)[8]) {
+  constexpr uint32_t H = 1u << (W - 1);
+  const float a = fabsf(u);
+  uint32_t j;
+  if constexpr (W == 1) {
+    j = 0;
+  } else if constexpr (W == 2) {
+    j = a > pb[1] ? 1u : 0u;
+  } else if constexpr (W == 3) {
+    const bool c1 = a > pb[2];
+    const bool c0 = a > (c1 ? pb[3] : pb[1]);
+    j = (c1 ? 2u : 0u) + (c0 ? 1u : 0u);
+  } else {
+    const bool c2 = a > pb[4];
+    const bool c1 = a > (c2 ? pb[6] : pb[2]);
+    const float t0 = c2 ? (c1 ? pb[7] : pb[5]) : (c1 ? pb[3] : pb[1]);
+    const bool c0 = a > t0;
+    j = (c2 ? 4u : 0u) + (c1 ? 2u : 0u) + (c0 ? 1u : 0u);
+  }
+  return u > 0.f ? H + j : H - 1u - j;
+}
+
+// 32 codes of width W from one 32-column TMEM chunk, packed LSB-first into W words.
+template <int W>
+__device__ __forceinline__ void pack_chunk(const uint32_t (&y)[32], float inv_nu, const float (&pb)[8],
+                                           uint32_t* out) {
+#pragma unroll
+  for (int w = 0; w < W; ++w) out[w] = 0u;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t c = sym_code<W>(__uint_as_float(y[j]) * inv_nu, pb);
+    const int bit = j * W, wi = bit >> 5, sh = bit & 31;
+    out[wi] |= c << sh;
+    if (sh + W > 32) out[wi + 1] |= c >> (32 - sh);
+  }
+}
+
+template <int B, int MIXED>
+struct TcFormat {
+  static constexpr int b0 = MIXED ? B + 1 : B;     // width of columns 0..63
+  static constexpr int b1 = B;                     // width of columns 64..127
+  static constexpr int words = 2 * b0 + 2 * b1;    // packed row, 32-bit words
+  static constexpr int bytes = 4 * words;
+};
+
+template <int B, int MIXED>
+__global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                    QuantArgs a) {
+  using namespace sm100;
+  using TF = TcFormat<B, MIXED>;
+  extern __shared__ __align__(16) unsigned char smem_tc[];
+  __shared__ __align__(8) uint64_t x_full[kTcStages], x_empty[kTcStages], t_full[2], t_empty[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ float s_pb[2][8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t raw = smem_u32(smem_tc);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* basep = smem_tc + (base - raw);
+  const uint32_t pih = base, pil = base + kTcTile, xs0 = base + 2 * kTcTile;
+
+  // Pi as the K-major B operand (row j = output coordinate, K = input
+  // coordinate), hi and lo bf16 halves, in the swizzled layout
+  for (int i = tid; i < kDim * kDim; i += kTcThreads) {
+    const int j = i >> 7, k = i & 127;
+    const float p = a.pi[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+    const int off = (k >> 6) * kTcBox + j * 128 + ((((k & 63) >> 3) ^ (j & 7)) << 4) + (k & 7) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(basep + off) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(basep + kTcTile + off) = lo;
+  }
+  if (tid < 16) {
+    const int seg = tid >> 3, i = tid & 7;
+    const int w = seg ? TF::b1 : TF::b0;
+    const int half = 1 << (w - 1);
+    s_pb[seg][i] = i < half ? a.bd[w * kBookSlots + half - 1 + i] : 0.f;
+  }
+  if (warp == 9) {
+    tmem_alloc(&s_tmem, kTcCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1 + 4);  // the MMA commit and the four epilogue warps
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&t_full[b], 1);
+      mbar_init(&t_empty[b], 4);
+    }
+    s_abort = 0;
+    mbar_fence_init();
+  }
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // B tiles visible to the tensor cores
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
+
+  if (warp == 8) {
+    // ---- producer
+    if (lane == 0) {
+      prefetch_tensormap(&xmap);
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+        const int s = i % kTcStages;
+        if (i >= kTcStages && !mbar_wait(&x_empty[s], ((i / kTcStages) - 1) & 1)) s_abort = 1;
+        if (s_abort) break;
+        mbar_expect_tx(&x_full[s], kTcTile);
+        tma_load_2d(xs0 + s * kTcTile, &xmap, 0, static_cast<int>(tile * kTcRows), &x_full[s]);
+        tma_load_2d(xs0 + s * kTcTile + kTcBox, &xmap, 64, static_cast<int>(tile * kTcRows), &x_full[s]);
+      }
+      // loads still in flight land before the CTA may exit
+      for (int k = i - kTcStages; k < i; ++k)
+        if (k >= 0) mbar_wait(&x_full[k % kTcStages], (k / kTcStages) & 1);
+    }
+  } else if (warp == 9) {
+    // ---- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTcRows, kDim);
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+        const int s = i % kTcStages, buf = i & 1;
+        if (!mbar_wait(&x_full[s], (i / kTcStages) & 1)) s_abort = 1;
+        if (i >= 2 && !s_abort && !mbar_wait(&t_empty[buf], ((i >> 1) - 1) & 1)) s_abort = 1;
+        if (s_abort) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * kDim;
+#pragma unroll
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t off = (k >> 2) * kTcBox + (k & 3) * 32;
+          const uint64_t ad = sw128_kmajor_desc(xs0 + s * kTcTile + off);
+          umma_bf16(d, ad, sw128_kmajor_desc(pih + off), idesc, k > 0);
+          umma_bf16(d, ad, sw128_kmajor_desc(pil + off), idesc, true);
+        }
+        umma_commit(&x_empty[s]);
+        umma_commit(&t_full[buf]);
+      }
+    }
+  } else {
+    // ---- epilogue: group g takes tiles i = g (mod 2); thread = TMEM lane = row
+    const int g = warp >> 2, q = warp & 3, r = 32 * q + lane;
+    float pb0[8], pb1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      pb0[k] = s_pb[0][k];
+      pb1[k] = s_pb[1][k];
+    }
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+      if ((i & 1) != g) continue;
+      if (s_abort) break;
+      const int s = i % kTcStages, buf = i & 1;
+      // norm of the row from the staged bf16 tile
+      if (!mbar_wait(&x_full[s], (i / kTcStages) & 1)) {
+        s_abort = 1;
+        break;
+      }
+      float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = xs0 + s * kTcTile + bx * kTcBox + r * 128 + ((c ^ (r & 7)) << 4);
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(addr));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+            ss2 = __ffma2_rn(f, f, ss2);
+          }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_empty[s]);
+      const float nu = sqrtf(ss2.x + ss2.y);
+      const float inv = nu > 0.f ? 1.f / nu : 0.f;
+      if (!mbar_wait(&t_full[buf], (i >> 1) & 1)) {
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t words[TF::words];
+      const uint32_t tbase = tmem + buf * kDim + (static_cast<uint32_t>(32 * q) << 16);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t y[32];
+        tmem_ld32(tbase + 32 * c, y);
+        tmem_wait_ld();
+        if (c < 2)
+          pack_chunk<TF::b0>(y, inv, pb0, words + c * TF::b0);
+        else
+          pack_chunk<TF::b1>(y, inv, pb1, words + 2 * TF::b0 + (c - 2) * TF::b1);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[buf]);
+      // outputs
+      const int64_t v = tile * kTcRows + r;
+      if (v < a.n) {
+        int64_t row = v;
+        if (a.append) {
+          int seq, head, pos;
+          row = append_row(a, v, &seq, &head, &pos);
+          if (row == -2) {
+            uint16_t* dst = a.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + v * kDim);
+#pragma unroll
+            for (int k = 0; k < kDim / 8; ++k) reinterpret_cast<uint4*>(dst)[k] = src[k];
+          }
+        }
+        if (row >= 0) {
+          if (!(nu > 0.f)) {
+#pragma unroll
+            for (int w = 0; w < TF::words; ++w) words[w] = 0u;
+          }
+          uint8_t* dst = a.codes + row * TF::bytes;
+          if constexpr (TF::bytes % 16 == 0) {
+#pragma unroll
+            for (int w = 0; w < TF::words; w += 4)
+              *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+          } else {
+#pragma unroll
+            for (int w = 0; w < TF::words; w += 2)
+              *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
+          }
+          a.norms[row] = nu;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcCols);
+  }
+  if (tid == 0 && s_abort && a.status) atomicOr(a.status, 4);
+}
+
 // Status bit 1: the append of a sequence was refused (capacity exceeded, or a
 // sequence index / stored length out of range); its length is unchanged.
 __global__ void bump_lens_kernel(const int32_t* seq_ids, int32_t* lens, int32_t* status, int n_seq,
@@ -383,7 +661,65 @@ int num_sms() {
 
 size_t quant_smem(int prod) { return sizeof(SmemQuant) + (prod ? sizeof(SmemProd) : 0); }
 
+// cuTensorMapEncodeTiled from the driver, looked up once (no link-time
+// dependency on libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+template <int B, int MIXED>
+tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<B, MIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+  if (e == cudaSuccess) {
+    quantize_tc_kernel<B, MIXED><<<grid, kTcThreads, kTcSmem, st>>>(map, a);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core quantize kernel launch");
+}
+
+// bf16 rows in MSE or mixed formats: tensor-core rotation.
+bool tc_eligible(const QuantArgs& a) {
+  return a.x_bf16 && !a.prod && a.mse_bits >= 1 && (a.mixed ? a.mse_bits == 3 : a.mse_bits <= 4) &&
+         a.n <= (int64_t(1) << 31) &&
+         (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 && encode_tiled() != nullptr;
+}
+
+tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(a.n)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTcRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode_tiled()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dims, strides,
+                                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
+  const int64_t tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  switch (a.mse_bits * 2 + a.mixed) {
+    case 2: return launch_tc<1, 0>(a, map, grid, st);
+    case 4: return launch_tc<2, 0>(a, map, grid, st);
+    case 6: return launch_tc<3, 0>(a, map, grid, st);
+    case 7: return launch_tc<3, 1>(a, map, grid, st);
+    case 8: return launch_tc<4, 0>(a, map, grid, st);
+    default: return fail(TQ_ERR_UNSUPPORTED, "tq_quantize: no tensor-core kernel for this format");
+  }
+}
+
 tq_status run_quantize(QuantArgs& a, cudaStream_t st) {
+  if (a.n <= 0) return TQ_OK;
+  if (tc_eligible(a)) return run_quantize_tc(a, st);
   const size_t smem = quant_smem(a.prod);
   const int64_t tiles = (a.n + kTile - 1) / kTile;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
@@ -404,8 +740,10 @@ void fill_format(QuantArgs& a, const tq_params* p, const FormatSpec& f) {
   a.mixed = f.mixed;
   a.prod = f.prod;
   a.code_bytes = f.code_bytes;
+  a.pi = p->pi32;
   a.pit = p->pit32;
   a.mt = p->mt32;
+  a.status = p->status32;
   a.cb = p->cb32;
   a.bd = p->bd32;
 }
@@ -449,6 +787,7 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
     a.n_sink = c->n_sink;
     a.cache_seqs = c->n_seq;
     a.sink = which ? c->v_sink : c->k_sink;
+    a.status = c->status;
     tq_status s = run_quantize(a, st);
     if (s != TQ_OK) return s;
   }
