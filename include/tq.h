@@ -133,9 +133,9 @@ tq_status tq_row_bytes(const tq_params* p, int which, int* code_bytes, int* qjl_
 /* Rotate, quantize and pack n vectors x ([n][d], fp32 or bf16, device) with
  * the K or V format of p into `out` (device planes sized for n rows).
  * Article section "Il metodo TurboQuant, in breve".  n = 0 is a no-op.
- * bf16 input in MSE or mixed formats (x 16-byte aligned) runs the rotation on
- * the tensor cores (tcgen05, Pi split into two bf16 halves, fp32
- * accumulation); fp32 input and prod formats use an fp32 SIMT kernel. */
+ * bf16 input (x 16-byte aligned) runs the rotation, and in prod formats the
+ * residual sketch, on the tensor cores (tcgen05, the matrices split into two
+ * bf16 halves, fp32 accumulation); fp32 input uses an fp32 SIMT kernel. */
 tq_status tq_quantize(const tq_params* p, const void* x, int x_dtype, int64_t n, int which,
                       const tq_packed* out, void* stream);
 

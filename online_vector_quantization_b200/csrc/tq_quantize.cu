@@ -584,6 +584,347 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   if (tid == 0 && s_abort && a.status) atomicOr(a.status, 4);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core quantize for prod formats (bf16 input): total bits = MB + 1,
+// an MB-bit MSE stage and the 1-bit QJL sketch of the residual.
+//
+// A sketch sign may differ from the exact one only where |(S r)_i| < 1e-5,
+// and a rotation error in the unit vector reaches (S r)_i amplified by the
+// norm of a row of S (about sqrt(m)), so both products run at about 24
+// significant bits:
+//   D1 = X (Pi_a + Pi_b + Pi_c)^T      rotation; x is exact in bf16, Pi is
+//                                       split into three bf16 terms
+//   D2 = 2^10 rho (M_hi + M_lo)^T      sketch, M = S Pi^T; rho = y / nu - c[idx]
+//                                       the rotated-domain residual, split
+//                                       into two fp16 terms (rho_lo M_lo dropped)
+// S r = S Pi^T rho because r = Pi^T rho, and only the sign of D2 is kept, so
+// the power-of-two scale on rho never needs undoing.  The epilogue writes the
+// rho halves into the TMEM columns of D1 it has just read, and the sketch
+// MMAs take their A operand from there.  Shared memory: Pi (96 KB), M (64 KB)
+// and one x tile per epilogue group (64 KB).
+// ---------------------------------------------------------------------------
+constexpr int kTpSmem = 3 * kTcTile + 2 * kTcTile + 2 * kTcTile + 1024;  // Pi a/b/c, M hi/lo, x x2, slack
+constexpr int kTpCols = 512;                                                // per group: D1 (128) | D2 (128)
+constexpr float kRhoScale = 1024.f;
+
+// Code and centroid of u for a width-W codebook symmetric about 0: pb = the
+// positive bounds (pb[0] = 0), pc = the positive centroids, ascending.
+template <int W>
+__device__ __forceinline__ uint32_t sym_code_c(float u, const float (&pb)[8], const float (&pc)[8], float& c) {
+  constexpr uint32_t H = 1u << (W - 1);
+  const float a = fabsf(u);
+  uint32_t j;
+  float m;
+  if constexpr (W == 1) {
+    j = 0;
+    m = pc[0];
+  } else if constexpr (W == 2) {
+    const bool c0 = a > pb[1];
+    j = c0 ? 1u : 0u;
+    m = c0 ? pc[1] : pc[0];
+  } else {
+    static_assert(W == 3, "prod MSE stages use 1..3 bits");
+    const bool c1 = a > pb[2];
+    const bool c0 = a > (c1 ? pb[3] : pb[1]);
+    j = (c1 ? 2u : 0u) + (c0 ? 1u : 0u);
+    m = c1 ? (c0 ? pc[3] : pc[2]) : (c0 ? pc[1] : pc[0]);
+  }
+  const bool pos = u > 0.f;
+  c = pos ? m : -m;
+  return pos ? H + j : H - 1u - j;
+}
+
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Swizzled K-major byte offset of element (row, k) in a 128 x 128 16-bit tile.
+__device__ __forceinline__ int sw128_off(int row, int k) {
+  return (k >> 6) * kTcBox + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2;
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                         QuantArgs a) {
+  using namespace sm100;
+  constexpr int CW = MB > 0 ? 4 * MB : 1;  // packed MSE words per row (unused for MB = 0)
+  extern __shared__ __align__(16) unsigned char smem_tp[];
+  __shared__ __align__(8) uint64_t x_full[2], x_empty[2], t1_full[2], rho_full[2], t2_full[2], t_empty[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ float s_pb[8], s_pc[8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t raw = smem_u32(smem_tp);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* basep = smem_tp + (base - raw);
+  const uint32_t pia = base, mh = base + 3 * kTcTile, xs0 = base + 5 * kTcTile;
+
+  // B operands: Pi (row j, K = input coordinate) in three bf16 terms, and
+  // M = S Pi^T (row i = sketch index, K = rotated coordinate j: M[i][j] =
+  // mt[j][i]) in two fp16 terms
+  for (int e = tid; e < kDim * kDim; e += kTcThreads) {
+    const int row = e >> 7, k = e & 127;
+    const int off = sw128_off(row, k);
+    const float p = a.pi[e];
+    const __nv_bfloat16 p0 = __float2bfloat16_rn(p);
+    const float r1 = p - __bfloat162float(p0);
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+    *reinterpret_cast<__nv_bfloat16*>(basep + off) = p0;
+    *reinterpret_cast<__nv_bfloat16*>(basep + kTcTile + off) = p1;
+    *reinterpret_cast<__nv_bfloat16*>(basep + 2 * kTcTile + off) = p2;
+    const float m = a.mt[k * kSketch + row];
+    const __half m0 = __float2half_rn(m);
+    *reinterpret_cast<__half*>(basep + 3 * kTcTile + off) = m0;
+    *reinterpret_cast<__half*>(basep + 4 * kTcTile + off) = __float2half_rn(m - __half2float(m0));
+  }
+  if constexpr (MB > 0) {
+    if (tid < 8) {
+      constexpr int half = 1 << (MB - 1);
+      s_pb[tid] = tid < half ? a.bd[MB * kBookSlots + half - 1 + tid] : 0.f;
+      s_pc[tid] = tid < half ? a.cb[MB * kBookSlots + half + tid] : 0.f;
+    }
+  }
+  if (warp == 9) {
+    tmem_alloc(&s_tmem, kTpCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&x_full[b], 1);
+      mbar_init(&x_empty[b], 1 + 4);  // the rotation MMAs' commit and the four warps reading the norm
+      mbar_init(&t1_full[b], 1);
+      mbar_init(&rho_full[b], 4);
+      mbar_init(&t2_full[b], 1);
+      mbar_init(&t_empty[b], 4);
+    }
+    s_abort = 0;
+    mbar_fence_init();
+  }
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
+
+  if (warp == 8) {
+    // ---- producer: tile i into the x stage of its epilogue group (i & 1)
+    if (lane == 0) {
+      prefetch_tensormap(&xmap);
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+        const int s = i & 1;
+        if (i >= 2 && !mbar_wait(&x_empty[s], ((i >> 1) - 1) & 1)) s_abort = 1;
+        if (s_abort) break;
+        mbar_expect_tx(&x_full[s], kTcTile);
+        tma_load_2d(xs0 + s * kTcTile, &xmap, 0, static_cast<int>(tile * kTcRows), &x_full[s]);
+        tma_load_2d(xs0 + s * kTcTile + kTcBox, &xmap, 64, static_cast<int>(tile * kTcRows), &x_full[s]);
+      }
+      for (int k = i - 2; k < i; ++k)  // loads still in flight land before the CTA may exit
+        if (k >= 0) mbar_wait(&x_full[k & 1], (k >> 1) & 1);
+    }
+  } else if (warp == 9) {
+    // ---- MMA issue: rotation of tile i, then the sketch of tile i - 1
+    if (lane == 0) {
+      constexpr uint32_t id_rot = idesc_bf16_f32(kTcRows, kDim);
+      constexpr uint32_t id_sk = idesc_f16_f32(kTcRows, kSketch);
+      auto sketch = [&](int j) {  // D2 of local tile j, A = the residual halves in D1's columns
+        const int b = j & 1;
+        if (!mbar_wait(&rho_full[b], (j >> 1) & 1)) {
+          s_abort = 1;
+          return;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + b * 256;
+        const uint32_t d = acc + 128;
+#pragma unroll
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t off = (k >> 2) * kTcBox + (k & 3) * 32;
+          const uint32_t ahi = acc + 32 * (k >> 1) + 8 * (k & 1), alo = ahi + 16;
+          const uint64_t bh = sw128_kmajor_desc(mh + off);
+          umma_f16_ts(d, ahi, bh, id_sk, k > 0);
+          umma_f16_ts(d, ahi, sw128_kmajor_desc(mh + kTcTile + off), id_sk, true);
+          umma_f16_ts(d, alo, bh, id_sk, true);
+        }
+        umma_commit(&t2_full[b]);
+      };
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+        const int b = i & 1;
+        if (!mbar_wait(&x_full[b], (i >> 1) & 1)) s_abort = 1;
+        if (i >= 2 && !s_abort && !mbar_wait(&t_empty[b], ((i >> 1) - 1) & 1)) s_abort = 1;
+        if (s_abort) break;
+        tc_fence_after();
+        const uint32_t d = tmem + b * 256;
+#pragma unroll
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t off = (k >> 2) * kTcBox + (k & 3) * 32;
+          const uint64_t ad = sw128_kmajor_desc(xs0 + b * kTcTile + off);
+          umma_bf16(d, ad, sw128_kmajor_desc(pia + off), id_rot, k > 0);
+          umma_bf16(d, ad, sw128_kmajor_desc(pia + kTcTile + off), id_rot, true);
+          umma_bf16(d, ad, sw128_kmajor_desc(pia + 2 * kTcTile + off), id_rot, true);
+        }
+        umma_commit(&x_empty[b]);
+        umma_commit(&t1_full[b]);
+        if (i >= 1) sketch(i - 1);
+        if (s_abort) break;
+      }
+      if (i >= 1 && !s_abort) sketch(i - 1);
+    }
+  } else {
+    // ---- epilogue: group g takes tiles i = g (mod 2); thread = TMEM lane = row
+    const int g = warp >> 2, q = warp & 3, r = 32 * q + lane;
+    float pb[8], pc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      pb[k] = s_pb[k];
+      pc[k] = s_pc[k];
+    }
+    const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+      if ((i & 1) != g) continue;
+      if (s_abort) break;
+      const int ph = (i >> 1) & 1;
+      const uint32_t xs = xs0 + g * kTcTile;
+      if (!mbar_wait(&x_full[g], ph)) {
+        s_abort = 1;
+        break;
+      }
+      float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = xs + bx * kTcBox + r * 128 + ((c ^ (r & 7)) << 4);
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(addr));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+            ss2 = __ffma2_rn(f, f, ss2);
+          }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_empty[g]);
+      const float nu = sqrtf(ss2.x + ss2.y);
+      const float inv = nu > 0.f ? 1.f / nu : 0.f;
+      if (!mbar_wait(&t1_full[g], ph)) {
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t words[CW];
+      float g2 = 0.f;
+      const uint32_t acc = tmem + g * 256 + lanes;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t y[32];
+        tmem_ld32(acc + 32 * c, y);
+        tmem_wait_ld();
+        if constexpr (MB > 0) {
+#pragma unroll
+          for (int w = 0; w < MB; ++w) words[c * MB + w] = 0u;
+        }
+        // residual of columns 32c..32c+31, scaled, as fp16 hi / lo pairs:
+        // hi in columns 32c..32c+15, lo in 32c+16..32c+31 (over the D1
+        // values just read)
+        uint32_t o[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float rr[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 2 * e + h;
+            const float u = __uint_as_float(y[j]) * inv;
+            if constexpr (MB > 0) {
+              float cv;
+              const uint32_t code = sym_code_c<MB>(u, pb, pc, cv);
+              const int bit = j * MB, wi = bit >> 5, sh = bit & 31;
+              words[c * MB + wi] |= code << sh;
+              if (sh + MB > 32) words[c * MB + wi + 1] |= code >> (32 - sh);
+              rr[h] = u - cv;
+            } else {
+              rr[h] = u;
+            }
+            g2 = fmaf(rr[h], rr[h], g2);
+          }
+          const float s0 = rr[0] * kRhoScale, s1 = rr[1] * kRhoScale;
+          const uint32_t hi = f16x2_bits(s0, s1);
+          const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
+          o[e] = hi;
+          o[16 + e] = f16x2_bits(s0 - __low2float(hh), s1 - __high2float(hh));
+        }
+        tmem_st32(acc + 32 * c, o);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rho_full[g]);
+      if (!mbar_wait(&t2_full[g], ph)) {
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t z[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t y[32];
+        tmem_ld32(acc + 128 + 32 * c, y);
+        tmem_wait_ld();
+        uint32_t bits = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) bits |= (__uint_as_float(y[j]) >= 0.f ? 1u : 0u) << j;
+        z[c] = bits;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[g]);
+      // outputs
+      const int64_t v = tile * kTcRows + r;
+      if (v < a.n) {
+        int64_t row = v;
+        if (a.append) {
+          int seq, head, pos;
+          row = append_row(a, v, &seq, &head, &pos);
+          if (row == -2) {
+            uint16_t* dst = a.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + v * kDim);
+#pragma unroll
+            for (int k = 0; k < kDim / 8; ++k) reinterpret_cast<uint4*>(dst)[k] = src[k];
+          }
+        }
+        if (row >= 0) {
+          const bool zero = !(nu > 0.f);
+          if constexpr (MB > 0) {
+            uint8_t* dst = a.codes + row * (16 * MB);
+#pragma unroll
+            for (int w = 0; w < CW; w += 4)
+              *reinterpret_cast<uint4*>(dst + 4 * w) =
+                  zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+          }
+          a.norms[row] = nu;
+          *reinterpret_cast<uint4*>(a.qjl + row * (kSketch / 8)) =
+              zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(z[0], z[1], z[2], z[3]);
+          a.res[row] = zero ? 0.f : sqrtf(g2);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTpCols);
+  }
+  if (tid == 0 && s_abort && a.status) atomicOr(a.status, 4);
+}
+
 // Status bit 1: the append of a sequence was refused (capacity exceeded, or a
 // sequence index / stored length out of range); its length is unchanged.
 __global__ void bump_lens_kernel(const int32_t* seq_ids, int32_t* lens, int32_t* status, int n_seq,
@@ -678,6 +1019,17 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
+template <int MB>
+tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
+  cudaError_t e =
+      cudaFuncSetAttribute(quantize_tc_prod_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTpSmem);
+  if (e == cudaSuccess) {
+    quantize_tc_prod_kernel<MB><<<grid, kTcThreads, kTpSmem, st>>>(map, a);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core prod quantize kernel launch");
+}
+
 template <int B, int MIXED>
 tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<B, MIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
@@ -688,10 +1040,11 @@ tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaSt
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core quantize kernel launch");
 }
 
-// bf16 rows in MSE or mixed formats: tensor-core rotation.
+// bf16 rows: tensor-core rotation (MSE 1..4 bits, mixed 3.5, prod 1..4).
 bool tc_eligible(const QuantArgs& a) {
-  return a.x_bf16 && !a.prod && a.mse_bits >= 1 && (a.mixed ? a.mse_bits == 3 : a.mse_bits <= 4) &&
-         a.n <= (int64_t(1) << 31) &&
+  const bool fmt_ok = a.prod ? (!a.mixed && a.mse_bits >= 0 && a.mse_bits <= 3)
+                             : (a.mse_bits >= 1 && (a.mixed ? a.mse_bits == 3 : a.mse_bits <= 4));
+  return a.x_bf16 && fmt_ok && a.n <= (int64_t(1) << 31) &&
          (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 && encode_tiled() != nullptr;
 }
 
@@ -707,6 +1060,15 @@ tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
   if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
   const int64_t tiles = (a.n + kTcRows - 1) / kTcRows;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  if (a.prod) {
+    switch (a.mse_bits) {
+      case 0: return launch_tc_prod<0>(a, map, grid, st);
+      case 1: return launch_tc_prod<1>(a, map, grid, st);
+      case 2: return launch_tc_prod<2>(a, map, grid, st);
+      case 3: return launch_tc_prod<3>(a, map, grid, st);
+      default: return fail(TQ_ERR_UNSUPPORTED, "tq_quantize: no tensor-core kernel for this format");
+    }
+  }
   switch (a.mse_bits * 2 + a.mixed) {
     case 2: return launch_tc<1, 0>(a, map, grid, st);
     case 4: return launch_tc<2, 0>(a, map, grid, st);
