@@ -282,12 +282,16 @@ def _flush_l2(torch, buf):
 
 
 def _time_call(torch, fn, iters, flush=None):
-    """Median device time (ms) of fn over iters calls, L2 flushed between calls."""
+    """Median device time (ms) of fn over iters calls, L2 flushed between calls.
+    A short device-side spin precedes the start event so that the host's
+    launch overhead for fn is hidden behind queued GPU work and the interval
+    measures fn's kernels only."""
     stream = torch.cuda.current_stream()
     times = []
     for _ in range(iters):
         if flush is not None:
             _flush_l2(torch, flush)
+        torch.cuda._sleep(200_000)  # ~0.1 ms of SM clocks
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -297,17 +301,36 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-def run_aux(tq, torch, kv_inputs, device, args):
-    """The other workloads, measured on the same GPU in the same run."""
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny")
+
+
+def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
+    """The other workloads, measured on the same GPU in the same run.  `only`
+    restricts the run to one of AUX_WORKLOADS and `formats` the quantize sweep
+    to some of mse1..4, prod1..4 (both for profiling one kernel)."""
     out = {}
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MB > L2
     iters = 10
+    if only in (None, "quantize-sweep"):
+        out["quantize_sweep_1M_bf16"] = _aux_sweep(tq, torch, kv_inputs, device, flush, iters, formats)
+    if only in (None, "prod3-gqa"):
+        out["decode_prod3_gqa_T32k"] = _aux_prod3(tq, torch, kv_inputs, device, flush, iters)
+    if only in (None, "k4v3-sink"):
+        out.update(_aux_k4v3(tq, torch, kv_inputs, device, flush, iters))
+    if only in (None, "tiny"):
+        out["decode_tiny_fp32_T4096"] = _aux_tiny(tq, torch, kv_inputs, device, iters)
+    return out
+
+
+def _aux_sweep(tq, torch, kv_inputs, device, flush, iters, formats):
     # quantize sweep: 32 kv-heads x 32768 tokens, bf16 with 4 outlier channels
     n = 32 * 32768
     x = kv_inputs.kv_vectors(n, D, key="sweep", device=device, dtype=torch.bfloat16, outliers=True)
     sweep = {}
     for mode, name in ((tq.TQ_MODE_MSE, "mse"), (tq.TQ_MODE_PROD, "prod")):
         for b in (1, 2, 3, 4):
+            if formats and f"{name}{b}" not in formats:
+                continue
             p = tq.Params(b, b, mode, mode)
             pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
             ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
@@ -315,8 +338,10 @@ def run_aux(tq, torch, kv_inputs, device, args):
             by = n * (D * 2 + cb + 4 + (qb + 4 if qb else 0))
             sweep[f"{name}{b}"] = {"mvec_per_s": round(n / (ms * 1e-3) / 1e6, 1), "ms": round(ms, 4),
                                    "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1)}
-    out["quantize_sweep_1M_bf16"] = sweep
-    del x
+    return sweep
+
+
+def _aux_prod3(tq, torch, kv_inputs, device, flush, iters):
     # GQA decode, prod mode: B=1, 32 q / 8 kv heads, T=32768, K/V 3-bit (2-bit MSE + QJL)
     T = 32768
     p = tq.Params(3, 3, tq.TQ_MODE_PROD, tq.TQ_MODE_PROD)
@@ -329,10 +354,13 @@ def run_aux(tq, torch, kv_inputs, device, args):
     o = torch.empty(1, 32, D, dtype=torch.bfloat16, device=device)
     ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, T, o, ws), iters, flush)
     by = 8 * T * 2 * (32 + 16 + 8)
-    out["decode_prod3_gqa_T32k"] = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1),
-                                    "bytes": by, "l2": "flushed between calls"}
-    del cache, k, v
+    return {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
+            "l2": "flushed between calls"}
+
+
+def _aux_k4v3(tq, torch, kv_inputs, device, flush, iters):
     # long-context asymmetric: B=4, 64 q / 8 kv, T=131072, sink 128 bf16, K4/V3, sparse V 1e-6
+    out = {}
     T = 131072
     p = tq.Params(4, 3)
     cache = tq.Cache(p, 4, 8, T - 128, 128, device=device)
@@ -359,7 +387,10 @@ def run_aux(tq, torch, kv_inputs, device, args):
         out[f"decode_k4v3_sink_T128k_{name}"] = {"ms": round(ms, 4), "gb_per_s_dense_equiv": round(by / (ms * 1e-3) / 1e9, 1),
                                                  "dense_bytes": by}
     assert int(cache.status.item()) == 0
-    del cache
+    return out
+
+
+def _aux_tiny(tq, torch, kv_inputs, device, iters):
     # tiny fp32 case: 4096 vectors, b=3, 1 head
     p = tq.Params(3, 3)
     x = kv_inputs.kv_vectors(4096, D, key="c1", device=device)
@@ -369,8 +400,21 @@ def run_aux(tq, torch, kv_inputs, device, args):
     ws = tq.decode_workspace(p, 1, 1, 1, 4096, device=device)
     o = torch.empty(1, 1, D, dtype=torch.float32, device=device)
     ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, 4096, o, ws), iters)
-    out["decode_tiny_fp32_T4096"] = {"ms": round(ms, 4)}
-    return out
+    return {"ms": round(ms, 4)}
+
+
+def run_aux_only(args):
+    """One auxiliary workload alone (for profiling a kernel): prints its JSON."""
+    import torch
+
+    import kv_inputs
+    import online_vector_quantization_b200 as tq
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    formats = set(args.formats.split(",")) if args.formats else None
+    out = run_aux(tq, torch, kv_inputs, device, args, only=args.aux_only, formats=formats)
+    print(json.dumps({"aux_only": args.aux_only, "aux": out}), flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -478,10 +522,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-units", type=int, default=2)
     ap.add_argument("--traffic", type=float, default=None, help=argparse.SUPPRESS)
+    ap.add_argument("--aux-only", choices=AUX_WORKLOADS, default=None,
+                    help="run one auxiliary workload alone and print its numbers (profiling)")
+    ap.add_argument("--formats", default=None, help="with --aux-only quantize-sweep: e.g. mse3,prod3")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.aux_only:
+        run_aux_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

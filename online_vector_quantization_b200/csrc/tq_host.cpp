@@ -2,6 +2,8 @@
 // Lloyd-Max codebooks), parameter objects, argument checking and the C ABI
 // entry points.  Device work is enqueued by the launchers in the .cu files.
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -274,6 +276,52 @@ tq_status tq_qjl_matrix(uint64_t seed, int m, int d, double* s) {
   return TQ_OK;
 }
 
+// The tensor-core quantize kernels take Pi (rotation) and M = S Pi^T (QJL
+// sketch of the rotated residual) as B operands: row n = output index, K =
+// input index, 16-bit values in the layout a TMA copy with 128-byte swizzle
+// produces (two 64-column boxes of 128 rows x 128 B; the 16-byte chunk c of
+// row r sits at chunk c ^ (r & 7)).  Pi is split into bf16 terms (two for
+// the MSE kernels, three for the prod kernels) and M into two fp16 terms, each
+// term rounding what the previous ones left of the fp64 value.
+static size_t sw128_offset(int row, int k) {
+  return static_cast<size_t>((k >> 6) * 16384 + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2);
+}
+
+static std::vector<uint8_t> tensor_core_images(const std::vector<double>& pi, const std::vector<double>& m_rowmajor) {
+  std::vector<uint8_t> img(static_cast<size_t>(kTcImgCount) * kTcImgBytes, 0);
+  auto put = [&](int which, int row, int k, uint16_t bits) {
+    std::memcpy(img.data() + static_cast<size_t>(which) * kTcImgBytes + sw128_offset(row, k), &bits, 2);
+  };
+  auto bf = [](double v, double* back) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(static_cast<float>(v));
+    *back = static_cast<double>(__bfloat162float(h));
+    uint16_t b;
+    std::memcpy(&b, &h, 2);
+    return b;
+  };
+  auto hf = [](double v, double* back) {
+    const __half h = __float2half_rn(static_cast<float>(v));
+    *back = static_cast<double>(__half2float(h));
+    uint16_t b;
+    std::memcpy(&b, &h, 2);
+    return b;
+  };
+  for (int row = 0; row < kDim; ++row)
+    for (int k = 0; k < kDim; ++k) {
+      const double p = pi[static_cast<size_t>(row) * kDim + k];
+      double h0, h1, h2;
+      put(kTcImgPiHi, row, k, bf(p, &h0));
+      put(kTcImgPiLo, row, k, bf(p - h0, &h1));
+      put(kTcImgPiA, row, k, bf(p, &h0));
+      put(kTcImgPiB, row, k, bf(p - h0, &h1));
+      put(kTcImgPiC, row, k, bf(p - h0 - h1, &h2));
+      const double mv = m_rowmajor[static_cast<size_t>(row) * kDim + k];
+      put(kTcImgMHi, row, k, hf(mv, &h0));
+      put(kTcImgMLo, row, k, hf(mv - h0, &h1));
+    }
+  return img;
+}
+
 tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   if (!cfg || !out) return fail(TQ_ERR_ARG, "tq_params_create: NULL argument");
   *out = nullptr;
@@ -311,11 +359,13 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
       st32[j * m + i] = static_cast<float>(p->s[i * d + j]);
     }
   // M = S Pi^T (fp64): (S r) = M (Pi r) for a residual r given in the rotated domain
+  std::vector<double> mt64(static_cast<size_t>(m) * d);  // M row-major [i][j]
   for (int i = 0; i < m; ++i)
     for (int j = 0; j < d; ++j) {
       double acc = 0.0;
       for (int k = 0; k < d; ++k) acc += p->s[i * d + k] * p->pi[j * d + k];
       mt32[j * m + i] = static_cast<float>(acc);
+      mt64[i * d + j] = acc;
     }
   for (int b = 1; b <= kMaxBits; ++b) {
     bool used = false;
@@ -341,7 +391,7 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
          o_st = take(st32.size() * 4), o_mt = take(mt32.size() * 4), o_pi64 = take(p->pi.size() * 8),
          o_s64 = take(p->s.size() * 8), o_cb = take(cb32.size() * 4), o_bd = take(bd32.size() * 4),
          o_cb64 = take(cb64.size() * 8), o_cbs = take(cbs32.size() * 4), o_sig = take(sig32.size() * 4),
-         o_status = take(sizeof(int32_t));
+         o_status = take(sizeof(int32_t)), o_img = take(static_cast<size_t>(kTcImgCount) * kTcImgBytes);
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->block, off);
   if (e != cudaSuccess) {
@@ -363,6 +413,8 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   p->cbs32 = reinterpret_cast<float*>(base + o_cbs);
   p->sig32 = reinterpret_cast<float*>(base + o_sig);
   p->status32 = reinterpret_cast<int32_t*>(base + o_status);
+  p->tc_img = reinterpret_cast<uint8_t*>(base + o_img);
+  const std::vector<uint8_t> img = tensor_core_images(p->pi, mt64);
   e = cudaMemset(p->status32, 0, sizeof(int32_t));
   if (e != cudaSuccess) {
     cudaFree(p->block);
@@ -375,7 +427,8 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
       {p->mt32, mt32.data(), mt32.size() * 4},   {p->pi64, p->pi.data(), p->pi.size() * 8},
       {p->s64, p->s.data(), p->s.size() * 8},    {p->cb32, cb32.data(), cb32.size() * 4},
       {p->bd32, bd32.data(), bd32.size() * 4},   {p->cb64, cb64.data(), cb64.size() * 8},
-      {p->cbs32, cbs32.data(), cbs32.size() * 4}, {p->sig32, sig32.data(), sig32.size() * 4}};
+      {p->cbs32, cbs32.data(), cbs32.size() * 4}, {p->sig32, sig32.data(), sig32.size() * 4},
+      {p->tc_img, img.data(), img.size()}};
   for (auto& c : copies) {
     e = cudaMemcpy(c.dst, c.src, c.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {

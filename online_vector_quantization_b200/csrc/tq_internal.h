@@ -55,7 +55,16 @@ struct tq_params {
   float* bd32 = nullptr;   // decision bounds [kMaxBits+1][16]
   double* cb64 = nullptr;  // centroids fp64 [kMaxBits+1][16]
   int32_t* status32 = nullptr;  // device word that plain quantize kernels OR error bits into
+  // Tensor-core B operands of the quantize kernels, each a 128 x 128 16-bit
+  // tile in the 128-byte-swizzled K-major layout (32 KB; see kTcImg*)
+  uint8_t* tc_img = nullptr;
 };
+
+namespace tq {
+constexpr int kTcImgBytes = 128 * 128 * 2;
+// images in tq_params::tc_img, in this order
+enum { kTcImgPiHi = 0, kTcImgPiLo, kTcImgPiA, kTcImgPiB, kTcImgPiC, kTcImgMHi, kTcImgMLo, kTcImgCount };
+}  // namespace tq
 
 namespace tq {
 

@@ -50,6 +50,7 @@ struct QuantArgs {
   int n_tok, hkv, capacity, n_sink, cache_seqs;
   uint16_t* sink;  // bf16 [n_seq][hkv][n_sink][d]
   int32_t* status;  // device word; bit 4 = a pipeline wait timed out
+  const uint8_t* tc_img;  // tensor-core B operand images (tq_params::tc_img)
 };
 
 struct SmemQuant {
@@ -391,27 +392,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   using namespace sm100;
   using TF = TcFormat<B, MIXED>;
   extern __shared__ __align__(16) unsigned char smem_tc[];
-  __shared__ __align__(8) uint64_t x_full[kTcStages], x_empty[kTcStages], t_full[2], t_empty[2];
+  __shared__ __align__(8) uint64_t x_full[kTcStages], x_empty[kTcStages], t_full[2], t_empty[2], b_full;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ float s_pb[2][8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t raw = smem_u32(smem_tc);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* basep = smem_tc + (base - raw);
   const uint32_t pih = base, pil = base + kTcTile, xs0 = base + 2 * kTcTile;
 
-  // Pi as the K-major B operand (row j = output coordinate, K = input
-  // coordinate), hi and lo bf16 halves, in the swizzled layout
-  for (int i = tid; i < kDim * kDim; i += kTcThreads) {
-    const int j = i >> 7, k = i & 127;
-    const float p = a.pi[i];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-    const int off = (k >> 6) * kTcBox + j * 128 + ((((k & 63) >> 3) ^ (j & 7)) << 4) + (k & 7) * 2;
-    *reinterpret_cast<__nv_bfloat16*>(basep + off) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(basep + kTcTile + off) = lo;
-  }
+  // Pi (row j = output coordinate, K = input coordinate) as bf16 hi and lo
+  // halves arrives by bulk copy from the prepared images
   if (tid < 16) {
     const int seg = tid >> 3, i = tid & 7;
     const int w = seg ? TF::b1 : TF::b0;
@@ -431,10 +422,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 4);
     }
+    mbar_init(&b_full, 1);
     s_abort = 0;
     mbar_fence_init();
   }
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // B tiles visible to the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -442,9 +433,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
 
   if (warp == 8) {
-    // ---- producer
+    // ---- producer: the B operand once, then the x tiles
     if (lane == 0) {
       prefetch_tensormap(&xmap);
+      mbar_expect_tx(&b_full, 2 * kTcTile);
+      bulk_g2s_addr(pih, a.tc_img + kTcImgPiHi * kTcImgBytes, kTcTile, &b_full);
+      bulk_g2s_addr(pil, a.tc_img + kTcImgPiLo * kTcImgBytes, kTcTile, &b_full);
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
         const int s = i % kTcStages;
@@ -457,11 +451,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
       // loads still in flight land before the CTA may exit
       for (int k = i - kTcStages; k < i; ++k)
         if (k >= 0) mbar_wait(&x_full[k % kTcStages], (k / kTcStages) & 1);
+      mbar_wait(&b_full, 0);
     }
   } else if (warp == 9) {
     // ---- MMA issue
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTcRows, kDim);
+      if (!mbar_wait(&b_full, 0)) s_abort = 1;
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
         const int s = i % kTcStages, buf = i & 1;
@@ -639,46 +635,24 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Swizzled K-major byte offset of element (row, k) in a 128 x 128 16-bit tile.
-__device__ __forceinline__ int sw128_off(int row, int k) {
-  return (k >> 6) * kTcBox + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2;
-}
-
 template <int MB>
 __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                          QuantArgs a) {
   using namespace sm100;
   constexpr int CW = MB > 0 ? 4 * MB : 1;  // packed MSE words per row (unused for MB = 0)
   extern __shared__ __align__(16) unsigned char smem_tp[];
-  __shared__ __align__(8) uint64_t x_full[2], x_empty[2], t1_full[2], rho_full[2], t2_full[2], t_empty[2];
+  __shared__ __align__(8) uint64_t x_full[2], x_empty[2], t1_full[2], rho_full[2], t2_full[2], t_empty[2], b_full;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ float s_pb[8], s_pc[8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t raw = smem_u32(smem_tp);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* basep = smem_tp + (base - raw);
   const uint32_t pia = base, mh = base + 3 * kTcTile, xs0 = base + 5 * kTcTile;
 
-  // B operands: Pi (row j, K = input coordinate) in three bf16 terms, and
-  // M = S Pi^T (row i = sketch index, K = rotated coordinate j: M[i][j] =
-  // mt[j][i]) in two fp16 terms
-  for (int e = tid; e < kDim * kDim; e += kTcThreads) {
-    const int row = e >> 7, k = e & 127;
-    const int off = sw128_off(row, k);
-    const float p = a.pi[e];
-    const __nv_bfloat16 p0 = __float2bfloat16_rn(p);
-    const float r1 = p - __bfloat162float(p0);
-    const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
-    *reinterpret_cast<__nv_bfloat16*>(basep + off) = p0;
-    *reinterpret_cast<__nv_bfloat16*>(basep + kTcTile + off) = p1;
-    *reinterpret_cast<__nv_bfloat16*>(basep + 2 * kTcTile + off) = p2;
-    const float m = a.mt[k * kSketch + row];
-    const __half m0 = __float2half_rn(m);
-    *reinterpret_cast<__half*>(basep + 3 * kTcTile + off) = m0;
-    *reinterpret_cast<__half*>(basep + 4 * kTcTile + off) = __float2half_rn(m - __half2float(m0));
-  }
+  // B operands by bulk copy from the prepared images: Pi (row j, K = input
+  // coordinate) in three bf16 terms, M = S Pi^T (row i = sketch index, K =
+  // rotated coordinate) in two fp16 terms
   if constexpr (MB > 0) {
     if (tid < 8) {
       constexpr int half = 1 << (MB - 1);
@@ -699,10 +673,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
       mbar_init(&t2_full[b], 1);
       mbar_init(&t_empty[b], 4);
     }
+    mbar_init(&b_full, 1);
     s_abort = 0;
     mbar_fence_init();
   }
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -710,9 +684,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
   const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
 
   if (warp == 8) {
-    // ---- producer: tile i into the x stage of its epilogue group (i & 1)
+    // ---- producer: the B operands once, then tile i into the x stage of its
+    // epilogue group (i & 1)
     if (lane == 0) {
       prefetch_tensormap(&xmap);
+      mbar_expect_tx(&b_full, 5 * kTcTile);
+      for (int k = 0; k < 3; ++k)
+        bulk_g2s_addr(pia + k * kTcTile, a.tc_img + (kTcImgPiA + k) * kTcImgBytes, kTcTile, &b_full);
+      for (int k = 0; k < 2; ++k)
+        bulk_g2s_addr(mh + k * kTcTile, a.tc_img + (kTcImgMHi + k) * kTcImgBytes, kTcTile, &b_full);
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
         const int s = i & 1;
@@ -724,12 +704,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
       }
       for (int k = i - 2; k < i; ++k)  // loads still in flight land before the CTA may exit
         if (k >= 0) mbar_wait(&x_full[k & 1], (k >> 1) & 1);
+      mbar_wait(&b_full, 0);
     }
   } else if (warp == 9) {
     // ---- MMA issue: rotation of tile i, then the sketch of tile i - 1
     if (lane == 0) {
       constexpr uint32_t id_rot = idesc_bf16_f32(kTcRows, kDim);
       constexpr uint32_t id_sk = idesc_f16_f32(kTcRows, kSketch);
+      if (!mbar_wait(&b_full, 0)) s_abort = 1;
       auto sketch = [&](int j) {  // D2 of local tile j, A = the residual halves in D1's columns
         const int b = j & 1;
         if (!mbar_wait(&rho_full[b], (j >> 1) & 1)) {
@@ -1106,6 +1088,7 @@ void fill_format(QuantArgs& a, const tq_params* p, const FormatSpec& f) {
   a.pit = p->pit32;
   a.mt = p->mt32;
   a.status = p->status32;
+  a.tc_img = p->tc_img;
   a.cb = p->cb32;
   a.bd = p->bd32;
 }
