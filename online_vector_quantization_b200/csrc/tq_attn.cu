@@ -40,8 +40,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 constexpr int kTok = 16;       // tokens per warp tile
 constexpr int kMaxG = 8;       // query heads per kv-head (MMA N = 8)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -383,6 +381,7 @@ struct DecodeArgs {
   int B, hkv, group, hq, capacity, n_sink, max_len, part_floats;
   int ctas;   // CTAs of the decode grid (pieces a unit can be cut into)
   int chunk;  // quantized tokens per scheduled chunk
+  int merge_chunk;  // pieces the merge kernel stages in shared memory at a time
   float* parts;
   const uint32_t* qfrag;
   void* out;
@@ -421,77 +420,88 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\
 //    Pi q for all heads (one output coordinate each), threads 128..255 form
 //    S q (prod keys); then the fp16 B-fragments are written.
 // ---------------------------------------------------------------------------
+constexpr int kQrotThreads = 512;
+constexpr int kQrotSplit = kQrotThreads / kDim;  // slices of the k range per output coordinate
+
 template <int KF>
-__global__ void __launch_bounds__(kThreads) qrot_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
   using KR = KRow<KF>;
   using FK = Fmt<KF>;
   extern __shared__ float4 s_mat4[];              // Pi^T [k][j], then S^T [k][j] (prod keys)
   __shared__ __align__(16) float qsT[kDim][kMaxG];  // query, [k][head]
   __shared__ float qt[kMaxG][kDim];
   __shared__ float qsk[kMaxG][kSketch];
+  __shared__ float s_p[kQrotSplit][kMaxG][kDim];  // partial sums over k slices
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = a.group;
   pdl_launch();  // the decode kernel's prologue and cache stream may start
   {
     // stage the matrices with asynchronous 16-byte copies, all in flight
-    constexpr int N4 = kDim * kDim / 4 / kThreads;
+    constexpr int N4 = kDim * kDim / 4 / kQrotThreads;
     const float4* pit4 = reinterpret_cast<const float4*>(a.pit);
 #pragma unroll
-    for (int i = 0; i < N4; ++i) cp_async16(smem_u32(s_mat4 + i * kThreads + tid), pit4 + i * kThreads + tid);
+    for (int i = 0; i < N4; ++i)
+      cp_async16(smem_u32(s_mat4 + i * kQrotThreads + tid), pit4 + i * kQrotThreads + tid);
     if constexpr (FK::prod) {
       const float4* st4 = reinterpret_cast<const float4*>(a.st);
 #pragma unroll
       for (int i = 0; i < N4; ++i)
-        cp_async16(smem_u32(s_mat4 + kDim * kDim / 4 + i * kThreads + tid), st4 + i * kThreads + tid);
+        cp_async16(smem_u32(s_mat4 + kDim * kDim / 4 + i * kQrotThreads + tid), st4 + i * kQrotThreads + tid);
     }
   }
-  for (int i = tid; i < kMaxG * kDim; i += kThreads) {
+  for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
     const int h = i % kMaxG, d = i / kMaxG;
     qsT[d][h] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
   }
   cp_async_wait_all();
   __syncthreads();
   const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
-  {
-    const int j = tid & (kDim - 1);
-    const bool sketch = tid >= kDim;
-    if (!sketch || FK::prod) {
-      const float* mat = reinterpret_cast<const float*>(s_mat4) + (sketch ? kDim * kDim : 0);
-      const float4* q4 = reinterpret_cast<const float4*>(&qsT[0][0]);
-      float acc[kMaxG];
+  // thread (j, ks) sums k in [ks * 32, ks * 32 + 32) for output coordinate j
+  // of every head; the slices are added in shared memory
+  const int j = tid & (kDim - 1), ks = tid >> 7;
+  const float4* q4 = reinterpret_cast<const float4*>(&qsT[0][0]);
+  for (int mtx = 0; mtx < (FK::prod ? 2 : 1); ++mtx) {
+    const float* mat = reinterpret_cast<const float*>(s_mat4) + mtx * kDim * kDim;
+    float acc[kMaxG];
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+    for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
 #pragma unroll 8
-      for (int k = 0; k < kDim; ++k) {
-        const float m = mat[k * kDim + j];
-        const float4 x0 = q4[2 * k], x1 = q4[2 * k + 1];
-        acc[0] = fmaf(m, x0.x, acc[0]);
-        acc[1] = fmaf(m, x0.y, acc[1]);
-        acc[2] = fmaf(m, x0.z, acc[2]);
-        acc[3] = fmaf(m, x0.w, acc[3]);
-        acc[4] = fmaf(m, x1.x, acc[4]);
-        acc[5] = fmaf(m, x1.y, acc[5]);
-        acc[6] = fmaf(m, x1.z, acc[6]);
-        acc[7] = fmaf(m, x1.w, acc[7]);
-      }
-      if (sketch) {
+    for (int kk = 0; kk < kDim / kQrotSplit; ++kk) {
+      const int k = ks * (kDim / kQrotSplit) + kk;
+      const float m = mat[k * kDim + j];
+      const float4 x0 = q4[2 * k], x1 = q4[2 * k + 1];
+      acc[0] = fmaf(m, x0.x, acc[0]);
+      acc[1] = fmaf(m, x0.y, acc[1]);
+      acc[2] = fmaf(m, x0.z, acc[2]);
+      acc[3] = fmaf(m, x0.w, acc[3]);
+      acc[4] = fmaf(m, x1.x, acc[4]);
+      acc[5] = fmaf(m, x1.y, acc[5]);
+      acc[6] = fmaf(m, x1.z, acc[6]);
+      acc[7] = fmaf(m, x1.w, acc[7]);
+    }
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) qsk[h][j] = acc[h] * scale;
+    for (int h = 0; h < kMaxG; ++h) s_p[ks][h][j] = acc[h];
+    __syncthreads();
+    for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
+      const int h = i / kDim, jj = i % kDim;
+      float v = 0.f;
+#pragma unroll
+      for (int s = 0; s < kQrotSplit; ++s) v += s_p[s][h][jj];
+      if (mtx == 1) {
+        qsk[h][jj] = v * scale;
       } else {
-        const int wj = FK::width(j);
-        const float f = wj > 0 ? scale / a.sig[wj] : 0.f;
-#pragma unroll
-        for (int h = 0; h < kMaxG; ++h) qt[h][j] = acc[h] * f;
+        const int wj = FK::width(jj);
+        qt[h][jj] = wj > 0 ? v * (scale / a.sig[wj]) : 0.f;
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
   // B fragments: lane (g, t) supplies column g; k-steps 0..7 from the MSE
   // segments, 8..15 from the QJL segment.  Unpacked: column g = head g, halves
   // hi (x = 0) and lo (x = 1).  Packed (group <= 4): column g < 4 = hi of head
   // g, column g >= 4 = lo of head g - 4, in x = 0.
   uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  for (int i = tid; i < 16 * 32; i += kThreads) {
+  for (int i = tid; i < 16 * 32; i += kQrotThreads) {
     const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
     int dims[4] = {0, 0, 0, 0};
     bool valid = true;
@@ -894,7 +904,9 @@ __device__ __forceinline__ void consumers_sync() {
 }
 
 
-// Partial slot: per head of the unit's group, [max, sum, accumulator].
+// Partial slot: per head of the unit's group, [max, sum, 2 unused, accumulator]
+// (kPartAcc floats before the accumulator keep every row 16-byte aligned).
+constexpr int kPartAcc = 4;
 __device__ __forceinline__ float* part_slot(const DecodeArgs& a, int64_t slot) {
   return a.parts + slot * a.group * a.part_floats;
 }
@@ -971,7 +983,7 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
           l += wl[w * kMaxG + h] * f;
         }
       }
-      dst[h * PF + 2 + lo + j] = s;
+      dst[h * PF + kPartAcc + lo + j] = s;
       if (pass == 0 && j == 0) {
         dst[h * PF + 0] = M;
         dst[h * PF + 1] = l;
@@ -1005,10 +1017,17 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Merge shared memory beyond the static arrays: sink weights [n_sink][8] and
-// piece weights [ctas][8].
-inline size_t merge_dyn_bytes(int n_sink, int ctas) {
-  return (static_cast<size_t>(n_sink) + ctas) * kMaxG * sizeof(float);
+// Merge shared memory beyond the static arrays: sink weights [n_sink][8],
+// piece maxima / weights and sums [ctas][8] each, and a staging buffer of
+// merge_chunk pieces (G x part_floats floats each).
+constexpr size_t kMergeStageBytes = 128 * 1024;
+inline int merge_chunk_pieces(int group, int part_floats) {
+  const size_t per = static_cast<size_t>(group) * part_floats * sizeof(float);
+  return static_cast<int>(std::max<size_t>(1, kMergeStageBytes / per));
+}
+inline size_t merge_dyn_bytes(int n_sink, int ctas, int group, int part_floats) {
+  return (static_cast<size_t>(n_sink) + 2 * static_cast<size_t>(ctas)) * kMaxG * sizeof(float) +
+         static_cast<size_t>(merge_chunk_pieces(group, part_floats)) * group * part_floats * sizeof(float);
 }
 
 template <int VF>
@@ -1026,7 +1045,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   __shared__ float s_ms[kMaxG], s_ls[kMaxG], s_M[kMaxG], s_L[kMaxG];
   __shared__ long long s_C, s_cu0;
   float* s_sc = reinterpret_cast<float*>(s_dyn4);  // [n_sink][8]
-  float* s_f = s_sc + a.n_sink * kMaxG;             // [pieces][8]
+  float* s_f = s_sc + a.n_sink * kMaxG;             // [pieces][8]: maxima, then weights
+  float* s_l = s_f + a.ctas * kMaxG;                // [pieces][8]: sums
+  float* s_part = s_l + a.ctas * kMaxG;             // staged pieces [merge_chunk][G][part_floats]
   const int u = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.group, P = a.ctas, CH = a.chunk, PF = a.part_floats;
@@ -1146,20 +1167,29 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     first = cta_of_chunk(cu0, C, P);
     n_p = cta_of_chunk(cu0 + ui.chunks - 1, C, P) - first + 1;
   }
-  if (warp < G) {  // warp h: the pieces' maxima, weights and sums for head h
+  // the maxima and sums of all pieces, gathered at once
+  for (int e = tid; e < n_p * G; e += NT) {
+    const int i = e / G, h = e % G;
+    float m = -INFINITY, l = 0.f;
+    if (cta_has_chunks(first + i, C, P)) {
+      const float* pp = part_slot(a, u + first + i) + h * PF;
+      m = __ldcg(pp);
+      l = __ldcg(pp + 1);
+    }
+    s_f[i * kMaxG + h] = m;
+    s_l[i * kMaxG + h] = l;
+  }
+  __syncthreads();
+  if (warp < G) {  // warp h: merged maximum, the pieces' weights and the sum for head h
     const int h = warp;
     float M = s_ms[h];
-    for (int i = lane; i < n_p; i += 32) {
-      const float m = cta_has_chunks(first + i, C, P) ? __ldcg(part_slot(a, u + first + i) + h * PF) : -INFINITY;
-      s_f[i * kMaxG + h] = m;
-      M = fmaxf(M, m);
-    }
+    for (int i = lane; i < n_p; i += 32) M = fmaxf(M, s_f[i * kMaxG + h]);
     M = warp_max(M);
     float L = 0.f;
     for (int i = lane; i < n_p; i += 32) {
       const float m = s_f[i * kMaxG + h];
       const float f = m > -INFINITY ? exp2f(m - M) : 0.f;
-      if (f != 0.f) L = fmaf(__ldcg(part_slot(a, u + first + i) + h * PF + 1), f, L);
+      L = fmaf(s_l[i * kMaxG + h], f, L);
       s_f[i * kMaxG + h] = f;
     }
     L = warp_sum(L);
@@ -1172,19 +1202,31 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   __syncthreads();
   if (has_pieces) {
     {
+      // the accumulators: consecutive slots, staged chunk by chunk with
+      // 16-byte asynchronous copies
       const int j = tid % WD, sl = tid / WD;
       float acc[kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
-      for (int i = sl; i < n_p; i += NS) {
-        const float* pp = part_slot(a, u + first + i) + 2 + j;
+      const int slot_floats = G * PF;
+      for (int c0 = 0; c0 < n_p; c0 += a.merge_chunk) {
+        const int cnt = min(a.merge_chunk, n_p - c0);
+        const float4* src = reinterpret_cast<const float4*>(part_slot(a, u + first + c0));
+        const int n16 = cnt * slot_floats / 4;
+        for (int e = tid; e < n16; e += NT) cp_async16(smem_u32(s_part) + 16 * e, src + e);
+        cp_async_wait_all();
+        __syncthreads();
+        for (int i = sl; i < cnt; i += NS) {
+          const float* pp = s_part + i * slot_floats + kPartAcc + j;
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
-          if (h < G) {
-            const float f = s_f[i * kMaxG + h];
-            if (f != 0.f) acc[h] = fmaf(__ldcg(pp + h * PF), f, acc[h]);
+          for (int h = 0; h < kMaxG; ++h) {
+            // weight 0: a piece of a CTA with an empty range, whose slot was
+            // not written in this call
+            const float f = h < G ? s_f[(c0 + i) * kMaxG + h] : 0.f;
+            if (f != 0.f) acc[h] = fmaf(pp[h * PF], f, acc[h]);
           }
         }
+        __syncthreads();  // the staging buffer is refilled
       }
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) s_red[(sl * kMaxG + h) * WD + j] = acc[h];
@@ -1522,12 +1564,12 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
   e = cudaFuncSetAttribute(qrot_kernel<KF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(qrot_smem));
   if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
-  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kThreads, qrot_smem, st>>>(a);
+  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kQrotThreads, qrot_smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas);
+  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, plan.group, plan.part_floats);
   if (merge_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(merge_kernel<VF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(merge_smem));
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
@@ -1561,7 +1603,7 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) 
   pl.group = hq / hkv;
   pl.max_len = max_len;
   pl.ctas = num_sms_cached() < kMaxPieces ? num_sms_cached() : kMaxPieces;
-  pl.part_floats = 2 + (p->fv.prod ? 2 * kDim : kDim);
+  pl.part_floats = kPartAcc + (p->fv.prod ? 2 * kDim : kDim);
   const size_t units = static_cast<size_t>(B) * hkv;
   const size_t qfrag = (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
   // piece (u, cta) uses slot u + cta: fewer than units + ctas slots
@@ -1596,6 +1638,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.max_len = plan.max_len;
   a.part_floats = plan.part_floats;
   a.ctas = plan.ctas;
+  a.merge_chunk = merge_chunk_pieces(plan.group, plan.part_floats);
   if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 4096");
   const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
   char* w = static_cast<char*>(ws);
