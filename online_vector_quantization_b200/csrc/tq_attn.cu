@@ -617,11 +617,42 @@ struct WarpState {
 template <bool PACK>
 using QFrag = uint32_t[8][2][PACK ? 1 : 2];
 
+// Token order inside a 16-token subtile.  MMA row / column k of a subtile
+// holds physical token pi[k] (K and V use the same order, so the scores,
+// softmax weights and V columns line up).  The order only changes which
+// shared-memory banks the code loads hit: lane (g, t) reads K rows pi[g],
+// pi[g + 8] and V rows pi[2t], pi[2t + 1], pi[2t + 8], pi[2t + 9], and rows of
+// 24..64 bytes make some orders collide less.  pi[k] is nibble k of the word;
+// the words come from a search over a model of these loads (bank_perm.py next
+// to this file), identity where no order helps.
+__host__ __device__ constexpr uint64_t token_order(int kf, int vf) {
+  return kf == 2 && vf == 2     ? 0xFE095427B86D1AC3ull
+         : kf == 4 && vf == 4   ? 0xB2CD41F863905AE7ull
+         : kf == 11 && vf == 11 ? 0x2AE619D534F8BC70ull
+         : kf == 18 && vf == 18 ? 0xB6C51FA82907D43Eull
+         : kf == 4 && vf == 2   ? 0xB856274109A3DEFCull
+         : kf == 3 && vf == 2   ? 0xC1B7502E948F3D6Aull
+                                : 0xFEDCBA9876543210ull;
+}
+
+// This lane's physical rows within a subtile: K rows (score rows g, g + 8)
+// and V rows (MMA columns 2t, 2t + 1, 2t + 8, 2t + 9).
+struct TokRows {
+  int kA, kB, v0, v1, v8, v9;
+};
+template <int KF, int VF>
+__device__ __forceinline__ TokRows tok_rows(int g, int t) {
+  constexpr uint64_t pi = token_order(KF, VF);
+  auto at = [](int k) { return static_cast<int>((pi >> (4 * k)) & 15u); };
+  return TokRows{at(g), at(g + 8), at(2 * t), at(2 * t + 1), at(2 * t + 8), at(2 * t + 9)};
+}
+
 // Scores of one 16-token subtile whose rows start at `srow` of the staged
 // planes: s2 (base 2) for tokens g (s2[0], s2[1]) and g+8 (s2[2], s2[3]),
 // columns 2t, 2t+1; masked tokens get -inf.  Two MMA accumulator chains.
 template <int KF, bool PACK>
-__device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, bool okA, bool okB, int g, int t,
+__device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
+                                               int g, int t,
                                                const QFrag<PACK>& bq, const QFrag<PACK>& bqs,
                                                uint32_t lut_a, uint32_t lut_b,
                                                uint32_t lane4, uint32_t lane8, uint32_t c1k, float (&s2)[4]) {
@@ -629,7 +660,7 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, bo
   using KR = KRow<KF>;
   constexpr int NX = PACK ? 1 : 2;
   const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
-  const int rA = srow + g, rB = srow + g + 8;
+  const int rA = srow + tr.kA, rB = srow + tr.kB;
   const uint32_t ka = u.kcodes + rA * FK::code_bytes;
   const uint32_t kb = u.kcodes + rB * FK::code_bytes;
   float ca[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -711,21 +742,22 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, bo
 // O^T += C_v^T P'^T for one 16-token subtile (rows from `srow`); p holds the
 // softmax weights of tokens g (p[0], p[1]) and g+8 (p[2], p[3]).
 template <int VF, int VMT>
-__device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, bool okA, bool okB, int g, int t,
+__device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
+                                           int g, int t,
                                            const float (&p)[4], uint32_t lut_a,
                                            uint32_t lut_b, uint32_t lane4, uint32_t lane8, uint32_t c1v,
                                            float (&oacc)[VMT][4]) {
   using FV = Fmt<VF>;
   using VR = VRow<VF>;
   const uint32_t one2 = 0x3C003C00u;
-  const float wA = okA ? ldsf(u.vnorm, (srow + g) * 4) : 0.f, wB = okB ? ldsf(u.vnorm, (srow + g + 8) * 4) : 0.f;
+  const float wA = okA ? ldsf(u.vnorm, (srow + tr.kA) * 4) : 0.f, wB = okB ? ldsf(u.vnorm, (srow + tr.kB) * 4) : 0.f;
   const uint32_t pb0 = movmatrix_t(h2bits(p[0] * wA, p[1] * wA));
   const uint32_t pb1 = movmatrix_t(h2bits(p[2] * wB, p[3] * wB));
-  const int v0 = srow + 2 * t;  // tokens v0, v0+1, v0+8, v0+9
-  const uint32_t r0p = u.vcodes + v0 * FV::code_bytes;
-  const uint32_t r1p = r0p + FV::code_bytes;
-  const uint32_t r8p = r0p + 8 * FV::code_bytes;
-  const uint32_t r9p = r0p + 9 * FV::code_bytes;
+  // rows of MMA columns 2t, 2t+1, 2t+8, 2t+9
+  const uint32_t r0p = u.vcodes + (srow + tr.v0) * FV::code_bytes;
+  const uint32_t r1p = u.vcodes + (srow + tr.v1) * FV::code_bytes;
+  const uint32_t r8p = u.vcodes + (srow + tr.v8) * FV::code_bytes;
+  const uint32_t r9p = u.vcodes + (srow + tr.v9) * FV::code_bytes;
   if constexpr (FV::nseg > 0) {
     constexpr int MT = VR::S0::MT;
     typename VR::S0 xa, xb, xc, xd;
@@ -754,14 +786,15 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, bool o
     for (int mt = 0; mt < MT; ++mt) mma16816(oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
   }
   if constexpr (FV::prod) {
-    const float uA = okA ? wA * ldsf(u.vres, (srow + g) * 4) : 0.f, uB = okB ? wB * ldsf(u.vres, (srow + g + 8) * 4) : 0.f;
+    const float uA = okA ? wA * ldsf(u.vres, (srow + tr.kA) * 4) : 0.f,
+                uB = okB ? wB * ldsf(u.vres, (srow + tr.kB) * 4) : 0.f;
     const uint32_t qb0 = movmatrix_t(h2bits(p[0] * uA, p[1] * uA));
     const uint32_t qb1 = movmatrix_t(h2bits(p[2] * uB, p[3] * uB));
     typename VR::Q xa, xb, xc, xd;
-    xa.load(u.vq + v0 * (kSketch / 8), g);
-    xb.load(u.vq + (v0 + 1) * (kSketch / 8), g);
-    xc.load(u.vq + (v0 + 8) * (kSketch / 8), g);
-    xd.load(u.vq + (v0 + 9) * (kSketch / 8), g);
+    xa.load(u.vq + (srow + tr.v0) * (kSketch / 8), g);
+    xb.load(u.vq + (srow + tr.v1) * (kSketch / 8), g);
+    xc.load(u.vq + (srow + tr.v8) * (kSketch / 8), g);
+    xd.load(u.vq + (srow + tr.v9) * (kSketch / 8), g);
     uint32_t r0[8], r08[8], r1[8], r18[8];
     VR::Q::decode(xa, xb, lut_a, lane4, lane8, one2, r0, r08);
     VR::Q::decode(xc, xd, lut_a, lane4, lane8, one2, r1, r18);
@@ -784,56 +817,96 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
                                              uint32_t c1k, uint32_t c1v, float thr) {
   constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
   constexpr bool second = WT == 2 * kTok;
-  const bool ok0A = row0 + g < nq, ok0B = row0 + g + 8 < nq;
-  const bool ok1A = row0 + kTok + g < nq, ok1B = row0 + kTok + g + 8 < nq;
+  const TokRows tr = tok_rows<KF, VF>(g, t);
+  const bool ok0A = row0 + tr.kA < nq, ok0B = row0 + tr.kB < nq;
+  const bool ok1A = row0 + kTok + tr.kA < nq, ok1B = row0 + kTok + tr.kB < nq;
   float s0[4], s1[4];
-  subtile_scores<KF, PACK>(u, srow, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
+  subtile_scores<KF, PACK>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
   if constexpr (second)
-    subtile_scores<KF, PACK>(u, srow + kTok, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
+    subtile_scores<KF, PACK>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
   // online softmax over the 32 tokens (base 2), columns 2t and 2t+1
-  float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
-  float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-  }
-  const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
-  const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
   float p0[4], p1[4];
-  p0[0] = fast_exp2(s0[0] - mn0);
-  p0[1] = fast_exp2(s0[1] - mn1);
-  p0[2] = fast_exp2(s0[2] - mn0);
-  p0[3] = fast_exp2(s0[3] - mn1);
-  p1[0] = fast_exp2(s1[0] - mn0);
-  p1[1] = fast_exp2(s1[1] - mn1);
-  p1[2] = fast_exp2(s1[2] - mn0);
-  p1[3] = fast_exp2(s1[3] - mn1);
-  float rs0 = (p0[0] + p0[2]) + (p1[0] + p1[2]), rs1 = (p0[1] + p0[3]) + (p1[1] + p1[3]);
+  if constexpr (!SPARSE) {
+    // Dense: the running maximum moves only when some lane sees a larger
+    // score (rare after the first tiles), and each lane keeps its own partial
+    // sum (the eight lanes of a column are added when the piece is written),
+    // so most tiles take no cross-lane step.
+    float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
+    float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
+    if (__any_sync(0xffffffffu, (mx0 > W.m0) | (mx1 > W.m1))) {
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
-    rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
-  }
-  W.l0 = fmaf(W.l0, al0, rs0);
-  W.l1 = fmaf(W.l1, al1, rs1);
-  W.m0 = mn0;
-  W.m1 = mn1;
-  if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
+      const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
+      W.l0 *= al0;
+      W.l1 *= al1;
 #pragma unroll
-    for (int i = 0; i < VMT; ++i) {
-      W.oacc[i][0] *= al0;
-      W.oacc[i][1] *= al1;
-      W.oacc[i][2] *= al0;
-      W.oacc[i][3] *= al1;
+      for (int i = 0; i < VMT; ++i) {
+        W.oacc[i][0] *= al0;
+        W.oacc[i][1] *= al1;
+        W.oacc[i][2] *= al0;
+        W.oacc[i][3] *= al1;
+      }
+      W.m0 = mn0;
+      W.m1 = mn1;
+    }
+    p0[0] = fast_exp2(s0[0] - W.m0);
+    p0[1] = fast_exp2(s0[1] - W.m1);
+    p0[2] = fast_exp2(s0[2] - W.m0);
+    p0[3] = fast_exp2(s0[3] - W.m1);
+    p1[0] = fast_exp2(s1[0] - W.m0);
+    p1[1] = fast_exp2(s1[1] - W.m1);
+    p1[2] = fast_exp2(s1[2] - W.m0);
+    p1[3] = fast_exp2(s1[3] - W.m1);
+    W.l0 += (p0[0] + p0[2]) + (p1[0] + p1[2]);
+    W.l1 += (p0[1] + p0[3]) + (p1[1] + p1[3]);
+  } else {
+    float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
+    float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
+    const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
+    p0[0] = fast_exp2(s0[0] - mn0);
+    p0[1] = fast_exp2(s0[1] - mn1);
+    p0[2] = fast_exp2(s0[2] - mn0);
+    p0[3] = fast_exp2(s0[3] - mn1);
+    p1[0] = fast_exp2(s1[0] - mn0);
+    p1[1] = fast_exp2(s1[1] - mn1);
+    p1[2] = fast_exp2(s1[2] - mn0);
+    p1[3] = fast_exp2(s1[3] - mn1);
+    float rs0 = (p0[0] + p0[2]) + (p1[0] + p1[2]), rs1 = (p0[1] + p0[3]) + (p1[1] + p1[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
+      rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
+    }
+    W.l0 = fmaf(W.l0, al0, rs0);
+    W.l1 = fmaf(W.l1, al1, rs1);
+    W.m0 = mn0;
+    W.m1 = mn1;
+    if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
+#pragma unroll
+      for (int i = 0; i < VMT; ++i) {
+        W.oacc[i][0] *= al0;
+        W.oacc[i][1] *= al1;
+        W.oacc[i][2] *= al0;
+        W.oacc[i][3] *= al1;
+      }
     }
   }
   if constexpr (!SPARSE) {
-    subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+    subtile_pv<VF, VMT>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if constexpr (second)
-      subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   } else {
     // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
     const float c0 = thr * W.l0, c1 = thr * W.l1;
@@ -845,9 +918,9 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
       p1[i + 1] = p1[i + 1] >= c1 ? p1[i + 1] : 0.f;
     }
     if (__any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f))
-      subtile_pv<VF, VMT>(u, srow, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if (second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f))
-      subtile_pv<VF, VMT>(u, srow + kTok, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   }
 }
 
@@ -919,8 +992,9 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t i, float 
 }
 
 // Cross-warp combine of one piece into partial slot `slot`, in 64-coordinate
-// slices of the accumulator (consumer threads).
-template <int KF, int VF, bool PACK>
+// slices of the accumulator (consumer threads).  LANE_SUMS: each lane holds
+// its own partial softmax sums (dense path), added over the column first.
+template <int KF, int VF, bool PACK, bool LANE_SUMS>
 __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& W, int64_t slot, float* sm,
                             int warp, int g, int t) {
   using FV = Fmt<VF>;
@@ -934,11 +1008,19 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
   float* wacc = wl + kConsumers * kMaxG;   // [warp][head][kSliceDims]
   float* dst = part_slot(a, slot);
   const int PF = a.part_floats;
+  float l0 = W.l0, l1 = W.l1;
+  if constexpr (LANE_SUMS) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+  }
   if (g == 0) {
     wm[warp * kMaxG + 2 * t] = W.m0;
     wm[warp * kMaxG + 2 * t + 1] = W.m1;
-    wl[warp * kMaxG + 2 * t] = W.l0;
-    wl[warp * kMaxG + 2 * t + 1] = W.l1;
+    wl[warp * kMaxG + 2 * t] = l0;
+    wl[warp * kMaxG + 2 * t + 1] = l1;
   }
 #pragma unroll 1
   for (int pass = 0; pass < WD / kSliceDims; ++pass) {
@@ -1413,15 +1495,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     if (lane == 0 && c0 < c1) {
       int u = s_u0, lc = s_lc0;
       UnitInfo ui = unit_info(a, u, CH);
-      long long k = 0;
-      for (long long c = c0; c < c1; ++c, ++k) {
+      const int nk = static_cast<int>(c1 - c0);
+      int s = 0;
+      uint32_t round = 0;  // parity of k / S
+      for (int k = 0; k < nk; ++k) {
         while (lc >= ui.chunks) {
           ++u;
           lc = 0;
           ui = unit_info(a, u, CH);
         }
-        const int s = static_cast<int>(k % S);
-        if (k >= S && !mbar_wait(&empty_bar[s], static_cast<uint32_t>((k / S - 1) & 1))) s_abort = 1;
+        if (k >= S && !mbar_wait(&empty_bar[s], round ^ 1u)) s_abort = 1;
         if (s_abort) break;
         const int64_t ubase = static_cast<int64_t>(u) * a.capacity;
         const int r0 = lc * CH;
@@ -1443,6 +1526,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
           bulk_g2s_addr(st + SL::vr, a.v_res + row, rows * 4, bar);
         }
         ++lc;
+        if (++s == S) {
+          s = 0;
+          round ^= 1u;
+        }
       }
     }
     return;
@@ -1464,34 +1551,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   UnitInfo ui{};
   int walk_u = s_u0, walk_lc = s_lc0;
   UnitInfo wui = c0 < c1 ? unit_info(a, walk_u, CH) : UnitInfo{};
-  long long k = 0;
-  for (long long c = c0; c < c1; ++c, ++k) {
+  const int nk = static_cast<int>(c1 - c0);
+  int s = 0;
+  uint32_t round = 0;  // parity of k / S
+  for (int k = 0; k < nk; ++k) {
     while (walk_lc >= wui.chunks) {
       ++walk_u;
       walk_lc = 0;
       wui = unit_info(a, walk_u, CH);
     }
     if (walk_u != u) {
-      if (u >= 0) write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
+      if (u >= 0) write_piece<KF, VF, PACK, !SPARSE>(a, wst, u + cta, scratch, warp, g, t);
       u = walk_u;
       ui = wui;
       const uint32_t* qf = a.qfrag + static_cast<int64_t>(u) * kQfragWords;
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
+      for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
           for (int x = 0; x < NX; ++x) {
-            bq[s][r][x] = qf[((s * 2 + r) * 2 + x) * 32 + lane];
-            if constexpr (FK::prod) bqs[s][r][x] = qf[(((8 + s) * 2 + r) * 2 + x) * 32 + lane];
+            bq[ks][r][x] = qf[((ks * 2 + r) * 2 + x) * 32 + lane];
+            if constexpr (FK::prod) bqs[ks][r][x] = qf[(((8 + ks) * 2 + r) * 2 + x) * 32 + lane];
           }
 #pragma unroll
       for (int i = 0; i < WarpState<KF, VF, PACK>::VMT; ++i) wst.oacc[i][0] = wst.oacc[i][1] = wst.oacc[i][2] = wst.oacc[i][3] = 0.f;
       wst.m0 = wst.m1 = -INFINITY;
       wst.l0 = wst.l1 = 0.f;
     }
-    const int s = static_cast<int>(k % S);
-    if (!s_abort && !mbar_wait(&full_bar[s], static_cast<uint32_t>((k / S) & 1))) s_abort = 1;
+    if (!s_abort && !mbar_wait(&full_bar[s], round)) s_abort = 1;
     const int row0 = walk_lc * CH + warp * WT;
     if (!s_abort && row0 < ui.nq) {
       const uint32_t st = stage_addr(s);
@@ -1510,8 +1598,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
     ++walk_lc;
+    if (++s == S) {
+      s = 0;
+      round ^= 1u;
+    }
   }
-  if (u >= 0) write_piece<KF, VF, PACK>(a, wst, u + cta, scratch, warp, g, t);
+  if (u >= 0) write_piece<KF, VF, PACK, !SPARSE>(a, wst, u + cta, scratch, warp, g, t);
   if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
 
