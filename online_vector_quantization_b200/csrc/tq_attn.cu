@@ -132,6 +132,20 @@ __device__ __forceinline__ uint4 lds128(uint32_t base, uint32_t off) {
   return v;
 }
 __device__ __forceinline__ float ldsf(uint32_t base, uint32_t off) { return __uint_as_float(lds32(base, off)); }
+// Lookup-table reads: the tables are written once before the main loop and
+// only read after it, so these loads are pure functions of their address and
+// the compiler may schedule them freely (the stage reads above stay ordered
+// by the pipeline's barriers).
+__device__ __forceinline__ uint32_t lut32(uint32_t base, uint32_t off) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(base + off));
+  return v;
+}
+__device__ __forceinline__ uint2 lut64(uint32_t base, uint32_t off) {
+  uint2 v;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(base + off));
+  return v;
+}
 
 // byte k of w placed at bits 8..15; bits 0..7 and 16..31 from lb (the lane
 // offset and the table base; lb's bits 8..15 are zero)
@@ -234,13 +248,13 @@ struct KChunk {
     constexpr int s = S;
     if constexpr (B == 4) {
       const uint32_t ww = w[s >> 1];
-      lo = lds32(smem, byte_addr(ww, lane4, 2 * (s & 1)));
-      hi = lds32(smem, byte_addr(ww, lane4, 2 * (s & 1) + 1));
+      lo = lut32(smem, byte_addr(ww, lane4, 2 * (s & 1)));
+      hi = lut32(smem, byte_addr(ww, lane4, 2 * (s & 1) + 1));
     } else if constexpr (B == 3) {
-      lo = lds32(smem, pair3<2 * S>(lane4 + 128));
-      hi = lds32(smem, pair3<2 * S + 1>(lane4 + 128));
+      lo = lut32(smem, pair3<2 * S>(lane4 + 128));
+      hi = lut32(smem, pair3<2 * S + 1>(lane4 + 128));
     } else if constexpr (B == 2) {
-      const uint2 v = lds64(smem, byte_addr(w[s >> 2], lane8, s & 3));
+      const uint2 v = lut64(smem, byte_addr(w[s >> 2], lane8, s & 3));
       lo = v.x;
       hi = v.y;
     } else {
@@ -302,8 +316,8 @@ struct VChunk {
         const uint32_t od = ((xa >> 4) & 0x0F0F0F0Fu) | (xb & 0xF0F0F0F0u);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          rg[4 * wd + k] = lds32(smem, byte_addr(ev, lane4, k));
-          rg8[4 * wd + k] = lds32(smem, byte_addr(od, lane4, k));
+          rg[4 * wd + k] = lut32(smem, byte_addr(ev, lane4, k));
+          rg8[4 * wd + k] = lut32(smem, byte_addr(od, lane4, k));
         }
       }
     } else if constexpr (B == 3) {
@@ -318,8 +332,8 @@ struct VChunk {
         const uint32_t od = ((xa >> 3) & E) | (xb & ~E);
         static_for<4>([&](auto kk) {
           constexpr int k = decltype(kk)::value;
-          rg[4 * h + k] = lds32(smem, addr6<6 * k>(ev, lb));
-          rg8[4 * h + k] = lds32(smem, addr6<6 * k>(od, lb));
+          rg[4 * h + k] = lut32(smem, addr6<6 * k>(ev, lb));
+          rg8[4 * h + k] = lut32(smem, addr6<6 * k>(od, lb));
         });
       });
     } else if constexpr (B == 2) {
@@ -328,8 +342,8 @@ struct VChunk {
       const uint32_t od = ((xa >> 2) & 0x33333333u) | (xb & 0xCCCCCCCCu);
 #pragma unroll
       for (int j = 0; j < MT / 2; ++j) {
-        const uint2 e = lds64(smem, byte_addr(ev, lane8, j));
-        const uint2 o = lds64(smem, byte_addr(od, lane8, j));
+        const uint2 e = lut64(smem, byte_addr(ev, lane8, j));
+        const uint2 o = lut64(smem, byte_addr(od, lane8, j));
         rg[2 * j] = e.x;
         rg[2 * j + 1] = e.y;
         rg8[2 * j] = o.x;
@@ -810,14 +824,13 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
 // lets their lookup and MMA chains interleave).  SPARSE: skip the PV MMAs of
 // a subtile whose weights are all below the sparse-V threshold.
 template <int KF, int VF, bool PACK, int WT, bool SPARSE>
-__device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int row0, int nq,
+__device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int row0, int nq, const TokRows& tr,
                                              WarpState<KF, VF, PACK>& W, const QFrag<PACK>& bq,
                                              const QFrag<PACK>& bqs, int g, int t, uint32_t lut_a,
                                              uint32_t lut_b, uint32_t lane4, uint32_t lane8,
                                              uint32_t c1k, uint32_t c1v, float thr) {
   constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
   constexpr bool second = WT == 2 * kTok;
-  const TokRows tr = tok_rows<KF, VF>(g, t);
   const bool ok0A = row0 + tr.kA < nq, ok0B = row0 + tr.kB < nq;
   const bool ok1A = row0 + kTok + tr.kA < nq, ok1B = row0 + kTok + tr.kB < nq;
   float s0[4], s1[4];
@@ -1542,6 +1555,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const float thr = a.sparse_thr;
+  const TokRows trows = tok_rows<KF, VF>(g, t);
 
   pdl_wait();  // the rotated query fragments
 
@@ -1592,7 +1606,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       sp.kres = st + SL::kr;
       sp.vq = st + SL::vq;
       sp.vres = st + SL::vr;
-      compute_tile<KF, VF, PACK, WT, SPARSE>(sp, warp * WT, row0, ui.nq, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
+      compute_tile<KF, VF, PACK, WT, SPARSE>(sp, warp * WT, row0, ui.nq, trows, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
                                  c1k, c1v, thr);
     }
     __syncwarp();
