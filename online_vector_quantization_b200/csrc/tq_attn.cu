@@ -1136,7 +1136,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   __shared__ float s_red[4 * kMaxG * kDim];       // slice partials
   __shared__ __align__(16) float s_acc[WD][kMaxG];  // merged accumulator, [j][head]
   __shared__ float s_osk[kMaxG][kDim];            // sink values, original domain
-  __shared__ float s_q[kMaxG][kDim];
+  __shared__ float s_q[kMaxG][4][33];  // query quarters, padded: the four quarters sit in different banks
   __shared__ float s_ms[kMaxG], s_ls[kMaxG], s_M[kMaxG], s_L[kMaxG];
   __shared__ long long s_C, s_cu0;
   float* s_sc = reinterpret_cast<float*>(s_dyn4);  // [n_sink][8]
@@ -1184,35 +1184,70 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   }
   // sink: scores with the original query, softmax weights, weighted values
   if (ui.ns > 0) {
-    for (int i = tid; i < kMaxG * kDim; i += NT) (&s_q[0][0])[i] = i < G * kDim ? load_q(a.q, a.q_bf16, orow + i) : 0.f;
+    for (int i = tid; i < kMaxG * kDim; i += NT)
+      s_q[i / kDim][(i % kDim) >> 5][i & 31] = i < G * kDim ? load_q(a.q, a.q_bf16, orow + i) : 0.f;
     __syncthreads();
-    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
-    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim;
+    // sink rows are staged through shared memory (the piece staging buffer,
+    // not yet in use) in chunks of up to SC tokens with 16-byte asynchronous
+    // copies, so each chunk costs one memory round trip
+    const char* ks = reinterpret_cast<const char*>(a.k_sink) + static_cast<int64_t>(u) * a.n_sink * kDim * 2;
+    const char* vs = reinterpret_cast<const char*>(a.v_sink) + static_cast<int64_t>(u) * a.n_sink * kDim * 2;
+    const __nv_bfloat16* srow = reinterpret_cast<const __nv_bfloat16*>(s_part);
+    const int SC = a.merge_chunk * G * PF * 4 / (kDim * 2);  // rows that fit the staging buffer
     const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
-    for (int t = warp; t < ui.ns; t += NT / 32) {
-      const __nv_bfloat16* kr = ks + static_cast<int64_t>(t) * kDim + 4 * lane;
-      float k4[4];
+    auto stage_rows = [&](const char* src, int c0, int cnt) {
+      const float4* s4 = reinterpret_cast<const float4*>(src + static_cast<int64_t>(c0) * kDim * 2);
+      for (int e = tid; e < cnt * kDim * 2 / 16; e += NT) cp_async16(smem_u32(s_part) + 16 * e, s4 + e);
+      cp_async_wait_all();
+      __syncthreads();
+    };
+    for (int c0 = 0; c0 < ui.ns; c0 += SC) {
+      const int cnt = min(SC, ui.ns - c0);
+      stage_rows(ks, c0, cnt);
+      // thread (token, quarter): dot products over 32 coordinates for every
+      // head, then added across the four quarters (adjacent lanes)
+      for (int tb = 0; tb < cnt; tb += NT / 4) {
+        const int tt = tb + (tid >> 2), qtr = tid & 3;
+        float d[kMaxG];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) k4[e] = __bfloat162float(kr[e]);
-      for (int h = 0; h < G; ++h) {
-        float d = 0.f;
+        for (int h = 0; h < kMaxG; ++h) d[h] = 0.f;
+        if (tt < cnt) {
+          const uint4* kr = reinterpret_cast<const uint4*>(srow + tt * kDim + 32 * qtr);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d = fmaf(k4[e], s_q[h][4 * lane + e], d);
-        d = warp_sum(d);
-        if (lane == 0) s_sc[t * kMaxG + h] = d * scale;
+          for (int c = 0; c < 4; ++c) {
+            const uint4 kw = kr[c];
+            const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float k0 = __uint_as_float(w4[e] << 16), k1 = __uint_as_float(w4[e] & 0xFFFF0000u);
+              const int j = 8 * c + 2 * e;
+#pragma unroll
+              for (int h = 0; h < kMaxG; ++h) d[h] = fmaf(k1, s_q[h][qtr][j + 1], fmaf(k0, s_q[h][qtr][j], d[h]));
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          d[h] += __shfl_xor_sync(0xffffffffu, d[h], 1);
+          d[h] += __shfl_xor_sync(0xffffffffu, d[h], 2);
+        }
+        if (tt < cnt && qtr == 0)
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h)
+            if (h < G) s_sc[(c0 + tt) * kMaxG + h] = d[h] * scale;
       }
+      __syncthreads();  // the staging buffer is refilled
     }
-    __syncthreads();
     if (warp < G) {  // warp h: max, weights and sum of head h
       const int h = warp;
       float mx = -INFINITY;
-      for (int t = lane; t < ui.ns; t += 32) mx = fmaxf(mx, s_sc[t * kMaxG + h]);
+      for (int tt = lane; tt < ui.ns; tt += 32) mx = fmaxf(mx, s_sc[tt * kMaxG + h]);
       mx = warp_max(mx);
       float sum = 0.f;
-      for (int t = lane; t < ui.ns; t += 32) {
-        const float p = exp2f(s_sc[t * kMaxG + h] - mx);
-        s_sc[t * kMaxG + h] = p;
-        sum += p;
+      for (int tt = lane; tt < ui.ns; tt += 32) {
+        const float pw = exp2f(s_sc[tt * kMaxG + h] - mx);
+        s_sc[tt * kMaxG + h] = pw;
+        sum += pw;
       }
       sum = warp_sum(sum);
       if (lane == 0) {
@@ -1225,17 +1260,22 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       float acc[kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
-      for (int t = sl4; t < ui.ns; t += 4) {
-        const float v = __bfloat162float(vs[static_cast<int64_t>(t) * kDim + o]);
-        const float4 p0 = s_dyn4[t * 2], p1 = s_dyn4[t * 2 + 1];
-        acc[0] = fmaf(p0.x, v, acc[0]);
-        acc[1] = fmaf(p0.y, v, acc[1]);
-        acc[2] = fmaf(p0.z, v, acc[2]);
-        acc[3] = fmaf(p0.w, v, acc[3]);
-        acc[4] = fmaf(p1.x, v, acc[4]);
-        acc[5] = fmaf(p1.y, v, acc[5]);
-        acc[6] = fmaf(p1.z, v, acc[6]);
-        acc[7] = fmaf(p1.w, v, acc[7]);
+      for (int c0 = 0; c0 < ui.ns; c0 += SC) {
+        const int cnt = min(SC, ui.ns - c0);
+        stage_rows(vs, c0, cnt);
+        for (int tt = sl4; tt < cnt; tt += 4) {
+          const float v = __bfloat162float(srow[tt * kDim + o]);
+          const float4 p0 = s_dyn4[(c0 + tt) * 2], p1 = s_dyn4[(c0 + tt) * 2 + 1];
+          acc[0] = fmaf(p0.x, v, acc[0]);
+          acc[1] = fmaf(p0.y, v, acc[1]);
+          acc[2] = fmaf(p0.z, v, acc[2]);
+          acc[3] = fmaf(p0.w, v, acc[3]);
+          acc[4] = fmaf(p1.x, v, acc[4]);
+          acc[5] = fmaf(p1.y, v, acc[5]);
+          acc[6] = fmaf(p1.z, v, acc[6]);
+          acc[7] = fmaf(p1.w, v, acc[7]);
+        }
+        __syncthreads();  // the staging buffer is refilled
       }
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) s_red[(sl4 * kMaxG + h) * kDim + o] = acc[h];
