@@ -839,13 +839,13 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
     subtile_scores<KF, PACK>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
-  // online softmax over the 32 tokens (base 2), columns 2t and 2t+1
+  // online softmax over the 32 tokens (base 2), columns 2t and 2t+1.  The
+  // running maximum moves only when some lane sees a larger score (rare
+  // after the first tiles), and each lane keeps its own partial sum (the
+  // eight lanes of a column are added when the piece is written), so most
+  // tiles take no cross-lane step.
   float p0[4], p1[4];
-  if constexpr (!SPARSE) {
-    // Dense: the running maximum moves only when some lane sees a larger
-    // score (rare after the first tiles), and each lane keeps its own partial
-    // sum (the eight lanes of a column are added when the piece is written),
-    // so most tiles take no cross-lane step.
+  {
     float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
     float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
     if (__any_sync(0xffffffffu, (mx0 > W.m0) | (mx1 > W.m1))) {
@@ -878,50 +878,15 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
     p1[3] = fast_exp2(s1[3] - W.m1);
     W.l0 += (p0[0] + p0[2]) + (p1[0] + p1[2]);
     W.l1 += (p0[1] + p0[3]) + (p1[1] + p1[3]);
-  } else {
-    float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
-    float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    const float mn0 = fmaxf(W.m0, mx0), mn1 = fmaxf(W.m1, mx1);
-    const float al0 = fast_exp2(W.m0 - mn0), al1 = fast_exp2(W.m1 - mn1);
-    p0[0] = fast_exp2(s0[0] - mn0);
-    p0[1] = fast_exp2(s0[1] - mn1);
-    p0[2] = fast_exp2(s0[2] - mn0);
-    p0[3] = fast_exp2(s0[3] - mn1);
-    p1[0] = fast_exp2(s1[0] - mn0);
-    p1[1] = fast_exp2(s1[1] - mn1);
-    p1[2] = fast_exp2(s1[2] - mn0);
-    p1[3] = fast_exp2(s1[3] - mn1);
-    float rs0 = (p0[0] + p0[2]) + (p1[0] + p1[2]), rs1 = (p0[1] + p0[3]) + (p1[1] + p1[3]);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      rs0 += __shfl_xor_sync(0xffffffffu, rs0, off);
-      rs1 += __shfl_xor_sync(0xffffffffu, rs1, off);
-    }
-    W.l0 = fmaf(W.l0, al0, rs0);
-    W.l1 = fmaf(W.l1, al1, rs1);
-    W.m0 = mn0;
-    W.m1 = mn1;
-    if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
-#pragma unroll
-      for (int i = 0; i < VMT; ++i) {
-        W.oacc[i][0] *= al0;
-        W.oacc[i][1] *= al1;
-        W.oacc[i][2] *= al0;
-        W.oacc[i][3] *= al1;
-      }
-    }
   }
   if constexpr (!SPARSE) {
     subtile_pv<VF, VMT>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if constexpr (second)
       subtile_pv<VF, VMT>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   } else {
-    // sparse V: exp(s - m)/l over the tokens seen so far bounds the final weight
+    // sparse V: exp(s - m) / l over the tokens seen so far bounds the final
+    // weight, and this lane's partial sum is at most l, so p < thr * l_lane
+    // only skips tokens whose final weight is below thr
     const float c0 = thr * W.l0, c1 = thr * W.l1;
 #pragma unroll
     for (int i = 0; i < 4; i += 2) {
@@ -1615,7 +1580,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       wui = unit_info(a, walk_u, CH);
     }
     if (walk_u != u) {
-      if (u >= 0) write_piece<KF, VF, PACK, !SPARSE>(a, wst, u + cta, scratch, warp, g, t);
+      if (u >= 0) write_piece<KF, VF, PACK, true>(a, wst, u + cta, scratch, warp, g, t);
       u = walk_u;
       ui = wui;
       const uint32_t* qf = a.qfrag + static_cast<int64_t>(u) * kQfragWords;
@@ -1657,7 +1622,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       round ^= 1u;
     }
   }
-  if (u >= 0) write_piece<KF, VF, PACK, !SPARSE>(a, wst, u + cta, scratch, warp, g, t);
+  if (u >= 0) write_piece<KF, VF, PACK, true>(a, wst, u + cta, scratch, warp, g, t);
   if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
 
