@@ -72,15 +72,19 @@ struct Fmt {
 
 // Shared-memory lookup tables.  Region A (row stride 256 B): bytes [0,128) of
 // row r hold, for each lane, half2(c4[r & 15], c4[r >> 4]); bytes [128, 256)
-// of rows r < 64 hold half2(c3[r & 7], c3[r >> 3]).  Region B (row stride
-// 256 B, 8 B per lane): four 2-bit centroids of byte r.  Entry (r, lane) sits
-// at r*256 + lane*4 (or *8): every lane hits its own bank.
+// of rows r < 64 hold half2(c3[r & 7], c3[r >> 3]) -- and, when region A spans
+// all 256 rows anyway (t3_wide), every row r holds the entry of r & 63, so a
+// 3-bit pair in the low six bits of any byte is looked up with one byte
+// permute.  Region B (row stride 256 B, 8 B per lane): four 2-bit centroids of
+// byte r.  Entry (r, lane) sits at r*256 + lane*4 (or *8): every lane hits its
+// own bank.
 template <int KF, int VF>
 struct Lut {
   static constexpr bool t4 = Fmt<KF>::uses(4) || Fmt<VF>::uses(4);
   static constexpr bool t3 = Fmt<KF>::uses(3) || Fmt<VF>::uses(3);
   static constexpr bool t2 = Fmt<KF>::uses(2) || Fmt<VF>::uses(2);
   static constexpr int region_a = (t4 || (t3 && t2)) ? 65536 : (t3 ? 16384 : 0);
+  static constexpr bool t3_wide = t3 && region_a == 65536;
   static constexpr int region_b_off = region_a;  // 0 or 65536: a 64 KB boundary
   static constexpr int bytes = region_a + (t2 ? 65536 : 0);
 };
@@ -241,12 +245,23 @@ struct KChunk {
     }
   }
 
-  // k-step S: (lo, hi) = A-fragment registers for k = 2t..2t+1 and 2t+8..2t+9
-  template <int S>
+  // k-step S: (lo, hi) = A-fragment registers for k = 2t..2t+1 and 2t+8..2t+9.
+  // T3W (3-bit): the pair table spans 256 rows, so the pair at bit 12S (6,
+  // 30: after a 6-bit shift; 12, 36 / 18, 42: after 12 / 18) is the low six
+  // bits of byte 0 or 3 of w[0] or of a funnel shift of (w[0], w[1]).
+  template <int S, bool T3W = false>
   __device__ __forceinline__ void decode(uint32_t smem, uint32_t lane4, uint32_t lane8,
                                          uint32_t c_bits, uint32_t& lo, uint32_t& hi) const {
     constexpr int s = S;
-    if constexpr (B == 4) {
+    if constexpr (B == 3 && T3W && ND == 64) {
+      const uint32_t lb = lane4 + 128;
+      const uint32_t w1 = w[WORDS > 1 ? 1 : 0];
+      constexpr int kb = S >= 2 ? 3 : 0;  // byte of the low field
+      const uint32_t src_lo = (S & 1) ? __funnelshift_r(w[0], w1, 12) : w[0];
+      const uint32_t src_hi = (S & 1) ? __funnelshift_r(w[0], w1, 18) : __funnelshift_r(w[0], w1, 6);
+      lo = lut32(smem, byte_addr(src_lo, lb, kb));
+      hi = lut32(smem, byte_addr(src_hi, lb, kb));
+    } else if constexpr (B == 4) {
       const uint32_t ww = w[s >> 1];
       lo = lut32(smem, byte_addr(ww, lane4, 2 * (s & 1)));
       hi = lut32(smem, byte_addr(ww, lane4, 2 * (s & 1) + 1));
@@ -664,7 +679,7 @@ __device__ __forceinline__ TokRows tok_rows(int g, int t) {
 // Scores of one 16-token subtile whose rows start at `srow` of the staged
 // planes: s2 (base 2) for tokens g (s2[0], s2[1]) and g+8 (s2[2], s2[3]),
 // columns 2t, 2t+1; masked tokens get -inf.  Two MMA accumulator chains.
-template <int KF, bool PACK>
+template <int KF, bool PACK, bool T3W>
 __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
                                                int g, int t,
                                                const QFrag<PACK>& bq, const QFrag<PACK>& bqs,
@@ -700,8 +715,8 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
     static_for<KR::S1::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      xa.template decode<s>(lut_a, lane4, lane8, c1k, la, ha);
-      xb.template decode<s>(lut_a, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s, T3W>(lut_a, lane4, lane8, c1k, la, ha);
+      xb.template decode<s, T3W>(lut_a, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x)
         mma16816(ca[(NX * s + x + 1) & 1], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
@@ -834,9 +849,9 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
   const bool ok0A = row0 + tr.kA < nq, ok0B = row0 + tr.kB < nq;
   const bool ok1A = row0 + kTok + tr.kA < nq, ok1B = row0 + kTok + tr.kB < nq;
   float s0[4], s1[4];
-  subtile_scores<KF, PACK>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
+  subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
   if constexpr (second)
-    subtile_scores<KF, PACK>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
+    subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
   // online softmax over the 32 tokens (base 2), columns 2t and 2t+1.  The
@@ -1432,9 +1447,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       }
     }
     if constexpr (L::t3) {
-      for (int i = tid; i < 64 * 32; i += kThreadsP) {
-        const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (r & 7)], cb[3 * kBookSlots + (r >> 3)]);
+      constexpr int rows = L::t3_wide ? 256 : 64;
+      for (int i = tid; i < rows * 32; i += kThreadsP) {
+        const int r = i >> 5, ln = i & 31, e = r & 63;
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
       }
     }
     if constexpr (L::t2) {
