@@ -242,10 +242,15 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     hk = [t.cpu().pin_memory() for t in st["ck"][:args.steps]]
     hv = [t.cpu().pin_memory() for t in st["cv"][:args.steps]]
     hq = [t.cpu().pin_memory() for t in st["qs"][:args.steps]]
-    hout = torch.empty(N_SEQ, HQ, D, dtype=torch.bfloat16).pin_memory()
-    dk = torch.empty_like(st["ck"][0])
-    dv = torch.empty_like(st["cv"][0])
-    dq = torch.empty_like(st["qs"][0])
+    hout = [torch.empty(N_SEQ, HQ, D, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    # double-buffered device inputs: the copy stream brings step j's chunk and
+    # queries in while the compute stream still decodes step j - 1
+    dk = [torch.empty_like(st["ck"][0]) for _ in range(2)]
+    dv = [torch.empty_like(st["cv"][0]) for _ in range(2)]
+    dq = [torch.empty_like(st["qs"][0]) for _ in range(2)]
+    copy_stream = torch.cuda.Stream(device=device)
+    copied = [torch.cuda.Event() for _ in range(args.steps)]
+    consumed = [torch.cuda.Event() for _ in range(args.steps)]
     # rewind the lengths so the e2e steps see the same contexts as the timed ones
     lens0 = torch.tensor([n + args.warmup * CHUNK for n in st["lens"]], dtype=torch.int32, device=device)
     cache.lens.copy_(lens0)
@@ -254,13 +259,21 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
         dist.barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    copy_stream.wait_event(t0)
     for j in range(args.steps):
-        dk.copy_(hk[j], non_blocking=True)
-        dv.copy_(hv[j], non_blocking=True)
-        dq.copy_(hq[j], non_blocking=True)
-        tq.tq_append(params, cache, st["ids"], dk, dv)
-        tq.tq_decode_attn(params, dq, cache, st["cap"], st["out"], st["ws"])
-        hout.copy_(st["out"], non_blocking=True)
+        b = j & 1
+        with torch.cuda.stream(copy_stream):
+            if j >= 2:
+                copy_stream.wait_event(consumed[j - 2])  # step j - 2 has read buffer b
+            dk[b].copy_(hk[j], non_blocking=True)
+            dv[b].copy_(hv[j], non_blocking=True)
+            dq[b].copy_(hq[j], non_blocking=True)
+            copied[j].record(copy_stream)
+        stream.wait_event(copied[j])
+        tq.tq_append(params, cache, st["ids"], dk[b], dv[b], stream=stream)
+        tq.tq_decode_attn(params, dq[b], cache, st["cap"], st["out"], st["ws"], stream=stream)
+        consumed[j].record(stream)
+        hout[b].copy_(st["out"], non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
@@ -301,7 +314,7 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny")
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa")
 
 
 def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
@@ -319,6 +332,8 @@ def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
         out.update(_aux_k4v3(tq, torch, kv_inputs, device, flush, iters))
     if only in (None, "tiny"):
         out["decode_tiny_fp32_T4096"] = _aux_tiny(tq, torch, kv_inputs, device, iters)
+    if only in (None, "bf16-sdpa"):
+        out["bf16_kv_decode_sdpa_stream_shapes"] = _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters)
     return out
 
 
@@ -401,6 +416,42 @@ def _aux_tiny(tq, torch, kv_inputs, device, iters):
     o = torch.empty(1, 1, D, dtype=torch.float32, device=device)
     ms = _time_call(torch, lambda: tq.tq_decode_attn(p, q, cache, 4096, o, ws), iters)
     return {"ms": round(ms, 4)}
+
+
+def _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters):
+    """Context for the packed cache: one decode step over an unquantized bf16
+    KV cache of the streaming workload's shapes (16 sequences, the same
+    contexts, 32 q / 8 kv heads), with PyTorch's fused attention (the fastest
+    backend that accepts the shapes), one call per sequence."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", 0))
+    gen = torch.Generator(device=device).manual_seed(0)
+    ks = [torch.randn(1, HKV, n, D, generator=gen, device=device, dtype=torch.bfloat16) for n in lens]
+    vs = [torch.randn(1, HKV, n, D, generator=gen, device=device, dtype=torch.bfloat16) for n in lens]
+    q = torch.randn(N_SEQ, 1, HQ, 1, D, generator=gen, device=device, dtype=torch.bfloat16)
+    by = sum(n * HKV * D * 2 * 2 for n in lens)
+    best = None
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION,
+                    SDPBackend.MATH):
+        try:
+            with sdpa_kernel([backend]):
+                def run():
+                    for s in range(N_SEQ):
+                        F.scaled_dot_product_attention(q[s], ks[s], vs[s], enable_gqa=True)
+                run()
+                torch.cuda.synchronize()
+                ms = _time_call(torch, run, iters, flush)
+        except RuntimeError:
+            continue
+        if best is None or ms < best[1]:
+            best = (backend.name, ms)
+    if best is None:
+        return {"unavailable": "no SDPA backend accepted the shapes"}
+    name, ms = best
+    return {"backend": name, "ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
+            "tokens_per_s_per_seq": round(1000.0 / ms, 1), "calls": N_SEQ}
 
 
 def run_aux_only(args):

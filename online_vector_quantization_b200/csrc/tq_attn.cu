@@ -1682,14 +1682,13 @@ cudaError_t launch_overlapped(Kernel kernel, dim3 grid, int threads, size_t smem
 
 template <int KF, int VF, bool PACK, bool SPARSE>
 tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<KF, VF, PACK, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem<decode_kernel<KF, VF, PACK, SPARSE>>(static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
   // the query rotation waits for all earlier work on the stream (the appends
   // that filled the cache); the two kernels after it overlap their prologues
   // with its tail
   const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
-  e = cudaFuncSetAttribute(qrot_kernel<KF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(qrot_smem));
+  e = ensure_dyn_smem<qrot_kernel<KF>>(static_cast<int>(qrot_smem));
   if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
   qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kQrotThreads, qrot_smem, st>>>(a);
   e = cudaGetLastError();
@@ -1698,7 +1697,7 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, plan.group, plan.part_floats);
   if (merge_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(merge_kernel<VF>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(merge_smem));
+    e = ensure_dyn_smem<merge_kernel<VF>>(static_cast<int>(merge_smem));
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
   }
   e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv), kMergeThreads, merge_smem, st, a);

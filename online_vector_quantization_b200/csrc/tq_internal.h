@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 #include <vector>
 
@@ -70,6 +71,28 @@ namespace tq {
 
 tq_status fail(tq_status st, const std::string& msg);
 tq_status cuda_fail(cudaError_t e, const char* what);
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, calling the runtime only the first time a larger value is
+// needed there (the attribute persists; the call costs host time on every
+// launch otherwise).  One instantiation, and so one record, per kernel.
+template <auto kernel>
+cudaError_t ensure_dyn_smem(int bytes) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> granted[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices)
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (granted[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  int cur = granted[dev].load(std::memory_order_relaxed);
+  while (cur < bytes && !granted[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+  }
+  return cudaSuccess;
+}
 
 // Kernel launchers (defined in the .cu files).
 tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x, int x_bf16,

@@ -1004,7 +1004,7 @@ EncodeTiledFn encode_tiled() {
 template <int MB>
 tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
   cudaError_t e =
-      cudaFuncSetAttribute(quantize_tc_prod_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTpSmem);
+      ensure_dyn_smem<quantize_tc_prod_kernel<MB>>(kTpSmem);
   if (e == cudaSuccess) {
     quantize_tc_prod_kernel<MB><<<grid, kTcThreads, kTpSmem, st>>>(map, a);
     e = cudaGetLastError();
@@ -1014,7 +1014,7 @@ tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap& map, int grid, c
 
 template <int B, int MIXED>
 tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<B, MIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+  cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED>>(kTcSmem);
   if (e == cudaSuccess) {
     quantize_tc_kernel<B, MIXED><<<grid, kTcThreads, kTcSmem, st>>>(map, a);
     e = cudaGetLastError();
@@ -1069,10 +1069,10 @@ tq_status run_quantize(QuantArgs& a, cudaStream_t st) {
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   cudaError_t e;
   if (a.x_bf16) {
-    e = cudaFuncSetAttribute(quantize_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = ensure_dyn_smem<quantize_kernel<1>>(static_cast<int>(smem));
     if (e == cudaSuccess) quantize_kernel<1><<<grid, kThreads, smem, st>>>(a);
   } else {
-    e = cudaFuncSetAttribute(quantize_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = ensure_dyn_smem<quantize_kernel<0>>(static_cast<int>(smem));
     if (e == cudaSuccess) quantize_kernel<0><<<grid, kThreads, smem, st>>>(a);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
