@@ -1434,35 +1434,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const int P = gridDim.x, cta = blockIdx.x;
   const int U = a.B * a.hkv;
 
-  // ---- lookup tables (all threads), schedule and barriers (thread 0)
-  {
-    __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
-    if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
-    __syncthreads();
-    const float* cb = s_cb;
-    if constexpr (L::t4) {
-      for (int i = tid; i < 256 * 32; i += kThreadsP) {
-        const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
-      }
-    }
-    if constexpr (L::t3) {
-      constexpr int rows = L::t3_wide ? 256 : 64;
-      for (int i = tid; i < rows * 32; i += kThreadsP) {
-        const int r = i >> 5, ln = i & 31, e = r & 63;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
-      }
-    }
-    if constexpr (L::t2) {
-      for (int i = tid; i < 256 * 32; i += kThreadsP) {
-        const int r = i >> 5, ln = i & 31;
-        uint2 v;
-        v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
-        v.y = h2bits(cb[2 * kBookSlots + ((r >> 4) & 3)], cb[2 * kBookSlots + (r >> 6)]);
-        *reinterpret_cast<uint2*>(lut_mem + L::region_b_off + r * 256 + ln * 8) = v;
-      }
-    }
-  }
+  // ---- codebooks to shared memory, schedule (warp 0) and barriers (thread 32);
+  // the producer starts streaming right after, while the consumers build
+  // the lookup tables
+  __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
+  if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
   if (warp == 0) {
     // schedule (one warp): total chunks C, this CTA's range [c0, c1) and the
     // unit / local chunk where it starts
@@ -1568,6 +1544,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     }
     return;
   }
+
+  // ---- lookup tables (consumer threads)
+  {
+    constexpr int NTC = kConsumers * 32;
+    const float* cb = s_cb;
+    if constexpr (L::t4) {
+      for (int i = tid; i < 256 * 32; i += NTC) {
+        const int r = i >> 5, ln = i & 31;
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
+      }
+    }
+    if constexpr (L::t3) {
+      constexpr int rows = L::t3_wide ? 256 : 64;
+      for (int i = tid; i < rows * 32; i += NTC) {
+        const int r = i >> 5, ln = i & 31, e = r & 63;
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
+      }
+    }
+    if constexpr (L::t2) {
+      for (int i = tid; i < 256 * 32; i += NTC) {
+        const int r = i >> 5, ln = i & 31;
+        uint2 v;
+        v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
+        v.y = h2bits(cb[2 * kBookSlots + ((r >> 4) & 3)], cb[2 * kBookSlots + (r >> 6)]);
+        *reinterpret_cast<uint2*>(lut_mem + L::region_b_off + r * 256 + ln * 8) = v;
+      }
+    }
+  }
+  consumers_sync();  // tables complete
 
   // ---- consumers
   // table bases are folded into the lane offsets (see kLutAddr)
