@@ -43,6 +43,7 @@ MASK64 = (1 << 64) - 1
 SPLITMIX_GAMMA = 0x9E3779B97F4A7C15
 TAG_ROTATION = 0
 TAG_QJL = 1
+TAG_HADAMARD_SIGNS = 2
 
 
 def splitmix64(state0: int, count: int, start: int = 0) -> np.ndarray:
@@ -102,6 +103,36 @@ def rotation(seed: int, d: int) -> np.ndarray:
     s = np.sign(np.diag(r))
     s[s == 0] = 1.0
     return q * s[None, :]
+
+
+def hadamard_signs(seed: int, d: int) -> np.ndarray:
+    """The random sign flips of the Hadamard rotation: s_j = -1 when the top
+    bit of SplitMix64 output j of stream (seed, TAG_HADAMARD_SIGNS) is set,
+    +1 otherwise."""
+    z = splitmix64(stream_state(seed, TAG_HADAMARD_SIGNS), d)
+    return np.where((z >> np.uint64(63)) == 1, -1.0, 1.0)
+
+
+def walsh_hadamard(d: int) -> np.ndarray:
+    """Sylvester's Walsh-Hadamard matrix: H[i][j] = (-1)^popcount(i & j)."""
+    i = np.arange(d)
+    bits = np.bitwise_and(i[:, None], i[None, :])
+    pop = np.zeros_like(bits)
+    while bits.any():
+        pop += bits & 1
+        bits >>= 1
+    return np.where(pop % 2 == 1, -1.0, 1.0)
+
+
+def hadamard_rotation(seed: int, d: int) -> np.ndarray:
+    """[P3] "Cosa aggiunge turboquant-mlx": the port realizes the random
+    rotation with a Hadamard transform.  Randomized with sign flips (the page
+    gives no detail; the plainest reading): Pi = H D / sqrt(d), D = diag(s),
+    so y = Pi u is the normalized Walsh-Hadamard transform of the sign-flipped
+    u.  d must be a power of two."""
+    if d <= 0 or d & (d - 1):
+        raise ValueError("the Hadamard rotation needs d a power of two")
+    return walsh_hadamard(d) * hadamard_signs(seed, d)[None, :] / math.sqrt(d)
 
 
 def qjl_matrix(seed: int, m: int, d: int) -> np.ndarray:
@@ -277,12 +308,18 @@ class Params:
     fmt_v: Format
     seed: int = 0
     m: int = 128
+    rotation: str = "haar"   # "haar" (dense Haar Pi) or "hadamard" (sign flips + Walsh-Hadamard)
     pi: np.ndarray = field(init=False)
     s: np.ndarray = field(init=False)
     books: dict = field(init=False)
 
     def __post_init__(self):
-        self.pi = rotation(self.seed, self.d)
+        if self.rotation == "haar":
+            self.pi = rotation(self.seed, self.d)
+        elif self.rotation == "hadamard":
+            self.pi = hadamard_rotation(self.seed, self.d)
+        else:
+            raise ValueError(f"unknown rotation {self.rotation!r}")
         self.s = qjl_matrix(self.seed, self.m, self.d)
         self.books = {}
         for f in (self.fmt_k, self.fmt_v):

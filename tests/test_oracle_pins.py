@@ -87,6 +87,74 @@ def test_rotation_is_haar():
     assert stats.kstest((1 + xs) / 2, stats.beta(a, a).cdf).pvalue > 1e-4
 
 
+# ---- Hadamard rotation ([P3] "Cosa aggiunge turboquant-mlx") ---------------
+
+def _sylvester(d):
+    # Independent construction of the Walsh-Hadamard matrix: H_1 = [1],
+    # H_2n = [[H_n, H_n], [H_n, -H_n]].
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def _fwht(v):
+    # In-place butterflies (an O(d log d) algorithm, not a matrix product).
+    v = v.copy()
+    n, hlen = v.shape[0], 1
+    while hlen < n:
+        for i in range(0, n, 2 * hlen):
+            a, b = v[i:i + hlen].copy(), v[i + hlen:i + 2 * hlen].copy()
+            v[i:i + hlen], v[i + hlen:i + 2 * hlen] = a + b, a - b
+        hlen *= 2
+    return v
+
+
+def test_hadamard_rotation_orthogonal_with_entries_pm_inv_sqrt_d():
+    for d in (8, 128, 512):
+        pi = o.hadamard_rotation(3, d)
+        assert np.max(np.abs(pi @ pi.T - np.eye(d))) < 1e-14
+        assert np.all(np.abs(np.abs(pi) - 1 / math.sqrt(d)) < 1e-16)
+        assert np.array_equal(o.walsh_hadamard(d), _sylvester(d))
+
+
+def test_hadamard_rotation_is_signed_fast_transform():
+    # y = Pi u is the normalised fast Walsh-Hadamard transform of the
+    # sign-flipped u: catches a transposed Pi (signs on rows, not columns).
+    d = 128
+    rng = np.random.default_rng(11)
+    s = o.hadamard_signs(7, d)
+    for _ in range(4):
+        u = rng.standard_normal(d)
+        want = _fwht(s * u) / math.sqrt(d)
+        assert np.max(np.abs(o.hadamard_rotation(7, d) @ u - want)) < 1e-13
+
+
+def test_hadamard_signs_balanced_and_seeded():
+    s = o.hadamard_signs(0, 1 << 14)
+    assert set(np.unique(s)) == {-1.0, 1.0}
+    assert abs(s.mean()) < 5 / math.sqrt(s.size)
+    assert not np.array_equal(o.hadamard_signs(0, 128), o.hadamard_signs(1, 128))
+
+
+@pytest.mark.parametrize("fmt", [o.Format(3), o.Format(3, mixed=True), o.Format(2, prod=True)])
+def test_hadamard_quantize_is_nearest_centroid_and_rotates_back(fmt):
+    p = o.Params(128, fmt, fmt, rotation="hadamard")
+    x = kv_inputs.kv_vectors(32, 128, key="hd", dtype=torch.bfloat16).double().numpy()
+    pk = o.quantize(p, x, "k")
+    widths = [fmt.mse_bits(j, 128) for j in range(128)]
+    idx = o.unpack_codes(pk.codes, widths)
+    y = (x / np.linalg.norm(x, axis=1, keepdims=True)) @ p.pi.T
+    for v in range(32):
+        for j in range(128):
+            if widths[j]:
+                assert idx[v, j] == int(np.argmin(np.abs(y[v, j] - p.books[widths[j]].centroids)))
+    if not fmt.prod:
+        xh = o.dequantize(p, pk, "k")
+        c = np.array([[p.books[widths[j]].centroids[idx[v, j]] for j in range(128)] for v in range(32)])
+        assert np.max(np.abs(xh @ p.pi.T / pk.norms.astype(np.float64)[:, None] - c)) < 1e-13
+
+
 def test_qjl_matrix_standard_normal_rows():
     s = o.qjl_matrix(0, 128, 128)
     assert s.shape == (128, 128)
