@@ -61,6 +61,7 @@ typedef enum {
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 typedef enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1 } tq_mode;
 typedef enum { TQ_K = 0, TQ_V = 1 } tq_which;
+typedef enum { TQ_ROT_HAAR = 0, TQ_ROT_HADAMARD = 1 } tq_rotation_kind;
 
 /* Parameters of one quantizer pair (keys and values may differ: the
  * asymmetric K/V setting of "Greetings from TurboQuant-MLX" (turboquant_plus
@@ -75,6 +76,7 @@ typedef struct {
   int mixed_k, mixed_v;  /* 0 or 1 */
   int m;                 /* QJL sketch size */
   uint64_t seed;
+  int rotation;          /* tq_rotation_kind: dense Haar Pi (0) or randomized Hadamard (1) */
 } tq_config;
 
 typedef struct tq_params tq_params;
@@ -104,6 +106,15 @@ tq_status tq_codebook(int d, int bits, double* centroids, double* bounds);
  * from SplitMix64 (stream seed ^ (0 << 32)) and Box-Muller, filled row-major.
  * Host array of d*d doubles, caller-owned.  Pure host function. */
 tq_status tq_rotation(uint64_t seed, int d, double* pi);
+
+/* Randomized Hadamard rotation, the port's realization of the random rotation
+ * (TurboQuant-MLX article, section "Cosa aggiunge turboquant-mlx"):
+ * Pi = H D / sqrt(d) with H the Walsh-Hadamard matrix (Sylvester order,
+ * H[i][j] = (-1)^popcount(i & j)) and D = diag(s), s_j = -1 when the top bit
+ * of SplitMix64 output j of stream seed ^ (2 << 32) is set, else +1.  d a
+ * power of two; host array of d*d doubles (row-major, y = Pi u), caller-owned.
+ * Pure host function. */
+tq_status tq_hadamard_rotation(uint64_t seed, int d, double* pi);
 
 /* QJL matrix S (m x d row-major, i.i.d. N(0,1)) from the stream
  * seed ^ (1 << 32).  Host array of m*d doubles.  Pure host function. */

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libtq.so")
 
 TQ_F32, TQ_BF16 = 0, 1
 TQ_MODE_MSE, TQ_MODE_PROD = 0, 1
+TQ_ROT_HAAR, TQ_ROT_HADAMARD = 0, 1
 TQ_K, TQ_V = 0, 1
 STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_ARG", 2: "TQ_ERR_UNSUPPORTED", 3: "TQ_ERR_ALIGN",
                 4: "TQ_ERR_CAPACITY", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_NOMEM"}
@@ -41,7 +42,7 @@ _dp = ctypes.POINTER(ctypes.c_double)
 class TqConfig(ctypes.Structure):
     _fields_ = [("d", c_int), ("bits_k", c_int), ("bits_v", c_int), ("mode_k", c_int),
                 ("mode_v", c_int), ("mixed_k", c_int), ("mixed_v", c_int), ("m", c_int),
-                ("seed", c_uint64)]
+                ("seed", c_uint64), ("rotation", c_int)]
 
 
 class TqPacked(ctypes.Structure):
@@ -62,6 +63,7 @@ class TqAttnFlags(ctypes.Structure):
 _SIGS = {
     "tq_codebook": (c_int, [c_int, c_int, _dp, _dp]),
     "tq_rotation": (c_int, [c_uint64, c_int, _dp]),
+    "tq_hadamard_rotation": (c_int, [c_uint64, c_int, _dp]),
     "tq_qjl_matrix": (c_int, [c_uint64, c_int, c_int, _dp]),
     "tq_params_create": (c_int, [ctypes.POINTER(TqConfig), ctypes.POINTER(c_void_p)]),
     "tq_params_destroy": (None, [c_void_p]),
@@ -130,6 +132,12 @@ def tq_rotation(seed: int, d: int) -> np.ndarray:
     return out
 
 
+def tq_hadamard_rotation(seed: int, d: int) -> np.ndarray:
+    out = np.zeros((d, d))
+    _check(_lib.tq_hadamard_rotation(seed, d, out.ctypes.data_as(_dp)))
+    return out
+
+
 def tq_qjl_matrix(seed: int, m: int, d: int) -> np.ndarray:
     out = np.zeros((m, d))
     _check(_lib.tq_qjl_matrix(seed, m, d, out.ctypes.data_as(_dp)))
@@ -142,8 +150,9 @@ class Params:
     """Owner of a tq_params handle (device tables on the current device)."""
 
     def __init__(self, bits_k: int, bits_v: int, mode_k: int = TQ_MODE_MSE, mode_v: int = TQ_MODE_MSE,
-                 mixed_k: int = 0, mixed_v: int = 0, seed: int = 0, d: int = 128, m: int = 128):
-        self.config = TqConfig(d, bits_k, bits_v, mode_k, mode_v, mixed_k, mixed_v, m, seed)
+                 mixed_k: int = 0, mixed_v: int = 0, seed: int = 0, d: int = 128, m: int = 128,
+                 rotation: int = 0):
+        self.config = TqConfig(d, bits_k, bits_v, mode_k, mode_v, mixed_k, mixed_v, m, seed, rotation)
         h = c_void_p()
         _check(_lib.tq_params_create(ctypes.byref(self.config), ctypes.byref(h)))
         self.handle = h.value

@@ -270,6 +270,29 @@ tq_status tq_rotation(uint64_t seed, int d, double* pi) {
   return TQ_OK;
 }
 
+tq_status tq_hadamard_rotation(uint64_t seed, int d, double* pi) {
+  if (!pi || d < 1 || (d & (d - 1))) return fail(TQ_ERR_ARG, "tq_hadamard_rotation: d must be a power of two");
+  // Sylvester doubling: H_2n = [[H_n, H_n], [H_n, -H_n]]
+  std::vector<double> h(static_cast<size_t>(d) * d, 0.0);
+  h[0] = 1.0;
+  for (int n = 1; n < d; n *= 2)
+    for (int i = 0; i < n; ++i)
+      for (int j = 0; j < n; ++j) {
+        const double v = h[static_cast<size_t>(i) * d + j];
+        h[static_cast<size_t>(i) * d + j + n] = v;
+        h[static_cast<size_t>(i + n) * d + j] = v;
+        h[static_cast<size_t>(i + n) * d + j + n] = -v;
+      }
+  const uint64_t s0 = seed ^ (uint64_t(2) << 32);
+  const double inv = 1.0 / std::sqrt(static_cast<double>(d));
+  for (int j = 0; j < d; ++j) {
+    const uint64_t z = splitmix_mix(s0 + uint64_t(j + 1) * 0x9E3779B97F4A7C15ull);
+    const double s = (z >> 63) ? -inv : inv;
+    for (int i = 0; i < d; ++i) pi[static_cast<size_t>(i) * d + j] = h[static_cast<size_t>(i) * d + j] * s;
+  }
+  return TQ_OK;
+}
+
 tq_status tq_qjl_matrix(uint64_t seed, int m, int d, double* s) {
   if (!s || m < 1 || d < 1) return fail(TQ_ERR_ARG, "tq_qjl_matrix: bad arguments");
   gaussian_stream(seed, 1, static_cast<size_t>(m) * d, s);
@@ -326,6 +349,8 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   if (!cfg || !out) return fail(TQ_ERR_ARG, "tq_params_create: NULL argument");
   *out = nullptr;
   if (cfg->d != kDim) return fail(TQ_ERR_UNSUPPORTED, "tq_params_create: d must be 128");
+  if (cfg->rotation != TQ_ROT_HAAR && cfg->rotation != TQ_ROT_HADAMARD)
+    return fail(TQ_ERR_ARG, "tq_params_create: unknown rotation kind");
   if (cfg->m != kSketch) return fail(TQ_ERR_UNSUPPORTED, "tq_params_create: m must be 128");
   std::string why;
   FormatSpec fk, fv;
@@ -340,7 +365,10 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   const int d = kDim, m = kSketch;
   p->pi.resize(static_cast<size_t>(d) * d);
   p->s.resize(static_cast<size_t>(m) * d);
-  tq_rotation(cfg->seed, d, p->pi.data());
+  if (cfg->rotation == TQ_ROT_HADAMARD)
+    tq_hadamard_rotation(cfg->seed, d, p->pi.data());
+  else
+    tq_rotation(cfg->seed, d, p->pi.data());
   tq_qjl_matrix(cfg->seed, m, d, p->s.data());
 
   // host staging of every device table

@@ -40,6 +40,17 @@ def test_rotation_matches_oracle(seed, d):
     assert np.max(np.abs(tq.tq_rotation(seed, d) - o.rotation(seed, d))) < 1e-12
 
 
+@pytest.mark.parametrize("seed,d", [(0, 128), (99, 128), (5, 8), (1, 512)])
+def test_hadamard_rotation_matches_oracle(seed, d):
+    assert np.array_equal(tq.tq_hadamard_rotation(seed, d), o.hadamard_rotation(seed, d))
+
+
+def test_hadamard_rotation_rejects_non_power_of_two():
+    with pytest.raises(tq.TqError) as e:
+        tq.tq_hadamard_rotation(0, 96)
+    assert e.value.status == 1
+
+
 def test_qjl_matrix_matches_oracle():
     assert np.max(np.abs(tq.tq_qjl_matrix(3, 128, 128) - o.qjl_matrix(3, 128, 128))) < 1e-14
 
@@ -57,5 +68,8 @@ def test_host_argument_errors():
     with pytest.raises(tq.TqError) as e:
         tq.Params(3, 3, mixed_k=1, mode_k=tq.TQ_MODE_PROD)
     assert e.value.status == 2
+    with pytest.raises(tq.TqError) as e:
+        tq.Params(3, 3, rotation=7)
+    assert e.value.status == 1
     assert tq._lib.tq_cache_bytes(None, 1, 1, 64, 0) == 0
     assert tq._lib.tq_decode_workspace_bytes(None, 1, 8, 8, 128) == 0
