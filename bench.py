@@ -342,17 +342,22 @@ def _aux_sweep(tq, torch, kv_inputs, device, flush, iters, formats):
     n = 32 * 32768
     x = kv_inputs.kv_vectors(n, D, key="sweep", device=device, dtype=torch.bfloat16, outliers=True)
     sweep = {}
-    for mode, name in ((tq.TQ_MODE_MSE, "mse"), (tq.TQ_MODE_PROD, "prod")):
-        for b in (1, 2, 3, 4):
-            if formats and f"{name}{b}" not in formats:
-                continue
-            p = tq.Params(b, b, mode, mode)
-            pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
-            ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
-            cb, qb = p.row_bytes(tq.TQ_K)
-            by = n * (D * 2 + cb + 4 + (qb + 4 if qb else 0))
-            sweep[f"{name}{b}"] = {"mvec_per_s": round(n / (ms * 1e-3) / 1e6, 1), "ms": round(ms, 4),
-                                   "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1)}
+    cases = [(mode, name, b, tq.TQ_ROT_HAAR, f"{name}{b}")
+             for mode, name in ((tq.TQ_MODE_MSE, "mse"), (tq.TQ_MODE_PROD, "prod")) for b in (1, 2, 3, 4)]
+    # the randomized Hadamard rotation in place of the Haar one (same kernels, another Pi)
+    cases += [(tq.TQ_MODE_MSE, "mse", 3, tq.TQ_ROT_HADAMARD, "mse3_hadamard"),
+              (tq.TQ_MODE_PROD, "prod", 3, tq.TQ_ROT_HADAMARD, "prod3_hadamard")]
+    for mode, name, b, rot, label in cases:
+        if formats and label not in formats:
+            continue
+        p = tq.Params(b, b, mode, mode, rotation=rot)
+        pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
+        ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
+        assert p.status() == 0
+        cb, qb = p.row_bytes(tq.TQ_K)
+        by = n * (D * 2 + cb + 4 + (qb + 4 if qb else 0))
+        sweep[label] = {"mvec_per_s": round(n / (ms * 1e-3) / 1e6, 1), "ms": round(ms, 4),
+                        "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1)}
     return sweep
 
 

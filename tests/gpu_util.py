@@ -20,10 +20,12 @@ def fmt(bits, prod=False, mixed=False):
     return o.Format(bits, prod=prod, mixed=mixed)
 
 
-def make_params(fk: o.Format, fv: o.Format, seed: int = 0):
+def make_params(fk: o.Format, fv: o.Format, seed: int = 0, rotation: str = "haar"):
+    kind = {"haar": tq.TQ_ROT_HAAR, "hadamard": tq.TQ_ROT_HADAMARD}[rotation]
     gp = tq.Params(fk.bits, fv.bits, tq.TQ_MODE_PROD if fk.prod else tq.TQ_MODE_MSE,
-                   tq.TQ_MODE_PROD if fv.prod else tq.TQ_MODE_MSE, int(fk.mixed), int(fv.mixed), seed=seed)
-    op = o.Params(128, fk, fv, seed=seed)
+                   tq.TQ_MODE_PROD if fv.prod else tq.TQ_MODE_MSE, int(fk.mixed), int(fv.mixed), seed=seed,
+                   rotation=kind)
+    op = o.Params(128, fk, fv, seed=seed, rotation=rotation)
     return gp, op
 
 

@@ -66,6 +66,30 @@ def test_quantize_many_tiles_per_cta(f):
 
 
 @pytest.mark.parametrize("f", FORMATS, ids=FMT_IDS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_quantize_parity_hadamard_rotation(f, dtype):
+    """The randomized Hadamard rotation (sign flips, then the normalized
+    Walsh-Hadamard transform) in place of the Haar rotation: both quantize
+    kernels (SIMT for fp32, tensor cores for bf16) across several tiles of
+    the persistent grid and a ragged tail."""
+    gp, op = gu.make_params(f, f, seed=11, rotation="hadamard")
+    n = 148 * 128 + 333
+    x = kv_inputs.kv_vectors(n, 128, key=("qh", f.bits, f.prod, f.mixed), dtype=dtype, outliers=True)
+    x[5] = 0
+    out = tq.Packed.empty(gp, n, tq.TQ_K)
+    tq.tq_quantize(gp, x.cuda(), tq.TQ_K, out)
+    torch.cuda.synchronize()
+    assert gp.status() == 0
+    got = gu.gpu_packed_to_numpy(out)
+    xd = x.double().numpy()
+    want = o.quantize(op, xd, "k")
+    skip = gu.compare_codes(op, f, xd, got, want) if f.code_bytes(128) else set()
+    assert np.allclose(got.norms, want.norms, rtol=1e-6, atol=0)
+    gu.compare_qjl(op, f, xd, got, want, skip)
+    assert not got.codes[5].any() and got.norms[5] == 0
+
+
+@pytest.mark.parametrize("f", FORMATS, ids=FMT_IDS)
 def test_dequantize_parity(f):
     gp, op = gu.make_params(f, f)
     n = 777
@@ -79,8 +103,8 @@ def test_dequantize_parity(f):
 
 
 def _decode_case(fk, fv, B, hq, hkv, T, lens, n_sink, thr, q_dtype=torch.bfloat16, out_dtype=torch.bfloat16,
-                 key="dec"):
-    gp, op = gu.make_params(fk, fv)
+                 key="dec", rotation="haar"):
+    gp, op = gu.make_params(fk, fv, rotation=rotation)
     k = kv_inputs.kv_vectors(B * hkv * T, 128, key=(key, "k"), dtype=torch.bfloat16)
     v = kv_inputs.kv_vectors(B * hkv * T, 128, key=(key, "v"), dtype=torch.bfloat16)
     kd = k.double().numpy().reshape(B, hkv, T, 128)
@@ -124,6 +148,15 @@ def test_decode_parity_formats(fk, fv):
     # several splits per sequence, ragged lengths, GQA group of 4
     got, want, _ = _decode_case(fk, fv, B=2, hq=8, hkv=2, T=2500, lens=[2500, 1777], n_sink=0, thr=0.0,
                                 key=("fmt", str(fk), str(fv)))
+    assert gu.rel_l2(got, want) < gu.ATTN_REL_L2
+
+
+@pytest.mark.parametrize("fk,fv", [(gu.fmt(4), gu.fmt(3)), (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)),
+                                   (gu.fmt(3, prod=True), gu.fmt(3, prod=True))], ids=["k4v3", "mixed", "prod3"])
+def test_decode_parity_hadamard_rotation(fk, fv):
+    # the query rotation and the output un-rotation use the Hadamard Pi
+    got, want, _ = _decode_case(fk, fv, B=2, hq=8, hkv=2, T=1500, lens=[1500, 999], n_sink=16, thr=0.0,
+                                key=("had", str(fk), str(fv)), rotation="hadamard")
     assert gu.rel_l2(got, want) < gu.ATTN_REL_L2
 
 
