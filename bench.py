@@ -93,10 +93,11 @@ class ClockSampler:
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device):
-    """Config: streaming append + decode.  Returns the state the step uses."""
+def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device, bits: int = 3):
+    """Config: streaming append + decode (mixed rows: bits + 0.5 bits per
+    channel, 3.5 by default).  Returns the state the step uses."""
     lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", rank))
-    params = tq.Params(3, 3, mixed_k=1, mixed_v=1, seed=0)
+    params = tq.Params(bits, bits, mixed_k=1, mixed_v=1, seed=0)
     cap = ((max(lens) + (n_steps + 1) * CHUNK + 63) // 64) * 64
     cache = tq.Cache(params, N_SEQ, HKV, cap, 0, device=device)
     # prefill (untimed): the prefix of each sequence through tq_append
@@ -314,7 +315,7 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa")
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "stream-2.5")
 
 
 def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
@@ -332,6 +333,8 @@ def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
         out.update(_aux_k4v3(tq, torch, kv_inputs, device, flush, iters))
     if only in (None, "tiny"):
         out["decode_tiny_fp32_T4096"] = _aux_tiny(tq, torch, kv_inputs, device, iters)
+    if only in (None, "stream-2.5"):
+        out["decode_mixed2.5_stream_shapes"] = _aux_stream25(tq, torch, kv_inputs, device, flush, iters)
     if only in (None, "bf16-sdpa"):
         out["bf16_kv_decode_sdpa_stream_shapes"] = _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters)
     return out
@@ -345,12 +348,14 @@ def _aux_sweep(tq, torch, kv_inputs, device, flush, iters, formats):
     cases = [(mode, name, b, tq.TQ_ROT_HAAR, f"{name}{b}")
              for mode, name in ((tq.TQ_MODE_MSE, "mse"), (tq.TQ_MODE_PROD, "prod")) for b in (1, 2, 3, 4)]
     # the randomized Hadamard rotation in place of the Haar one (same kernels, another Pi)
+    cases += [(tq.TQ_MODE_MSE, "mixed", 2, tq.TQ_ROT_HAAR, "mixed2.5"), (tq.TQ_MODE_MSE, "mixed", 3, tq.TQ_ROT_HAAR, "mixed3.5")]
     cases += [(tq.TQ_MODE_MSE, "mse", 3, tq.TQ_ROT_HADAMARD, "mse3_hadamard"),
               (tq.TQ_MODE_PROD, "prod", 3, tq.TQ_ROT_HADAMARD, "prod3_hadamard")]
     for mode, name, b, rot, label in cases:
         if formats and label not in formats:
             continue
-        p = tq.Params(b, b, mode, mode, rotation=rot)
+        mixed = int(name == "mixed")
+        p = tq.Params(b, b, mode, mode, mixed, mixed, rotation=rot)
         pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
         ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
         assert p.status() == 0
@@ -407,6 +412,23 @@ def _aux_k4v3(tq, torch, kv_inputs, device, flush, iters):
         out[f"decode_k4v3_sink_T128k_{name}"] = {"ms": round(ms, 4), "gb_per_s_dense_equiv": round(by / (ms * 1e-3) / 1e9, 1),
                                                  "dense_bytes": by}
     assert int(cache.status.item()) == 0
+    return out
+
+
+def _aux_stream25(tq, torch, kv_inputs, device, flush, iters):
+    """The decode call of the streaming workload (16 sequences, the same
+    contexts, 32 q / 8 kv heads) over 2.5-bit rows (64 rotated channels at
+    3 bits, 64 at 2: 40-byte code rows)."""
+    st = build_stream_workload(tq, torch, kv_inputs, 0, 1, device, bits=2)
+    p, cache = st["params"], st["cache"]
+    ms = _time_call(torch, lambda: tq.tq_decode_attn(p, st["qs"][0], cache, st["cap"], st["out"], st["ws"]),
+                    iters, flush)
+    assert int(cache.status.item()) == 0
+    row = p.row_bytes(tq.TQ_K)[0] + 4
+    by = sum(HKV * n * 2 * row for n in st["lens"]) + 2 * N_SEQ * HQ * D * 2
+    out = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
+           "l2": "flushed between calls"}
+    del st, cache
     return out
 
 

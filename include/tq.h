@@ -67,8 +67,9 @@ typedef enum { TQ_ROT_HAAR = 0, TQ_ROT_HADAMARD = 1 } tq_rotation_kind;
  * asymmetric K/V setting of "Greetings from TurboQuant-MLX" (turboquant_plus
  * issue 59) and of the TurboQuant-MLX article, section "Cosa aggiunge").
  * bits_*: total bits per channel.  mixed_*: 1 puts the first d/2 rotated
- * channels at bits+1 ("3.5 bits per channel" with bits = 3, article section
- * "Il metodo TurboQuant, in breve"); MSE mode only.  seed drives Pi and S. */
+ * channels at bits+1 ("3.5 bits per channel" with bits = 3 and "2.5 bits per
+ * channel" with bits = 2, article section "Il metodo TurboQuant, in breve");
+ * MSE mode only, bits 2 or 3 (else TQ_ERR_UNSUPPORTED).  seed drives Pi and S. */
 typedef struct {
   int d;
   int bits_k, bits_v;
@@ -229,7 +230,9 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
  * their bf16 keys and values directly.  A sequence with no tokens gives a
  * zero output.  max_len: host bound on lens (longer sequences are cut to it
  * and bit 2 is set in cache->status).  n_sink above 4096 gives
- * TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the query rotation,
+ * TQ_ERR_UNSUPPORTED.  K/V formats with a decode kernel: equal formats
+ * (MSE 1..4 bits, mixed 2.5 and 3.5, prod 1..4) and the asymmetric MSE pairs
+ * K4/V3, K4/V2, K3/V2; any other pair gives TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the query rotation,
  * the persistent decode kernel and the merge; the last two are launched with
  * programmatic stream serialization and overlap their prologues with the
  * previous kernel's tail. */

@@ -658,6 +658,7 @@ __host__ __device__ constexpr uint64_t token_order(int kf, int vf) {
   return kf == 2 && vf == 2     ? 0xFE095427B86D1AC3ull
          : kf == 4 && vf == 4   ? 0xB2CD41F863905AE7ull
          : kf == 11 && vf == 11 ? 0x2AE619D534F8BC70ull
+         : kf == 10 && vf == 10 ? 0xA428EC6031F97DB5ull
          : kf == 18 && vf == 18 ? 0xB6C51FA82907D43Eull
          : kf == 4 && vf == 2   ? 0xB856274109A3DEFCull
          : kf == 3 && vf == 2   ? 0xC1B7502E948F3D6Aull
@@ -702,8 +703,8 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
     static_for<KR::S0::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      xa.template decode<s>(lk, lane4, lane8, c1k, la, ha);
-      xb.template decode<s>(lk, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s, T3W>(lk, lane4, lane8, c1k, la, ha);
+      xb.template decode<s, T3W>(lk, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x) mma16816(ca[(NX * s + x) & 1], la, lb, ha, hb, bq[s][0][x], bq[s][1][x]);
     });
@@ -712,11 +713,12 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
     typename KR::S1 xa, xb;
     xa.load(ka, t);
     xb.load(kb, t);
+    const uint32_t lk = FK::b1 == 2 ? lut_b : lut_a;
     static_for<KR::S1::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      xa.template decode<s, T3W>(lut_a, lane4, lane8, c1k, la, ha);
-      xb.template decode<s, T3W>(lut_a, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s, T3W>(lk, lane4, lane8, c1k, la, ha);
+      xb.template decode<s, T3W>(lk, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x)
         mma16816(ca[(NX * s + x + 1) & 1], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
@@ -809,8 +811,9 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
     xc.load(r8p, g);
     xd.load(r9p, g);
     uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
-    VR::S1::decode(xa, xb, lut_a, lane4, lane8, c1v, r0, r08);
-    VR::S1::decode(xc, xd, lut_a, lane4, lane8, c1v, r1, r18);
+    const uint32_t lut = FV::b1 == 2 ? lut_b : lut_a;
+    VR::S1::decode(xa, xb, lut, lane4, lane8, c1v, r0, r08);
+    VR::S1::decode(xc, xd, lut, lane4, lane8, c1v, r1, r18);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) mma16816(oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
   }
@@ -1795,6 +1798,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   TQ_CASE(fid(3, 0, 0), fid(3, 0, 0))
   TQ_CASE(fid(4, 0, 0), fid(4, 0, 0))
   TQ_CASE(fid(3, 1, 0), fid(3, 1, 0))
+  TQ_CASE(fid(2, 1, 0), fid(2, 1, 0))
   TQ_CASE(fid(0, 0, 1), fid(0, 0, 1))
   TQ_CASE(fid(1, 0, 1), fid(1, 0, 1))
   TQ_CASE(fid(2, 0, 1), fid(2, 0, 1))

@@ -241,7 +241,10 @@ static bool make_format(int bits, int mode, int mixed, FormatSpec* f, std::strin
   f->mixed = mixed;
   f->mse_bits = f->prod ? bits - 1 : bits;
   if (mixed && f->prod) { *why = "mixed rows are supported in MSE mode only"; return false; }
-  if (mixed && bits != 3) { *why = "mixed rows are supported for bits = 3 (3.5 bits per channel) only"; return false; }
+  if (mixed && bits != 2 && bits != 3) {
+    *why = "mixed rows are supported for bits = 2 and 3 (2.5 and 3.5 bits per channel) only";
+    return false;
+  }
   f->code_bytes = mixed ? 8 * (2 * f->mse_bits + 1) : 16 * f->mse_bits;
   f->qjl_bytes = f->prod ? kSketch / 8 : 0;
   return true;

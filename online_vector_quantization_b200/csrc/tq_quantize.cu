@@ -1022,10 +1022,10 @@ tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaSt
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core quantize kernel launch");
 }
 
-// bf16 rows: tensor-core rotation (MSE 1..4 bits, mixed 3.5, prod 1..4).
+// bf16 rows: tensor-core rotation (MSE 1..4 bits, mixed 2.5 and 3.5, prod 1..4).
 bool tc_eligible(const QuantArgs& a) {
   const bool fmt_ok = a.prod ? (!a.mixed && a.mse_bits >= 0 && a.mse_bits <= 3)
-                             : (a.mse_bits >= 1 && (a.mixed ? a.mse_bits == 3 : a.mse_bits <= 4));
+                             : (a.mse_bits >= 1 && (a.mixed ? (a.mse_bits == 2 || a.mse_bits == 3) : a.mse_bits <= 4));
   return a.x_bf16 && fmt_ok && a.n <= (int64_t(1) << 31) &&
          (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 && encode_tiled() != nullptr;
 }
@@ -1054,6 +1054,7 @@ tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
   switch (a.mse_bits * 2 + a.mixed) {
     case 2: return launch_tc<1, 0>(a, map, grid, st);
     case 4: return launch_tc<2, 0>(a, map, grid, st);
+    case 5: return launch_tc<2, 1>(a, map, grid, st);
     case 6: return launch_tc<3, 0>(a, map, grid, st);
     case 7: return launch_tc<3, 1>(a, map, grid, st);
     case 8: return launch_tc<4, 0>(a, map, grid, st);

@@ -69,6 +69,9 @@ def test_host_argument_errors():
         tq.Params(3, 3, mixed_k=1, mode_k=tq.TQ_MODE_PROD)
     assert e.value.status == 2
     with pytest.raises(tq.TqError) as e:
+        tq.Params(4, 4, mixed_k=1)
+    assert e.value.status == 2
+    with pytest.raises(tq.TqError) as e:
         tq.Params(3, 3, rotation=7)
     assert e.value.status == 1
     assert tq._lib.tq_cache_bytes(None, 1, 1, 64, 0) == 0

@@ -18,9 +18,9 @@ if not torch.cuda.is_available():  # collected on CPU machines, run on the GPU machine
 import online_vector_quantization_b200 as tq  # noqa: E402
 import gpu_util as gu  # noqa: E402
 
-FORMATS = [gu.fmt(1), gu.fmt(2), gu.fmt(3), gu.fmt(4), gu.fmt(3, mixed=True),
+FORMATS = [gu.fmt(1), gu.fmt(2), gu.fmt(3), gu.fmt(4), gu.fmt(3, mixed=True), gu.fmt(2, mixed=True),
            gu.fmt(1, prod=True), gu.fmt(2, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True)]
-FMT_IDS = ["mse1", "mse2", "mse3", "mse4", "mixed3.5", "prod1", "prod2", "prod3", "prod4"]
+FMT_IDS = ["mse1", "mse2", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod1", "prod2", "prod3", "prod4"]
 
 
 @pytest.mark.parametrize("f", FORMATS, ids=FMT_IDS)
@@ -135,12 +135,13 @@ DECODE_FORMATS = [
     (gu.fmt(2), gu.fmt(2)),
     (gu.fmt(1), gu.fmt(1)),
     (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)),
+    (gu.fmt(2, mixed=True), gu.fmt(2, mixed=True)),
     (gu.fmt(3, prod=True), gu.fmt(3, prod=True)),
     (gu.fmt(2, prod=True), gu.fmt(2, prod=True)),
     (gu.fmt(4, prod=True), gu.fmt(4, prod=True)),
     (gu.fmt(1, prod=True), gu.fmt(1, prod=True)),
 ]
-DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "mixed", "prod3", "prod2", "prod4", "prod1"]
+DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "mixed", "mixed2.5", "prod3", "prod2", "prod4", "prod1"]
 
 
 @pytest.mark.parametrize("fk,fv", DECODE_FORMATS, ids=DEC_IDS)
@@ -198,7 +199,9 @@ def test_decode_length_above_bound_sets_status():
 
 
 @pytest.mark.parametrize("fk,fv,n_sink", [(gu.fmt(4), gu.fmt(3), 8), (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True), 0),
-                                          (gu.fmt(3, prod=True), gu.fmt(3, prod=True), 0)], ids=["k4v3sink", "mixed", "prod3"])
+                                          (gu.fmt(2, mixed=True), gu.fmt(2, mixed=True), 4),
+                                          (gu.fmt(3, prod=True), gu.fmt(3, prod=True), 0)],
+                         ids=["k4v3sink", "mixed", "mixed2.5sink", "prod3"])
 def test_append_parity(fk, fv, n_sink):
     gp, op = gu.make_params(fk, fv)
     n_seq, hkv, cap = 3, 2, 256

@@ -229,6 +229,24 @@ def test_distortion_bounds_and_page_cosines():
         assert round(math.sqrt(1 - o.mse_distortion(book(128, b))), 3) == cos
 
 
+@pytest.mark.parametrize("b", [2, 3])
+def test_mixed_row_distortion_is_mean_of_its_two_widths(b):
+    # "3.5 / 2.5 bits per channel" (article, "Il metodo TurboQuant, in
+    # breve"): half the rotated coordinates at b+1 bits, half at b.  For
+    # uniform unit vectors every rotated coordinate follows the sphere law, so
+    # the expected squared error of the round trip is (D_b + D_{b+1}) / 2.
+    fmt = o.Format(b, mixed=True)
+    p = o.Params(128, fmt, fmt)
+    rng = np.random.default_rng(40 + b)
+    u = rng.standard_normal((8192, 128))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    err = np.sum((o.dequantize(p, o.quantize(p, u, "k"), "k") - u) ** 2, axis=1)
+    want = 0.5 * (o.mse_distortion(book(128, b)) + o.mse_distortion(book(128, b + 1)))
+    assert abs(err.mean() - want) < 5 * err.std() / math.sqrt(err.size)
+    # and it lies strictly between the two uniform widths' distortions
+    assert o.mse_distortion(book(128, b + 1)) < err.mean() < o.mse_distortion(book(128, b))
+
+
 def test_end_to_end_cosine_matches_pages():
     p = o.Params(128, o.Format(3), o.Format(4))
     for row in _table("pages_cosine.txt"):
@@ -243,7 +261,7 @@ def test_end_to_end_cosine_matches_pages():
 # ---- quantize / pack -------------------------------------------------------
 
 @pytest.mark.parametrize("fmt", [o.Format(1), o.Format(2), o.Format(3), o.Format(4),
-                                 o.Format(3, mixed=True), o.Format(3, prod=True)])
+                                 o.Format(3, mixed=True), o.Format(2, mixed=True), o.Format(3, prod=True)])
 def test_quantize_is_brute_force_nearest_centroid(fmt):
     p = o.Params(128, fmt, fmt)
     x = kv_inputs.kv_vectors(64, 128, key="bf", dtype=torch.bfloat16).double().numpy()
@@ -270,20 +288,23 @@ def test_pack_golden_b3():
     assert np.array_equal(o.unpack_codes(got, [3] * 128), codes)
 
 
-def test_pack_golden_mixed():
-    rows = _kv("pack_mixed43.txt")
+@pytest.mark.parametrize("name,bits,row", [("pack_mixed43.txt", 3, 56), ("pack_mixed32.txt", 2, 40)])
+def test_pack_golden_mixed(name, bits, row):
+    rows = _kv(name)
     codes = np.zeros((1, 128), dtype=np.int64)
     for kv in rows["set"].split():
         j, c = kv.split("=")
         codes[0, int(j)] = int(c)
-    want = bytearray(56)
+    want = bytearray(row)
     for kv in rows["bytes"].split():
         i, v = kv.split("=")
         want[int(i)] = int(v, 16)
-    fmt = o.Format(3, mixed=True)
+    fmt = o.Format(bits, mixed=True)
     widths = [fmt.mse_bits(j, 128) for j in range(128)]
-    assert fmt.code_bytes(128) == 56
-    assert o.pack_codes(codes, widths).tobytes() == bytes(want)
+    assert fmt.code_bytes(128) == row
+    got = o.pack_codes(codes, widths)
+    assert got.tobytes() == bytes(want)
+    assert np.array_equal(o.unpack_codes(got, widths), codes)
 
 
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
