@@ -76,7 +76,8 @@ struct Fmt {
 // all 256 rows anyway (t3_wide), every row r holds the entry of r & 63, so a
 // 3-bit pair in the low six bits of any byte is looked up with one byte
 // permute.  Region B (row stride 256 B, 8 B per lane): four 2-bit centroids of
-// byte r.  Entry (r, lane) sits at r*256 + lane*4 (or *8): every lane hits its
+// byte r.  With 2- and 3-bit widths only (t2a), bytes [0, 128) of region A row
+// r hold half2(c2[r & 3], c2[(r >> 2) & 3]) instead, and there is no region B.  Entry (r, lane) sits at r*256 + lane*4 (or *8): every lane hits its
 // own bank.
 template <int KF, int VF>
 struct Lut {
@@ -85,8 +86,11 @@ struct Lut {
   static constexpr bool t2 = Fmt<KF>::uses(2) || Fmt<VF>::uses(2);
   static constexpr int region_a = (t4 || (t3 && t2)) ? 65536 : (t3 ? 16384 : 0);
   static constexpr bool t3_wide = t3 && region_a == 65536;
+  // 2-bit and 3-bit widths without 4-bit ones: the 2-bit pair table takes the
+  // free bytes [0, 128) of region A instead of a region B of its own
+  static constexpr bool t2a = t2 && t3 && !t4;
   static constexpr int region_b_off = region_a;  // 0 or 65536: a 64 KB boundary
-  static constexpr int bytes = region_a + (t2 ? 65536 : 0);
+  static constexpr int bytes = region_a + (t2 && !t2a ? 65536 : 0);
 };
 
 // The tables live at shared-window address kLutAddr (64 KB aligned), so a
@@ -249,7 +253,9 @@ struct KChunk {
   // T3W (3-bit): the pair table spans 256 rows, so the pair at bit 12S (6,
   // 30: after a 6-bit shift; 12, 36 / 18, 42: after 12 / 18) is the low six
   // bits of byte 0 or 3 of w[0] or of a funnel shift of (w[0], w[1]).
-  template <int S, bool T3W = false>
+  // T2A (2-bit): the pair table in region A; the pair in the high nibble of a
+  // byte is looked up after a 4-bit shift of the word.
+  template <int S, bool T3W = false, bool T2A = false>
   __device__ __forceinline__ void decode(uint32_t smem, uint32_t lane4, uint32_t lane8,
                                          uint32_t c_bits, uint32_t& lo, uint32_t& hi) const {
     constexpr int s = S;
@@ -268,6 +274,10 @@ struct KChunk {
     } else if constexpr (B == 3) {
       lo = lut32(smem, pair3<2 * S>(lane4 + 128));
       hi = lut32(smem, pair3<2 * S + 1>(lane4 + 128));
+    } else if constexpr (B == 2 && T2A) {
+      const uint32_t ww = w[s >> 2];
+      lo = lut32(smem, byte_addr(ww, lane4, s & 3));
+      hi = lut32(smem, byte_addr(ww >> 4, lane4, s & 3));
     } else if constexpr (B == 2) {
       const uint2 v = lut64(smem, byte_addr(w[s >> 2], lane8, s & 3));
       lo = v.x;
@@ -319,6 +329,7 @@ struct VChunk {
   }
 
   // rows g (coordinate 2mt) and g+8 (2mt+1) for every m-tile, tokens (A, B)
+  template <bool T2A = false>
   __device__ __forceinline__ static void decode(const VChunk& a, const VChunk& b, uint32_t smem,
                                                 uint32_t lane4, uint32_t lane8, uint32_t c_bits,
                                                 uint32_t (&rg)[MT], uint32_t (&rg8)[MT]) {
@@ -357,12 +368,19 @@ struct VChunk {
       const uint32_t od = ((xa >> 2) & 0x33333333u) | (xb & 0xCCCCCCCCu);
 #pragma unroll
       for (int j = 0; j < MT / 2; ++j) {
-        const uint2 e = lut64(smem, byte_addr(ev, lane8, j));
-        const uint2 o = lut64(smem, byte_addr(od, lane8, j));
-        rg[2 * j] = e.x;
-        rg[2 * j + 1] = e.y;
-        rg8[2 * j] = o.x;
-        rg8[2 * j + 1] = o.y;
+        if constexpr (T2A) {
+          rg[2 * j] = lut32(smem, byte_addr(ev, lane4, j));
+          rg[2 * j + 1] = lut32(smem, byte_addr(ev >> 4, lane4, j));
+          rg8[2 * j] = lut32(smem, byte_addr(od, lane4, j));
+          rg8[2 * j + 1] = lut32(smem, byte_addr(od >> 4, lane4, j));
+        } else {
+          const uint2 e = lut64(smem, byte_addr(ev, lane8, j));
+          const uint2 o = lut64(smem, byte_addr(od, lane8, j));
+          rg[2 * j] = e.x;
+          rg[2 * j + 1] = e.y;
+          rg8[2 * j] = o.x;
+          rg8[2 * j + 1] = o.y;
+        }
       }
     } else {
       const uint32_t wv = (static_cast<uint32_t>(a.x) & 0xFFFFu) | (static_cast<uint32_t>(b.x) << 16);
@@ -680,7 +698,7 @@ __device__ __forceinline__ TokRows tok_rows(int g, int t) {
 // Scores of one 16-token subtile whose rows start at `srow` of the staged
 // planes: s2 (base 2) for tokens g (s2[0], s2[1]) and g+8 (s2[2], s2[3]),
 // columns 2t, 2t+1; masked tokens get -inf.  Two MMA accumulator chains.
-template <int KF, bool PACK, bool T3W>
+template <int KF, bool PACK, bool T3W, bool T2A>
 __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
                                                int g, int t,
                                                const QFrag<PACK>& bq, const QFrag<PACK>& bqs,
@@ -703,8 +721,8 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
     static_for<KR::S0::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      xa.template decode<s, T3W>(lk, lane4, lane8, c1k, la, ha);
-      xb.template decode<s, T3W>(lk, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s, T3W, T2A>(lk, lane4, lane8, c1k, la, ha);
+      xb.template decode<s, T3W, T2A>(lk, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x) mma16816(ca[(NX * s + x) & 1], la, lb, ha, hb, bq[s][0][x], bq[s][1][x]);
     });
@@ -717,8 +735,8 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
     static_for<KR::S1::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
       uint32_t la, ha, lb, hb;
-      xa.template decode<s, T3W>(lk, lane4, lane8, c1k, la, ha);
-      xb.template decode<s, T3W>(lk, lane4, lane8, c1k, lb, hb);
+      xa.template decode<s, T3W, T2A>(lk, lane4, lane8, c1k, la, ha);
+      xb.template decode<s, T3W, T2A>(lk, lane4, lane8, c1k, lb, hb);
 #pragma unroll
       for (int x = 0; x < NX; ++x)
         mma16816(ca[(NX * s + x + 1) & 1], la, lb, ha, hb, bq[KR::S0::KSTEPS + s][0][x], bq[KR::S0::KSTEPS + s][1][x]);
@@ -772,7 +790,7 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
 
 // O^T += C_v^T P'^T for one 16-token subtile (rows from `srow`); p holds the
 // softmax weights of tokens g (p[0], p[1]) and g+8 (p[2], p[3]).
-template <int VF, int VMT>
+template <int VF, int VMT, bool T2A>
 __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
                                            int g, int t,
                                            const float (&p)[4], uint32_t lut_a,
@@ -798,8 +816,8 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
     xd.load(r9p, g);
     uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
     const uint32_t lut = FV::b0 == 2 ? lut_b : lut_a;
-    VR::S0::decode(xa, xb, lut, lane4, lane8, c1v, r0, r08);
-    VR::S0::decode(xc, xd, lut, lane4, lane8, c1v, r1, r18);
+    VR::S0::template decode<T2A>(xa, xb, lut, lane4, lane8, c1v, r0, r08);
+    VR::S0::template decode<T2A>(xc, xd, lut, lane4, lane8, c1v, r1, r18);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) mma16816(oacc[mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
   }
@@ -812,8 +830,8 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
     xd.load(r9p, g);
     uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
     const uint32_t lut = FV::b1 == 2 ? lut_b : lut_a;
-    VR::S1::decode(xa, xb, lut, lane4, lane8, c1v, r0, r08);
-    VR::S1::decode(xc, xd, lut, lane4, lane8, c1v, r1, r18);
+    VR::S1::template decode<T2A>(xa, xb, lut, lane4, lane8, c1v, r0, r08);
+    VR::S1::template decode<T2A>(xc, xd, lut, lane4, lane8, c1v, r1, r18);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) mma16816(oacc[VR::S0::MT + mt], r0[mt], r08[mt], r1[mt], r18[mt], pb0, pb1);
   }
@@ -852,9 +870,9 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
   const bool ok0A = row0 + tr.kA < nq, ok0B = row0 + tr.kB < nq;
   const bool ok1A = row0 + kTok + tr.kA < nq, ok1B = row0 + kTok + tr.kB < nq;
   float s0[4], s1[4];
-  subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
+  subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
   if constexpr (second)
-    subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
+    subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
   // online softmax over the 32 tokens (base 2), columns 2t and 2t+1.  The
@@ -898,9 +916,9 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
     W.l1 += (p0[1] + p0[3]) + (p1[1] + p1[3]);
   }
   if constexpr (!SPARSE) {
-    subtile_pv<VF, VMT>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+    subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if constexpr (second)
-      subtile_pv<VF, VMT>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   } else {
     // sparse V: exp(s - m) / l over the tokens seen so far bounds the final
     // weight, and this lane's partial sum is at most l, so p < thr * l_lane
@@ -914,9 +932,9 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
       p1[i + 1] = p1[i + 1] >= c1 ? p1[i + 1] : 0.f;
     }
     if (__any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f))
-      subtile_pv<VF, VMT>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if (second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f))
-      subtile_pv<VF, VMT>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   }
 }
 
@@ -1565,7 +1583,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
         *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
       }
     }
-    if constexpr (L::t2) {
+    if constexpr (L::t2a) {
+      for (int i = tid; i < 256 * 32; i += NTC) {
+        const int r = i >> 5, ln = i & 31;
+        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) =
+            h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
+      }
+    } else if constexpr (L::t2) {
       for (int i = tid; i < 256 * 32; i += NTC) {
         const int r = i >> 5, ln = i & 31;
         uint2 v;

@@ -134,6 +134,8 @@ DECODE_FORMATS = [
     (gu.fmt(4), gu.fmt(4)),
     (gu.fmt(2), gu.fmt(2)),
     (gu.fmt(1), gu.fmt(1)),
+    (gu.fmt(3), gu.fmt(2)),
+    (gu.fmt(4), gu.fmt(2)),
     (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)),
     (gu.fmt(2, mixed=True), gu.fmt(2, mixed=True)),
     (gu.fmt(3, prod=True), gu.fmt(3, prod=True)),
@@ -141,7 +143,7 @@ DECODE_FORMATS = [
     (gu.fmt(4, prod=True), gu.fmt(4, prod=True)),
     (gu.fmt(1, prod=True), gu.fmt(1, prod=True)),
 ]
-DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "mixed", "mixed2.5", "prod3", "prod2", "prod4", "prod1"]
+DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "k3v2", "k4v2", "mixed", "mixed2.5", "prod3", "prod2", "prod4", "prod1"]
 
 
 @pytest.mark.parametrize("fk,fv", DECODE_FORMATS, ids=DEC_IDS)
