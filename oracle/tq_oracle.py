@@ -495,3 +495,32 @@ def decode_attention(p: Params, q: np.ndarray, cache: Cache, lens, hkv: int,
         for h in hs:
             out[b, h] = attend_one(q[b, h], keys, vals, ns, sparse_v_threshold)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Inner-product search over a quantized database.  [P3] "Il metodo TurboQuant,
+# in breve": besides the KV cache, the paper applies the quantizer to
+# similarity search, in place of product quantization.  [reading] The score of
+# a database row for a query is the inner product of the query with the row's
+# reconstruction, <q, x_hat> (in prod mode the unbiased estimate of <q, x>);
+# a search returns the k best rows per query, larger score first, equal scores
+# in row order, and pads with score -inf and row -1 when the database holds
+# fewer than k rows.
+# ---------------------------------------------------------------------------
+
+def ip_scores(p: Params, q: np.ndarray, pk: Packed, which: str = "k") -> np.ndarray:
+    """Scores (Q, n) of queries q (Q, d) against the packed rows pk."""
+    return np.asarray(q, dtype=np.float64) @ dequantize(p, pk, which).T
+
+
+def ip_search(p: Params, q: np.ndarray, pk: Packed, k: int, which: str = "k"):
+    """Top-k rows per query: (scores (Q, k), rows (Q, k))."""
+    s = ip_scores(p, q, pk, which)
+    nq, n = s.shape
+    scores = np.full((nq, k), -np.inf)
+    rows = np.full((nq, k), -1, dtype=np.int64)
+    for i in range(nq):
+        order = np.lexsort((np.arange(n), -s[i]))[:k]  # score descending, then row ascending
+        scores[i, :order.size] = s[i, order]
+        rows[i, :order.size] = order
+    return scores, rows

@@ -466,3 +466,48 @@ def test_decode_attention_gqa_sink_and_rotated_domain_identity():
             assert np.allclose(keys[ns:] @ q[b, h], s_rot, rtol=1e-10, atol=1e-10)
             vals = np.concatenate([v[b, g, :ns], o.dequantize(p, vr, "v")[:n - ns]])
             assert np.allclose(out[b, h], _loops_attention(q[b, h], keys, vals, ns, 0.0), atol=1e-12)
+
+
+# ---- inner-product search ----------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [o.Format(3), o.Format(2, mixed=True)])
+def test_ip_search_is_brute_force_top_k(fmt):
+    # brute force in the rotated domain: score = nu * sum_j (Pi q)_j c[idx_j]
+    # (no reconstruction, no Pi^T), then a plain sort by (-score, row)
+    p = o.Params(128, fmt, fmt)
+    x = kv_inputs.kv_vectors(61, 128, key="ipb").double().numpy()
+    x[40] = x[3]  # exact ties: the lower row comes first
+    x[41] = x[3]
+    pk = o.quantize(p, x, "k")
+    widths = [fmt.mse_bits(j, 128) for j in range(128)]
+    idx = o.unpack_codes(pk.codes, widths)
+    q = np.random.default_rng(6).standard_normal((4, 128))
+    q[1] = 3.0 * x[3] / np.linalg.norm(x[3])  # the tied rows are this query's best
+    want_s = np.zeros((4, 61))
+    for i in range(4):
+        qr = p.pi @ q[i]
+        for r in range(61):
+            acc = 0.0
+            for j in range(128):
+                acc += qr[j] * p.books[widths[j]].centroids[idx[r, j]]
+            want_s[i, r] = float(pk.norms[r]) * acc
+    assert np.max(np.abs(o.ip_scores(p, q, pk) - want_s)) < 1e-12 * np.max(np.abs(want_s))
+    scores, rows = o.ip_search(p, q, pk, 9)
+    for i in range(4):
+        brute = sorted(range(61), key=lambda r: (-want_s[i, r], r))[:9]
+        assert rows[i].tolist() == brute
+        assert np.allclose(scores[i], want_s[i, brute], rtol=1e-12, atol=0)
+    assert rows[1, :3].tolist() == [3, 40, 41]
+
+
+def test_ip_search_pads_short_databases():
+    fmt = o.Format(2, prod=True)
+    p = o.Params(128, fmt, fmt)
+    x = kv_inputs.kv_vectors(3, 128, key="ips").double().numpy()
+    q = np.random.default_rng(7).standard_normal((2, 128))
+    scores, rows = o.ip_search(p, q, o.quantize(p, x, "k"), 5)
+    assert (rows[:, 3:] == -1).all() and np.isneginf(scores[:, 3:]).all()
+    assert sorted(rows[0, :3].tolist()) == [0, 1, 2]
+    empty = o.quantize(p, np.zeros((0, 128)), "k")
+    scores, rows = o.ip_search(p, q, empty, 4)
+    assert (rows == -1).all() and np.isneginf(scores).all()
