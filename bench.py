@@ -335,7 +335,7 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "stream-2.5")
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "stream-2.5", "search")
 
 
 def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
@@ -355,6 +355,8 @@ def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
         out["decode_tiny_fp32_T4096"] = _aux_tiny(tq, torch, kv_inputs, device, iters)
     if only in (None, "stream-2.5"):
         out["decode_mixed2.5_stream_shapes"] = _aux_stream25(tq, torch, kv_inputs, device, flush, iters)
+    if only in (None, "search"):
+        out["ip_search_4M"] = _aux_search(tq, torch, kv_inputs, device, flush, iters, formats)
     if only in (None, "bf16-sdpa"):
         out["bf16_kv_decode_sdpa_stream_shapes"] = _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters)
     return out
@@ -449,6 +451,38 @@ def _aux_stream25(tq, torch, kv_inputs, device, flush, iters):
     out = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
            "l2": "flushed between calls"}
     del st, cache
+    return out
+
+
+def _aux_search(tq, torch, kv_inputs, device, flush, iters, formats):
+    """Inner-product search: a database of 2^22 vectors (d = 128, bf16 with
+    lognormal norms and outlier channels, quantized on the GPU), top-10 rows
+    for 8 and for 32 bf16 queries; bytes are the packed rows read once per
+    group of 8 queries."""
+    n = 1 << 22
+    x = kv_inputs.kv_vectors(n, D, key="search-db", device=device, dtype=torch.bfloat16, outliers=True)
+    out = {}
+    ws = tq.search_workspace(device=device)
+    for name, bits, mode in (("prod3", 3, tq.TQ_MODE_PROD), ("mse4", 4, tq.TQ_MODE_MSE)):
+        if formats and name not in formats:
+            continue
+        p = tq.Params(bits, bits, mode, mode)
+        pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
+        tq.tq_quantize(p, x, tq.TQ_K, pk)
+        cb, qb = p.row_bytes(tq.TQ_K)
+        row = cb + 4 + (qb + 4 if qb else 0)
+        for nq in (8, 32):
+            q = kv_inputs.queries((nq, D), key=("search-q", nq), device=device)
+            sc = torch.empty(nq, 10, device=device)
+            rw = torch.empty(nq, 10, dtype=torch.int64, device=device)
+            ms = _time_call(torch, lambda: tq.tq_search(p, tq.TQ_K, pk, n, q, 10, sc, rw, ws), iters, flush)
+            by = n * row * ((nq + 7) // 8)
+            out[f"{name}_q{nq}_k10"] = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1),
+                                        "bytes": by, "queries_per_s": round(nq / (ms * 1e-3), 1)}
+        assert p.status() == 0
+        del pk
+    del x
+    out["l2"] = "flushed between calls"
     return out
 
 

@@ -261,6 +261,36 @@ tq_status tq_decode_attn_noalloc(const tq_params* p, const void* q, int q_dtype,
 /* Message for the last failed call on this host thread ("" if none). */
 const char* tq_last_error(void);
 
+/* ---- inner-product search ---------------------------------------------- */
+
+/* Workspace bytes of tq_search on the current device (the same for every
+ * database size and number of queries). */
+size_t tq_search_workspace_bytes(void);
+
+/* Top-k inner-product search over a database of n rows quantized with the
+ * `which` format of p (tq_quantize output: device planes, 16-byte aligned),
+ * the second application of the quantizer in the TurboQuant-MLX article,
+ * section "Il metodo TurboQuant, in breve" (similarity search in place of
+ * product quantization).  Row i scores <q_j, x^_i> for query j, the inner
+ * product with the row's reconstruction: ||x_i|| (<Pi q_j, c[idx_i]> +
+ * sqrt(pi/2)/m ||r_i|| <S q_j, z_i>) in prod mode (the unbiased estimate of
+ * <q_j, x_i>), the first term alone in MSE mode.
+ *   q:      [n_queries][d] (q_dtype), device, 16-byte aligned.
+ *   scores: [n_queries][k] fp32, rows: [n_queries][k] int64, device,
+ *           caller-owned: per query the k best rows, larger score first,
+ *           equal scores in row order; with n < k the tail holds score -inf
+ *           and row -1.
+ * Scores come from fp16 tensor-core products with fp32 accumulation: rows
+ * whose scores differ by less than about 1e-3 of ||q|| ||x|| may come in
+ * either order.  1 <= k <= 32 (TQ_ERR_UNSUPPORTED above), 0 <= n < 2^31,
+ * n_queries >= 1 (the database is read once per group of 8 queries).
+ * workspace: device, >= tq_search_workspace_bytes() bytes, 16-byte aligned;
+ * calls sharing it must not overlap.  Asynchronous on `stream`; error bits
+ * go to the params status word (tq_params_status). */
+tq_status tq_search(const tq_params* p, int which, const tq_packed* db, int64_t n, const void* q, int q_dtype,
+                    int n_queries, int k, float* scores, int64_t* rows, void* workspace, size_t ws_bytes,
+                    void* stream);
+
 #ifdef __cplusplus
 }
 #endif

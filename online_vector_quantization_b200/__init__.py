@@ -82,6 +82,9 @@ _SIGS = {
                                c_int, c_void_p, c_size_t, ctypes.POINTER(TqAttnFlags), c_void_p]),
     "tq_decode_attn_noalloc": (c_int, [c_void_p, c_void_p, c_int, ctypes.POINTER(TqCache), c_int, c_int, c_int,
                                        c_void_p, c_int, ctypes.POINTER(TqAttnFlags), c_void_p]),
+    "tq_search_workspace_bytes": (c_size_t, []),
+    "tq_search": (c_int, [c_void_p, c_int, ctypes.POINTER(TqPacked), c_int64, c_void_p, c_int, c_int, c_int,
+                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "tq_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -293,3 +296,25 @@ def tq_decode_attn_noalloc(params: Params, q, cache: Cache, max_len: int, out, s
     flags = TqAttnFlags(sparse_v_threshold, 0)
     _check(_lib.tq_decode_attn_noalloc(params.handle, _ptr(q), _dtype_code(q), ctypes.byref(cache.struct), B, hq,
                                        max_len, _ptr(out), _dtype_code(out), ctypes.byref(flags), _stream(stream)))
+
+
+# ---- inner-product search ----------------------------------------------------
+
+def tq_search_workspace_bytes() -> int:
+    return _lib.tq_search_workspace_bytes()
+
+
+def search_workspace(device="cuda"):
+    """Allocate a workspace for tq_search."""
+    import torch
+    return torch.empty(tq_search_workspace_bytes(), dtype=torch.uint8, device=device)
+
+
+def tq_search(params: Params, which: int, db: Packed, n: int, q, k: int, scores, rows, workspace, stream=None):
+    """q: (n_queries, d) CUDA tensor (fp32 or bf16); scores: (n_queries, k)
+    fp32 and rows: (n_queries, k) int64 CUDA tensors."""
+    assert q.is_contiguous() and scores.is_contiguous() and rows.is_contiguous()
+    st = db.struct()
+    _check(_lib.tq_search(params.handle, which, ctypes.byref(st), n, _ptr(q), _dtype_code(q), q.shape[0], k,
+                          _ptr(scores), _ptr(rows), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(stream)))

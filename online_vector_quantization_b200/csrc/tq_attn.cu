@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "tq_internal.h"
 #include "tq_sm100.cuh"
@@ -442,6 +443,13 @@ struct DecodeArgs {
   float sparse_thr;
   int pack;          // 1: group <= 4, query hi/lo halves share one MMA (columns g and g+4)
   uint32_t dyn_bytes;  // dynamic shared memory granted to the decode kernel
+  float qscale;      // factor on the rotated query: log2(e)/sqrt(d) for attention, 1 for search
+  // inner-product search only
+  int64_t n_db;            // database rows (k_* planes)
+  int topk;                // k <= kSearchMaxK
+  uint64_t* cand;          // per (query, CTA) candidate lists [group][ctas][32]
+  float* out_scores;       // [group][topk]
+  int64_t* out_rows;       // [group][topk]
 };
 
 __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
   }
   cp_async_wait_all();
   __syncthreads();
-  const float scale = kLog2e * rsqrtf(static_cast<float>(kDim));
+  const float scale = a.qscale;
   // thread (j, ks) sums k in [ks * 32, ks * 32 + 32) for output coordinate j
   // of every head; the slices are added in shared memory
   const int j = tid & (kDim - 1), ks = tid >> 7;
@@ -1411,6 +1419,42 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   }
 }
 
+// The lookup tables of a format pair (see Lut), written by the consumer
+// threads (thread index tid < kConsumers * 32) from the sigma-scaled
+// centroids cb staged in shared memory.
+template <typename L>
+__device__ __forceinline__ void build_luts(unsigned char* lut_mem, const float* cb, int tid) {
+  constexpr int NTC = kConsumers * 32;
+  if constexpr (L::t4) {
+    for (int i = tid; i < 256 * 32; i += NTC) {
+      const int r = i >> 5, ln = i & 31;
+      *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
+    }
+  }
+  if constexpr (L::t3) {
+    constexpr int rows = L::t3_wide ? 256 : 64;
+    for (int i = tid; i < rows * 32; i += NTC) {
+      const int r = i >> 5, ln = i & 31, e = r & 63;
+      *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
+    }
+  }
+  if constexpr (L::t2a) {
+    for (int i = tid; i < 256 * 32; i += NTC) {
+      const int r = i >> 5, ln = i & 31;
+      *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) =
+          h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
+    }
+  } else if constexpr (L::t2) {
+    for (int i = tid; i < 256 * 32; i += NTC) {
+      const int r = i >> 5, ln = i & 31;
+      uint2 v;
+      v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
+      v.y = h2bits(cb[2 * kBookSlots + ((r >> 4) & 3)], cb[2 * kBookSlots + (r >> 6)]);
+      *reinterpret_cast<uint2*>(lut_mem + L::region_b_off + r * 256 + ln * 8) = v;
+    }
+  }
+}
+
 template <int KF, int VF, bool PACK, bool SPARSE>
 __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
@@ -1567,38 +1611,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   }
 
   // ---- lookup tables (consumer threads)
-  {
-    constexpr int NTC = kConsumers * 32;
-    const float* cb = s_cb;
-    if constexpr (L::t4) {
-      for (int i = tid; i < 256 * 32; i += NTC) {
-        const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb[4 * kBookSlots + (r & 15)], cb[4 * kBookSlots + (r >> 4)]);
-      }
-    }
-    if constexpr (L::t3) {
-      constexpr int rows = L::t3_wide ? 256 : 64;
-      for (int i = tid; i < rows * 32; i += NTC) {
-        const int r = i >> 5, ln = i & 31, e = r & 63;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + 128 + ln * 4) = h2bits(cb[3 * kBookSlots + (e & 7)], cb[3 * kBookSlots + (e >> 3)]);
-      }
-    }
-    if constexpr (L::t2a) {
-      for (int i = tid; i < 256 * 32; i += NTC) {
-        const int r = i >> 5, ln = i & 31;
-        *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) =
-            h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
-      }
-    } else if constexpr (L::t2) {
-      for (int i = tid; i < 256 * 32; i += NTC) {
-        const int r = i >> 5, ln = i & 31;
-        uint2 v;
-        v.x = h2bits(cb[2 * kBookSlots + (r & 3)], cb[2 * kBookSlots + ((r >> 2) & 3)]);
-        v.y = h2bits(cb[2 * kBookSlots + ((r >> 4) & 3)], cb[2 * kBookSlots + (r >> 6)]);
-        *reinterpret_cast<uint2*>(lut_mem + L::region_b_off + r * 256 + ln * 8) = v;
-      }
-    }
-  }
+  build_luts<L>(lut_mem, s_cb, tid);
   consumers_sync();  // tables complete
 
   // ---- consumers
@@ -1675,6 +1688,340 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// 4. Inner-product search over a quantized database (the method page's second
+//    application: similarity search in place of product quantization).  Every
+//    database row is scored with the estimator the decode kernel uses,
+//    <q, x^> = ||x|| (<Pi q, c[idx]> + sqrt(pi/2)/m ||r|| <S q, z>) (query
+//    scale 1 instead of log2(e)/sqrt(d)), and the k best rows per query are
+//    kept: larger score first, equal scores in row order.
+//
+//    search_kernel: persistent, the decode kernel's producer / consumer
+//    pipeline over contiguous ranges of database chunks (K planes only).
+//    Each consumer warp keeps, per query, its best candidates as a sorted
+//    column across its lanes (lane j = j-th best); a subtile's scores are
+//    first tested against the lanes' thresholds (the k-th best score) with one
+//    vote, and only candidates that pass are inserted.  At the end the 15
+//    warps' lists of each query are merged into the CTA's list.
+//    search_merge_kernel: one CTA per query merges the CTAs' lists.
+// ---------------------------------------------------------------------------
+constexpr int kSearchMaxK = 32;      // one list entry per lane
+constexpr int kSearchMaxCtas = 256;  // bound on the search grid (merge stages all lists)
+
+// Candidate key: the score in an order-preserving unsigned form above the
+// complemented row, so a larger key is a better candidate (ties on the score
+// go to the lower row).  0 stands for "no candidate".
+__device__ __forceinline__ uint64_t cand_key(float v, uint32_t row) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(o) << 32) | static_cast<uint64_t>(~row);
+}
+__device__ __forceinline__ float key_score(uint64_t key) {
+  if (key == 0) return -INFINITY;
+  const uint32_t o = static_cast<uint32_t>(key >> 32);
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+__device__ __forceinline__ int64_t key_row(uint64_t key) {
+  return key == 0 ? -1 : static_cast<int64_t>(~static_cast<uint32_t>(key));
+}
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+
+// Insert the candidates cA, cB (0: none) of the lanes into one query's list.
+// Lanes below k hold the list; a candidate that does not beat entry k-1 is
+// dropped.
+__device__ __forceinline__ void topk_offer(uint64_t& list, uint64_t cA, uint64_t cB, int lane, int k) {
+  unsigned mA = __ballot_sync(0xffffffffu, cA != 0);
+  unsigned mB = __ballot_sync(0xffffffffu, cB != 0);
+  while (mA | mB) {
+    const bool fromA = mA != 0;
+    const int src = __ffs(fromA ? mA : mB) - 1;
+    const uint64_t c = __shfl_sync(0xffffffffu, fromA ? cA : cB, src);
+    if (fromA)
+      mA &= mA - 1;
+    else
+      mB &= mB - 1;
+    const int pos = __popc(__ballot_sync(0xffffffffu, list > c));
+    const uint64_t up = __shfl_up_sync(0xffffffffu, list, 1);
+    if (pos < k) {
+      if (lane == pos)
+        list = c;
+      else if (lane > pos)
+        list = up;
+    }
+  }
+}
+
+// Offer one 16-token subtile: lane (g, t) holds the scores of rows rowA
+// (s[0], s[1]) and rowB (s[2], s[3]) for queries 2t and 2t + 1; thr0 / thr1
+// are the current k-th best scores of those two queries (-inf while a list
+// is not full).
+template <int G>
+__device__ __forceinline__ void offer_subtile(uint64_t (&list)[G], float& thr0, float& thr1, const float (&s)[4],
+                                              bool okA, bool okB, uint32_t rowA, uint32_t rowB, int t, int lane,
+                                              int Q, int k) {
+  const bool pass = (2 * t < Q && ((okA && s[0] >= thr0) || (okB && s[2] >= thr0))) ||
+                    (2 * t + 1 < Q && ((okA && s[1] >= thr1) || (okB && s[3] >= thr1)));
+  if (!__any_sync(0xffffffffu, pass)) return;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    if (h >= Q) break;
+    const bool own = t == (h >> 1);
+    const float th = (h & 1) ? thr1 : thr0;
+    const float va = s[h & 1], vb = s[2 + (h & 1)];
+    const uint64_t cA = (own && okA && va >= th) ? cand_key(va, rowA) : 0;
+    const uint64_t cB = (own && okB && vb >= th) ? cand_key(vb, rowB) : 0;
+    topk_offer(list[h], cA, cB, lane, k);
+    const float kth = key_score(__shfl_sync(0xffffffffu, list[h], k - 1));
+    if (own) {
+      if (h & 1)
+        thr1 = kth;
+      else
+        thr0 = kth;
+    }
+  }
+}
+
+template <int KF, bool PACK>
+__global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
+  using FK = Fmt<KF>;
+  using L = Lut<KF, 0>;
+  using CF = DecodeCfg<KF, 0>;
+  constexpr int CH = CF::CH, WT = CF::WT, S = CF::S;
+  using SL = StageLayout<KF, 0, CH>;
+  constexpr int NX = PACK ? 1 : 2;
+  constexpr int kRowBytes = FK::code_bytes + 4 + (FK::prod ? kSketch / 8 + 4 : 0);
+  extern __shared__ __align__(128) unsigned char smem[];
+  pdl_launch();  // the merge kernel may be scheduled as CTAs retire
+  // shared-memory layout as in decode_kernel
+  const uint32_t dyn0 = smem_u32(smem);
+  uint32_t low0 = (dyn0 + 127u) & ~127u, n_low = 0;
+  while (n_low < S && low0 + (n_low + 1) * SL::bytes <= kLutAddr) ++n_low;
+  const uint32_t high0 = kLutAddr + L::bytes;
+  uint32_t end = high0 + (S - n_low) * SL::bytes, scratch_addr;
+  if (low0 + n_low * SL::bytes + kScratchBytes <= kLutAddr) {
+    scratch_addr = low0 + n_low * SL::bytes;
+  } else {
+    scratch_addr = end;
+    end += kScratchBytes;
+  }
+  if (dyn0 > kLutAddr || end > dyn0 + a.dyn_bytes) {
+    if (threadIdx.x == 0) atomicOr(a.status, 8);
+    return;
+  }
+  auto stage_addr = [&](int s) -> uint32_t {
+    return s < static_cast<int>(n_low) ? low0 + s * SL::bytes : high0 + (s - n_low) * SL::bytes;
+  };
+  uint64_t* scratch = reinterpret_cast<uint64_t*>(smem + (scratch_addr - dyn0));
+  unsigned char* lut_mem = smem + (kLutAddr - dyn0);
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ volatile int s_abort;
+  __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int P = gridDim.x, cta = blockIdx.x;
+  const int Q = a.group, k = a.topk;
+  const int64_t n = a.n_db;
+  const int64_t C = (n + CH - 1) / CH;
+  const int64_t c0 = range_start(cta, C, P), c1 = range_start(cta + 1, C, P);
+  if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
+  if (tid == 32) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kConsumers);
+    }
+    s_abort = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumers) {
+    // ---- producer: rows in groups of four by bulk copy (every plane slice a
+    // multiple of 16 bytes), the last n % 4 rows by plain copies
+    if (lane == 0 && c0 < c1) {
+      const int nk = static_cast<int>(c1 - c0);
+      int s = 0;
+      uint32_t round = 0;
+      for (int kk = 0; kk < nk; ++kk) {
+        if (kk >= S && !mbar_wait(&empty_bar[s], round ^ 1u)) s_abort = 1;
+        if (s_abort) break;
+        const int64_t r0 = (c0 + kk) * CH;
+        const int rows = static_cast<int>(n - r0 < CH ? n - r0 : CH);
+        const int rows4 = rows & ~3;
+        const uint32_t st = stage_addr(s);
+        unsigned char* stp = smem + (st - dyn0);
+        for (int r = rows4; r < rows; ++r) {
+          const int64_t row = r0 + r;
+          for (int w = 0; w < FK::code_bytes / 4; ++w)
+            reinterpret_cast<uint32_t*>(stp + SL::kc + r * FK::code_bytes)[w] =
+                reinterpret_cast<const uint32_t*>(a.k_codes + row * FK::code_bytes)[w];
+          reinterpret_cast<float*>(stp + SL::kn)[r] = a.k_norms[row];
+          if constexpr (FK::prod) {
+            for (int w = 0; w < kSketch / 32; ++w)
+              reinterpret_cast<uint32_t*>(stp + SL::kq + r * (kSketch / 8))[w] =
+                  reinterpret_cast<const uint32_t*>(a.k_qjl + row * (kSketch / 8))[w];
+            reinterpret_cast<float*>(stp + SL::kr)[r] = a.k_res[row];
+          }
+        }
+        uint64_t* bar = &full_bar[s];
+        if (rows4 > 0) {
+          mbar_expect_tx(bar, static_cast<uint32_t>(rows4) * kRowBytes);
+          if constexpr (FK::code_bytes > 0)
+            bulk_g2s_addr(st + SL::kc, a.k_codes + r0 * FK::code_bytes, rows4 * FK::code_bytes, bar);
+          bulk_g2s_addr(st + SL::kn, a.k_norms + r0, rows4 * 4, bar);
+          if constexpr (FK::prod) {
+            bulk_g2s_addr(st + SL::kq, a.k_qjl + r0 * (kSketch / 8), rows4 * (kSketch / 8), bar);
+            bulk_g2s_addr(st + SL::kr, a.k_res + r0, rows4 * 4, bar);
+          }
+        } else {
+          mbar_arrive(bar);
+        }
+        if (++s == S) {
+          s = 0;
+          round ^= 1u;
+        }
+      }
+      // bulk copies still in flight land before the CTA may exit
+      for (int kk = nk - S; kk < nk; ++kk)
+        if (kk >= 0) mbar_wait(&full_bar[kk % S], (kk / S) & 1);
+    }
+    return;
+  }
+
+  // ---- lookup tables (consumer threads)
+  build_luts<L>(lut_mem, s_cb, tid);
+  consumers_sync();  // tables complete
+  const uint32_t lut_a = 0, lut_b = 0;
+  const uint32_t lane4 = kLutAddr | (lane * 4), lane8 = (kLutAddr + L::region_b_off) | (lane * 8);
+  const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
+  const TokRows tr = tok_rows<KF, 0>(g, t);
+
+  pdl_wait();  // the rotated query fragments
+  QFrag<PACK> bq, bqs;
+  {
+    const uint32_t* qf = a.qfrag;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int x = 0; x < NX; ++x) {
+          bq[ks][r][x] = qf[((ks * 2 + r) * 2 + x) * 32 + lane];
+          if constexpr (FK::prod) bqs[ks][r][x] = qf[(((8 + ks) * 2 + r) * 2 + x) * 32 + lane];
+        }
+  }
+  uint64_t list[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) list[h] = 0;
+  float thr0 = -INFINITY, thr1 = -INFINITY;
+
+  const int nk = static_cast<int>(c1 - c0);
+  int s = 0;
+  uint32_t round = 0;
+  for (int kk = 0; kk < nk; ++kk) {
+    if (!s_abort && !mbar_wait(&full_bar[s], round)) s_abort = 1;
+    const int64_t row0 = (c0 + kk) * CH + warp * WT;
+    const bool abort_w = __shfl_sync(0xffffffffu, static_cast<int>(s_abort), 0) != 0;  // one view per warp
+    if (!abort_w && row0 < n) {
+      const uint32_t st = stage_addr(s);
+      UnitPlanes sp;
+      sp.kcodes = st + SL::kc;
+      sp.knorm = st + SL::kn;
+      sp.kq = st + SL::kq;
+      sp.kres = st + SL::kr;
+      sp.vcodes = sp.vnorm = sp.vq = sp.vres = 0;
+#pragma unroll
+      for (int sub = 0; sub < WT / kTok; ++sub) {
+        const int64_t rb = row0 + sub * kTok;
+        const bool okA = rb + tr.kA < n, okB = rb + tr.kB < n;
+        float sc[4];
+        subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, okA, okB, g, t, bq, bqs,
+                                                      lut_a, lut_b, lane4, lane8, c1k, sc);
+        offer_subtile<kMaxG>(list, thr0, thr1, sc, okA, okB, static_cast<uint32_t>(rb + tr.kA),
+                             static_cast<uint32_t>(rb + tr.kB), t, lane, Q, k);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if (++s == S) {
+      s = 0;
+      round ^= 1u;
+    }
+  }
+
+  // ---- the CTA's list per query: merge the consumer warps' lists
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) scratch[(warp * kMaxG + h) * 32 + lane] = list[h];
+  consumers_sync();
+  if (warp < Q) {
+    const int h = warp;
+    int pos = 0;
+    uint64_t head = lane < kConsumers ? scratch[(lane * kMaxG + h) * 32] : 0;
+    uint64_t* dst = a.cand + (static_cast<int64_t>(h) * P + cta) * 32;
+    for (int r = 0; r < 32; ++r) {
+      const uint64_t best = warp_max_u64(head);
+      if (lane == 0) dst[r] = best;
+      if (best != 0 && head == best) {  // keys are unique apart from 0
+        ++pos;
+        head = pos < 32 ? scratch[(lane * kMaxG + h) * 32 + pos] : 0;
+      }
+    }
+  }
+  if (s_abort && tid == 0) atomicOr(a.status, 4);
+}
+
+// One CTA per query: the top k of the CTAs' sorted lists.
+constexpr int kSearchMergeThreads = 256;
+__global__ void __launch_bounds__(kSearchMergeThreads) search_merge_kernel(DecodeArgs a) {
+  extern __shared__ uint64_t s_keys[];  // [ctas][32]
+  const int h = blockIdx.x, P = a.ctas, k = a.topk, tid = threadIdx.x, lane = tid & 31;
+  pdl_wait();  // the CTAs' lists
+  const uint64_t* src = a.cand + static_cast<int64_t>(h) * P * 32;
+  for (int i = tid; i < P * 32; i += kSearchMergeThreads) s_keys[i] = src[i];
+  __syncthreads();
+  if (tid >= 32) return;
+  // lane owns lists lane, lane + 32, ... (at most kSearchMaxCtas / 32)
+  constexpr int J = kSearchMaxCtas / 32;
+  int pos[J];
+  uint64_t head[J];
+  uint64_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int l = lane + 32 * j;
+    pos[j] = 0;
+    head[j] = l < P ? s_keys[l * 32] : 0;
+    mine = head[j] > mine ? head[j] : mine;
+  }
+  float* os = a.out_scores + static_cast<int64_t>(h) * k;
+  int64_t* orow = a.out_rows + static_cast<int64_t>(h) * k;
+  for (int r = 0; r < k; ++r) {
+    const uint64_t best = warp_max_u64(mine);
+    if (lane == 0) {
+      os[r] = key_score(best);
+      orow[r] = key_row(best);
+    }
+    if (best != 0 && mine == best) {
+      uint64_t m = 0;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        if (head[j] == best) {
+          ++pos[j];
+          head[j] = pos[j] < 32 ? s_keys[(lane + 32 * j) * 32 + pos[j]] : 0;
+        }
+        m = head[j] > m ? head[j] : m;
+      }
+      mine = m;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 int num_sms_cached() {
@@ -1691,6 +2038,11 @@ template <int KF, int VF>
 size_t decode_smem_bytes() {
   using CF = DecodeCfg<KF, VF>;
   return static_cast<size_t>(plan_end(CF::stage, CF::S, CF::lut, kScratchBytes) - kDynBaseMax);
+}
+template <int KF, int VF>
+constexpr bool decode_smem_bytes_fits() {
+  using CF = DecodeCfg<KF, VF>;
+  return plan_end(CF::stage, CF::S, CF::lut, kScratchBytes) <= kSmemEnd;
 }
 
 // Launch with programmatic stream serialization: the kernel may start before
@@ -1750,6 +2102,28 @@ tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
 }
 
 constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 3) | (prod << 4); }
+
+template <int KF, bool PACK>
+tq_status run_search(DecodeArgs& a, int groups_ctas, cudaStream_t st) {
+  static_assert(decode_smem_bytes_fits<KF, 0>(), "no shared-memory plan for this search format");
+  cudaError_t e = ensure_dyn_smem<search_kernel<KF, PACK>>(kSmemBudget);
+  if (e != cudaSuccess) return cuda_fail(e, "search kernel attribute");
+  const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
+  e = ensure_dyn_smem<qrot_kernel<KF>>(static_cast<int>(qrot_smem));
+  if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
+  qrot_kernel<KF><<<dim3(1, 1), kQrotThreads, qrot_smem, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
+  e = launch_overlapped(search_kernel<KF, PACK>, dim3(groups_ctas), kThreadsP, kSmemBudget, st, a);
+  if (e != cudaSuccess) return cuda_fail(e, "search kernel launch");
+  const size_t merge_smem = static_cast<size_t>(groups_ctas) * 32 * sizeof(uint64_t);
+  if (merge_smem > 48 * 1024) {
+    e = ensure_dyn_smem<search_merge_kernel>(static_cast<int>(merge_smem));
+    if (e != cudaSuccess) return cuda_fail(e, "search merge attribute");
+  }
+  e = launch_overlapped(search_merge_kernel, dim3(a.group), kSearchMergeThreads, merge_smem, st, a);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "search merge launch");
+}
 
 }  // namespace
 
@@ -1812,6 +2186,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.cbs = p->cbs32;
   a.sig = p->sig32;
   a.sparse_thr = sparse_thr;
+  a.qscale = kLog2e / std::sqrt(static_cast<float>(kDim));
 
   const int kf = p->fk.id(), vf = p->fv.id();
 #define TQ_CASE(K, V) \
@@ -1833,6 +2208,72 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   TQ_CASE(fid(3, 0, 0), fid(2, 0, 0))
 #undef TQ_CASE
   return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: this K/V format pair has no decode kernel");
+}
+
+int search_ctas() { return std::min(num_sms_cached(), kSearchMaxCtas); }
+
+size_t search_workspace_bytes() {
+  return static_cast<size_t>(kQfragWords) * sizeof(uint32_t) +
+         static_cast<size_t>(kMaxG) * search_ctas() * 32 * sizeof(uint64_t);
+}
+
+int search_max_k() { return kSearchMaxK; }
+
+tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed* db, int64_t n, const void* q,
+                        int q_bf16, int n_queries, int k, float* scores, int64_t* rows, void* ws,
+                        cudaStream_t st) {
+  const int P = search_ctas();
+  char* w = static_cast<char*>(ws);
+  for (int g0 = 0; g0 < n_queries; g0 += kMaxG) {
+    // one pass over the database per group of up to kMaxG queries
+    DecodeArgs a{};
+    a.group = std::min(kMaxG, n_queries - g0);
+    a.q = static_cast<const char*>(q) + static_cast<size_t>(g0) * kDim * (q_bf16 ? 2 : 4);
+    a.q_bf16 = q_bf16;
+    a.k_codes = db->codes;
+    a.k_norms = db->norms;
+    a.k_qjl = db->qjl;
+    a.k_res = db->res_norms;
+    a.status = p->status32;
+    a.B = 1;
+    a.hkv = 1;
+    a.hq = a.group;
+    a.ctas = P;
+    a.qfrag = reinterpret_cast<uint32_t*>(w);
+    a.cand = reinterpret_cast<uint64_t*>(w + kQfragWords * sizeof(uint32_t));
+    a.pit = p->pit32;
+    a.st = p->st32;
+    a.pi = p->pi32;
+    a.s = p->s32;
+    a.cbs = p->cbs32;
+    a.sig = p->sig32;
+    a.pack = a.group <= 4;
+    a.dyn_bytes = kSmemBudget;
+    a.qscale = 1.f;
+    a.n_db = n;
+    a.topk = k;
+    a.out_scores = scores + static_cast<size_t>(g0) * k;
+    a.out_rows = rows + static_cast<size_t>(g0) * k;
+    tq_status r = TQ_ERR_UNSUPPORTED;
+    const int kf = f.id();
+#define TQ_CASE(K)                                                                           \
+  if (kf == (K)) r = a.pack ? run_search<(K), true>(a, P, st) : run_search<(K), false>(a, P, st); \
+  else
+    TQ_CASE(fid(1, 0, 0))
+    TQ_CASE(fid(2, 0, 0))
+    TQ_CASE(fid(3, 0, 0))
+    TQ_CASE(fid(4, 0, 0))
+    TQ_CASE(fid(2, 1, 0))
+    TQ_CASE(fid(3, 1, 0))
+    TQ_CASE(fid(0, 0, 1))
+    TQ_CASE(fid(1, 0, 1))
+    TQ_CASE(fid(2, 0, 1))
+    TQ_CASE(fid(3, 0, 1))
+    return fail(TQ_ERR_UNSUPPORTED, "tq_search: no search kernel for this format");
+#undef TQ_CASE
+    if (r != TQ_OK) return r;
+  }
+  return TQ_OK;
 }
 
 }  // namespace tq

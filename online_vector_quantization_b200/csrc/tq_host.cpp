@@ -658,4 +658,29 @@ tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const t
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t tq_search_workspace_bytes(void) { return search_workspace_bytes(); }
+
+tq_status tq_search(const tq_params* p, int which, const tq_packed* db, int64_t n, const void* q, int q_dtype,
+                    int n_queries, int k, float* scores, int64_t* rows, void* workspace, size_t ws_bytes,
+                    void* stream) {
+  if (!p) return fail(TQ_ERR_ARG, "tq_search: NULL params");
+  if ((which != TQ_K && which != TQ_V) || (q_dtype != TQ_F32 && q_dtype != TQ_BF16) || n < 0 ||
+      n > INT32_MAX - 1 || n_queries < 1 || k < 1)
+    return fail(TQ_ERR_ARG, "tq_search: bad which, dtype, n, n_queries or k");
+  if (k > search_max_k()) return fail(TQ_ERR_UNSUPPORTED, "tq_search: k above 32");
+  if (!q || !scores || !rows || !workspace) return fail(TQ_ERR_ARG, "tq_search: NULL q, scores, rows or workspace");
+  if (!aligned16(q) || !aligned16(workspace))
+    return fail(TQ_ERR_ALIGN, "tq_search: q and workspace must be 16-byte aligned");
+  if (ws_bytes < search_workspace_bytes()) return fail(TQ_ERR_CAPACITY, "tq_search: workspace too small");
+  const FormatSpec& f = which == TQ_K ? p->fk : p->fv;
+  if (n > 0) {
+    tq_status st = check_packed(f, db, "tq_search");
+    if (st != TQ_OK) return st;
+  } else if (!db) {
+    return fail(TQ_ERR_ARG, "tq_search: NULL database");
+  }
+  return launch_search(p, f, db, n, q, q_dtype == TQ_BF16, n_queries, k, scores, rows, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

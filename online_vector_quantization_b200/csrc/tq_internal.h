@@ -111,5 +111,10 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len);
 tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c,
                         const DecodePlan& plan, void* out, int out_bf16, void* ws,
                         float sparse_thr, cudaStream_t st);
+size_t search_workspace_bytes();
+int search_max_k();
+tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed* db, int64_t n, const void* q,
+                        int q_bf16, int n_queries, int k, float* scores, int64_t* rows, void* ws,
+                        cudaStream_t st);
 
 }  // namespace tq

@@ -10,7 +10,9 @@ busy), checked on sampled outputs the oracle computes one by one:
 - long-context K4/V3 decode with a 128-token bf16 sink, planted keys and
   sparse V (B=4, 64 q / 8 kv, T=131072): two sampled (sequence, kv-head) units;
 - the streaming step (16 sequences, U[8192, 65536] contexts, mixed 3.5-bit,
-  prefill, one 64-token append, one decode): two sampled units.
+  prefill, one 64-token append, one decode): two sampled units;
+- the inner-product search (2^22 prod 3-bit rows, 8 queries, top-10): the
+  returned rows against the oracle's scores and a 200,000-row sample.
 """
 import numpy as np
 import pytest
@@ -186,3 +188,32 @@ def test_full_stream_step_sampled():
         got = unit_packed(cache, f, "k", b, h, lens[b])
         got = o.Packed(got.codes[rows], got.norms[rows], got.qjl[rows], got.res_norms[rows])
         check_unit_codes(op, f, "k", st["ck"][0][b, :, h].double().cpu().numpy(), got)
+
+
+def test_full_search_sampled():
+    """The search workload bench.py times (2^22 prod 3-bit rows, 8 queries,
+    top-10): the returned rows' scores against the oracle's, and no row of a
+    200,000-row sample (plus every returned row) beats the returned ones by
+    more than the score tolerance."""
+    import test_gpu_search as ts
+
+    n, nq, k = 1 << 22, 8, 10
+    f = gu.fmt(3, prod=True)
+    gp, op = gu.make_params(f, f)
+    x = kv_inputs.kv_vectors(n, D, key="search-db", device="cuda", dtype=torch.bfloat16, outliers=True)
+    pk = tq.Packed.empty(gp, n, tq.TQ_K)
+    tq.tq_quantize(gp, x, tq.TQ_K, pk)
+    q = kv_inputs.queries((nq, D), key=("search-q", nq), device="cuda")
+    sc = torch.empty(nq, k, device="cuda")
+    rw = torch.empty(nq, k, dtype=torch.int64, device="cuda")
+    tq.tq_search(gp, tq.TQ_K, pk, n, q, k, sc, rw, tq.search_workspace())
+    torch.cuda.synchronize()
+    assert gp.status() == 0
+    got_s, got_r = sc.cpu().numpy(), rw.cpu().numpy()
+    rows = np.unique(np.concatenate([np.random.default_rng(3).choice(n, 200000, replace=False), got_r.ravel()]))
+    idx = torch.from_numpy(rows).cuda()
+    sub = o.Packed(pk.codes[idx].cpu().numpy(), pk.norms[idx].cpu().numpy(), pk.qjl[idx].cpu().numpy(),
+                   pk.res_norms[idx].cpu().numpy())
+    qd = q.double().cpu().numpy()
+    all_s = o.ip_scores(op, qd, sub, "k")
+    ts.check_topk(qd, got_s, got_r, all_s, pk.norms.cpu().numpy(), k, cand_rows=rows)
