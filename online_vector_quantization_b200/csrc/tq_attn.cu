@@ -1699,9 +1699,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
 //    pipeline over contiguous ranges of database chunks (K planes only).
 //    Each consumer warp keeps, per query, its best candidates as a sorted
 //    column across its lanes (lane j = j-th best); a subtile's scores are
-//    first tested against the lanes' thresholds (the k-th best score) with one
-//    vote, and only candidates that pass are inserted.  At the end the 15
-//    warps' lists of each query are merged into the CTA's list.
+//    first tested against a per-query bound shared by the CTA's warps (the
+//    best k-th score of any warp's list), and only rows that reach it are
+//    inserted.  At the end the 15 warps' lists of each query are merged into
+//    the CTA's list.
 //    search_merge_kernel: one CTA per query merges the CTAs' lists.
 // ---------------------------------------------------------------------------
 constexpr int kSearchMaxK = 32;      // one list entry per lane
@@ -1757,33 +1758,45 @@ __device__ __forceinline__ void topk_offer(uint64_t& list, uint64_t cA, uint64_t
   }
 }
 
+// Order-preserving unsigned form of a score and back (ord_score(-inf) =
+// 0x007FFFFF: the "no bound yet" threshold).
+__device__ __forceinline__ uint32_t ord_score(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_score(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+constexpr uint32_t kNoBound = 0x007FFFFFu;  // ord_score(-inf)
+
 // Offer one 16-token subtile: lane (g, t) holds the scores of rows rowA
-// (s[0], s[1]) and rowB (s[2], s[3]) for queries 2t and 2t + 1; thr0 / thr1
-// are the current k-th best scores of those two queries (-inf while a list
-// is not full).
+// (s[0], s[1]) and rowB (s[2], s[3]) for queries 2t and 2t + 1.  s_thr[h]
+// (shared by the CTA's warps) is the best k-th score any warp's list of query
+// h holds: a row scoring below it has k better rows already listed, so it
+// cannot be in the result.  One reduction finds the queries with rows at or
+// above their bound; only those are offered to the warp's lists.
 template <int G>
-__device__ __forceinline__ void offer_subtile(uint64_t (&list)[G], float& thr0, float& thr1, const float (&s)[4],
-                                              bool okA, bool okB, uint32_t rowA, uint32_t rowB, int t, int lane,
-                                              int Q, int k) {
-  const bool pass = (2 * t < Q && ((okA && s[0] >= thr0) || (okB && s[2] >= thr0))) ||
-                    (2 * t + 1 < Q && ((okA && s[1] >= thr1) || (okB && s[3] >= thr1)));
-  if (!__any_sync(0xffffffffu, pass)) return;
+__device__ __forceinline__ void offer_subtile(uint64_t (&list)[G], uint32_t* s_thr, const float (&s)[4], bool okA,
+                                              bool okB, uint32_t rowA, uint32_t rowB, int t, int lane, int Q,
+                                              int k) {
+  const int h0 = 2 * t, h1 = 2 * t + 1;
+  const float b0 = h0 < Q ? unord_score(s_thr[h0 & (G - 1)]) : INFINITY;
+  const float b1 = h1 < Q ? unord_score(s_thr[h1 & (G - 1)]) : INFINITY;
+  const bool p0 = (okA && s[0] >= b0) || (okB && s[2] >= b0);
+  const bool p1 = (okA && s[1] >= b1) || (okB && s[3] >= b1);
+  const unsigned heads = __reduce_or_sync(0xffffffffu, (p0 ? 1u << h0 : 0u) | (p1 ? 1u << h1 : 0u));
+  if (heads == 0) return;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    if (h >= Q) break;
+    if (!(heads & (1u << h))) continue;
     const bool own = t == (h >> 1);
-    const float th = (h & 1) ? thr1 : thr0;
+    const float th = (h & 1) ? b1 : b0;
     const float va = s[h & 1], vb = s[2 + (h & 1)];
     const uint64_t cA = (own && okA && va >= th) ? cand_key(va, rowA) : 0;
     const uint64_t cB = (own && okB && vb >= th) ? cand_key(vb, rowB) : 0;
     topk_offer(list[h], cA, cB, lane, k);
-    const float kth = key_score(__shfl_sync(0xffffffffu, list[h], k - 1));
-    if (own) {
-      if (h & 1)
-        thr1 = kth;
-      else
-        thr0 = kth;
-    }
+    const uint64_t kth = __shfl_sync(0xffffffffu, list[h], k - 1);
+    if (lane == 0 && kth != 0) atomicMax(&s_thr[h], static_cast<uint32_t>(kth >> 32));
   }
 }
 
@@ -1823,6 +1836,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ volatile int s_abort;
   __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
+  __shared__ uint32_t s_thr[kMaxG];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int P = gridDim.x, cta = blockIdx.x;
   const int Q = a.group, k = a.topk;
@@ -1830,6 +1844,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   const int64_t C = (n + CH - 1) / CH;
   const int64_t c0 = range_start(cta, C, P), c1 = range_start(cta + 1, C, P);
   if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
+  if (tid >= 96 && tid < 96 + kMaxG) s_thr[tid - 96] = kNoBound;
   if (tid == 32) {
 #pragma unroll
     for (int i = 0; i < S; ++i) {
@@ -1919,7 +1934,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   uint64_t list[kMaxG];
 #pragma unroll
   for (int h = 0; h < kMaxG; ++h) list[h] = 0;
-  float thr0 = -INFINITY, thr1 = -INFINITY;
 
   const int nk = static_cast<int>(c1 - c0);
   int s = 0;
@@ -1943,7 +1957,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
         float sc[4];
         subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, okA, okB, g, t, bq, bqs,
                                                       lut_a, lut_b, lane4, lane8, c1k, sc);
-        offer_subtile<kMaxG>(list, thr0, thr1, sc, okA, okB, static_cast<uint32_t>(rb + tr.kA),
+        offer_subtile<kMaxG>(list, s_thr, sc, okA, okB, static_cast<uint32_t>(rb + tr.kA),
                              static_cast<uint32_t>(rb + tr.kB), t, lane, Q, k);
       }
     }
