@@ -1733,27 +1733,26 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
   return v;
 }
 
-// Insert the candidates cA, cB (0: none) of the lanes into one query's list.
+// Insert the candidates c[i] (0: none) of the lanes into one query's list.
 // Lanes below k hold the list; a candidate that does not beat entry k-1 is
 // dropped.
-__device__ __forceinline__ void topk_offer(uint64_t& list, uint64_t cA, uint64_t cB, int lane, int k) {
-  unsigned mA = __ballot_sync(0xffffffffu, cA != 0);
-  unsigned mB = __ballot_sync(0xffffffffu, cB != 0);
-  while (mA | mB) {
-    const bool fromA = mA != 0;
-    const int src = __ffs(fromA ? mA : mB) - 1;
-    const uint64_t c = __shfl_sync(0xffffffffu, fromA ? cA : cB, src);
-    if (fromA)
-      mA &= mA - 1;
-    else
-      mB &= mB - 1;
-    const int pos = __popc(__ballot_sync(0xffffffffu, list > c));
-    const uint64_t up = __shfl_up_sync(0xffffffffu, list, 1);
-    if (pos < k) {
-      if (lane == pos)
-        list = c;
-      else if (lane > pos)
-        list = up;
+template <int NC>
+__device__ __forceinline__ void topk_offer(uint64_t& list, const uint64_t (&c)[NC], int lane, int k) {
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    unsigned m = __ballot_sync(0xffffffffu, c[i] != 0);
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      const uint64_t cc = __shfl_sync(0xffffffffu, c[i], src);
+      const int pos = __popc(__ballot_sync(0xffffffffu, list > cc));
+      const uint64_t up = __shfl_up_sync(0xffffffffu, list, 1);
+      if (pos < k) {
+        if (lane == pos)
+          list = cc;
+        else if (lane > pos)
+          list = up;
+      }
     }
   }
 }
@@ -1769,21 +1768,26 @@ __device__ __forceinline__ float unord_score(uint32_t o) {
 }
 constexpr uint32_t kNoBound = 0x007FFFFFu;  // ord_score(-inf)
 
-// Offer one 16-token subtile: lane (g, t) holds the scores of rows rowA
-// (s[0], s[1]) and rowB (s[2], s[3]) for queries 2t and 2t + 1.  s_thr[h]
-// (shared by the CTA's warps) is the best k-th score any warp's list of query
-// h holds: a row scoring below it has k better rows already listed, so it
-// cannot be in the result.  One reduction finds the queries with rows at or
-// above their bound; only those are offered to the warp's lists.
-template <int G>
-__device__ __forceinline__ void offer_subtile(uint64_t (&list)[G], uint32_t* s_thr, const float (&s)[4], bool okA,
-                                              bool okB, uint32_t rowA, uint32_t rowB, int t, int lane, int Q,
-                                              int k) {
+// Offer the NS 16-token subtiles of one warp tile: for subtile i, lane
+// (g, t) holds the scores of rows row[i][0] (s[i][0], s[i][1]) and row[i][1]
+// (s[i][2], s[i][3]) for queries 2t and 2t + 1 (ok[i][*]: the row exists).
+// s_thr[h] (shared by the CTA's warps) is the best k-th score any warp's
+// list of query h holds: a row scoring below it has k better rows listed
+// already, so it cannot be in the result.  One reduction finds the queries
+// with rows at or above their bound; only those are offered to the lists.
+template <int G, int NS>
+__device__ __forceinline__ void offer_tile(uint64_t (&list)[G], uint32_t* s_thr, const float (&s)[NS][4],
+                                           const bool (&ok)[NS][2], const uint32_t (&row)[NS][2], int t, int lane,
+                                           int Q, int k) {
   const int h0 = 2 * t, h1 = 2 * t + 1;
   const float b0 = h0 < Q ? unord_score(s_thr[h0 & (G - 1)]) : INFINITY;
   const float b1 = h1 < Q ? unord_score(s_thr[h1 & (G - 1)]) : INFINITY;
-  const bool p0 = (okA && s[0] >= b0) || (okB && s[2] >= b0);
-  const bool p1 = (okA && s[1] >= b1) || (okB && s[3] >= b1);
+  bool p0 = false, p1 = false;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    p0 |= (ok[i][0] && s[i][0] >= b0) || (ok[i][1] && s[i][2] >= b0);
+    p1 |= (ok[i][0] && s[i][1] >= b1) || (ok[i][1] && s[i][3] >= b1);
+  }
   const unsigned heads = __reduce_or_sync(0xffffffffu, (p0 ? 1u << h0 : 0u) | (p1 ? 1u << h1 : 0u));
   if (heads == 0) return;
 #pragma unroll
@@ -1791,10 +1795,14 @@ __device__ __forceinline__ void offer_subtile(uint64_t (&list)[G], uint32_t* s_t
     if (!(heads & (1u << h))) continue;
     const bool own = t == (h >> 1);
     const float th = (h & 1) ? b1 : b0;
-    const float va = s[h & 1], vb = s[2 + (h & 1)];
-    const uint64_t cA = (own && okA && va >= th) ? cand_key(va, rowA) : 0;
-    const uint64_t cB = (own && okB && vb >= th) ? cand_key(vb, rowB) : 0;
-    topk_offer(list[h], cA, cB, lane, k);
+    uint64_t c[2 * NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+      const float va = s[i][h & 1], vb = s[i][2 + (h & 1)];
+      c[2 * i] = (own && ok[i][0] && va >= th) ? cand_key(va, row[i][0]) : 0;
+      c[2 * i + 1] = (own && ok[i][1] && vb >= th) ? cand_key(vb, row[i][1]) : 0;
+    }
+    topk_offer(list[h], c, lane, k);
     const uint64_t kth = __shfl_sync(0xffffffffu, list[h], k - 1);
     if (lane == 0 && kth != 0) atomicMax(&s_thr[h], static_cast<uint32_t>(kth >> 32));
   }
@@ -1950,16 +1958,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
       sp.kq = st + SL::kq;
       sp.kres = st + SL::kr;
       sp.vcodes = sp.vnorm = sp.vq = sp.vres = 0;
+      // both subtiles' scores first (their lookup and MMA chains
+      // interleave), then one offer
+      constexpr int NS = WT / kTok;
+      float sc[NS][4];
+      bool ok[NS][2];
+      uint32_t rows[NS][2];
 #pragma unroll
-      for (int sub = 0; sub < WT / kTok; ++sub) {
+      for (int sub = 0; sub < NS; ++sub) {
         const int64_t rb = row0 + sub * kTok;
-        const bool okA = rb + tr.kA < n, okB = rb + tr.kB < n;
-        float sc[4];
-        subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, okA, okB, g, t, bq, bqs,
-                                                      lut_a, lut_b, lane4, lane8, c1k, sc);
-        offer_subtile<kMaxG>(list, s_thr, sc, okA, okB, static_cast<uint32_t>(rb + tr.kA),
-                             static_cast<uint32_t>(rb + tr.kB), t, lane, Q, k);
+        ok[sub][0] = rb + tr.kA < n;
+        ok[sub][1] = rb + tr.kB < n;
+        rows[sub][0] = static_cast<uint32_t>(rb + tr.kA);
+        rows[sub][1] = static_cast<uint32_t>(rb + tr.kB);
+        subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, ok[sub][0], ok[sub][1], g, t,
+                                                      bq, bqs, lut_a, lut_b, lane4, lane8, c1k, sc[sub]);
       }
+      offer_tile<kMaxG, NS>(list, s_thr, sc, ok, rows, t, lane, Q, k);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
