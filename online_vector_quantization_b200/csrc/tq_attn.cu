@@ -1733,28 +1733,37 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
   return v;
 }
 
-// Insert the candidates c[i] (0: none) of the lanes into one query's list.
-// Lanes below k hold the list; a candidate that does not beat entry k-1 is
-// dropped.
-template <int NC>
-__device__ __forceinline__ void topk_offer(uint64_t& list, const uint64_t (&c)[NC], int lane, int k) {
-#pragma unroll
-  for (int i = 0; i < NC; ++i) {
-    unsigned m = __ballot_sync(0xffffffffu, c[i] != 0);
-    while (m) {
-      const int src = __ffs(m) - 1;
-      m &= m - 1;
-      const uint64_t cc = __shfl_sync(0xffffffffu, c[i], src);
-      const int pos = __popc(__ballot_sync(0xffffffffu, list > cc));
-      const uint64_t up = __shfl_up_sync(0xffffffffu, list, 1);
-      if (pos < k) {
-        if (lane == pos)
-          list = cc;
-        else if (lane > pos)
-          list = up;
-      }
+// Insert the candidates c0..c3 (0: none) of the lanes into one query's list
+// (lane j holds entry j).  Lanes below k hold the list; a candidate that does
+// not beat entry k-1 is dropped.  Kept compact (one loop, no unrolling): it
+// runs only for the rare rows that reach the bound.
+__device__ __noinline__ uint64_t topk_offer(uint64_t ent, uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3,
+                                            int lane, int k) {
+  unsigned m0 = __ballot_sync(0xffffffffu, c0 != 0), m1 = __ballot_sync(0xffffffffu, c1 != 0);
+  unsigned m2 = __ballot_sync(0xffffffffu, c2 != 0), m3 = __ballot_sync(0xffffffffu, c3 != 0);
+#pragma unroll 1
+  while (m0 | m1 | m2 | m3) {
+    // the lowest pending lane of the first non-empty candidate set
+    const int w = m0 ? 0 : m1 ? 1 : m2 ? 2 : 3;
+    const unsigned m = w == 0 ? m0 : w == 1 ? m1 : w == 2 ? m2 : m3;
+    const uint64_t c = w == 0 ? c0 : w == 1 ? c1 : w == 2 ? c2 : c3;
+    const int src = __ffs(m) - 1;
+    const unsigned rest = m & (m - 1);
+    m0 = w == 0 ? rest : m0;
+    m1 = w == 1 ? rest : m1;
+    m2 = w == 2 ? rest : m2;
+    m3 = w == 3 ? rest : m3;
+    const uint64_t cc = __shfl_sync(0xffffffffu, c, src);
+    const int pos = __popc(__ballot_sync(0xffffffffu, ent > cc));
+    const uint64_t up = __shfl_up_sync(0xffffffffu, ent, 1);
+    if (pos < k) {
+      if (lane == pos)
+        ent = cc;
+      else if (lane > pos)
+        ent = up;
     }
   }
+  return ent;
 }
 
 // Order-preserving unsigned form of a score and back (ord_score(-inf) =
@@ -1771,39 +1780,42 @@ constexpr uint32_t kNoBound = 0x007FFFFFu;  // ord_score(-inf)
 // Offer the NS 16-token subtiles of one warp tile: for subtile i, lane
 // (g, t) holds the scores of rows row[i][0] (s[i][0], s[i][1]) and row[i][1]
 // (s[i][2], s[i][3]) for queries 2t and 2t + 1 (ok[i][*]: the row exists).
-// s_thr[h] (shared by the CTA's warps) is the best k-th score any warp's
-// list of query h holds: a row scoring below it has k better rows listed
-// already, so it cannot be in the result.  One reduction finds the queries
-// with rows at or above their bound; only those are offered to the lists.
-template <int G, int NS>
-__device__ __forceinline__ void offer_tile(uint64_t (&list)[G], uint32_t* s_thr, const float (&s)[NS][4],
+// The warp's lists live in shared memory, lists[h * 32 + j] = entry j of
+// query h.  s_thr[h] (shared by the CTA's warps) is the best k-th score any
+// warp's list of query h holds: a row scoring below it has k better rows
+// listed already, so it cannot be in the result.  One reduction finds the
+// queries with rows at or above their bound; only those are offered.
+template <int NS>
+__device__ __forceinline__ void offer_tile(uint64_t* lists, uint32_t* s_thr, const float (&s)[NS][4],
                                            const bool (&ok)[NS][2], const uint32_t (&row)[NS][2], int t, int lane,
                                            int Q, int k) {
+  static_assert(NS == 1 || NS == 2, "one or two subtiles per warp tile");
   const int h0 = 2 * t, h1 = 2 * t + 1;
-  const float b0 = h0 < Q ? unord_score(s_thr[h0 & (G - 1)]) : INFINITY;
-  const float b1 = h1 < Q ? unord_score(s_thr[h1 & (G - 1)]) : INFINITY;
+  const float b0 = h0 < Q ? unord_score(s_thr[h0 & (kMaxG - 1)]) : INFINITY;
+  const float b1 = h1 < Q ? unord_score(s_thr[h1 & (kMaxG - 1)]) : INFINITY;
   bool p0 = false, p1 = false;
 #pragma unroll
   for (int i = 0; i < NS; ++i) {
     p0 |= (ok[i][0] && s[i][0] >= b0) || (ok[i][1] && s[i][2] >= b0);
     p1 |= (ok[i][0] && s[i][1] >= b1) || (ok[i][1] && s[i][3] >= b1);
   }
-  const unsigned heads = __reduce_or_sync(0xffffffffu, (p0 ? 1u << h0 : 0u) | (p1 ? 1u << h1 : 0u));
-  if (heads == 0) return;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    if (!(heads & (1u << h))) continue;
-    const bool own = t == (h >> 1);
-    const float th = (h & 1) ? b1 : b0;
-    uint64_t c[2 * NS];
+  unsigned heads = __reduce_or_sync(0xffffffffu, (p0 ? 1u << h0 : 0u) | (p1 ? 1u << h1 : 0u));
+#pragma unroll 1
+  while (heads) {
+    const int h = __ffs(heads) - 1;
+    heads &= heads - 1;
+    const bool own = t == (h >> 1), odd = h & 1;
+    const float th = odd ? b1 : b0;
+    uint64_t c[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int i = 0; i < NS; ++i) {
-      const float va = s[i][h & 1], vb = s[i][2 + (h & 1)];
+      const float va = odd ? s[i][1] : s[i][0], vb = odd ? s[i][3] : s[i][2];
       c[2 * i] = (own && ok[i][0] && va >= th) ? cand_key(va, row[i][0]) : 0;
       c[2 * i + 1] = (own && ok[i][1] && vb >= th) ? cand_key(vb, row[i][1]) : 0;
     }
-    topk_offer(list[h], c, lane, k);
-    const uint64_t kth = __shfl_sync(0xffffffffu, list[h], k - 1);
+    const uint64_t ent = topk_offer(lists[h * 32 + lane], c[0], c[1], c[2], c[3], lane, k);
+    lists[h * 32 + lane] = ent;
+    const uint64_t kth = __shfl_sync(0xffffffffu, ent, k - 1);
     if (lane == 0 && kth != 0) atomicMax(&s_thr[h], static_cast<uint32_t>(kth >> 32));
   }
 }
@@ -1939,9 +1951,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
           if constexpr (FK::prod) bqs[ks][r][x] = qf[(((8 + ks) * 2 + r) * 2 + x) * 32 + lane];
         }
   }
-  uint64_t list[kMaxG];
+  // this warp's lists of the queries: [h][32] in the scratch area
+  uint64_t* lists = scratch + warp * kMaxG * 32;
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) list[h] = 0;
+  for (int h = 0; h < kMaxG; ++h) lists[h * 32 + lane] = 0;
 
   const int nk = static_cast<int>(c1 - c0);
   int s = 0;
@@ -1974,7 +1987,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
         subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, ok[sub][0], ok[sub][1], g, t,
                                                       bq, bqs, lut_a, lut_b, lane4, lane8, c1k, sc[sub]);
       }
-      offer_tile<kMaxG, NS>(list, s_thr, sc, ok, rows, t, lane, Q, k);
+      offer_tile<NS>(lists, s_thr, sc, ok, rows, t, lane, Q, k);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
@@ -1985,8 +1998,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   }
 
   // ---- the CTA's list per query: merge the consumer warps' lists
-#pragma unroll
-  for (int h = 0; h < kMaxG; ++h) scratch[(warp * kMaxG + h) * 32 + lane] = list[h];
   consumers_sync();
   if (warp < Q) {
     const int h = warp;
