@@ -450,6 +450,8 @@ struct DecodeArgs {
   uint64_t* cand;          // per (query, CTA) candidate lists [group][ctas][32]
   float* out_scores;       // [group][topk]
   int64_t* out_rows;       // [group][topk]
+  const uint32_t* bound_in;  // per-query starting bound (ordered score) or null
+  uint32_t* bound_out;       // the merge writes the k-th best score here instead of results
 };
 
 __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t i) {
@@ -1937,7 +1939,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const TokRows tr = tok_rows<KF, 0>(g, t);
 
-  pdl_wait();  // the rotated query fragments
+  pdl_wait();  // the rotated query fragments (and the starting bounds)
+  if (a.bound_in && tid < Q) atomicMax(&s_thr[tid], a.bound_in[tid]);
   QFrag<PACK> bq, bqs;
   {
     const uint32_t* qf = a.qfrag;
@@ -2043,8 +2046,13 @@ __global__ void __launch_bounds__(kSearchMergeThreads) search_merge_kernel(Decod
   for (int r = 0; r < k; ++r) {
     const uint64_t best = warp_max_u64(mine);
     if (lane == 0) {
-      os[r] = key_score(best);
-      orow[r] = key_row(best);
+      if (a.bound_out) {
+        // k rows score at least the k-th best: a bound for the full pass
+        if (r == k - 1) a.bound_out[h] = best != 0 ? static_cast<uint32_t>(best >> 32) : kNoBound;
+      } else {
+        os[r] = key_score(best);
+        orow[r] = key_row(best);
+      }
     }
     if (best != 0 && mine == best) {
       uint64_t m = 0;
@@ -2146,6 +2154,14 @@ constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 3) | (p
 template <int KF, bool PACK>
 tq_status run_search(DecodeArgs& a, int groups_ctas, cudaStream_t st) {
   static_assert(decode_smem_bytes_fits<KF, 0>(), "no shared-memory plan for this search format");
+  // A large database is searched twice: first its leading rows, one chunk
+  // per CTA, whose k-th best score per query becomes the starting bound of
+  // the full pass (k rows reach it, so rows below it are never results);
+  // the full pass then inserts few rows into its lists.
+  const int64_t n_pre = static_cast<int64_t>(groups_ctas) * DecodeCfg<KF, 0>::CH;
+  const bool prefix = a.bound_out != nullptr && a.n_db >= 8 * n_pre;
+  uint32_t* bound = a.bound_out;
+  a.bound_out = nullptr;
   cudaError_t e = ensure_dyn_smem<search_kernel<KF, PACK>>(kSmemBudget);
   if (e != cudaSuccess) return cuda_fail(e, "search kernel attribute");
   const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
@@ -2154,13 +2170,24 @@ tq_status run_search(DecodeArgs& a, int groups_ctas, cudaStream_t st) {
   qrot_kernel<KF><<<dim3(1, 1), kQrotThreads, qrot_smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
-  e = launch_overlapped(search_kernel<KF, PACK>, dim3(groups_ctas), kThreadsP, kSmemBudget, st, a);
-  if (e != cudaSuccess) return cuda_fail(e, "search kernel launch");
   const size_t merge_smem = static_cast<size_t>(groups_ctas) * 32 * sizeof(uint64_t);
   if (merge_smem > 48 * 1024) {
     e = ensure_dyn_smem<search_merge_kernel>(static_cast<int>(merge_smem));
     if (e != cudaSuccess) return cuda_fail(e, "search merge attribute");
   }
+  a.bound_in = nullptr;
+  if (prefix) {
+    DecodeArgs pre = a;
+    pre.n_db = n_pre;
+    pre.bound_out = bound;
+    e = launch_overlapped(search_kernel<KF, PACK>, dim3(groups_ctas), kThreadsP, kSmemBudget, st, pre);
+    if (e != cudaSuccess) return cuda_fail(e, "search kernel launch");
+    e = launch_overlapped(search_merge_kernel, dim3(a.group), kSearchMergeThreads, merge_smem, st, pre);
+    if (e != cudaSuccess) return cuda_fail(e, "search merge launch");
+    a.bound_in = bound;
+  }
+  e = launch_overlapped(search_kernel<KF, PACK>, dim3(groups_ctas), kThreadsP, kSmemBudget, st, a);
+  if (e != cudaSuccess) return cuda_fail(e, "search kernel launch");
   e = launch_overlapped(search_merge_kernel, dim3(a.group), kSearchMergeThreads, merge_smem, st, a);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "search merge launch");
 }
@@ -2254,7 +2281,7 @@ int search_ctas() { return std::min(num_sms_cached(), kSearchMaxCtas); }
 
 size_t search_workspace_bytes() {
   return static_cast<size_t>(kQfragWords) * sizeof(uint32_t) +
-         static_cast<size_t>(kMaxG) * search_ctas() * 32 * sizeof(uint64_t);
+         static_cast<size_t>(kMaxG) * search_ctas() * 32 * sizeof(uint64_t) + 256;
 }
 
 int search_max_k() { return kSearchMaxK; }
@@ -2281,6 +2308,8 @@ tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed
     a.ctas = P;
     a.qfrag = reinterpret_cast<uint32_t*>(w);
     a.cand = reinterpret_cast<uint64_t*>(w + kQfragWords * sizeof(uint32_t));
+    a.bound_out = reinterpret_cast<uint32_t*>(w + kQfragWords * sizeof(uint32_t) +
+                                              static_cast<size_t>(kMaxG) * P * 32 * sizeof(uint64_t));
     a.pit = p->pit32;
     a.st = p->st32;
     a.pi = p->pi32;

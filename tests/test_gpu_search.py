@@ -170,3 +170,17 @@ def test_search_rejects_bad_arguments():
     with pytest.raises(tq.TqError) as e:
         tq.tq_search(gp, tq.TQ_K, pk, 64, q, 4, s, r, ws[:100])
     assert e.value.status == 4
+
+
+def test_search_with_bound_pass():
+    # a database large enough for the leading-rows pass that seeds the bound
+    f = gu.fmt(3)
+    n = 8 * 148 * 480 + 1001
+    gp, op, x, pk = build_db(f, n, "srl", boost=(70000, n - 2))
+    xd = x.double().numpy()
+    qd = queries(xd, 5, "srlq", planted=[(1, 70000), (3, n - 2)])
+    q = torch.from_numpy(qd).to(torch.bfloat16)
+    qd = q.double().numpy()
+    got_s, got_r = run_search(gp, tq.TQ_K, pk, n, q, 16)
+    opk = to_oracle(pk, n)
+    check_topk(qd, got_s, got_r, o.ip_scores(op, qd, opk, "k"), opk.norms, 16)
