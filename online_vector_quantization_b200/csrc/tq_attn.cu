@@ -708,15 +708,19 @@ __device__ __forceinline__ TokRows tok_rows(int g, int t) {
 // Scores of one 16-token subtile whose rows start at `srow` of the staged
 // planes: s2 (base 2) for tokens g (s2[0], s2[1]) and g+8 (s2[2], s2[3]),
 // columns 2t, 2t+1; masked tokens get -inf.  Two MMA accumulator chains.
-template <int KF, bool PACK, bool T3W, bool T2A>
+// HI: the query's fp16 high halves only (column g = head g, no low halves):
+// one MMA per k-step for up to 8 heads, scores within about 2^-12 of
+// ||q|| ||x|| (the search's precision; attention keeps both halves).
+template <int KF, bool PACK, bool T3W, bool T2A, bool HI = false>
 __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
                                                int g, int t,
-                                               const QFrag<PACK>& bq, const QFrag<PACK>& bqs,
+                                               const QFrag<PACK || HI>& bq, const QFrag<PACK || HI>& bqs,
                                                uint32_t lut_a, uint32_t lut_b,
                                                uint32_t lane4, uint32_t lane8, uint32_t c1k, float (&s2)[4]) {
+  static_assert(!(PACK && HI), "packed halves or high halves only");
   using FK = Fmt<KF>;
   using KR = KRow<KF>;
-  constexpr int NX = PACK ? 1 : 2;
+  constexpr int NX = (PACK || HI) ? 1 : 2;
   const uint32_t one2 = 0x3C003C00u;  // half2(1, 1)
   const int rA = srow + tr.kA, rB = srow + tr.kB;
   const uint32_t ka = u.kcodes + rA * FK::code_bytes;
@@ -1829,7 +1833,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   using CF = DecodeCfg<KF, 0>;
   constexpr int CH = CF::CH, WT = CF::WT, S = CF::S;
   using SL = StageLayout<KF, 0, CH>;
-  constexpr int NX = PACK ? 1 : 2;
+  // up to 4 queries: high and low halves packed in one MMA; more: high halves only
+  constexpr bool HI = !PACK;
   constexpr int kRowBytes = FK::code_bytes + 4 + (FK::prod ? kSketch / 8 + 4 : 0);
   extern __shared__ __align__(128) unsigned char smem[];
   pdl_launch();  // the merge kernel may be scheduled as CTAs retire
@@ -1941,18 +1946,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
 
   pdl_wait();  // the rotated query fragments (and the starting bounds)
   if (a.bound_in && tid < Q) atomicMax(&s_thr[tid], a.bound_in[tid]);
-  QFrag<PACK> bq, bqs;
+  QFrag<true> bq, bqs;  // slot 0: packed halves, or (unpacked layout) the high halves
   {
     const uint32_t* qf = a.qfrag;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int x = 0; x < NX; ++x) {
-          bq[ks][r][x] = qf[((ks * 2 + r) * 2 + x) * 32 + lane];
-          if constexpr (FK::prod) bqs[ks][r][x] = qf[(((8 + ks) * 2 + r) * 2 + x) * 32 + lane];
-        }
+      for (int r = 0; r < 2; ++r) {
+        bq[ks][r][0] = qf[((ks * 2 + r) * 2 + 0) * 32 + lane];
+        if constexpr (FK::prod) bqs[ks][r][0] = qf[(((8 + ks) * 2 + r) * 2 + 0) * 32 + lane];
+      }
   }
   // this warp's lists of the queries: [h][32] in the scratch area
   uint64_t* lists = scratch + warp * kMaxG * 32;
@@ -1987,8 +1990,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
         ok[sub][1] = rb + tr.kB < n;
         rows[sub][0] = static_cast<uint32_t>(rb + tr.kA);
         rows[sub][1] = static_cast<uint32_t>(rb + tr.kB);
-        subtile_scores<KF, PACK, L::t3_wide, L::t2a>(sp, warp * WT + sub * kTok, tr, ok[sub][0], ok[sub][1], g, t,
-                                                      bq, bqs, lut_a, lut_b, lane4, lane8, c1k, sc[sub]);
+        subtile_scores<KF, PACK, L::t3_wide, L::t2a, HI>(sp, warp * WT + sub * kTok, tr, ok[sub][0], ok[sub][1], g,
+                                                          t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, sc[sub]);
       }
       offer_tile<NS>(lists, s_thr, sc, ok, rows, t, lane, Q, k);
     }

@@ -23,9 +23,10 @@ import online_vector_quantization_b200 as tq  # noqa: E402
 import gpu_util as gu  # noqa: E402
 
 D = 128
-# score tolerance per unit of ||q|| * ||x||: fp16 centroid and query-half
-# rounding (relative ~1e-4 after the per-width scaling) summed over 128
-# coordinates with fp32 accumulation, with margin
+# score tolerance per unit of ||q|| * max ||x||: the query in fp16 (high
+# halves only for more than 4 queries: at most 2^-12 relative per coordinate,
+# about 2^-12 / sqrt(128) summed with random signs), centroids near-exact in
+# fp16 after the per-width scaling, fp32 accumulation
 SCORE_TOL = 2e-4
 
 
