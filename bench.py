@@ -133,16 +133,22 @@ DECODE_TRAFFIC = {"source_sha256": "5eb66211a806211958dd2cd9d530b4da17b3d718fcde
                   "bytes": 489154816}
 
 
-def decode_traffic():
+def decode_sources_sha256():
+    """sha256 over the decode kernel's sources (tq_decode_common.cuh, then tq_attn.cu)."""
     import hashlib
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "online_vector_quantization_b200", "csrc",
-                       "tq_attn.cu")
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "online_vector_quantization_b200", "csrc")
+    h = hashlib.sha256()
     try:
-        with open(src, "rb") as f:
-            same = hashlib.sha256(f.read()).hexdigest() == DECODE_TRAFFIC["source_sha256"]
+        for name in ("tq_decode_common.cuh", "tq_attn.cu"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
     except OSError:
-        same = False
-    return DECODE_TRAFFIC["bytes"] if same else None
+        return None
+    return h.hexdigest()
+
+
+def decode_traffic():
+    return DECODE_TRAFFIC["bytes"] if decode_sources_sha256() == DECODE_TRAFFIC["source_sha256"] else None
 
 
 def step_bytes(lens_now):

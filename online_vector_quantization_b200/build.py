@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtq.so")
-SOURCES = ["tq_host.cpp", "tq_quantize.cu", "tq_attn.cu", "tq_noalloc.cu"]
+SOURCES = ["tq_host.cpp", "tq_quantize.cu", "tq_attn.cu", "tq_search.cu", "tq_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
