@@ -106,6 +106,37 @@ __device__ __noinline__ uint64_t topk_offer(uint64_t ent, uint64_t c0, uint64_t 
 }
 
 
+// Merge up to 32 candidates at once into a list (lane j holds entry j, both
+// sorted by a bitonic network): the candidates c0..c3 of the eight lanes
+// (g, t) that own a query are gathered one per lane (tile row L from lane
+// (L & 7, t), component (L >> 4) * 2 + ((L >> 3) & 1)), sorted descending,
+// and the list keeps the 32 largest of both (elementwise maximum against the
+// reversed candidates, then a bitonic clean-up).  Cheaper than one insertion
+// per candidate when many rows reach the bound (the first tiles).
+__device__ __noinline__ uint64_t topk_merge32(uint64_t ent, uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3,
+                                              int t_own, int lane) {
+  const int src = ((lane & 7) << 2) | t_own, comp = ((lane >> 4) << 1) | ((lane >> 3) & 1);
+  const uint64_t v0 = __shfl_sync(0xffffffffu, c0, src), v1 = __shfl_sync(0xffffffffu, c1, src);
+  const uint64_t v2 = __shfl_sync(0xffffffffu, c2, src), v3 = __shfl_sync(0xffffffffu, c3, src);
+  uint64_t key = comp == 0 ? v0 : comp == 1 ? v1 : comp == 2 ? v2 : v3;
+#pragma unroll
+  for (int k2 = 2; k2 <= 32; k2 <<= 1)
+#pragma unroll
+    for (int j = k2 >> 1; j > 0; j >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool keep_max = ((lane & j) == 0) == ((lane & k2) == 0);
+      key = keep_max ? (o > key ? o : key) : (o < key ? o : key);
+    }
+  const uint64_t rev = __shfl_sync(0xffffffffu, key, 31 - lane);
+  uint64_t m = ent > rev ? ent : rev;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, m, j);
+    m = (lane & j) == 0 ? (o > m ? o : m) : (o < m ? o : m);
+  }
+  return m;
+}
+
 // Offer the NS 16-token subtiles of one warp tile: for subtile i, lane
 // (g, t) holds the scores of rows row[i][0] (s[i][0], s[i][1]) and row[i][1]
 // (s[i][2], s[i][3]) for queries 2t and 2t + 1 (ok[i][*]: the row exists).
@@ -142,7 +173,10 @@ __device__ __forceinline__ void offer_tile(uint64_t* lists, uint32_t* s_thr, con
       c[2 * i] = (own && ok[i][0] && va >= th) ? cand_key(va, row[i][0]) : 0;
       c[2 * i + 1] = (own && ok[i][1] && vb >= th) ? cand_key(vb, row[i][1]) : 0;
     }
-    const uint64_t ent = topk_offer(lists[h * 32 + lane], c[0], c[1], c[2], c[3], lane, k);
+    const int n_c = __popc(__ballot_sync(0xffffffffu, c[0] != 0)) + __popc(__ballot_sync(0xffffffffu, c[1] != 0)) +
+                    __popc(__ballot_sync(0xffffffffu, c[2] != 0)) + __popc(__ballot_sync(0xffffffffu, c[3] != 0));
+    const uint64_t ent = n_c > 6 ? topk_merge32(lists[h * 32 + lane], c[0], c[1], c[2], c[3], h >> 1, lane)
+                                 : topk_offer(lists[h * 32 + lane], c[0], c[1], c[2], c[3], lane, k);
     lists[h * 32 + lane] = ent;
     const uint64_t kth = __shfl_sync(0xffffffffu, ent, k - 1);
     if (lane == 0 && kth != 0) atomicMax(&s_thr[h], static_cast<uint32_t>(kth >> 32));
@@ -333,7 +367,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
     int pos = 0;
     uint64_t head = lane < kConsumers ? scratch[(lane * kMaxG + h) * 32] : 0;
     uint64_t* dst = a.cand + (static_cast<int64_t>(h) * P + cta) * 32;
-    for (int r = 0; r < 32; ++r) {
+    // the CTA's k best (the grid's k best are among the CTAs' k best)
+    for (int r = 0; r < k; ++r) {
       const uint64_t best = warp_max_u64(head);
       if (lane == 0) dst[r] = best;
       if (best != 0 && head == best) {  // keys are unique apart from 0
@@ -341,6 +376,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
         head = pos < 32 ? scratch[(lane * kMaxG + h) * 32 + pos] : 0;
       }
     }
+    if (lane >= k) dst[lane] = 0;
   }
   if (s_abort && tid == 0) atomicOr(a.status, 4);
 }
@@ -351,8 +387,10 @@ __global__ void __launch_bounds__(kSearchMergeThreads) search_merge_kernel(Decod
   extern __shared__ uint64_t s_keys[];  // [ctas][32]
   const int h = blockIdx.x, P = a.ctas, k = a.topk, tid = threadIdx.x, lane = tid & 31;
   pdl_wait();  // the CTAs' lists
+  // all 16-byte pieces of the lists in flight at once
   const uint64_t* src = a.cand + static_cast<int64_t>(h) * P * 32;
-  for (int i = tid; i < P * 32; i += kSearchMergeThreads) s_keys[i] = src[i];
+  for (int i = tid; i < P * 16; i += kSearchMergeThreads) cp_async16(smem_u32(s_keys + 2 * i), src + 2 * i);
+  cp_async_wait_all();
   __syncthreads();
   if (tid >= 32) return;
   // lane owns lists lane, lane + 32, ... (at most kSearchMaxCtas / 32)
