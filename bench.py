@@ -96,7 +96,7 @@ class ClockSampler:
 def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device, bits: int = 3):
     """Config: streaming append + decode (mixed rows: bits + 0.5 bits per
     channel, 3.5 by default).  Returns the state the step uses."""
-    lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", rank))
+    lens = rank_sequence_lengths(kv_inputs, rank)
     params = tq.Params(bits, bits, mixed_k=1, mixed_v=1, seed=0)
     cap = ((max(lens) + (n_steps + 1) * CHUNK + 63) // 64) * 64
     cache = tq.Cache(params, N_SEQ, HKV, cap, 0, device=device)
@@ -149,6 +149,21 @@ def decode_sources_sha256():
 
 def decode_traffic():
     return DECODE_TRAFFIC["bytes"] if decode_sources_sha256() == DECODE_TRAFFIC["source_sha256"] else None
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """The largest of one per-rank number over all ranks (every rank calls it,
+    in the same order): multi-GPU times are the slowest rank's."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_sequence_lengths(kv_inputs, rank: int):
+    """The streaming workload's context lengths on one rank: every rank (GPU)
+    holds its own 16 sequences (weak scaling, no data shared between ranks)."""
+    return kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", rank))
 
 
 def step_bytes(lens_now):
@@ -206,9 +221,7 @@ def run_gpu(args):
     total_ms = t0.elapsed_time(t1)
     decode_ms = [a.elapsed_time(b) for a, b in d_events]
     if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, device)
     append_b, decode_b = 0, 0
     for j in range(args.steps):
         a, d = step_bytes([n + j * CHUNK for n in lens_at_timing])
@@ -305,9 +318,7 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, device)
     total = 0
     for j in range(args.steps):
         a, d = step_bytes([n + (args.warmup + j) * CHUNK for n in st["lens"]])
