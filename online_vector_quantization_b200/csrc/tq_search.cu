@@ -39,6 +39,10 @@ using namespace sm100;
 
 constexpr int kSearchMaxK = 32;      // one list entry per lane
 constexpr int kSearchMaxCtas = 256;  // bound on the search grid (merge stages all lists)
+// the consumer warps' candidate lists ([warp][query][32] keys) live in the
+// scratch area of the decode kernel's shared-memory plan
+static_assert(kConsumers * kMaxG * 32 * sizeof(uint64_t) <= kScratchBytes, "search lists exceed the scratch area");
+static_assert(kMaxG <= kConsumers, "one merging warp per query");
 
 // Order-preserving unsigned form of a score and back (ord_score(-inf) =
 // 0x007FFFFF: the "no bound yet" threshold).
