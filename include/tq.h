@@ -99,7 +99,9 @@ typedef struct {
  * TurboQuant, in breve" (optimal scalar quantizer for the known distribution)
  * and section "Cosa aggiunge turboquant-mlx" (Lloyd-Max).  Writes 2^bits
  * ascending centroids and the 2^bits - 1 midpoints between them (host
- * arrays, caller-owned).  Any d >= 3 and bits in 1..8.  Pure host function. */
+ * arrays, caller-owned).  Any d >= 3 and bits in 1..8: up to 4 bits by the
+ * plain Lloyd iteration, above by Newton's method on the same conditions
+ * (the plain iteration slows down as the levels grow).  Pure host function. */
 tq_status tq_codebook(int d, int bits, double* centroids, double* bounds);
 
 /* Seeded random rotation Pi (d x d row-major, y = Pi u): Haar orthogonal,

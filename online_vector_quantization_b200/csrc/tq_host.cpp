@@ -173,7 +173,115 @@ struct SphereCoordinate {
   double first_moment(double a, double b) const { return moment_prim(a) - moment_prim(b); }
 };
 
+// Standard normal quantile by bisection on erfc (start values only).
+static double normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// The Lloyd map: T_k = (first moment) / (mass) of f over the cell of c_k.
+static void lloyd_map(const SphereCoordinate& f, const GaussLegendre& gl, const std::vector<double>& c,
+                      std::vector<double>& T, std::vector<double>& m0) {
+  const int levels = static_cast<int>(c.size());
+  for (int k = 0; k < levels; ++k) {
+    const double lo = k == 0 ? -1.0 : 0.5 * (c[k - 1] + c[k]);
+    const double hi = k == levels - 1 ? 1.0 : 0.5 * (c[k] + c[k + 1]);
+    m0[k] = f.mass(lo, hi, gl);
+    T[k] = f.first_moment(lo, hi) / m0[k];
+  }
+}
+
+// More than 16 levels: the plain iteration's contraction approaches 1, so the
+// fixed point c = T(c) is found by Newton's method.  With t_k the midpoints
+// and f_k = f(t_k), dT_k/dc_{k+1} = f_k (t_k - T_k) / (2 M0_k) and
+// dT_k/dc_{k-1} = f_{k-1} (T_k - t_{k-1}) / (2 M0_k), dT_k/dc_k their sum:
+// the Jacobian of c - T(c) is tridiagonal (Thomas algorithm).  Start: the
+// high-resolution optimum of a Gaussian of variance 1/d (point density ~
+// f^(1/3): Gaussian quantiles of variance 3/d), then 50 plain steps; Newton
+// steps are halved while they do not reduce max |c - T(c)| or break the order.
+static tq_status lloyd_max_newton(int d, int bits, double* centroids, double* bounds) {
+  const int L = 1 << bits;
+  SphereCoordinate f(d);
+  GaussLegendre gl(48);
+  std::vector<double> c(L), T(L), m0(L), cn(L), Tn(L), m0n(L), step(L);
+  const double s3 = std::sqrt(3.0 / d);
+  for (int k = 0; k < L; ++k) c[k] = s3 * normal_quantile((k + 0.5) / L);
+  for (int it = 0; it < 50; ++it) {
+    lloyd_map(f, gl, c, T, m0);
+    c = T;
+  }
+  lloyd_map(f, gl, c, T, m0);
+  auto max_abs_g = [&](const std::vector<double>& cc, const std::vector<double>& tt) {
+    double g = 0.0;
+    for (int k = 0; k < L; ++k) g = std::max(g, std::fabs(cc[k] - tt[k]));
+    return g;
+  };
+  std::vector<double> diag(L), sup(L), sub(L), rhs(L);
+  for (int it = 0; it < 100; ++it) {
+    // J = I - dT, rows k: sub[k] (column k-1), diag[k], sup[k] (column k+1)
+    for (int k = 0; k < L; ++k) {
+      double up = 0.0, dn = 0.0;
+      if (k + 1 < L) {
+        const double t = 0.5 * (c[k] + c[k + 1]);
+        up = f.density(t) * (t - T[k]) / (2.0 * m0[k]);
+      }
+      if (k > 0) {
+        const double t = 0.5 * (c[k - 1] + c[k]);
+        dn = f.density(t) * (T[k] - t) / (2.0 * m0[k]);
+      }
+      diag[k] = 1.0 - up - dn;
+      sup[k] = -up;
+      sub[k] = -dn;
+      rhs[k] = -(c[k] - T[k]);
+    }
+    // Thomas algorithm
+    for (int k = 1; k < L; ++k) {
+      const double w = sub[k] / diag[k - 1];
+      diag[k] -= w * sup[k - 1];
+      rhs[k] -= w * rhs[k - 1];
+    }
+    step[L - 1] = rhs[L - 1] / diag[L - 1];
+    for (int k = L - 2; k >= 0; --k) step[k] = (rhs[k] - sup[k] * step[k + 1]) / diag[k];
+    const double g0 = max_abs_g(c, T);
+    double lam = 1.0;
+    for (;;) {
+      bool ok = true;
+      for (int k = 0; k < L; ++k) {
+        cn[k] = c[k] + lam * step[k];
+        if (k > 0 && !(cn[k] > cn[k - 1])) ok = false;
+      }
+      if (!(cn[0] > -1.0) || !(cn[L - 1] < 1.0)) ok = false;
+      if (ok) {
+        lloyd_map(f, gl, cn, Tn, m0n);
+        if (max_abs_g(cn, Tn) < g0 || lam < 1e-6) break;
+      }
+      lam *= 0.5;
+      if (lam < 1e-9) return fail(TQ_ERR_ARG, "tq_codebook: Newton iteration did not converge");
+    }
+    double moved = 0.0, cmax = 0.0;
+    for (int k = 0; k < L; ++k) {
+      moved = std::max(moved, std::fabs(cn[k] - c[k]));
+      cmax = std::max(cmax, std::fabs(cn[k]));
+    }
+    c.swap(cn);
+    T.swap(Tn);
+    m0.swap(m0n);
+    if (moved <= 1e-15 * cmax) break;
+  }
+  for (int k = 0; k < L; ++k) centroids[k] = c[k];
+  for (int k = 0; k + 1 < L; ++k) bounds[k] = 0.5 * (c[k] + c[k + 1]);
+  return TQ_OK;
+}
+
 static tq_status lloyd_max(int d, int bits, double* centroids, double* bounds) {
+  if (bits > 4) return lloyd_max_newton(d, bits, centroids, bounds);
   const int levels = 1 << bits;
   SphereCoordinate f(d);
   GaussLegendre gl(48);

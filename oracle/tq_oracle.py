@@ -219,7 +219,17 @@ def lloyd_max(d: int, bits: int, tol: float = 1e-15, max_iter: int = 100000) -> 
       t_k = (c_k + c_{k+1}) / 2             (nearest-neighbour boundaries)
       c_k = int x f / int f over [t_{k-1}, t_k]  (centroid condition)
     until no centroid moves by more than ``tol`` (relative to max |c|).
+    Above 4 bits the plain iteration converges too slowly (its contraction
+    approaches 1 as the levels grow), so the same two conditions are solved
+    by Newton's method instead (lloyd_max_newton).
     """
+    if bits > 4:
+        return lloyd_max_newton(d, bits, tol)
+    return lloyd_iteration(d, bits, tol, max_iter)
+
+
+def lloyd_iteration(d: int, bits: int, tol: float = 1e-15, max_iter: int = 100000) -> Codebook:
+    """The plain Lloyd-Max iteration of lloyd_max, for any number of bits."""
     levels = 1 << bits
     nd = NormalDist()
     c = np.array([nd.inv_cdf((k + 0.5) / levels) for k in range(levels)]) / math.sqrt(d)
@@ -231,6 +241,59 @@ def lloyd_max(d: int, bits: int, tol: float = 1e-15, max_iter: int = 100000) -> 
         c_new = cell_first_moment(lo, hi, d) / cell_mass(lo, hi, d)
         moved = np.max(np.abs(c_new - c))
         c = c_new
+        if moved <= tol * np.max(np.abs(c)):
+            break
+    return Codebook(d, bits, c, 0.5 * (c[:-1] + c[1:]), it)
+
+
+def lloyd_max_newton(d: int, bits: int, tol: float = 1e-15, max_iter: int = 100, warm: int = 50) -> Codebook:
+    """The fixed point of the Lloyd map of lloyd_max, T_k(c) = M1_k / M0_k
+    (first moment over mass of f over [t_{k-1}, t_k], t_k the midpoints),
+    found by Newton's method on G(c) = c - T(c).  With f_k = f(t_k):
+      dT_k/dc_{k+1} = f_k (t_k - T_k) / (2 M0_k)
+      dT_k/dc_{k-1} = f_{k-1} (T_k - t_{k-1}) / (2 M0_k)
+      dT_k/dc_k     = the sum of the two
+    so the Jacobian I - dT is tridiagonal.  Start: the high-resolution optimum
+    for a Gaussian of variance 1/d (point density proportional to f^(1/3):
+    Gaussian quantiles of variance 3/d), then ``warm`` plain Lloyd steps.
+    Steps are halved while they do not reduce max |G| or break the order of
+    the centroids.
+    """
+    levels = 1 << bits
+    nd = NormalDist()
+    c = np.array([nd.inv_cdf((k + 0.5) / levels) for k in range(levels)]) * math.sqrt(3.0 / d)
+
+    def lloyd_map(c):
+        t = 0.5 * (c[:-1] + c[1:])
+        lo = np.concatenate(([-1.0], t))
+        hi = np.concatenate((t, [1.0]))
+        m0 = cell_mass(lo, hi, d)
+        return cell_first_moment(lo, hi, d) / m0, m0, t
+
+    for _ in range(warm):
+        c = lloyd_map(c)[0]
+    T, m0, t = lloyd_map(c)
+    G = c - T
+    it = 0
+    for it in range(1, max_iter + 1):
+        ft = coord_density(t, d)
+        up = ft * (t - T[:-1]) / (2 * m0[:-1])   # dT_k/dc_{k+1}, k < L-1
+        lo = ft * (T[1:] - t) / (2 * m0[1:])     # dT_{k+1}/dc_k
+        jac = np.eye(levels)
+        jac -= np.diag(np.concatenate((up, [0.0])) + np.concatenate(([0.0], lo)))
+        jac -= np.diag(up, 1) + np.diag(lo, -1)
+        step = np.linalg.solve(jac, -G)
+        lam = 1.0
+        while True:
+            cn = c + lam * step
+            if np.all(np.diff(cn) > 0) and cn[0] > -1.0 and cn[-1] < 1.0:
+                Tn, m0n, tn = lloyd_map(cn)
+                Gn = cn - Tn
+                if np.max(np.abs(Gn)) < np.max(np.abs(G)) or lam < 1e-6:
+                    break
+            lam *= 0.5
+        moved = np.max(np.abs(cn - c))
+        c, T, m0, t, G = cn, Tn, m0n, tn, Gn
         if moved <= tol * np.max(np.abs(c)):
             break
     return Codebook(d, bits, c, 0.5 * (c[:-1] + c[1:]), it)

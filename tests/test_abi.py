@@ -27,7 +27,8 @@ def test_every_declared_symbol_is_exported():
         assert n in tq.EXPORTED, n
 
 
-@pytest.mark.parametrize("d,b", [(128, 1), (128, 2), (128, 3), (128, 4), (64, 3), (256, 2)])
+@pytest.mark.parametrize("d,b", [(128, 1), (128, 2), (128, 3), (128, 4), (64, 3), (256, 2), (128, 5), (64, 7),
+                                 (128, 8)])
 def test_codebook_matches_oracle(d, b):
     c, t = tq.tq_codebook(d, b)
     ref = o.lloyd_max(d, b)

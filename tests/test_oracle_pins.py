@@ -511,3 +511,33 @@ def test_ip_search_pads_short_databases():
     empty = o.quantize(p, np.zeros((0, 128)), "k")
     scores, rows = o.ip_search(p, q, empty, 4)
     assert (rows == -1).all() and np.isneginf(scores).all()
+
+
+# ---- codebooks above 4 bits (Newton on the Lloyd conditions) ----------------
+
+@pytest.mark.parametrize("b", [2, 3, 4, 5])
+def test_newton_reaches_the_lloyd_iteration_fixed_point(b):
+    # two algorithms for the same conditions: the plain iteration (run to
+    # convergence) and Newton's method from the high-resolution start
+    it = o.lloyd_iteration(128, b)
+    nw = o.lloyd_max_newton(128, b)
+    assert np.max(np.abs(it.centroids - nw.centroids)) < 1e-13
+
+
+@pytest.mark.parametrize("b", [6, 8])
+def test_many_level_codebook_conditions(b):
+    d = 128
+    cb = book(d, b)
+    c = cb.centroids
+    assert np.all(np.diff(c) > 0) and np.max(np.abs(c + c[::-1])) < 1e-13
+    lo = np.concatenate(([-1.0], cb.bounds))
+    hi = np.concatenate((cb.bounds, [1.0]))
+    # centroid condition, cell by cell, against an independent quadrature
+    from scipy import integrate as si
+    for k in (0, 1, len(c) // 2 - 1, len(c) // 2, len(c) - 1):
+        m0 = si.quad(lambda x: o.coord_density(x, d), lo[k], hi[k], epsabs=0, epsrel=1e-13)[0]
+        m1 = si.quad(lambda x: x * o.coord_density(x, d), lo[k], hi[k], epsabs=0, epsrel=1e-13)[0]
+        assert abs(m1 / m0 - c[k]) < 1e-12 * max(abs(c[k]), 1e-3)
+    # the rate-distortion sandwich of the article ("within about 2.7x")
+    dist = o.mse_distortion(cb)
+    assert 4.0 ** -b <= dist <= math.sqrt(3) * math.pi / 2 * 4.0 ** -b
