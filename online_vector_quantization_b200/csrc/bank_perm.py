@@ -145,10 +145,10 @@ def search(fk, fv, chunk, seed=1, restarts=8, iters=20000):
 # instantiations; ids as in tq_attn.cu: mse | mixed << 3 | prod << 4
 PAIRS = [
     (1, 1, fmt(1), fmt(1), 480), (2, 2, fmt(2), fmt(2), 480), (3, 3, fmt(3), fmt(3), 480),
-    (4, 4, fmt(4), fmt(4), 480), (11, 11, fmt(3, True), fmt(3, True), 480), (10, 10, fmt(2, True), fmt(2, True), 480),
-    (16, 16, fmt(0, prod=True), fmt(0, prod=True), 240), (17, 17, fmt(1, prod=True), fmt(1, prod=True), 240),
-    (18, 18, fmt(2, prod=True), fmt(2, prod=True), 240), (19, 19, fmt(3, prod=True), fmt(3, prod=True), 240),
-    (4, 3, fmt(4), fmt(3), 480), (4, 2, fmt(4), fmt(2), 480), (3, 2, fmt(3), fmt(2), 480),
+    (4, 4, fmt(4), fmt(4), 240), (11, 11, fmt(3, True), fmt(3, True), 480), (10, 10, fmt(2, True), fmt(2, True), 480),
+    (16, 16, fmt(0, prod=True), fmt(0, prod=True), 480), (17, 17, fmt(1, prod=True), fmt(1, prod=True), 480),
+    (18, 18, fmt(2, prod=True), fmt(2, prod=True), 480), (19, 19, fmt(3, prod=True), fmt(3, prod=True), 480),
+    (4, 3, fmt(4), fmt(3), 480), (4, 2, fmt(4), fmt(2), 240), (3, 2, fmt(3), fmt(2), 480),
 ]
 
 if __name__ == "__main__":
