@@ -77,3 +77,32 @@ def test_host_argument_errors():
     assert e.value.status == 1
     assert tq._lib.tq_cache_bytes(None, 1, 1, 64, 0) == 0
     assert tq._lib.tq_decode_workspace_bytes(None, 1, 8, 8, 128) == 0
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/tq.h compiles as C99 with warnings as errors, and a C program
+    links against libtq.so and calls a host entry point through it."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(tq.__file__)
+    prog = tmp_path / "probe.c"
+    prog.write_text(
+        '#include "tq.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        "  double c[8], t[7];\n"
+        "  if (tq_codebook(128, 3, c, t) != TQ_OK) return 1;\n"
+        "  if (tq_codebook(2, 3, c, t) != TQ_ERR_ARG) return 2;\n"
+        '  printf("%.12f\\n", c[7]);\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "probe"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.dirname(HEADER), str(prog),
+                        "-L", lib_dir, "-ltq", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert abs(float(r.stdout) - o.lloyd_max(128, 3).centroids[7]) < 1e-12
