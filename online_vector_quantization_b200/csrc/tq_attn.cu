@@ -340,7 +340,9 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
 }
 
 // ---------------------------------------------------------------------------
-// 3. merge: one CTA per unit (sequence, kv-head), all heads of its group.
+// 3. merge: one CTA per unit (sequence, kv-head) and group of merge_heads
+//    query heads (all heads of the unit's group, or one head each when the
+//    units are too few to fill the GPU otherwise).
 //    The unit's quantized tokens were streamed as pieces by consecutive CTAs
 //    of the decode grid; its bf16 sink tokens are attended here.  Partial
 //    results are combined by their maxima (the usual online-softmax merge),
@@ -365,8 +367,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Merge shared memory beyond the static arrays: sink weights [n_sink][8],
 // piece maxima / weights and sums [ctas][8] each, and a staging buffer of
-// merge_chunk pieces (G x part_floats floats each).
-constexpr size_t kMergeStageBytes = 128 * 1024;
+// merge_chunk pieces (the CTA's heads x part_floats floats each).  Small
+// enough for two merge CTAs per SM.
+constexpr size_t kMergeStageBytes = 32 * 1024;
 inline int merge_chunk_pieces(int group, int part_floats) {
   const size_t per = static_cast<size_t>(group) * part_floats * sizeof(float);
   return static_cast<int>(std::max<size_t>(1, kMergeStageBytes / per));
@@ -396,9 +399,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   float* s_part = s_l + a.ctas * kMaxG;             // staged pieces [merge_chunk][G][part_floats]
   const int u = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = a.group, P = a.ctas, CH = a.chunk, PF = a.part_floats;
+  const int G = a.merge_heads, h0 = blockIdx.y * G;  // this CTA's heads: h0 .. h0 + G - 1 of the group
+  const int P = a.ctas, CH = a.chunk, PF = a.part_floats;
   const int b = u / a.hkv, kvh = u % a.hkv;
-  const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * G) * kDim;  // head 0 of the group
+  // head h0 of the unit's group
+  const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * a.group + h0) * kDim;
   const UnitInfo ui = unit_info(a, u, CH);
   if (ui.len == 0) {
     for (int i = tid; i < G * kDim; i += NT) store_out(a, orow + i, 0.f);
@@ -558,7 +563,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     const int i = e / G, h = e % G;
     float m = -INFINITY, l = 0.f;
     if (cta_has_chunks(first + i, C, P)) {
-      const float* pp = part_slot(a, u + first + i) + h * PF;
+      const float* pp = part_slot(a, u + first + i) + (h0 + h) * PF;
       m = __ldcg(pp);
       l = __ldcg(pp + 1);
     }
@@ -594,12 +599,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       float acc[kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
-      const int slot_floats = G * PF;
+      // this CTA's heads of each piece: G x PF consecutive floats at head h0
+      const int slot_floats = G * PF, per4 = slot_floats / 4;
       for (int c0 = 0; c0 < n_p; c0 += a.merge_chunk) {
         const int cnt = min(a.merge_chunk, n_p - c0);
-        const float4* src = reinterpret_cast<const float4*>(part_slot(a, u + first + c0));
-        const int n16 = cnt * slot_floats / 4;
-        for (int e = tid; e < n16; e += NT) cp_async16(smem_u32(s_part) + 16 * e, src + e);
+        const int n16 = cnt * per4;
+        for (int e = tid; e < n16; e += NT) {
+          const int i = e / per4, q4 = e - i * per4;
+          const float4* src = reinterpret_cast<const float4*>(part_slot(a, u + first + c0 + i) + h0 * PF);
+          cp_async16(smem_u32(s_part) + 16 * e, src + q4);
+        }
         cp_async_wait_all();
         __syncthreads();
         for (int i = sl; i < cnt; i += NS) {
@@ -916,12 +925,13 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, plan.group, plan.part_floats);
+  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, a.merge_heads, plan.part_floats);
   if (merge_smem > 48 * 1024) {
     e = ensure_dyn_smem<merge_kernel<VF>>(static_cast<int>(merge_smem));
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
   }
-  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv), kMergeThreads, merge_smem, st, a);
+  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv, plan.group / a.merge_heads), kMergeThreads,
+                        merge_smem, st, a);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "merge kernel launch");
 }
 
@@ -985,7 +995,13 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.max_len = plan.max_len;
   a.part_floats = plan.part_floats;
   a.ctas = plan.ctas;
-  a.merge_chunk = merge_chunk_pieces(plan.group, plan.part_floats);
+  // few units (small batches, long contexts): one merge CTA per (unit, head)
+  // so the merge work spreads over the GPU; otherwise one per unit
+  {
+    const long long units = static_cast<long long>(plan.B) * plan.hkv;
+    a.merge_heads = units * plan.group <= 2LL * num_sms_cached() ? 1 : plan.group;
+  }
+  a.merge_chunk = merge_chunk_pieces(a.merge_heads, plan.part_floats);
   if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 4096");
   const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
   char* w = static_cast<char*>(ws);

@@ -416,6 +416,7 @@ struct DecodeArgs {
   int ctas;   // CTAs of the decode grid (pieces a unit can be cut into)
   int chunk;  // quantized tokens per scheduled chunk
   int merge_chunk;  // pieces the merge kernel stages in shared memory at a time
+  int merge_heads;  // query heads per merge CTA (the group, or 1: one CTA per (unit, head))
   float* parts;
   const uint32_t* qfrag;
   void* out;
