@@ -925,11 +925,10 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  // static and dynamic shared memory together pass 48 KB: opt in every time
   const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, a.merge_heads, plan.part_floats);
-  if (merge_smem > 48 * 1024) {
-    e = ensure_dyn_smem<merge_kernel<VF>>(static_cast<int>(merge_smem));
-    if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
-  }
+  e = ensure_dyn_smem<merge_kernel<VF>>(static_cast<int>(merge_smem));
+  if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
   e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv, plan.group / a.merge_heads), kMergeThreads,
                         merge_smem, st, a);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "merge kernel launch");
