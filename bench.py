@@ -132,19 +132,26 @@ def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device,
 # The sources changed after the capture only outside decode_kernel (the merge
 # kernel, the host launch code, and one argument field only the merge reads),
 # so the figure is tied to the sources as they are now.
-DECODE_TRAFFIC = {"source_sha256": "edd013d35f9330d2c8dd8fc2026d5c97276b0ebfffa738b1bc048a8beaf768ec",
+DECODE_TRAFFIC = {"source_sha256": "b426d03d3fc4c2860cffb7da0929aa5341593ed4587e754872505fa7a1cd5f34",
                   "bytes": 489391104}
 
 
 def decode_sources_sha256():
-    """sha256 over the decode kernel's sources (tq_decode_common.cuh, then tq_attn.cu)."""
+    """sha256 over the decode kernel's sources (tq_decode_common.cuh, then
+    tq_attn.cu) with comments and blank lines removed, so that only code
+    changes invalidate a captured traffic figure."""
     import hashlib
+    import re
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "online_vector_quantization_b200", "csrc")
     h = hashlib.sha256()
     try:
         for name in ("tq_decode_common.cuh", "tq_attn.cu"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+            with open(os.path.join(csrc, name)) as f:
+                text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+            for line in text.splitlines():
+                code = re.sub(r"//.*$", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     except OSError:
         return None
     return h.hexdigest()

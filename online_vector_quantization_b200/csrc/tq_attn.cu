@@ -23,8 +23,11 @@
 //      (two or four codes per lookup, no bank conflicts), so no fp16 tile is
 //      ever written back to memory.  Warps merge in shared memory and the CTA
 //      writes one (m, l, acc) partial per piece of a (sequence, kv-head).
-//   3. merge_kernel: one CTA per (sequence, query head) attends the bf16 sink,
-//      combines the pieces and applies Pi^T / S^T once.
+//   3. merge_kernel: one CTA per (sequence, kv-head), or per (sequence,
+//      query head) for small batches, attends the bf16 sink, combines the
+//      pieces and applies Pi^T / S^T once.  (qrot_kernel, the formats, tables
+//      and subtile scoring live in tq_decode_common.cuh, shared with the
+//      inner-product search.)
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
