@@ -18,8 +18,8 @@ Sources (page title, section):
   [P5] "Why TurboQuant saves DGX twice" (NVIDIA developer forum): PolarQuant +
        QJL residual correction, 3.5-bit, no calibration, online per token.
 
-Readings where the pages are silent are marked [reading]; every one of them is
-listed in the design doc.  Pins: every function below is checked by
+Readings where the pages are silent are marked [reading] where they are
+used.  Pins: every function below is checked by
 ``tests/test_oracle_pins.py`` against something other than itself; none is
 "parity unpinned".
 """
