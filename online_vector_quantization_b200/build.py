@@ -26,9 +26,12 @@ def nvcc() -> str:
 
 
 def build(verbose: bool = False, ptxas_info: bool = False) -> str:
+    """Compile every source (in parallel, one nvcc per source) and link."""
+    from concurrent.futures import ThreadPoolExecutor
+
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    cmds, objs = [], []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
         obj = os.path.join(objdir, src + ".o")
@@ -40,8 +43,14 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
                 cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd))
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as pool:
+        for r in list(pool.map(lambda c: subprocess.run(c, capture_output=not verbose, text=True), cmds)):
+            if r.returncode != 0:
+                import sys
+                sys.stderr.write((r.stdout or "") + (r.stderr or ""))
+                raise subprocess.CalledProcessError(r.returncode, r.args, r.stdout, r.stderr)
     link = [nvcc(), "-shared", "-o", LIB, *objs, *ARCH]
     if verbose:
         print(" ".join(link))
