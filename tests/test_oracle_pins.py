@@ -261,7 +261,8 @@ def test_end_to_end_cosine_matches_pages():
 # ---- quantize / pack -------------------------------------------------------
 
 @pytest.mark.parametrize("fmt", [o.Format(1), o.Format(2), o.Format(3), o.Format(4),
-                                 o.Format(3, mixed=True), o.Format(2, mixed=True), o.Format(3, prod=True)])
+                                 o.Format(3, mixed=True), o.Format(2, mixed=True), o.Format(3, prod=True),
+                                 o.Format(8)])
 def test_quantize_is_brute_force_nearest_centroid(fmt):
     p = o.Params(128, fmt, fmt)
     x = kv_inputs.kv_vectors(64, 128, key="bf", dtype=torch.bfloat16).double().numpy()
@@ -541,3 +542,12 @@ def test_many_level_codebook_conditions(b):
     # the rate-distortion sandwich of the article ("within about 2.7x")
     dist = o.mse_distortion(cb)
     assert 4.0 ** -b <= dist <= math.sqrt(3) * math.pi / 2 * 4.0 ** -b
+
+
+def test_eight_bit_rows_are_bytes():
+    # 8-bit codes (the K8 setting of the article's "Cosa aggiunge"): code j is byte j
+    fmt = o.Format(8)
+    assert fmt.code_bytes(128) == 128
+    idx = np.random.default_rng(9).integers(0, 256, size=(5, 128))
+    packed = o.pack_codes(idx, [8] * 128)
+    assert np.array_equal(packed, idx.astype(np.uint8))
