@@ -362,7 +362,7 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "stream-2.5", "search")
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "fp8-kv", "stream-2.5", "search")
 
 
 def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
@@ -386,6 +386,8 @@ def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
         out["ip_search_4M"] = _aux_search(tq, torch, kv_inputs, device, flush, iters, formats)
     if only in (None, "bf16-sdpa"):
         out["bf16_kv_decode_sdpa_stream_shapes"] = _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters)
+    if only in (None, "fp8-kv"):
+        out["fp8_kv_decode_stream_shapes"] = _aux_fp8_kv(torch, kv_inputs, device, flush, iters)
     return out
 
 
@@ -460,6 +462,13 @@ def _aux_k4v3(tq, torch, kv_inputs, device, flush, iters):
         by = 4 * 8 * ((T - 128) * (68 + 52) + 128 * 512)
         out[f"decode_k4v3_sink_T128k_{name}"] = {"ms": round(ms, 4), "gb_per_s_dense_equiv": round(by / (ms * 1e-3) / 1e9, 1),
                                                  "dense_bytes": by}
+    # what the sparse-V rule dropped in one call (device tallies, untimed)
+    stats = torch.zeros(4, dtype=torch.int64, device=device)
+    tq.tq_decode_attn(p, q, cache, T, o, ws, 1e-6, sparse_v_stats=stats)
+    examined, dropped, tiles, skipped = (int(x) for x in stats.cpu())
+    out["decode_k4v3_sink_T128k_sparse_v"].update(
+        {"weights_dropped": round(dropped / max(examined, 1), 4), "tiles_skipped": round(skipped / max(tiles, 1), 4),
+         "weights_examined": examined, "tiles_examined": tiles})
     assert int(cache.status.item()) == 0
     return out
 
@@ -562,6 +571,44 @@ def _aux_bf16_sdpa(torch, kv_inputs, device, flush, iters):
             "tokens_per_s_per_seq": round(1000.0 / ms, 1), "calls": N_SEQ}
 
 
+def _aux_fp8_kv(torch, kv_inputs, device, flush, iters):
+    """Context for the packed cache: one decode step over an FP8 (e4m3) KV
+    cache of the streaming workload's shapes (16 sequences, the same contexts,
+    32 q / 8 kv heads), with FlashInfer's decode kernel (one call per
+    sequence, the faster of its CUDA-core and tensor-core variants)."""
+    try:
+        import flashinfer
+    except Exception as e:  # pragma: no cover - depends on the image
+        return {"unavailable": f"flashinfer import failed: {e}"}
+    lens = kv_inputs.sequence_lengths(N_SEQ, LEN_LO, LEN_HI, key=("stream-lens", 0))
+    gen = torch.Generator(device=device).manual_seed(0)
+    f8 = torch.float8_e4m3fn
+    ks = [torch.randn(n, HKV, D, generator=gen, device=device).to(f8) for n in lens]
+    vs = [torch.randn(n, HKV, D, generator=gen, device=device).to(f8) for n in lens]
+    q = torch.randn(N_SEQ, HQ, D, generator=gen, device=device, dtype=torch.bfloat16)
+    by = sum(n * HKV * D * 2 for n in lens)
+    best, errors = None, []
+    for tc in (False, True):
+        try:
+            def run():
+                for s in range(N_SEQ):
+                    flashinfer.single_decode_with_kv_cache(q[s], ks[s], vs[s], use_tensor_cores=tc)
+            run()
+            torch.cuda.synchronize()
+            ms = _time_call(torch, run, iters, flush)
+        except Exception as e:
+            errors.append(f"use_tensor_cores={tc}: {type(e).__name__}: {str(e)[:200]}")
+            continue
+        if best is None or ms < best[1]:
+            best = (tc, ms)
+    if best is None:
+        return {"unavailable": "; ".join(errors)}
+    tc, ms = best
+    return {"backend": f"flashinfer {flashinfer.__version__} single_decode_with_kv_cache "
+                       f"(use_tensor_cores={tc})", "ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1),
+            "bytes": by, "tokens_per_s_per_seq": round(1000.0 / ms, 1), "calls": N_SEQ}
+
+
 def run_aux_only(args):
     """One auxiliary workload alone (for profiling a kernel): prints its JSON."""
     import torch
@@ -580,10 +627,11 @@ def run_aux_only(args):
 # Oracle timing (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
 
-def _oracle_unit_sample(n_units: int):
-    """Build oracle state for n_units (sequence, kv-head) units of the
-    streaming workload (untimed) and return a function doing one step on them:
-    quantize a 64-token chunk of K and V and decode the unit's 4 query heads."""
+def _oracle_units(unit_ids):
+    """Build oracle state for some (sequence, kv-head) units of the streaming
+    workload (untimed) and return a function doing one step on them: quantize
+    a 64-token chunk of K and V, append it and decode the unit's 4 query heads.
+    Unit u holds a context as long as sequence u mod 16."""
     import numpy as np
     import torch
 
@@ -594,7 +642,7 @@ def _oracle_unit_sample(n_units: int):
     f = o.Format(3, mixed=True)
     op = o.Params(128, f, f)
     units = []
-    for u in range(n_units):
+    for u in unit_ids:
         s = u % N_SEQ
         n = lens[s]
         k = kv_inputs.kv_vectors(n, D, key=("oracle-k", s, u), dtype=torch.bfloat16).double().numpy()
@@ -624,48 +672,118 @@ def _oracle_unit_sample(n_units: int):
     return one_step
 
 
-def _threads():
+_WORKER_STEP = None
+
+
+def _oracle_worker_init(unit_ids):
+    """Pool worker: one BLAS thread per process, then the worker's units."""
+    global _WORKER_STEP
     try:
-        import numpy  # noqa: F401
-        from threadpoolctl import threadpool_info
-        info = threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] or [1])
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+    _WORKER_STEP = _oracle_units(unit_ids)
+
+
+def _oracle_worker_step(_):
+    return _WORKER_STEP()
+
+
+def _host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
 
 
-def cpu_baseline_stream(args):
-    step = _oracle_unit_sample(args.cpu_units)
+class OraclePool:
+    """The oracle over independent units on all host cores: one spawned
+    process per core (started before any GPU work of the caller matters, and
+    by spawn, never fork), each owning units_per_worker units; a step runs one
+    oracle step in every worker at once."""
+
+    def __init__(self, units_per_worker: int, workers: int | None = None):
+        import multiprocessing as mp
+        # every host core, up to 32 processes (each holds its units' oracle
+        # state and a copy of the numpy / torch runtime)
+        self.workers = workers or min(_host_cores(), 32)
+        self.units = self.workers * units_per_worker
+        ctx = mp.get_context("spawn")
+        self._pools = []
+        # one single-process pool per worker so each gets its own unit ids
+        for w in range(self.workers):
+            ids = list(range(w * units_per_worker, (w + 1) * units_per_worker))
+            self._pools.append(ctx.Pool(1, initializer=_oracle_worker_init, initargs=(ids,)))
+
+    def step(self) -> int:
+        res = [p.apply_async(_oracle_worker_step, (0,)) for p in self._pools]
+        return sum(r.get() for r in res)
+
+    def close(self):
+        for p in self._pools:
+            p.terminate()
+            p.join()
+
+
+def cpu_baseline_stream(args, pool=None):
+    """The oracle timed on the host: all cores (a spawn process pool over
+    independent units) and one thread on one unit."""
+    own = pool is None
+    if own:
+        pool = OraclePool(args.cpu_units)
+    pool.step()  # warm-up: every worker has built its units and run once
     t = time.perf_counter()
-    nbytes = step()
+    nbytes = pool.step()
     dt = time.perf_counter() - t
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"{args.cpu_units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step "
-                      f"(64-token append + 4-head decode each), fp64 numpy, {dt:.1f} s"}
+    workers, units = pool.workers, pool.units
+    if own:
+        pool.close()
+    # one thread, one unit
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(1)
+    except Exception:
+        lim = None
+    one = _oracle_units([0])
+    one()
+    t1 = time.perf_counter()
+    b1 = one()
+    d1 = time.perf_counter() - t1
+    if lim is not None:
+        lim.restore_original_limits()
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": f"{units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step (64-token append "
+                      f"+ 4-head decode each), fp64 numpy oracle, {workers} processes x 1 thread, {dt:.1f} s; "
+                      f"the whole step's 128 units would take about {dt * N_SEQ * HKV / units:.1f} s",
+            "single_thread": {"value": round(b1 / d1 / 1e9, 5), "unit": "GB/s", "units": 1, "s": round(d1, 2)}}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    step = _oracle_unit_sample(args.cpu_units)
-    for _ in range(args.warmup):
-        step()
-    t = time.perf_counter()
-    nbytes = 0
-    for _ in range(args.steps):
-        nbytes += step()
-    dt = time.perf_counter() - t
+    pool = OraclePool(args.cpu_units)
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        t = time.perf_counter()
+        nbytes = 0
+        for _ in range(args.steps):
+            nbytes += pool.step()
+        dt = time.perf_counter() - t
+    finally:
+        pool.close()
     value = nbytes / dt / 1e9
-    sample = (f"{args.cpu_units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step per step "
-              "(64-token append + 4-head decode each), fp64 numpy oracle on host cores")
+    sample = (f"{pool.units} of {N_SEQ * HKV} (sequence, kv-head) units of the streaming step per step "
+              f"(64-token append + 4-head decode each), fp64 numpy oracle, {pool.workers} processes x 1 thread")
     line = {"impl": "reference", "metric": "decode-attn packed-KV GB/s (streaming append + decode step)",
             "value": round(value, 4), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "streaming append + decode: 16 seqs, ctx U[8192,65536], 64-token bf16 chunk, "
                                    "mixed 3.5-bit K/V, 32 q / 8 kv heads, d=128 (bounded sample)"},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": pool.workers, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -679,7 +797,7 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-aux", action="store_true", help="skip the auxiliary workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--cpu-units", type=int, default=2)
+    ap.add_argument("--cpu-units", type=int, default=1, help="oracle units per host core (CPU baseline)")
     ap.add_argument("--aux-only", choices=AUX_WORKLOADS, default=None,
                     help="run one auxiliary workload alone and print its numbers (profiling)")
     ap.add_argument("--formats", default=None, help="with --aux-only quantize-sweep: e.g. mse3,prod3")

@@ -164,14 +164,32 @@ tq_status tq_dequantize(const tq_params* p, const tq_packed* in, int64_t n, int 
 /* A cache for n_seq sequences x n_kv_heads heads.  Token t of a sequence is
  * kept unquantized in bf16 if t < n_sink (attention sink, "Greetings from
  * TurboQuant-MLX", item 1) and is quantized row t - n_sink otherwise.
- * Every plane is laid out [n_seq][n_kv_heads][capacity][row] (sink planes
- * [n_seq][n_kv_heads][n_sink][d]); capacity is a multiple of 64 and counts
- * quantized rows.  lens: device int32 [n_seq], tokens held per sequence
- * (sink included); the caller zeroes it for an empty cache.  status: device
- * int32 word; kernels OR error bits into it (1 = append past capacity,
- * 2 = a length above the bound given to tq_decode_attn, 4 = a decode wait on
- * the copy pipeline gave up after its time limit, 8 = the decode kernel's
- * shared-memory layout did not fit; after 4 or 8 the outputs are invalid). */
+ * capacity is a multiple of 64 and counts quantized rows.  Planes are laid
+ * out per unit: [n_seq][n_kv_heads][...] with a unit's data contiguous.
+ *  - norms, res_norms: [capacity] fp32; qjl: [capacity][m/8] bytes (row order).
+ *  - sink planes: [n_sink][d] bf16.
+ *  - code planes (k_codes, v_codes): [capacity / 16] tiles of 16 rows,
+ *    16 * code_bytes bytes each, arranged for the decode kernel rather than
+ *    in row order.  Write and read them through tq_append,
+ *    tq_cache_write_rows and tq_cache_read_rows.  Inside a tile, lane
+ *    L = 4g + t (g, t in 0..7, 0..3) of the decoding warp owns a block of
+ *    code_bytes / 2 bytes: for keys, of tokens g and g + 8, the bytes of the
+ *    packed row holding quarter t of each code segment ([A.seg0 | B.seg0 |
+ *    A.seg1 | B.seg1], A = token g, B = token g + 8); for values, of tokens
+ *    2t, 2t+1, 2t+8, 2t+9 (a, b, c, d), eighth g of each segment ([a.seg0 |
+ *    b.seg0 | c.seg0 | d.seg0 | a.seg1 | ... | d.seg1]).  A segment is the
+ *    whole row (uniform widths) or one of its two halves of 64 coordinates
+ *    (mixed rows); every such piece is a whole number of bytes.  The blocks
+ *    are stored as columns: the first 16 bytes of every lane (lane L's at
+ *    offset 16 L), then the next 16, then 8, then 4, as the block's size
+ *    needs.  So each lane reads its share with one load per column and the
+ *    warp's loads never share a shared-memory bank.
+ * lens: device int32 [n_seq], tokens held per sequence (sink included); the
+ * caller zeroes it for an empty cache.  status: device int32 word; kernels OR
+ * error bits into it (1 = append past capacity, 2 = a length above the bound
+ * given to tq_decode_attn, 4 = a decode wait on the copy pipeline gave up
+ * after its time limit, 8 = the decode kernel's shared-memory layout did not
+ * fit; after 4 or 8 the outputs are invalid). */
 typedef struct {
   int n_seq, n_kv_heads, capacity, n_sink;
   uint8_t* k_codes; float* k_norms; uint8_t* k_qjl; float* k_res_norms;
@@ -201,17 +219,40 @@ tq_status tq_cache_bind(const tq_params* p, void* base, size_t bytes, int n_seq,
 tq_status tq_append(const tq_params* p, const tq_cache* cache, const int32_t* seq_ids,
                     const void* k, const void* v, int dtype, int n_tok, int n_seq, void* stream);
 
+/* Copy n packed rows (tq_quantize's row format, device planes `rows`, 16-byte
+ * aligned) into quantized rows row0 .. row0 + n - 1 of unit (seq, kv_head) of
+ * the cache, K side (which = TQ_K) or V side: codes into the tiled code plane,
+ * norms, and in prod mode the QJL rows and residual norms.  lens and the sink
+ * are not touched.  For importing rows quantized elsewhere (or by the
+ * oracle in tests).  row0 + n > capacity gives TQ_ERR_CAPACITY.
+ * Asynchronous on `stream`. */
+tq_status tq_cache_write_rows(const tq_params* p, const tq_cache* cache, int which, int seq, int kv_head,
+                              int row0, int64_t n, const tq_packed* rows, void* stream);
+
+/* The reverse: quantized rows row0 .. row0 + n - 1 of unit (seq, kv_head)
+ * into packed rows (tq_quantize's format).  Asynchronous on `stream`. */
+tq_status tq_cache_read_rows(const tq_params* p, const tq_cache* cache, int which, int seq, int kv_head,
+                             int row0, int64_t n, const tq_packed* rows, void* stream);
+
 /* ---- decode attention --------------------------------------------------- */
 
 /* sparse_v_threshold: V of a quantized token is left out when an upper bound
  * on its softmax weight is below this value (0 = off); the softmax
  * denominator keeps every token ("Greetings from TurboQuant-MLX", item 3:
- * 1e-6).  The bound used is exp(s - m)/l over the tokens seen so far, which
- * is never below the final weight, so no token the exact rule keeps is
- * skipped. */
+ * 1e-6).  The bound used is exp(s - m) / max(l, 1) with m the running maximum
+ * of the scores seen so far by the decoding warp and l a partial sum of their
+ * weights; it is never below the final weight, so no token the exact rule
+ * keeps is skipped.  The value work of a 32-token tile is skipped when all its
+ * (token, query head) weights are dropped.
+ * sparse_v_stats: NULL, or a device array of 4 uint64 (8-byte aligned) that
+ * the call adds its tallies to when sparse V is on (the caller zeroes it):
+ * [0] (quantized token, query head) weights examined, [1] weights dropped,
+ * [2] 32-token warp tiles examined, [3] tiles whose value work was skipped.
+ * reserved must be 0. */
 typedef struct {
   float sparse_v_threshold;
   int reserved;
+  unsigned long long* sparse_v_stats;
 } tq_attn_flags;
 
 /* Workspace bytes for tq_decode_attn on B sequences with n_kv_heads heads,
@@ -250,12 +291,15 @@ tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const t
  * synchronization).  No counterpart in the method's pages: it only changes
  * where the workspace lives.  The workspace is a fixed 8 MiB array in device
  * memory defined by the library (every GPU that loads the library holds it
- * until the process exits); a call that would need more returns
- * TQ_ERR_CAPACITY.  No cudaMalloc, cudaFree or other allocation happens.  The
- * first call on each device looks up the array's address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * All calls share the array and each one clears what must start at zero, so
- * calls that overlap on the GPU (for example on two streams) race. */
+ * until the process exits); a call that would need more than 8 MiB (see
+ * tq_decode_workspace_bytes) returns TQ_ERR_CAPACITY.  Arguments are checked
+ * exactly as tq_decode_attn checks them.  No cudaMalloc, cudaFree or other
+ * allocation happens.  The first call on each device looks up the array's
+ * address (cudaGetSymbolAddress), and so does the first call after the
+ * device's context was replaced (cudaDeviceReset); make such a call before any
+ * stream capture.  No call clears the array and none needs to: every word a
+ * kernel reads was written earlier in the same call.  All calls share the
+ * array, so calls that overlap on the GPU (for example on two streams) race. */
 tq_status tq_decode_attn_noalloc(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
                                  int B, int hq, int max_len, void* out, int out_dtype,
                                  const tq_attn_flags* flags, void* stream);

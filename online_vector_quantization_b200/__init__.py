@@ -57,7 +57,7 @@ class TqCache(ctypes.Structure):
 
 
 class TqAttnFlags(ctypes.Structure):
-    _fields_ = [("sparse_v_threshold", c_float), ("reserved", c_int)]
+    _fields_ = [("sparse_v_threshold", c_float), ("reserved", c_int), ("sparse_v_stats", c_void_p)]
 
 
 _SIGS = {
@@ -76,6 +76,10 @@ _SIGS = {
                               ctypes.POINTER(TqCache)]),
     "tq_append": (c_int, [c_void_p, ctypes.POINTER(TqCache), c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                           c_void_p]),
+    "tq_cache_write_rows": (c_int, [c_void_p, ctypes.POINTER(TqCache), c_int, c_int, c_int, c_int, c_int64,
+                                    ctypes.POINTER(TqPacked), c_void_p]),
+    "tq_cache_read_rows": (c_int, [c_void_p, ctypes.POINTER(TqCache), c_int, c_int, c_int, c_int, c_int64,
+                                   ctypes.POINTER(TqPacked), c_void_p]),
     "tq_decode_workspace_bytes": (c_size_t, [c_void_p, c_int, c_int, c_int, c_int]),
     "tq_decode_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
     "tq_decode_attn": (c_int, [c_void_p, c_void_p, c_int, ctypes.POINTER(TqCache), c_int, c_int, c_int, c_void_p,
@@ -240,8 +244,12 @@ class Cache:
         self.n_seq, self.n_kv_heads, self.capacity, self.n_sink = n_seq, n_kv_heads, capacity, n_sink
 
     def plane(self, name: str, dtype, row_elems: int):
-        """View of one plane as a tensor [n_seq][n_kv_heads][rows][row_elems]."""
+        """View of one row-ordered plane (norms, qjl, res_norms, sink) as a
+        tensor [n_seq][n_kv_heads][rows][row_elems].  The code planes are
+        tiled: use read_rows / write_rows for them."""
         import torch
+        if name.endswith("_codes"):
+            raise ValueError("code planes are tiled; use Cache.read_rows / Cache.write_rows")
         ptr = getattr(self.struct, name)
         if not ptr:
             return None
@@ -251,6 +259,22 @@ class Cache:
         off = ptr - self.buffer.data_ptr()
         flat = self.buffer[off: off + count * itemsize].view(dtype)
         return flat.view(self.n_seq, self.n_kv_heads, rows, row_elems)
+
+
+def tq_cache_write_rows(params: Params, cache: Cache, which: int, seq: int, kv_head: int, row0: int,
+                        rows: Packed, n: int, stream=None):
+    """Copy n packed rows into quantized rows row0.. of unit (seq, kv_head)."""
+    st = rows.struct()
+    _check(_lib.tq_cache_write_rows(params.handle, ctypes.byref(cache.struct), which, seq, kv_head, row0, n,
+                                    ctypes.byref(st), _stream(stream)))
+
+
+def tq_cache_read_rows(params: Params, cache: Cache, which: int, seq: int, kv_head: int, row0: int,
+                       rows: Packed, n: int, stream=None):
+    """Copy quantized rows row0 .. row0 + n - 1 of unit (seq, kv_head) out as packed rows."""
+    st = rows.struct()
+    _check(_lib.tq_cache_read_rows(params.handle, ctypes.byref(cache.struct), which, seq, kv_head, row0, n,
+                                   ctypes.byref(st), _stream(stream)))
 
 
 def tq_append(params: Params, cache: Cache, seq_ids, k, v, stream=None):
@@ -278,10 +302,11 @@ def decode_workspace(params: Params, B: int, hq: int, n_kv_heads: int, max_len: 
 
 
 def tq_decode_attn(params: Params, q, cache: Cache, max_len: int, out, workspace,
-                   sparse_v_threshold: float = 0.0, stream=None):
-    """q, out: (B, hq, d) CUDA tensors (fp32 or bf16)."""
+                   sparse_v_threshold: float = 0.0, stream=None, sparse_v_stats=None):
+    """q, out: (B, hq, d) CUDA tensors (fp32 or bf16).  sparse_v_stats: None
+    or a (4,) int64 CUDA tensor the call adds its sparse-V tallies to."""
     B, hq = q.shape[0], q.shape[1]
-    flags = TqAttnFlags(sparse_v_threshold, 0)
+    flags = TqAttnFlags(sparse_v_threshold, 0, _ptr(sparse_v_stats))
     _check(_lib.tq_decode_attn(params.handle, _ptr(q), _dtype_code(q), ctypes.byref(cache.struct), B, hq,
                                max_len, _ptr(out), _dtype_code(out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), ctypes.byref(flags),
@@ -289,11 +314,11 @@ def tq_decode_attn(params: Params, q, cache: Cache, max_len: int, out, workspace
 
 
 def tq_decode_attn_noalloc(params: Params, q, cache: Cache, max_len: int, out, sparse_v_threshold: float = 0.0,
-                           stream=None):
+                           stream=None, sparse_v_stats=None):
     """tq_decode_attn with the library's fixed device scratch instead of a
     caller workspace (see include/tq.h)."""
     B, hq = q.shape[0], q.shape[1]
-    flags = TqAttnFlags(sparse_v_threshold, 0)
+    flags = TqAttnFlags(sparse_v_threshold, 0, _ptr(sparse_v_stats))
     _check(_lib.tq_decode_attn_noalloc(params.handle, _ptr(q), _dtype_code(q), ctypes.byref(cache.struct), B, hq,
                                        max_len, _ptr(out), _dtype_code(out), ctypes.byref(flags), _stream(stream)))
 

@@ -59,18 +59,18 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
   const float wA = okA ? ldsf(u.vnorm, (srow + tr.kA) * 4) : 0.f, wB = okB ? ldsf(u.vnorm, (srow + tr.kB) * 4) : 0.f;
   const uint32_t pb0 = movmatrix_t(h2bits(p[0] * wA, p[1] * wA));
   const uint32_t pb1 = movmatrix_t(h2bits(p[2] * wB, p[3] * wB));
-  // rows of MMA columns 2t, 2t+1, 2t+8, 2t+9
-  const uint32_t r0p = u.vcodes + (srow + tr.v0) * FV::code_bytes;
-  const uint32_t r1p = u.vcodes + (srow + tr.v1) * FV::code_bytes;
-  const uint32_t r8p = u.vcodes + (srow + tr.v8) * FV::code_bytes;
-  const uint32_t r9p = u.vcodes + (srow + tr.v9) * FV::code_bytes;
+  // tiled V codes (tq_layout.cuh): this lane's block holds tokens 2t, 2t+1,
+  // 2t+8, 2t+9 (MMA columns) of the subtile, its eighth g of each segment
+  constexpr CodeTile CT = code_tile<VF>();
+  [[maybe_unused]] LaneBlock<VF> blk;
+  if constexpr (FV::nseg > 0) blk.load(u.vcodes + (srow >> 4) * CT.tile_bytes(), 4 * g + t);
   if constexpr (FV::nseg > 0) {
     constexpr int MT = VR::S0::MT;
     typename VR::S0 xa, xb, xc, xd;
-    xa.load(r0p, g);
-    xb.load(r1p, g);
-    xc.load(r8p, g);
-    xd.load(r9p, g);
+    xa.template from_block<CT.voff(0, 0)>(blk);
+    xb.template from_block<CT.voff(1, 0)>(blk);
+    xc.template from_block<CT.voff(2, 0)>(blk);
+    xd.template from_block<CT.voff(3, 0)>(blk);
     uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
     const uint32_t lut = FV::b0 == 2 ? lut_b : lut_a;
     VR::S0::template decode<T2A>(xa, xb, lut, lane4, lane8, c1v, r0, r08);
@@ -81,10 +81,10 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
   if constexpr (FV::nseg > 1) {
     constexpr int MT = VR::S1::MT;
     typename VR::S1 xa, xb, xc, xd;
-    xa.load(r0p, g);
-    xb.load(r1p, g);
-    xc.load(r8p, g);
-    xd.load(r9p, g);
+    xa.template from_block<CT.voff(0, 1)>(blk);
+    xb.template from_block<CT.voff(1, 1)>(blk);
+    xc.template from_block<CT.voff(2, 1)>(blk);
+    xd.template from_block<CT.voff(3, 1)>(blk);
     uint32_t r0[MT], r08[MT], r1[MT], r18[MT];
     const uint32_t lut = FV::b1 == 2 ? lut_b : lut_a;
     VR::S1::template decode<T2A>(xa, xb, lut, lane4, lane8, c1v, r0, r08);
@@ -110,26 +110,34 @@ __device__ __forceinline__ void subtile_pv(const UnitPlanes& u, int srow, const 
   }
 }
 
+// Sparse-V tallies of one lane (summed over the grid when the caller asks for
+// them): (token, query head) weights examined and dropped, 32-token warp
+// tiles examined and tiles whose value work was skipped.
+struct SparseTally {
+  unsigned examined = 0, dropped = 0, tiles = 0, tiles_skipped = 0;
+};
+
 // One warp tile of 32 tokens (two 16-token subtiles) starting at stage row
 // `srow`, unit-relative row `row0`; tokens at or past `nq` are masked (their
 // scores are -inf and their value weights 0, so a subtile past the end adds
 // nothing; computing it anyway keeps the two subtiles free of branches, which
-// lets their lookup and MMA chains interleave).  SPARSE: skip the PV MMAs of
-// a subtile whose weights are all below the sparse-V threshold.
-template <int KF, int VF, bool PACK, int WT, bool SPARSE>
+// lets their lookup and MMA chains interleave).  SPARSE: 0 dense; 1 sparse V
+// (weights below the bound are dropped, and the PV work of a tile whose
+// weights are all dropped is skipped); 2 the same with tallies.
+template <int KF, int VF, bool PACK, int WT, int SPARSE>
 __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int row0, int nq, const TokRows& tr,
                                              WarpState<KF, VF, PACK>& W, const QFrag<PACK>& bq,
                                              const QFrag<PACK>& bqs, int g, int t, uint32_t lut_a,
                                              uint32_t lut_b, uint32_t lane4, uint32_t lane8,
-                                             uint32_t c1k, uint32_t c1v, float thr) {
+                                             uint32_t c1k, uint32_t c1v, float thr, int group, SparseTally& tally) {
   constexpr int VMT = WarpState<KF, VF, PACK>::VMT;
   constexpr bool second = WT == 2 * kTok;
   const bool ok0A = row0 + tr.kA < nq, ok0B = row0 + tr.kB < nq;
   const bool ok1A = row0 + kTok + tr.kA < nq, ok1B = row0 + kTok + tr.kB < nq;
   float s0[4], s1[4];
-  subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
+  subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a, false, true>(u, srow, tr, ok0A, ok0B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s0);
   if constexpr (second)
-    subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
+    subtile_scores<KF, PACK, Lut<KF, VF>::t3_wide, Lut<KF, VF>::t2a, false, true>(u, srow + kTok, tr, ok1A, ok1B, g, t, bq, bqs, lut_a, lut_b, lane4, lane8, c1k, s1);
   else
     s1[0] = s1[1] = s1[2] = s1[3] = -INFINITY;
   // online softmax over the 32 tokens (base 2), columns 2t and 2t+1.  The
@@ -172,26 +180,50 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
     W.l0 += (p0[0] + p0[2]) + (p1[0] + p1[2]);
     W.l1 += (p0[1] + p0[3]) + (p1[1] + p1[3]);
   }
-  if constexpr (!SPARSE) {
+  if constexpr (SPARSE == 0) {
     subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
     if constexpr (second)
       subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
   } else {
-    // sparse V: exp(s - m) / l over the tokens seen so far bounds the final
-    // weight, and this lane's partial sum is at most l, so p < thr * l_lane
-    // only skips tokens whose final weight is below thr
-    const float c0 = thr * W.l0, c1 = thr * W.l1;
+    // Sparse V ("Greetings from TurboQuant-MLX", item 3): the value of a token
+    // whose weight is below thr is left out (the denominator keeps it).  The
+    // final weight is exp(s - M) / L with M, L the max and sum over all the
+    // unit's tokens; exp(s - m) / l_w with m, l_w this warp's running max and
+    // sum is never below it, and l_w is at least this lane's partial sum and
+    // at least 1 (the token at the running max counts exp(0)).  So a weight
+    // below thr * max(l_lane, 1) is below thr in the end: no token the exact
+    // rule keeps is dropped.
+    const float c0 = thr * fmaxf(W.l0, 1.f), c1 = thr * fmaxf(W.l1, 1.f);
+    const bool col0 = 2 * t < group, col1 = 2 * t + 1 < group;  // real heads (packed: the hi columns)
+    const bool okr[4] = {ok0A, ok0B, ok1A, ok1B};
+    float* pp[4] = {&p0[0], &p0[2], &p1[0], &p1[2]};
+    bool keep = false;
 #pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-      p0[i] = p0[i] >= c0 ? p0[i] : 0.f;
-      p0[i + 1] = p0[i + 1] >= c1 ? p0[i + 1] : 0.f;
-      p1[i] = p1[i] >= c0 ? p1[i] : 0.f;
-      p1[i + 1] = p1[i + 1] >= c1 ? p1[i + 1] : 0.f;
+    for (int r = 0; r < 4; ++r) {
+      float* pr = pp[r];
+      const bool d0 = pr[0] < c0, d1 = pr[1] < c1;
+      if constexpr (SPARSE == 2) {
+        if (okr[r]) {
+          tally.examined += col0 + col1;
+          tally.dropped += (col0 && d0) + (col1 && d1);
+        }
+      }
+      pr[0] = d0 ? 0.f : pr[0];
+      pr[1] = d1 ? 0.f : pr[1];
+      // columns past the group (empty heads) never keep a tile alive
+      keep |= (col0 && pr[0] > 0.f) | (col1 && pr[1] > 0.f);
     }
-    if (__any_sync(0xffffffffu, (p0[0] + p0[1] + p0[2] + p0[3]) > 0.f))
+    if constexpr (SPARSE == 2) ++tally.tiles;
+    // the value work is skipped only when every weight of the warp tile was
+    // dropped; otherwise both subtiles run without branches, as on the dense
+    // path (a per-subtile branch costs more than it saves at GQA widths)
+    if (__any_sync(0xffffffffu, keep)) {
       subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow, tr, ok0A, ok0B, g, t, p0, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
-    if (second && __any_sync(0xffffffffu, (p1[0] + p1[1] + p1[2] + p1[3]) > 0.f))
-      subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+      if constexpr (second)
+        subtile_pv<VF, VMT, Lut<KF, VF>::t2a>(u, srow + kTok, tr, ok1A, ok1B, g, t, p1, lut_a, lut_b, lane4, lane8, c1v, W.oacc);
+    } else if constexpr (SPARSE == 2) {
+      ++tally.tiles_skipped;
+    }
   }
 }
 
@@ -674,7 +706,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
 }
 
 
-template <int KF, int VF, bool PACK, bool SPARSE>
+template <int KF, int VF, bool PACK, int SPARSE>
 __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   using FK = Fmt<KF>;
   using FV = Fmt<VF>;
@@ -840,7 +872,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const float thr = a.sparse_thr;
-  const TokRows trows = tok_rows<KF, VF>(g, t);
+  const TokRows trows = tok_rows(g, t);
 
   pdl_wait();  // the rotated query fragments
 
@@ -853,6 +885,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const int nk = static_cast<int>(c1 - c0);
   int s = 0;
   uint32_t round = 0;  // parity of k / S
+  SparseTally tally;
   for (int k = 0; k < nk; ++k) {
     while (walk_lc >= wui.chunks) {
       ++walk_u;
@@ -892,7 +925,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       sp.vq = st + SL::vq;
       sp.vres = st + SL::vr;
       compute_tile<KF, VF, PACK, WT, SPARSE>(sp, warp * WT, row0, ui.nq, trows, wst, bq, bqs, g, t, lut_a, lut_b, lane4, lane8,
-                                 c1k, c1v, thr);
+                                             c1k, c1v, thr, a.group, tally);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
@@ -904,6 +937,20 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   }
   if (u >= 0) write_piece<KF, VF, PACK, true>(a, wst, u + cta, scratch, warp, g, t);
   if (s_abort && tid == 0) atomicOr(a.status, 4);
+  if constexpr (SPARSE == 2) {
+    {
+      unsigned long long v[4] = {tally.examined, tally.dropped, lane == 0 ? tally.tiles : 0u,
+                                 lane == 0 ? tally.tiles_skipped : 0u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) atomicAdd(a.sv_stats + i, v[i]);
+    }
+  }
 }
 
 
@@ -913,7 +960,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
 
 
 
-template <int KF, int VF, bool PACK, bool SPARSE>
+template <int KF, int VF, bool PACK, int SPARSE>
 tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaStream_t st) {
   cudaError_t e = ensure_dyn_smem<decode_kernel<KF, VF, PACK, SPARSE>>(static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
@@ -945,9 +992,11 @@ tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
   a.dyn_bytes = static_cast<uint32_t>(smem);
   a.pack = plan.group <= 4;
   a.chunk = DecodeCfg<KF, VF>::CH;
+  if (a.sparse_thr > 0.f && a.sv_stats)
+    return a.pack ? run_decode_v<KF, VF, true, 2>(a, plan, smem, st) : run_decode_v<KF, VF, false, 2>(a, plan, smem, st);
   if (a.sparse_thr > 0.f)
-    return a.pack ? run_decode_v<KF, VF, true, true>(a, plan, smem, st) : run_decode_v<KF, VF, false, true>(a, plan, smem, st);
-  return a.pack ? run_decode_v<KF, VF, true, false>(a, plan, smem, st) : run_decode_v<KF, VF, false, false>(a, plan, smem, st);
+    return a.pack ? run_decode_v<KF, VF, true, 1>(a, plan, smem, st) : run_decode_v<KF, VF, false, 1>(a, plan, smem, st);
+  return a.pack ? run_decode_v<KF, VF, true, 0>(a, plan, smem, st) : run_decode_v<KF, VF, false, 0>(a, plan, smem, st);
 }
 
 
@@ -972,7 +1021,8 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) 
 }
 
 tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c, const DecodePlan& plan,
-                        void* out, int out_bf16, void* ws, float sparse_thr, cudaStream_t st) {
+                        void* out, int out_bf16, void* ws, float sparse_thr, unsigned long long* sv_stats,
+                        cudaStream_t st) {
   DecodeArgs a{};
   a.q = q;
   a.q_bf16 = q_bf16;
@@ -1019,6 +1069,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.cbs = p->cbs32;
   a.sig = p->sig32;
   a.sparse_thr = sparse_thr;
+  a.sv_stats = sv_stats;
   a.qscale = kLog2e / std::sqrt(static_cast<float>(kDim));
 
   const int kf = p->fk.id(), vf = p->fv.id();

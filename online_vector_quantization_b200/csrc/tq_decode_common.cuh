@@ -20,6 +20,7 @@
 #include <cmath>
 
 #include "tq_internal.h"
+#include "tq_layout.cuh"
 #include "tq_sm100.cuh"
 
 namespace tq {
@@ -224,6 +225,12 @@ struct KChunk {
     }
   }
 
+  // the lane's piece at byte OFF of its lane block in a tiled code plane
+  template <int OFF, typename Blk>
+  __device__ __forceinline__ void from_block(const Blk& blk) {
+    blk.template words<OFF, WORDS>(w);
+  }
+
   // 64-bit window holding the 6-bit field p (3-bit chunks)
   template <int P>
   __device__ __forceinline__ uint32_t pair3(uint32_t lb) const {
@@ -315,6 +322,16 @@ struct VChunk {
     }
   }
 
+  // the token's piece (ND * B / 64 bytes) at byte OFF of the lane block
+  template <int OFF, typename Blk>
+  __device__ __forceinline__ void from_block(const Blk& blk) {
+    constexpr int bits = ND * B / 8;
+    uint32_t v[2];
+    blk.template words<OFF, 2>(v);
+    const uint64_t y = static_cast<uint64_t>(v[0]) | (static_cast<uint64_t>(v[1]) << 32);
+    x = bits == 64 ? y : (y & ((1ull << bits) - 1ull));
+  }
+
   // rows g (coordinate 2mt) and g+8 (2mt+1) for every m-tile, tokens (A, B)
   template <bool T2A = false>
   __device__ __forceinline__ static void decode(const VChunk& a, const VChunk& b, uint32_t smem,
@@ -397,6 +414,47 @@ struct VRow {
   using Q = VChunk<1, 128, 0>;
 };
 
+// One lane's block of a tiled code plane (see tq_layout.cuh): loaded with one
+// 16-, 8- and 4-byte shared load per column, conflict-free across the warp.
+template <int F>
+__host__ __device__ constexpr CodeTile code_tile() {
+  return make_code_tile(Fmt<F>::mse, Fmt<F>::mixed, Fmt<F>::code_bytes);
+}
+
+template <int F>
+struct LaneBlock {
+  static constexpr CodeTile CT = code_tile<F>();
+  static constexpr int WORDS = CT.lane_bytes() / 4 > 0 ? CT.lane_bytes() / 4 : 1;
+  uint32_t w[WORDS];
+
+  // tile: shared address of the 16-token tile
+  __device__ __forceinline__ void load(uint32_t tile, int lane) {
+    static_for<CT.c16()>([&](auto jj) {
+      constexpr int j = decltype(jj)::value;
+      const uint4 v = lds128(tile, j * 512 + lane * 16);
+      w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+    });
+    if constexpr (CT.c8() > 0) {
+      const uint2 v = lds64(tile, 512 * CT.c16() + lane * 8);
+      w[4 * CT.c16()] = v.x;
+      w[4 * CT.c16() + 1] = v.y;
+    }
+    if constexpr (CT.c4() > 0) w[4 * CT.c16() + 2 * CT.c8()] = lds32(tile, 512 * CT.c16() + 256 * CT.c8() + lane * 4);
+  }
+
+  // NW little-endian words starting at byte OFF of the block (bytes past the
+  // block's end are unspecified)
+  template <int OFF, int NW>
+  __device__ __forceinline__ void words(uint32_t (&out)[NW]) const {
+    constexpr int w0 = OFF / 4, sh = (OFF % 4) * 8;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const uint32_t lo = w[min(w0 + i, WORDS - 1)], hi = w[min(w0 + i + 1, WORDS - 1)];
+      out[i] = sh == 0 ? lo : __funnelshift_r(lo, hi, sh);
+    }
+  }
+};
+
 struct DecodeArgs {
   const void* q;
   int q_bf16;
@@ -428,6 +486,7 @@ struct DecodeArgs {
   const float* cbs;  // sigma-scaled centroids [5][16] (the values the MMAs see)
   const float* sig;  // sigma per width [5]
   float sparse_thr;
+  unsigned long long* sv_stats;  // sparse-V tallies [4] (device) or null
   int pack;          // 1: group <= 4, query hi/lo halves share one MMA (columns g and g+4)
   uint32_t dyn_bytes;  // dynamic shared memory granted to the decode kernel
   float qscale;      // factor on the rotated query: log2(e)/sqrt(d) for attention, 1 for search
@@ -661,35 +720,15 @@ struct WarpState {
 template <bool PACK>
 using QFrag = uint32_t[8][2][PACK ? 1 : 2];
 
-// Token order inside a 16-token subtile.  MMA row / column k of a subtile
-// holds physical token pi[k] (K and V use the same order, so the scores,
-// softmax weights and V columns line up).  The order only changes which
-// shared-memory banks the code loads hit: lane (g, t) reads K rows pi[g],
-// pi[g + 8] and V rows pi[2t], pi[2t + 1], pi[2t + 8], pi[2t + 9], and rows of
-// 24..64 bytes make some orders collide less.  pi[k] is nibble k of the word;
-// the words come from a search over a model of these loads (bank_perm.py next
-// to this file), identity where no order helps.
-__host__ __device__ constexpr uint64_t token_order(int kf, int vf) {
-  return kf == 2 && vf == 2     ? 0xFE095427B86D1AC3ull
-         : kf == 4 && vf == 4   ? 0xB2CD41F863905AE7ull
-         : kf == 11 && vf == 11 ? 0x2AE619D534F8BC70ull
-         : kf == 10 && vf == 10 ? 0xA428EC6031F97DB5ull
-         : kf == 18 && vf == 18 ? 0xB6C51FA82907D43Eull
-         : kf == 4 && vf == 2   ? 0xB856274109A3DEFCull
-         : kf == 3 && vf == 2   ? 0xC1B7502E948F3D6Aull
-                                : 0xFEDCBA9876543210ull;
-}
-
-// This lane's physical rows within a subtile: K rows (score rows g, g + 8)
-// and V rows (MMA columns 2t, 2t + 1, 2t + 8, 2t + 9).
+// This lane's rows within a 16-token subtile: K rows (score rows g, g + 8)
+// and V rows (MMA columns 2t, 2t + 1, 2t + 8, 2t + 9).  In a tiled code plane
+// the tile layout already gives every lane its own banks, so tokens sit in
+// MMA row / column order.
 struct TokRows {
   int kA, kB, v0, v1, v8, v9;
 };
-template <int KF, int VF>
 __device__ __forceinline__ TokRows tok_rows(int g, int t) {
-  constexpr uint64_t pi = token_order(KF, VF);
-  auto at = [](int k) { return static_cast<int>((pi >> (4 * k)) & 15u); };
-  return TokRows{at(g), at(g + 8), at(2 * t), at(2 * t + 1), at(2 * t + 8), at(2 * t + 9)};
+  return TokRows{g, g + 8, 2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
 }
 
 // Scores of one 16-token subtile whose rows start at `srow` of the staged
@@ -698,7 +737,10 @@ __device__ __forceinline__ TokRows tok_rows(int g, int t) {
 // HI: the query's fp16 high halves only (column g = head g, no low halves):
 // one MMA per k-step for up to 8 heads, scores within about 2^-12 of
 // ||q|| ||x|| (the search's precision; attention keeps both halves).
-template <int KF, bool PACK, bool T3W, bool T2A, bool HI = false>
+// TILED: the K code plane is a tiled cache plane (tq_layout.cuh: token g and
+// g + 8 of the subtile are this lane's rows A and B); otherwise rows are
+// packed rows in token order tr (the search's database).
+template <int KF, bool PACK, bool T3W, bool T2A, bool HI = false, bool TILED = false>
 __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, const TokRows& tr, bool okA, bool okB,
                                                int g, int t,
                                                const QFrag<PACK || HI>& bq, const QFrag<PACK || HI>& bqs,
@@ -714,10 +756,17 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
   const uint32_t kb = u.kcodes + rB * FK::code_bytes;
   float ca[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float cq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  [[maybe_unused]] LaneBlock<KF> blk;
+  if constexpr (TILED && FK::nseg > 0) blk.load(u.kcodes + (srow >> 4) * code_tile<KF>().tile_bytes(), 4 * g + t);
   if constexpr (FK::nseg > 0) {
     typename KR::S0 xa, xb;
-    xa.load(ka, t);
-    xb.load(kb, t);
+    if constexpr (TILED) {
+      xa.template from_block<code_tile<KF>().koff(0, 0)>(blk);
+      xb.template from_block<code_tile<KF>().koff(1, 0)>(blk);
+    } else {
+      xa.load(ka, t);
+      xb.load(kb, t);
+    }
     const uint32_t lk = FK::b0 == 2 ? lut_b : lut_a;
     static_for<KR::S0::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;
@@ -730,8 +779,13 @@ __device__ __forceinline__ void subtile_scores(const UnitPlanes& u, int srow, co
   }
   if constexpr (FK::nseg > 1) {
     typename KR::S1 xa, xb;
-    xa.load(ka, t);
-    xb.load(kb, t);
+    if constexpr (TILED) {
+      xa.template from_block<code_tile<KF>().koff(0, 1)>(blk);
+      xb.template from_block<code_tile<KF>().koff(1, 1)>(blk);
+    } else {
+      xa.load(ka, t);
+      xb.load(kb, t);
+    }
     const uint32_t lk = FK::b1 == 2 ? lut_b : lut_a;
     static_for<KR::S1::KSTEPS>([&](auto ss) {
       constexpr int s = decltype(ss)::value;

@@ -358,6 +358,53 @@ static bool make_format(int bits, int mode, int mixed, FormatSpec* f, std::strin
   return true;
 }
 
+// ---- argument checks shared by the entry points --------------------------
+
+static bool aligned16_ptr(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+tq_status check_cache(const tq_params* p, const tq_cache* c, const char* who) {
+  if (!c) return fail(TQ_ERR_ARG, std::string(who) + ": NULL cache");
+  if (c->n_seq < 1 || c->n_kv_heads < 1 || c->capacity < 0 || c->capacity % 64 || c->n_sink < 0)
+    return fail(TQ_ERR_ARG, std::string(who) + ": bad cache sizes");
+  if (!c->lens || !c->status || !c->k_norms || !c->v_norms || (p->fk.code_bytes && !c->k_codes) ||
+      (p->fv.code_bytes && !c->v_codes) || (p->fk.prod && (!c->k_qjl || !c->k_res_norms)) ||
+      (p->fv.prod && (!c->v_qjl || !c->v_res_norms)) || (c->n_sink && (!c->k_sink || !c->v_sink)))
+    return fail(TQ_ERR_ARG, std::string(who) + ": a cache plane is NULL");
+  const void* planes[] = {c->k_codes, c->k_norms, c->k_qjl, c->k_res_norms, c->v_codes,
+                          c->v_norms, c->v_qjl, c->v_res_norms, c->k_sink, c->v_sink};
+  for (const void* pl : planes)
+    if (pl && !aligned16_ptr(pl)) return fail(TQ_ERR_ALIGN, std::string(who) + ": cache planes must be 16-byte aligned");
+  return TQ_OK;
+}
+
+tq_status check_decode_call(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache, int B, int hq,
+                            int max_len, const void* out, int out_dtype, const tq_attn_flags* flags,
+                            const char* who, DecodePlan* plan, float* thr, unsigned long long** sv_stats) {
+  const std::string w(who);
+  if (!p) return fail(TQ_ERR_ARG, w + ": NULL params");
+  tq_status st = check_cache(p, cache, who);
+  if (st != TQ_OK) return st;
+  if (B < 1 || B > cache->n_seq || hq < 1 || max_len < 0 || (q_dtype != TQ_F32 && q_dtype != TQ_BF16) ||
+      (out_dtype != TQ_F32 && out_dtype != TQ_BF16))
+    return fail(TQ_ERR_ARG, w + ": bad B, hq, max_len or dtype");
+  const int hkv = cache->n_kv_heads;
+  if (hq % hkv) return fail(TQ_ERR_ARG, w + ": hq must be a multiple of n_kv_heads");
+  if (hq / hkv > 8) return fail(TQ_ERR_UNSUPPORTED, w + ": at most 8 query heads per kv-head");
+  if (max_len > cache->capacity + cache->n_sink) return fail(TQ_ERR_ARG, w + ": max_len above the cache's capacity");
+  if (!q || !out) return fail(TQ_ERR_ARG, w + ": NULL q or out");
+  if (!aligned16_ptr(q) || !aligned16_ptr(out)) return fail(TQ_ERR_ALIGN, w + ": q and out must be 16-byte aligned");
+  const float t = flags ? flags->sparse_v_threshold : 0.f;
+  if (!(t >= 0.f) || t >= 1.f) return fail(TQ_ERR_ARG, w + ": sparse_v_threshold must be in [0, 1)");
+  if (flags && flags->reserved != 0) return fail(TQ_ERR_ARG, w + ": flags->reserved must be 0");
+  unsigned long long* stats = flags ? flags->sparse_v_stats : nullptr;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7))
+    return fail(TQ_ERR_ALIGN, w + ": sparse_v_stats must be 8-byte aligned");
+  *thr = t;
+  *sv_stats = stats;
+  *plan = plan_decode(p, B, hq, hkv, max_len);
+  return TQ_OK;
+}
+
 }  // namespace tq
 
 using namespace tq;
@@ -701,21 +748,6 @@ tq_status tq_cache_bind(const tq_params* p, void* base, size_t bytes, int n_seq,
   return TQ_OK;
 }
 
-static tq_status check_cache(const tq_params* p, const tq_cache* c, const char* who) {
-  if (!c) return fail(TQ_ERR_ARG, std::string(who) + ": NULL cache");
-  if (c->n_seq < 1 || c->n_kv_heads < 1 || c->capacity < 0 || c->capacity % 64 || c->n_sink < 0)
-    return fail(TQ_ERR_ARG, std::string(who) + ": bad cache sizes");
-  if (!c->lens || !c->status || !c->k_norms || !c->v_norms || (p->fk.code_bytes && !c->k_codes) ||
-      (p->fv.code_bytes && !c->v_codes) || (p->fk.prod && (!c->k_qjl || !c->k_res_norms)) ||
-      (p->fv.prod && (!c->v_qjl || !c->v_res_norms)) || (c->n_sink && (!c->k_sink || !c->v_sink)))
-    return fail(TQ_ERR_ARG, std::string(who) + ": a cache plane is NULL");
-  const void* planes[] = {c->k_codes, c->k_norms, c->k_qjl, c->k_res_norms, c->v_codes,
-                          c->v_norms, c->v_qjl, c->v_res_norms, c->k_sink, c->v_sink};
-  for (const void* pl : planes)
-    if (pl && !aligned16(pl)) return fail(TQ_ERR_ALIGN, std::string(who) + ": cache planes must be 16-byte aligned");
-  return TQ_OK;
-}
-
 tq_status tq_append(const tq_params* p, const tq_cache* cache, const int32_t* seq_ids, const void* k,
                     const void* v, int dtype, int n_tok, int n_seq, void* stream) {
   if (!p) return fail(TQ_ERR_ARG, "tq_append: NULL params");
@@ -728,6 +760,31 @@ tq_status tq_append(const tq_params* p, const tq_cache* cache, const int32_t* se
   if (!aligned16(k) || !aligned16(v)) return fail(TQ_ERR_ALIGN, "tq_append: inputs must be 16-byte aligned");
   return launch_append(p, cache, seq_ids, k, v, dtype == TQ_BF16, n_tok, n_seq,
                        static_cast<cudaStream_t>(stream));
+}
+
+static tq_status cache_rows(const tq_params* p, const tq_cache* cache, int which, int seq, int kv_head, int row0,
+                            int64_t n, const tq_packed* rows, void* stream, int to_cache, const char* who) {
+  if (!p) return fail(TQ_ERR_ARG, std::string(who) + ": NULL params");
+  tq_status st = check_cache(p, cache, who);
+  if (st != TQ_OK) return st;
+  if ((which != TQ_K && which != TQ_V) || seq < 0 || seq >= cache->n_seq || kv_head < 0 ||
+      kv_head >= cache->n_kv_heads || row0 < 0 || n < 0)
+    return fail(TQ_ERR_ARG, std::string(who) + ": bad which, seq, kv_head, row0 or n");
+  if (row0 + n > cache->capacity) return fail(TQ_ERR_CAPACITY, std::string(who) + ": rows past the cache's capacity");
+  if (n == 0) return TQ_OK;
+  st = check_packed(which == TQ_K ? p->fk : p->fv, rows, who);
+  if (st != TQ_OK) return st;
+  return launch_cache_rows(p, cache, which, seq, kv_head, row0, n, rows, to_cache, static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_cache_write_rows(const tq_params* p, const tq_cache* cache, int which, int seq, int kv_head, int row0,
+                              int64_t n, const tq_packed* rows, void* stream) {
+  return cache_rows(p, cache, which, seq, kv_head, row0, n, rows, stream, 1, "tq_cache_write_rows");
+}
+
+tq_status tq_cache_read_rows(const tq_params* p, const tq_cache* cache, int which, int seq, int kv_head, int row0,
+                             int64_t n, const tq_packed* rows, void* stream) {
+  return cache_rows(p, cache, which, seq, kv_head, row0, n, rows, stream, 0, "tq_cache_read_rows");
 }
 
 size_t tq_decode_workspace_bytes(const tq_params* p, int B, int hq, int n_kv_heads, int max_len) {
@@ -744,25 +801,16 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
 tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache, int B,
                          int hq, int max_len, void* out, int out_dtype, void* workspace, size_t ws_bytes,
                          const tq_attn_flags* flags, void* stream) {
-  if (!p) return fail(TQ_ERR_ARG, "tq_decode_attn: NULL params");
-  tq_status st = check_cache(p, cache, "tq_decode_attn");
+  DecodePlan plan;
+  float thr = 0.f;
+  unsigned long long* sv_stats = nullptr;
+  tq_status st = check_decode_call(p, q, q_dtype, cache, B, hq, max_len, out, out_dtype, flags, "tq_decode_attn",
+                                   &plan, &thr, &sv_stats);
   if (st != TQ_OK) return st;
-  if (B < 1 || B > cache->n_seq || hq < 1 || max_len < 0 || (q_dtype != TQ_F32 && q_dtype != TQ_BF16) ||
-      (out_dtype != TQ_F32 && out_dtype != TQ_BF16))
-    return fail(TQ_ERR_ARG, "tq_decode_attn: bad B, hq, max_len or dtype");
-  const int hkv = cache->n_kv_heads;
-  if (hq % hkv) return fail(TQ_ERR_ARG, "tq_decode_attn: hq must be a multiple of n_kv_heads");
-  if (hq / hkv > 8) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: at most 8 query heads per kv-head");
-  if (max_len > cache->capacity + cache->n_sink)
-    return fail(TQ_ERR_ARG, "tq_decode_attn: max_len above the cache's capacity");
-  if (!q || !out || !workspace) return fail(TQ_ERR_ARG, "tq_decode_attn: NULL q, out or workspace");
-  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
-    return fail(TQ_ERR_ALIGN, "tq_decode_attn: q, out and workspace must be 16-byte aligned");
-  DecodePlan plan = plan_decode(p, B, hq, hkv, max_len);
+  if (!workspace) return fail(TQ_ERR_ARG, "tq_decode_attn: NULL workspace");
+  if (!aligned16(workspace)) return fail(TQ_ERR_ALIGN, "tq_decode_attn: workspace must be 16-byte aligned");
   if (ws_bytes < plan.ws_total_bytes) return fail(TQ_ERR_CAPACITY, "tq_decode_attn: workspace too small");
-  float thr = flags ? flags->sparse_v_threshold : 0.f;
-  if (!(thr >= 0.f) || thr >= 1.f) return fail(TQ_ERR_ARG, "tq_decode_attn: sparse_v_threshold must be in [0, 1)");
-  return launch_decode(p, q, q_dtype == TQ_BF16, cache, plan, out, out_dtype == TQ_BF16, workspace, thr,
+  return launch_decode(p, q, q_dtype == TQ_BF16, cache, plan, out, out_dtype == TQ_BF16, workspace, thr, sv_stats,
                        static_cast<cudaStream_t>(stream));
 }
 

@@ -100,6 +100,8 @@ tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x
 tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* seq_ids,
                         const void* k, const void* v, int x_bf16, int n_tok, int n_seq,
                         cudaStream_t st);
+tq_status launch_cache_rows(const tq_params* p, const tq_cache* c, int which, int seq, int kv_head, int row0,
+                            int64_t n, const tq_packed* rows, int to_cache, cudaStream_t st);
 tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_packed* in,
                             int64_t n, float* out, cudaStream_t st);
 
@@ -108,9 +110,15 @@ struct DecodePlan {
   size_t ws_total_bytes;
 };
 DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len);
+// Argument checks of a cache and of a whole decode call (tq_decode_attn and
+// tq_decode_attn_noalloc share them): on success *plan and *thr are set.
+tq_status check_cache(const tq_params* p, const tq_cache* c, const char* who);
+tq_status check_decode_call(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache, int B, int hq,
+                            int max_len, const void* out, int out_dtype, const tq_attn_flags* flags,
+                            const char* who, DecodePlan* plan, float* thr, unsigned long long** sv_stats);
 tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c,
                         const DecodePlan& plan, void* out, int out_bf16, void* ws,
-                        float sparse_thr, cudaStream_t st);
+                        float sparse_thr, unsigned long long* sv_stats, cudaStream_t st);
 size_t search_workspace_bytes();
 int search_max_k();
 tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed* db, int64_t n, const void* q,

@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include "tq_internal.h"
+#include "tq_layout.cuh"
 #include "tq_sm100.cuh"
 
 namespace tq {
@@ -43,8 +44,9 @@ struct QuantArgs {
   float* norms;
   uint8_t* qjl;
   float* res;
-  // append destination
+  // append destination (code planes tiled, tq_layout.cuh; kside: the keys' arrangement)
   int append;
+  int kside;
   const int32_t* seq_ids;
   const int32_t* lens;
   int n_tok, hkv, capacity, n_sink, cache_seqs;
@@ -85,6 +87,55 @@ __device__ int64_t append_row(const QuantArgs& a, int64_t v, int* seq_out, int* 
   const int pos = len + tok;
   if (pos < a.n_sink) return -2;                           // sink token
   return (static_cast<int64_t>(seq) * a.hkv + head) * a.capacity + (pos - a.n_sink);
+}
+
+// n bytes of a packed row (32-bit words, nw of them) from row byte src to dst,
+// in the widest stores the destination's alignment allows.
+__device__ __forceinline__ void store_row_bytes(uint8_t* dst, const uint32_t* words, int nw, int src, int n) {
+  while (n > 0) {
+    const int w = src >> 2, sh = 8 * (src & 3);
+    const uint32_t lo = words[w], hi = w + 1 < nw ? words[w + 1] : 0u;
+    const uint32_t v = sh ? __funnelshift_r(lo, hi, sh) : lo;
+    const uintptr_t ad = reinterpret_cast<uintptr_t>(dst);
+    if (n >= 4 && (ad & 3) == 0) {
+      *reinterpret_cast<uint32_t*>(dst) = v;
+      dst += 4; src += 4; n -= 4;
+    } else if (n >= 2 && (ad & 1) == 0) {
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
+      dst += 2; src += 2; n -= 2;
+    } else {
+      *dst = static_cast<uint8_t>(v);
+      dst += 1; src += 1; n -= 1;
+    }
+  }
+}
+
+// Store the code words of a packed row as token (row & 15) of its 16-token
+// tile in a tiled cache code plane (tq_layout.cuh).  row = unit * capacity +
+// quantized position (capacity a multiple of 64, so tiles never straddle
+// units).  Each piece is a contiguous run of the packed row and of its lane
+// block; a run is split where the lane block changes column.
+__device__ __forceinline__ void store_tiled_codes(uint8_t* plane, const CodeTile& ct, bool kside, int64_t row,
+                                                  const uint32_t* words) {
+  uint8_t* tile = plane + (row >> 4) * ct.tile_bytes();
+  const int tok = static_cast<int>(row & 15), nw = ct.cb / 4;
+  for (int s = 0; s < ct.nseg; ++s) {
+    const int parts = kside ? 4 : 8;
+    const int pb = kside ? ct.kpiece(s) : ct.vpiece(s);
+    const int off = kside ? ct.koff(tok >> 3, s) : ct.voff((tok & 1) + 2 * (tok >> 3), s);
+    for (int q = 0; q < parts; ++q) {
+      const int L = kside ? 4 * (tok & 7) + q : 4 * q + ((tok & 7) >> 1);
+      int src = ct.seg_byte(s) + q * pb, p = off, n = pb;
+      while (n > 0) {
+        // bytes of this column left from lane-block byte p
+        const int c16 = 16 * ct.c16(), c8 = c16 + 8 * ct.c8();
+        const int room = p < c16 ? 16 - (p & 15) : p < c8 ? 8 - ((p - c16) & 7) : 4 - ((p - c8) & 3);
+        const int m = n < room ? n : room;
+        store_row_bytes(tile + ct.tile_off(L, p), words, nw, src, m);
+        src += m; p += m; n -= m;
+      }
+    }
+  }
 }
 
 template <int BF16>
@@ -262,12 +313,21 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_kernel(QuantArgs a) {
 
     // pack codes and write norms
     const int words = a.code_bytes / 4;
-    for (int it = tid; it < kTile * words; it += kThreads) {
-      const int v = it / words, w = it % words;
-      const int64_t row = s.row[v];
-      if (row < 0) continue;
-      reinterpret_cast<uint32_t*>(a.codes + row * a.code_bytes)[w] =
-          pack_word(s.codes[v], w, a.mse_bits, a.mixed);
+    if (a.append) {
+      // a cache's tiled code plane: one thread per row
+      if (words > 0 && tid < kTile && s.row[tid] >= 0) {
+        uint32_t rw[kMaxBits * 4];
+        for (int w = 0; w < words; ++w) rw[w] = pack_word(s.codes[tid], w, a.mse_bits, a.mixed);
+        store_tiled_codes(a.codes, make_code_tile(a.mse_bits, a.mixed, a.code_bytes), a.kside, s.row[tid], rw);
+      }
+    } else {
+      for (int it = tid; it < kTile * words; it += kThreads) {
+        const int v = it / words, w = it % words;
+        const int64_t row = s.row[v];
+        if (row < 0) continue;
+        reinterpret_cast<uint32_t*>(a.codes + row * a.code_bytes)[w] =
+            pack_word(s.codes[v], w, a.mse_bits, a.mixed);
+      }
     }
     if (tid < kTile && s.row[tid] >= 0) a.norms[s.row[tid]] = s.nu[tid];
 
@@ -556,15 +616,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
             for (int w = 0; w < TF::words; ++w) words[w] = 0u;
           }
-          uint8_t* dst = a.codes + row * TF::bytes;
-          if constexpr (TF::bytes % 16 == 0) {
-#pragma unroll
-            for (int w = 0; w < TF::words; w += 4)
-              *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+          if (a.append) {
+            constexpr CodeTile CT = make_code_tile(B, MIXED, TF::bytes);
+            store_tiled_codes(a.codes, CT, a.kside, row, words);
           } else {
+            uint8_t* dst = a.codes + row * TF::bytes;
+            if constexpr (TF::bytes % 16 == 0) {
 #pragma unroll
-            for (int w = 0; w < TF::words; w += 2)
-              *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
+              for (int w = 0; w < TF::words; w += 4)
+                *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+            } else {
+#pragma unroll
+              for (int w = 0; w < TF::words; w += 2)
+                *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
+            }
           }
           a.norms[row] = nu;
         }
@@ -884,11 +949,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
         if (row >= 0) {
           const bool zero = !(nu > 0.f);
           if constexpr (MB > 0) {
-            uint8_t* dst = a.codes + row * (16 * MB);
+            if (zero) {
 #pragma unroll
-            for (int w = 0; w < CW; w += 4)
-              *reinterpret_cast<uint4*>(dst + 4 * w) =
-                  zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+              for (int w = 0; w < CW; ++w) words[w] = 0u;
+            }
+            if (a.append) {
+              constexpr CodeTile CT = make_code_tile(MB, 0, 16 * MB);
+              store_tiled_codes(a.codes, CT, a.kside, row, words);
+            } else {
+              uint8_t* dst = a.codes + row * (16 * MB);
+#pragma unroll
+              for (int w = 0; w < CW; w += 4)
+                *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+            }
           }
           a.norms[row] = nu;
           *reinterpret_cast<uint4*>(a.qjl + row * (kSketch / 8)) =
@@ -918,6 +991,41 @@ __global__ void bump_lens_kernel(const int32_t* seq_ids, int32_t* lens, int32_t*
     atomicOr(status, 1);
   else
     lens[seq] += n_tok;
+}
+
+// Row import / export between packed rows (tq_quantize's format) and the
+// quantized rows of one cache unit: codes converted to / from the tiled code
+// plane, norms, QJL rows and residual norms copied.  One thread per row.
+__global__ void cache_rows_kernel(int to_cache, CodeTile ct, int kside, uint8_t* codes, float* norms, uint8_t* qjl,
+                                  float* res, int64_t unit_row0, uint8_t* r_codes, float* r_norms, uint8_t* r_qjl,
+                                  float* r_res, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int64_t row = unit_row0 + i;
+  if (ct.nseg > 0) {
+    uint8_t* tile = codes + (row >> 4) * ct.tile_bytes();
+    uint8_t* prow = r_codes + i * ct.cb;
+    if (to_cache) {
+      uint32_t w[kMaxBits * 4];
+      for (int k = 0; k < ct.cb / 4; ++k) w[k] = reinterpret_cast<const uint32_t*>(prow)[k];
+      store_tiled_codes(codes, ct, kside, row, w);
+    } else {
+      for_each_tile_byte(ct, kside, static_cast<int>(row & 15), [&](int src, int dst) { prow[src] = tile[dst]; });
+    }
+  }
+  if (to_cache) {
+    norms[row] = r_norms[i];
+    if (qjl) {
+      for (int k = 0; k < kSketch / 8; ++k) qjl[row * (kSketch / 8) + k] = r_qjl[i * (kSketch / 8) + k];
+      res[row] = r_res[i];
+    }
+  } else {
+    r_norms[i] = norms[row];
+    if (qjl) {
+      for (int k = 0; k < kSketch / 8; ++k) r_qjl[i * (kSketch / 8) + k] = qjl[row * (kSketch / 8) + k];
+      r_res[i] = res[row];
+    }
+  }
 }
 
 // x_hat = nu (Pi^T c + sqrt(pi/2)/m gamma S^T z), fp64 accumulation.
@@ -1125,6 +1233,7 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
     a.qjl = which ? c->v_qjl : c->k_qjl;
     a.res = which ? c->v_res_norms : c->k_res_norms;
     a.append = 1;
+    a.kside = which == 0;
     a.seq_ids = seq_ids;
     a.lens = c->lens;
     a.n_tok = n_tok;
@@ -1141,6 +1250,22 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
                                                         c->n_sink + c->capacity, c->n_seq);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "append length update");
+}
+
+tq_status launch_cache_rows(const tq_params* p, const tq_cache* c, int which, int seq, int kv_head, int row0,
+                            int64_t n, const tq_packed* rows, int to_cache, cudaStream_t st) {
+  if (n == 0) return TQ_OK;
+  const FormatSpec& f = which == TQ_K ? p->fk : p->fv;
+  const CodeTile ct = make_code_tile(f.mse_bits, f.mixed, f.code_bytes);
+  const int64_t unit_row0 = (static_cast<int64_t>(seq) * c->n_kv_heads + kv_head) * c->capacity + row0;
+  const bool k = which == TQ_K;
+  const int64_t blocks = (n + 127) / 128;
+  cache_rows_kernel<<<static_cast<unsigned>(blocks), 128, 0, st>>>(
+      to_cache, ct, k, k ? c->k_codes : c->v_codes, k ? c->k_norms : c->v_norms, f.prod ? (k ? c->k_qjl : c->v_qjl) : nullptr,
+      f.prod ? (k ? c->k_res_norms : c->v_res_norms) : nullptr, unit_row0, rows->codes, rows->norms,
+      f.prod ? rows->qjl : nullptr, f.prod ? rows->res_norms : nullptr, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, to_cache ? "tq_cache_write_rows" : "tq_cache_read_rows");
 }
 
 tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_packed* in, int64_t n,

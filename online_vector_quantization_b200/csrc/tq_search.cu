@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   const uint32_t lut_a = 0, lut_b = 0;
   const uint32_t lane4 = kLutAddr | (lane * 4), lane8 = (kLutAddr + L::region_b_off) | (lane * 8);
   const uint32_t c1k = FK::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
-  const TokRows tr = tok_rows<KF, 0>(g, t);
+  const TokRows tr = tok_rows(g, t);
 
   pdl_wait();  // the rotated query fragments (and the starting bounds)
   if (a.bound_in && tid < Q) atomicMax(&s_thr[tid], a.bound_in[tid]);

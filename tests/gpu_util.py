@@ -101,28 +101,39 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
 
+def side_id(side: str) -> int:
+    return tq.TQ_K if side == "k" else tq.TQ_V
+
+
+def read_unit_rows(cache: tq.Cache, f: o.Format, side: str, b: int, h: int, row0: int, n: int) -> o.Packed:
+    """Quantized rows row0 .. row0 + n - 1 of unit (b, h), as packed rows
+    (tq_cache_read_rows: the code planes are tiled)."""
+    out = tq.Packed.empty(cache.params, max(n, 1), side_id(side))
+    tq.tq_cache_read_rows(cache.params, cache, side_id(side), b, h, row0, out, n)
+    torch.cuda.synchronize()
+    pk = gpu_packed_to_numpy(out)
+    return o.Packed(pk.codes[:n], pk.norms[:n], pk.qjl[:n], pk.res_norms[:n])
+
+
+def write_unit_rows(cache: tq.Cache, side: str, b: int, h: int, row0: int, pk: o.Packed):
+    n = pk.norms.shape[0]
+    if n:
+        tq.tq_cache_write_rows(cache.params, cache, side_id(side), b, h, row0, numpy_packed_to_gpu(pk), n)
+
+
 def fill_cache_from_oracle(cache: tq.Cache, op: o.Params, ocache: o.Cache, lens, B, hkv):
-    """Write oracle-packed rows and bf16 sink rows into a GPU cache."""
-    gp_planes = {}
-    for name, dtype, elems in (("k_codes", torch.uint8, op.fmt_k.code_bytes(128)),
-                               ("v_codes", torch.uint8, op.fmt_v.code_bytes(128)),
-                               ("k_norms", torch.float32, 1), ("v_norms", torch.float32, 1),
-                               ("k_qjl", torch.uint8, 16), ("v_qjl", torch.uint8, 16),
-                               ("k_res_norms", torch.float32, 1), ("v_res_norms", torch.float32, 1),
-                               ("k_sink", torch.bfloat16, 128), ("v_sink", torch.bfloat16, 128)):
-        gp_planes[name] = cache.plane(name, dtype, elems)
+    """Write oracle-packed rows (tq_cache_write_rows) and bf16 sink rows into a
+    GPU cache."""
+    sinks = {side: cache.plane(side + "_sink", torch.bfloat16, 128) for side in ("k", "v")}
     for b in range(B):
         for h in range(hkv):
             ns = min(cache.n_sink, lens[b])
             nq = lens[b] - ns
             for side, rows, sink in (("k", ocache.k_rows[b, h], ocache.k_sink[b, h]),
                                      ("v", ocache.v_rows[b, h], ocache.v_sink[b, h])):
-                if gp_planes[side + "_codes"] is not None and rows.codes.shape[1]:
-                    gp_planes[side + "_codes"][b, h, :nq] = torch.from_numpy(rows.codes[:nq]).cuda()
-                gp_planes[side + "_norms"][b, h, :nq, 0] = torch.from_numpy(rows.norms[:nq]).cuda()
-                if gp_planes[side + "_qjl"] is not None:
-                    gp_planes[side + "_qjl"][b, h, :nq] = torch.from_numpy(rows.qjl[:nq]).cuda()
-                    gp_planes[side + "_res_norms"][b, h, :nq, 0] = torch.from_numpy(rows.res_norms[:nq]).cuda()
+                write_unit_rows(cache, side, b, h, 0,
+                                o.Packed(rows.codes[:nq], rows.norms[:nq], rows.qjl[:nq], rows.res_norms[:nq]))
                 if ns:
-                    gp_planes[side + "_sink"][b, h, :ns] = torch.from_numpy(sink[:ns]).to(torch.bfloat16).cuda()
+                    sinks[side][b, h, :ns] = torch.from_numpy(sink[:ns]).to(torch.bfloat16).cuda()
+    torch.cuda.synchronize()
     cache.lens.copy_(torch.tensor(lens, dtype=torch.int32))

@@ -34,14 +34,7 @@ D = 128
 
 def unit_packed(cache, f: o.Format, side: str, b: int, h: int, rows: int) -> o.Packed:
     """The packed rows [0, rows) of plane side (k or v) of unit (b, h)."""
-    codes = cache.plane(side + "_codes", torch.uint8, f.code_bytes(D))
-    norms = cache.plane(side + "_norms", torch.float32, 1)
-    qjl = cache.plane(side + "_qjl", torch.uint8, 16) if f.prod else None
-    res = cache.plane(side + "_res_norms", torch.float32, 1) if f.prod else None
-    return o.Packed(codes[b, h, :rows].cpu().numpy() if codes is not None else np.zeros((rows, 0), np.uint8),
-                    norms[b, h, :rows, 0].cpu().numpy(),
-                    qjl[b, h, :rows].cpu().numpy() if qjl is not None else np.zeros((rows, 0), np.uint8),
-                    res[b, h, :rows, 0].cpu().numpy() if res is not None else np.zeros(rows, np.float32))
+    return gu.read_unit_rows(cache, f, side, b, h, 0, rows)
 
 
 def oracle_cache_from_gpu(cache, fk, fv, units, lens):

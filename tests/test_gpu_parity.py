@@ -225,17 +225,13 @@ def test_append_parity(fk, fv, n_sink):
                 xs = x[s_in, :, h].double().numpy()
                 pos = np.arange(start[seq], start[seq] + n_tok)
                 qpos = pos[pos >= n_sink] - n_sink
-                want = o.quantize(op, xs[pos >= n_sink], side)
-                codes = cache.plane(side + "_codes", torch.uint8, f.code_bytes(128))
-                norms = cache.plane(side + "_norms", torch.float32, 1)
-                got = o.Packed(codes[seq, h, qpos].cpu().numpy() if codes is not None else np.zeros((len(qpos), 0), np.uint8),
-                               norms[seq, h, qpos, 0].cpu().numpy(),
-                               cache.plane(side + "_qjl", torch.uint8, 16)[seq, h, qpos].cpu().numpy() if f.prod else np.zeros((len(qpos), 0), np.uint8),
-                               cache.plane(side + "_res_norms", torch.float32, 1)[seq, h, qpos, 0].cpu().numpy() if f.prod else np.zeros(len(qpos), np.float32))
-                xq = xs[pos >= n_sink]
-                skip = gu.compare_codes(op, f, xq, got, want) if f.code_bytes(128) else set()
-                assert np.allclose(got.norms, want.norms, rtol=1e-6)
-                gu.compare_qjl(op, f, xq, got, want, skip)
+                if len(qpos):
+                    want = o.quantize(op, xs[pos >= n_sink], side)
+                    got = gu.read_unit_rows(cache, f, side, seq, h, int(qpos[0]), len(qpos))
+                    xq = xs[pos >= n_sink]
+                    skip = gu.compare_codes(op, f, xq, got, want) if f.code_bytes(128) else set()
+                    assert np.allclose(got.norms, want.norms, rtol=1e-6)
+                    gu.compare_qjl(op, f, xq, got, want, skip)
                 if n_sink and (pos < n_sink).any():
                     sink = cache.plane(side + "_sink", torch.bfloat16, 128)
                     sp = pos[pos < n_sink]
@@ -269,3 +265,281 @@ def test_gpu_built_cache_attention_matches_oracle_built():
     ocache = o.cache_from_vectors(op, kd, vd, 0)
     want = o.decode_attention(op, q.double().numpy(), ocache, [T, T], hkv)
     assert gu.rel_l2(out.float().cpu().numpy(), want) < gu.ATTN_REL_L2
+
+
+GQA_FORMATS = [(gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)), (gu.fmt(4), gu.fmt(3)),
+               (gu.fmt(3, prod=True), gu.fmt(3, prod=True)), (gu.fmt(1), gu.fmt(1))]
+
+
+@pytest.mark.parametrize("group", [1, 2, 3, 5, 6, 7, 8])
+@pytest.mark.parametrize("fk,fv", GQA_FORMATS, ids=["mixed", "k4v3", "prod3", "k1v1"])
+def test_decode_parity_gqa_groups(fk, fv, group):
+    """Every query-head group size the boundary accepts: groups of up to 4 pack
+    the query's high and low halves into spare MMA columns (3 leaves two of the
+    eight columns empty), larger groups run unpacked with 8 - group empty
+    columns."""
+    got, want, _ = _decode_case(fk, fv, B=2, hq=2 * group, hkv=2, T=1100, lens=[1100, 613], n_sink=0, thr=0.0,
+                                key=("gqa", str(fk), group))
+    assert gu.rel_l2(got, want) < gu.ATTN_REL_L2
+
+
+def _oracle_weights(op, q, ocache, b, kvh, group, nq):
+    """Final softmax weights (group, nq) of the quantized tokens of one unit
+    (no sink), by plain attention over the oracle's dequantized keys."""
+    kr = ocache.k_rows[b, kvh]
+    keys = o.dequantize(op, o.Packed(kr.codes[:nq], kr.norms[:nq], kr.qjl[:nq], kr.res_norms[:nq]), "k")
+    s = q[b, kvh * group:(kvh + 1) * group] @ keys.T / math.sqrt(128)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("fk,fv,group", [(gu.fmt(4), gu.fmt(3), 4), (gu.fmt(4), gu.fmt(3), 8),
+                                         (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True), 4)],
+                         ids=["k4v3g4", "k4v3g8", "mixedg4"])
+def test_decode_sparse_v_drops_and_matches_oracle(fk, fv, group):
+    """Peaked queries (N(0,1) scaled by 8): most softmax weights fall below
+    1e-6, the kernel drops their values and skips whole tiles, and the output
+    still matches the oracle's exact rule (drop a token's value when its final
+    weight is below the threshold).  The kernel's bound is conservative: every
+    weight it drops is one the exact rule drops."""
+    B, hkv, T, thr = 2, 2, 3000, 1e-6
+    hq = hkv * group
+    gp, op = gu.make_params(fk, fv)
+    key = ("sparse", str(fk), group)
+    k = kv_inputs.kv_vectors(B * hkv * T, 128, key=(key, "k"), dtype=torch.bfloat16)
+    v = kv_inputs.kv_vectors(B * hkv * T, 128, key=(key, "v"), dtype=torch.bfloat16)
+    q = (kv_inputs.queries((B, hq, 128), key=(key, "q"), dtype=torch.float32) * 8).to(torch.bfloat16)
+    ocache = o.cache_from_vectors(op, k.double().numpy().reshape(B, hkv, T, 128),
+                                  v.double().numpy().reshape(B, hkv, T, 128), 0)
+    lens = [T, 2345]
+    qd = q.double().numpy()
+    want = o.decode_attention(op, qd, ocache, lens, hkv, thr)
+    cache = tq.Cache(gp, B, hkv, ((T + 63) // 64) * 64, 0)
+    gu.fill_cache_from_oracle(cache, op, ocache, lens, B, hkv)
+    ws = tq.decode_workspace(gp, B, hq, hkv, T)
+    out = torch.empty(B, hq, 128, dtype=torch.bfloat16, device="cuda")
+    stats = torch.zeros(4, dtype=torch.int64, device="cuda")
+    tq.tq_decode_attn(gp, q.cuda(), cache, T, out, ws, thr, sparse_v_stats=stats)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    examined, dropped, tiles, skipped = (int(x) for x in stats.cpu())
+    exact_dropped = sum(int((_oracle_weights(op, qd, ocache, b, h, group, lens[b]) < thr).sum())
+                        for b in range(B) for h in range(hkv))
+    print(f"sparse V: kernel dropped {dropped}/{examined} weights ({dropped / examined:.3f}), exact rule "
+          f"{exact_dropped / examined:.3f}; tiles skipped {skipped}/{tiles} ({skipped / tiles:.3f})")
+    assert examined == sum(lens) * hkv * group
+    assert dropped / examined > 0.5
+    assert dropped <= exact_dropped
+    assert gu.rel_l2(out.float().cpu().numpy(), want) < gu.ATTN_REL_L2
+
+
+def test_decode_sparse_v_skips_whole_tiles():
+    """A value tile's work is skipped only when all its (token, head) weights
+    are dropped.  One unit of 2 x 148 x 480 tokens (two 480-token chunks per
+    CTA of the persistent grid): in even chunks the first token of every
+    32-token warp tile is a strong key (norm 30, cos 0.99 with the query), the
+    rest are ordinary keys, whose scores then sit ~20 below the running
+    maximum.  Every warp meets a strong key before its odd-chunk tiles, which
+    hold ordinary keys only and are skipped; the output matches the oracle's
+    exact rule."""
+    fk, fv = gu.fmt(4), gu.fmt(3)
+    gp, op = gu.make_params(fk, fv)
+    T, thr = 2 * 148 * 480, 1e-6
+    q = kv_inputs.queries((1, 1, 128), key=("skip", "q"), dtype=torch.float32)
+    k = kv_inputs.kv_vectors(T, 128, key=("skip", "k"), dtype=torch.float32)
+    v = kv_inputs.kv_vectors(T, 128, key=("skip", "v"), dtype=torch.float32)
+    pos = np.arange(T)
+    strong = ((pos // 480) % 2 == 0) & (pos % 32 == 0)
+    qh = q[0, 0] / q[0, 0].norm()
+    w = kv_inputs.kv_vectors(int(strong.sum()), 128, key=("skip", "w"), dtype=torch.float32)
+    w = w - (w @ qh)[:, None] * qh[None]
+    w = w / w.norm(dim=1, keepdim=True)
+    k[torch.from_numpy(strong)] = 30.0 * (0.99 * qh[None] + (1 - 0.99 ** 2) ** 0.5 * w)
+    k = k.to(torch.bfloat16)
+    v = v.to(torch.bfloat16)
+    q = q.to(torch.bfloat16)
+    ocache = o.cache_from_vectors(op, k.double().numpy()[None, None], v.double().numpy()[None, None], 0)
+    want = o.decode_attention(op, q.double().numpy(), ocache, [T], 1, thr)
+    cache = tq.Cache(gp, 1, 1, T, 0)
+    gu.fill_cache_from_oracle(cache, op, ocache, [T], 1, 1)
+    ws = tq.decode_workspace(gp, 1, 1, 1, T)
+    out = torch.empty(1, 1, 128, dtype=torch.bfloat16, device="cuda")
+    stats = torch.zeros(4, dtype=torch.int64, device="cuda")
+    tq.tq_decode_attn(gp, q.cuda(), cache, T, out, ws, thr, sparse_v_stats=stats)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    examined, dropped, tiles, skipped = (int(x) for x in stats.cpu())
+    print(f"sparse V, planted keys: dropped {dropped}/{examined}, tiles skipped {skipped}/{tiles}")
+    assert examined == T and tiles == T // 32
+    assert skipped / tiles > 0.45 and dropped / examined > 0.9
+    assert gu.rel_l2(out.float().cpu().numpy(), want) < gu.ATTN_REL_L2
+
+
+def test_config1_tiny_fp32_end_to_end():
+    """The tiny MSE-only configuration as stated: 4096 fp32 vectors (d = 128,
+    lognormal norms), 3-bit codes quantized on the GPU, dequantized, then
+    appended to a one-head cache as keys and values alike and attended by one
+    fp32 query; the GPU-built cache against the oracle's own."""
+    f = gu.fmt(3)
+    gp, op = gu.make_params(f, f)
+    n = 4096
+    x = kv_inputs.kv_vectors(n, 128, key="c1")
+    xd = x.double().numpy()
+    pk = tq.Packed.empty(gp, n, tq.TQ_K)
+    tq.tq_quantize(gp, x.cuda(), tq.TQ_K, pk)
+    torch.cuda.synchronize()
+    got = gu.gpu_packed_to_numpy(pk)
+    want_pk = o.quantize(op, xd, "k")
+    gu.compare_codes(op, f, xd, got, want_pk)
+    assert np.allclose(got.norms, want_pk.norms, rtol=1e-6, atol=0)
+    # dequantization of the GPU's codes, against the oracle's on the same codes
+    xh = torch.empty(n, 128, dtype=torch.float32, device="cuda")
+    tq.tq_dequantize(gp, pk, n, tq.TQ_K, xh)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(xh.cpu().numpy() - o.dequantize(op, got, "k"))) <= gu.DEQUANT_ATOL
+    # K = V = the same vectors through the streaming append (fp32 input)
+    cache = tq.Cache(gp, 1, 1, n, 0)
+    xs = x.view(1, n, 1, 128).cuda()
+    tq.tq_append(gp, cache, torch.zeros(1, dtype=torch.int32, device="cuda"), xs, xs)
+    torch.cuda.synchronize()
+    assert cache.lens.cpu().tolist() == [n] and int(cache.status.item()) == 0
+    assert np.array_equal(gu.read_unit_rows(cache, f, "k", 0, 0, 0, n).codes, got.codes)
+    assert np.array_equal(gu.read_unit_rows(cache, f, "v", 0, 0, 0, n).codes, got.codes)
+    q = kv_inputs.queries((1, 1, 128), key="c1q", dtype=torch.float32)
+    ws = tq.decode_workspace(gp, 1, 1, 1, n)
+    out = torch.empty(1, 1, 128, dtype=torch.float32, device="cuda")
+    tq.tq_decode_attn(gp, q.cuda(), cache, n, out, ws)
+    torch.cuda.synchronize()
+    ocache = o.cache_from_vectors(op, xd[None, None], xd[None, None], 0)
+    want = o.decode_attention(op, q.double().numpy(), ocache, [n], 1)
+    err = gu.rel_l2(out.cpu().numpy(), want)
+    print(f"config 1 (fp32 query and output, GPU-built cache vs the oracle's): rel L2 {err:.3e}")
+    assert err < gu.ATTN_REL_L2
+
+
+ALL_CODE_FORMATS = [gu.fmt(1), gu.fmt(2), gu.fmt(3), gu.fmt(4), gu.fmt(3, mixed=True), gu.fmt(2, mixed=True),
+                    gu.fmt(2, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True)]
+ALL_CODE_IDS = ["mse1", "mse2", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod2", "prod3", "prod4"]
+
+
+def _tile_spec_offsets(f, side):
+    """The tiled code layout as include/tq.h states it, written out on its
+    own: for token i (0..15) of a tile, the tile byte of every byte of its
+    packed row.  Lane L = 4g + t; a key lane owns tokens g, g + 8 and quarter
+    t of each segment, a value lane tokens 2t, 2t+1, 2t+8, 2t+9 and eighth g;
+    lane blocks of code_bytes / 2 bytes are stored as 16-, 16-, 8- and 4-byte
+    columns in that order."""
+    cb = f.code_bytes(128)
+    w = [f.mse_bits(j, 128) for j in range(128)]
+    segs = [(0, 64), (64, 128)] if f.mixed else [(0, 128)]
+    seg_start = [sum(w[:a]) // 8 for a, _ in segs]
+    seg_bytes = [sum(w[a:b]) // 8 for a, b in segs]
+    lb = cb // 2
+    cols = []
+    rest = lb
+    for width in (16, 16, 8, 4):
+        if rest >= width:
+            cols.append(width)
+            rest -= width
+    assert rest == 0
+
+    def tile_byte(lane, p):
+        base = 0
+        for width in cols:
+            if p < width:
+                return base + lane * width + p
+            p -= width
+            base += 32 * width
+        raise AssertionError
+
+    table = {}
+    for tok in range(16):
+        m = {}
+        for si, (sb, nb) in enumerate(zip(seg_start, seg_bytes)):
+            if side == "k":
+                g, role, parts = tok % 8, tok // 8, 4
+                piece = nb // 4
+                prior = sum(2 * (seg_bytes[x] // 4) for x in range(si))
+                for t in range(parts):
+                    for i in range(piece):
+                        m[sb + t * piece + i] = tile_byte(4 * g + t, prior + role * piece + i)
+            else:
+                t, member = (tok % 8) // 2, tok % 2 + 2 * (tok // 8)
+                piece = nb // 8
+                prior = sum(4 * (seg_bytes[x] // 8) for x in range(si))
+                for g in range(8):
+                    for i in range(piece):
+                        m[sb + g * piece + i] = tile_byte(4 * g + t, prior + member * piece + i)
+        assert sorted(m) == list(range(cb))
+        table[tok] = m
+    assert sorted(v for m in table.values() for v in m.values()) == list(range(16 * cb))
+    return table
+
+
+@pytest.mark.parametrize("f", ALL_CODE_FORMATS, ids=ALL_CODE_IDS)
+@pytest.mark.parametrize("side", ["k", "v"])
+def test_cache_rows_round_trip_and_tile_layout(f, side):
+    """tq_cache_write_rows / tq_cache_read_rows round-trip arbitrary packed rows
+    at a ragged offset, and the code plane holds them exactly as the tile
+    layout of include/tq.h says."""
+    fk = f if side == "k" else gu.fmt(1)
+    fv = f if side == "v" else gu.fmt(1)
+    gp, op = gu.make_params(fk, fv)
+    cap, n, row0 = 256, 150, 37
+    cache = tq.Cache(gp, 2, 3, cap, 0)
+    rng = np.random.default_rng(7)
+    cb = f.code_bytes(128)
+    pk = o.Packed(rng.integers(0, 256, (n, cb), dtype=np.uint8), rng.random(n).astype(np.float32),
+                  rng.integers(0, 256, (n, 16 if f.prod else 0), dtype=np.uint8),
+                  rng.random(n).astype(np.float32) if f.prod else np.zeros(n, np.float32))
+    gu.write_unit_rows(cache, side, 1, 2, row0, pk)
+    back = gu.read_unit_rows(cache, f, side, 1, 2, row0, n)
+    assert np.array_equal(back.codes, pk.codes) and np.array_equal(back.norms, pk.norms)
+    if f.prod:
+        assert np.array_equal(back.qjl, pk.qjl) and np.array_equal(back.res_norms, pk.res_norms)
+    # the raw code plane of unit (1, 2) against the stated layout
+    plane = cache.buffer[getattr(cache.struct, side + "_codes") - cache.buffer.data_ptr():]
+    unit = plane[(1 * 3 + 2) * cap * cb:(1 * 3 + 2 + 1) * cap * cb].cpu().numpy().reshape(cap // 16, 16 * cb)
+    spec = _tile_spec_offsets(f, side)
+    for r in range(n):
+        pos = row0 + r
+        tile, tok = divmod(pos, 16)
+        offs = spec[tok]
+        assert all(unit[tile, offs[j]] == pk.codes[r, j] for j in range(cb)), r
+    # the other units are untouched
+    other = plane[:cap * cb].cpu().numpy()
+    assert not other.any()
+
+
+@pytest.mark.parametrize("fk,fv", [(gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)), (gu.fmt(4), gu.fmt(3)),
+                                   (gu.fmt(3, prod=True), gu.fmt(3, prod=True)), (gu.fmt(2, mixed=True),
+                                                                                  gu.fmt(2, mixed=True))],
+                         ids=["mixed3.5", "k4v3", "prod3", "mixed2.5"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_append_rows_equal_quantize_rows(fk, fv, dtype):
+    """Appending in ragged 64-token chunks stores, bit for bit, the rows
+    tq_quantize produces for the same vectors (both kernels families: tensor
+    cores for bf16, SIMT for fp32), at every tile position."""
+    gp, _ = gu.make_params(fk, fv)
+    hkv, T = 2, 203
+    cache = tq.Cache(gp, 1, hkv, 256, 3)
+    k = kv_inputs.kv_vectors(T * hkv, 128, key=("ar", "k"), dtype=dtype).view(1, T, hkv, 128).cuda()
+    v = kv_inputs.kv_vectors(T * hkv, 128, key=("ar", "v"), dtype=dtype).view(1, T, hkv, 128).cuda()
+    ids = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for c0 in range(0, T, 64):
+        tq.tq_append(gp, cache, ids, k[:, c0:c0 + 64].contiguous(), v[:, c0:c0 + 64].contiguous())
+    torch.cuda.synchronize()
+    assert cache.lens.cpu().tolist() == [T] and int(cache.status.item()) == 0
+    for side, x, which in (("k", k, tq.TQ_K), ("v", v, tq.TQ_V)):
+        f = fk if side == "k" else fv
+        for h in range(hkv):
+            xs = x[0, 3:, h].contiguous()
+            ref = tq.Packed.empty(gp, T - 3, which)
+            tq.tq_quantize(gp, xs, which, ref)
+            torch.cuda.synchronize()
+            want = gu.gpu_packed_to_numpy(ref)
+            got = gu.read_unit_rows(cache, f, side, 0, h, 0, T - 3)
+            assert np.array_equal(got.codes, want.codes), (side, h)
+            assert np.array_equal(got.norms, want.norms)
+            if f.prod:
+                assert np.array_equal(got.qjl, want.qjl) and np.array_equal(got.res_norms, want.res_norms)
