@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "tq_internal.h"
 #include "tq_layout.cuh"
 #include "tq_sm100.cuh"
@@ -137,6 +139,96 @@ __device__ __forceinline__ void store_tiled_codes(uint8_t* plane, const CodeTile
     }
   }
 }
+
+// The same store with the format known at compile time (the tensor-core
+// kernels): every piece's row bytes, lane-block offset, column and alignment
+// are constants, the row's words stay in registers, and each run is written
+// with the widest stores its alignment allows (tiles are 16-byte aligned).
+template <int MSE, int MIXED, int CB>
+struct TiledStore {
+  static constexpr CodeTile CT = make_code_tile(MSE, MIXED, CB);
+
+  template <int SRC>
+  static __device__ __forceinline__ uint32_t get4(const uint32_t* w) {
+    constexpr int i = SRC / 4, sh = 8 * (SRC % 4);
+    if constexpr (sh == 0)
+      return w[i];
+    else if constexpr (i + 1 < CB / 4)
+      return __funnelshift_r(w[i], w[i + 1], sh);
+    else
+      return w[i] >> sh;
+  }
+
+  // N bytes from row byte SRC to byte LOFF of lane L's block
+  template <int SRC, int N, int LOFF>
+  static __device__ __forceinline__ void piece(uint8_t* tile, int L, const uint32_t* w) {
+    if constexpr (N > 0) {
+      constexpr int e16 = 16 * CT.c16(), e8 = e16 + 8 * CT.c8();
+      constexpr int width = LOFF < e16 ? 16 : LOFF < e8 ? 8 : 4;
+      constexpr int cstart = LOFF < e16 ? (LOFF / 16) * 16 : LOFF < e8 ? e16 : e8;
+      constexpr int cbase = LOFF < e16 ? (LOFF / 16) * 512 : LOFF < e8 ? 512 * CT.c16() : 512 * CT.c16() + 256 * CT.c8();
+      constexpr int inoff = LOFF - cstart, room = width - inoff, m0 = N < room ? N : room;
+      constexpr int M = (width >= 8 && inoff % 8 == 0 && m0 >= 8) ? 8
+                        : (inoff % 4 == 0 && m0 >= 4)               ? 4
+                        : (inoff % 2 == 0 && m0 >= 2)               ? 2
+                                                                    : 1;
+      uint8_t* dst = tile + cbase + L * width + inoff;
+      if constexpr (M == 8)
+        *reinterpret_cast<uint2*>(dst) = make_uint2(get4<SRC>(w), get4<SRC + 4>(w));
+      else if constexpr (M == 4)
+        *reinterpret_cast<uint32_t*>(dst) = get4<SRC>(w);
+      else if constexpr (M == 2)
+        *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(get4<SRC>(w));
+      else
+        *dst = static_cast<uint8_t>(get4<SRC>(w));
+      piece<SRC + M, N - M, LOFF + M>(tile, L, w);
+    }
+  }
+
+  // keys: the pieces of token role ROLE (0: token g, 1: token g + 8), quarters Q.. of segment S..
+  template <int ROLE, int S = 0, int Q = 0>
+  static __device__ __forceinline__ void kpieces(uint8_t* tile, int g, const uint32_t* w) {
+    if constexpr (S < CT.nseg) {
+      if constexpr (Q < 4) {
+        piece<CT.seg_byte(S) + Q * CT.kpiece(S), CT.kpiece(S), CT.koff(ROLE, S)>(tile, 4 * g + Q, w);
+        kpieces<ROLE, S, Q + 1>(tile, g, w);
+      } else {
+        kpieces<ROLE, S + 1, 0>(tile, g, w);
+      }
+    }
+  }
+  // values: the pieces of member M (token 2t, 2t+1, 2t+8, 2t+9), eighths G.. of segment S..
+  template <int M, int S = 0, int G = 0>
+  static __device__ __forceinline__ void vpieces(uint8_t* tile, int t, const uint32_t* w) {
+    if constexpr (S < CT.nseg) {
+      if constexpr (G < 8) {
+        piece<CT.seg_byte(S) + G * CT.vpiece(S), CT.vpiece(S), CT.voff(M, S)>(tile, 4 * G + t, w);
+        vpieces<M, S, G + 1>(tile, t, w);
+      } else {
+        vpieces<M, S + 1, 0>(tile, t, w);
+      }
+    }
+  }
+
+  static __device__ __forceinline__ void row(uint8_t* plane, bool kside, int64_t r, const uint32_t* w) {
+    uint8_t* tile = plane + (r >> 4) * CT.tile_bytes();
+    const int tok = static_cast<int>(r & 15);
+    if (kside) {
+      if (tok < 8)
+        kpieces<0>(tile, tok, w);
+      else
+        kpieces<1>(tile, tok - 8, w);
+    } else {
+      const int t = (tok & 7) >> 1;
+      switch ((tok & 1) + 2 * (tok >> 3)) {
+        case 0: vpieces<0>(tile, t, w); break;
+        case 1: vpieces<1>(tile, t, w); break;
+        case 2: vpieces<2>(tile, t, w); break;
+        default: vpieces<3>(tile, t, w); break;
+      }
+    }
+  }
+};
 
 template <int BF16>
 __device__ void load_tile(const QuantArgs& a, SmemQuant& s, int64_t v0) {
@@ -617,8 +709,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
             for (int w = 0; w < TF::words; ++w) words[w] = 0u;
           }
           if (a.append) {
-            constexpr CodeTile CT = make_code_tile(B, MIXED, TF::bytes);
-            store_tiled_codes(a.codes, CT, a.kside, row, words);
+            TiledStore<B, MIXED, TF::bytes>::row(a.codes, a.kside, row, words);
           } else {
             uint8_t* dst = a.codes + row * TF::bytes;
             if constexpr (TF::bytes % 16 == 0) {
@@ -954,8 +1045,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
               for (int w = 0; w < CW; ++w) words[w] = 0u;
             }
             if (a.append) {
-              constexpr CodeTile CT = make_code_tile(MB, 0, 16 * MB);
-              store_tiled_codes(a.codes, CT, a.kside, row, words);
+              TiledStore<MB, 0, 16 * MB>::row(a.codes, a.kside, row, words);
             } else {
               uint8_t* dst = a.codes + row * (16 * MB);
 #pragma unroll
@@ -1218,9 +1308,54 @@ tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x
   return run_quantize(a, st);
 }
 
+namespace {
+
+// The values' quantize kernel of an append runs on a side stream of the
+// library, concurrently with the keys' kernel on the caller's stream: for a
+// streaming chunk each grid holds a fraction of the SMs, so the two overlap
+// instead of queueing.  The side stream forks from and joins the caller's
+// stream through events (both recorded and waited inside one critical
+// section, so concurrent callers cannot cross their dependencies); the
+// pattern is valid under stream capture.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kSideDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kSideDevices];
+
+tq_status side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_append: cudaGetDevice");
+  if (dev < 0 || dev >= kSideDevices) return fail(TQ_ERR_UNSUPPORTED, "tq_append: device index too large");
+  SideStream& s = g_side[dev];
+  if (!s.stream) {
+    e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      s = SideStream{};
+      return cuda_fail(e, "tq_append: side stream");
+    }
+  }
+  *out = &s;
+  return TQ_OK;
+}
+
+}  // namespace
+
 tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* seq_ids, const void* k,
                         const void* v, int x_bf16, int n_tok, int n_seq, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(n_seq) * n_tok * c->n_kv_heads;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* side = nullptr;
+  tq_status sst = side_stream(&side);
+  if (sst != TQ_OK) return sst;
+  cudaError_t fe = cudaEventRecord(side->fork, st);
+  if (fe == cudaSuccess) fe = cudaStreamWaitEvent(side->stream, side->fork, 0);
+  if (fe != cudaSuccess) return cuda_fail(fe, "tq_append: fork");
   for (int which = 0; which < 2; ++which) {
     const FormatSpec& f = which ? p->fv : p->fk;
     QuantArgs a{};
@@ -1243,9 +1378,16 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
     a.cache_seqs = c->n_seq;
     a.sink = which ? c->v_sink : c->k_sink;
     a.status = c->status;
-    tq_status s = run_quantize(a, st);
-    if (s != TQ_OK) return s;
+    tq_status s = run_quantize(a, which ? side->stream : st);
+    if (s != TQ_OK) {
+      // keep the side stream joined to the caller's stream even on failure
+      if (cudaEventRecord(side->join, side->stream) == cudaSuccess) cudaStreamWaitEvent(st, side->join, 0);
+      return s;
+    }
   }
+  fe = cudaEventRecord(side->join, side->stream);
+  if (fe == cudaSuccess) fe = cudaStreamWaitEvent(st, side->join, 0);
+  if (fe != cudaSuccess) return cuda_fail(fe, "tq_append: join");
   bump_lens_kernel<<<(n_seq + 127) / 128, 128, 0, st>>>(seq_ids, c->lens, c->status, n_seq, n_tok,
                                                         c->n_sink + c->capacity, c->n_seq);
   cudaError_t e = cudaGetLastError();
