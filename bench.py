@@ -93,11 +93,13 @@ class ClockSampler:
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device, bits: int = 3):
+def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device, bits: int = 3, params=None):
     """Config: streaming append + decode (mixed rows: bits + 0.5 bits per
-    channel, 3.5 by default).  Returns the state the step uses."""
+    channel, 3.5 by default; `params` replaces the format).  Returns the
+    state the step uses."""
     lens = rank_sequence_lengths(kv_inputs, rank)
-    params = tq.Params(bits, bits, mixed_k=1, mixed_v=1, seed=0)
+    if params is None:
+        params = tq.Params(bits, bits, mixed_k=1, mixed_v=1, seed=0)
     cap = ((max(lens) + (n_steps + 1) * CHUNK + 63) // 64) * 64
     cache = tq.Cache(params, N_SEQ, HKV, cap, 0, device=device)
     # prefill (untimed): the prefix of each sequence through tq_append
@@ -127,13 +129,10 @@ def build_stream_workload(tq, torch, kv_inputs, rank: int, n_steps: int, device,
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch of
-# this workload (one ncu capture: 485.12 MB read, 4.27 MB written), valid for
+# this workload (one ncu capture: 485.20 MB read, 5.02 MB written), valid for
 # the kernel source it was taken on only: reported as null once that changes.
-# The sources changed after the capture only outside decode_kernel (the merge
-# kernel, the host launch code, and one argument field only the merge reads),
-# so the figure is tied to the sources as they are now.
-DECODE_TRAFFIC = {"source_sha256": "b426d03d3fc4c2860cffb7da0929aa5341593ed4587e754872505fa7a1cd5f34",
-                  "bytes": 489391104}
+DECODE_TRAFFIC = {"source_sha256": "c4760886ffed909ddd5d38bc37cef1cfe6e39a91834deb57bfbfebcd87d39a31",
+                  "bytes": 490224384}
 
 
 def decode_sources_sha256():
@@ -362,7 +361,8 @@ def _time_call(torch, fn, iters, flush=None):
     return statistics.median(times)
 
 
-AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "fp8-kv", "stream-2.5", "search")
+AUX_WORKLOADS = ("quantize-sweep", "prod3-gqa", "k4v3-sink", "tiny", "bf16-sdpa", "fp8-kv", "stream-2.5", "stream-k8v3",
+                 "search")
 
 
 def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
@@ -382,6 +382,8 @@ def run_aux(tq, torch, kv_inputs, device, args, only=None, formats=None):
         out["decode_tiny_fp32_T4096"] = _aux_tiny(tq, torch, kv_inputs, device, iters)
     if only in (None, "stream-2.5"):
         out["decode_mixed2.5_stream_shapes"] = _aux_stream25(tq, torch, kv_inputs, device, flush, iters)
+    if only in (None, "stream-k8v3"):
+        out["decode_k8v3_stream_shapes"] = _aux_stream_k8v3(tq, torch, kv_inputs, device, flush, iters)
     if only in (None, "search"):
         out["ip_search_4M"] = _aux_search(tq, torch, kv_inputs, device, flush, iters, formats)
     if only in (None, "bf16-sdpa"):
@@ -402,11 +404,13 @@ def _aux_sweep(tq, torch, kv_inputs, device, flush, iters, formats):
     cases += [(tq.TQ_MODE_MSE, "mixed", 2, tq.TQ_ROT_HAAR, "mixed2.5"), (tq.TQ_MODE_MSE, "mixed", 3, tq.TQ_ROT_HAAR, "mixed3.5")]
     cases += [(tq.TQ_MODE_MSE, "mse", 3, tq.TQ_ROT_HADAMARD, "mse3_hadamard"),
               (tq.TQ_MODE_PROD, "prod", 3, tq.TQ_ROT_HADAMARD, "prod3_hadamard")]
+    # 8-bit codes (256 centroids), the key side of the K8/V3 pair
+    cases += [(tq.TQ_MODE_MSE, "mse", 8, tq.TQ_ROT_HAAR, "mse8")]
     for mode, name, b, rot, label in cases:
         if formats and label not in formats:
             continue
         mixed = int(name == "mixed")
-        p = tq.Params(b, b, mode, mode, mixed, mixed, rotation=rot)
+        p = tq.Params(b, b if b <= 4 else 3, mode, mode, mixed, mixed, rotation=rot)
         pk = tq.Packed.empty(p, n, tq.TQ_K, device=device)
         ms = _time_call(torch, lambda: tq.tq_quantize(p, x, tq.TQ_K, pk), iters, flush)
         assert p.status() == 0
@@ -484,6 +488,22 @@ def _aux_stream25(tq, torch, kv_inputs, device, flush, iters):
     assert int(cache.status.item()) == 0
     row = p.row_bytes(tq.TQ_K)[0] + 4
     by = sum(HKV * n * 2 * row for n in st["lens"]) + 2 * N_SEQ * HQ * D * 2
+    out = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
+           "l2": "flushed between calls"}
+    del st, cache
+    return out
+
+
+def _aux_stream_k8v3(tq, torch, kv_inputs, device, flush, iters):
+    """The decode call of the streaming workload's shapes with 8-bit keys
+    (128-byte code rows, 256 centroids) and 3-bit values (48-byte rows)."""
+    st = build_stream_workload(tq, torch, kv_inputs, 0, 1, device, params=tq.Params(8, 3, seed=0))
+    p, cache = st["params"], st["cache"]
+    ms = _time_call(torch, lambda: tq.tq_decode_attn(p, st["qs"][0], cache, st["cap"], st["out"], st["ws"]),
+                    iters, flush)
+    assert int(cache.status.item()) == 0
+    row = p.row_bytes(tq.TQ_K)[0] + 4 + p.row_bytes(tq.TQ_V)[0] + 4
+    by = sum(HKV * n * row for n in st["lens"]) + 2 * N_SEQ * HQ * D * 2
     out = {"ms": round(ms, 4), "gb_per_s": round(by / (ms * 1e-3) / 1e9, 1), "bytes": by,
            "l2": "flushed between calls"}
     del st, cache

@@ -24,7 +24,8 @@
  *    thread.  Inputs must be finite: NaN or Inf inputs give unspecified codes
  *    but never an out-of-bounds access.
  *  - Sizes: d = 128 and m = 128 in this version (TQ_ERR_UNSUPPORTED
- *    otherwise); bits in 1..4 (MSE) or 1..4 total (prod, 1 = QJL only).
+ *    otherwise); bits in 1..4 or 8 (MSE; 8 = one byte per code, 256
+ *    centroids, uniform rows only) or 1..4 total (prod, 1 = QJL only).
  *
  * Packed row format (both sides of the library agree on it; the pages only
  * say that codes live at "unconventional bit widths", NVIDIA forum post "Why
@@ -181,15 +182,17 @@ tq_status tq_dequantize(const tq_params* p, const tq_packed* in, int64_t n, int 
  *    whole row (uniform widths) or one of its two halves of 64 coordinates
  *    (mixed rows); every such piece is a whole number of bytes.  The blocks
  *    are stored as columns: the first 16 bytes of every lane (lane L's at
- *    offset 16 L), then the next 16, then 8, then 4, as the block's size
- *    needs.  So each lane reads its share with one load per column and the
+ *    offset 16 L), then the next 16 and so on while 16 bytes remain, then 8,
+ *    then 4, as the block's size needs.  So each lane reads its share with one load per column and the
  *    warp's loads never share a shared-memory bank.
  * lens: device int32 [n_seq], tokens held per sequence (sink included); the
- * caller zeroes it for an empty cache.  status: device int32 word; kernels OR
- * error bits into it (1 = append past capacity, 2 = a length above the bound
- * given to tq_decode_attn, 4 = a decode wait on the copy pipeline gave up
- * after its time limit, 8 = the decode kernel's shared-memory layout did not
- * fit; after 4 or 8 the outputs are invalid). */
+ * caller zeroes it for an empty cache.  status: device int32 word, zeroed by
+ * the caller with the cache; kernels OR error bits into its low 16 bits (1 =
+ * append past capacity, 2 = a length above the bound given to
+ * tq_decode_attn, 4 = a decode wait on the copy pipeline gave up after its
+ * time limit, 8 = the decode kernel's shared-memory layout did not fit; after
+ * 4 or 8 the outputs are invalid).  Bits 16..31 count the CTAs of a running
+ * tq_append and are zero again when it ends. */
 typedef struct {
   int n_seq, n_kv_heads, capacity, n_sink;
   uint8_t* k_codes; float* k_norms; uint8_t* k_qjl; float* k_res_norms;
@@ -215,7 +218,12 @@ tq_status tq_cache_bind(const tq_params* p, void* base, size_t bytes, int n_seq,
  * [n_seq][n_tok][n_kv_heads][d] in dtype.  Tokens land at positions
  * lens[s] .. lens[s] + n_tok - 1 (sink or quantized row), then lens[s] grows
  * by n_tok, all in stream order.  A sequence that would pass
- * n_sink + capacity is left unchanged and bit 1 is set in cache->status. */
+ * n_sink + capacity is left unchanged and bit 1 is set in cache->status.
+ * When K and V share a format and dtype is bf16 one kernel quantizes both;
+ * otherwise the keys' kernel runs on `stream` and the values' on a side
+ * stream of the library's, joined back before the call returns.  The CTA that
+ * finishes last updates lens (no separate launch), so appends to one cache
+ * must not overlap on the GPU. */
 tq_status tq_append(const tq_params* p, const tq_cache* cache, const int32_t* seq_ids,
                     const void* k, const void* v, int dtype, int n_tok, int n_seq, void* stream);
 
@@ -275,10 +283,12 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
  * and bit 2 is set in cache->status).  n_sink above 4096 gives
  * TQ_ERR_UNSUPPORTED.  K/V formats with a decode kernel: equal formats
  * (MSE 1..4 bits, mixed 2.5 and 3.5, prod 1..4) and the asymmetric MSE pairs
- * K4/V3, K4/V2, K3/V2; any other pair gives TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the query rotation,
- * the persistent decode kernel and the merge; the last two are launched with
- * programmatic stream serialization and overlap their prologues with the
- * previous kernel's tail. */
+ * K4/V3, K4/V2, K3/V2 and K8/V3 (8-bit keys); any other pair gives
+ * TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the
+ * query rotation, the persistent decode kernel and the merge; the last two
+ * are launched with programmatic stream serialization and overlap their
+ * prologues with the previous kernel's tail.  Nothing in the workspace needs
+ * to start at zero. */
 tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
                          int B, int hq, int max_len, void* out, int out_dtype,
                          void* workspace, size_t ws_bytes, const tq_attn_flags* flags,

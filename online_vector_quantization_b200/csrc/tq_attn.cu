@@ -10,11 +10,11 @@
 // (same page, item 1) follow the header tq.h.
 //
 // Kernels of one decode step
-//   1. qrot_kernel: q -> Pi q (and S q), scaled by log2(e)/sqrt(d), stored as
-//      fp16 MMA B-fragments in the workspace, once per (sequence, kv-head).
-//   2. decode_kernel: persistent, one CTA per SM; a producer warp streams
+//   1. decode_kernel: persistent, one CTA per SM; a producer warp streams
 //      the packed cache into shared memory with bulk copies, fifteen consumer
-//      warps walk 16-token tiles of it:
+//      warps rotate the query at each (sequence, kv-head) unit they start
+//      (q -> Pi q and S q, scaled by log2(e)/sqrt(d), as fp16 MMA
+//      B-fragments) and walk 16-token tiles of the stream:
 //        scores S^T[16 tok x 8 heads] = C_k[16 x 128] Q~^T  (mma.sync m16n8k16)
 //        online softmax (base 2), sparse-V mask, P' = p * ||v||
 //        O^T[128 x 8 heads] += C_v^T[128 x 16 tok] P'^T    (mma.sync m16n8k16)
@@ -23,11 +23,11 @@
 //      (two or four codes per lookup, no bank conflicts), so no fp16 tile is
 //      ever written back to memory.  Warps merge in shared memory and the CTA
 //      writes one (m, l, acc) partial per piece of a (sequence, kv-head).
-//   3. merge_kernel: one CTA per (sequence, kv-head), or per (sequence,
+//   2. merge_kernel: one CTA per (sequence, kv-head), or per (sequence,
 //      query head) for small batches, attends the bf16 sink, combines the
-//      pieces and applies Pi^T / S^T once.  (qrot_kernel, the formats, tables
-//      and subtile scoring live in tq_decode_common.cuh, shared with the
-//      inner-product search.)
+//      pieces and applies Pi^T / S^T once.  (The formats, tables and subtile
+//      scoring live in tq_decode_common.cuh, shared with the inner-product
+//      search.)
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -242,8 +242,13 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
 // at most U + P - 1 of them.  The merge kernel finds a unit's pieces from the
 // same schedule.  No CTA waits for another.
 // ---------------------------------------------------------------------------
+// A unit with quantized tokens occupies slack + chunks slots of the list:
+// `slack` (a.unit_slack) empty slots model the fixed cost a CTA pays when it
+// starts a unit (combining the previous piece, rotating the query, merging),
+// so CTAs whose ranges cross more units get fewer chunks.  Empty slots are
+// skipped by the producer and the consumers alike.
 struct UnitInfo {
-  int len, ns, nq, chunks;
+  int len, ns, nq, chunks, slack, slots;
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u, int kChunk) {
@@ -254,14 +259,17 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u, int kC
   r.ns = min(a.n_sink, len);
   r.nq = len - r.ns;
   r.chunks = (r.nq + kChunk - 1) / kChunk;
+  r.slack = r.chunks > 0 ? a.unit_slack : 0;
+  r.slots = r.chunks + r.slack;
   return r;
 }
 
 
-// Chunks of each kv-head unit of sequence b (all units of a sequence are alike).
-__device__ __forceinline__ int seq_chunks(const DecodeArgs& a, int b, int kChunk) {
+// Slots of each kv-head unit of sequence b (all units of a sequence are alike).
+__device__ __forceinline__ int seq_slots(const DecodeArgs& a, int b, int kChunk) {
   const int len = min(max(a.lens[b], 0), a.max_len);
-  return (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
+  const int ch = (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
+  return ch > 0 ? ch + a.unit_slack : 0;
 }
 
 // CTA whose range holds chunk c: the largest i with i*C/P <= c.
@@ -290,9 +298,11 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t i, float 
     reinterpret_cast<float*>(a.out)[i] = v;
 }
 
-// Cross-warp combine of one piece into partial slot `slot`, in 64-coordinate
-// slices of the accumulator (consumer threads).  LANE_SUMS: each lane holds
-// its own partial softmax sums (dense path), added over the column first.
+// Cross-warp combine of one piece into partial slot `slot` (consumer
+// threads).  Every warp rescales its accumulator to the CTA's maximum before
+// storing it, so the combine is a plain sum over warps, done in 64-coordinate
+// slices of the accumulator.  LANE_SUMS: each lane holds its own partial
+// softmax sums (dense path), added over the column first.
 template <int KF, int VF, bool PACK, bool LANE_SUMS>
 __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& W, int64_t slot, float* sm,
                             int warp, int g, int t) {
@@ -321,6 +331,27 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
     wl[warp * kMaxG + 2 * t] = l0;
     wl[warp * kMaxG + 2 * t + 1] = l1;
   }
+  consumers_sync();
+  // this lane's two columns: the CTA's maximum and this warp's factor
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kConsumers; ++w) {
+    M0 = fmaxf(M0, wm[w * kMaxG + 2 * t]);
+    M1 = fmaxf(M1, wm[w * kMaxG + 2 * t + 1]);
+  }
+  const float f0 = W.m0 > -INFINITY ? exp2f(W.m0 - M0) : 0.f;
+  const float f1 = W.m1 > -INFINITY ? exp2f(W.m1 - M1) : 0.f;
+  if (tid < a.group) {  // the piece's maximum and sum of head tid
+    const int h = tid;
+    float M = -INFINITY, l = 0.f;
+    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
+    for (int w = 0; w < kConsumers; ++w) {
+      const float mw = wm[w * kMaxG + h];
+      if (mw > -INFINITY) l = fmaf(wl[w * kMaxG + h], exp2f(mw - M), l);
+    }
+    dst[h * PF + 0] = M;
+    dst[h * PF + 1] = l;
+  }
 #pragma unroll 1
   for (int pass = 0; pass < WD / kSliceDims; ++pass) {
     const int lo = pass * kSliceDims;
@@ -342,33 +373,21 @@ __device__ void write_piece(const DecodeArgs& a, const WarpState<KF, VF, PACK>& 
       float* w0 = wacc + (warp * kMaxG + 2 * t) * kSliceDims - lo;
       float* w1 = wacc + (warp * kMaxG + 2 * t + 1) * kSliceDims - lo;
       if (d0 >= lo && d0 < lo + kSliceDims) {
-        w0[d0] = W.oacc[mt][0];
-        w1[d0] = W.oacc[mt][1];
+        w0[d0] = W.oacc[mt][0] * f0;
+        w1[d0] = W.oacc[mt][1] * f1;
       }
       if (d1 >= lo && d1 < lo + kSliceDims) {
-        w0[d1] = W.oacc[mt][2];
-        w1[d1] = W.oacc[mt][3];
+        w0[d1] = W.oacc[mt][2] * f0;
+        w1[d1] = W.oacc[mt][3] * f1;
       }
     }
     consumers_sync();
     for (int i = tid; i < a.group * kSliceDims; i += NT) {
       const int h = i / kSliceDims, j = i % kSliceDims;
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, wm[w * kMaxG + h]);
-      float s = 0.f, l = 0.f;
-      for (int w = 0; w < kConsumers; ++w) {
-        const float mw = wm[w * kMaxG + h];
-        if (mw > -INFINITY) {
-          const float f = exp2f(mw - M);
-          s += wacc[(w * kMaxG + h) * kSliceDims + j] * f;
-          l += wl[w * kMaxG + h] * f;
-        }
-      }
-      dst[h * PF + kPartAcc + lo + j] = s;
-      if (pass == 0 && j == 0) {
-        dst[h * PF + 0] = M;
-        dst[h * PF + 1] = l;
-      }
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) acc += wacc[(w * kMaxG + h) * kSliceDims + j];
+      dst[h * PF + kPartAcc + lo + j] = acc;
     }
     consumers_sync();
   }
@@ -459,7 +478,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   if (warp == 0 && ui.chunks > 0) {
     long long tot = 0, before = 0;
     for (int v = lane; v < a.B; v += 32) {
-      const int ch = seq_chunks(a, v, CH);
+      const int ch = seq_slots(a, v, CH);
       tot += ch;
       if (v < b) before += ch;
     }
@@ -470,7 +489,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     }
     if (lane == 0) {
       s_C = tot * a.hkv;
-      s_cu0 = before * a.hkv + static_cast<long long>(kvh) * ui.chunks;
+      s_cu0 = before * a.hkv + static_cast<long long>(kvh) * ui.slots + ui.slack;
     }
   }
   // sink: scores with the original query, softmax weights, weighted values
@@ -740,7 +759,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     return s < static_cast<int>(n_low) ? low0 + s * SL::bytes : high0 + (s - n_low) * SL::bytes;
   };
   float* scratch = reinterpret_cast<float*>(smem + (scratch_addr - dyn0));
-  unsigned char* lut_mem = smem + (kLutAddr - dyn0);
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ long long s_c0, s_c1;
@@ -750,17 +768,34 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const int P = gridDim.x, cta = blockIdx.x;
   const int U = a.B * a.hkv;
 
-  // ---- codebooks to shared memory, schedule (warp 0) and barriers (thread 32);
-  // the producer starts streaming right after, while the consumers build
-  // the lookup tables
-  __shared__ float s_cb[(kMaxBits + 1) * kBookSlots];
-  if (tid < (kMaxBits + 1) * kBookSlots) s_cb[tid] = a.cbs[tid];
+  // ---- barriers (thread 32); the producer starts the copy of the lookup
+  // tables (built once per parameter set) while warp 0 computes the schedule
+  __shared__ __align__(8) uint64_t lut_bar;
+  if (tid == 32) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kConsumers);
+    }
+    mbar_init(&lut_bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if constexpr (L::bytes > 0) {
+    if (tid == kConsumers * 32) {
+      mbar_expect_tx(&lut_bar, L::bytes);
+      constexpr int kPart = 32768;
+#pragma unroll
+      for (int off = 0; off < L::bytes; off += kPart)
+        bulk_g2s_addr(kLutAddr + off, a.lut_img + off, min(kPart, L::bytes - off), &lut_bar);
+    }
+  }
   if (warp == 0) {
     // schedule (one warp): total chunks C, this CTA's range [c0, c1) and the
     // unit / local chunk where it starts
     long long C = 0;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
-      int ch = b0 + lane < a.B ? seq_chunks(a, b0 + lane, CH) : 0;
+      int ch = b0 + lane < a.B ? seq_slots(a, b0 + lane, CH) : 0;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, off);
       C += ch;
@@ -771,7 +806,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     long long base = 0;
     for (int b0 = 0; b0 < a.B && c0 < c1; b0 += 32) {
       const int b = b0 + lane;
-      const long long ch = b < a.B ? seq_chunks(a, b, CH) : 0;
+      const long long ch = b < a.B ? seq_slots(a, b, CH) : 0;
       long long incl = ch;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -805,14 +840,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       s_abort = 0;
     }
   }
-  if (tid == 32) {
-#pragma unroll
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], kConsumers);
-    }
-    mbar_fence_init();
-  }
   __syncthreads();
   const long long c0 = s_c0, c1 = s_c1;
 
@@ -822,18 +849,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       int u = s_u0, lc = s_lc0;
       UnitInfo ui = unit_info(a, u, CH);
       const int nk = static_cast<int>(c1 - c0);
-      int s = 0;
-      uint32_t round = 0;  // parity of k / S
+      int s = 0, n_streamed = 0;
+      uint32_t round = 0;  // parity of (chunks streamed) / S
       for (int k = 0; k < nk; ++k) {
-        while (lc >= ui.chunks) {
+        while (lc >= ui.slots) {
           ++u;
           lc = 0;
           ui = unit_info(a, u, CH);
         }
-        if (k >= S && !mbar_wait(&empty_bar[s], round ^ 1u)) s_abort = 1;
+        if (lc < ui.slack) {  // an empty slot
+          ++lc;
+          continue;
+        }
+        if (n_streamed >= S && !mbar_wait(&empty_bar[s], round ^ 1u)) s_abort = 1;
         if (s_abort) break;
+        ++n_streamed;
         const int64_t ubase = static_cast<int64_t>(u) * a.capacity;
-        const int r0 = lc * CH;
+        const int r0 = (lc - ui.slack) * CH;
         const int rows = min(CH, (ui.nq + kTok - 1) / kTok * kTok - r0);  // <= capacity - r0
         const uint32_t st = stage_addr(s);
         uint64_t* bar = &full_bar[s];
@@ -861,9 +893,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     return;
   }
 
-  // ---- lookup tables (consumer threads)
-  build_luts<L>(lut_mem, s_cb, tid);
-  consumers_sync();  // tables complete
+  bool luts_ready = L::bytes == 0;  // waited for before the first tile
+  bool frags_ready = false;         // the rotated query, waited for at the first unit
 
   // ---- consumers
   // table bases are folded into the lane offsets (see kLutAddr)
@@ -873,8 +904,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const uint32_t c1v = FV::mse == 1 ? h2bits(a.cbs[1 * kBookSlots + 1], a.cbs[1 * kBookSlots + 1]) : 0u;
   const float thr = a.sparse_thr;
   const TokRows trows = tok_rows(g, t);
-
-  pdl_wait();  // the rotated query fragments
 
   WarpState<KF, VF, PACK> wst;
   QFrag<PACK> bq, bqs;
@@ -887,15 +916,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   uint32_t round = 0;  // parity of k / S
   SparseTally tally;
   for (int k = 0; k < nk; ++k) {
-    while (walk_lc >= wui.chunks) {
+    while (walk_lc >= wui.slots) {
       ++walk_u;
       walk_lc = 0;
       wui = unit_info(a, walk_u, CH);
+    }
+    if (walk_lc < wui.slack) {  // an empty slot
+      ++walk_lc;
+      continue;
     }
     if (walk_u != u) {
       if (u >= 0) write_piece<KF, VF, PACK, true>(a, wst, u + cta, scratch, warp, g, t);
       u = walk_u;
       ui = wui;
+      if (!frags_ready) {
+        pdl_wait();  // the query rotation kernel's fragments
+        frags_ready = true;
+      }
       const uint32_t* qf = a.qfrag + static_cast<int64_t>(u) * kQfragWords;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
@@ -911,8 +948,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
       wst.m0 = wst.m1 = -INFINITY;
       wst.l0 = wst.l1 = 0.f;
     }
+    if (!luts_ready) {
+      if (!mbar_wait(&lut_bar, 0)) s_abort = 1;
+      luts_ready = true;
+    }
     if (!s_abort && !mbar_wait(&full_bar[s], round)) s_abort = 1;
-    const int row0 = walk_lc * CH + warp * WT;
+    const int row0 = (walk_lc - ui.slack) * CH + warp * WT;
     if (!s_abort && row0 < ui.nq) {
       const uint32_t st = stage_addr(s);
       UnitPlanes sp;
@@ -936,6 +977,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     }
   }
   if (u >= 0) write_piece<KF, VF, PACK, true>(a, wst, u + cta, scratch, warp, g, t);
+  if (!luts_ready) mbar_wait(&lut_bar, 0);  // no copy may target a finished CTA
   if (s_abort && tid == 0) atomicOr(a.status, 4);
   if constexpr (SPARSE == 2) {
     {
@@ -965,8 +1007,9 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   cudaError_t e = ensure_dyn_smem<decode_kernel<KF, VF, PACK, SPARSE>>(static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
   // the query rotation waits for all earlier work on the stream (the appends
-  // that filled the cache); the two kernels after it overlap their prologues
-  // with its tail
+  // that filled the cache); the decode kernel after it starts its prologue
+  // (tables, schedule, first bulk copies) while the rotation runs, and the
+  // merge kernel overlaps its prologue with the decode kernel's tail
   const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
   e = ensure_dyn_smem<qrot_kernel<KF>>(static_cast<int>(qrot_smem));
   if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
@@ -992,6 +1035,8 @@ tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
   a.dyn_bytes = static_cast<uint32_t>(smem);
   a.pack = plan.group <= 4;
   a.chunk = DecodeCfg<KF, VF>::CH;
+  // a unit start costs about two 480-token chunks of streaming
+  a.unit_slack = std::max(1, 960 / DecodeCfg<KF, VF>::CH);
   if (a.sparse_thr > 0.f && a.sv_stats)
     return a.pack ? run_decode_v<KF, VF, true, 2>(a, plan, smem, st) : run_decode_v<KF, VF, false, 2>(a, plan, smem, st);
   if (a.sparse_thr > 0.f)
@@ -1003,6 +1048,74 @@ tq_status run_decode(DecodeArgs& a, const DecodePlan& plan, cudaStream_t st) {
 
 }  // namespace
 
+namespace {
+// The lookup tables of a format pair, built once into global memory: the
+// decode kernel's shared-memory table region, byte for byte.
+template <int KF, int VF>
+__global__ void __launch_bounds__(kConsumers * 32) lut_image_kernel(unsigned char* img, const float* cbs,
+                                                                       const float* cbs8) {
+  build_luts<Lut<KF, VF>>(img, cbs, threadIdx.x, cbs8);
+}
+
+template <int KF, int VF>
+size_t lut_bytes_of() {
+  return Lut<KF, VF>::bytes;
+}
+
+template <int K, int V>
+struct PairTag {
+  static constexpr int kf = K, vf = V;
+};
+
+// Calls fn(PairTag<KF, VF>{}) for a format pair with a decode kernel;
+// returns false otherwise.
+template <typename Fn>
+bool dispatch_pair(int kf, int vf, Fn&& fn) {
+#define TQ_PAIR(K, V)                \
+  if (kf == (K) && vf == (V)) {      \
+    fn(PairTag<(K), (V)>{});         \
+    return true;                     \
+  }
+  TQ_PAIR(fid(1, 0, 0), fid(1, 0, 0))
+  TQ_PAIR(fid(2, 0, 0), fid(2, 0, 0))
+  TQ_PAIR(fid(3, 0, 0), fid(3, 0, 0))
+  TQ_PAIR(fid(4, 0, 0), fid(4, 0, 0))
+  TQ_PAIR(fid(3, 1, 0), fid(3, 1, 0))
+  TQ_PAIR(fid(2, 1, 0), fid(2, 1, 0))
+  TQ_PAIR(fid(0, 0, 1), fid(0, 0, 1))
+  TQ_PAIR(fid(1, 0, 1), fid(1, 0, 1))
+  TQ_PAIR(fid(2, 0, 1), fid(2, 0, 1))
+  TQ_PAIR(fid(3, 0, 1), fid(3, 0, 1))
+  TQ_PAIR(fid(4, 0, 0), fid(3, 0, 0))
+  TQ_PAIR(fid(4, 0, 0), fid(2, 0, 0))
+  TQ_PAIR(fid(3, 0, 0), fid(2, 0, 0))
+  TQ_PAIR(fid(8, 0, 0), fid(3, 0, 0))
+#undef TQ_PAIR
+  return false;
+}
+}  // namespace
+
+size_t decode_lut_bytes(const FormatSpec& fk, const FormatSpec& fv) {
+  size_t bytes = 0;
+  dispatch_pair(fk.id(), fv.id(), [&](auto tag) {
+    using T = decltype(tag);
+    bytes = lut_bytes_of<T::kf, T::vf>();
+  });
+  return bytes;
+}
+
+tq_status build_decode_luts(tq_params* p) {
+  cudaError_t e = cudaSuccess;
+  dispatch_pair(p->fk.id(), p->fv.id(), [&](auto tag) {
+    using T = decltype(tag);
+    if (Lut<T::kf, T::vf>::bytes == 0) return;
+    lut_image_kernel<T::kf, T::vf><<<1, kConsumers * 32>>>(p->lut_img, p->cbs32, p->cbs8_32);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
+  });
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_params_create: decode lookup tables");
+}
+
 DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) {
   DecodePlan pl{};
   pl.B = B;
@@ -1013,10 +1126,11 @@ DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len) 
   pl.ctas = num_sms_cached() < kMaxPieces ? num_sms_cached() : kMaxPieces;
   pl.part_floats = kPartAcc + (p->fv.prod ? 2 * kDim : kDim);
   const size_t units = static_cast<size_t>(B) * hkv;
-  const size_t qfrag = (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
   // piece (u, cta) uses slot u + cta: fewer than units + ctas slots
   const size_t slots = units + pl.ctas;
-  pl.ws_total_bytes = qfrag + slots * pl.group * pl.part_floats * sizeof(float);
+  pl.ws_qfrag_bytes = (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
+  pl.ws_parts_bytes = (slots * pl.group * pl.part_floats * sizeof(float) + 255) & ~size_t(255);
+  pl.ws_total_bytes = pl.ws_qfrag_bytes + pl.ws_parts_bytes;
   return pl;
 }
 
@@ -1055,11 +1169,8 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   }
   a.merge_chunk = merge_chunk_pieces(a.merge_heads, plan.part_floats);
   if (c->n_sink > kMaxSink) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: n_sink above 4096");
-  const size_t units = static_cast<size_t>(plan.B) * plan.hkv;
-  char* w = static_cast<char*>(ws);
-  a.qfrag = reinterpret_cast<uint32_t*>(w);
-  w += (units * kQfragWords * sizeof(uint32_t) + 255) & ~size_t(255);
-  a.parts = reinterpret_cast<float*>(w);
+  a.qfrag = static_cast<uint32_t*>(ws);
+  a.parts = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.ws_qfrag_bytes);
   a.out = out;
   a.out_bf16 = out_bf16;
   a.pit = p->pit32;
@@ -1067,6 +1178,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.pi = p->pi32;
   a.s = p->s32;
   a.cbs = p->cbs32;
+  a.lut_img = p->lut_img;
   a.sig = p->sig32;
   a.sparse_thr = sparse_thr;
   a.sv_stats = sv_stats;
@@ -1090,6 +1202,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   TQ_CASE(fid(4, 0, 0), fid(3, 0, 0))
   TQ_CASE(fid(4, 0, 0), fid(2, 0, 0))
   TQ_CASE(fid(3, 0, 0), fid(2, 0, 0))
+  TQ_CASE(fid(8, 0, 0), fid(3, 0, 0))
 #undef TQ_CASE
   return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attn: this K/V format pair has no decode kernel");
 }

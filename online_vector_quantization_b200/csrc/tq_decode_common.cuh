@@ -39,15 +39,15 @@ constexpr float kQjlScale = 1.2533141373155003f / kSketch;  // sqrt(pi/2)/m
 constexpr int kQfragWords = 16 * 2 * 2 * 32;
 
 // ---------------------------------------------------------------------------
-// Formats (id = mse_bits | mixed << 3 | prod << 4).  Segments of the MSE row:
+// Formats (id = mse_bits | mixed << 4 | prod << 5).  Segments of the MSE row:
 // one uniform segment of 128 coordinates, or (mixed) 64 coordinates at
 // mse+1 bits followed by 64 at mse bits.
 // ---------------------------------------------------------------------------
 template <int F>
 struct Fmt {
-  static constexpr int mse = F & 7;
-  static constexpr bool mixed = (F >> 3) & 1;
-  static constexpr bool prod = (F >> 4) & 1;
+  static constexpr int mse = F & 15;
+  static constexpr bool mixed = (F >> 4) & 1;
+  static constexpr bool prod = (F >> 5) & 1;
   static constexpr int nseg = mixed ? 2 : (mse > 0 ? 1 : 0);
   static constexpr int code_bytes = mixed ? 8 * (2 * mse + 1) : 16 * mse;
   static constexpr int b0 = mixed ? mse + 1 : mse;
@@ -65,14 +65,19 @@ struct Fmt {
 // 3-bit pair in the low six bits of any byte is looked up with one byte
 // permute.  Region B (row stride 256 B, 8 B per lane): four 2-bit centroids of
 // byte r.  With 2- and 3-bit widths only (t2a), bytes [0, 128) of region A row
-// r hold half2(c2[r & 3], c2[(r >> 2) & 3]) instead, and there is no region B.  Entry (r, lane) sits at r*256 + lane*4 (or *8): every lane hits its
-// own bank.
+// r hold half2(c2[r & 3], c2[(r >> 2) & 3]) instead, and there is no region B.
+// With 8-bit keys (t8), bytes [0, 128) of row r hold half2(c8[r], c8[r]): one
+// code byte, one lookup.  Entry (r, lane) sits at r*256 + lane*4 (or *8):
+// every lane hits its own bank.
 template <int KF, int VF>
 struct Lut {
+  static constexpr bool t8 = Fmt<KF>::uses(8);
   static constexpr bool t4 = Fmt<KF>::uses(4) || Fmt<VF>::uses(4);
   static constexpr bool t3 = Fmt<KF>::uses(3) || Fmt<VF>::uses(3);
   static constexpr bool t2 = Fmt<KF>::uses(2) || Fmt<VF>::uses(2);
-  static constexpr int region_a = (t4 || (t3 && t2)) ? 65536 : (t3 ? 16384 : 0);
+  static_assert(!Fmt<VF>::uses(8), "8-bit codes are decoded on the key side only");
+  static_assert(!(t8 && (t4 || t2)), "8-bit keys pair with 3-bit (or 1-bit) values");
+  static constexpr int region_a = (t8 || t4 || (t3 && t2)) ? 65536 : (t3 ? 16384 : 0);
   static constexpr bool t3_wide = t3 && region_a == 65536;
   // 2-bit and 3-bit widths without 4-bit ones: the 2-bit pair table takes the
   // free bytes [0, 128) of region A instead of a region B of its own
@@ -261,6 +266,13 @@ struct KChunk {
       const uint32_t src_hi = (S & 1) ? __funnelshift_r(w[0], w1, 18) : __funnelshift_r(w[0], w1, 6);
       lo = lut32(smem, byte_addr(src_lo, lb, kb));
       hi = lut32(smem, byte_addr(src_hi, lb, kb));
+    } else if constexpr (B == 8) {
+      // one lookup per code byte; the low halves of two entries form a pair
+      const uint32_t ww = w[s];
+      const uint32_t e0 = lut32(smem, byte_addr(ww, lane4, 0)), e1 = lut32(smem, byte_addr(ww, lane4, 1));
+      const uint32_t e2 = lut32(smem, byte_addr(ww, lane4, 2)), e3 = lut32(smem, byte_addr(ww, lane4, 3));
+      lo = __byte_perm(e0, e1, 0x5410);
+      hi = __byte_perm(e2, e3, 0x5410);
     } else if constexpr (B == 4) {
       const uint32_t ww = w[s >> 1];
       lo = lut32(smem, byte_addr(ww, lane4, 2 * (s & 1)));
@@ -473,10 +485,12 @@ struct DecodeArgs {
   int B, hkv, group, hq, capacity, n_sink, max_len, part_floats;
   int ctas;   // CTAs of the decode grid (pieces a unit can be cut into)
   int chunk;  // quantized tokens per scheduled chunk
+  int unit_slack;  // empty schedule slots at the start of each unit
   int merge_chunk;  // pieces the merge kernel stages in shared memory at a time
   int merge_heads;  // query heads per merge CTA (the group, or 1: one CTA per (unit, head))
   float* parts;
   const uint32_t* qfrag;
+
   void* out;
   int out_bf16;
   const float* pit;  // Pi^T
@@ -484,6 +498,7 @@ struct DecodeArgs {
   const float* pi;   // Pi
   const float* s;    // S
   const float* cbs;  // sigma-scaled centroids [5][16] (the values the MMAs see)
+  const uint8_t* lut_img;  // the decode kernel's lookup tables, prebuilt (params)
   const float* sig;  // sigma per width [5]
   float sparse_thr;
   unsigned long long* sv_stats;  // sparse-V tallies [4] (device) or null
@@ -517,6 +532,58 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // are visible (a no-op in a kernel launched without the attribute).
 __device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// B fragments of a rotated query: lane (g, t) supplies column g; k-steps 0..7
+// from the MSE segments, 8..15 from the QJL segment.  Unpacked: column g =
+// head g, halves hi (x = 0) and lo (x = 1).  Packed (group <= 4): column g < 4
+// = hi of head g, column g >= 4 = lo of head g - 4, in x = 0.  qt: [8][128]
+// rotated, scaled query (MSE coordinates); qsk: [8][128] sketch S q (prod
+// keys).  Threads tid = 0.. of nthreads write the kQfragWords words of dst.
+template <int KF>
+__device__ __forceinline__ void write_qfrag(const float* qt, const float* qsk, int pack, uint32_t* dst, int tid,
+                                            int nthreads) {
+  using KR = KRow<KF>;
+  using FK = Fmt<KF>;
+  for (int i = tid; i < 16 * 32; i += nthreads) {
+    const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
+    int dims[4] = {0, 0, 0, 0};
+    bool valid = true;
+    const bool qjl = ks >= 8;
+    if (!qjl) {
+      if (FK::nseg == 0) {
+        valid = false;
+      } else if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
+        for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
+      } else {
+        for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
+      }
+    } else {
+      if (!FK::prod) valid = false;
+      for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
+    }
+    const int head = pack ? (g & 3) : g;
+    const float* src = (qjl ? qsk : qt) + head * kDim;
+    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
+    if (valid) {
+      for (int r = 0; r < 2; ++r) {
+        const float x0 = src[dims[2 * r]], x1 = src[dims[2 * r + 1]];
+        const __half2 h = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(h);
+        hi[r] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[r] = h2bits(x0 - hf.x, x1 - hf.y);
+      }
+    }
+    for (int r = 0; r < 2; ++r) {
+      if (pack) {
+        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = g < 4 ? hi[r] : lo[r];
+        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = 0;
+      } else {
+        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
+        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
+      }
+    }
+  }
+}
 
 // ---------------------------------------------------------------------------
 // 1. query rotation: one CTA per (sequence, kv-head).  Threads 0..127 form
@@ -599,50 +666,8 @@ __global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
     }
     __syncthreads();
   }
-  // B fragments: lane (g, t) supplies column g; k-steps 0..7 from the MSE
-  // segments, 8..15 from the QJL segment.  Unpacked: column g = head g, halves
-  // hi (x = 0) and lo (x = 1).  Packed (group <= 4): column g < 4 = hi of head
-  // g, column g >= 4 = lo of head g - 4, in x = 0.
   uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  for (int i = tid; i < 16 * 32; i += kQrotThreads) {
-    const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
-    int dims[4] = {0, 0, 0, 0};
-    bool valid = true;
-    const bool qjl = ks >= 8;
-    if (!qjl) {
-      if (FK::nseg == 0) {
-        valid = false;
-      } else if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
-        for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
-      } else {
-        for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
-      }
-    } else {
-      if (!FK::prod) valid = false;
-      for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
-    }
-    const int head = a.pack ? (g & 3) : g;
-    const float* src = qjl ? qsk[head] : qt[head];
-    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
-    if (valid) {
-      for (int r = 0; r < 2; ++r) {
-        const float x0 = src[dims[2 * r]], x1 = src[dims[2 * r + 1]];
-        const __half2 h = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(h);
-        hi[r] = *reinterpret_cast<const uint32_t*>(&h);
-        lo[r] = h2bits(x0 - hf.x, x1 - hf.y);
-      }
-    }
-    for (int r = 0; r < 2; ++r) {
-      if (a.pack) {
-        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = g < 4 ? hi[r] : lo[r];
-        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = 0;
-      } else {
-        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
-        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
-      }
-    }
-  }
+  write_qfrag<KF>(&qt[0][0], &qsk[0][0], a.pack, dst, tid, kQrotThreads);
 }
 
 // Shared addresses of the planes of one staged chunk.
@@ -851,10 +876,17 @@ __device__ __forceinline__ void consumers_sync() {
 
 // The lookup tables of a format pair (see Lut), written by the consumer
 // threads (thread index tid < kConsumers * 32) from the sigma-scaled
-// centroids cb staged in shared memory.
+// centroids cb (widths 1..4) and cb8 (the 8-bit codebook, 8-bit keys only).
 template <typename L>
-__device__ __forceinline__ void build_luts(unsigned char* lut_mem, const float* cb, int tid) {
+__device__ __forceinline__ void build_luts(unsigned char* lut_mem, const float* cb, int tid,
+                                           const float* cb8 = nullptr) {
   constexpr int NTC = kConsumers * 32;
+  if constexpr (L::t8) {
+    for (int i = tid; i < 256 * 32; i += NTC) {
+      const int r = i >> 5, ln = i & 31;
+      *reinterpret_cast<uint32_t*>(lut_mem + r * 256 + ln * 4) = h2bits(cb8[r], cb8[r]);
+    }
+  }
   if constexpr (L::t4) {
     for (int i = tid; i < 256 * 32; i += NTC) {
       const int r = i >> 5, ln = i & 31;
@@ -925,7 +957,7 @@ cudaError_t launch_overlapped(Kernel kernel, dim3 grid, int threads, size_t smem
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 3) | (prod << 4); }
+constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 4) | (prod << 5); }
 
 }  // namespace
 }  // namespace tq

@@ -342,7 +342,8 @@ static double codebook_sigma(const double* c, int levels) {
 
 static bool make_format(int bits, int mode, int mixed, FormatSpec* f, std::string* why) {
   if (mode != TQ_MODE_MSE && mode != TQ_MODE_PROD) { *why = "mode must be MSE or PROD"; return false; }
-  if (bits < 1 || bits > 4) { *why = "bits must be in 1..4"; return false; }
+  const bool wide = bits == kWideBits && mode == TQ_MODE_MSE && mixed == 0;
+  if ((bits < 1 || bits > 4) && !wide) { *why = "bits must be in 1..4, or 8 in MSE mode (unmixed rows)"; return false; }
   if (mixed != 0 && mixed != 1) { *why = "mixed must be 0 or 1"; return false; }
   f->total_bits = bits;
   f->prod = mode == TQ_MODE_PROD;
@@ -532,7 +533,47 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   // host staging of every device table
   std::vector<float> pi32(d * d), pit32(d * d), s32(m * d), st32(d * m), mt32(d * m);
   std::vector<float> cb32((kMaxBits + 1) * kBookSlots, 0.f), bd32((kMaxBits + 1) * kBookSlots, 0.f);
-  std::vector<float> cbs32((kMaxBits + 1) * kBookSlots, 0.f), sig32(kMaxBits + 1, 1.f);
+  std::vector<float> cbs32((kMaxBits + 1) * kBookSlots, 0.f), sig32(kSigSlots, 1.f);
+  std::vector<float> cb8_32(256, 0.f), cbs8_32(256, 0.f), bd8_32(256, INFINITY);
+  std::vector<double> cb8_64(256, 0.0), pit64(static_cast<size_t>(d) * d);
+  std::vector<float> cell8;  // pairs {count, bound}
+  for (int r = 0; r < d; ++r)
+    for (int c = 0; c < d; ++c) pit64[static_cast<size_t>(c) * d + r] = p->pi[static_cast<size_t>(r) * d + c];
+  if (fk.wide() || fv.wide()) {
+    double c[256], t[255];
+    lloyd_max(d, kWideBits, c, t);
+    const double sg = codebook_sigma(c, 256);
+    sig32[kWideBits] = static_cast<float>(sg);
+    for (int k = 0; k < 256; ++k) {
+      cb8_32[k] = static_cast<float>(c[k]);
+      cbs8_32[k] = static_cast<float>(c[k] * static_cast<double>(sig32[kWideBits]));
+      cb8_64[k] = c[k];
+    }
+    for (int k = 0; k < 255; ++k) bd8_32[k] = static_cast<float>(t[k]);
+    // cells over |u| no wider than the closest two positive bounds, so each
+    // holds at most one bound: the code of |u| is the count at the cell's
+    // start plus 1 if |u| passes the cell's bound
+    double min_gap = INFINITY;
+    for (int k = 128; k + 1 < 255; ++k) min_gap = std::min(min_gap, t[k + 1] - t[k]);
+    const float w = static_cast<float>(0.99 * min_gap);
+    const int n_cells = static_cast<int>(std::ceil(t[254] / w)) + 2;
+    if (n_cells > kCell8Max) { delete p; return fail(TQ_ERR_UNSUPPORTED, "tq_params_create: 8-bit code cells"); }
+    cell8.resize(2 * static_cast<size_t>(n_cells));
+    for (int cidx = 0; cidx < n_cells; ++cidx) {
+      const float lo = cidx * w, hi = (cidx + 1) * w;
+      int cnt = 0;
+      float inside = INFINITY;
+      for (int k = 128; k < 255; ++k) {  // the positive bounds t[128..254]
+        const float b = static_cast<float>(t[k]);
+        if (b <= lo) ++cnt;
+        else if (b < hi) inside = std::min(inside, b);
+      }
+      cell8[2 * cidx] = static_cast<float>(cnt);
+      cell8[2 * cidx + 1] = inside;
+    }
+    p->cell8_n = n_cells;
+    p->cell8_inv_w = 1.f / w;
+  }
   std::vector<double> cb64((kMaxBits + 1) * kBookSlots, 0.0);
   for (int r = 0; r < d; ++r)
     for (int c = 0; c < d; ++c) {
@@ -577,7 +618,11 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
          o_st = take(st32.size() * 4), o_mt = take(mt32.size() * 4), o_pi64 = take(p->pi.size() * 8),
          o_s64 = take(p->s.size() * 8), o_cb = take(cb32.size() * 4), o_bd = take(bd32.size() * 4),
          o_cb64 = take(cb64.size() * 8), o_cbs = take(cbs32.size() * 4), o_sig = take(sig32.size() * 4),
-         o_status = take(sizeof(int32_t)), o_img = take(static_cast<size_t>(kTcImgCount) * kTcImgBytes);
+         o_status = take(sizeof(int32_t)), o_img = take(static_cast<size_t>(kTcImgCount) * kTcImgBytes),
+         o_cb8 = take(256 * 4), o_cbs8 = take(256 * 4), o_bd8 = take(256 * 4), o_cb864 = take(256 * 8),
+         o_cell8 = take(cell8.size() * 4), o_pit64 = take(pit64.size() * 8);
+  p->lut_bytes = decode_lut_bytes(p->fk, p->fv);
+  const size_t o_lut = take(p->lut_bytes);
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->block, off);
   if (e != cudaSuccess) {
@@ -600,6 +645,13 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
   p->sig32 = reinterpret_cast<float*>(base + o_sig);
   p->status32 = reinterpret_cast<int32_t*>(base + o_status);
   p->tc_img = reinterpret_cast<uint8_t*>(base + o_img);
+  p->lut_img = p->lut_bytes ? reinterpret_cast<uint8_t*>(base + o_lut) : nullptr;
+  p->cb8_32 = reinterpret_cast<float*>(base + o_cb8);
+  p->cbs8_32 = reinterpret_cast<float*>(base + o_cbs8);
+  p->bd8_32 = reinterpret_cast<float*>(base + o_bd8);
+  p->cb8_64 = reinterpret_cast<double*>(base + o_cb864);
+  p->cell8 = cell8.empty() ? nullptr : reinterpret_cast<float2*>(base + o_cell8);
+  p->pit64 = reinterpret_cast<double*>(base + o_pit64);
   const std::vector<uint8_t> img = tensor_core_images(p->pi, mt64);
   e = cudaMemset(p->status32, 0, sizeof(int32_t));
   if (e != cudaSuccess) {
@@ -614,13 +666,25 @@ tq_status tq_params_create(const tq_config* cfg, tq_params** out) {
       {p->s64, p->s.data(), p->s.size() * 8},    {p->cb32, cb32.data(), cb32.size() * 4},
       {p->bd32, bd32.data(), bd32.size() * 4},   {p->cb64, cb64.data(), cb64.size() * 8},
       {p->cbs32, cbs32.data(), cbs32.size() * 4}, {p->sig32, sig32.data(), sig32.size() * 4},
-      {p->tc_img, img.data(), img.size()}};
+      {p->tc_img, img.data(), img.size()},       {p->cb8_32, cb8_32.data(), 256 * 4},
+      {p->cbs8_32, cbs8_32.data(), 256 * 4},     {p->bd8_32, bd8_32.data(), 256 * 4},
+      {p->cb8_64, cb8_64.data(), 256 * 8},       {p->cell8, cell8.data(), cell8.size() * 4},
+      {p->pit64, pit64.data(), pit64.size() * 8}};
   for (auto& c : copies) {
+    if (c.n == 0) continue;
     e = cudaMemcpy(c.dst, c.src, c.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
       cudaFree(p->block);
       delete p;
       return cuda_fail(e, "tq_params_create: upload");
+    }
+  }
+  if (p->lut_bytes) {
+    const tq_status st = build_decode_luts(p);
+    if (st != TQ_OK) {
+      cudaFree(p->block);
+      delete p;
+      return st;
     }
   }
   *out = p;

@@ -14,8 +14,11 @@ namespace tq {
 
 constexpr int kDim = 128;       // head dimension handled by the kernels
 constexpr int kSketch = 128;    // QJL sketch size m
-constexpr int kMaxBits = 4;     // largest MSE code width used by the kernels
-constexpr int kBookSlots = 16;  // centroid slots per width in device tables
+constexpr int kMaxBits = 4;     // largest MSE width of the small codebook tables
+constexpr int kBookSlots = 16;  // centroid slots per width in those tables
+constexpr int kWideBits = 8;    // the 8-bit MSE width (256 levels) has tables of its own
+constexpr int kSigSlots = kWideBits + 1;  // sigma per width, 0..8
+constexpr int kCell8Max = 512;  // code-search cells of the 8-bit codebook (quantize kernels)
 
 // One quantizer format (keys or values).
 //   mse_bits: width of the uniform MSE part (bits, or bits-1 in prod mode);
@@ -29,8 +32,9 @@ struct FormatSpec {
   int prod = 0;
   int code_bytes = 0;
   int qjl_bytes = 0;
-  int id() const { return mse_bits | (mixed << 3) | (prod << 4); }
+  int id() const { return mse_bits | (mixed << 4) | (prod << 5); }
   int width(int j) const { return (mixed && j < kDim / 2) ? mse_bits + 1 : mse_bits; }
+  bool wide() const { return mse_bits == kWideBits; }
 };
 
 }  // namespace tq
@@ -52,13 +56,31 @@ struct tq_params {
   double* s64 = nullptr;   // S  [m][d] fp64 (dequantize)
   float* cb32 = nullptr;   // centroids [kMaxBits+1][16] (row b = width b)
   float* cbs32 = nullptr;  // centroids times sigma_b, the values fed to fp16 MMAs
-  float* sig32 = nullptr;  // sigma_b [kMaxBits+1]: scale making sigma_b*c near-exact in fp16
+  float* sig32 = nullptr;  // sigma_b [kSigSlots]: scale making sigma_b*c near-exact in fp16
   float* bd32 = nullptr;   // decision bounds [kMaxBits+1][16]
   double* cb64 = nullptr;  // centroids fp64 [kMaxBits+1][16]
   int32_t* status32 = nullptr;  // device word that plain quantize kernels OR error bits into
+  // 8-bit MSE codebook (256 levels): centroids, sigma-scaled centroids (the
+  // decode tables), the 255 decision bounds, fp64 centroids (dequantize) and
+  // the code-search cells of the positive half: cell c of width 1/cell8_inv_w
+  // holds {number of positive bounds at or below its start, the one bound
+  // inside it or +inf}.  Pi^T in fp64 for the 8-bit SIMT quantizer.
+  float* cb8_32 = nullptr;
+  float* cbs8_32 = nullptr;
+  float* bd8_32 = nullptr;
+  double* cb8_64 = nullptr;
+  float2* cell8 = nullptr;
+  int cell8_n = 0;
+  float cell8_inv_w = 0.f;
+  double* pit64 = nullptr;
   // Tensor-core B operands of the quantize kernels, each a 128 x 128 16-bit
   // tile in the 128-byte-swizzled K-major layout (32 KB; see kTcImg*)
   uint8_t* tc_img = nullptr;
+  // The decode kernel's shared-memory lookup tables for the (fk, fv) pair,
+  // built once on the device (tq_attn.cu) and bulk-copied by every decode
+  // CTA at its start; lut_bytes = 0 when the pair has no decode kernel.
+  uint8_t* lut_img = nullptr;
+  size_t lut_bytes = 0;
 };
 
 namespace tq {
@@ -107,6 +129,8 @@ tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_pa
 
 struct DecodePlan {
   int B, hq, hkv, group, max_len, ctas, part_floats;
+  size_t ws_qfrag_bytes;  // rotated-query fragments, then
+  size_t ws_parts_bytes;  // the split partials
   size_t ws_total_bytes;
 };
 DecodePlan plan_decode(const tq_params* p, int B, int hq, int hkv, int max_len);
@@ -119,6 +143,10 @@ tq_status check_decode_call(const tq_params* p, const void* q, int q_dtype, cons
 tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_cache* c,
                         const DecodePlan& plan, void* out, int out_bf16, void* ws,
                         float sparse_thr, unsigned long long* sv_stats, cudaStream_t st);
+// Size of the decode lookup-table image of a format pair (0: no decode
+// kernel), and its construction into p->lut_img (legacy stream, synchronized).
+size_t decode_lut_bytes(const FormatSpec& fk, const FormatSpec& fv);
+tq_status build_decode_luts(tq_params* p);
 size_t search_workspace_bytes();
 int search_max_k();
 tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed* db, int64_t n, const void* q,

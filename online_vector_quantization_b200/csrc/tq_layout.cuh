@@ -18,7 +18,8 @@
 // that holds the lane's coordinates, copied as is.  Every piece is a whole
 // number of bytes, so a byte of the tile belongs to exactly one token.
 // A lane block is code_bytes / 2 bytes, stored as columns: the first 16 bytes
-// of every lane (lane L's at 16 L), then the next 16 (if any), then 8, then 4.
+// of every lane (lane L's at 16 L), then the next 16 while 16 remain, then 8,
+// then 4.
 #pragma once
 
 #include <stdint.h>

@@ -41,6 +41,11 @@ struct QuantArgs {
   const float* mt;   // (S Pi^T)^T [d][m]
   const float* cb;   // [5][16]
   const float* bd;   // [5][16]
+  // 8-bit codebook (mse_bits == 8): code-search cells, fp64 Pi^T
+  const float2* cell8;
+  int cell8_n;
+  float cell8_inv_w;
+  const double* pit64;
   // plain destination (row = vector index)
   uint8_t* codes;
   float* norms;
@@ -50,12 +55,74 @@ struct QuantArgs {
   int append;
   int kside;
   const int32_t* seq_ids;
-  const int32_t* lens;
+  int32_t* lens;
   int n_tok, hkv, capacity, n_sink, cache_seqs;
   uint16_t* sink;  // bf16 [n_seq][hkv][n_sink][d]
   int32_t* status;  // device word; bit 4 = a pipeline wait timed out
   const uint8_t* tc_img;  // tensor-core B operand images (tq_params::tc_img)
+  // A second plane (the tensor-core kernels, appends whose K and V formats
+  // are equal): one launch quantizes the keys (plane 0, the fields above) and
+  // the values (plane 1, these, in the values' arrangement); tiles
+  // [0, tiles of n) are plane 0's, the next as many plane 1's.
+  int planes;
+  const void* x2;
+  uint8_t* codes2;
+  float* norms2;
+  uint8_t* qjl2;
+  float* res2;
+  uint16_t* sink2;
+  // Folded length update of an append: every CTA of the append's kernels
+  // (arrive_total of them) counts itself in bits 16..31 of the cache's status
+  // word once it has read lens for the last time; the last one adds n_tok to
+  // the length of each of the n_seq_in appended sequences (or flags bit 1)
+  // and returns the count to zero.  0 = no update in this launch.
+  int arrive_total;
+  int n_seq_in;
 };
+
+// The input and destinations of plane pl.
+struct PlaneDst {
+  const void* x;
+  uint8_t* codes;
+  float* norms;
+  uint8_t* qjl;
+  float* res;
+  uint16_t* sink;
+  int kside;
+};
+__device__ __forceinline__ PlaneDst plane_dst(const QuantArgs& a, int pl) {
+  return pl ? PlaneDst{a.x2, a.codes2, a.norms2, a.qjl2, a.res2, a.sink2, 0}
+            : PlaneDst{a.x, a.codes, a.norms, a.qjl, a.res, a.sink, a.kside};
+}
+
+// The end of an append kernel's CTA (every thread calls it, after the CTA's
+// last read of lens): see QuantArgs::arrive_total.  A sequence whose append
+// does not fit (or whose index or stored length is out of range) keeps its
+// length, and bit 1 is set in the status word.
+__device__ void append_arrive(const QuantArgs& a, int count = 1) {
+  if (!a.append || a.arrive_total <= 0) return;
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int old = atomicAdd(a.status, count << 16);
+    s_last = ((old >> 16) & 0xFFFF) + count == a.arrive_total;
+    if (s_last) __threadfence();
+  }
+  __syncthreads();
+  if (!s_last) return;
+  const int limit = a.n_sink + a.capacity;
+  for (int i = threadIdx.x; i < a.n_seq_in; i += blockDim.x) {
+    const int seq = a.seq_ids[i];
+    const int len = (seq >= 0 && seq < a.cache_seqs) ? __ldcg(a.lens + seq) : -1;
+    if (len < 0 || len + a.n_tok > limit)
+      atomicOr(a.status, 1);
+    else
+      a.lens[seq] = len + a.n_tok;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAnd(a.status, 0xFFFF);
+}
 
 struct SmemQuant {
   float pit[kDim][kDim];     // pit[k][j] = Pi[j][k]
@@ -461,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_kernel(QuantArgs a) {
       }
     }
   }
+  append_arrive(a);
 }
 
 // ---------------------------------------------------------------------------
@@ -488,6 +556,7 @@ constexpr int kTcTile = 2 * kTcBox;               // one 128 x 128 bf16 tile: 32
 constexpr int kTcThreads = 10 * 32;
 constexpr int kTcSmem = 2 * kTcTile + kTcStages * kTcTile + 1024;  // Pi hi/lo, x ring, alignment slack
 constexpr int kTcCols = 256;                      // TMEM columns: two 128-column accumulators
+constexpr int kTcSmemWide = 3 * kTcTile + 3 * kTcTile + 1024;  // 8-bit: Pi a/b/c, three x stages
 
 // Code of u for a width-W codebook whose decision bounds are symmetric about
 // 0: pb[i] = the i-th positive bound (pb[0] = 0 is the middle one).  Equals the
@@ -515,6 +584,17 @@ __device__ __forceinline__ uint32_t sym_code(float u, const float (&pb)[8]) {
   return u > 0.f ? H + j : H - 1u - j;
 }
 
+// 8-bit code of u from the cell table of the positive half (cells hold the
+// count of positive bounds at or below their start and the one bound inside
+// them): the count of bounds strictly below u, except on exact ties.
+__device__ __forceinline__ uint32_t code8(float u, const float2* cells, int n_cells, float inv_w) {
+  const float a = fabsf(u);
+  const int c = min(static_cast<int>(a * inv_w), n_cells - 1);
+  const float2 cell = cells[c];
+  const uint32_t j = static_cast<uint32_t>(cell.x) + (a > cell.y ? 1u : 0u);
+  return u > 0.f ? 128u + j : 127u - j;
+}
+
 // 32 codes of width W from one 32-column TMEM chunk, packed LSB-first into W words.
 template <int W>
 __device__ __forceinline__ void pack_chunk(const uint32_t (&y)[32], float inv_nu, const float (&pb)[8],
@@ -540,22 +620,30 @@ struct TcFormat {
 
 template <int B, int MIXED>
 __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                    const __grid_constant__ CUtensorMap xmap2,
                                                                     QuantArgs a) {
   using namespace sm100;
   using TF = TcFormat<B, MIXED>;
+  // 8-bit codes: Pi in three bf16 terms (the 255 bounds sit ~1.5e-3 apart,
+  // so the rotation must be good to ~1e-8) and one fewer x stage to make room
+  constexpr bool kWide = B == kWideBits;
+  constexpr int NPI = kWide ? 3 : 2, NST = kWide ? 3 : kTcStages;
   extern __shared__ __align__(16) unsigned char smem_tc[];
-  __shared__ __align__(8) uint64_t x_full[kTcStages], x_empty[kTcStages], t_full[2], t_empty[2], b_full;
+  __shared__ __align__(8) uint64_t x_full[NST], x_empty[NST], t_full[2], t_empty[2], b_full;
+  __shared__ float2 s_cell8[kWide ? kCell8Max : 1];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ float s_pb[2][8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t raw = smem_u32(smem_tc);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t pih = base, pil = base + kTcTile, xs0 = base + 2 * kTcTile;
+  const uint32_t pih = base, pil = base + kTcTile, xs0 = base + NPI * kTcTile;
 
   // Pi (row j = output coordinate, K = input coordinate) as bf16 hi and lo
   // halves arrives by bulk copy from the prepared images
-  if (tid < 16) {
+  if constexpr (kWide) {
+    for (int i = tid; i < a.cell8_n; i += kTcThreads) s_cell8[i] = a.cell8[i];
+  } else if (tid < 16) {
     const int seg = tid >> 3, i = tid & 7;
     const int w = seg ? TF::b1 : TF::b0;
     const int half = 1 << (w - 1);
@@ -566,7 +654,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 1 + 4);  // the MMA commit and the four epilogue warps
     }
@@ -582,27 +670,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int64_t plane_tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int64_t n_tiles = plane_tiles * a.planes;
 
   if (warp == 8) {
     // ---- producer: the B operand once, then the x tiles
     if (lane == 0) {
       prefetch_tensormap(&xmap);
-      mbar_expect_tx(&b_full, 2 * kTcTile);
-      bulk_g2s_addr(pih, a.tc_img + kTcImgPiHi * kTcImgBytes, kTcTile, &b_full);
-      bulk_g2s_addr(pil, a.tc_img + kTcImgPiLo * kTcImgBytes, kTcTile, &b_full);
+      if (a.planes > 1) prefetch_tensormap(&xmap2);
+      mbar_expect_tx(&b_full, NPI * kTcTile);
+      if constexpr (kWide) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          bulk_g2s_addr(pih + t * kTcTile, a.tc_img + (kTcImgPiA + t) * kTcImgBytes, kTcTile, &b_full);
+      } else {
+        bulk_g2s_addr(pih, a.tc_img + kTcImgPiHi * kTcImgBytes, kTcTile, &b_full);
+        bulk_g2s_addr(pil, a.tc_img + kTcImgPiLo * kTcImgBytes, kTcTile, &b_full);
+      }
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
-        const int s = i % kTcStages;
-        if (i >= kTcStages && !mbar_wait(&x_empty[s], ((i / kTcStages) - 1) & 1)) s_abort = 1;
+        const int s = i % NST;
+        if (i >= NST && !mbar_wait(&x_empty[s], ((i / NST) - 1) & 1)) s_abort = 1;
         if (s_abort) break;
         mbar_expect_tx(&x_full[s], kTcTile);
-        tma_load_2d(xs0 + s * kTcTile, &xmap, 0, static_cast<int>(tile * kTcRows), &x_full[s]);
-        tma_load_2d(xs0 + s * kTcTile + kTcBox, &xmap, 64, static_cast<int>(tile * kTcRows), &x_full[s]);
+        const int pl = tile >= plane_tiles;
+        const CUtensorMap* map = pl ? &xmap2 : &xmap;
+        const int row0 = static_cast<int>((tile - pl * plane_tiles) * kTcRows);
+        tma_load_2d(xs0 + s * kTcTile, map, 0, row0, &x_full[s]);
+        tma_load_2d(xs0 + s * kTcTile + kTcBox, map, 64, row0, &x_full[s]);
       }
       // loads still in flight land before the CTA may exit
-      for (int k = i - kTcStages; k < i; ++k)
-        if (k >= 0) mbar_wait(&x_full[k % kTcStages], (k / kTcStages) & 1);
+      for (int k = i - NST; k < i; ++k)
+        if (k >= 0) mbar_wait(&x_full[k % NST], (k / NST) & 1);
       mbar_wait(&b_full, 0);
     }
   } else if (warp == 9) {
@@ -612,8 +711,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
       if (!mbar_wait(&b_full, 0)) s_abort = 1;
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
-        const int s = i % kTcStages, buf = i & 1;
-        if (!mbar_wait(&x_full[s], (i / kTcStages) & 1)) s_abort = 1;
+        const int s = i % NST, buf = i & 1;
+        if (!mbar_wait(&x_full[s], (i / NST) & 1)) s_abort = 1;
         if (i >= 2 && !s_abort && !mbar_wait(&t_empty[buf], ((i >> 1) - 1) & 1)) s_abort = 1;
         if (s_abort) break;
         tc_fence_after();
@@ -624,6 +723,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
           const uint64_t ad = sw128_kmajor_desc(xs0 + s * kTcTile + off);
           umma_bf16(d, ad, sw128_kmajor_desc(pih + off), idesc, k > 0);
           umma_bf16(d, ad, sw128_kmajor_desc(pil + off), idesc, true);
+          if constexpr (kWide) umma_bf16(d, ad, sw128_kmajor_desc(pih + 2 * kTcTile + off), idesc, true);
         }
         umma_commit(&x_empty[s]);
         umma_commit(&t_full[buf]);
@@ -642,9 +742,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
       if ((i & 1) != g) continue;
       if (s_abort) break;
-      const int s = i % kTcStages, buf = i & 1;
+      const int s = i % NST, buf = i & 1;
       // norm of the row from the staged bf16 tile
-      if (!mbar_wait(&x_full[s], (i / kTcStages) & 1)) {
+      if (!mbar_wait(&x_full[s], (i / NST) & 1)) {
         s_abort = 1;
         break;
       }
@@ -681,24 +781,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
         uint32_t y[32];
         tmem_ld32(tbase + 32 * c, y);
         tmem_wait_ld();
-        if (c < 2)
+        if constexpr (kWide) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            uint32_t wd = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              wd |= code8(__uint_as_float(y[4 * jj + e]) * inv, s_cell8, a.cell8_n, a.cell8_inv_w) << (8 * e);
+            words[8 * c + jj] = wd;
+          }
+        } else if (c < 2) {
           pack_chunk<TF::b0>(y, inv, pb0, words + c * TF::b0);
-        else
+        } else {
           pack_chunk<TF::b1>(y, inv, pb1, words + 2 * TF::b0 + (c - 2) * TF::b1);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[buf]);
       // outputs
-      const int64_t v = tile * kTcRows + r;
+      const int pl = tile >= plane_tiles;
+      const PlaneDst pd = plane_dst(a, pl);
+      const int64_t v = (tile - pl * plane_tiles) * kTcRows + r;
       if (v < a.n) {
         int64_t row = v;
         if (a.append) {
           int seq, head, pos;
           row = append_row(a, v, &seq, &head, &pos);
           if (row == -2) {
-            uint16_t* dst = a.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + v * kDim);
+            uint16_t* dst = pd.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(pd.x) + v * kDim);
 #pragma unroll
             for (int k = 0; k < kDim / 8; ++k) reinterpret_cast<uint4*>(dst)[k] = src[k];
           }
@@ -709,9 +821,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
             for (int w = 0; w < TF::words; ++w) words[w] = 0u;
           }
           if (a.append) {
-            TiledStore<B, MIXED, TF::bytes>::row(a.codes, a.kside, row, words);
+            TiledStore<B, MIXED, TF::bytes>::row(pd.codes, pd.kside, row, words);
           } else {
-            uint8_t* dst = a.codes + row * TF::bytes;
+            uint8_t* dst = pd.codes + row * TF::bytes;
             if constexpr (TF::bytes % 16 == 0) {
 #pragma unroll
               for (int w = 0; w < TF::words; w += 4)
@@ -722,7 +834,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
                 *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
             }
           }
-          a.norms[row] = nu;
+          pd.norms[row] = nu;
         }
       }
     }
@@ -734,6 +846,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
     tmem_dealloc(tmem, kTcCols);
   }
   if (tid == 0 && s_abort && a.status) atomicOr(a.status, 4);
+  append_arrive(a);
 }
 
 // ---------------------------------------------------------------------------
@@ -793,6 +906,7 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
 
 template <int MB>
 __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                         const __grid_constant__ CUtensorMap xmap2,
                                                                          QuantArgs a) {
   using namespace sm100;
   constexpr int CW = MB > 0 ? 4 * MB : 1;  // packed MSE words per row (unused for MB = 0)
@@ -837,13 +951,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const int64_t n_tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int64_t plane_tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int64_t n_tiles = plane_tiles * a.planes;
 
   if (warp == 8) {
     // ---- producer: the B operands once, then tile i into the x stage of its
     // epilogue group (i & 1)
     if (lane == 0) {
       prefetch_tensormap(&xmap);
+      if (a.planes > 1) prefetch_tensormap(&xmap2);
       mbar_expect_tx(&b_full, 5 * kTcTile);
       for (int k = 0; k < 3; ++k)
         bulk_g2s_addr(pia + k * kTcTile, a.tc_img + (kTcImgPiA + k) * kTcImgBytes, kTcTile, &b_full);
@@ -855,8 +971,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
         if (i >= 2 && !mbar_wait(&x_empty[s], ((i >> 1) - 1) & 1)) s_abort = 1;
         if (s_abort) break;
         mbar_expect_tx(&x_full[s], kTcTile);
-        tma_load_2d(xs0 + s * kTcTile, &xmap, 0, static_cast<int>(tile * kTcRows), &x_full[s]);
-        tma_load_2d(xs0 + s * kTcTile + kTcBox, &xmap, 64, static_cast<int>(tile * kTcRows), &x_full[s]);
+        const int pl = tile >= plane_tiles;
+        const CUtensorMap* map = pl ? &xmap2 : &xmap;
+        const int row0 = static_cast<int>((tile - pl * plane_tiles) * kTcRows);
+        tma_load_2d(xs0 + s * kTcTile, map, 0, row0, &x_full[s]);
+        tma_load_2d(xs0 + s * kTcTile + kTcBox, map, 64, row0, &x_full[s]);
       }
       for (int k = i - 2; k < i; ++k)  // loads still in flight land before the CTA may exit
         if (k >= 0) mbar_wait(&x_full[k & 1], (k >> 1) & 1);
@@ -1024,15 +1143,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[g]);
       // outputs
-      const int64_t v = tile * kTcRows + r;
+      const int pl = tile >= plane_tiles;
+      const PlaneDst pd = plane_dst(a, pl);
+      const int64_t v = (tile - pl * plane_tiles) * kTcRows + r;
       if (v < a.n) {
         int64_t row = v;
         if (a.append) {
           int seq, head, pos;
           row = append_row(a, v, &seq, &head, &pos);
           if (row == -2) {
-            uint16_t* dst = a.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + v * kDim);
+            uint16_t* dst = pd.sink + ((static_cast<int64_t>(seq) * a.hkv + head) * a.n_sink + pos) * kDim;
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(pd.x) + v * kDim);
 #pragma unroll
             for (int k = 0; k < kDim / 8; ++k) reinterpret_cast<uint4*>(dst)[k] = src[k];
           }
@@ -1045,18 +1166,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
               for (int w = 0; w < CW; ++w) words[w] = 0u;
             }
             if (a.append) {
-              TiledStore<MB, 0, 16 * MB>::row(a.codes, a.kside, row, words);
+              TiledStore<MB, 0, 16 * MB>::row(pd.codes, pd.kside, row, words);
             } else {
-              uint8_t* dst = a.codes + row * (16 * MB);
+              uint8_t* dst = pd.codes + row * (16 * MB);
 #pragma unroll
               for (int w = 0; w < CW; w += 4)
                 *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
             }
           }
-          a.norms[row] = nu;
-          *reinterpret_cast<uint4*>(a.qjl + row * (kSketch / 8)) =
+          pd.norms[row] = nu;
+          *reinterpret_cast<uint4*>(pd.qjl + row * (kSketch / 8)) =
               zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(z[0], z[1], z[2], z[3]);
-          a.res[row] = zero ? 0.f : sqrtf(g2);
+          pd.res[row] = zero ? 0.f : sqrtf(g2);
         }
       }
     }
@@ -1068,20 +1189,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
     tmem_dealloc(tmem, kTpCols);
   }
   if (tid == 0 && s_abort && a.status) atomicOr(a.status, 4);
+  append_arrive(a);
 }
 
-// Status bit 1: the append of a sequence was refused (capacity exceeded, or a
-// sequence index / stored length out of range); its length is unchanged.
-__global__ void bump_lens_kernel(const int32_t* seq_ids, int32_t* lens, int32_t* status, int n_seq,
-                                 int n_tok, int limit, int cache_seqs) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_seq) return;
-  const int seq = seq_ids[i];
-  if (seq < 0 || seq >= cache_seqs || lens[seq] < 0 || lens[seq] + n_tok > limit)
-    atomicOr(status, 1);
-  else
-    lens[seq] += n_tok;
+// 8-bit codes for rows the tensor-core kernel does not take (fp32 input):
+// one block per vector, thread j = rotated coordinate j.  The rotation runs
+// in fp64 from Pi^T in fp64: the 255 bounds of the 8-bit codebook sit
+// ~1.5e-3 apart near 0, where an fp32 rotation error of ~1e-7 would move more
+// codes across a bound than the parity contract allows.
+__global__ void __launch_bounds__(kDim) quantize8_kernel(QuantArgs a) {
+  __shared__ double xs[kDim];
+  __shared__ double red[kDim / 32];
+  __shared__ __align__(16) uint32_t words[kDim / 4];
+  __shared__ float2 s_cell8[kCell8Max];
+  __shared__ long long s_row;
+  __shared__ int s_seq, s_head, s_pos;
+  const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+  for (int i = j; i < a.cell8_n; i += kDim) s_cell8[i] = a.cell8[i];
+  for (int64_t v = blockIdx.x; v < a.n; v += gridDim.x) {
+    const double xj = a.x_bf16 ? static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(a.x)[v * kDim + j]))
+                               : static_cast<double>(static_cast<const float*>(a.x)[v * kDim + j]);
+    if (j == 0) {
+      int seq = 0, head = 0, pos = 0;
+      s_row = a.append ? append_row(a, v, &seq, &head, &pos) : v;
+      s_seq = seq;
+      s_head = head;
+      s_pos = pos;
+    }
+    xs[j] = xj;
+    double sq = xj * xj;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if (lane == 0) red[warp] = sq;
+    __syncthreads();
+    const int64_t row = s_row;
+    if (row == -2) {  // a sink token: kept in bf16
+      a.sink[((static_cast<int64_t>(s_seq) * a.hkv + s_head) * a.n_sink + s_pos) * kDim + j] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(static_cast<float>(xj)));
+    } else if (row >= 0) {
+      const double nu = sqrt(red[0] + red[1] + red[2] + red[3]);
+      double y = 0.0;
+#pragma unroll 8
+      for (int k = 0; k < kDim; ++k) y = fma(a.pit64[k * kDim + j], xs[k], y);
+      const uint32_t code =
+          nu > 0.0 ? code8(static_cast<float>(y / nu), s_cell8, a.cell8_n, a.cell8_inv_w) : 0u;
+      // four codes per word, lane-wise
+      const uint32_t part = code << (8 * (j & 3));
+      const uint32_t w4 = part | __shfl_xor_sync(0xffffffffu, part, 1);
+      const uint32_t w = w4 | __shfl_xor_sync(0xffffffffu, w4, 2);
+      if ((j & 3) == 0) words[j >> 2] = w;
+      __syncthreads();
+      if (a.append) {
+        if (j == 0) store_tiled_codes(a.codes, make_code_tile(kWideBits, 0, 16 * kWideBits), a.kside, row, words);
+      } else if (j < kDim / 4) {
+        reinterpret_cast<uint32_t*>(a.codes + row * (16 * kWideBits))[j] = words[j];
+      }
+      if (j == 0) a.norms[row] = static_cast<float>(nu);
+    }
+    __syncthreads();
+  }
+  append_arrive(a);
 }
+
+// Arrivals on behalf of `count` CTAs of an append kernel that could not be
+// launched, so that the length update still happens once and the count
+// returns to zero.
+__global__ void append_arrive_kernel(QuantArgs a, int count) { append_arrive(a, count); }
 
 // Row import / export between packed rows (tq_quantize's format) and the
 // quantized rows of one cache unit: codes converted to / from the tiled code
@@ -1123,7 +1296,7 @@ constexpr int kDeqVecs = 8;
 __global__ void __launch_bounds__(kDim) dequantize_kernel(
     const uint8_t* codes, const float* norms, const uint8_t* qjl, const float* res, int64_t n,
     int mse_bits, int mixed, int prod, int code_bytes, const double* pi64, const double* s64,
-    const double* cb64, float* out) {
+    const double* cb64, const double* cb8_64, float* out) {
   __shared__ double chat[kDeqVecs][kDim];
   __shared__ double zs[kDeqVecs][kSketch];
   const int i = threadIdx.x;
@@ -1139,7 +1312,7 @@ __global__ void __launch_bounds__(kDim) dequantize_kernel(
         uint32_t w = row[bit >> 3];
         if ((bit & 7) + b > 8) w |= static_cast<uint32_t>(row[(bit >> 3) + 1]) << 8;
         const int idx = (w >> (bit & 7)) & ((1u << b) - 1);
-        c = cb64[b * kBookSlots + idx];
+        c = b == kWideBits ? cb8_64[idx] : cb64[b * kBookSlots + idx];
       }
       if (prod) z = ((qjl[gv * (kSketch / 8) + (i >> 3)] >> (i & 7)) & 1) ? 1.0 : -1.0;
     }
@@ -1200,72 +1373,101 @@ EncodeTiledFn encode_tiled() {
 }
 
 template <int MB>
-tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
+tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
   cudaError_t e =
       ensure_dyn_smem<quantize_tc_prod_kernel<MB>>(kTpSmem);
   if (e == cudaSuccess) {
-    quantize_tc_prod_kernel<MB><<<grid, kTcThreads, kTpSmem, st>>>(map, a);
+    quantize_tc_prod_kernel<MB><<<grid, kTcThreads, kTpSmem, st>>>(maps[0], maps[1], a);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core prod quantize kernel launch");
 }
 
 template <int B, int MIXED>
-tq_status launch_tc(const QuantArgs& a, const CUtensorMap& map, int grid, cudaStream_t st) {
-  cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED>>(kTcSmem);
+tq_status launch_tc(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
+  constexpr int smem = B == kWideBits ? kTcSmemWide : kTcSmem;
+  cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED>>(smem);
   if (e == cudaSuccess) {
-    quantize_tc_kernel<B, MIXED><<<grid, kTcThreads, kTcSmem, st>>>(map, a);
+    quantize_tc_kernel<B, MIXED><<<grid, kTcThreads, smem, st>>>(maps[0], maps[1], a);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core quantize kernel launch");
 }
 
-// bf16 rows: tensor-core rotation (MSE 1..4 bits, mixed 2.5 and 3.5, prod 1..4).
-bool tc_eligible(const QuantArgs& a) {
-  const bool fmt_ok = a.prod ? (!a.mixed && a.mse_bits >= 0 && a.mse_bits <= 3)
-                             : (a.mse_bits >= 1 && (a.mixed ? (a.mse_bits == 2 || a.mse_bits == 3) : a.mse_bits <= 4));
-  return a.x_bf16 && fmt_ok && a.n <= (int64_t(1) << 31) &&
-         (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 && encode_tiled() != nullptr;
+bool tc_format(const QuantArgs& a) {
+  return a.prod ? (!a.mixed && a.mse_bits >= 0 && a.mse_bits <= 3)
+                : (a.mse_bits >= 1 && (a.mixed ? (a.mse_bits == 2 || a.mse_bits == 3)
+                                               : (a.mse_bits <= 4 || a.mse_bits == kWideBits)));
 }
 
-tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(a.n)};
+// bf16 rows: tensor-core rotation (MSE 1..4 and 8 bits, mixed 2.5 and 3.5, prod 1..4).
+bool tc_eligible(const QuantArgs& a) {
+  return a.x_bf16 && tc_format(a) && a.n <= (int64_t(1) << 31) &&
+         (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
+         (a.planes < 2 || (reinterpret_cast<uintptr_t>(a.x2) & 15) == 0) && encode_tiled() != nullptr;
+}
+
+// The grid run_quantize launches for a (the CTAs an append's length update
+// counts).
+int64_t quantize_grid(const QuantArgs& a) {
+  if (a.n <= 0) return 0;
+  if (tc_eligible(a)) return std::min<int64_t>(((a.n + kTcRows - 1) / kTcRows) * a.planes, num_sms());
+  if (a.mse_bits == kWideBits) return std::min<int64_t>(a.n, 64LL * num_sms());
+  return std::min<int64_t>((a.n + kTile - 1) / kTile, num_sms());
+}
+
+bool encode_rows(CUtensorMap* map, const void* x, int64_t n) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(n)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim) * 2};
   const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTcRows)};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = encode_tiled()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dims, strides,
-                                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
-  const int64_t tiles = (a.n + kTcRows - 1) / kTcRows;
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  return encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
+  CUtensorMap maps[2];
+  if (!encode_rows(&maps[0], a.x, a.n)) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
+  if (a.planes > 1) {
+    if (!encode_rows(&maps[1], a.x2, a.n)) return fail(TQ_ERR_CUDA, "tq_append: cuTensorMapEncodeTiled failed");
+  } else {
+    maps[1] = maps[0];
+  }
+  const int grid = static_cast<int>(quantize_grid(a));
   if (a.prod) {
     switch (a.mse_bits) {
-      case 0: return launch_tc_prod<0>(a, map, grid, st);
-      case 1: return launch_tc_prod<1>(a, map, grid, st);
-      case 2: return launch_tc_prod<2>(a, map, grid, st);
-      case 3: return launch_tc_prod<3>(a, map, grid, st);
+      case 0: return launch_tc_prod<0>(a, maps, grid, st);
+      case 1: return launch_tc_prod<1>(a, maps, grid, st);
+      case 2: return launch_tc_prod<2>(a, maps, grid, st);
+      case 3: return launch_tc_prod<3>(a, maps, grid, st);
       default: return fail(TQ_ERR_UNSUPPORTED, "tq_quantize: no tensor-core kernel for this format");
     }
   }
   switch (a.mse_bits * 2 + a.mixed) {
-    case 2: return launch_tc<1, 0>(a, map, grid, st);
-    case 4: return launch_tc<2, 0>(a, map, grid, st);
-    case 5: return launch_tc<2, 1>(a, map, grid, st);
-    case 6: return launch_tc<3, 0>(a, map, grid, st);
-    case 7: return launch_tc<3, 1>(a, map, grid, st);
-    case 8: return launch_tc<4, 0>(a, map, grid, st);
+    case 2: return launch_tc<1, 0>(a, maps, grid, st);
+    case 4: return launch_tc<2, 0>(a, maps, grid, st);
+    case 5: return launch_tc<2, 1>(a, maps, grid, st);
+    case 6: return launch_tc<3, 0>(a, maps, grid, st);
+    case 7: return launch_tc<3, 1>(a, maps, grid, st);
+    case 8: return launch_tc<4, 0>(a, maps, grid, st);
+    case 16: return launch_tc<kWideBits, 0>(a, maps, grid, st);
     default: return fail(TQ_ERR_UNSUPPORTED, "tq_quantize: no tensor-core kernel for this format");
   }
 }
 
+// Launches the quantize kernel for a (a.planes == 2 only where tc_eligible).
 tq_status run_quantize(QuantArgs& a, cudaStream_t st) {
   if (a.n <= 0) return TQ_OK;
   if (tc_eligible(a)) return run_quantize_tc(a, st);
+  if (a.planes != 1) return fail(TQ_ERR_UNSUPPORTED, "two-plane quantize needs the tensor-core kernels");
+  const int64_t grid = quantize_grid(a);
+  if (a.mse_bits == kWideBits) {
+    quantize8_kernel<<<static_cast<unsigned>(grid), kDim, 0, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "8-bit quantize kernel launch");
+  }
   const size_t smem = quant_smem(a.prod);
-  const int64_t tiles = (a.n + kTile - 1) / kTile;
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   cudaError_t e;
   if (a.x_bf16) {
     e = ensure_dyn_smem<quantize_kernel<1>>(static_cast<int>(smem));
@@ -1290,6 +1492,10 @@ void fill_format(QuantArgs& a, const tq_params* p, const FormatSpec& f) {
   a.tc_img = p->tc_img;
   a.cb = p->cb32;
   a.bd = p->bd32;
+  a.cell8 = p->cell8;
+  a.cell8_n = p->cell8_n;
+  a.cell8_inv_w = p->cell8_inv_w;
+  a.pit64 = p->pit64;
 }
 
 }  // namespace
@@ -1298,6 +1504,7 @@ tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x
                           const tq_packed* out, cudaStream_t st) {
   QuantArgs a{};
   fill_format(a, p, f);
+  a.planes = 1;
   a.x = x;
   a.x_bf16 = x_bf16;
   a.n = n;
@@ -1349,17 +1556,13 @@ tq_status side_stream(SideStream** out) {
 tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* seq_ids, const void* k,
                         const void* v, int x_bf16, int n_tok, int n_seq, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(n_seq) * n_tok * c->n_kv_heads;
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  SideStream* side = nullptr;
-  tq_status sst = side_stream(&side);
-  if (sst != TQ_OK) return sst;
-  cudaError_t fe = cudaEventRecord(side->fork, st);
-  if (fe == cudaSuccess) fe = cudaStreamWaitEvent(side->stream, side->fork, 0);
-  if (fe != cudaSuccess) return cuda_fail(fe, "tq_append: fork");
+  QuantArgs q[2];
   for (int which = 0; which < 2; ++which) {
     const FormatSpec& f = which ? p->fv : p->fk;
-    QuantArgs a{};
+    QuantArgs& a = q[which];
+    a = QuantArgs{};
     fill_format(a, p, f);
+    a.planes = 1;
     a.x = which ? v : k;
     a.x_bf16 = x_bf16;
     a.n = n;
@@ -1378,20 +1581,44 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
     a.cache_seqs = c->n_seq;
     a.sink = which ? c->v_sink : c->k_sink;
     a.status = c->status;
-    tq_status s = run_quantize(a, which ? side->stream : st);
-    if (s != TQ_OK) {
-      // keep the side stream joined to the caller's stream even on failure
-      if (cudaEventRecord(side->join, side->stream) == cudaSuccess) cudaStreamWaitEvent(st, side->join, 0);
-      return s;
-    }
+    a.n_seq_in = n_seq;
   }
+  // equal K and V formats on the tensor-core kernels: one launch for both
+  QuantArgs both = q[0];
+  both.planes = 2;
+  both.x2 = v;
+  both.codes2 = c->v_codes;
+  both.norms2 = c->v_norms;
+  both.qjl2 = c->v_qjl;
+  both.res2 = c->v_res_norms;
+  both.sink2 = c->v_sink;
+  if (p->fk.id() == p->fv.id() && tc_eligible(both)) {
+    both.arrive_total = static_cast<int>(quantize_grid(both));
+    return run_quantize(both, st);
+  }
+  // otherwise K on the caller's stream and V on a side stream, concurrently;
+  // the last CTA of either kernel updates the lengths
+  const int64_t g0 = quantize_grid(q[0]), total = g0 + quantize_grid(q[1]);
+  if (total > 0xFFFF) return fail(TQ_ERR_UNSUPPORTED, "tq_append: too many CTAs for the length update");
+  q[0].arrive_total = q[1].arrive_total = static_cast<int>(total);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* side = nullptr;
+  tq_status sst = side_stream(&side);
+  if (sst != TQ_OK) return sst;
+  cudaError_t fe = cudaEventRecord(side->fork, st);
+  if (fe == cudaSuccess) fe = cudaStreamWaitEvent(side->stream, side->fork, 0);
+  if (fe != cudaSuccess) return cuda_fail(fe, "tq_append: fork");
+  tq_status s = run_quantize(q[0], st);
+  if (s == TQ_OK) {
+    s = run_quantize(q[1], side->stream);
+    // K's CTAs are counting already: arrive for the values' kernel
+    if (s != TQ_OK) append_arrive_kernel<<<1, 128, 0, st>>>(q[0], static_cast<int>(total - g0));
+  }
+  // the side stream is joined to the caller's stream even on failure
   fe = cudaEventRecord(side->join, side->stream);
   if (fe == cudaSuccess) fe = cudaStreamWaitEvent(st, side->join, 0);
-  if (fe != cudaSuccess) return cuda_fail(fe, "tq_append: join");
-  bump_lens_kernel<<<(n_seq + 127) / 128, 128, 0, st>>>(seq_ids, c->lens, c->status, n_seq, n_tok,
-                                                        c->n_sink + c->capacity, c->n_seq);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "append length update");
+  if (s != TQ_OK) return s;
+  return fe == cudaSuccess ? TQ_OK : cuda_fail(fe, "tq_append: join");
 }
 
 tq_status launch_cache_rows(const tq_params* p, const tq_cache* c, int which, int seq, int kv_head, int row0,
@@ -1416,7 +1643,7 @@ tq_status launch_dequantize(const tq_params* p, const FormatSpec& f, const tq_pa
   if (blocks > 0x7fffffff) return fail(TQ_ERR_UNSUPPORTED, "tq_dequantize: n too large");
   dequantize_kernel<<<static_cast<unsigned>(blocks), kDim, 0, st>>>(
       in->codes, in->norms, in->qjl, in->res_norms, n, f.mse_bits, f.mixed, f.prod, f.code_bytes, p->pi64,
-      p->s64, p->cb64, out);
+      p->s64, p->cb64, p->cb8_64, out);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "dequantize kernel launch");
 }

@@ -66,6 +66,13 @@ def test_host_argument_errors():
     with pytest.raises(tq.TqError) as e:
         tq.Params(5, 3)
     assert e.value.status == 2
+    for bad in (dict(bits_k=6), dict(bits_k=8, mode_k=tq.TQ_MODE_PROD), dict(bits_k=8, mixed_k=1)):
+        # 8-bit codes: MSE mode, uniform rows only
+        args = dict(bits_k=3, bits_v=3)
+        args.update(bad)
+        with pytest.raises(tq.TqError) as e:
+            tq.Params(args.pop("bits_k"), args.pop("bits_v"), **args)
+        assert e.value.status == 2, bad
     with pytest.raises(tq.TqError) as e:
         tq.Params(3, 3, mixed_k=1, mode_k=tq.TQ_MODE_PROD)
     assert e.value.status == 2

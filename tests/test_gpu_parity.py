@@ -142,8 +142,10 @@ DECODE_FORMATS = [
     (gu.fmt(2, prod=True), gu.fmt(2, prod=True)),
     (gu.fmt(4, prod=True), gu.fmt(4, prod=True)),
     (gu.fmt(1, prod=True), gu.fmt(1, prod=True)),
+    (gu.fmt(8), gu.fmt(3)),
 ]
-DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "k3v2", "k4v2", "mixed", "mixed2.5", "prod3", "prod2", "prod4", "prod1"]
+DEC_IDS = ["k3v3", "k4v3", "k4v4", "k2v2", "k1v1", "k3v2", "k4v2", "mixed", "mixed2.5", "prod3", "prod2", "prod4", "prod1",
+           "k8v3"]
 
 
 @pytest.mark.parametrize("fk,fv", DECODE_FORMATS, ids=DEC_IDS)
@@ -202,8 +204,9 @@ def test_decode_length_above_bound_sets_status():
 
 @pytest.mark.parametrize("fk,fv,n_sink", [(gu.fmt(4), gu.fmt(3), 8), (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True), 0),
                                           (gu.fmt(2, mixed=True), gu.fmt(2, mixed=True), 4),
-                                          (gu.fmt(3, prod=True), gu.fmt(3, prod=True), 0)],
-                         ids=["k4v3sink", "mixed", "mixed2.5sink", "prod3"])
+                                          (gu.fmt(3, prod=True), gu.fmt(3, prod=True), 0),
+                                          (gu.fmt(8), gu.fmt(3), 8)],
+                         ids=["k4v3sink", "mixed", "mixed2.5sink", "prod3", "k8v3sink"])
 def test_append_parity(fk, fv, n_sink):
     gp, op = gu.make_params(fk, fv)
     n_seq, hkv, cap = 3, 2, 256
@@ -268,11 +271,11 @@ def test_gpu_built_cache_attention_matches_oracle_built():
 
 
 GQA_FORMATS = [(gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)), (gu.fmt(4), gu.fmt(3)),
-               (gu.fmt(3, prod=True), gu.fmt(3, prod=True)), (gu.fmt(1), gu.fmt(1))]
+               (gu.fmt(3, prod=True), gu.fmt(3, prod=True)), (gu.fmt(1), gu.fmt(1)), (gu.fmt(8), gu.fmt(3))]
 
 
 @pytest.mark.parametrize("group", [1, 2, 3, 5, 6, 7, 8])
-@pytest.mark.parametrize("fk,fv", GQA_FORMATS, ids=["mixed", "k4v3", "prod3", "k1v1"])
+@pytest.mark.parametrize("fk,fv", GQA_FORMATS, ids=["mixed", "k4v3", "prod3", "k1v1", "k8v3"])
 def test_decode_parity_gqa_groups(fk, fv, group):
     """Every query-head group size the boundary accepts: groups of up to 4 pack
     the query's high and low halves into spare MMA columns (3 leaves two of the
@@ -335,21 +338,22 @@ def test_decode_sparse_v_drops_and_matches_oracle(fk, fv, group):
 
 def test_decode_sparse_v_skips_whole_tiles():
     """A value tile's work is skipped only when all its (token, head) weights
-    are dropped.  One unit of 2 x 148 x 480 tokens (two 480-token chunks per
-    CTA of the persistent grid): in even chunks the first token of every
-    32-token warp tile is a strong key (norm 30, cos 0.99 with the query), the
-    rest are ordinary keys, whose scores then sit ~20 below the running
-    maximum.  Every warp meets a strong key before its odd-chunk tiles, which
-    hold ordinary keys only and are skipped; the output matches the oracle's
-    exact rule."""
+    are dropped, and a warp can only tell once it has met a large score.  One
+    unit of 6 x 148 x 480 tokens (several 480-token chunks per CTA of the
+    persistent grid): in every third chunk the first token of every 32-token
+    tile is a strong key (norm 30, cos 0.99 with the query); the rest are
+    ordinary keys, whose scores sit ~20 below.  Warps meet a strong key early in
+    their range and then skip the tiles of ordinary keys after it, whatever
+    the exact chunk ranges of the CTAs; the output matches the oracle's exact
+    rule."""
     fk, fv = gu.fmt(4), gu.fmt(3)
     gp, op = gu.make_params(fk, fv)
-    T, thr = 2 * 148 * 480, 1e-6
+    T, thr = 6 * 148 * 480, 1e-6
     q = kv_inputs.queries((1, 1, 128), key=("skip", "q"), dtype=torch.float32)
     k = kv_inputs.kv_vectors(T, 128, key=("skip", "k"), dtype=torch.float32)
     v = kv_inputs.kv_vectors(T, 128, key=("skip", "v"), dtype=torch.float32)
     pos = np.arange(T)
-    strong = ((pos // 480) % 2 == 0) & (pos % 32 == 0)
+    strong = ((pos // 480) % 3 == 0) & (pos % 32 == 0)
     qh = q[0, 0] / q[0, 0].norm()
     w = kv_inputs.kv_vectors(int(strong.sum()), 128, key=("skip", "w"), dtype=torch.float32)
     w = w - (w @ qh)[:, None] * qh[None]
@@ -371,7 +375,7 @@ def test_decode_sparse_v_skips_whole_tiles():
     examined, dropped, tiles, skipped = (int(x) for x in stats.cpu())
     print(f"sparse V, planted keys: dropped {dropped}/{examined}, tiles skipped {skipped}/{tiles}")
     assert examined == T and tiles == T // 32
-    assert skipped / tiles > 0.45 and dropped / examined > 0.9
+    assert skipped / tiles > 0.3 and dropped / examined > 0.6
     assert gu.rel_l2(out.float().cpu().numpy(), want) < gu.ATTN_REL_L2
 
 
@@ -418,8 +422,8 @@ def test_config1_tiny_fp32_end_to_end():
 
 
 ALL_CODE_FORMATS = [gu.fmt(1), gu.fmt(2), gu.fmt(3), gu.fmt(4), gu.fmt(3, mixed=True), gu.fmt(2, mixed=True),
-                    gu.fmt(2, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True)]
-ALL_CODE_IDS = ["mse1", "mse2", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod2", "prod3", "prod4"]
+                    gu.fmt(2, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True), gu.fmt(8)]
+ALL_CODE_IDS = ["mse1", "mse2", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod2", "prod3", "prod4", "mse8"]
 
 
 def _tile_spec_offsets(f, side):
@@ -427,17 +431,17 @@ def _tile_spec_offsets(f, side):
     own: for token i (0..15) of a tile, the tile byte of every byte of its
     packed row.  Lane L = 4g + t; a key lane owns tokens g, g + 8 and quarter
     t of each segment, a value lane tokens 2t, 2t+1, 2t+8, 2t+9 and eighth g;
-    lane blocks of code_bytes / 2 bytes are stored as 16-, 16-, 8- and 4-byte
-    columns in that order."""
+    lane blocks of code_bytes / 2 bytes are stored as 16-byte columns while
+    16 bytes remain, then an 8- and a 4-byte column as needed."""
     cb = f.code_bytes(128)
     w = [f.mse_bits(j, 128) for j in range(128)]
     segs = [(0, 64), (64, 128)] if f.mixed else [(0, 128)]
     seg_start = [sum(w[:a]) // 8 for a, _ in segs]
     seg_bytes = [sum(w[a:b]) // 8 for a, b in segs]
     lb = cb // 2
-    cols = []
-    rest = lb
-    for width in (16, 16, 8, 4):
+    cols = [16] * (lb // 16)
+    rest = lb % 16
+    for width in (8, 4):
         if rest >= width:
             cols.append(width)
             rest -= width
@@ -513,8 +517,9 @@ def test_cache_rows_round_trip_and_tile_layout(f, side):
 
 @pytest.mark.parametrize("fk,fv", [(gu.fmt(3, mixed=True), gu.fmt(3, mixed=True)), (gu.fmt(4), gu.fmt(3)),
                                    (gu.fmt(3, prod=True), gu.fmt(3, prod=True)), (gu.fmt(2, mixed=True),
-                                                                                  gu.fmt(2, mixed=True))],
-                         ids=["mixed3.5", "k4v3", "prod3", "mixed2.5"])
+                                                                                  gu.fmt(2, mixed=True)),
+                                   (gu.fmt(8), gu.fmt(3))],
+                         ids=["mixed3.5", "k4v3", "prod3", "mixed2.5", "k8v3"])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 def test_append_rows_equal_quantize_rows(fk, fv, dtype):
     """Appending in ragged 64-token chunks stores, bit for bit, the rows
@@ -543,3 +548,144 @@ def test_append_rows_equal_quantize_rows(fk, fv, dtype):
             assert np.array_equal(got.norms, want.norms)
             if f.prod:
                 assert np.array_equal(got.qjl, want.qjl) and np.array_equal(got.res_norms, want.res_norms)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit codes (256 centroids, one byte per coordinate): the fp32 path rotates
+# in fp64 on the SIMT cores, the bf16 path on the tensor cores with a
+# three-term split of Pi; both search the codebook through uniform cells.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("rotation", ["haar", "hadamard"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_quantize_parity_8bit(dtype, rotation):
+    f = gu.fmt(8)
+    gp, op = gu.make_params(f, gu.fmt(3), seed=5, rotation=rotation)
+    # bf16: several 128-row tiles per CTA of the persistent grid and a ragged
+    # tail; fp32: one vector per block, a ragged count
+    n = 148 * 128 * 3 + 77 if dtype == torch.bfloat16 else 3001
+    x = kv_inputs.kv_vectors(n, 128, key=("q8", rotation), dtype=dtype, outliers=True)
+    x[9] = 0
+    out = tq.Packed.empty(gp, n, tq.TQ_K)
+    tq.tq_quantize(gp, x.cuda(), tq.TQ_K, out)
+    torch.cuda.synchronize()
+    assert gp.status() == 0
+    got = gu.gpu_packed_to_numpy(out)
+    xd = x.double().numpy()
+    want = o.quantize(op, xd, "k")
+    gu.compare_codes(op, f, xd, got, want)
+    assert np.allclose(got.norms, want.norms, rtol=1e-6, atol=0)
+    assert not got.codes[9].any() and got.norms[9] == 0
+    # the levels are reached across the range (all 256 on the larger bf16
+    # set; the outermost few are rare in 3001 vectors)
+    assert len(np.unique(got.codes)) >= (256 if n > 10000 else 248)
+
+
+def test_dequantize_parity_8bit():
+    gp, op = gu.make_params(gu.fmt(8), gu.fmt(3))
+    n = 555
+    x = kv_inputs.kv_vectors(n, 128, key="dq8", dtype=torch.bfloat16, outliers=True)
+    want_pk = o.quantize(op, x.double().numpy(), "k")
+    want = o.dequantize(op, want_pk, "k")
+    out = torch.empty(n, 128, dtype=torch.float32, device="cuda")
+    tq.tq_dequantize(gp, gu.numpy_packed_to_gpu(want_pk), n, tq.TQ_K, out)
+    assert np.max(np.abs(out.cpu().numpy() - want)) <= gu.DEQUANT_ATOL
+
+
+def test_decode_k8v3_beats_k4v3_on_the_same_vectors():
+    """8-bit keys reach the exact (unquantized-key) attention more closely
+    than 4-bit keys over the same values: the decode kernel reads the wider
+    codes without losing what they add."""
+    B, hq, hkv, T = 2, 8, 2, 1500
+    lens = [1500, 1111]
+    k = kv_inputs.kv_vectors(B * hkv * T, 128, key=("k8cmp", "k"), dtype=torch.bfloat16)
+    v = kv_inputs.kv_vectors(B * hkv * T, 128, key=("k8cmp", "v"), dtype=torch.bfloat16)
+    q = kv_inputs.queries((B, hq, 128), key=("k8cmp", "q"))
+    kd = k.double().numpy().reshape(B, hkv, T, 128)
+    vd = v.double().numpy().reshape(B, hkv, T, 128)
+    errs = {}
+    for kb in (4, 8):
+        gp, op = gu.make_params(gu.fmt(kb), gu.fmt(3))
+        ocache = o.cache_from_vectors(op, kd, vd, 0)
+        # exact keys, the values as quantized: isolates the keys' error
+        exact = np.zeros((B, hq, 128))
+        group = hq // hkv
+        for b in range(B):
+            for h in range(hq):
+                kvh = h // group
+                vr = ocache.v_rows[b, kvh]
+                n = lens[b]
+                vals = o.dequantize(op, o.Packed(vr.codes[:n], vr.norms[:n], vr.qjl[:n], vr.res_norms[:n]), "v")
+                s = kd[b, kvh, :n] @ q[b, h].double().numpy() / math.sqrt(128)
+                w = np.exp(s - s.max())
+                exact[b, h] = (w / w.sum()) @ vals
+        cache = tq.Cache(gp, B, hkv, ((T + 63) // 64) * 64, 0)
+        gu.fill_cache_from_oracle(cache, op, ocache, lens, B, hkv)
+        ws = tq.decode_workspace(gp, B, hq, hkv, T)
+        out = torch.empty(B, hq, 128, dtype=torch.float32, device="cuda")
+        tq.tq_decode_attn(gp, q.cuda(), cache, T, out, ws)
+        torch.cuda.synchronize()
+        errs[kb] = gu.rel_l2(out.cpu().numpy(), exact)
+    print(f"rel L2 vs exact keys: K4 {errs[4]:.3e}  K8 {errs[8]:.3e}")
+    assert errs[8] < 0.25 * errs[4]
+
+
+@pytest.mark.parametrize("fk,fv,dtype", [(gu.fmt(3, mixed=True), gu.fmt(3, mixed=True), torch.bfloat16),
+                                         (gu.fmt(3, prod=True), gu.fmt(3, prod=True), torch.bfloat16),
+                                         (gu.fmt(4), gu.fmt(3), torch.bfloat16),
+                                         (gu.fmt(3, mixed=True), gu.fmt(3, mixed=True), torch.float32),
+                                         (gu.fmt(8), gu.fmt(3), torch.float32)],
+                         ids=["mixed-one-launch", "prod3-one-launch", "k4v3-two-kernels", "mixed-f32", "k8v3-f32"])
+def test_append_length_update_folded(fk, fv, dtype):
+    """The last CTA of an append updates lens (no separate launch): ragged
+    appends to shuffled subsets of the sequences leave every length exact,
+    the stored rows equal to tq_quantize's, and the status word (the CTA count
+    in its high half included) back at zero; an append that does not fit
+    leaves its sequence's length alone and sets bit 1 only."""
+    gp, _ = gu.make_params(fk, fv)
+    n_seq, hkv, cap, n_sink = 5, 2, 512, 4
+    cache = tq.Cache(gp, n_seq, hkv, cap, n_sink)
+    rng = np.random.default_rng(31)
+    expect = [0] * n_seq
+    held = {s: [] for s in range(n_seq)}  # (k, v) chunks per sequence, in order
+    for step in range(12):
+        n_tok = int(rng.integers(1, 41))
+        seqs = [int(s) for s in rng.permutation(n_seq)[:int(rng.integers(1, n_seq + 1))]]
+        k = kv_inputs.kv_vectors(len(seqs) * n_tok * hkv, 128, key=("fold", "k", step), dtype=dtype)
+        v = kv_inputs.kv_vectors(len(seqs) * n_tok * hkv, 128, key=("fold", "v", step), dtype=dtype)
+        k = k.view(len(seqs), n_tok, hkv, 128)
+        v = v.view(len(seqs), n_tok, hkv, 128)
+        tq.tq_append(gp, cache, torch.tensor(seqs, dtype=torch.int32, device="cuda"), k.cuda(), v.cuda())
+        for i, s in enumerate(seqs):
+            expect[s] += n_tok
+            held[s].append((k[i], v[i]))
+        torch.cuda.synchronize()
+        assert cache.lens.cpu().tolist() == expect, step
+        assert int(cache.status.item()) == 0, step
+    # the quantized rows of two sequences against tq_quantize of the same vectors
+    for s in (0, 3):
+        if expect[s] <= n_sink:
+            continue
+        for side, which, f in (("k", tq.TQ_K, fk), ("v", tq.TQ_V, fv)):
+            x = torch.cat([kv[0 if side == "k" else 1] for kv in held[s]], 0)  # (len, hkv, d)
+            for h in range(hkv):
+                xs = x[n_sink:, h].contiguous().cuda()
+                ref = tq.Packed.empty(gp, xs.shape[0], which)
+                tq.tq_quantize(gp, xs, which, ref)
+                torch.cuda.synchronize()
+                want = gu.gpu_packed_to_numpy(ref)
+                got = gu.read_unit_rows(cache, f, side, s, h, 0, xs.shape[0])
+                assert np.array_equal(got.codes, want.codes), (s, side, h)
+                assert np.array_equal(got.norms, want.norms)
+    # refused: neither sequence 2 nor 4 can take 600 more tokens; then 8 fit
+    big = kv_inputs.kv_vectors(2 * 600 * hkv, 128, key="fold-big", dtype=dtype).view(2, 600, hkv, 128)
+    seqs = torch.tensor([2, 4], dtype=torch.int32, device="cuda")
+    tq.tq_append(gp, cache, seqs, big.cuda(), big.cuda())
+    torch.cuda.synchronize()
+    assert cache.lens.cpu().tolist() == expect
+    assert int(cache.status.item()) == 1
+    small = big[:, :8].contiguous().cuda()
+    cache.status.zero_()
+    tq.tq_append(gp, cache, torch.tensor([4], dtype=torch.int32, device="cuda"), small[:1], small[:1])
+    torch.cuda.synchronize()
+    expect[4] += 8
+    assert cache.lens.cpu().tolist() == expect and int(cache.status.item()) == 0
