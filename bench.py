@@ -473,6 +473,19 @@ def _aux_k4v3(tq, torch, kv_inputs, device, flush, iters):
     out["decode_k4v3_sink_T128k_sparse_v"].update(
         {"weights_dropped": round(dropped / max(examined, 1), 4), "tiles_skipped": round(skipped / max(tiles, 1), 4),
          "weights_examined": examined, "tiles_examined": tiles})
+    # the same cache with peaked queries (x 8): where whole tiles fall below
+    # the threshold for every head of the group, sparse V skips their values
+    qp = q * 8
+    for thr, name in ((1e-6, "sparse_v"), (0.0, "dense")):
+        ms = _time_call(torch, lambda: tq.tq_decode_attn(p, qp, cache, T, o, ws, thr), iters, flush)
+        by = 4 * 8 * ((T - 128) * (68 + 52) + 128 * 512)
+        out[f"decode_k4v3_sink_T128k_peaked_{name}"] = {"ms": round(ms, 4),
+                                                        "gb_per_s_dense_equiv": round(by / (ms * 1e-3) / 1e9, 1)}
+    stats.zero_()
+    tq.tq_decode_attn(p, qp, cache, T, o, ws, 1e-6, sparse_v_stats=stats)
+    examined, dropped, tiles, skipped = (int(x) for x in stats.cpu())
+    out["decode_k4v3_sink_T128k_peaked_sparse_v"].update(
+        {"weights_dropped": round(dropped / max(examined, 1), 4), "tiles_skipped": round(skipped / max(tiles, 1), 4)})
     assert int(cache.status.item()) == 0
     return out
 

@@ -188,12 +188,18 @@ __device__ __forceinline__ void compute_tile(const UnitPlanes& u, int srow, int 
     // Sparse V ("Greetings from TurboQuant-MLX", item 3): the value of a token
     // whose weight is below thr is left out (the denominator keeps it).  The
     // final weight is exp(s - M) / L with M, L the max and sum over all the
-    // unit's tokens; exp(s - m) / l_w with m, l_w this warp's running max and
-    // sum is never below it, and l_w is at least this lane's partial sum and
-    // at least 1 (the token at the running max counts exp(0)).  So a weight
-    // below thr * max(l_lane, 1) is below thr in the end: no token the exact
-    // rule keeps is dropped.
-    const float c0 = thr * fmaxf(W.l0, 1.f), c1 = thr * fmaxf(W.l1, 1.f);
+    // unit's tokens; exp(s - m) / l_c with m this warp's running max and l_c
+    // the sum over the tokens this warp's column has seen (the eight lanes'
+    // partial sums) is never below it, and l_c >= 1 (the token at the running
+    // max counts exp(0)).  So a weight below thr * max(l_c, 1) is below thr in
+    // the end: no token the exact rule keeps is dropped.
+    float lc0 = W.l0, lc1 = W.l1;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      lc0 += __shfl_xor_sync(0xffffffffu, lc0, off);
+      lc1 += __shfl_xor_sync(0xffffffffu, lc1, off);
+    }
+    const float c0 = thr * fmaxf(lc0, 1.f), c1 = thr * fmaxf(lc1, 1.f);
     const bool col0 = 2 * t < group, col1 = 2 * t + 1 < group;  // real heads (packed: the hi columns)
     const bool okr[4] = {ok0A, ok0B, ok1A, ok1B};
     float* pp[4] = {&p0[0], &p0[2], &p1[0], &p1[2]};
@@ -251,9 +257,11 @@ struct UnitInfo {
   int len, ns, nq, chunks, slack, slots;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u, int kChunk) {
+// lens: the cache's lengths (global), or the decode kernel's copy of them in
+// shared memory.
+__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, const int* lens, int u, int kChunk) {
   const int b = u / a.hkv;
-  const int len = min(max(a.lens[b], 0), a.max_len);
+  const int len = min(max(lens[b], 0), a.max_len);
   UnitInfo r;
   r.len = len;
   r.ns = min(a.n_sink, len);
@@ -266,8 +274,8 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, int u, int kC
 
 
 // Slots of each kv-head unit of sequence b (all units of a sequence are alike).
-__device__ __forceinline__ int seq_slots(const DecodeArgs& a, int b, int kChunk) {
-  const int len = min(max(a.lens[b], 0), a.max_len);
+__device__ __forceinline__ int seq_slots(const DecodeArgs& a, const int* lens, int b, int kChunk) {
+  const int len = min(max(lens[b], 0), a.max_len);
   const int ch = (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
   return ch > 0 ? ch + a.unit_slack : 0;
 }
@@ -428,29 +436,31 @@ inline int merge_chunk_pieces(int group, int part_floats) {
   const size_t per = static_cast<size_t>(group) * part_floats * sizeof(float);
   return static_cast<int>(std::max<size_t>(1, kMergeStageBytes / per));
 }
-inline size_t merge_dyn_bytes(int n_sink, int ctas, int group, int part_floats) {
-  return (static_cast<size_t>(n_sink) + 2 * static_cast<size_t>(ctas)) * kMaxG * sizeof(float) +
+inline size_t merge_dyn_bytes(int n_sink, int ctas, int group, int part_floats, int mh) {
+  return (static_cast<size_t>(n_sink) + 2 * static_cast<size_t>(ctas)) * mh * sizeof(float) +
          static_cast<size_t>(merge_chunk_pieces(group, part_floats)) * group * part_floats * sizeof(float);
 }
 
-template <int VF>
+// MH: heads per CTA the kernel is compiled for (1, 4 or 8; a.merge_heads <= MH).
+template <int VF, int MH>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
+  static_assert(MH == 1 || MH == 4 || MH == 8, "heads per merge CTA");
   using FV = Fmt<VF>;
   constexpr int NT = kMergeThreads;
   constexpr int WD = FV::prod ? 2 * kDim : kDim;  // accumulator: rotated | sketch
   constexpr int NS = NT / WD;                     // piece slices of the accumulation
   constexpr int RS = WD / 4;                      // matrix rows per un-rotation slice
   extern __shared__ float4 s_dyn4[];
-  __shared__ float s_red[4 * kMaxG * kDim];       // slice partials
-  __shared__ __align__(16) float s_acc[WD][kMaxG];  // merged accumulator, [j][head]
-  __shared__ float s_osk[kMaxG][kDim];            // sink values, original domain
-  __shared__ float s_q[kMaxG][4][33];  // query quarters, padded: the four quarters sit in different banks
-  __shared__ float s_ms[kMaxG], s_ls[kMaxG], s_M[kMaxG], s_L[kMaxG];
+  __shared__ float s_red[4 * MH * kDim];       // slice partials
+  __shared__ __align__(16) float s_acc[WD][MH];  // merged accumulator, [j][head]
+  __shared__ float s_osk[MH][kDim];            // sink values, original domain
+  __shared__ float s_q[MH][4][33];  // query quarters, padded: the four quarters sit in different banks
+  __shared__ float s_ms[MH], s_ls[MH], s_M[MH], s_L[MH];
   __shared__ long long s_C, s_cu0;
-  float* s_sc = reinterpret_cast<float*>(s_dyn4);  // [n_sink][8]
-  float* s_f = s_sc + a.n_sink * kMaxG;             // [pieces][8]: maxima, then weights
-  float* s_l = s_f + a.ctas * kMaxG;                // [pieces][8]: sums
-  float* s_part = s_l + a.ctas * kMaxG;             // staged pieces [merge_chunk][G][part_floats]
+  float* s_sc = reinterpret_cast<float*>(s_dyn4);  // [n_sink][MH]
+  float* s_f = s_sc + a.n_sink * MH;             // [pieces][MH]: maxima, then weights
+  float* s_l = s_f + a.ctas * MH;                // [pieces][MH]: sums
+  float* s_part = s_l + a.ctas * MH;             // staged pieces [merge_chunk][G][part_floats]
   const int u = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.merge_heads, h0 = blockIdx.y * G;  // this CTA's heads: h0 .. h0 + G - 1 of the group
@@ -458,7 +468,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   const int b = u / a.hkv, kvh = u % a.hkv;
   // head h0 of the unit's group
   const int64_t orow = (static_cast<int64_t>(b) * a.hq + kvh * a.group + h0) * kDim;
-  const UnitInfo ui = unit_info(a, u, CH);
+  const UnitInfo ui = unit_info(a, a.lens, u, CH);
   if (ui.len == 0) {
     for (int i = tid; i < G * kDim; i += NT) store_out(a, orow + i, 0.f);
     return;
@@ -478,7 +488,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   if (warp == 0 && ui.chunks > 0) {
     long long tot = 0, before = 0;
     for (int v = lane; v < a.B; v += 32) {
-      const int ch = seq_slots(a, v, CH);
+      const int ch = seq_slots(a, a.lens, v, CH);
       tot += ch;
       if (v < b) before += ch;
     }
@@ -494,7 +504,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   }
   // sink: scores with the original query, softmax weights, weighted values
   if (ui.ns > 0) {
-    for (int i = tid; i < kMaxG * kDim; i += NT)
+    for (int i = tid; i < MH * kDim; i += NT)
       s_q[i / kDim][(i % kDim) >> 5][i & 31] = i < G * kDim ? load_q(a.q, a.q_bf16, orow + i) : 0.f;
     __syncthreads();
     // sink rows are staged through shared memory (the piece staging buffer,
@@ -518,9 +528,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       // head, then added across the four quarters (adjacent lanes)
       for (int tb = 0; tb < cnt; tb += NT / 4) {
         const int tt = tb + (tid >> 2), qtr = tid & 3;
-        float d[kMaxG];
+        float d[MH];
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) d[h] = 0.f;
+        for (int h = 0; h < MH; ++h) d[h] = 0.f;
         if (tt < cnt) {
           const uint4* kr = reinterpret_cast<const uint4*>(srow + tt * kDim + 32 * qtr);
 #pragma unroll
@@ -532,31 +542,31 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
               const float k0 = __uint_as_float(w4[e] << 16), k1 = __uint_as_float(w4[e] & 0xFFFF0000u);
               const int j = 8 * c + 2 * e;
 #pragma unroll
-              for (int h = 0; h < kMaxG; ++h) d[h] = fmaf(k1, s_q[h][qtr][j + 1], fmaf(k0, s_q[h][qtr][j], d[h]));
+              for (int h = 0; h < MH; ++h) d[h] = fmaf(k1, s_q[h][qtr][j + 1], fmaf(k0, s_q[h][qtr][j], d[h]));
             }
           }
         }
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
+        for (int h = 0; h < MH; ++h) {
           d[h] += __shfl_xor_sync(0xffffffffu, d[h], 1);
           d[h] += __shfl_xor_sync(0xffffffffu, d[h], 2);
         }
         if (tt < cnt && qtr == 0)
 #pragma unroll
-          for (int h = 0; h < kMaxG; ++h)
-            if (h < G) s_sc[(c0 + tt) * kMaxG + h] = d[h] * scale;
+          for (int h = 0; h < MH; ++h)
+            if (h < G) s_sc[(c0 + tt) * MH + h] = d[h] * scale;
       }
       __syncthreads();  // the staging buffer is refilled
     }
     if (warp < G) {  // warp h: max, weights and sum of head h
       const int h = warp;
       float mx = -INFINITY;
-      for (int tt = lane; tt < ui.ns; tt += 32) mx = fmaxf(mx, s_sc[tt * kMaxG + h]);
+      for (int tt = lane; tt < ui.ns; tt += 32) mx = fmaxf(mx, s_sc[tt * MH + h]);
       mx = warp_max(mx);
       float sum = 0.f;
       for (int tt = lane; tt < ui.ns; tt += 32) {
-        const float pw = exp2f(s_sc[tt * kMaxG + h] - mx);
-        s_sc[tt * kMaxG + h] = pw;
+        const float pw = exp2f(s_sc[tt * MH + h] - mx);
+        s_sc[tt * MH + h] = pw;
         sum += pw;
       }
       sum = warp_sum(sum);
@@ -567,36 +577,39 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     }
     __syncthreads();
     {
-      float acc[kMaxG];
+      float acc[MH];
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+      for (int h = 0; h < MH; ++h) acc[h] = 0.f;
       for (int c0 = 0; c0 < ui.ns; c0 += SC) {
         const int cnt = min(SC, ui.ns - c0);
         stage_rows(vs, c0, cnt);
         for (int tt = sl4; tt < cnt; tt += 4) {
           const float v = __bfloat162float(srow[tt * kDim + o]);
-          const float4 p0 = s_dyn4[(c0 + tt) * 2], p1 = s_dyn4[(c0 + tt) * 2 + 1];
-          acc[0] = fmaf(p0.x, v, acc[0]);
-          acc[1] = fmaf(p0.y, v, acc[1]);
-          acc[2] = fmaf(p0.z, v, acc[2]);
-          acc[3] = fmaf(p0.w, v, acc[3]);
-          acc[4] = fmaf(p1.x, v, acc[4]);
-          acc[5] = fmaf(p1.y, v, acc[5]);
-          acc[6] = fmaf(p1.z, v, acc[6]);
-          acc[7] = fmaf(p1.w, v, acc[7]);
+          if constexpr (MH == 1) {
+            acc[0] = fmaf(s_sc[c0 + tt], v, acc[0]);
+          } else {
+#pragma unroll
+            for (int q4 = 0; q4 < MH / 4; ++q4) {
+              const float4 pw = s_dyn4[(c0 + tt) * (MH / 4) + q4];
+              acc[4 * q4] = fmaf(pw.x, v, acc[4 * q4]);
+              acc[4 * q4 + 1] = fmaf(pw.y, v, acc[4 * q4 + 1]);
+              acc[4 * q4 + 2] = fmaf(pw.z, v, acc[4 * q4 + 2]);
+              acc[4 * q4 + 3] = fmaf(pw.w, v, acc[4 * q4 + 3]);
+            }
+          }
         }
         __syncthreads();  // the staging buffer is refilled
       }
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) s_red[(sl4 * kMaxG + h) * kDim + o] = acc[h];
+      for (int h = 0; h < MH; ++h) s_red[(sl4 * MH + h) * kDim + o] = acc[h];
     }
     __syncthreads();
     for (int i = tid; i < G * kDim; i += NT) {
       const int h = i / kDim, j = i % kDim;
-      s_osk[h][j] = s_red[(0 * kMaxG + h) * kDim + j] + s_red[(1 * kMaxG + h) * kDim + j] +
-                    s_red[(2 * kMaxG + h) * kDim + j] + s_red[(3 * kMaxG + h) * kDim + j];
+      s_osk[h][j] = s_red[(0 * MH + h) * kDim + j] + s_red[(1 * MH + h) * kDim + j] +
+                    s_red[(2 * MH + h) * kDim + j] + s_red[(3 * MH + h) * kDim + j];
     }
-  } else if (tid < kMaxG) {
+  } else if (tid < MH) {
     s_ms[tid] = -INFINITY;
     s_ls[tid] = 0.f;
   }
@@ -621,21 +634,21 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       m = __ldcg(pp);
       l = __ldcg(pp + 1);
     }
-    s_f[i * kMaxG + h] = m;
-    s_l[i * kMaxG + h] = l;
+    s_f[i * MH + h] = m;
+    s_l[i * MH + h] = l;
   }
   __syncthreads();
   if (warp < G) {  // warp h: merged maximum, the pieces' weights and the sum for head h
     const int h = warp;
     float M = s_ms[h];
-    for (int i = lane; i < n_p; i += 32) M = fmaxf(M, s_f[i * kMaxG + h]);
+    for (int i = lane; i < n_p; i += 32) M = fmaxf(M, s_f[i * MH + h]);
     M = warp_max(M);
     float L = 0.f;
     for (int i = lane; i < n_p; i += 32) {
-      const float m = s_f[i * kMaxG + h];
+      const float m = s_f[i * MH + h];
       const float f = m > -INFINITY ? exp2f(m - M) : 0.f;
-      L = fmaf(s_l[i * kMaxG + h], f, L);
-      s_f[i * kMaxG + h] = f;
+      L = fmaf(s_l[i * MH + h], f, L);
+      s_f[i * MH + h] = f;
     }
     L = warp_sum(L);
     if (lane == 0) {
@@ -650,9 +663,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       // the accumulators: consecutive slots, staged chunk by chunk with
       // 16-byte asynchronous copies
       const int j = tid % WD, sl = tid / WD;
-      float acc[kMaxG];
+      float acc[MH];
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+      for (int h = 0; h < MH; ++h) acc[h] = 0.f;
       // this CTA's heads of each piece: G x PF consecutive floats at head h0
       const int slot_floats = G * PF, per4 = slot_floats / 4;
       for (int c0 = 0; c0 < n_p; c0 += a.merge_chunk) {
@@ -668,56 +681,59 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
         for (int i = sl; i < cnt; i += NS) {
           const float* pp = s_part + i * slot_floats + kPartAcc + j;
 #pragma unroll
-          for (int h = 0; h < kMaxG; ++h) {
+          for (int h = 0; h < MH; ++h) {
             // weight 0: a piece of a CTA with an empty range, whose slot was
             // not written in this call
-            const float f = h < G ? s_f[(c0 + i) * kMaxG + h] : 0.f;
+            const float f = h < G ? s_f[(c0 + i) * MH + h] : 0.f;
             if (f != 0.f) acc[h] = fmaf(pp[h * PF], f, acc[h]);
           }
         }
         __syncthreads();  // the staging buffer is refilled
       }
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) s_red[(sl * kMaxG + h) * WD + j] = acc[h];
+      for (int h = 0; h < MH; ++h) s_red[(sl * MH + h) * WD + j] = acc[h];
     }
     __syncthreads();
-    for (int i = tid; i < kMaxG * WD; i += NT) {
-      const int j = i / kMaxG, h = i % kMaxG;
+    for (int i = tid; i < MH * WD; i += NT) {
+      const int j = i / MH, h = i % MH;
       float v = 0.f;
 #pragma unroll
-      for (int sl = 0; sl < NS; ++sl) v += s_red[(sl * kMaxG + h) * WD + j];
+      for (int sl = 0; sl < NS; ++sl) v += s_red[(sl * MH + h) * WD + j];
       if (j < kDim) v = FV::width(j) > 0 ? v / a.sig[FV::width(j)] : 0.f;
       s_acc[j][h] = h < G ? v : 0.f;
     }
     __syncthreads();
     // un-rotation: out_h[o] = sum_j Pi[j][o] A_h[j] + sqrt(pi/2)/m sum_j S[j][o] B_h[j]
-    float r[kMaxG];
+    float r[MH];
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) r[h] = 0.f;
-    const float4* acc4 = reinterpret_cast<const float4*>(&s_acc[sl4 * RS][0]);
+    for (int h = 0; h < MH; ++h) r[h] = 0.f;
 #pragma unroll
     for (int jj = 0; jj < RS; ++jj) {
-      const float4 x0 = acc4[2 * jj], x1 = acc4[2 * jj + 1];
-      r[0] = fmaf(pm[jj], x0.x, r[0]);
-      r[1] = fmaf(pm[jj], x0.y, r[1]);
-      r[2] = fmaf(pm[jj], x0.z, r[2]);
-      r[3] = fmaf(pm[jj], x0.w, r[3]);
-      r[4] = fmaf(pm[jj], x1.x, r[4]);
-      r[5] = fmaf(pm[jj], x1.y, r[5]);
-      r[6] = fmaf(pm[jj], x1.z, r[6]);
-      r[7] = fmaf(pm[jj], x1.w, r[7]);
+      if constexpr (MH == 1) {
+        r[0] = fmaf(pm[jj], s_acc[sl4 * RS + jj][0], r[0]);
+      } else {
+        const float4* acc4 = reinterpret_cast<const float4*>(&s_acc[sl4 * RS + jj][0]);
+#pragma unroll
+        for (int q4 = 0; q4 < MH / 4; ++q4) {
+          const float4 x = acc4[q4];
+          r[4 * q4] = fmaf(pm[jj], x.x, r[4 * q4]);
+          r[4 * q4 + 1] = fmaf(pm[jj], x.y, r[4 * q4 + 1]);
+          r[4 * q4 + 2] = fmaf(pm[jj], x.z, r[4 * q4 + 2]);
+          r[4 * q4 + 3] = fmaf(pm[jj], x.w, r[4 * q4 + 3]);
+        }
+      }
     }
     __syncthreads();  // s_red is reused
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) s_red[(sl4 * kMaxG + h) * kDim + o] = r[h];
+    for (int h = 0; h < MH; ++h) s_red[(sl4 * MH + h) * kDim + o] = r[h];
     __syncthreads();
   }
   for (int i = tid; i < G * kDim; i += NT) {
     const int h = i / kDim, j = i % kDim;
     float v = 0.f;
     if (has_pieces)
-      v = s_red[(0 * kMaxG + h) * kDim + j] + s_red[(1 * kMaxG + h) * kDim + j] + s_red[(2 * kMaxG + h) * kDim + j] +
-          s_red[(3 * kMaxG + h) * kDim + j];
+      v = s_red[(0 * MH + h) * kDim + j] + s_red[(1 * MH + h) * kDim + j] + s_red[(2 * MH + h) * kDim + j] +
+          s_red[(3 * MH + h) * kDim + j];
     if (ui.ns > 0) v = fmaf(s_M[h], s_osk[h][j], v);
     const float L = s_L[h];
     store_out(a, orow + i, L > 0.f ? v / L : 0.f);
@@ -767,6 +783,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int P = gridDim.x, cta = blockIdx.x;
   const int U = a.B * a.hkv;
+  // the lengths, read once: every later unit lookup is a shared-memory load
+  constexpr int kLenCache = 128;
+  __shared__ int s_len[kLenCache];
+  if (a.B <= kLenCache)
+    for (int b = tid; b < a.B; b += kThreadsP) s_len[b] = a.lens[b];
+  const int* lens = a.B <= kLenCache ? s_len : a.lens;
 
   // ---- barriers (thread 32); the producer starts the copy of the lookup
   // tables (built once per parameter set) while warp 0 computes the schedule
@@ -795,7 +817,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     // unit / local chunk where it starts
     long long C = 0;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
-      int ch = b0 + lane < a.B ? seq_slots(a, b0 + lane, CH) : 0;
+      int ch = b0 + lane < a.B ? seq_slots(a, lens, b0 + lane, CH) : 0;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, off);
       C += ch;
@@ -806,7 +828,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     long long base = 0;
     for (int b0 = 0; b0 < a.B && c0 < c1; b0 += 32) {
       const int b = b0 + lane;
-      const long long ch = b < a.B ? seq_slots(a, b, CH) : 0;
+      const long long ch = b < a.B ? seq_slots(a, lens, b, CH) : 0;
       long long incl = ch;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -831,7 +853,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     }
     if (cta == 0)
       for (int b = lane; b < a.B; b += 32)
-        if (a.lens[b] > a.max_len) atomicOr(a.status, 2);
+        if (lens[b] > a.max_len) atomicOr(a.status, 2);
     if (lane == 0) {
       s_c0 = c0;
       s_c1 = c1;
@@ -847,7 +869,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     // ---- producer: one lane streams the CTA's chunks through the stages
     if (lane == 0 && c0 < c1) {
       int u = s_u0, lc = s_lc0;
-      UnitInfo ui = unit_info(a, u, CH);
+      UnitInfo ui = unit_info(a, lens, u, CH);
       const int nk = static_cast<int>(c1 - c0);
       int s = 0, n_streamed = 0;
       uint32_t round = 0;  // parity of (chunks streamed) / S
@@ -855,7 +877,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
         while (lc >= ui.slots) {
           ++u;
           lc = 0;
-          ui = unit_info(a, u, CH);
+          ui = unit_info(a, lens, u, CH);
         }
         if (lc < ui.slack) {  // an empty slot
           ++lc;
@@ -910,7 +932,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   int u = -1;
   UnitInfo ui{};
   int walk_u = s_u0, walk_lc = s_lc0;
-  UnitInfo wui = c0 < c1 ? unit_info(a, walk_u, CH) : UnitInfo{};
+  UnitInfo wui = c0 < c1 ? unit_info(a, lens, walk_u, CH) : UnitInfo{};
   const int nk = static_cast<int>(c1 - c0);
   int s = 0;
   uint32_t round = 0;  // parity of k / S
@@ -919,7 +941,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
     while (walk_lc >= wui.slots) {
       ++walk_u;
       walk_lc = 0;
-      wui = unit_info(a, walk_u, CH);
+      wui = unit_info(a, lens, walk_u, CH);
     }
     if (walk_lc < wui.slack) {  // an empty slot
       ++walk_lc;
@@ -1010,21 +1032,23 @@ tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaS
   // that filled the cache); the decode kernel after it starts its prologue
   // (tables, schedule, first bulk copies) while the rotation runs, and the
   // merge kernel overlaps its prologue with the decode kernel's tail
-  const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
-  e = ensure_dyn_smem<qrot_kernel<KF>>(static_cast<int>(qrot_smem));
-  if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
-  qrot_kernel<KF><<<dim3(plan.hkv, plan.B), kQrotThreads, qrot_smem, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_qrot<KF>(a, plan.B, plan.hkv, st);
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   // static and dynamic shared memory together pass 48 KB: opt in every time
-  const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, a.merge_heads, plan.part_floats);
-  e = ensure_dyn_smem<merge_kernel<VF>>(static_cast<int>(merge_smem));
-  if (e != cudaSuccess) return cuda_fail(e, "merge kernel attribute");
-  e = launch_overlapped(merge_kernel<VF>, dim3(plan.B * plan.hkv, plan.group / a.merge_heads), kMergeThreads,
-                        merge_smem, st, a);
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "merge kernel launch");
+  auto merge = [&](auto mh) -> tq_status {
+    constexpr int MH = decltype(mh)::value;
+    const size_t merge_smem = merge_dyn_bytes(a.n_sink, plan.ctas, a.merge_heads, plan.part_floats, MH);
+    cudaError_t me = ensure_dyn_smem<merge_kernel<VF, MH>>(static_cast<int>(merge_smem));
+    if (me == cudaSuccess) me = ensure_max_carveout<merge_kernel<VF, MH>>();
+    if (me != cudaSuccess) return cuda_fail(me, "merge kernel attribute");
+    me = launch_overlapped(merge_kernel<VF, MH>, dim3(plan.B * plan.hkv, plan.group / a.merge_heads), kMergeThreads,
+                           merge_smem, st, a);
+    return me == cudaSuccess ? TQ_OK : cuda_fail(me, "merge kernel launch");
+  };
+  if (a.merge_heads == 1) return merge(IntC<1>{});
+  return a.merge_heads <= 4 ? merge(IntC<4>{}) : merge(IntC<8>{});
 }
 
 template <int KF, int VF>

@@ -536,138 +536,141 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\
 // B fragments of a rotated query: lane (g, t) supplies column g; k-steps 0..7
 // from the MSE segments, 8..15 from the QJL segment.  Unpacked: column g =
 // head g, halves hi (x = 0) and lo (x = 1).  Packed (group <= 4): column g < 4
-// = hi of head g, column g >= 4 = lo of head g - 4, in x = 0.  qt: [8][128]
-// rotated, scaled query (MSE coordinates); qsk: [8][128] sketch S q (prod
-// keys).  Threads tid = 0.. of nthreads write the kQfragWords words of dst.
+// = hi of head g, column g >= 4 = lo of head g - 4, in x = 0.  Word
+// ((ks * 2 + r) * 2 + x) * 32 + lane of a unit's kQfragWords.
+//
+// The coordinates behind the words of k-step ks for lane quarter t (dims[0..3]
+// = halves lo.x, lo.y, hi.x, hi.y); false where the format leaves the k-step
+// unused.  All four lie in one 32-coordinate block (block 0 for an unused
+// k-step).
 template <int KF>
-__device__ __forceinline__ void write_qfrag(const float* qt, const float* qsk, int pack, uint32_t* dst, int tid,
-                                            int nthreads) {
+__host__ __device__ __forceinline__ bool qfrag_dims(int ks, int t, int (&dims)[4]) {
   using KR = KRow<KF>;
   using FK = Fmt<KF>;
-  for (int i = tid; i < 16 * 32; i += nthreads) {
-    const int ks = i / 32, lane = i % 32, g = lane >> 2, t = lane & 3;
-    int dims[4] = {0, 0, 0, 0};
-    bool valid = true;
-    const bool qjl = ks >= 8;
-    if (!qjl) {
-      if (FK::nseg == 0) {
-        valid = false;
-      } else if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
-        for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
-      } else {
-        for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
-      }
+  for (int e = 0; e < 4; ++e) dims[e] = 0;
+  if (ks < 8) {
+    if (FK::nseg == 0) return false;
+    if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
+      for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
     } else {
-      if (!FK::prod) valid = false;
-      for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
+      for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
     }
-    const int head = pack ? (g & 3) : g;
-    const float* src = (qjl ? qsk : qt) + head * kDim;
-    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
-    if (valid) {
+    return true;
+  }
+  if (!FK::prod) return false;
+  for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// 1. query rotation: Pi q (MSE keys) and S q (prod keys) as fp16 fragments.
+//    One CTA per (32-coordinate slice of one matrix, kv-head, sequence):
+//    blockIdx.x = 4 * m + slice, m = 0 for Pi (formats with MSE codes), the
+//    last m for S (prod keys).  Thread (jj, ks) sums k in [16 ks, 16 ks + 16)
+//    for output coordinate 32 slice + jj of every head, the 8 partial sums
+//    meet in shared memory, and the slice writes the fragment words whose
+//    coordinates it holds (qfrag_dims keeps each word inside one slice).
+// ---------------------------------------------------------------------------
+constexpr int kQrotThreads = 256;
+constexpr int kQrotSlice = 32;                          // output coordinates per CTA
+constexpr int kQrotKSplit = kQrotThreads / kQrotSlice;  // slices of the k range
+constexpr int kQrotK = kDim / kQrotKSplit;              // k per thread
+
+template <int KF>
+constexpr int qrot_matrices() {
+  return (Fmt<KF>::nseg > 0 ? 1 : 0) + (Fmt<KF>::prod ? 1 : 0);
+}
+
+template <int KF>
+__global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
+  using FK = Fmt<KF>;
+  __shared__ __align__(16) float qsT[kDim][kMaxG];  // query, [k][head]
+  __shared__ float s_p[kQrotKSplit][kMaxG][kQrotSlice];
+  __shared__ float s_v[kMaxG][kQrotSlice];          // the slice's scaled outputs
+  const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int m = (FK::nseg > 0 ? 0 : 1) + static_cast<int>(blockIdx.x) / 4, sl = blockIdx.x % 4;
+  const int G = a.group;
+  pdl_launch();  // the decode kernel's prologue and cache stream may start
+  const int jj = tid % kQrotSlice, kq = tid / kQrotSlice, j = sl * kQrotSlice + jj;
+  // this thread's matrix entries (Pi^T or S^T, [k][j]: coalesced over j)
+  const float* mat = m ? a.st : a.pit;
+  float mv[kQrotK];
+#pragma unroll
+  for (int i = 0; i < kQrotK; ++i) mv[i] = __ldg(mat + (kq * kQrotK + i) * kDim + j);
+  for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
+    const int h = i % kMaxG, d = i / kMaxG;
+    qsT[d][h] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
+  }
+  __syncthreads();
+  float acc[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+  const float4* q4 = reinterpret_cast<const float4*>(&qsT[0][0]);
+#pragma unroll
+  for (int i = 0; i < kQrotK; ++i) {
+    const int k = kq * kQrotK + i;
+    const float4 x0 = q4[2 * k], x1 = q4[2 * k + 1];
+    acc[0] = fmaf(mv[i], x0.x, acc[0]);
+    acc[1] = fmaf(mv[i], x0.y, acc[1]);
+    acc[2] = fmaf(mv[i], x0.z, acc[2]);
+    acc[3] = fmaf(mv[i], x0.w, acc[3]);
+    acc[4] = fmaf(mv[i], x1.x, acc[4]);
+    acc[5] = fmaf(mv[i], x1.y, acc[5]);
+    acc[6] = fmaf(mv[i], x1.z, acc[6]);
+    acc[7] = fmaf(mv[i], x1.w, acc[7]);
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) s_p[kq][h][jj] = acc[h];
+  __syncthreads();
+  {
+    const int h = tid / kQrotSlice;  // kQrotThreads = kMaxG * kQrotSlice
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < kQrotKSplit; ++i) v += s_p[i][h][jj];
+    if (m == 0) {
+      const int wj = FK::width(j);
+      v = wj > 0 ? v * (a.qscale / a.sig[wj]) : 0.f;
+    } else {
+      v *= a.qscale;
+    }
+    s_v[h][jj] = v;
+  }
+  __syncthreads();
+  // the words of this matrix's k-steps whose coordinates lie in the slice
+  uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
+  {
+    const int ks = 8 * m + tid / 32, lane = tid % 32, g = lane >> 2, t = lane & 3;
+    int dims[4];
+    if (qfrag_dims<KF>(ks, t, dims) && dims[0] / kQrotSlice == sl) {
+      const int head = a.pack ? (g & 3) : g;
+      const float* src = &s_v[head][0];
+      const int o = sl * kQrotSlice;
+#pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const float x0 = src[dims[2 * r]], x1 = src[dims[2 * r + 1]];
-        const __half2 h = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(h);
-        hi[r] = *reinterpret_cast<const uint32_t*>(&h);
-        lo[r] = h2bits(x0 - hf.x, x1 - hf.y);
-      }
-    }
-    for (int r = 0; r < 2; ++r) {
-      if (pack) {
-        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = g < 4 ? hi[r] : lo[r];
-        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = 0;
-      } else {
-        dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi[r];
-        dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo[r];
+        const float x0 = src[dims[2 * r] - o], x1 = src[dims[2 * r + 1] - o];
+        const __half2 hv = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(hv);
+        const uint32_t hi = *reinterpret_cast<const uint32_t*>(&hv);
+        const uint32_t lo = h2bits(x0 - hf.x, x1 - hf.y);
+        if (a.pack) {
+          dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = g < 4 ? hi : lo;
+          dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = 0;
+        } else {
+          dst[((ks * 2 + r) * 2 + 0) * 32 + lane] = hi;
+          dst[((ks * 2 + r) * 2 + 1) * 32 + lane] = lo;
+        }
       }
     }
   }
 }
 
-// ---------------------------------------------------------------------------
-// 1. query rotation: one CTA per (sequence, kv-head).  Threads 0..127 form
-//    Pi q for all heads (one output coordinate each), threads 128..255 form
-//    S q (prod keys); then the fp16 B-fragments are written.
-// ---------------------------------------------------------------------------
-constexpr int kQrotThreads = 512;
-constexpr int kQrotSplit = kQrotThreads / kDim;  // slices of the k range per output coordinate
-
+// The query rotation of B sequences x hkv kv-heads.
 template <int KF>
-__global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
-  using KR = KRow<KF>;
-  using FK = Fmt<KF>;
-  extern __shared__ float4 s_mat4[];              // Pi^T [k][j], then S^T [k][j] (prod keys)
-  __shared__ __align__(16) float qsT[kDim][kMaxG];  // query, [k][head]
-  __shared__ float qt[kMaxG][kDim];
-  __shared__ float qsk[kMaxG][kSketch];
-  __shared__ float s_p[kQrotSplit][kMaxG][kDim];  // partial sums over k slices
-  const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int G = a.group;
-  pdl_launch();  // the decode kernel's prologue and cache stream may start
-  {
-    // stage the matrices with asynchronous 16-byte copies, all in flight
-    constexpr int N4 = kDim * kDim / 4 / kQrotThreads;
-    const float4* pit4 = reinterpret_cast<const float4*>(a.pit);
-#pragma unroll
-    for (int i = 0; i < N4; ++i)
-      cp_async16(smem_u32(s_mat4 + i * kQrotThreads + tid), pit4 + i * kQrotThreads + tid);
-    if constexpr (FK::prod) {
-      const float4* st4 = reinterpret_cast<const float4*>(a.st);
-#pragma unroll
-      for (int i = 0; i < N4; ++i)
-        cp_async16(smem_u32(s_mat4 + kDim * kDim / 4 + i * kQrotThreads + tid), st4 + i * kQrotThreads + tid);
-    }
-  }
-  for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
-    const int h = i % kMaxG, d = i / kMaxG;
-    qsT[d][h] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  const float scale = a.qscale;
-  // thread (j, ks) sums k in [ks * 32, ks * 32 + 32) for output coordinate j
-  // of every head; the slices are added in shared memory
-  const int j = tid & (kDim - 1), ks = tid >> 7;
-  const float4* q4 = reinterpret_cast<const float4*>(&qsT[0][0]);
-  for (int mtx = 0; mtx < (FK::prod ? 2 : 1); ++mtx) {
-    const float* mat = reinterpret_cast<const float*>(s_mat4) + mtx * kDim * kDim;
-    float acc[kMaxG];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
-#pragma unroll 8
-    for (int kk = 0; kk < kDim / kQrotSplit; ++kk) {
-      const int k = ks * (kDim / kQrotSplit) + kk;
-      const float m = mat[k * kDim + j];
-      const float4 x0 = q4[2 * k], x1 = q4[2 * k + 1];
-      acc[0] = fmaf(m, x0.x, acc[0]);
-      acc[1] = fmaf(m, x0.y, acc[1]);
-      acc[2] = fmaf(m, x0.z, acc[2]);
-      acc[3] = fmaf(m, x0.w, acc[3]);
-      acc[4] = fmaf(m, x1.x, acc[4]);
-      acc[5] = fmaf(m, x1.y, acc[5]);
-      acc[6] = fmaf(m, x1.z, acc[6]);
-      acc[7] = fmaf(m, x1.w, acc[7]);
-    }
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) s_p[ks][h][j] = acc[h];
-    __syncthreads();
-    for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
-      const int h = i / kDim, jj = i % kDim;
-      float v = 0.f;
-#pragma unroll
-      for (int s = 0; s < kQrotSplit; ++s) v += s_p[s][h][jj];
-      if (mtx == 1) {
-        qsk[h][jj] = v * scale;
-      } else {
-        const int wj = FK::width(jj);
-        qt[h][jj] = wj > 0 ? v * (scale / a.sig[wj]) : 0.f;
-      }
-    }
-    __syncthreads();
-  }
-  uint32_t* dst = const_cast<uint32_t*>(a.qfrag) + (static_cast<int64_t>(b) * a.hkv + kvh) * kQfragWords;
-  write_qfrag<KF>(&qt[0][0], &qsk[0][0], a.pack, dst, tid, kQrotThreads);
+cudaError_t launch_qrot(const DecodeArgs& a, int B, int hkv, cudaStream_t st) {
+  const cudaError_t e = ensure_max_carveout<qrot_kernel<KF>>();
+  if (e != cudaSuccess) return e;
+  qrot_kernel<KF><<<dim3(4 * qrot_matrices<KF>(), hkv, B), kQrotThreads, 0, st>>>(a);
+  return cudaGetLastError();
 }
 
 // Shared addresses of the planes of one staged chunk.

@@ -116,6 +116,23 @@ cudaError_t ensure_dyn_smem(int bytes) {
   return cudaSuccess;
 }
 
+// Prefer the largest shared-memory carveout for a small kernel that runs
+// right before or after the decode kernel (query rotation, merge): an SM
+// whose carveout already fits the decode kernel's 226 KB takes its CTA as
+// soon as the small kernel's CTAs leave, without reconfiguring first.
+template <auto kernel>
+cudaError_t ensure_max_carveout() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
 // Kernel launchers (defined in the .cu files).
 tq_status launch_quantize(const tq_params* p, const FormatSpec& f, const void* x, int x_bf16,
                           int64_t n, const tq_packed* out, cudaStream_t st);

@@ -450,11 +450,7 @@ tq_status run_search(DecodeArgs& a, int groups_ctas, cudaStream_t st) {
   a.bound_out = nullptr;
   cudaError_t e = ensure_dyn_smem<search_kernel<KF, PACK>>(kSmemBudget);
   if (e != cudaSuccess) return cuda_fail(e, "search kernel attribute");
-  const size_t qrot_smem = static_cast<size_t>(Fmt<KF>::prod ? 2 : 1) * kDim * kDim * sizeof(float);
-  e = ensure_dyn_smem<qrot_kernel<KF>>(static_cast<int>(qrot_smem));
-  if (e != cudaSuccess) return cuda_fail(e, "query rotation attribute");
-  qrot_kernel<KF><<<dim3(1, 1), kQrotThreads, qrot_smem, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_qrot<KF>(a, 1, 1, st);
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   const size_t merge_smem = static_cast<size_t>(groups_ctas) * 32 * sizeof(uint64_t);
   if (merge_smem > 48 * 1024) {
