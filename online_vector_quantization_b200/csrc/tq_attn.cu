@@ -625,14 +625,35 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     first = cta_of_chunk(cu0, C, P);
     n_p = cta_of_chunk(cu0 + ui.chunks - 1, C, P) - first + 1;
   }
-  // the maxima and sums of all pieces, gathered at once
+  // this CTA's heads of each piece: G x PF consecutive floats at head h0,
+  // staged with 16-byte asynchronous copies, merge_chunk pieces at a time
+  const int slot_floats = G * PF, per4 = slot_floats / 4;
+  auto stage = [&](int c0, int cnt) {
+    for (int e = tid; e < cnt * per4; e += NT) {
+      const int i = e / per4, q4 = e - i * per4;
+      const float4* src = reinterpret_cast<const float4*>(part_slot(a, u + first + c0 + i) + h0 * PF);
+      cp_async16(smem_u32(s_part) + 16 * e, src + q4);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+  };
+  // usually every piece fits one staging pass: the maxima and sums are then
+  // read from the staged copies, one memory round trip after the wait
+  const bool one_pass = has_pieces && n_p <= a.merge_chunk;
+  if (one_pass) stage(0, n_p);
   for (int e = tid; e < n_p * G; e += NT) {
     const int i = e / G, h = e % G;
     float m = -INFINITY, l = 0.f;
     if (cta_has_chunks(first + i, C, P)) {
-      const float* pp = part_slot(a, u + first + i) + (h0 + h) * PF;
-      m = __ldcg(pp);
-      l = __ldcg(pp + 1);
+      if (one_pass) {
+        const float* pp = s_part + i * slot_floats + h * PF;
+        m = pp[0];
+        l = pp[1];
+      } else {
+        const float* pp = part_slot(a, u + first + i) + (h0 + h) * PF;
+        m = __ldcg(pp);
+        l = __ldcg(pp + 1);
+      }
     }
     s_f[i * MH + h] = m;
     s_l[i * MH + h] = l;
@@ -660,24 +681,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   __syncthreads();
   if (has_pieces) {
     {
-      // the accumulators: consecutive slots, staged chunk by chunk with
-      // 16-byte asynchronous copies
+      // the accumulators (already staged in the one-pass case)
       const int j = tid % WD, sl = tid / WD;
       float acc[MH];
 #pragma unroll
       for (int h = 0; h < MH; ++h) acc[h] = 0.f;
-      // this CTA's heads of each piece: G x PF consecutive floats at head h0
-      const int slot_floats = G * PF, per4 = slot_floats / 4;
       for (int c0 = 0; c0 < n_p; c0 += a.merge_chunk) {
         const int cnt = min(a.merge_chunk, n_p - c0);
-        const int n16 = cnt * per4;
-        for (int e = tid; e < n16; e += NT) {
-          const int i = e / per4, q4 = e - i * per4;
-          const float4* src = reinterpret_cast<const float4*>(part_slot(a, u + first + c0 + i) + h0 * PF);
-          cp_async16(smem_u32(s_part) + 16 * e, src + q4);
-        }
-        cp_async_wait_all();
-        __syncthreads();
+        if (!one_pass) stage(c0, cnt);
         for (int i = sl; i < cnt; i += NS) {
           const float* pp = s_part + i * slot_floats + kPartAcc + j;
 #pragma unroll
@@ -688,7 +699,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
             if (f != 0.f) acc[h] = fmaf(pp[h * PF], f, acc[h]);
           }
         }
-        __syncthreads();  // the staging buffer is refilled
+        if (!one_pass) __syncthreads();  // the staging buffer is refilled
       }
 #pragma unroll
       for (int h = 0; h < MH; ++h) s_red[(sl * MH + h) * WD + j] = acc[h];
@@ -1028,11 +1039,12 @@ template <int KF, int VF, bool PACK, int SPARSE>
 tq_status run_decode_v(DecodeArgs& a, const DecodePlan& plan, size_t smem, cudaStream_t st) {
   cudaError_t e = ensure_dyn_smem<decode_kernel<KF, VF, PACK, SPARSE>>(static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel attribute");
-  // the query rotation waits for all earlier work on the stream (the appends
-  // that filled the cache); the decode kernel after it starts its prologue
+  // the query rotation loads its matrix entries while the previous kernel on
+  // the stream (the append that filled the cache, say) finishes, and reads
+  // the query only after it; the decode kernel after it starts its prologue
   // (tables, schedule, first bulk copies) while the rotation runs, and the
   // merge kernel overlaps its prologue with the decode kernel's tail
-  e = launch_qrot<KF>(a, plan.B, plan.hkv, st);
+  e = launch_qrot<KF>(a, plan.B, plan.hkv, st, true);
   if (e != cudaSuccess) return cuda_fail(e, "query rotation launch");
   e = launch_overlapped(decode_kernel<KF, VF, PACK, SPARSE>, dim3(plan.ctas), kThreadsP, smem, st, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

@@ -549,17 +549,23 @@ __host__ __device__ __forceinline__ bool qfrag_dims(int ks, int t, int (&dims)[4
   using FK = Fmt<KF>;
   for (int e = 0; e < 4; ++e) dims[e] = 0;
   if (ks < 8) {
-    if (FK::nseg == 0) return false;
-    if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
-      for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
+    if constexpr (FK::nseg == 0) {
+      return false;
     } else {
-      for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
+      if (FK::nseg == 1 || ks < KR::S0::KSTEPS) {
+        for (int e = 0; e < 4; ++e) dims[e] = KR::S0::dim(0, t, ks, e);
+      } else {
+        for (int e = 0; e < 4; ++e) dims[e] = KR::S1::dim(64, t, ks - KR::S0::KSTEPS, e);
+      }
+      return true;
     }
+  }
+  if constexpr (!FK::prod) {
+    return false;
+  } else {
+    for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
     return true;
   }
-  if (!FK::prod) return false;
-  for (int e = 0; e < 4; ++e) dims[e] = KR::Q::dim(0, t, ks - 8, e);
-  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -590,13 +596,17 @@ __global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
   const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int m = (FK::nseg > 0 ? 0 : 1) + static_cast<int>(blockIdx.x) / 4, sl = blockIdx.x % 4;
   const int G = a.group;
-  pdl_launch();  // the decode kernel's prologue and cache stream may start
   const int jj = tid % kQrotSlice, kq = tid / kQrotSlice, j = sl * kQrotSlice + jj;
   // this thread's matrix entries (Pi^T or S^T, [k][j]: coalesced over j)
   const float* mat = m ? a.st : a.pit;
   float mv[kQrotK];
 #pragma unroll
   for (int i = 0; i < kQrotK; ++i) mv[i] = __ldg(mat + (kq * kQrotK + i) * kDim + j);
+  // Launched behind the previous kernel on the stream (an append, say), the
+  // matrix loads above overlap its tail; the query, and the cache lengths the
+  // decode kernel reads, are only read once that kernel has finished.
+  pdl_wait();
+  pdl_launch();  // the decode kernel's prologue and cache stream may start
   for (int i = tid; i < kMaxG * kDim; i += kQrotThreads) {
     const int h = i % kMaxG, d = i / kMaxG;
     qsT[d][h] = h < G ? load_q(a.q, a.q_bf16, (static_cast<int64_t>(b) * a.hq + kvh * G + h) * kDim + d) : 0.f;
@@ -664,14 +674,6 @@ __global__ void __launch_bounds__(kQrotThreads) qrot_kernel(DecodeArgs a) {
   }
 }
 
-// The query rotation of B sequences x hkv kv-heads.
-template <int KF>
-cudaError_t launch_qrot(const DecodeArgs& a, int B, int hkv, cudaStream_t st) {
-  const cudaError_t e = ensure_max_carveout<qrot_kernel<KF>>();
-  if (e != cudaSuccess) return e;
-  qrot_kernel<KF><<<dim3(4 * qrot_matrices<KF>(), hkv, B), kQrotThreads, 0, st>>>(a);
-  return cudaGetLastError();
-}
 
 // Shared addresses of the planes of one staged chunk.
 struct UnitPlanes {
@@ -958,6 +960,18 @@ cudaError_t launch_overlapped(Kernel kernel, dim3 grid, int threads, size_t smem
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// The query rotation of B sequences x hkv kv-heads; overlapped: launched with
+// programmatic stream serialization (see qrot_kernel).
+template <int KF>
+cudaError_t launch_qrot(const DecodeArgs& a, int B, int hkv, cudaStream_t st, bool overlapped = false) {
+  const cudaError_t e = ensure_max_carveout<qrot_kernel<KF>>();
+  if (e != cudaSuccess) return e;
+  const dim3 grid(4 * qrot_matrices<KF>(), hkv, B);
+  if (overlapped) return launch_overlapped(qrot_kernel<KF>, grid, kQrotThreads, 0, st, a);
+  qrot_kernel<KF><<<grid, kQrotThreads, 0, st>>>(a);
+  return cudaGetLastError();
 }
 
 constexpr int fid(int mse, int mixed, int prod) { return mse | (mixed << 4) | (prod << 5); }

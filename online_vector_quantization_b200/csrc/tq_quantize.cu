@@ -80,6 +80,11 @@ struct QuantArgs {
   int n_seq_in;
 };
 
+// Lets the next kernel on the stream, when it is launched with programmatic
+// stream serialization (the decode call's query rotation), start its own
+// independent prologue; it waits for this grid before reading its outputs.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // The input and destinations of plane pl.
 struct PlaneDst {
   const void* x;
@@ -367,6 +372,7 @@ template <int BF16>
 __global__ void __launch_bounds__(kThreads, 1) quantize_kernel(QuantArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SmemQuant& s = *reinterpret_cast<SmemQuant*>(smem_raw);
+  launch_dependents();
   SmemProd* sp = a.prod ? reinterpret_cast<SmemProd*>(smem_raw + sizeof(SmemQuant)) : nullptr;
   __shared__ float cb_s[kMaxBits + 1][kBookSlots];
   __shared__ float bd_s[kMaxBits + 1][kBookSlots];
@@ -624,6 +630,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
                                                                     QuantArgs a) {
   using namespace sm100;
   using TF = TcFormat<B, MIXED>;
+  launch_dependents();
   // 8-bit codes: Pi in three bf16 terms (the 255 bounds sit ~1.5e-3 apart,
   // so the rotation must be good to ~1e-8) and one fewer x stage to make room
   constexpr bool kWide = B == kWideBits;
@@ -910,6 +917,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
                                                                          QuantArgs a) {
   using namespace sm100;
   constexpr int CW = MB > 0 ? 4 * MB : 1;  // packed MSE words per row (unused for MB = 0)
+  launch_dependents();
   extern __shared__ __align__(16) unsigned char smem_tp[];
   __shared__ __align__(8) uint64_t x_full[2], x_empty[2], t1_full[2], rho_full[2], t2_full[2], t_empty[2], b_full;
   __shared__ uint32_t s_tmem;
@@ -1200,6 +1208,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_prod_kernel(const _
 __global__ void __launch_bounds__(kDim) quantize8_kernel(QuantArgs a) {
   __shared__ double xs[kDim];
   __shared__ double red[kDim / 32];
+  launch_dependents();
   __shared__ __align__(16) uint32_t words[kDim / 4];
   __shared__ float2 s_cell8[kCell8Max];
   __shared__ long long s_row;
