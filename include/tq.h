@@ -285,10 +285,12 @@ tq_status tq_decode_workspace_init(void* workspace, size_t ws_bytes, void* strea
  * (MSE 1..4 bits, mixed 2.5 and 3.5, prod 1..4) and the asymmetric MSE pairs
  * K4/V3, K4/V2, K3/V2 and K8/V3 (8-bit keys); any other pair gives
  * TQ_ERR_UNSUPPORTED.  Three kernels run on the stream: the
- * query rotation, the persistent decode kernel and the merge; the last two
- * are launched with programmatic stream serialization and overlap their
- * prologues with the previous kernel's tail.  Nothing in the workspace needs
- * to start at zero. */
+ * query rotation, the persistent decode kernel and the merge, each launched
+ * with programmatic stream serialization so that its prologue overlaps the
+ * previous kernel's tail; the rotation reads q only after the kernel before
+ * it on the stream has finished, so q and the cache may be written by the
+ * work just before the call.  Nothing in the workspace needs to start at
+ * zero. */
 tq_status tq_decode_attn(const tq_params* p, const void* q, int q_dtype, const tq_cache* cache,
                          int B, int hq, int max_len, void* out, int out_dtype,
                          void* workspace, size_t ws_bytes, const tq_attn_flags* flags,

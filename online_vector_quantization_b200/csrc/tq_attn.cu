@@ -258,8 +258,10 @@ struct UnitInfo {
 };
 
 // lens: the cache's lengths (global), or the decode kernel's copy of them in
-// shared memory.
-__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, const int* lens, int u, int kChunk) {
+// shared memory.  Read as volatile: a kernel launched with programmatic
+// stream serialization may run beside the one that wrote them, so they are
+// fetched from L2, never from a stale L1 line.
+__device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, const volatile int* lens, int u, int kChunk) {
   const int b = u / a.hkv;
   const int len = min(max(lens[b], 0), a.max_len);
   UnitInfo r;
@@ -274,7 +276,7 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeArgs& a, const int* le
 
 
 // Slots of each kv-head unit of sequence b (all units of a sequence are alike).
-__device__ __forceinline__ int seq_slots(const DecodeArgs& a, const int* lens, int b, int kChunk) {
+__device__ __forceinline__ int seq_slots(const DecodeArgs& a, const volatile int* lens, int b, int kChunk) {
   const int len = min(max(lens[b], 0), a.max_len);
   const int ch = (len - min(a.n_sink, len) + kChunk - 1) / kChunk;
   return ch > 0 ? ch + a.unit_slack : 0;
@@ -798,8 +800,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) decode_kernel(DecodeArgs a) {
   constexpr int kLenCache = 128;
   __shared__ int s_len[kLenCache];
   if (a.B <= kLenCache)
-    for (int b = tid; b < a.B; b += kThreadsP) s_len[b] = a.lens[b];
-  const int* lens = a.B <= kLenCache ? s_len : a.lens;
+    for (int b = tid; b < a.B; b += kThreadsP) s_len[b] = __ldcg(a.lens + b);
+  const volatile int* lens = a.B <= kLenCache ? s_len : a.lens;
 
   // ---- barriers (thread 32); the producer starts the copy of the lookup
   // tables (built once per parameter set) while warp 0 computes the schedule

@@ -155,7 +155,7 @@ __device__ int64_t append_row(const QuantArgs& a, int64_t v, int* seq_out, int* 
   *head_out = head;
   *pos_out = 0;
   if (seq < 0 || seq >= a.cache_seqs) return -1;          // rejected by the length update
-  const int len = a.lens[seq];
+  const int len = __ldcg(a.lens + seq);  // written by the previous append's last CTA
   *pos_out = len + tok;
   if (len < 0 || len + a.n_tok > a.n_sink + a.capacity) return -1;
   const int pos = len + tok;
