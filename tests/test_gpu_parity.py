@@ -689,3 +689,36 @@ def test_append_length_update_folded(fk, fv, dtype):
     torch.cuda.synchronize()
     expect[4] += 8
     assert cache.lens.cpu().tolist() == expect and int(cache.status.item()) == 0
+
+
+def test_decode_reads_query_and_cache_written_just_before():
+    """The decode call's kernels start under programmatic stream
+    serialization, overlapping the previous kernel's tail: a query produced by
+    the kernel right before the call, after an append that filled the cache,
+    must still be read as written.  Each call is compared with the same call
+    made after a full synchronization."""
+    fk = fv = gu.fmt(3, mixed=True)
+    gp, _ = gu.make_params(fk, fv)
+    B, hkv, hq, T = 3, 2, 8, 700
+    k = kv_inputs.kv_vectors(B * T * hkv, 128, key=("pdl", "k"), dtype=torch.bfloat16).view(B, T, hkv, 128).cuda()
+    v = kv_inputs.kv_vectors(B * T * hkv, 128, key=("pdl", "v"), dtype=torch.bfloat16).view(B, T, hkv, 128).cuda()
+    base = kv_inputs.queries((B, hq, 128), key=("pdl", "q"), dtype=torch.float32).cuda()
+    ids = torch.arange(B, dtype=torch.int32, device="cuda")
+    ws = tq.decode_workspace(gp, B, hq, hkv, T)
+    for trial in range(3):
+        cache = tq.Cache(gp, B, hkv, 704, 0)
+        out_fast = torch.empty(B, hq, 128, dtype=torch.bfloat16, device="cuda")
+        for c0 in range(0, T, 64):
+            c1 = min(T, c0 + 64)
+            tq.tq_append(gp, cache, ids, k[:, c0:c1].contiguous(), v[:, c0:c1].contiguous())
+        # the query comes from a kernel launched just before the decode call
+        q = (base * (1.0 + 0.5 * trial)).to(torch.bfloat16)
+        tq.tq_decode_attn(gp, q, cache, T, out_fast, ws)
+        torch.cuda.synchronize()
+        out_sync = torch.empty_like(out_fast)
+        q2 = q.clone()
+        torch.cuda.synchronize()
+        tq.tq_decode_attn(gp, q2, cache, T, out_sync, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out_fast, out_sync), trial
+        assert cache.lens.cpu().tolist() == [T] * B and int(cache.status.item()) == 0
