@@ -338,6 +338,8 @@ size_t tq_search_workspace_bytes(void);
  *           caller-owned: per query the k best rows, larger score first,
  *           equal scores in row order; with n < k the tail holds score -inf
  *           and row -1.
+ * Every format tq_params_create accepts is searchable (MSE 1..4 and 8 bits,
+ * mixed 2.5 and 3.5, prod 1..4).
  * Scores come from fp16 tensor-core products with fp32 accumulation: rows
  * whose scores differ by less than about 1e-3 of ||q|| ||x|| may come in
  * either order.  1 <= k <= 32 (TQ_ERR_UNSUPPORTED above), 0 <= n < 2^31,

@@ -1216,6 +1216,7 @@ tq_status launch_decode(const tq_params* p, const void* q, int q_bf16, const tq_
   a.pi = p->pi32;
   a.s = p->s32;
   a.cbs = p->cbs32;
+  a.cbs8 = p->cbs8_32;
   a.lut_img = p->lut_img;
   a.sig = p->sig32;
   a.sparse_thr = sparse_thr;

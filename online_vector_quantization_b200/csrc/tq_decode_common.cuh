@@ -210,7 +210,11 @@ struct KChunk {
   // row: shared address of the token's code row
   __device__ __forceinline__ void load(uint32_t row, int t) {
     const int o = BYTE0 + t * BYTES;
-    if constexpr (BYTES == 16) {
+    if constexpr (BYTES == 32) {
+      const uint4 v0 = lds128(row, o), v1 = lds128(row, o + 16);
+      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    } else if constexpr (BYTES == 16) {
       const uint4 v = lds128(row, o);
       w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     } else if constexpr (BYTES == 12) {
@@ -498,6 +502,7 @@ struct DecodeArgs {
   const float* pi;   // Pi
   const float* s;    // S
   const float* cbs;  // sigma-scaled centroids [5][16] (the values the MMAs see)
+  const float* cbs8;  // sigma-scaled 8-bit centroids [256] (8-bit formats)
   const uint8_t* lut_img;  // the decode kernel's lookup tables, prebuilt (params)
   const float* sig;  // sigma per width [5]
   float sparse_thr;

@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) search_kernel(DecodeArgs a) {
   }
 
   // ---- lookup tables (consumer threads)
-  build_luts<L>(lut_mem, s_cb, tid);
+  build_luts<L>(lut_mem, s_cb, tid, a.cbs8);
   consumers_sync();  // tables complete
   const uint32_t lut_a = 0, lut_b = 0;
   const uint32_t lane4 = kLutAddr | (lane * 4), lane8 = (kLutAddr + L::region_b_off) | (lane * 8);
@@ -514,6 +514,7 @@ tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed
     a.pi = p->pi32;
     a.s = p->s32;
     a.cbs = p->cbs32;
+    a.cbs8 = p->cbs8_32;
     a.sig = p->sig32;
     a.pack = a.group <= 4;
     a.dyn_bytes = kSmemBudget;
@@ -537,6 +538,7 @@ tq_status launch_search(const tq_params* p, const FormatSpec& f, const tq_packed
     TQ_CASE(fid(1, 0, 1))
     TQ_CASE(fid(2, 0, 1))
     TQ_CASE(fid(3, 0, 1))
+    TQ_CASE(fid(8, 0, 0))
     return fail(TQ_ERR_UNSUPPORTED, "tq_search: no search kernel for this format");
 #undef TQ_CASE
     if (r != TQ_OK) return r;

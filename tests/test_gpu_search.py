@@ -102,8 +102,8 @@ def queries(xd, nq, key, planted=()):
 
 
 SEARCH_FORMATS = [gu.fmt(1), gu.fmt(3), gu.fmt(4), gu.fmt(3, mixed=True), gu.fmt(2, mixed=True),
-                  gu.fmt(1, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True)]
-SEARCH_IDS = ["mse1", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod1", "prod3", "prod4"]
+                  gu.fmt(1, prod=True), gu.fmt(3, prod=True), gu.fmt(4, prod=True), gu.fmt(8)]
+SEARCH_IDS = ["mse1", "mse3", "mse4", "mixed3.5", "mixed2.5", "prod1", "prod3", "prod4", "mse8"]
 
 
 @pytest.mark.parametrize("f", SEARCH_FORMATS, ids=SEARCH_IDS)
