@@ -379,7 +379,7 @@ def test_decode_sparse_v_skips_whole_tiles():
     assert gu.rel_l2(out.float().cpu().numpy(), want) < gu.ATTN_REL_L2
 
 
-def test_config1_tiny_fp32_end_to_end():
+def test_tiny_fp32_quantize_append_decode_end_to_end():
     """The tiny MSE-only configuration as stated: 4096 fp32 vectors (d = 128,
     lognormal norms), 3-bit codes quantized on the GPU, dequantized, then
     appended to a one-head cache as keys and values alike and attended by one
@@ -417,7 +417,7 @@ def test_config1_tiny_fp32_end_to_end():
     ocache = o.cache_from_vectors(op, xd[None, None], xd[None, None], 0)
     want = o.decode_attention(op, q.double().numpy(), ocache, [n], 1)
     err = gu.rel_l2(out.cpu().numpy(), want)
-    print(f"config 1 (fp32 query and output, GPU-built cache vs the oracle's): rel L2 {err:.3e}")
+    print(f"tiny fp32 case (4096 vectors, fp32 query and output, GPU-built cache vs the oracle's): rel L2 {err:.3e}")
     assert err < gu.ATTN_REL_L2
 
 
