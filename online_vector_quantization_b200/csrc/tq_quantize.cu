@@ -107,12 +107,13 @@ __device__ __forceinline__ PlaneDst plane_dst(const QuantArgs& a, int pl) {
 __device__ void append_arrive(const QuantArgs& a, int count = 1) {
   if (!a.append || a.arrive_total <= 0) return;
   __shared__ int s_last;
+  // No fence: every read of lens in this CTA has been consumed (its rows
+  // computed) before the barrier, nothing in this kernel reads the rows it
+  // writes, and later kernels on the stream see all of it at its end.
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     const int old = atomicAdd(a.status, count << 16);
     s_last = ((old >> 16) & 0xFFFF) + count == a.arrive_total;
-    if (s_last) __threadfence();
   }
   __syncthreads();
   if (!s_last) return;
