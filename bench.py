@@ -273,7 +273,10 @@ def run_gpu(args):
             "clocks": clocks,
             # per step: append = quantize K, quantize V, length update;
             # decode = query rotation, decode kernel, merge
-            "gpu_launches": args.steps * 6,
+            # per step: one append launch (K and V planes of the equal mixed
+            # formats together) and the decode call's query rotation, decode
+            # kernel and merge
+            "gpu_launches": args.steps * 4,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "aux": aux,
