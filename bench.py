@@ -271,8 +271,6 @@ def run_gpu(args):
                          "bytes_per_launch": int(decode_bytes_per_launch), "traffic": decode_traffic(),
                          "traffic_kernel": "decode_kernel alone (ncu capture)"},
             "clocks": clocks,
-            # per step: append = quantize K, quantize V, length update;
-            # decode = query rotation, decode kernel, merge
             # per step: one append launch (K and V planes of the equal mixed
             # formats together) and the decode call's query rotation, decode
             # kernel and merge
