@@ -78,7 +78,13 @@ struct QuantArgs {
   // and returns the count to zero.  0 = no update in this launch.
   int arrive_total;
   int n_seq_in;
+  // Append input in head-major tiles (the MSE tensor-core kernel): tile =
+  // 128 consecutive tokens (over the n_seq_in x n_tok chunk, token-major) of
+  // one kv-head, so a warp's 32 rows go to consecutive rows of one cache unit
+  // and its tiled stores land in a few tiles instead of eight units.
+  int head_major;
 };
+
 
 // Lets the next kernel on the stream, when it is launched with programmatic
 // stream serialization (the decode call's query rotation), start its own
@@ -625,6 +631,23 @@ struct TcFormat {
   static constexpr int bytes = 4 * words;
 };
 
+// Tiles of one plane, and the row of tile-local row r (-1: past the end).
+__host__ __device__ __forceinline__ int64_t plane_tile_count(const QuantArgs& a) {
+  if (a.head_major) {
+    const int64_t nt = a.n / a.hkv;
+    return ((nt + kTcRows - 1) / kTcRows) * a.hkv;
+  }
+  return (a.n + kTcRows - 1) / kTcRows;
+}
+__device__ __forceinline__ int64_t tile_row(const QuantArgs& a, int64_t lt, int r) {
+  if (a.head_major) {
+    const int64_t ts = (lt / a.hkv) * kTcRows + r;  // token index over the chunk
+    return ts < a.n / a.hkv ? ts * a.hkv + lt % a.hkv : -1;
+  }
+  const int64_t v = lt * kTcRows + r;
+  return v < a.n ? v : -1;
+}
+
 template <int B, int MIXED>
 __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                     const __grid_constant__ CUtensorMap xmap2,
@@ -678,7 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const int64_t plane_tiles = (a.n + kTcRows - 1) / kTcRows;
+  const int64_t plane_tiles = plane_tile_count(a);
   const int64_t n_tiles = plane_tiles * a.planes;
 
   if (warp == 8) {
@@ -703,9 +726,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
         mbar_expect_tx(&x_full[s], kTcTile);
         const int pl = tile >= plane_tiles;
         const CUtensorMap* map = pl ? &xmap2 : &xmap;
-        const int row0 = static_cast<int>((tile - pl * plane_tiles) * kTcRows);
-        tma_load_2d(xs0 + s * kTcTile, map, 0, row0, &x_full[s]);
-        tma_load_2d(xs0 + s * kTcTile + kTcBox, map, 64, row0, &x_full[s]);
+        const int64_t lt = tile - pl * plane_tiles;
+        if (a.head_major) {
+          const int head = static_cast<int>(lt % a.hkv), t0 = static_cast<int>((lt / a.hkv) * kTcRows);
+          tma_load_3d(xs0 + s * kTcTile, map, 0, head, t0, &x_full[s]);
+          tma_load_3d(xs0 + s * kTcTile + kTcBox, map, 64, head, t0, &x_full[s]);
+        } else {
+          const int row0 = static_cast<int>(lt * kTcRows);
+          tma_load_2d(xs0 + s * kTcTile, map, 0, row0, &x_full[s]);
+          tma_load_2d(xs0 + s * kTcTile + kTcBox, map, 64, row0, &x_full[s]);
+        }
       }
       // loads still in flight land before the CTA may exit
       for (int k = i - NST; k < i; ++k)
@@ -810,8 +840,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
       // outputs
       const int pl = tile >= plane_tiles;
       const PlaneDst pd = plane_dst(a, pl);
-      const int64_t v = (tile - pl * plane_tiles) * kTcRows + r;
-      if (v < a.n) {
+      const int64_t v = tile_row(a, tile - pl * plane_tiles, r);
+      if (v >= 0) {
         int64_t row = v;
         if (a.append) {
           int seq, head, pos;
@@ -1421,7 +1451,7 @@ bool tc_eligible(const QuantArgs& a) {
 // counts).
 int64_t quantize_grid(const QuantArgs& a) {
   if (a.n <= 0) return 0;
-  if (tc_eligible(a)) return std::min<int64_t>(((a.n + kTcRows - 1) / kTcRows) * a.planes, num_sms());
+  if (tc_eligible(a)) return std::min<int64_t>(plane_tile_count(a) * a.planes, num_sms());
   if (a.mse_bits == kWideBits) return std::min<int64_t>(a.n, 64LL * num_sms());
   return std::min<int64_t>((a.n + kTile - 1) / kTile, num_sms());
 }
@@ -1436,11 +1466,26 @@ bool encode_rows(CUtensorMap* map, const void* x, int64_t n) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same rows as [tokens][heads][d]: a box of 128 tokens of one head.
+bool encode_heads(CUtensorMap* map, const void* x, int64_t n, int hkv) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(hkv),
+                              static_cast<cuuint64_t>(n / hkv)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDim) * 2, static_cast<cuuint64_t>(kDim) * 2 * hkv};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kTcRows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_tiled()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 tq_status run_quantize_tc(const QuantArgs& a, cudaStream_t st) {
   CUtensorMap maps[2];
-  if (!encode_rows(&maps[0], a.x, a.n)) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
+  auto encode = [&](CUtensorMap* m, const void* x) {
+    return a.head_major ? encode_heads(m, x, a.n, a.hkv) : encode_rows(m, x, a.n);
+  };
+  if (!encode(&maps[0], a.x)) return fail(TQ_ERR_CUDA, "tq_quantize: cuTensorMapEncodeTiled failed");
   if (a.planes > 1) {
-    if (!encode_rows(&maps[1], a.x2, a.n)) return fail(TQ_ERR_CUDA, "tq_append: cuTensorMapEncodeTiled failed");
+    if (!encode(&maps[1], a.x2)) return fail(TQ_ERR_CUDA, "tq_append: cuTensorMapEncodeTiled failed");
   } else {
     maps[1] = maps[0];
   }
@@ -1592,6 +1637,7 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
     a.sink = which ? c->v_sink : c->k_sink;
     a.status = c->status;
     a.n_seq_in = n_seq;
+    a.head_major = !f.prod && tc_eligible(a);
   }
   // equal K and V formats on the tensor-core kernels: one launch for both
   QuantArgs both = q[0];

@@ -60,6 +60,14 @@ __device__ __forceinline__ void bulk_g2s_addr(uint32_t dst, const void* src, uin
 // 2-D tiled tensor copy of the box at element coordinates (x, y) of `map`
 // (x innermost; x * element size must be a multiple of 16 bytes).  Rows past
 // the tensor's end arrive as zeros; the full box counts toward the barrier.
+// 3-D tiled tensor copy of the box at element coordinates (x, y, z).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
