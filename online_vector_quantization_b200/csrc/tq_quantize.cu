@@ -639,16 +639,19 @@ __host__ __device__ __forceinline__ int64_t plane_tile_count(const QuantArgs& a)
   }
   return (a.n + kTcRows - 1) / kTcRows;
 }
+template <bool HM>
 __device__ __forceinline__ int64_t tile_row(const QuantArgs& a, int64_t lt, int r) {
-  if (a.head_major) {
+  if constexpr (HM) {
     const int64_t ts = (lt / a.hkv) * kTcRows + r;  // token index over the chunk
     return ts < a.n / a.hkv ? ts * a.hkv + lt % a.hkv : -1;
+  } else {
+    const int64_t v = lt * kTcRows + r;
+    return v < a.n ? v : -1;
   }
-  const int64_t v = lt * kTcRows + r;
-  return v < a.n ? v : -1;
 }
 
-template <int B, int MIXED>
+// HM: a.head_major (compiled apart so that the row-major path keeps its code).
+template <int B, int MIXED, bool HM>
 __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                     const __grid_constant__ CUtensorMap xmap2,
                                                                     QuantArgs a) {
@@ -701,7 +704,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const int64_t plane_tiles = plane_tile_count(a);
+  const int64_t plane_tiles = HM ? ((a.n / a.hkv + kTcRows - 1) / kTcRows) * a.hkv : (a.n + kTcRows - 1) / kTcRows;
   const int64_t n_tiles = plane_tiles * a.planes;
 
   if (warp == 8) {
@@ -727,7 +730,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
         const int pl = tile >= plane_tiles;
         const CUtensorMap* map = pl ? &xmap2 : &xmap;
         const int64_t lt = tile - pl * plane_tiles;
-        if (a.head_major) {
+        if constexpr (HM) {
           const int head = static_cast<int>(lt % a.hkv), t0 = static_cast<int>((lt / a.hkv) * kTcRows);
           tma_load_3d(xs0 + s * kTcTile, map, 0, head, t0, &x_full[s]);
           tma_load_3d(xs0 + s * kTcTile + kTcBox, map, 64, head, t0, &x_full[s]);
@@ -840,7 +843,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
       // outputs
       const int pl = tile >= plane_tiles;
       const PlaneDst pd = plane_dst(a, pl);
-      const int64_t v = tile_row(a, tile - pl * plane_tiles, r);
+      const int64_t v = tile_row<HM>(a, tile - pl * plane_tiles, r);
       if (v >= 0) {
         int64_t row = v;
         if (a.append) {
@@ -1423,15 +1426,19 @@ tq_status launch_tc_prod(const QuantArgs& a, const CUtensorMap* maps, int grid, 
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core prod quantize kernel launch");
 }
 
-template <int B, int MIXED>
-tq_status launch_tc(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
+template <int B, int MIXED, bool HM>
+tq_status launch_tc_hm(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
   constexpr int smem = B == kWideBits ? kTcSmemWide : kTcSmem;
-  cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED>>(smem);
+  cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED, HM>>(smem);
   if (e == cudaSuccess) {
-    quantize_tc_kernel<B, MIXED><<<grid, kTcThreads, smem, st>>>(maps[0], maps[1], a);
+    quantize_tc_kernel<B, MIXED, HM><<<grid, kTcThreads, smem, st>>>(maps[0], maps[1], a);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tensor-core quantize kernel launch");
+}
+template <int B, int MIXED>
+tq_status launch_tc(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
+  return a.head_major ? launch_tc_hm<B, MIXED, true>(a, maps, grid, st) : launch_tc_hm<B, MIXED, false>(a, maps, grid, st);
 }
 
 bool tc_format(const QuantArgs& a) {
