@@ -200,37 +200,74 @@ def run_gpu(args):
     params, cache = st["params"], st["cache"]
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        tq.tq_append(params, cache, st["ids"], st["ck"][i], st["cv"][i])
-        ev_d0.record(stream)
-        tq.tq_decode_attn(params, st["qs"][i], cache, st["cap"], st["out"], st["ws"])
-        ev_d1.record(stream)
+    def step(i, evs=None):
+        # on the current stream: the default stream, or the capture stream
+        s = torch.cuda.current_stream()
+        tq.tq_append(params, cache, st["ids"], st["ck"][i], st["cv"][i], stream=s)
+        if evs is not None:
+            evs[0].record(s)
+        tq.tq_decode_attn(params, st["qs"][i], cache, st["cap"], st["out"], st["ws"], stream=s)
+        if evs is not None:
+            evs[1].record(s)
 
-    ev_d0, ev_d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    lens_at_timing = [n + args.warmup * CHUNK for n in st["lens"]]
+    lens_t = torch.tensor(lens_at_timing, dtype=torch.int32, device=device)
+    # The K timed steps are captured once in a CUDA graph (capturing runs
+    # nothing) and replayed as one launch.  A second capture of the same steps
+    # records timing events around every decode call for the roofline; it is
+    # replayed after the timed region (lengths rewound), since an event
+    # between the append and the decode call's first kernel holds that kernel
+    # until the append has finished (no programmatic overlap).
+    d_events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+                for _ in range(args.steps)]
+    graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(device=device)
+    with torch.cuda.graph(graph, stream=cap_stream):
+        for j in range(args.steps):
+            step(args.warmup + j)
+    with torch.cuda.graph(graph_ev, stream=cap_stream):
+        for j in range(args.steps):
+            step(args.warmup + j, d_events[j])
+    torch.cuda.synchronize()
+    assert cache.lens.cpu().tolist() == lens_at_timing
     if world > 1:
         dist.barrier()
-    lens_at_timing = [n + args.warmup * CHUNK for n in st["lens"]]
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    d_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
     torch.cuda.synchronize()
     t0.record(stream)
-    for j in range(args.steps):
-        ev_d0, ev_d1 = d_events[j]
-        step(args.warmup + j)
+    graph.replay()
     t1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
+
+    def rerun(fn):
+        cache.lens.copy_(lens_t)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    # the same steps with the decode calls bracketed by events, and issued
+    # call by call from the host
+    ev_ms = rerun(graph_ev.replay)
+    eager_ms = rerun(lambda: [step(args.warmup + j) for j in range(args.steps)])
+    del graph, graph_ev
     total_ms = t0.elapsed_time(t1)
     decode_ms = [a.elapsed_time(b) for a, b in d_events]
     if world > 1:
         total_ms = max_over_ranks(total_ms, dist, device)
+        eager_ms = max_over_ranks(eager_ms, dist, device)
+        ev_ms = max_over_ranks(ev_ms, dist, device)
     append_b, decode_b = 0, 0
     for j in range(args.steps):
         a, d = step_bytes([n + j * CHUNK for n in lens_at_timing])
@@ -263,6 +300,9 @@ def run_gpu(args):
                        "seq_lens": st["lens"], "l2": "inputs larger than L2 (cache read ~570 MB per step)",
                        "tokens_per_s_per_seq": round(1000.0 / ms_per_step, 2),
                        "decode_ms": round(avg_decode_s * 1e3, 4),
+                       "launch": "the timed steps captured in one CUDA graph (one replay)",
+                       "eager_ms_per_step": round(eager_ms / args.steps, 4),
+                       "decode_events_ms_per_step": round(ev_ms / args.steps, 4),
                        "append_plus_decode_bytes_per_step": (append_b + decode_b) // args.steps,
                        "parallelism": f"replicas x{world}"},
             "roofline": {"kernel": "decode_kernel<mixed3.5,mixed3.5> (+qrot, merge)", "bound": "hbm",
@@ -307,7 +347,6 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     def bring_in(j):
         b = j & 1
         with torch.cuda.stream(copy_stream):
@@ -318,6 +357,8 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
             dq[b].copy_(hq[j], non_blocking=True)
             copied[j].record(copy_stream)
 
+    # (1) eager: every call issued from the host loop
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     copy_stream.wait_event(t0)
     bring_in(0)
@@ -334,7 +375,58 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
         hout[b].copy_(st["out"], non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
+    eager_ms = t0.elapsed_time(t1)
+
+    # (2) the same calls captured once per step (before the timed region) in a
+    # CUDA graph and replayed.  Graph j appends and decodes step j; beside
+    # them, on a forked branch, it copies step j + 1's inputs in and step
+    # j - 1's result out (outputs double-buffered on the device), so neither
+    # the copies nor the host's per-call launch work sit on the step's path.
+    # One graph per step because every step reads its own pinned host buffers.
+    cache.lens.copy_(lens0)
+    dout = [st["out"], torch.empty_like(st["out"])]
+    cap_stream = torch.cuda.Stream(device=device)
+    graphs = []
+    for j in range(args.steps):
+        b = j & 1
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            branch = j + 1 < args.steps or j >= 1
+            if branch:
+                fork, join = torch.cuda.Event(), torch.cuda.Event()
+                fork.record(cap_stream)
+                copy_stream.wait_event(fork)
+                with torch.cuda.stream(copy_stream):
+                    if j + 1 < args.steps:
+                        nb = (j + 1) & 1
+                        dk[nb].copy_(hk[j + 1], non_blocking=True)
+                        dv[nb].copy_(hv[j + 1], non_blocking=True)
+                        dq[nb].copy_(hq[j + 1], non_blocking=True)
+                    if j >= 1:
+                        hout[1 - b].copy_(dout[1 - b], non_blocking=True)
+                    join.record(copy_stream)
+            tq.tq_append(params, cache, st["ids"], dk[b], dv[b], stream=cap_stream)
+            tq.tq_decode_attn(params, dq[b], cache, st["cap"], dout[b], st["ws"], stream=cap_stream)
+            if branch:
+                cap_stream.wait_event(join)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    dk[0].copy_(hk[0], non_blocking=True)
+    dv[0].copy_(hv[0], non_blocking=True)
+    dq[0].copy_(hq[0], non_blocking=True)
+    for g in graphs:
+        g.replay()
+    last = (args.steps - 1) & 1
+    hout[last].copy_(dout[last], non_blocking=True)  # the last step's result
+    t1.record(stream)
+    torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
+    assert int(cache.status.item()) == 0
+    del graphs
     # the same copies alone (no kernels): how much of the step is PCIe
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(copy_stream)
@@ -351,6 +443,7 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     if world > 1:
         ms = max_over_ranks(ms, dist, device)
         copy_ms = max_over_ranks(copy_ms, dist, device)
+        eager_ms = max_over_ranks(eager_ms, dist, device)
     total = 0
     for j in range(args.steps):
         a, d = step_bytes([n + (args.warmup + j) * CHUNK for n in st["lens"]])
@@ -358,7 +451,9 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     h2d = 2 * N_SEQ * CHUNK * HKV * D * 2 + N_SEQ * HQ * D * 2
     return {"value": round(total * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms / args.steps, 4),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": N_SEQ * HQ * D * 2,
-            "copies_alone_ms_per_step": round(copy_ms / args.steps, 4)}
+            "copies_alone_ms_per_step": round(copy_ms / args.steps, 4),
+            "launch": "one CUDA graph per step of the public calls (captured before the timed region)",
+            "eager_ms_per_step": round(eager_ms / args.steps, 4)}
 
 
 def _flush_l2(torch, buf):
