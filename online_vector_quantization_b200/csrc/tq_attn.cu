@@ -447,6 +447,7 @@ inline size_t merge_dyn_bytes(int n_sink, int ctas, int group, int part_floats, 
 template <int VF, int MH>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   static_assert(MH == 1 || MH == 4 || MH == 8, "heads per merge CTA");
+  pdl_launch();  // the next append's kernel may set itself up meanwhile (it waits for this grid)
   using FV = Fmt<VF>;
   constexpr int NT = kMergeThreads;
   constexpr int WD = FV::prod ? 2 * kDim : kDim;  // accumulator: rotated | sketch

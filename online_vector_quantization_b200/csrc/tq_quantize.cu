@@ -78,6 +78,11 @@ struct QuantArgs {
   // and returns the count to zero.  0 = no update in this launch.
   int arrive_total;
   int n_seq_in;
+  // Launched with programmatic stream serialization (the tensor-core kernel
+  // of an append): the CTAs may start while the previous kernel on the stream
+  // still runs, and set up shared memory, barriers and tensor memory before
+  // they wait for it; every global access comes after the wait.
+  int overlapped;
   // Append input in head-major tiles (the MSE tensor-core kernel): tile =
   // 128 consecutive tokens (over the n_seq_in x n_tok chunk, token-major) of
   // one kv-head, so a warp's 32 rows go to consecutive rows of one cache unit
@@ -90,6 +95,11 @@ struct QuantArgs {
 // stream serialization (the decode call's query rotation), start its own
 // independent prologue; it waits for this grid before reading its outputs.
 __device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// Waits until the previous kernel on the stream has finished and its writes
+// are visible (returns at once when this grid was launched without
+// programmatic stream serialization).
+__device__ __forceinline__ void wait_prerequisites() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 // The input and destinations of plane pl.
 struct PlaneDst {
@@ -703,6 +713,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) quantize_tc_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // everything above touched only shared memory, tensor memory and the
+  // parameter tables; the input, the cache and its lengths come after
+  wait_prerequisites();
   const uint32_t tmem = s_tmem;
   const int64_t plane_tiles = HM ? ((a.n / a.hkv + kTcRows - 1) / kTcRows) * a.hkv : (a.n + kTcRows - 1) / kTcRows;
   const int64_t n_tiles = plane_tiles * a.planes;
@@ -1430,7 +1443,19 @@ template <int B, int MIXED, bool HM>
 tq_status launch_tc_hm(const QuantArgs& a, const CUtensorMap* maps, int grid, cudaStream_t st) {
   constexpr int smem = B == kWideBits ? kTcSmemWide : kTcSmem;
   cudaError_t e = ensure_dyn_smem<quantize_tc_kernel<B, MIXED, HM>>(smem);
-  if (e == cudaSuccess) {
+  if (e == cudaSuccess && a.overlapped) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, quantize_tc_kernel<B, MIXED, HM>, maps[0], maps[1], a);
+  } else if (e == cudaSuccess) {
     quantize_tc_kernel<B, MIXED, HM><<<grid, kTcThreads, smem, st>>>(maps[0], maps[1], a);
     e = cudaGetLastError();
   }
@@ -1657,6 +1682,7 @@ tq_status launch_append(const tq_params* p, const tq_cache* c, const int32_t* se
   both.sink2 = c->v_sink;
   if (p->fk.id() == p->fv.id() && tc_eligible(both)) {
     both.arrive_total = static_cast<int>(quantize_grid(both));
+    both.overlapped = 1;
     return run_quantize(both, st);
   }
   // otherwise K on the caller's stream and V on a side stream, concurrently;
