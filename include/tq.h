@@ -19,6 +19,12 @@
  *    allocates the parameter tables once and tq_params_destroy frees them.
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
  *    default stream).  Device calls only enqueue work and never synchronize.
+ *    tq_append and tq_decode_attn may therefore be captured into a CUDA
+ *    graph on a capturing stream (tq_append's side stream, used when K and V
+ *    formats differ, forks from and joins back into it) once each has been
+ *    called eagerly on the device, which sets the kernels' attributes; a
+ *    replay reads the lengths on the device, so it appends after and
+ *    attends over whatever the cache holds at replay time.
  *  - Errors: every call returns a tq_status; TQ_OK is 0.  On failure nothing
  *    is enqueued and tq_last_error() returns a message for the calling host
  *    thread.  Inputs must be finite: NaN or Inf inputs give unspecified codes
