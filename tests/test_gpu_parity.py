@@ -722,3 +722,54 @@ def test_decode_reads_query_and_cache_written_just_before():
         torch.cuda.synchronize()
         assert torch.equal(out_fast, out_sync), trial
         assert cache.lens.cpu().tolist() == [T] * B and int(cache.status.item()) == 0
+
+
+def test_back_to_back_steps_match_synchronized_steps():
+    """The append's kernel starts under programmatic stream serialization
+    right after the previous step's merge (which lets it launch early), and
+    its input comes from the kernel just before it: step after step without a
+    synchronization, every decode output and the final lengths must equal
+    those of the same steps with a full synchronization around every call."""
+    fk = fv = gu.fmt(3, mixed=True)
+    gp, _ = gu.make_params(fk, fv)
+    B, hkv, hq, chunk, steps = 4, 2, 8, 48, 6
+    lens0 = [130, 0, 515, 64]
+    k = kv_inputs.kv_vectors(steps * B * chunk * hkv, 128, key=("b2b", "k"), dtype=torch.float32).view(steps, B, chunk, hkv, 128).cuda()
+    v = kv_inputs.kv_vectors(steps * B * chunk * hkv, 128, key=("b2b", "v"), dtype=torch.float32).view(steps, B, chunk, hkv, 128).cuda()
+    qs = kv_inputs.queries((steps, B, hq, 128), key=("b2b", "q"), dtype=torch.float32).cuda()
+    ids = torch.arange(B, dtype=torch.int32, device="cuda")
+    cap = 896
+
+    def prefilled():
+        cache = tq.Cache(gp, B, hkv, cap, 0)
+        for s, n in enumerate(lens0):
+            if n:
+                x = kv_inputs.kv_vectors(n * hkv, 128, key=("b2b-pre", s), dtype=torch.bfloat16).view(1, n, hkv, 128).cuda()
+                tq.tq_append(gp, cache, torch.tensor([s], dtype=torch.int32, device="cuda"), x, x)
+        torch.cuda.synchronize()
+        return cache
+
+    outs = {}
+    for mode in ("sync", "fast"):
+        cache = prefilled()
+        ws = tq.decode_workspace(gp, B, hq, hkv, cap)
+        outs[mode] = []
+        for i in range(steps):
+            # the chunk and the query are written by the kernels just before the calls
+            kc, vc = k[i].to(torch.bfloat16), v[i].to(torch.bfloat16)
+            q = qs[i].to(torch.bfloat16)
+            if mode == "sync":
+                torch.cuda.synchronize()
+            tq.tq_append(gp, cache, ids, kc, vc)
+            if mode == "sync":
+                torch.cuda.synchronize()
+            out = torch.empty(B, hq, 128, dtype=torch.bfloat16, device="cuda")
+            tq.tq_decode_attn(gp, q, cache, cap, out, ws)
+            if mode == "sync":
+                torch.cuda.synchronize()
+            outs[mode].append(out)
+        torch.cuda.synchronize()
+        assert cache.lens.cpu().tolist() == [n + steps * chunk for n in lens0], mode
+        assert int(cache.status.item()) == 0, mode
+    for i in range(steps):
+        assert torch.equal(outs["fast"][i], outs["sync"][i]), i
