@@ -379,35 +379,41 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
 
     # (2) the same calls captured once per step (before the timed region) in a
     # CUDA graph and replayed.  Graph j appends and decodes step j; beside
-    # them, on a forked branch, it copies step j + 1's inputs in and step
+    # them, on forked branches, it copies step j + 1's inputs in and step
     # j - 1's result out (outputs double-buffered on the device), so neither
     # the copies nor the host's per-call launch work sit on the step's path.
     # One graph per step because every step reads its own pinned host buffers.
     cache.lens.copy_(lens0)
     dout = [st["out"], torch.empty_like(st["out"])]
     cap_stream = torch.cuda.Stream(device=device)
+    out_stream = torch.cuda.Stream(device=device)
     graphs = []
     for j in range(args.steps):
         b = j & 1
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap_stream):
-            branch = j + 1 < args.steps or j >= 1
-            if branch:
+            # two branches, one per copy direction, so the result copy does
+            # not queue behind the input copies
+            joins = []
+            for active, cs in ((j + 1 < args.steps, copy_stream), (j >= 1, out_stream)):
+                if not active:
+                    continue
                 fork, join = torch.cuda.Event(), torch.cuda.Event()
                 fork.record(cap_stream)
-                copy_stream.wait_event(fork)
-                with torch.cuda.stream(copy_stream):
-                    if j + 1 < args.steps:
+                cs.wait_event(fork)
+                with torch.cuda.stream(cs):
+                    if cs is copy_stream:
                         nb = (j + 1) & 1
                         dk[nb].copy_(hk[j + 1], non_blocking=True)
                         dv[nb].copy_(hv[j + 1], non_blocking=True)
                         dq[nb].copy_(hq[j + 1], non_blocking=True)
-                    if j >= 1:
+                    else:
                         hout[1 - b].copy_(dout[1 - b], non_blocking=True)
-                    join.record(copy_stream)
+                    join.record(cs)
+                joins.append(join)
             tq.tq_append(params, cache, st["ids"], dk[b], dv[b], stream=cap_stream)
             tq.tq_decode_attn(params, dq[b], cache, st["cap"], dout[b], st["ws"], stream=cap_stream)
-            if branch:
+            for join in joins:
                 cap_stream.wait_event(join)
         graphs.append(g)
     torch.cuda.synchronize()
@@ -427,16 +433,22 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     ms = t0.elapsed_time(t1)
     assert int(cache.status.item()) == 0
     del graphs
-    # the same copies alone (no kernels): how much of the step is PCIe
+    # the same copies alone (no kernels, each direction on its own stream): how
+    # much of the step is PCIe
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(copy_stream)
-    with torch.cuda.stream(copy_stream):
-        for j in range(args.steps):
-            b = j & 1
+    out_stream.wait_event(c0)
+    for j in range(args.steps):
+        b = j & 1
+        with torch.cuda.stream(copy_stream):
             dk[b].copy_(hk[j], non_blocking=True)
             dv[b].copy_(hv[j], non_blocking=True)
             dq[b].copy_(hq[j], non_blocking=True)
+        with torch.cuda.stream(out_stream):
             hout[b].copy_(st["out"], non_blocking=True)
+    done = torch.cuda.Event()
+    done.record(out_stream)
+    copy_stream.wait_event(done)
     c1.record(copy_stream)
     torch.cuda.synchronize()
     copy_ms = c0.elapsed_time(c1)
