@@ -223,12 +223,14 @@ def run_gpu(args):
     # until the append has finished (no programmatic overlap).
     d_events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
                 for _ in range(args.steps)]
+    # (thread-local capture: a CUDA call from another thread of the process,
+    # such as a communication library's watchdog, does not void the capture)
     graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream(device=device)
-    with torch.cuda.graph(graph, stream=cap_stream):
+    with torch.cuda.graph(graph, stream=cap_stream, capture_error_mode="thread_local"):
         for j in range(args.steps):
             step(args.warmup + j)
-    with torch.cuda.graph(graph_ev, stream=cap_stream):
+    with torch.cuda.graph(graph_ev, stream=cap_stream, capture_error_mode="thread_local"):
         for j in range(args.steps):
             step(args.warmup + j, d_events[j])
     torch.cuda.synchronize()
@@ -391,7 +393,7 @@ def run_e2e(tq, torch, kv_inputs, args, st, rank, device, world):
     for j in range(args.steps):
         b = j & 1
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap_stream):
+        with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
             # two branches, one per copy direction, so the result copy does
             # not queue behind the input copies
             joins = []
